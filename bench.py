@@ -1,0 +1,443 @@
+#!/usr/bin/env python3
+"""Samba block prefill benchmark on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl samba|reference]
+
+Workload: long-context prefill, batch 1, L = 131072 tokens through a stack of 4
+bf16 Samba blocks (d_model 2048, d_inner 4096, d_state 16, d_conv 4, dt_rank 128,
+32/4 heads of 64, window 2048, SwiGLU 8192).  One step = the whole stack over one
+sequence.  Metric: prefill tokens/s per block = B*L / (step time / 4), summed over
+ranks (each rank runs its own replica: no data-path collective).
+
+Printed JSON line (rank 0): value (device time, inputs resident in HBM), e2e
+(same metric through the C ABI with pinned host input/output copied inside the
+timed region), roofline of the dominant kernel (from a CUDA-event attribution
+pass over the same kernels), the oracle CPU baseline, clocks sampled during the
+timed region.  `--impl reference` times the fp64 CPU oracle on a bounded sample
+of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from sliding_window_attention_samba_b200 import inputs as I  # noqa: E402
+
+WORKLOAD = "prefill_bf16_L131072_x4"
+METRIC = "prefill tokens/s per Samba block at L=128K"
+UNIT = "tokens/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="samba", choices=["samba", "reference"])
+    ap.add_argument("--seq-len", type=int, default=None, help="override L (parity/debug runs only)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), d.get("bf16_tflops_sustained", 1400.0), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# the CUDA path
+# ---------------------------------------------------------------------------
+def make_stack(torch, L, shape, n_blocks, seed, dev):
+    """Random-init weights of the stack on the device (N(0, 0.02) matrices,
+    S4D-Real A, D = 1, Delta bias in [1e-3, 1e-1], unit norm gains)."""
+    g = torch.Generator(device=dev)
+    blocks = []
+    s = shape
+    bf = torch.bfloat16
+    for li in range(n_blocks):
+        g.manual_seed(I.tensor_key(seed, f"stack.L{li}") & ((1 << 63) - 1))
+
+        def mat(o, i):
+            return (torch.randn(o, i, generator=g, device=dev) * 0.02).to(bf)
+
+        w = {f"norm{i}": torch.ones(s.d_model, device=dev) for i in range(4)}
+        w["W_in"] = mat(2 * s.d_inner, s.d_model)
+        w["conv_w"] = torch.randn(s.d_inner, s.d_conv, generator=g, device=dev) * 0.02
+        w["conv_b"] = None
+        w["W_x"] = mat(s.dt_rank + 2 * s.d_state, s.d_inner)
+        w["W_dt"] = mat(s.d_inner, s.dt_rank)
+        w["dt_bias"] = torch.from_numpy(I.dt_bias_init(seed, f"stack.L{li}.dt_bias", s.d_inner)).to(dev)
+        w["A_log"] = torch.from_numpy(I.a_log_init(s.d_inner, s.d_state)).to(dev)
+        w["D"] = torch.ones(s.d_inner, device=dev)
+        w["W_out"] = mat(s.d_model, s.d_inner)
+        w["Wq"] = mat(s.n_q * s.head_dim, s.d_model)
+        w["Wk"] = mat(s.n_kv * s.head_dim, s.d_model)
+        w["Wv"] = mat(s.n_kv * s.head_dim, s.d_model)
+        w["Wo"] = mat(s.d_model, s.n_q * s.head_dim)
+        for m in (1, 2):
+            w[f"mlp{m}_W1"] = mat(s.d_ff, s.d_model)
+            w[f"mlp{m}_W2"] = mat(s.d_ff, s.d_model)
+            w[f"mlp{m}_W3"] = mat(s.d_model, s.d_ff)
+        blocks.append((w, L.make_weights(w)))
+    return blocks
+
+
+def gemm_list(s, T):
+    """(name, M, N, K, epilogue, flops) of every projection in one block, in launch order."""
+    R, N16 = s.dt_rank, s.d_state
+    qkvw = (s.n_q + 2 * s.n_kv) * s.head_dim
+    g = [("in_proj", T, 2 * s.d_inner, s.d_model, 0),
+         ("x_proj", T, R + 2 * N16, s.d_inner, 0),
+         ("dt_proj", T, s.d_inner, R, 3),
+         ("out_proj", T, s.d_model, s.d_inner, 1),
+         ("mlp1_up", T, s.d_ff, s.d_model, 2),
+         ("mlp1_down", T, s.d_model, s.d_ff, 1),
+         ("qkv", T, qkvw, s.d_model, 0),
+         ("o_proj", T, s.d_model, s.n_q * s.head_dim, 1),
+         ("mlp2_up", T, s.d_ff, s.d_model, 2),
+         ("mlp2_down", T, s.d_model, s.d_ff, 1)]
+    return [(n, M, N, K, e, 2.0 * M * N * K * (2 if e == 2 else 1)) for (n, M, N, K, e) in g]
+
+
+def swa_flops(s, Bn, Ln):
+    w = s.window
+    pairs = Ln * w - w * (w - 1) / 2 if Ln >= w else Ln * (Ln + 1) / 2
+    return 4.0 * s.head_dim * s.n_q * pairs * Bn
+
+
+def attribution_pass(torch, L, s, blocks, x, T, Bn, Ln, reps=2):
+    """Times each kernel of one block separately through the component entry
+    points (same kernels, same shapes, same stream) with CUDA events."""
+    dev = x.device
+    bf = torch.bfloat16
+    st = torch.cuda.current_stream()
+    w, _ = blocks[0]
+    xn = torch.empty(T, s.d_model, device=dev, dtype=bf)
+    hz = torch.empty(T, 2 * s.d_inner, device=dev, dtype=bf)
+    u = torch.empty(T, s.d_inner, device=dev, dtype=bf)
+    xdbl = torch.empty(T, s.dt_rank + 2 * s.d_state, device=dev, dtype=bf)
+    dlt = torch.empty(T, s.d_inner, device=dev, dtype=bf)
+    y = torch.empty(T, s.d_inner, device=dev, dtype=bf)
+    big = torch.empty(T, s.d_ff, device=dev, dtype=bf)
+    xo = torch.empty(T, s.d_model, device=dev, dtype=bf)
+    q = torch.empty(Bn, Ln, s.n_q, s.head_dim, device=dev, dtype=bf).normal_()
+    kk = torch.empty(Bn, Ln, s.n_kv, s.head_dim, device=dev, dtype=bf).normal_()
+    vv = torch.empty_like(kk).normal_()
+    o = torch.empty_like(q)
+    times = {}
+
+    def timed(name, fn):
+        for _ in range(reps + 1):  # first call is a warm-up
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(st)
+            fn()
+            e1.record(st)
+            e1.synchronize()
+            times.setdefault(name, []).append(e0.elapsed_time(e1) * 1e-3)
+        times[name] = times[name][1:]
+
+    timed("rmsnorm", lambda: L.samba_rmsnorm(x, w["norm0"], xn, T, s.d_model, s.norm_eps, 1))
+    W = {"in_proj": (w["W_in"], None, xn, hz), "x_proj": (w["W_x"], None, u, xdbl),
+         "dt_proj": (w["W_dt"], None, None, dlt), "out_proj": (w["W_out"], None, y, xo),
+         "mlp1_up": (w["mlp1_W1"], w["mlp1_W2"], xn, big), "mlp1_down": (w["mlp1_W3"], None, big, xo),
+         "qkv": (w["Wq"], None, xn, None), "o_proj": (w["Wo"], None, o, xo)}
+    for (name, M, N, K, e, fl) in gemm_list(s, T):
+        if name in ("mlp2_up", "mlp2_down"):
+            continue
+        Wm, W2, a_in, out = W[name]
+        a_t = torch.empty(M, K, device=dev, dtype=bf).normal_() if a_in is None or a_in.shape[1] != K else a_in
+        o_t = torch.empty(M, N, device=dev, dtype=bf) if out is None or out.shape[1] != N else out
+        Wt = Wm if Wm.shape == (N, K) else torch.empty(N, K, device=dev, dtype=bf).normal_()
+        timed(name, lambda a_t=a_t, Wt=Wt, W2=W2, o_t=o_t, M=M, N=N, K=K, e=e: L.samba_linear(
+            a_t, Wt, W2, w["dt_bias"] if e == 3 else None, x if e == 1 else None, o_t, M, N, K, e, 1))
+    timed("conv", lambda: L.samba_causal_conv1d(hz, 2 * s.d_inner, w["conv_w"], None, u, None, Bn, Ln, s.d_inner,
+                                                 s.d_conv, 1))
+    timed("scan", lambda: _scan_contig(torch, L, s, w, u, dlt, hz, y, Bn, Ln))
+    timed("swa", lambda: L.samba_swa_fwd(q, kk, vv, o, Bn, Ln, s.n_q, s.n_kv, s.head_dim, s.window, 0.0, 0, 0.0, 1))
+    return {k: sum(v) / len(v) for k, v in times.items()}
+
+
+_SCAN_BUFS = {}
+
+
+def _scan_contig(torch, L, s, w, u, dlt, hz, y, Bn, Ln):
+    """Selective scan on contiguous [B, L, D] operands of the block's sizes."""
+    key = (Bn, Ln)
+    if key not in _SCAN_BUFS:
+        dev = u.device
+        T = Bn * Ln
+        _SCAN_BUFS[key] = (torch.empty(T, s.d_inner, device=dev, dtype=torch.bfloat16).normal_(),
+                           torch.empty(T, s.d_state, device=dev, dtype=torch.bfloat16).normal_(),
+                           torch.empty(T, s.d_state, device=dev, dtype=torch.bfloat16).normal_())
+    z, Bm, Cm = _SCAN_BUFS[key]
+    L.samba_selective_scan(u, dlt, None, 0, w["A_log"], Bm, Cm, w["D"], z, None, None, y, Bn, Ln, s.d_inner,
+                           s.d_state, 1)
+
+
+def run_cuda(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from sliding_window_attention_samba_b200 import _lib as L
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    shape, Bn, Ln, n_blocks, seed = I.WORKLOADS[WORKLOAD]
+    if args.seq_len:
+        Ln = args.seq_len
+    s = shape
+    T = Bn * Ln
+    cfg = L.make_config(s)
+    blocks = make_stack(torch, L, s, n_blocks, seed + 1000 * rank, dev)
+    ws_bytes = L.samba_block_workspace_size(cfg, Bn, Ln)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    gx = torch.Generator(device=dev)
+    gx.manual_seed(I.tensor_key(seed + rank, "stack.x") & ((1 << 63) - 1))
+    x0 = torch.randn(Bn, Ln, s.d_model, generator=gx, device=dev).to(torch.bfloat16)
+    bufs = [torch.empty_like(x0), torch.empty_like(x0)]
+    stream = torch.cuda.current_stream()
+
+    def step(x_in):
+        cur = x_in
+        for i, (_, wst) in enumerate(blocks):
+            out = bufs[i % 2]
+            L.samba_block_fwd(cfg, wst, cur, out, None, None, Bn, Ln, ws, ws_bytes)
+            cur = out
+        return cur
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step(x0)
+    torch.cuda.synchronize()
+    assert L.samba_get_error() == 0, "device error during warm-up"
+
+    # ---- device-timed region (inputs resident; activations >> L2, no flush needed)
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step(x0)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    t_dev = e0.elapsed_time(e1) * 1e-3
+    assert L.samba_get_error() == 0, "device error in the timed region"
+
+    # ---- end to end: pinned host input -> device -> stack -> host output, per step
+    xh = x0.cpu().pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    xd = torch.empty_like(x0)
+    barrier()
+    torch.cuda.synchronize()
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.steps):
+        xd.copy_(xh, non_blocking=True)
+        out = step(xd)
+        yh.copy_(out, non_blocking=True)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    t_e2e = f0.elapsed_time(f1) * 1e-3
+
+    # ---- per-kernel attribution (same kernels and shapes, one block)
+    kt = attribution_pass(torch, L, s, blocks, x0.view(T, s.d_model), T, Bn, Ln) if rank == 0 else {}
+
+    def tmax(t):
+        if world == 1:
+            return t
+        tt = torch.tensor([t], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        return float(tt.item())
+
+    t_dev, t_e2e = tmax(t_dev), tmax(t_e2e)
+    return dict(t_dev=t_dev, t_e2e=t_e2e, clocks=clk, kt=kt, s=s, Bn=Bn, Ln=Ln, n_blocks=n_blocks,
+                h2d=xh.numel() * 2, d2h=yh.numel() * 2)
+
+
+def kernel_report(kt, s, T, Bn, Ln, peaks):
+    hbm, tf_burst, tf_sus, src = peaks
+    gl = gemm_list(s, T)
+    g_flops = sum(fl for (n, M, N, K, e, fl) in gl if n in kt)
+    g_time = sum(kt[n] for (n, *_r) in gl if n in kt)
+    n_g = len([1 for (n, *_r) in gl if n in kt])
+    rep = {"gemm": {"tflops": g_flops / g_time / 1e12, "frac_of_" + src + "_bf16_peak": g_flops / g_time / 1e12 / tf_sus,
+                    "per_gemm_tflops": {n: round(fl / kt[n] / 1e12, 1) for (n, M, N, K, e, fl) in gl if n in kt}}}
+    scan_bytes = T * (8 * s.d_inner + 4 * s.d_state)
+    rep["scan"] = {"gbs": scan_bytes / kt["scan"] / 1e9, "frac_of_" + src + "_hbm": scan_bytes / kt["scan"] / 1e9 / hbm,
+                   "ms": kt["scan"] * 1e3}
+    sf = swa_flops(s, Bn, Ln)
+    rep["swa"] = {"tflops": sf / kt["swa"] / 1e12, "frac_of_" + src + "_bf16_peak": sf / kt["swa"] / 1e12 / tf_sus,
+                  "ms": kt["swa"] * 1e3}
+    conv_bytes = T * s.d_inner * 4
+    rep["conv"] = {"gbs": conv_bytes / kt["conv"] / 1e9, "ms": kt["conv"] * 1e3}
+    rep["rmsnorm"] = {"gbs": T * s.d_model * 4 / kt["rmsnorm"] / 1e9, "ms": kt["rmsnorm"] * 1e3}
+    roof = {"bound": "tensor", "achieved": round(g_flops / n_g / (g_time / n_g) / 1e12, 2), "peak": tf_sus,
+            "unit": "TFLOP/s", "frac": round(g_flops / g_time / 1e12 / tf_sus, 4), "traffic": None,
+            "kernel": "gemm_tc (all projections of a block, flop-weighted)", "peak_source": src + " sustained bf16"}
+    return roof, rep
+
+
+# ---------------------------------------------------------------------------
+# the oracle (CPU baseline / reference arm)
+# ---------------------------------------------------------------------------
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def oracle_sample(sample_len=1024):
+    """fp64 oracle of one block at the workload's shapes on a bounded sample:
+    batch 1, the first `sample_len` tokens.  Returns (tokens/s per block, desc)."""
+    from oracle import samba_oracle as O
+    shape = I.WORKLOADS[WORKLOAD][0]
+    W = I.block_weights(shape, 2)
+    x = I.block_input(shape, 2, 1, sample_len)
+    t0 = time.perf_counter()
+    O.block_fwd(x, W, shape)
+    dt = time.perf_counter() - t0
+    return sample_len / dt, f"1 block, batch 1, first {sample_len} tokens of the L=131072 sequence (fp64 numpy)"
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    shape, Bn, Ln, n_blocks, _ = I.WORKLOADS[WORKLOAD]
+    if args.seq_len:
+        Ln = args.seq_len
+    cfgd = {"workload": WORKLOAD, "model": "samba block stack (random init)", "global_batch": Bn * max(world, 1),
+            "seq_len": Ln, "n_blocks": n_blocks, "d_model": shape.d_model, "window": shape.window,
+            "parallelism": f"replicas{max(world, 1)}", "l2": "activations per block >> 126 MB L2; no flush needed"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        vals = []
+        for i in range(args.warmup + args.steps):
+            v, desc = oracle_sample(256)
+            if i >= args.warmup:
+                vals.append(v)
+        v = statistics.mean(vals)
+        print(json.dumps({"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+                          "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+                          "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfgd,
+                          "cpu_baseline": {"value": v, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                                           "sample": desc},
+                          "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
+        return
+
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        import datetime
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    r = run_cuda(args, rank, world, local_rank)
+    peaks = load_peaks()
+    if rank == 0:
+        tok_block = Bn * Ln * world  # tokens through each block, all ranks
+        value = tok_block / (r["t_dev"] / args.steps / n_blocks)
+        e2e = tok_block / (r["t_e2e"] / args.steps / n_blocks)
+        roof, rep = kernel_report(r["kt"], r["s"], Bn * Ln, Bn, Ln, peaks)
+        cpu = None
+        if not args.no_cpu_baseline:
+            v, desc = oracle_sample(1024)
+            cpu = {"value": v, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle", "sample": desc}
+        launches_per_block = 4 + 10 + 1 + 1 + 1 + 1  # norms, projections, conv, scan, rope table, swa
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": r["t_dev"] / args.steps * 1e3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfgd,
+                "e2e": {"value": e2e, "unit": UNIT, "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
+                "roofline": roof, "kernels": rep, "cpu_baseline": cpu, "clocks": r["clocks"],
+                "gpu_launches": launches_per_block * n_blocks * args.steps}
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,234 @@
+/*
+ * samba.h - C ABI of the B200 (sm_100a) Samba block library (libsamba.so).
+ *
+ * What is computed follows the page "Samba: Simple Hybrid State Space Models
+ * for Efficient Unlimited Context Language Modeling" (a long-form summary of
+ * arXiv 2406.07522), cited as [Samba <section>, <sub-heading>].  The block is
+ * Mamba -> SwiGLU MLP -> sliding-window attention -> SwiGLU MLP, every layer
+ * pre-RMSNorm with a residual add [Samba 3.2 "Big-Picture Architecture"].
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller, 16-byte
+ *     aligned, contiguous row-major with the innermost dimension last, unless an
+ *     argument says otherwise.  The library allocates no device memory: scratch
+ *     space comes from the caller through (workspace, workspace_bytes), sized by
+ *     the matching *_workspace_size query.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream).  The return value reports argument validation and launch errors
+ *     only.  Errors detected on the device (a bounded wait that gave up, a
+ *     failed device-side check) are latched in a device error word that
+ *     samba_get_error() reads.
+ *   - Activations and weight matrices are `samba_dtype` (fp32 or bf16); per-channel
+ *     parameters (norm gains, conv taps, dt bias, A_log, D) and the SSM state are
+ *     fp32.  Arithmetic is fp32 (fp32 accumulation on the tensor cores).
+ *   - Weight matrices are stored [out_features, in_features] row-major, i.e. the
+ *     transpose of the pages' X W notation.
+ *   - No exception, C++ type or torch type crosses this boundary; the library is
+ *     stateless apart from the device error word and is reentrant.
+ */
+#ifndef SAMBA_H_
+#define SAMBA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SAMBA_OK = 0,
+  SAMBA_ERR_INVALID_ARG = 1,  /* NULL where data is required, bad size, workspace too small */
+  SAMBA_ERR_UNSUPPORTED = 2,  /* valid but not handled by these kernels (misaligned, N != 16, ...) */
+  SAMBA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed (launch, tensor-map encode) */
+  SAMBA_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up (from samba_get_error) */
+  SAMBA_ERR_DEVICE = 5        /* a device-side check failed (from samba_get_error) */
+} samba_status;
+
+typedef enum { SAMBA_F32 = 0, SAMBA_BF16 = 1 } samba_dtype;
+
+typedef void* samba_stream; /* cudaStream_t */
+
+/* Human-readable name of a status code (static string). */
+const char* samba_status_string(samba_status s);
+
+/* Library version string (static). */
+const char* samba_version(void);
+
+/* Synchronises `stream`, returns and clears the device error word of the
+ * current device: SAMBA_OK, SAMBA_ERR_TIMEOUT or SAMBA_ERR_DEVICE, or
+ * SAMBA_ERR_CUDA if the synchronisation itself failed. */
+samba_status samba_get_error(samba_stream stream);
+
+/* ------------------------------------------------------------------------
+ * Selective scan (S6)  [Samba 3.4 "The State Space Model Update (S6)",
+ *                        "Input-Dependent Selective Gating", "Gated Output"]
+ *
+ *   Delta_t = dt_softplus ? log(1 + exp(dt_t + dt_bias)) : dt_t (+ dt_bias)
+ *   h_t     = exp(Delta_t * A) (.) h_{t-1} + (Delta_t * u_t) * B_t,  A = -exp(A_log)
+ *   y_t     = <C_t, h_t> + Dskip * u_t,  then  y_t *= SiLU(z_t)  if z != NULL
+ *
+ *   u, dt, z, y : [B, L, D] dtype        Bm, Cm : [B, L, N] dtype
+ *   A_log       : [D, N] fp32            dt_bias, Dskip : [D] fp32 or NULL (0)
+ *   h0          : [B, D, N] fp32 initial state or NULL (zeros)
+ *   hT          : [B, D, N] fp32 state after the last token, or NULL
+ * Requirements: N == 16, D % 32 == 0, B >= 1, L >= 0.  L == 0 copies h0 (or
+ * zeros) into hT.  The state is kept in fp32 throughout.
+ * ---------------------------------------------------------------------- */
+size_t samba_selective_scan_workspace_size(int B, int L, int D, int N);
+
+samba_status samba_selective_scan(const void* u, const void* dt, const float* dt_bias, int dt_softplus,
+                                  const float* A_log, const void* Bm, const void* Cm, const float* Dskip,
+                                  const void* z, const float* h0, float* hT, void* y, int B, int L, int D,
+                                  int N, samba_dtype dtype, void* workspace, size_t workspace_bytes,
+                                  samba_stream stream);
+
+/* ------------------------------------------------------------------------
+ * Causal sliding-window attention with grouped-query heads and RoPE
+ *   [Samba 3.4 "Window Specification", "Positional Encoding", "Implementation"]
+ *
+ *   qr = RoPE(q, pos0 + t), kr = RoPE(k, pos0 + t)   (rope_base == 0: no rotation)
+ *   o[b,t,h] = sum_{s = max(0, t-window+1)}^{t} softmax_s(scale * qr[b,t,h] . kr[b,s,g(h)]) v[b,s,g(h)]
+ *   g(h) = h / (Hq / Hkv);  scale = softmax_scale > 0 ? softmax_scale : 1/sqrt(head_dim)
+ *
+ *   q, o : [B, L, Hq, head_dim] dtype      k, v : [B, L, Hkv, head_dim] dtype
+ * RoPE pairs channel i with i + head_dim/2 and uses theta_i = rope_base^(-2i/head_dim);
+ * angles are formed from fp64 tables so that positions up to 2^30 keep ~1e-7 rad.
+ * Requirements: Hq % Hkv == 0, head_dim in {16, 32, 64, 128}, window >= 1,
+ * pos0 >= 0, pos0 + L <= 2^30.  With rope_base != 0 the rotated copies of q and k
+ * live in the workspace.
+ * ---------------------------------------------------------------------- */
+size_t samba_swa_workspace_size(int B, int L, int Hq, int Hkv, int head_dim, float rope_base,
+                                samba_dtype dtype);
+
+samba_status samba_swa_fwd(const void* q, const void* k, const void* v, void* o, int B, int L, int Hq, int Hkv,
+                           int head_dim, int window, float rope_base, int64_t pos0, float softmax_scale,
+                           samba_dtype dtype, void* workspace, size_t workspace_bytes, samba_stream stream);
+
+/* ------------------------------------------------------------------------
+ * Building blocks of the block (also used by it)
+ * ---------------------------------------------------------------------- */
+
+/* RMSNorm [Samba 3.2]: out[r,:] = x[r,:] / sqrt(mean(x[r,:]^2) + eps) * g.
+ * x, out: [rows, dim] dtype (may alias); g: [dim] fp32.  dim % 8 == 0. */
+samba_status samba_rmsnorm(const void* x, const float* g, void* out, int64_t rows, int dim, float eps,
+                           samba_dtype dtype, samba_stream stream);
+
+/* Short convolution [Samba 3.4 "Input Projection and Short Convolution"]:
+ *   u[b,t,c] = SiLU( sum_{j<k} w[c,j] * x[b, t-(k-1)+j, c] + bias[c] ),  x before t = 0 is 0.
+ * x: [B, L, *] dtype with row stride ld_x elements (>= D); w: [D, k] fp32;
+ * bias: [D] fp32 or NULL; u: [B, L, D] dtype; conv_state: [B, D, k-1] dtype
+ * receiving the last k-1 inputs (oldest first; zeros where L < k-1), or NULL.
+ * Requirements: 2 <= k <= 8, D % 8 == 0. */
+samba_status samba_causal_conv1d(const void* x, int64_t ld_x, const float* w, const float* bias, void* u,
+                                 void* conv_state, int B, int L, int D, int k, samba_dtype dtype,
+                                 samba_stream stream);
+
+typedef enum {
+  SAMBA_EPI_NONE = 0,          /* out = x W^T */
+  SAMBA_EPI_RESIDUAL = 1,      /* out = resid + x W^T            (resid [M, N] dtype, may alias out) */
+  SAMBA_EPI_SWIGLU = 2,        /* out = (x W^T) * SiLU(x W2^T)   [Samba 3.4 "SwiGLU Formulation"] */
+  SAMBA_EPI_SOFTPLUS_BIAS = 3  /* out = log(1 + exp(x W^T + bias))  (bias [N] fp32) */
+} samba_epilogue;
+
+/* Dense projection out[M, N] = epilogue(x[M, K] W[N, K]^T) with fp32 accumulation.
+ * W2 only for SWIGLU ([N, K]); bias only for SOFTPLUS_BIAS; resid only for RESIDUAL.
+ * Requirements: K % 8 == 0, N % 8 == 0. */
+samba_status samba_linear(const void* x, const void* W, const void* W2, const float* bias, const void* resid,
+                          void* out, int64_t M, int N, int K, samba_epilogue epilogue, samba_dtype dtype,
+                          samba_stream stream);
+
+/* ------------------------------------------------------------------------
+ * The Samba block (prefill)                                  [Samba 3.2, 3.4]
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  int d_model;   /* model width d_m */
+  int d_inner;   /* Mamba expanded width d_e (2 d_m in the pages) */
+  int d_state;   /* SSM state size d_s (16) */
+  int d_conv;    /* short-conv kernel size k (4) */
+  int dt_rank;   /* low-rank Delta bottleneck d_r (d_m / 16) */
+  int n_q;       /* query heads */
+  int n_kv;      /* key/value heads (GQA groups) */
+  int head_dim;  /* per-head width */
+  int window;    /* sliding window w (keys t-w+1 .. t) */
+  int d_ff;      /* SwiGLU hidden width d_p */
+  float rope_base; /* RoPE base (10000); 0 disables RoPE */
+  float norm_eps;  /* RMSNorm epsilon */
+  samba_dtype dtype;
+} samba_block_config;
+
+typedef struct {
+  const float* norm_g[4]; /* [d_model] gains before Mamba, MLP1, SWA, MLP2 */
+  const void* W_in;       /* [2*d_inner, d_model]: rows [0,d_inner) = W_in (x branch), rest = W_g (gate z) */
+  const float* conv_w;    /* [d_inner, d_conv] */
+  const float* conv_b;    /* [d_inner] or NULL */
+  const void* W_x;        /* [dt_rank + 2*d_state, d_inner]: rows = W_r | W_b | W_c */
+  const void* W_dt;       /* [d_inner, dt_rank]  (W_q of the pages) */
+  const float* dt_bias;   /* [d_inner] */
+  const float* A_log;     /* [d_inner, d_state]; A = -exp(A_log) */
+  const float* Dskip;     /* [d_inner] */
+  const void* W_out;      /* [d_model, d_inner] */
+  const void* Wq;         /* [n_q*head_dim, d_model] */
+  const void* Wk;         /* [n_kv*head_dim, d_model] */
+  const void* Wv;         /* [n_kv*head_dim, d_model] */
+  const void* Wo;         /* [d_model, n_q*head_dim] */
+  const void* mlp1_W1;    /* [d_ff, d_model]  value branch */
+  const void* mlp1_W2;    /* [d_ff, d_model]  SiLU gate branch */
+  const void* mlp1_W3;    /* [d_model, d_ff] */
+  const void* mlp2_W1;
+  const void* mlp2_W2;
+  const void* mlp2_W3;
+} samba_block_weights;
+
+/* Decode state of one block, all caller-owned device buffers. */
+typedef struct {
+  float* ssm;     /* [B, d_inner, d_state] fp32 recurrent state */
+  void* conv;     /* [B, d_inner, d_conv-1] dtype: last d_conv-1 pre-conv inputs, oldest first */
+  void* k_ring;   /* [B, window, n_kv, head_dim] dtype: post-RoPE keys, slot = position mod window */
+  void* v_ring;   /* [B, window, n_kv, head_dim] dtype */
+  int64_t* pos;   /* [B] number of tokens seen so far (the next token's position) */
+} samba_decode_state;
+
+/* Optional taps of intermediate results (each NULL or [B, L, d_model] dtype). */
+typedef struct {
+  void* branch[4]; /* f(RMSNorm(x)) of Mamba, MLP1, SWA, MLP2, before the residual add */
+  void* resid[3];  /* residual stream after Mamba, MLP1, SWA (x_out is the fourth) */
+} samba_block_taps;
+
+size_t samba_block_workspace_size(const samba_block_config* cfg, int B, int L);
+
+/* One block over a fresh sequence (positions 0..L-1):
+ *   x1 = x  + Mamba(RMSNorm(x)); x2 = x1 + MLP1(RMSNorm(x1));
+ *   x3 = x2 + SWA(RMSNorm(x2));  x_out = x3 + MLP2(RMSNorm(x3)).
+ * x_in, x_out: [B, L, d_model] dtype (must not alias).  If st != NULL it is
+ * overwritten with the decode state after the last token (SSM state, the last
+ * d_conv-1 pre-conv inputs, the last min(L, window) post-RoPE keys/values in
+ * their ring slots, pos[b] = L).  taps may be NULL.
+ * Requirements: d_state == 16, head_dim == 64 for bf16 (16..128 for fp32),
+ * d_model, d_inner, d_ff multiples of 64, n_q % n_kv == 0. */
+samba_status samba_block_fwd(const samba_block_config* cfg, const samba_block_weights* w, const void* x_in,
+                             void* x_out, samba_decode_state* st, const samba_block_taps* taps, int B, int L,
+                             void* workspace, size_t workspace_bytes, samba_stream stream);
+
+/* ------------------------------------------------------------------------
+ * The Samba block, one decode step per sequence (constant cost per token;
+ * [Samba 5 / Figure 2b discussion of decoding; the blog page's ring-buffer KV])
+ *
+ * x_t, y_t: [B, d_model] dtype.  For each row b with p = pos[b]: the Mamba layer
+ * advances the conv state and the SSM state by one step; the SWA layer writes
+ * RoPE(k)/v at ring slot p mod window and attends over the min(p+1, window)
+ * most recent slots; pos[b] becomes p + 1.  All state updates are in place and
+ * read positions from device memory, so the call can be captured in a CUDA graph
+ * and replayed.
+ * ---------------------------------------------------------------------- */
+size_t samba_step_workspace_size(const samba_block_config* cfg, int B);
+
+samba_status samba_step(const samba_block_config* cfg, const samba_block_weights* w, const void* x_t, void* y_t,
+                        samba_decode_state* st, int B, void* workspace, size_t workspace_bytes,
+                        samba_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAMBA_H_ */

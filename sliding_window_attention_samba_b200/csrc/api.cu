@@ -1,0 +1,601 @@
+// C ABI of libsamba: validation, workspace carving and the launch sequences of
+// the Samba block prefill and decode step [Samba 3.2 "Big-Picture
+// Architecture"; 3.4 "Detailed, Sentence-Based Technical Breakdown"].
+#include <mutex>
+#include <set>
+#include <utility>
+#include <string.h>
+
+#include "common.cuh"
+#include "decode.h"
+#include "kernels.h"
+
+namespace samba {
+
+// ---------------------------------------------------------------------------
+// Device error word
+// ---------------------------------------------------------------------------
+__device__ int g_error_word = 0;
+
+int* device_error_word() {
+  static int* addr[64] = {nullptr};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<int*>(p);
+  }
+  return addr[dev];
+}
+
+// ---------------------------------------------------------------------------
+// Per-(kernel, device) record of raised shared-memory limits
+// ---------------------------------------------------------------------------
+static std::mutex g_attr_mu;
+static std::set<std::pair<const void*, int>> g_attr_done;
+bool smem_attr_done(const void* kern, int dev) {
+  std::lock_guard<std::mutex> lk(g_attr_mu);
+  return g_attr_done.count({kern, dev}) != 0;
+}
+void smem_attr_mark(const void* kern, int dev) {
+  std::lock_guard<std::mutex> lk(g_attr_mu);
+  g_attr_done.insert({kern, dev});
+}
+
+// ---------------------------------------------------------------------------
+// Tensor maps through the driver entry point (no link-time libcuda dependency)
+// ---------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool make_tmap(CUtensorMap* m, const void* base, samba_dtype dt, int rank, const uint64_t* dims,
+               const uint64_t* strides_elems, const uint32_t* box, CUtensorMapSwizzle swz) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const size_t es = dtype_size(dt);
+  cuuint64_t gdim[5], gstride[4];
+  cuuint32_t bdim[5], estride[5];
+  for (int i = 0; i < rank; ++i) {
+    gdim[i] = dims[i];
+    bdim[i] = box[i];
+    estride[i] = 1;
+  }
+  for (int i = 0; i < rank - 1; ++i) gstride[i] = strides_elems[i] * es;
+  CUresult r = fn(m, dt == SAMBA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                  (cuuint32_t)rank, const_cast<void*>(base), gdim, gstride, bdim, estride,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------------------
+// Workspace carving (256-byte aligned sub-buffers)
+// ---------------------------------------------------------------------------
+struct Carve {
+  size_t off = 0;
+  size_t take(size_t bytes) {
+    const size_t o = off;
+    off = (off + bytes + 255) & ~size_t(255);
+    return o;
+  }
+};
+
+struct BlockPlan {
+  size_t tab, xn, hz, u, xdbl, dlt, y, x1, x2, x3, hmlp, qkv, o, total;
+  int xdw, qkvw;
+};
+
+static BlockPlan plan_block(const samba_block_config& c, int64_t T) {
+  BlockPlan p;
+  const size_t es = dtype_size(c.dtype);
+  p.xdw = c.dt_rank + 2 * c.d_state;
+  p.qkvw = (c.n_q + 2 * c.n_kv) * c.head_dim;
+  Carve cv;
+  p.tab = cv.take(rope_table_bytes(c.head_dim));
+  p.xn = cv.take(T * c.d_model * es);
+  p.hz = cv.take(T * 2 * c.d_inner * es);
+  p.u = cv.take(T * c.d_inner * es);
+  p.xdbl = cv.take(T * p.xdw * es);
+  p.dlt = cv.take(T * c.d_inner * es);
+  p.y = cv.take(T * c.d_inner * es);
+  p.x1 = cv.take(T * c.d_model * es);
+  p.x2 = cv.take(T * c.d_model * es);
+  p.x3 = cv.take(T * c.d_model * es);
+  p.hmlp = cv.take(T * c.d_ff * es);
+  p.qkv = cv.take(T * p.qkvw * es);
+  p.o = cv.take(T * c.n_q * c.head_dim * es);
+  p.total = cv.off + 256;  // slack for aligning the caller's base pointer
+  return p;
+}
+
+static samba_status validate_cfg(const samba_block_config* c) {
+  if (!c) return SAMBA_ERR_INVALID_ARG;
+  if (c->d_model <= 0 || c->d_inner <= 0 || c->d_state <= 0 || c->d_conv <= 0 || c->dt_rank <= 0 || c->n_q <= 0 ||
+      c->n_kv <= 0 || c->head_dim <= 0 || c->window <= 0 || c->d_ff <= 0)
+    return SAMBA_ERR_INVALID_ARG;
+  if (c->dtype != SAMBA_F32 && c->dtype != SAMBA_BF16) return SAMBA_ERR_INVALID_ARG;
+  if (c->n_q % c->n_kv) return SAMBA_ERR_INVALID_ARG;
+  if (c->d_state != 16 || c->d_conv < 2 || c->d_conv > 8) return SAMBA_ERR_UNSUPPORTED;
+  if (c->head_dim != 16 && c->head_dim != 32 && c->head_dim != 64) return SAMBA_ERR_UNSUPPORTED;
+  if (c->d_model % 64 || c->d_inner % 64 || c->d_ff % 64) return SAMBA_ERR_UNSUPPORTED;
+  const size_t es = dtype_size(c->dtype);
+  if ((c->dt_rank * es) % 16) return SAMBA_ERR_UNSUPPORTED;
+  return SAMBA_OK;
+}
+
+static samba_status validate_weights(const samba_block_weights* w) {
+  if (!w) return SAMBA_ERR_INVALID_ARG;
+  const void* req[] = {w->norm_g[0], w->norm_g[1], w->norm_g[2], w->norm_g[3], w->W_in, w->conv_w, w->W_x,
+                       w->W_dt, w->dt_bias, w->A_log, w->Dskip, w->W_out, w->Wq, w->Wk, w->Wv, w->Wo,
+                       w->mlp1_W1, w->mlp1_W2, w->mlp1_W3, w->mlp2_W1, w->mlp2_W2, w->mlp2_W3};
+  for (const void* p : req)
+    if (!p) return SAMBA_ERR_INVALID_ARG;
+  for (const void* p : req)
+    if (!aligned16(p)) return SAMBA_ERR_UNSUPPORTED;
+  return SAMBA_OK;
+}
+
+#define TRY(x)                            \
+  do {                                    \
+    samba_status s_ = (x);                \
+    if (s_ != SAMBA_OK) return s_;        \
+  } while (0)
+
+static GemmArgs gemm1(const void* A, int64_t lda, const void* W, int64_t M, int N, int K, void* out, int64_t ldo,
+                      samba_dtype dt) {
+  GemmArgs g;
+  g.A = A;
+  g.lda = lda;
+  g.nseg = 1;
+  g.seg[0].W = W;
+  g.seg[0].n = N;
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.out = out;
+  g.ldo = ldo;
+  g.dtype = dt;
+  return g;
+}
+
+// SwiGLU MLP sub-layer: x_next = x + W3 ((W1 xn) * SiLU(W2 xn))  [Samba 3.4 "SwiGLU Formulation"]
+static samba_status mlp_sublayer(const samba_block_config& c, const float* g, const void* W1, const void* W2,
+                                 const void* W3, const void* x, void* x_next, void* xn, void* hmlp, void* tap,
+                                 int64_t T, cudaStream_t st) {
+  TRY(launch_rmsnorm(x, c.d_model, g, xn, c.d_model, T, c.d_model, c.norm_eps, c.dtype, st));
+  GemmArgs up = gemm1(xn, c.d_model, W1, T, c.d_ff, c.d_model, hmlp, c.d_ff, c.dtype);
+  up.seg[0].W2 = W2;
+  up.epi = kEpiSwiglu;
+  TRY(launch_gemm(up, st));
+  GemmArgs dn = gemm1(hmlp, c.d_ff, W3, T, c.d_model, c.d_ff, x_next, c.d_model, c.dtype);
+  dn.epi = kEpiResid;
+  dn.resid = x;
+  dn.ldr = c.d_model;
+  dn.tap = tap;
+  dn.ldt = c.d_model;
+  return launch_gemm(dn, st);
+}
+
+}  // namespace samba
+
+using namespace samba;
+
+extern "C" {
+
+const char* samba_status_string(samba_status s) {
+  switch (s) {
+    case SAMBA_OK: return "SAMBA_OK";
+    case SAMBA_ERR_INVALID_ARG: return "SAMBA_ERR_INVALID_ARG";
+    case SAMBA_ERR_UNSUPPORTED: return "SAMBA_ERR_UNSUPPORTED";
+    case SAMBA_ERR_CUDA: return "SAMBA_ERR_CUDA";
+    case SAMBA_ERR_TIMEOUT: return "SAMBA_ERR_TIMEOUT";
+    case SAMBA_ERR_DEVICE: return "SAMBA_ERR_DEVICE";
+  }
+  return "SAMBA_ERR_UNKNOWN";
+}
+
+const char* samba_version(void) { return "samba-b200 0.1 (sm_100a)"; }
+
+samba_status samba_get_error(samba_stream stream) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return SAMBA_ERR_CUDA;
+  int* w = device_error_word();
+  if (!w) return SAMBA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, w, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return SAMBA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(w, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return SAMBA_ERR_CUDA;
+  }
+  return v == kErrTimeout ? SAMBA_ERR_TIMEOUT : (v ? SAMBA_ERR_DEVICE : SAMBA_OK);
+}
+
+// ------------------------------------------------------------------ scan
+size_t samba_selective_scan_workspace_size(int, int, int, int) { return 0; }
+
+samba_status samba_selective_scan(const void* u, const void* dt, const float* dt_bias, int dt_softplus,
+                                  const float* A_log, const void* Bm, const void* Cm, const float* Dskip,
+                                  const void* z, const float* h0, float* hT, void* y, int B, int L, int D, int N,
+                                  samba_dtype dtype, void*, size_t, samba_stream stream) {
+  if (dtype != SAMBA_F32 && dtype != SAMBA_BF16) return SAMBA_ERR_INVALID_ARG;
+  ScanArgs a;
+  a.u = u;
+  a.dt = dt;
+  a.z = z;
+  a.Bm = Bm;
+  a.Cm = Cm;
+  a.y = y;
+  a.ld_u = a.ld_dt = a.ld_z = a.ld_y = D;
+  a.ld_bc = N;
+  a.dt_bias = dt_bias;
+  a.A_log = A_log;
+  a.Dskip = Dskip;
+  a.h0 = h0;
+  a.hT = hT;
+  a.B = B;
+  a.L = L;
+  a.D = D;
+  a.N = N;
+  a.softplus = dt_softplus != 0;
+  a.dtype = dtype;
+  return launch_selective_scan(a, (cudaStream_t)stream);
+}
+
+// ------------------------------------------------------------------ SWA
+size_t samba_swa_workspace_size(int B, int L, int Hq, int Hkv, int head_dim, float rope_base, samba_dtype dtype) {
+  if (rope_base == 0.f || B <= 0 || L <= 0) return 0;
+  Carve cv;
+  const size_t es = dtype_size(dtype);
+  cv.take(rope_table_bytes(head_dim));
+  cv.take((size_t)B * L * Hq * head_dim * es);
+  cv.take((size_t)B * L * Hkv * head_dim * es);
+  return cv.off + 256;
+}
+
+samba_status samba_swa_fwd(const void* q, const void* k, const void* v, void* o, int B, int L, int Hq, int Hkv,
+                           int head_dim, int window, float rope_base, int64_t pos0, float softmax_scale,
+                           samba_dtype dtype, void* workspace, size_t workspace_bytes, samba_stream stream) {
+  cudaStream_t st = (cudaStream_t)stream;
+  if (dtype != SAMBA_F32 && dtype != SAMBA_BF16) return SAMBA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !o || B < 1 || L < 0 || Hq < 1 || Hkv < 1 || window < 1 || pos0 < 0 || rope_base < 0.f)
+    return SAMBA_ERR_INVALID_ARG;
+  if (Hq % Hkv) return SAMBA_ERR_INVALID_ARG;
+  if (head_dim != 16 && head_dim != 32 && head_dim != 64 && head_dim != 128) return SAMBA_ERR_UNSUPPORTED;
+  if (pos0 + (int64_t)L > (int64_t(1) << 30)) return SAMBA_ERR_UNSUPPORTED;
+  if (L == 0) return SAMBA_OK;
+  SwaArgs a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.ld_q = (int64_t)Hq * head_dim;
+  a.ld_k = a.ld_v = (int64_t)Hkv * head_dim;
+  a.ld_o = (int64_t)Hq * head_dim;
+  a.B = B;
+  a.L = L;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.d = head_dim;
+  a.window = window;
+  a.scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)head_dim);
+  a.dtype = dtype;
+  if (rope_base != 0.f) {
+    const size_t need = samba_swa_workspace_size(B, L, Hq, Hkv, head_dim, rope_base, dtype);
+    if (!workspace || workspace_bytes < need) return SAMBA_ERR_INVALID_ARG;
+    char* base = (char*)(((uintptr_t)workspace + 255) & ~uintptr_t(255));
+    Carve cv;
+    const size_t es = dtype_size(dtype);
+    float2* tab = (float2*)(base + cv.take(rope_table_bytes(head_dim)));
+    void* qr = base + cv.take((size_t)B * L * Hq * head_dim * es);
+    void* kr = base + cv.take((size_t)B * L * Hkv * head_dim * es);
+    TRY(launch_build_rope_table(tab, head_dim, rope_base, st));
+    TRY(launch_rope_apply(q, qr, B, L, Hq, head_dim, pos0, tab, dtype, st));
+    TRY(launch_rope_apply(k, kr, B, L, Hkv, head_dim, pos0, tab, dtype, st));
+    a.q = qr;
+    a.k = kr;
+  }
+  return launch_swa(a, st);
+}
+
+// ------------------------------------------------------------------ pieces
+samba_status samba_rmsnorm(const void* x, const float* g, void* out, int64_t rows, int dim, float eps,
+                           samba_dtype dtype, samba_stream stream) {
+  return launch_rmsnorm(x, dim, g, out, dim, rows, dim, eps, dtype, (cudaStream_t)stream);
+}
+
+samba_status samba_causal_conv1d(const void* x, int64_t ld_x, const float* w, const float* bias, void* u,
+                                 void* conv_state, int B, int L, int D, int k, samba_dtype dtype,
+                                 samba_stream stream) {
+  ConvArgs a;
+  a.x = x;
+  a.ld_x = ld_x;
+  a.w = w;
+  a.bias = bias;
+  a.u = u;
+  a.state = conv_state;
+  a.B = B;
+  a.L = L;
+  a.D = D;
+  a.k = k;
+  a.dtype = dtype;
+  return launch_causal_conv(a, (cudaStream_t)stream);
+}
+
+samba_status samba_linear(const void* x, const void* W, const void* W2, const float* bias, const void* resid,
+                          void* out, int64_t M, int N, int K, samba_epilogue epilogue, samba_dtype dtype,
+                          samba_stream stream) {
+  if (K % 8 || N % 8) return SAMBA_ERR_UNSUPPORTED;
+  GemmArgs g = gemm1(x, K, W, M, N, K, out, N, dtype);
+  switch (epilogue) {
+    case SAMBA_EPI_NONE: g.epi = kEpiNone; break;
+    case SAMBA_EPI_RESIDUAL: g.epi = kEpiResid; g.resid = resid; g.ldr = N; break;
+    case SAMBA_EPI_SWIGLU: g.epi = kEpiSwiglu; g.seg[0].W2 = W2; break;
+    case SAMBA_EPI_SOFTPLUS_BIAS: g.epi = kEpiSoftplus; g.bias = bias; break;
+    default: return SAMBA_ERR_INVALID_ARG;
+  }
+  return launch_gemm(g, (cudaStream_t)stream);
+}
+
+// ------------------------------------------------------------------ block
+size_t samba_block_workspace_size(const samba_block_config* cfg, int B, int L) {
+  if (validate_cfg(cfg) != SAMBA_OK || B < 1 || L < 0) return 0;
+  return plan_block(*cfg, (int64_t)B * L).total;
+}
+
+samba_status samba_block_fwd(const samba_block_config* cfg, const samba_block_weights* w, const void* x_in,
+                             void* x_out, samba_decode_state* stt, const samba_block_taps* taps, int B, int L,
+                             void* workspace, size_t workspace_bytes, samba_stream stream) {
+  TRY(validate_cfg(cfg));
+  TRY(validate_weights(w));
+  if (!x_in || !x_out || B < 1 || L < 0 || x_in == x_out) return SAMBA_ERR_INVALID_ARG;
+  if (stt && (!stt->ssm || !stt->conv || !stt->k_ring || !stt->v_ring || !stt->pos)) return SAMBA_ERR_INVALID_ARG;
+  const samba_block_config& c = *cfg;
+  const int64_t T = (int64_t)B * L;
+  const BlockPlan P = plan_block(c, T);
+  if (!workspace || workspace_bytes < P.total) return SAMBA_ERR_INVALID_ARG;
+  if (!aligned16(x_in) || !aligned16(x_out)) return SAMBA_ERR_UNSUPPORTED;
+  cudaStream_t st = (cudaStream_t)stream;
+  const samba_dtype dt = c.dtype;
+  char* base = (char*)(((uintptr_t)workspace + 255) & ~uintptr_t(255));
+  auto buf = [&](size_t off) -> void* { return base + off; };
+  const int Di = c.d_inner, Dm = c.d_model, N = c.d_state, R = c.dt_rank;
+  const size_t es = dtype_size(dt);
+  void* x1 = (taps && taps->resid[0]) ? taps->resid[0] : buf(P.x1);
+  void* x2 = (taps && taps->resid[1]) ? taps->resid[1] : buf(P.x2);
+  void* x3 = (taps && taps->resid[2]) ? taps->resid[2] : buf(P.x3);
+  void* xn = buf(P.xn);
+  char* hz = (char*)buf(P.hz);
+  char* xdbl = (char*)buf(P.xdbl);
+  char* qkv = (char*)buf(P.qkv);
+  float2* tab = (float2*)buf(P.tab);
+
+  if (T == 0) {
+    if (stt) {
+      TRY(launch_pos_update(stt->pos, B, 0, true, st));
+      ScanArgs z;  // zero SSM state
+      (void)z;
+      cudaMemsetAsync(stt->ssm, 0, (size_t)B * Di * N * sizeof(float), st);
+      cudaMemsetAsync(stt->conv, 0, (size_t)B * Di * (c.d_conv - 1) * es, st);
+    }
+    return SAMBA_OK;
+  }
+
+  // ---- Mamba sub-layer [Samba 3.4 "The Mamba Layer"]
+  TRY(launch_rmsnorm(x_in, Dm, w->norm_g[0], xn, Dm, T, Dm, c.norm_eps, dt, st));
+  TRY(launch_gemm(gemm1(xn, Dm, w->W_in, T, 2 * Di, Dm, hz, 2 * Di, dt), st));  // H | X W_g
+  {
+    ConvArgs ca;
+    ca.x = hz;
+    ca.ld_x = 2 * Di;
+    ca.w = w->conv_w;
+    ca.bias = w->conv_b;
+    ca.u = buf(P.u);
+    ca.state = stt ? stt->conv : nullptr;
+    ca.B = B;
+    ca.L = L;
+    ca.D = Di;
+    ca.k = c.d_conv;
+    ca.dtype = dt;
+    TRY(launch_causal_conv(ca, st));
+  }
+  TRY(launch_gemm(gemm1(buf(P.u), Di, w->W_x, T, P.xdw, Di, xdbl, P.xdw, dt), st));  // dt_low | B | C
+  {
+    GemmArgs g = gemm1(xdbl, P.xdw, w->W_dt, T, Di, R, buf(P.dlt), Di, dt);  // Delta = softplus(.. + b)
+    g.epi = kEpiSoftplus;
+    g.bias = w->dt_bias;
+    TRY(launch_gemm(g, st));
+  }
+  {
+    ScanArgs a;
+    a.u = buf(P.u);
+    a.dt = buf(P.dlt);
+    a.z = hz + (size_t)Di * es;
+    a.Bm = xdbl + (size_t)R * es;
+    a.Cm = xdbl + (size_t)(R + N) * es;
+    a.y = buf(P.y);
+    a.ld_u = a.ld_dt = a.ld_y = Di;
+    a.ld_z = 2 * Di;
+    a.ld_bc = P.xdw;
+    a.A_log = w->A_log;
+    a.Dskip = w->Dskip;
+    a.hT = stt ? stt->ssm : nullptr;
+    a.B = B;
+    a.L = L;
+    a.D = Di;
+    a.N = N;
+    a.softplus = false;
+    a.dtype = dt;
+    TRY(launch_selective_scan(a, st));
+  }
+  {
+    GemmArgs g = gemm1(buf(P.y), Di, w->W_out, T, Dm, Di, x1, Dm, dt);
+    g.epi = kEpiResid;
+    g.resid = x_in;
+    g.ldr = Dm;
+    g.tap = taps ? taps->branch[0] : nullptr;
+    g.ldt = Dm;
+    TRY(launch_gemm(g, st));
+  }
+  // ---- MLP 1
+  TRY(mlp_sublayer(c, w->norm_g[1], w->mlp1_W1, w->mlp1_W2, w->mlp1_W3, x1, x2, xn, buf(P.hmlp),
+                   taps ? taps->branch[1] : nullptr, T, st));
+  // ---- SWA sub-layer [Samba 3.4 "The Sliding Window Attention (SWA) Layer"]
+  TRY(launch_rmsnorm(x2, Dm, w->norm_g[2], xn, Dm, T, Dm, c.norm_eps, dt, st));
+  const int hd = c.head_dim;
+  const int qw = c.n_q * hd, kvw = c.n_kv * hd;
+  {
+    GemmArgs g = gemm1(xn, Dm, w->Wq, T, P.qkvw, Dm, qkv, P.qkvw, dt);
+    g.nseg = 3;
+    g.seg[0].W = w->Wq;
+    g.seg[0].n = qw;
+    g.seg[1].W = w->Wk;
+    g.seg[1].n = kvw;
+    g.seg[2].W = w->Wv;
+    g.seg[2].n = kvw;
+    if (c.rope_base != 0.f) {
+      TRY(launch_build_rope_table(tab, hd, c.rope_base, st));
+      g.epi = kEpiRope;
+      g.rope_cols = qw + kvw;
+      g.head_dim = hd;
+      g.seq_len = L;
+      g.pos0 = 0;
+      g.rope_tab = tab;
+    }
+    TRY(launch_gemm(g, st));
+  }
+  {
+    SwaArgs a;
+    a.q = qkv;
+    a.k = qkv + (size_t)qw * es;
+    a.v = qkv + (size_t)(qw + kvw) * es;
+    a.o = buf(P.o);
+    a.ld_q = a.ld_k = a.ld_v = P.qkvw;
+    a.ld_o = qw;
+    a.B = B;
+    a.L = L;
+    a.Hq = c.n_q;
+    a.Hkv = c.n_kv;
+    a.d = hd;
+    a.window = c.window;
+    a.scale = 1.0f / sqrtf((float)hd);
+    a.dtype = dt;
+    TRY(launch_swa(a, st));
+  }
+  if (stt) TRY(launch_ring_fill(qkv, P.qkvw, qw, qw + kvw, stt->k_ring, stt->v_ring, B, L, c.window, kvw, dt, st));
+  {
+    GemmArgs g = gemm1(buf(P.o), qw, w->Wo, T, Dm, qw, x3, Dm, dt);
+    g.epi = kEpiResid;
+    g.resid = x2;
+    g.ldr = Dm;
+    g.tap = taps ? taps->branch[2] : nullptr;
+    g.ldt = Dm;
+    TRY(launch_gemm(g, st));
+  }
+  // ---- MLP 2
+  TRY(mlp_sublayer(c, w->norm_g[3], w->mlp2_W1, w->mlp2_W2, w->mlp2_W3, x3, x_out, xn, buf(P.hmlp),
+                   taps ? taps->branch[3] : nullptr, T, st));
+  if (stt) TRY(launch_pos_update(stt->pos, B, L, true, st));
+  return SAMBA_OK;
+}
+
+// ------------------------------------------------------------------ decode step
+size_t samba_step_workspace_size(const samba_block_config* cfg, int B) {
+  if (validate_cfg(cfg) != SAMBA_OK || B < 1) return 0;
+  return plan_block(*cfg, B).total;
+}
+
+samba_status samba_step(const samba_block_config* cfg, const samba_block_weights* w, const void* x_t, void* y_t,
+                        samba_decode_state* stt, int B, void* workspace, size_t workspace_bytes,
+                        samba_stream stream) {
+  TRY(validate_cfg(cfg));
+  TRY(validate_weights(w));
+  if (!x_t || !y_t || !stt || B < 1 || x_t == y_t) return SAMBA_ERR_INVALID_ARG;
+  if (!stt->ssm || !stt->conv || !stt->k_ring || !stt->v_ring || !stt->pos) return SAMBA_ERR_INVALID_ARG;
+  const samba_block_config& c = *cfg;
+  const BlockPlan P = plan_block(c, B);
+  if (!workspace || workspace_bytes < P.total) return SAMBA_ERR_INVALID_ARG;
+  if (!aligned16(x_t) || !aligned16(y_t)) return SAMBA_ERR_UNSUPPORTED;
+  cudaStream_t st = (cudaStream_t)stream;
+  const samba_dtype dt = c.dtype;
+  char* base = (char*)(((uintptr_t)workspace + 255) & ~uintptr_t(255));
+  auto buf = [&](size_t off) -> void* { return base + off; };
+  const int Di = c.d_inner, Dm = c.d_model, N = c.d_state, R = c.dt_rank;
+  const size_t es = dtype_size(dt);
+  void* xn = buf(P.xn);
+  char* hz = (char*)buf(P.hz);
+  char* xdbl = (char*)buf(P.xdbl);
+  char* qkv = (char*)buf(P.qkv);
+  float2* tab = (float2*)buf(P.tab);
+  void *x1 = buf(P.x1), *x2 = buf(P.x2), *x3 = buf(P.x3);
+
+  // ---- Mamba, one step
+  TRY(launch_rmsnorm(x_t, Dm, w->norm_g[0], xn, Dm, B, Dm, c.norm_eps, dt, st));
+  TRY(launch_gemm(gemm1(xn, Dm, w->W_in, B, 2 * Di, Dm, hz, 2 * Di, dt), st));
+  TRY(launch_conv_step(hz, 2 * Di, w->conv_w, w->conv_b, stt->conv, buf(P.u), B, Di, c.d_conv, dt, st));
+  TRY(launch_gemm(gemm1(buf(P.u), Di, w->W_x, B, P.xdw, Di, xdbl, P.xdw, dt), st));
+  {
+    GemmArgs g = gemm1(xdbl, P.xdw, w->W_dt, B, Di, R, buf(P.dlt), Di, dt);
+    g.epi = kEpiSoftplus;
+    g.bias = w->dt_bias;
+    TRY(launch_gemm(g, st));
+  }
+  TRY(launch_scan_step(buf(P.u), buf(P.dlt), hz + (size_t)Di * es, 2 * Di, xdbl, P.xdw, R, w->A_log, w->Dskip,
+                       stt->ssm, buf(P.y), B, Di, dt, st));
+  {
+    GemmArgs g = gemm1(buf(P.y), Di, w->W_out, B, Dm, Di, x1, Dm, dt);
+    g.epi = kEpiResid;
+    g.resid = x_t;
+    g.ldr = Dm;
+    TRY(launch_gemm(g, st));
+  }
+  TRY(mlp_sublayer(c, w->norm_g[1], w->mlp1_W1, w->mlp1_W2, w->mlp1_W3, x1, x2, xn, buf(P.hmlp), nullptr, B, st));
+  // ---- SWA over the ring
+  TRY(launch_rmsnorm(x2, Dm, w->norm_g[2], xn, Dm, B, Dm, c.norm_eps, dt, st));
+  const int hd = c.head_dim;
+  const int qw = c.n_q * hd, kvw = c.n_kv * hd;
+  {
+    GemmArgs g = gemm1(xn, Dm, w->Wq, B, P.qkvw, Dm, qkv, P.qkvw, dt);
+    g.nseg = 3;
+    g.seg[0].W = w->Wq;
+    g.seg[0].n = qw;
+    g.seg[1].W = w->Wk;
+    g.seg[1].n = kvw;
+    g.seg[2].W = w->Wv;
+    g.seg[2].n = kvw;
+    if (c.rope_base != 0.f) {
+      TRY(launch_build_rope_table(tab, hd, c.rope_base, st));
+      g.epi = kEpiRope;
+      g.rope_cols = qw + kvw;
+      g.head_dim = hd;
+      g.pos_dev = stt->pos;
+      g.rope_tab = tab;
+    }
+    TRY(launch_gemm(g, st));
+  }
+  TRY(launch_ring_write(qkv, P.qkvw, qw, qw + kvw, stt->pos, stt->k_ring, stt->v_ring, B, c.window, kvw, dt, st));
+  TRY(launch_attn_decode(qkv, P.qkvw, stt->pos, stt->k_ring, stt->v_ring, buf(P.o), B, c.n_q, c.n_kv, hd, c.window,
+                         1.0f / sqrtf((float)hd), dt, st));
+  {
+    GemmArgs g = gemm1(buf(P.o), qw, w->Wo, B, Dm, qw, x3, Dm, dt);
+    g.epi = kEpiResid;
+    g.resid = x2;
+    g.ldr = Dm;
+    TRY(launch_gemm(g, st));
+  }
+  TRY(mlp_sublayer(c, w->norm_g[3], w->mlp2_W1, w->mlp2_W2, w->mlp2_W3, x3, y_t, xn, buf(P.hmlp), nullptr, B, st));
+  return launch_pos_update(stt->pos, B, 1, false, st);
+}
+
+}  // extern "C"

@@ -1,0 +1,247 @@
+// HBM-bound helper kernels: RMSNorm, causal depthwise conv + SiLU, RoPE tables
+// and the standalone RoPE rotation.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace samba {
+
+// ===========================================================================
+// RMSNorm [Samba 3.2: every layer is preceded by an RMSNorm]
+//   out = x / sqrt(mean(x^2) + eps) * g
+// One warp per row; 8-element vector accesses; fp32 sum of squares.
+// ===========================================================================
+template <typename T>
+__global__ void rmsnorm_kernel(const T* __restrict__ x, int64_t ld_x, const float* __restrict__ g,
+                               T* __restrict__ out, int64_t ld_out, int64_t rows, int dim, float eps) {
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const T* xr = x + row * ld_x;
+  T* orow = out + row * ld_out;
+  float ss = 0.f;
+  for (int c = lane * 8; c < dim; c += 256) {
+    float f[8];
+    load8(xr + c, f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ss = fmaf(f[i], f[i], ss);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float r = rsqrtf(ss / (float)dim + eps);
+  for (int c = lane * 8; c < dim; c += 256) {
+    float f[8], gg[8];
+    load8(xr + c, f);
+    load8(g + c, gg);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) f[i] = f[i] * r * gg[i];
+    store8(orow + c, f);
+  }
+}
+
+samba_status launch_rmsnorm(const void* x, int64_t ld_x, const float* g, void* out, int64_t ld_out, int64_t rows,
+                            int dim, float eps, samba_dtype dt, cudaStream_t st) {
+  if (!x || !g || !out || rows < 0 || dim <= 0) return SAMBA_ERR_INVALID_ARG;
+  if (dim % 8 || ld_x % 8 || ld_out % 8 || !aligned16(x) || !aligned16(out) || !aligned16(g))
+    return SAMBA_ERR_UNSUPPORTED;
+  if (rows == 0) return SAMBA_OK;
+  const int warps = 8;
+  dim3 grid((unsigned)((rows + warps - 1) / warps));
+  if (dt == SAMBA_BF16)
+    rmsnorm_kernel<bf16><<<grid, warps * 32, 0, st>>>((const bf16*)x, ld_x, g, (bf16*)out, ld_out, rows, dim, eps);
+  else
+    rmsnorm_kernel<float><<<grid, warps * 32, 0, st>>>((const float*)x, ld_x, g, (float*)out, ld_out, rows, dim,
+                                                       eps);
+  SAMBA_CHECK_LAUNCH();
+  return SAMBA_OK;
+}
+
+// ===========================================================================
+// Short convolution [Samba 3.4 "Input Projection and Short Convolution"]
+//   u[b,t,c] = SiLU(sum_j w[c,j] x[b,t-(k-1)+j,c] + bias[c])
+// A thread owns 8 consecutive channels and a run of kRun tokens, keeping the
+// last k-1 inputs in registers (each input is read once from HBM per run plus
+// k-1 halo rows).  Also writes the conv state (last k-1 inputs) when asked.
+// ===========================================================================
+constexpr int kConvRun = 32;
+constexpr int kMaxK = 8;
+
+template <typename T, int K>
+__global__ void conv_silu_kernel(const T* __restrict__ x, int64_t ld_x, const float* __restrict__ w,
+                                 const float* __restrict__ bias, T* __restrict__ u, T* __restrict__ state, int L,
+                                 int D) {
+  const int cg = blockIdx.x * blockDim.x + threadIdx.x;  // channel group of 8
+  const int c0 = cg * 8;
+  const int t0 = blockIdx.y * kConvRun;
+  const int b = blockIdx.z;
+  if (c0 >= D) return;
+  float wr[8][K], bb[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+#pragma unroll
+    for (int j = 0; j < K; ++j) wr[i][j] = w[(size_t)(c0 + i) * K + j];
+    bb[i] = bias ? bias[c0 + i] : 0.f;
+  }
+  const T* xb = x + (size_t)b * L * ld_x + c0;
+  float hist[K][8];  // hist[j] = x[t-(K-1)+j]
+#pragma unroll
+  for (int j = 0; j < K - 1; ++j) {
+    const int t = t0 - (K - 1) + j;
+    if (t >= 0) load8(xb + (size_t)t * ld_x, hist[j]);
+    else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) hist[j][i] = 0.f;
+    }
+  }
+  const int tend = min(t0 + kConvRun, L);
+  for (int t = t0; t < tend; ++t) {
+    load8(xb + (size_t)t * ld_x, hist[K - 1]);
+    float o[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float acc = bb[i];
+#pragma unroll
+      for (int j = 0; j < K; ++j) acc = fmaf(wr[i][j], hist[j][i], acc);
+      if constexpr (sizeof(T) == 4) o[i] = acc * sigmoid_acc(acc);
+      else o[i] = acc * sigmoid_fast(acc);
+    }
+    store8(u + ((size_t)b * L + t) * D + c0, o);
+#pragma unroll
+    for (int j = 0; j < K - 1; ++j)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) hist[j][i] = hist[j + 1][i];
+  }
+  // conv state: the last K-1 inputs of the sequence, oldest first, [B, D, K-1]
+  if (state && t0 <= L - 1 && L - 1 < t0 + kConvRun) {
+    for (int j = 0; j < K - 1; ++j) {
+      const int t = L - (K - 1) + j;
+      float f[8];
+      if (t >= 0) load8(xb + (size_t)t * ld_x, f);
+      else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) f[i] = 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) state[((size_t)b * D + c0 + i) * (K - 1) + j] = Elt<T>::from_f(f[i]);
+    }
+  }
+}
+
+template <typename T>
+__global__ void conv_state_zero_kernel(T* state, size_t n) {
+  size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
+  if (i < n) state[i] = Elt<T>::from_f(0.f);
+}
+
+template <typename T, int K>
+samba_status launch_conv_k(const ConvArgs& a, cudaStream_t st) {
+  const int groups = a.D / 8;
+  dim3 block(128);
+  dim3 grid((groups + 127) / 128, (a.L + kConvRun - 1) / kConvRun, a.B);
+  conv_silu_kernel<T, K><<<grid, block, 0, st>>>((const T*)a.x, a.ld_x, a.w, a.bias, (T*)a.u, (T*)a.state, a.L,
+                                                 a.D);
+  SAMBA_CHECK_LAUNCH();
+  return SAMBA_OK;
+}
+
+template <typename T>
+samba_status launch_conv_t(const ConvArgs& a, cudaStream_t st) {
+  switch (a.k) {
+    case 2: return launch_conv_k<T, 2>(a, st);
+    case 3: return launch_conv_k<T, 3>(a, st);
+    case 4: return launch_conv_k<T, 4>(a, st);
+    case 5: return launch_conv_k<T, 5>(a, st);
+    case 6: return launch_conv_k<T, 6>(a, st);
+    case 7: return launch_conv_k<T, 7>(a, st);
+    case 8: return launch_conv_k<T, 8>(a, st);
+  }
+  return SAMBA_ERR_UNSUPPORTED;
+}
+
+samba_status launch_causal_conv(const ConvArgs& a, cudaStream_t st) {
+  if (!a.x || !a.w || !a.u || a.B < 1 || a.L < 0 || a.D < 1 || a.ld_x < a.D) return SAMBA_ERR_INVALID_ARG;
+  if (a.k < 2 || a.k > kMaxK || a.D % 8 || a.ld_x % 8 || !aligned16(a.x) || !aligned16(a.u))
+    return SAMBA_ERR_UNSUPPORTED;
+  if (a.L == 0) {
+    if (a.state) {
+      const size_t n = (size_t)a.B * a.D * (a.k - 1);
+      if (a.dtype == SAMBA_BF16) conv_state_zero_kernel<bf16><<<(unsigned)((n + 255) / 256), 256, 0, st>>>((bf16*)a.state, n);
+      else conv_state_zero_kernel<float><<<(unsigned)((n + 255) / 256), 256, 0, st>>>((float*)a.state, n);
+      SAMBA_CHECK_LAUNCH();
+    }
+    return SAMBA_OK;
+  }
+  return a.dtype == SAMBA_BF16 ? launch_conv_t<bf16>(a, st) : launch_conv_t<float>(a, st);
+}
+
+// ===========================================================================
+// RoPE tables [Samba 3.4 "Positional Encoding": base 10000, standard RoPE]
+//   tab[l][r][i] = (cos, sin)(r * 1024^l * theta_i),  theta_i = base^(-2i/d)
+// built in fp64 so that a position p = a*2^20 + b*2^10 + c is rotated by the
+// product of three table rotations with ~1e-7 rad error up to p < 2^30.
+// ===========================================================================
+size_t rope_table_bytes(int head_dim) {
+  return (size_t)kRopeLevels * kRopeRadix * (head_dim / 2) * sizeof(float2);
+}
+
+__global__ void build_rope_table_kernel(float2* tab, int half, int head_dim, double base) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  const int total = kRopeLevels * kRopeRadix * half;
+  if (idx >= total) return;
+  const int i = idx % half;
+  const int r = (idx / half) % kRopeRadix;
+  const int l = idx / (half * kRopeRadix);
+  const double theta = pow(base, -2.0 * (double)i / (double)head_dim);
+  const double scale = l == 0 ? 1.0 : (l == 1 ? 1024.0 : 1048576.0);
+  const double ang = (double)r * scale * theta;
+  double s, c;
+  sincos(ang, &s, &c);
+  tab[idx] = make_float2((float)c, (float)s);
+}
+
+samba_status launch_build_rope_table(float2* tab, int head_dim, float base, cudaStream_t st) {
+  const int half = head_dim / 2;
+  const int total = kRopeLevels * kRopeRadix * half;
+  build_rope_table_kernel<<<(total + 255) / 256, 256, 0, st>>>(tab, half, head_dim, (double)base);
+  SAMBA_CHECK_LAUNCH();
+  return SAMBA_OK;
+}
+
+template <typename T>
+__global__ void rope_apply_kernel(const T* __restrict__ x, T* __restrict__ out, int64_t rows, int L, int H,
+                                  int head_dim, int64_t pos0, const float2* __restrict__ tab) {
+  // one thread per (row, head, i < half)
+  const int half = head_dim / 2;
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t total = rows * H * half;
+  if (idx >= total) return;
+  const int i = (int)(idx % half);
+  const int64_t rh = idx / half;  // row * H + h
+  const int64_t row = rh / H;
+  const int64_t p = pos0 + row % L;
+  const float2 c0 = tab[(0 * kRopeRadix + (p & 1023)) * half + i];
+  const float2 c1 = tab[(1 * kRopeRadix + ((p >> 10) & 1023)) * half + i];
+  const float2 c2 = tab[(2 * kRopeRadix + ((p >> 20) & 1023)) * half + i];
+  float cr = c0.x * c1.x - c0.y * c1.y, sr = c0.x * c1.y + c0.y * c1.x;
+  const float cs = cr * c2.x - sr * c2.y, sn = cr * c2.y + sr * c2.x;
+  const T* xp = x + rh * head_dim;
+  const float a = Elt<T>::to_f(xp[i]), bq = Elt<T>::to_f(xp[i + half]);
+  T* op = out + rh * head_dim;
+  op[i] = Elt<T>::from_f(a * cs - bq * sn);
+  op[i + half] = Elt<T>::from_f(bq * cs + a * sn);
+}
+
+samba_status launch_rope_apply(const void* x, void* out, int B, int L, int H, int head_dim, int64_t pos0,
+                               const float2* tab, samba_dtype dt, cudaStream_t st) {
+  const int64_t rows = (int64_t)B * L;
+  const int64_t total = rows * H * (head_dim / 2);
+  if (total == 0) return SAMBA_OK;
+  const unsigned grid = (unsigned)((total + 255) / 256);
+  if (dt == SAMBA_BF16)
+    rope_apply_kernel<bf16><<<grid, 256, 0, st>>>((const bf16*)x, (bf16*)out, rows, L, H, head_dim, pos0, tab);
+  else
+    rope_apply_kernel<float><<<grid, 256, 0, st>>>((const float*)x, (float*)out, rows, L, H, head_dim, pos0, tab);
+  SAMBA_CHECK_LAUNCH();
+  return SAMBA_OK;
+}
+
+}  // namespace samba

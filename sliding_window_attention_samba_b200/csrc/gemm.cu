@@ -1,0 +1,513 @@
+// Dense projections out = epilogue(A W^T) of the Samba block: Mamba in/x/dt/out
+// projections, the SwiGLU MLP and the attention Q/K/V/O projections
+// [Samba 3.4: eqs. H = X W_in, Delta = Softplus(U W_r W_q + b), B = U W_b,
+// C = U W_c, O = (Y (.) SiLU(X W_g)) W_out, "SwiGLU Formulation"].
+//
+// Two kernels:
+//  * gemm_tc: bf16 operands, fp32 accumulation on the 5th-generation tensor
+//    cores.  Persistent, warp specialised (warp 0: TMA producer, warp 1: MMA
+//    issuer + TMEM owner, warps 2-5: epilogue).  A 4-stage ring of 128x64 A and
+//    up to 256x64 B tiles in 128-byte-swizzled shared memory feeds
+//    tcgen05.mma (M=128, N<=256, K=16) issued by one thread into a double
+//    buffered 2x256-column TMEM accumulator, so the epilogue of one tile
+//    overlaps the main loop of the next.  Epilogues (residual add, SwiGLU,
+//    softplus+bias, RoPE) are fused on the TMEM read-out.
+//  * gemm_simt: CUDA-core fp32 FMA tiles, used for fp32 data (no TF32: its
+//    ~1e-3 error would break the fp32 tolerance) and for shapes the tensor-core
+//    kernel does not take.
+#include <stdlib.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace samba {
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// Shared epilogue pieces
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int64_t rope_position(const GemmArgs& a, int64_t row) {
+  return a.pos_dev ? a.pos_dev[row] : a.pos0 + row % a.seq_len;
+}
+// (cos, sin) of p * theta_i from the three-level fp64-built table
+__device__ __forceinline__ float2 rope_cs(const float2* __restrict__ tab, int half, int64_t p, int i) {
+  const float2 c0 = tab[(0 * kRopeRadix + (p & 1023)) * half + i];
+  const float2 c1 = tab[(1 * kRopeRadix + ((p >> 10) & 1023)) * half + i];
+  const float2 c2 = tab[(2 * kRopeRadix + ((p >> 20) & 1023)) * half + i];
+  const float cr = c0.x * c1.x - c0.y * c1.y, sr = c0.x * c1.y + c0.y * c1.x;
+  return make_float2(cr * c2.x - sr * c2.y, cr * c2.y + sr * c2.x);
+}
+
+template <typename T>
+__device__ __forceinline__ float silu_t(float g) {
+  if constexpr (sizeof(T) == 4) return g * sigmoid_acc(g);
+  else return g * sigmoid_fast(g);
+}
+template <typename T>
+__device__ __forceinline__ float softplus_t(float x) {
+  if constexpr (sizeof(T) == 4) return softplus_acc(x);
+  else return softplus_fast(x);
+}
+
+__device__ __forceinline__ void seg_lookup(const GemmArgs& a, int n, int& s, int& row) {
+  int base = 0;
+  s = 0;
+  while (s < a.nseg - 1 && n >= base + a.seg[s].n) {
+    base += a.seg[s].n;
+    ++s;
+  }
+  row = n - base;
+}
+
+// ===========================================================================
+// CUDA-core kernel: 64x64 tile, 256 threads x (4x4) outputs, BK = 16
+// ===========================================================================
+constexpr int SB_M = 64, SB_N = 64, SB_K = 16;
+
+template <typename T, int EPI>
+__global__ void __launch_bounds__(256) gemm_simt_kernel(const GemmArgs a) {
+  __shared__ float As[SB_K][SB_M + 4];
+  __shared__ float Bs[SB_K][SB_N + 4];
+  __shared__ float B2s[EPI == kEpiSwiglu ? SB_K : 1][SB_N + 4];
+  __shared__ float Cs[SB_M][SB_N + 1];
+  const int tid = threadIdx.x;
+  const int64_t m0 = (int64_t)blockIdx.y * SB_M;
+  const int n0 = blockIdx.x * SB_N;
+  const T* A = (const T*)a.A;
+  const int ty = tid / 16, tx = tid % 16;
+  float acc[4][4] = {}, acc2[4][4] = {};
+
+  // loader coordinates: row lr (0..63), k offset lk (0,4,8,12)
+  const int lr = tid / 4, lk = (tid % 4) * 4;
+  const int64_t arow = m0 + lr;
+  const int bn = n0 + lr;
+  int bseg = 0, brow = 0;
+  if (bn < a.N) seg_lookup(a, bn, bseg, brow);
+  const T* Wrow = bn < a.N ? (const T*)a.seg[bseg].W + (size_t)brow * a.K : nullptr;
+  const T* W2row = (EPI == kEpiSwiglu && bn < a.N) ? (const T*)a.seg[bseg].W2 + (size_t)brow * a.K : nullptr;
+
+  for (int k0 = 0; k0 < a.K; k0 += SB_K) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int k = k0 + lk + j;
+      As[lk + j][lr] = (arow < a.M && k < a.K) ? Elt<T>::to_f(A[arow * a.lda + k]) : 0.f;
+      Bs[lk + j][lr] = (Wrow && k < a.K) ? Elt<T>::to_f(Wrow[k]) : 0.f;
+      if (EPI == kEpiSwiglu) B2s[lk + j][lr] = (W2row && k < a.K) ? Elt<T>::to_f(W2row[k]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < SB_K; ++kk) {
+      float av[4], bv[4], b2v[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        av[i] = As[kk][ty * 4 + i];
+        bv[i] = Bs[kk][tx * 4 + i];
+        if (EPI == kEpiSwiglu) b2v[i] = B2s[kk][tx * 4 + i];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+          if (EPI == kEpiSwiglu) acc2[i][j] = fmaf(av[i], b2v[j], acc2[i][j]);
+        }
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      Cs[ty * 4 + i][tx * 4 + j] = EPI == kEpiSwiglu ? acc[i][j] * silu_t<T>(acc2[i][j]) : acc[i][j];
+  __syncthreads();
+
+  T* out = (T*)a.out;
+  for (int e = tid; e < SB_M * SB_N; e += 256) {
+    const int r = e / SB_N, c = e % SB_N;
+    const int64_t row = m0 + r;
+    const int col = n0 + c;
+    if (row >= a.M || col >= a.N) continue;
+    float v = Cs[r][c];
+    if (EPI == kEpiResid) {
+      if (a.tap) ((T*)a.tap)[row * a.ldt + col] = Elt<T>::from_f(v);
+      v += Elt<T>::to_f(((const T*)a.resid)[row * a.ldr + col]);
+    } else if (EPI == kEpiSoftplus) {
+      v = softplus_t<T>(v + a.bias[col]);
+    } else if (EPI == kEpiRope) {
+      if (col < a.rope_cols) {
+        const int hd = a.head_dim, half = hd / 2;
+        const int j = col % hd;
+        const int cb = c - j;  // head start within the tile
+        const int i = j % half;
+        const float x1 = Cs[r][cb + i], x2 = Cs[r][cb + i + half];
+        const float2 cs = rope_cs(a.rope_tab, half, rope_position(a, row), i);
+        v = j < half ? x1 * cs.x - x2 * cs.y : x2 * cs.x + x1 * cs.y;
+      }
+    }
+    out[row * a.ldo + col] = Elt<T>::from_f(v);
+  }
+}
+
+template <typename T>
+samba_status simt_dispatch(const GemmArgs& a, cudaStream_t st) {
+  dim3 grid((a.N + SB_N - 1) / SB_N, (unsigned)((a.M + SB_M - 1) / SB_M));
+  switch (a.epi) {
+    case kEpiNone: gemm_simt_kernel<T, kEpiNone><<<grid, 256, 0, st>>>(a); break;
+    case kEpiResid: gemm_simt_kernel<T, kEpiResid><<<grid, 256, 0, st>>>(a); break;
+    case kEpiSwiglu: gemm_simt_kernel<T, kEpiSwiglu><<<grid, 256, 0, st>>>(a); break;
+    case kEpiSoftplus: gemm_simt_kernel<T, kEpiSoftplus><<<grid, 256, 0, st>>>(a); break;
+    case kEpiRope: gemm_simt_kernel<T, kEpiRope><<<grid, 256, 0, st>>>(a); break;
+    default: return SAMBA_ERR_INVALID_ARG;
+  }
+  SAMBA_CHECK_LAUNCH();
+  return SAMBA_OK;
+}
+
+// ===========================================================================
+// tcgen05 kernel
+// ===========================================================================
+constexpr int TC_BM = 128, TC_BK = 64, TC_STAGES = 4, TC_MAXN = 256;
+constexpr int TC_THREADS = 192;
+constexpr uint32_t TC_A_BYTES = TC_BM * TC_BK * 2;
+constexpr uint32_t TC_B_BYTES = TC_MAXN * TC_BK * 2;
+
+struct TcSmem {
+  bf16 A[TC_STAGES][TC_BM * TC_BK];
+  bf16 B[TC_STAGES][TC_MAXN * TC_BK];
+  uint64_t full[TC_STAGES], empty[TC_STAGES], tfull[2], tempty[2];
+  uint32_t tmem_base;
+};
+
+struct TcParams {
+  CUtensorMap tmA;
+  CUtensorMap tmB[3];
+  CUtensorMap tmB2;
+  GemmArgs a;
+  int bn;          // output columns per tile
+  int umma_n;      // accumulator columns per tile (2*bn for SwiGLU)
+  int n_tiles, m_tiles, k_blocks;
+  int seg_start[3];
+};
+
+__device__ __forceinline__ void tc_tile_coords(const TcParams& p, int tile, int& mt, int& nt) {
+  mt = tile / p.n_tiles;
+  nt = tile % p.n_tiles;
+}
+
+template <int EPI>
+__device__ __forceinline__ void tc_epilogue_tile(const TcParams& p, uint32_t tbase, int64_t row, int nt) {
+  const GemmArgs& a = p.a;
+  const bool in_range = row < a.M;
+  const int col0 = nt * p.bn;
+  bf16* out = (bf16*)a.out;
+  uint32_t r[32], r2[32];
+  if (EPI == kEpiSwiglu) {
+    for (int cc = 0; cc < p.bn; cc += 32) {
+      tmem_ld32(tbase + cc, r);
+      tmem_ld32(tbase + p.bn + cc, r2);
+      tmem_wait_ld();
+      if (in_range) {
+        float f[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float g = __uint_as_float(r2[i]);
+          f[i] = __uint_as_float(r[i]) * (g * sigmoid_fast(g));
+        }
+        bf16* o = out + row * a.ldo + col0 + cc;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) store8(o + 8 * i, f + 8 * i);
+      }
+    }
+    return;
+  }
+  if (EPI == kEpiRope && col0 < a.rope_cols) {
+    // heads of 64 columns: rotate (i, i+32) pairs
+    const int half = a.head_dim / 2;  // 32
+    const int64_t pos = in_range ? rope_position(a, row) : 0;
+    for (int hc = 0; hc < p.bn; hc += 2 * half) {
+      tmem_ld32(tbase + hc, r);
+      tmem_ld32(tbase + hc + half, r2);
+      tmem_wait_ld();
+      if (in_range) {
+        float lo[32], hi[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float2 cs = rope_cs(a.rope_tab, half, pos, i);
+          const float x1 = __uint_as_float(r[i]), x2 = __uint_as_float(r2[i]);
+          lo[i] = x1 * cs.x - x2 * cs.y;
+          hi[i] = x2 * cs.x + x1 * cs.y;
+        }
+        bf16* o = out + row * a.ldo + col0 + hc;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          store8(o + 8 * i, lo + 8 * i);
+          store8(o + half + 8 * i, hi + 8 * i);
+        }
+      }
+    }
+    return;
+  }
+  for (int cc = 0; cc < p.bn; cc += 32) {
+    tmem_ld32(tbase + cc, r);
+    tmem_wait_ld();
+    if (!in_range) continue;
+    float f[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(r[i]);
+    const int col = col0 + cc;
+    if (EPI == kEpiResid) {
+      if (a.tap) {
+        bf16* t = (bf16*)a.tap + row * a.ldt + col;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) store8(t + 8 * i, f + 8 * i);
+      }
+      const bf16* rs = (const bf16*)a.resid + row * a.ldr + col;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float g[8];
+        load8(rs + 8 * i, g);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) f[8 * i + j] += g[j];
+      }
+    } else if (EPI == kEpiSoftplus) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) f[i] = softplus_fast(f[i] + a.bias[col + i]);
+    }
+    bf16* o = out + row * a.ldo + col;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) store8(o + 8 * i, f + 8 * i);
+  }
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_constant__ TcParams p, int* err) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  TcSmem& S = *reinterpret_cast<TcSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = warp_id_sync();
+  const int lane = threadIdx.x & 31;
+  const int ntiles = p.m_tiles * p.n_tiles;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < TC_STAGES; ++s) {
+      mbar_init(&S.full[s], 1);
+      mbar_init(&S.empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&S.tfull[i], 1);
+      mbar_init(&S.tempty[i], 4);
+    }
+    fence_mbar_init();
+    tma_prefetch_desc(&p.tmA);
+    for (int i = 0; i < p.a.nseg; ++i) tma_prefetch_desc(&p.tmB[i]);
+    if (EPI == kEpiSwiglu) tma_prefetch_desc(&p.tmB2);
+  }
+  if (warp == 1) {
+    tmem_alloc(&S.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+
+  if (warp == 0) {
+    // ---------------- TMA producer
+    if (elect_one()) {
+      const uint32_t bytes = TC_A_BYTES + (uint32_t)p.umma_n * TC_BK * 2;
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        int mt, nt;
+        tc_tile_coords(p, tile, mt, nt);
+        int seg = 0;
+        while (seg < p.a.nseg - 1 && nt * p.bn >= p.seg_start[seg + 1]) ++seg;
+        const int brow = nt * p.bn - p.seg_start[seg];
+        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+          const int s = it % TC_STAGES;
+          const uint32_t j = it / TC_STAGES;
+          if (!mbar_wait(&S.empty[s], (j & 1) ^ 1, err)) { ok = false; break; }
+          mbar_arrive_expect_tx(&S.full[s], bytes);
+          tma_load_2d(S.A[s], &p.tmA, &S.full[s], kb * TC_BK, mt * TC_BM);
+          if (EPI == kEpiSwiglu) {
+            tma_load_2d(S.B[s], &p.tmB[0], &S.full[s], kb * TC_BK, brow);
+            tma_load_2d(S.B[s] + p.bn * TC_BK, &p.tmB2, &S.full[s], kb * TC_BK, brow);
+          } else {
+            tma_load_2d(S.B[s], &p.tmB[seg], &S.full[s], kb * TC_BK, brow);
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    const uint32_t idesc = idesc_bf16_f32(TC_BM, p.umma_n);
+    if (elect_one()) {
+      int it = 0, tc = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tc) {
+        const int acc = tc & 1;
+        const uint32_t use = tc >> 1;
+        if (!mbar_wait(&S.tempty[acc], (use & 1) ^ 1, err)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + acc * TC_MAXN;
+        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+          const int s = it % TC_STAGES;
+          const uint32_t j = it / TC_STAGES;
+          if (!mbar_wait(&S.full[s], j & 1, err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(S.A[s]);
+          const uint32_t b_base = smem_u32(S.B[s]);
+#pragma unroll
+          for (int k = 0; k < TC_BK / 16; ++k) {
+            const uint64_t ad = smem_desc(a_base + k * 32, 16, 1024, kLayoutSw128);
+            const uint64_t bd = smem_desc(b_base + k * 32, 16, 1024, kLayoutSw128);
+            umma_f16_ss(d_tmem, ad, bd, idesc, (kb | k) != 0);
+          }
+          umma_commit(&S.empty[s]);
+        }
+        if (ok) umma_commit(&S.tfull[acc]);
+      }
+    }
+  } else {
+    // ---------------- epilogue warps 2..5 -> TMEM lane quadrant warp % 4
+    const int q = warp & 3;
+    int tc = 0;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tc) {
+      int mt, nt;
+      tc_tile_coords(p, tile, mt, nt);
+      const int acc = tc & 1;
+      const uint32_t use = tc >> 1;
+      if (!mbar_wait(&S.tfull[acc], use & 1, err)) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem + acc * TC_MAXN + ((uint32_t)(q * 32) << 16);
+      const int64_t row = (int64_t)mt * TC_BM + q * 32 + lane;
+      tc_epilogue_tile<EPI>(p, tbase, row, nt);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.tempty[acc]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+bool tc_bn_for(const GemmArgs& a, int& bn) {
+  if (a.epi == kEpiSwiglu) {
+    bn = 128;
+    return a.nseg == 1 && a.N % 128 == 0;
+  }
+  if (a.nseg == 1 && a.N <= TC_MAXN && a.N % 32 == 0) {
+    bn = a.N;
+    return true;
+  }
+  for (int cand : {256, 128, 64, 32}) {
+    bool okc = true;
+    for (int s = 0; s < a.nseg; ++s) okc = okc && (a.seg[s].n % cand == 0);
+    if (okc) {
+      bn = cand;
+      return true;
+    }
+  }
+  return false;
+}
+
+template <int EPI>
+samba_status tc_launch(TcParams& p, cudaStream_t st) {
+  const size_t smem = sizeof(TcSmem) + 1024;
+  auto kern = gemm_tc_kernel<EPI>;
+  if (!ensure_smem_attr(kern, smem))
+    return SAMBA_ERR_CUDA;
+  const int ntiles = p.m_tiles * p.n_tiles;
+  const int grid = ntiles < num_sms() ? ntiles : num_sms();
+  kern<<<grid, TC_THREADS, smem, st>>>(p, device_error_word());
+  SAMBA_CHECK_LAUNCH();
+  return SAMBA_OK;
+}
+
+}  // namespace
+
+bool gemm_tc_supported(const GemmArgs& a) {
+  if (a.dtype != SAMBA_BF16 || a.K % TC_BK != 0 || a.lda % 8 || a.ldo % 8 || a.M < 1) return false;
+  if (!aligned16(a.A) || !aligned16(a.out)) return false;
+  int bn;
+  if (!tc_bn_for(a, bn)) return false;
+  if (a.epi == kEpiRope && (a.head_dim != 64 || a.rope_cols % 64 != 0)) return false;
+  if (a.epi == kEpiResid && (a.ldr % 8 || (a.tap && a.ldt % 8))) return false;
+  for (int s = 0; s < a.nseg; ++s)
+    if (!aligned16(a.seg[s].W) || (a.seg[s].W2 && !aligned16(a.seg[s].W2))) return false;
+  return true;
+}
+
+samba_status launch_gemm_tc(const GemmArgs& a, cudaStream_t st) {
+  if (!gemm_tc_supported(a)) return SAMBA_ERR_UNSUPPORTED;
+  TcParams p;
+  memset(&p, 0, sizeof(p));
+  p.a = a;
+  tc_bn_for(a, p.bn);
+  p.umma_n = a.epi == kEpiSwiglu ? 2 * p.bn : p.bn;
+  p.n_tiles = a.N / p.bn;
+  p.m_tiles = (int)((a.M + TC_BM - 1) / TC_BM);
+  p.k_blocks = a.K / TC_BK;
+  {
+    uint64_t dims[2] = {(uint64_t)a.K, (uint64_t)a.M};
+    uint64_t strides[1] = {(uint64_t)a.lda};
+    uint32_t box[2] = {TC_BK, TC_BM};
+    if (!make_tmap(&p.tmA, a.A, SAMBA_BF16, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return SAMBA_ERR_CUDA;
+  }
+  int start = 0;
+  const uint32_t brows = (uint32_t)(a.epi == kEpiSwiglu ? p.bn : p.bn);
+  for (int s = 0; s < a.nseg; ++s) {
+    p.seg_start[s] = start;
+    uint64_t dims[2] = {(uint64_t)a.K, (uint64_t)a.seg[s].n};
+    uint64_t strides[1] = {(uint64_t)a.K};
+    uint32_t box[2] = {TC_BK, brows};
+    if (!make_tmap(&p.tmB[s], a.seg[s].W, SAMBA_BF16, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return SAMBA_ERR_CUDA;
+    if (a.epi == kEpiSwiglu &&
+        !make_tmap(&p.tmB2, a.seg[s].W2, SAMBA_BF16, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return SAMBA_ERR_CUDA;
+    start += a.seg[s].n;
+  }
+  switch (a.epi) {
+    case kEpiNone: return tc_launch<kEpiNone>(p, st);
+    case kEpiResid: return tc_launch<kEpiResid>(p, st);
+    case kEpiSwiglu: return tc_launch<kEpiSwiglu>(p, st);
+    case kEpiSoftplus: return tc_launch<kEpiSoftplus>(p, st);
+    case kEpiRope: return tc_launch<kEpiRope>(p, st);
+  }
+  return SAMBA_ERR_INVALID_ARG;
+}
+
+samba_status launch_gemm_simt(const GemmArgs& a, cudaStream_t st) {
+  if (a.M == 0) return SAMBA_OK;
+  return a.dtype == SAMBA_BF16 ? simt_dispatch<bf16>(a, st) : simt_dispatch<float>(a, st);
+}
+
+static bool force_simt() {
+  const char* e = getenv("SAMBA_GEMM_KERNEL");
+  return e && e[0] == 's';
+}
+
+samba_status launch_gemm(const GemmArgs& a, cudaStream_t st) {
+  if (!a.A || !a.out || a.M < 0 || a.N <= 0 || a.K <= 0 || a.nseg < 1 || a.nseg > 3) return SAMBA_ERR_INVALID_ARG;
+  int nsum = 0;
+  for (int s = 0; s < a.nseg; ++s) {
+    if (!a.seg[s].W || a.seg[s].n <= 0) return SAMBA_ERR_INVALID_ARG;
+    if (a.epi == kEpiSwiglu && !a.seg[s].W2) return SAMBA_ERR_INVALID_ARG;
+    nsum += a.seg[s].n;
+  }
+  if (nsum != a.N) return SAMBA_ERR_INVALID_ARG;
+  if (a.epi == kEpiResid && !a.resid) return SAMBA_ERR_INVALID_ARG;
+  if (a.epi == kEpiSoftplus && !a.bias) return SAMBA_ERR_INVALID_ARG;
+  if (a.epi == kEpiRope && (!a.rope_tab || a.head_dim <= 0 || a.rope_cols % a.head_dim)) return SAMBA_ERR_INVALID_ARG;
+  if (a.M == 0) return SAMBA_OK;
+  if (!force_simt() && gemm_tc_supported(a)) return launch_gemm_tc(a, st);
+  if (a.epi == kEpiRope && 64 % a.head_dim != 0) return SAMBA_ERR_UNSUPPORTED;
+  return launch_gemm_simt(a, st);
+}
+
+}  // namespace samba

@@ -1,0 +1,113 @@
+// Internal launcher interfaces of libsamba (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/samba.h"
+
+namespace samba {
+
+// ---------------- selective scan ----------------
+struct ScanArgs {
+  const void* u = nullptr;
+  const void* dt = nullptr;
+  const void* z = nullptr;
+  const void* Bm = nullptr;
+  const void* Cm = nullptr;
+  void* y = nullptr;
+  int64_t ld_u = 0, ld_dt = 0, ld_z = 0, ld_bc = 0, ld_y = 0;  // row strides (elements)
+  const float* dt_bias = nullptr;
+  const float* A_log = nullptr;
+  const float* Dskip = nullptr;
+  const float* h0 = nullptr;
+  float* hT = nullptr;
+  int B = 0, L = 0, D = 0, N = 0;
+  bool softplus = true;
+  samba_dtype dtype = SAMBA_BF16;
+};
+samba_status validate_scan(const ScanArgs& a);
+samba_status launch_selective_scan(const ScanArgs& a, cudaStream_t st);
+
+// ---------------- RoPE ----------------
+// Table of (cos, sin) pairs: [3][1024][half] float2 for angle p * theta_i with
+// p = a*2^20 + b*2^10 + c; entries built in fp64.
+constexpr int kRopeLevels = 3;
+constexpr int kRopeRadix = 1024;
+size_t rope_table_bytes(int head_dim);
+samba_status launch_build_rope_table(float2* tab, int head_dim, float base, cudaStream_t st);
+// out[b,t,h,:] = RoPE(x[b,t,h,:], pos0 + t); x may alias out.
+samba_status launch_rope_apply(const void* x, void* out, int B, int L, int H, int head_dim, int64_t pos0,
+                               const float2* tab, samba_dtype dt, cudaStream_t st);
+
+// ---------------- RMSNorm ----------------
+samba_status launch_rmsnorm(const void* x, int64_t ld_x, const float* g, void* out, int64_t ld_out, int64_t rows,
+                            int dim, float eps, samba_dtype dt, cudaStream_t st);
+
+// ---------------- causal conv ----------------
+struct ConvArgs {
+  const void* x = nullptr;
+  int64_t ld_x = 0;
+  const float* w = nullptr;
+  const float* bias = nullptr;
+  void* u = nullptr;
+  void* state = nullptr;
+  int B = 0, L = 0, D = 0, k = 0;
+  samba_dtype dtype = SAMBA_BF16;
+};
+samba_status launch_causal_conv(const ConvArgs& a, cudaStream_t st);
+
+// ---------------- dense projections ----------------
+enum GemmEpi : int { kEpiNone = 0, kEpiResid = 1, kEpiSwiglu = 2, kEpiSoftplus = 3, kEpiRope = 4 };
+
+struct GemmSeg {
+  const void* W = nullptr;   // [n, K] row-major (row stride K)
+  const void* W2 = nullptr;  // SwiGLU gate weights [n, K]
+  int n = 0;                 // output columns of this segment
+};
+
+struct GemmArgs {
+  const void* A = nullptr;  // [M, K], row stride lda
+  int64_t lda = 0;
+  int nseg = 1;
+  GemmSeg seg[3];           // B operand, segments concatenated along N
+  int64_t M = 0;
+  int N = 0, K = 0;         // N = sum of seg[i].n
+  int epi = kEpiNone;
+  void* out = nullptr;      // [M, N], row stride ldo
+  int64_t ldo = 0;
+  const void* resid = nullptr;  // kEpiResid: out = resid + acc
+  int64_t ldr = 0;
+  void* tap = nullptr;          // kEpiResid: optional copy of acc (before the residual add)
+  int64_t ldt = 0;
+  const float* bias = nullptr;  // kEpiSoftplus
+  // kEpiRope: columns [0, rope_cols) are rotated per head of head_dim;
+  // position = pos_dev ? pos_dev[row] : pos0 + row % seq_len.
+  int rope_cols = 0, head_dim = 0, seq_len = 1;
+  int64_t pos0 = 0;
+  const int64_t* pos_dev = nullptr;
+  const float2* rope_tab = nullptr;
+  samba_dtype dtype = SAMBA_BF16;
+};
+samba_status launch_gemm(const GemmArgs& a, cudaStream_t st);       // picks the kernel
+samba_status launch_gemm_simt(const GemmArgs& a, cudaStream_t st);  // CUDA-core fp32 FMA kernel
+samba_status launch_gemm_tc(const GemmArgs& a, cudaStream_t st);    // tcgen05 kernel (bf16)
+bool gemm_tc_supported(const GemmArgs& a);
+
+// ---------------- sliding-window attention ----------------
+struct SwaArgs {
+  const void* q = nullptr;  // [B, L, Hq, d] rows of stride ld_q elements per token
+  const void* k = nullptr;  // [B, L, Hkv, d]
+  const void* v = nullptr;
+  void* o = nullptr;        // [B, L, Hq, d]
+  int64_t ld_q = 0, ld_k = 0, ld_v = 0, ld_o = 0;  // elements between consecutive tokens
+  int B = 0, L = 0, Hq = 0, Hkv = 0, d = 0, window = 0;
+  float scale = 0.f;
+  samba_dtype dtype = SAMBA_BF16;
+};
+samba_status launch_swa(const SwaArgs& a, cudaStream_t st);
+samba_status launch_swa_simt(const SwaArgs& a, cudaStream_t st);
+samba_status launch_swa_tc(const SwaArgs& a, cudaStream_t st);
+bool swa_tc_supported(const SwaArgs& a);
+
+}  // namespace samba

@@ -1,0 +1,299 @@
+// Chunked selective scan (S6) for sm_100a.
+//
+// Computes, per batch row b and channel d [Samba 3.4 "The State Space Model
+// Update (S6)", "Input-Dependent Selective Gating", "Gated Output"]:
+//   Delta_t = softplus(dt_t + bias)            (or dt_t + bias)
+//   h_t     = exp(Delta_t A) (.) h_{t-1} + Delta_t u_t B_t
+//   y_t     = <C_t, h_t> + D u_t,   y_t *= SiLU(z_t)
+//
+// Design (one CTA = 32 channels of one batch row, the whole sequence):
+//   * 64-token chunks of u, dt, z (32 channels wide) and B, C (16 wide) are
+//     staged through shared memory by TMA, NSTAGE deep.
+//   * 8 warps split each chunk in time: warp w owns tokens [8w, 8w+8), lane l
+//     owns channel l and its 16 fp32 states in registers.
+//   * Walk 1: each lane runs its 8 tokens from a zero state, keeping the 8x16
+//     decays exp(Delta A) in registers, and publishes (prod of decays, end state).
+//   * Combine: 256 threads each own two (channel, state) pairs and chain the
+//     8 warp aggregates sequentially from the carry of the previous chunk
+//     (kept in registers across chunks); this yields every warp's entry state.
+//   * Walk 2: each lane re-runs its tokens from the right entry state with the
+//     cached decays (one exp per element in total), emits y into a shared tile
+//     written back by a TMA store.
+// No inter-CTA communication, no workspace, no spin waits except the TMA
+// mbarrier waits (bounded, error word on timeout).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace samba {
+
+namespace {
+
+constexpr int kCh = 32;       // channels per CTA
+constexpr int kWarps = 8;     // time sub-chunks per chunk
+constexpr int kTs = 8;        // tokens per warp sub-chunk
+constexpr int kChunk = kWarps * kTs;  // 64 tokens
+constexpr int kN = 16;        // state size
+constexpr int kStages = 3;
+constexpr int kThreads = kWarps * 32;
+
+template <typename T>
+struct ScanSmem {
+  T u[kStages][kChunk * kCh];
+  T dt[kStages][kChunk * kCh];
+  T z[kStages][kChunk * kCh];
+  T Bm[kStages][kChunk * kN];
+  T Cm[kStages][kChunk * kN];
+  T y[2][kChunk * kCh];
+  float aggP[kWarps][kN][kCh];
+  float aggH[kWarps][kN][kCh];
+  uint64_t full[kStages];
+};
+
+template <typename T>
+__device__ __forceinline__ void load16(const T* p, float* f) {
+  load8(p, f);
+  load8(p + 8, f + 8);
+}
+
+template <typename T, bool kSoftplus, bool kHasZ>
+__global__ void __launch_bounds__(kThreads, 1)
+    scan_chunked_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_dt,
+                        const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_B,
+                        const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ CUtensorMap tm_y,
+                        const float* __restrict__ A_log, const float* __restrict__ dt_bias,
+                        const float* __restrict__ Dskip, const float* __restrict__ h0, float* __restrict__ hT,
+                        int L, int D, int* err) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  ScanSmem<T>& S = *reinterpret_cast<ScanSmem<T>*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const int d0 = blockIdx.x * kCh;
+  const int b = blockIdx.y;
+  const int d = d0 + lane;
+  const int nchunk = (L + kChunk - 1) / kChunk;
+
+  constexpr uint32_t kStageBytes = (3 * kChunk * kCh + 2 * kChunk * kN) * sizeof(T);
+  const uint32_t stage_bytes = kHasZ ? kStageBytes : kStageBytes - kChunk * kCh * sizeof(T);
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(&S.full[s], 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_u);
+    tma_prefetch_desc(&tm_dt);
+    tma_prefetch_desc(&tm_B);
+    tma_prefetch_desc(&tm_C);
+    tma_prefetch_desc(&tm_y);
+    if (kHasZ) tma_prefetch_desc(&tm_z);
+  }
+  __syncthreads();
+
+  auto issue = [&](int c) {
+    const int s = c % kStages;
+    const int t0 = c * kChunk;
+    mbar_arrive_expect_tx(&S.full[s], stage_bytes);
+    tma_load_3d(S.u[s], &tm_u, &S.full[s], d0, t0, b);
+    tma_load_3d(S.dt[s], &tm_dt, &S.full[s], d0, t0, b);
+    if (kHasZ) tma_load_3d(S.z[s], &tm_z, &S.full[s], d0, t0, b);
+    tma_load_3d(S.Bm[s], &tm_B, &S.full[s], 0, t0, b);
+    tma_load_3d(S.Cm[s], &tm_C, &S.full[s], 0, t0, b);
+  };
+  if (tid == 0)
+    for (int c = 0; c < kStages - 1 && c < nchunk; ++c) issue(c);
+
+  // Per-lane constants: A * log2(e) so that exp(Delta A) = 2^(Delta A log2 e).
+  float A2[kN];
+#pragma unroll
+  for (int n = 0; n < kN; ++n) A2[n] = -expf(A_log[(size_t)d * kN + n]) * 1.4426950408889634f;
+  const float bias = dt_bias ? dt_bias[d] : 0.f;
+  const float Dd = Dskip ? Dskip[d] : 0.f;
+
+  // Combine-role ownership: channel cl, states cn and cn+1; their carries.
+  const int cl = tid & 31;
+  const int cn = (tid >> 5) * 2;
+  float carry[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j)
+    carry[j] = h0 ? h0[((size_t)b * D + d0 + cl) * kN + cn + j] : 0.f;
+
+  bool ok = true;
+  for (int c = 0; c < nchunk; ++c) {
+    const int s = c % kStages;
+    if (tid == 0 && c + kStages - 1 < nchunk) issue(c + kStages - 1);
+    ok = mbar_wait(&S.full[s], (c / kStages) & 1, err);
+    if (__syncthreads_or(!ok)) break;
+
+    const int tb = warp * kTs;           // first token of this warp within the chunk
+    const int tg = c * kChunk + tb;      // global index of that token
+    float dA[kTs][kN];
+    float du[kTs];
+    float h[kN];
+#pragma unroll
+    for (int n = 0; n < kN; ++n) h[n] = 0.f;
+
+    // ---- walk 1: local scan from zero, decays cached
+#pragma unroll
+    for (int i = 0; i < kTs; ++i) {
+      const int row = tb + i;
+      float dtv = Elt<T>::to_f(S.dt[s][row * kCh + lane]) + bias;
+      float delta;
+      if (kSoftplus) {
+        if constexpr (sizeof(T) == 4) delta = softplus_acc(dtv);
+        else delta = softplus_fast(dtv);
+      } else {
+        delta = dtv;
+      }
+      float uv = Elt<T>::to_f(S.u[s][row * kCh + lane]);
+      if (tg + i >= L) { delta = 0.f; uv = 0.f; }
+      du[i] = delta * uv;
+      float Bt[kN];
+      load16(&S.Bm[s][row * kN], Bt);
+#pragma unroll
+      for (int n = 0; n < kN; ++n) {
+        dA[i][n] = ex2_approx(delta * A2[n]);
+        h[n] = fmaf(dA[i][n], h[n], du[i] * Bt[n]);
+      }
+    }
+#pragma unroll
+    for (int n = 0; n < kN; ++n) {
+      float p = dA[0][n];
+#pragma unroll
+      for (int i = 1; i < kTs; ++i) p *= dA[i][n];
+      S.aggP[warp][n][lane] = p;
+      S.aggH[warp][n][lane] = h[n];
+    }
+    __syncthreads();
+
+    // ---- combine across the 8 warps, chained from the previous chunk's carry
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      float H = carry[j];
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const float P = S.aggP[w][cn + j][cl];
+        const float hl = S.aggH[w][cn + j][cl];
+        S.aggH[w][cn + j][cl] = H;
+        H = fmaf(P, H, hl);
+      }
+      carry[j] = H;
+    }
+    if (tid == 0) tma_store_wait_read<1>();  // y tile (c & 1) free again
+    __syncthreads();
+
+    // ---- walk 2: exact states from the entry state, outputs
+#pragma unroll
+    for (int n = 0; n < kN; ++n) h[n] = S.aggH[warp][n][lane];
+    T* ytile = S.y[c & 1];
+#pragma unroll
+    for (int i = 0; i < kTs; ++i) {
+      const int row = tb + i;
+      float Bt[kN], Ct[kN];
+      load16(&S.Bm[s][row * kN], Bt);
+      load16(&S.Cm[s][row * kN], Ct);
+      float y = 0.f;
+#pragma unroll
+      for (int n = 0; n < kN; ++n) {
+        h[n] = fmaf(dA[i][n], h[n], du[i] * Bt[n]);
+        y = fmaf(Ct[n], h[n], y);
+      }
+      const float uv = Elt<T>::to_f(S.u[s][row * kCh + lane]);
+      y = fmaf(Dd, uv, y);
+      if (kHasZ) {
+        const float zv = Elt<T>::to_f(S.z[s][row * kCh + lane]);
+        if constexpr (sizeof(T) == 4) y *= zv * sigmoid_acc(zv);
+        else y *= zv * sigmoid_fast(zv);
+      }
+      ytile[row * kCh + lane] = Elt<T>::from_f(y);
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      tma_store_3d(&tm_y, ytile, d0, c * kChunk, b);
+      tma_store_commit();
+    }
+  }
+  if (tid == 0) tma_store_wait_all<0>();
+  if (ok && hT) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) hT[((size_t)b * D + d0 + cl) * kN + cn + j] = carry[j];
+  }
+}
+
+__global__ void copy_state_kernel(const float* __restrict__ h0, float* __restrict__ hT, size_t n) {
+  size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
+  if (i < n) hT[i] = h0 ? h0[i] : 0.f;
+}
+
+template <typename T>
+bool make_rows_map(CUtensorMap* m, const void* base, int64_t ld, int width, int box_w, int L, int B) {
+  const samba_dtype dt = Elt<T>::id;
+  uint64_t dims[3] = {(uint64_t)width, (uint64_t)L, (uint64_t)B};
+  uint64_t strides[2] = {(uint64_t)ld, (uint64_t)ld * (uint64_t)L};
+  uint32_t box[3] = {(uint32_t)box_w, (uint32_t)kChunk, 1};
+  return make_tmap(m, base, dt, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+template <typename T, bool kSoftplus, bool kHasZ>
+samba_status launch_typed(const ScanArgs& a, cudaStream_t st) {
+  CUtensorMap mu, mdt, mz, mB, mC, my;
+  bool ok = make_rows_map<T>(&mu, a.u, a.ld_u, a.D, kCh, a.L, a.B) &&
+            make_rows_map<T>(&mdt, a.dt, a.ld_dt, a.D, kCh, a.L, a.B) &&
+            make_rows_map<T>(&mB, a.Bm, a.ld_bc, kN, kN, a.L, a.B) &&
+            make_rows_map<T>(&mC, a.Cm, a.ld_bc, kN, kN, a.L, a.B) &&
+            make_rows_map<T>(&my, a.y, a.ld_y, a.D, kCh, a.L, a.B);
+  if (kHasZ) ok = ok && make_rows_map<T>(&mz, a.z, a.ld_z, a.D, kCh, a.L, a.B);
+  else mz = mu;
+  if (!ok) return SAMBA_ERR_CUDA;
+  const size_t smem = sizeof(ScanSmem<T>) + 128;
+  auto kern = scan_chunked_kernel<T, kSoftplus, kHasZ>;
+  if (!ensure_smem_attr(kern, smem))
+    return SAMBA_ERR_CUDA;
+  dim3 grid(a.D / kCh, a.B);
+  kern<<<grid, kThreads, smem, st>>>(mu, mdt, mz, mB, mC, my, a.A_log, a.dt_bias, a.Dskip, a.h0, a.hT, a.L, a.D,
+                                     device_error_word());
+  SAMBA_CHECK_LAUNCH();
+  return SAMBA_OK;
+}
+
+template <typename T>
+samba_status launch_dispatch(const ScanArgs& a, cudaStream_t st) {
+  if (a.softplus) {
+    return a.z ? launch_typed<T, true, true>(a, st) : launch_typed<T, true, false>(a, st);
+  }
+  return a.z ? launch_typed<T, false, true>(a, st) : launch_typed<T, false, false>(a, st);
+}
+
+}  // namespace
+
+samba_status validate_scan(const ScanArgs& a) {
+  if (!a.u || !a.dt || !a.A_log || !a.Bm || !a.Cm || !a.y) return SAMBA_ERR_INVALID_ARG;
+  if (a.B < 1 || a.L < 0 || a.D < 1 || a.N < 1) return SAMBA_ERR_INVALID_ARG;
+  if (a.N != kN || a.D % kCh != 0) return SAMBA_ERR_UNSUPPORTED;
+  const size_t es = dtype_size(a.dtype);
+  const void* ptrs[] = {a.u, a.dt, a.Bm, a.Cm, a.y, a.z};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return SAMBA_ERR_UNSUPPORTED;
+  const int64_t lds[] = {a.ld_u, a.ld_dt, a.ld_bc, a.ld_y, a.z ? a.ld_z : a.ld_u};
+  for (int64_t ld : lds)
+    if ((ld * (int64_t)es) % 16 != 0) return SAMBA_ERR_UNSUPPORTED;
+  if (a.ld_u < a.D || a.ld_dt < a.D || a.ld_y < a.D || a.ld_bc < a.N || (a.z && a.ld_z < a.D))
+    return SAMBA_ERR_INVALID_ARG;
+  return SAMBA_OK;
+}
+
+samba_status launch_selective_scan(const ScanArgs& a, cudaStream_t st) {
+  samba_status v = validate_scan(a);
+  if (v != SAMBA_OK) return v;
+  if (a.L == 0) {
+    if (a.hT) {
+      const size_t n = (size_t)a.B * a.D * a.N;
+      copy_state_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(a.h0, a.hT, n);
+      SAMBA_CHECK_LAUNCH();
+    }
+    return SAMBA_OK;
+  }
+  return a.dtype == SAMBA_BF16 ? launch_dispatch<bf16>(a, st) : launch_dispatch<float>(a, st);
+}
+
+}  // namespace samba

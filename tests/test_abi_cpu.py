@@ -1,0 +1,83 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point include/samba.h declares, and rejects bad arguments before
+touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "samba.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(samba_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sliding_window_attention_samba_b200 import _lib
+    return _lib
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 14
+    h = lib.lib_handle()
+    for n in names:
+        assert hasattr(h, n), n
+
+
+def test_status_strings_and_version(lib):
+    assert lib.samba_status_string(0) == "SAMBA_OK"
+    assert lib.samba_status_string(4) == "SAMBA_ERR_TIMEOUT"
+    assert "sm_100a" in lib.samba_version()
+
+
+def test_structs_match_header_layout(lib):
+    # 10 ints + 2 floats + enum
+    assert ctypes.sizeof(lib.BlockConfig) == 13 * 4
+    assert ctypes.sizeof(lib.BlockWeights) == 23 * 8
+    assert ctypes.sizeof(lib.DecodeState) == 5 * 8
+    assert ctypes.sizeof(lib.BlockTaps) == 7 * 8
+
+
+def test_workspace_sizes_host_only(lib):
+    from sliding_window_attention_samba_b200 import inputs as I
+    cfg = lib.make_config(I.WIDE)
+    small = lib.samba_block_workspace_size(cfg, 1, 128)
+    big = lib.samba_block_workspace_size(cfg, 4, 4096)
+    assert 0 < small < big
+    # tokens x (d_model*5 + 2 d_inner*... ) bytes: at least the in_proj output must fit
+    assert big >= 4 * 4096 * 2 * I.WIDE.d_inner * 2
+    bad = lib.make_config(I.WIDE)
+    bad.d_state = 8
+    assert lib.samba_block_workspace_size(bad, 1, 128) == 0
+    assert lib.samba_selective_scan_workspace_size(1, 4096, 4096, 16) == 0
+    assert lib.samba_swa_workspace_size(1, 4096, 32, 4, 64, 0.0, 1) == 0
+    assert lib.samba_swa_workspace_size(1, 4096, 32, 4, 64, 10000.0, 1) >= 4096 * 36 * 64 * 2
+
+
+def test_invalid_arguments_rejected_before_launch(lib):
+    h = lib.lib_handle()
+    # NULL inputs to the scan
+    rc = h.samba_selective_scan(None, None, None, 1, None, None, None, None, None, None, None, None,
+                                1, 16, 32, 16, 1, None, 0, None)
+    assert rc == 1
+    # unsupported state size (valid pointers are never dereferenced on this path)
+    fake = ctypes.c_void_p(1 << 20)
+    rc = h.samba_selective_scan(fake, fake, None, 1, fake, fake, fake, None, None, None, None, fake,
+                                1, 16, 32, 8, 1, None, 0, None)
+    assert rc == 2
+    # GQA heads must divide
+    rc = h.samba_swa_fwd(fake, fake, fake, fake, 1, 16, 6, 4, 64, 8, ctypes.c_float(0.0), 0,
+                         ctypes.c_float(0.0), 1, None, 0, None)
+    assert rc == 1
+    # block: missing weights
+    from sliding_window_attention_samba_b200 import inputs as I
+    cfg = lib.make_config(I.TINY)
+    w = lib.BlockWeights()
+    with pytest.raises(lib.SambaError):
+        lib.samba_block_fwd(cfg, w, 1 << 20, 2 << 20, None, None, 1, 8, 1 << 22, 1 << 30, 0)

@@ -1,0 +1,118 @@
+"""Selective scan (samba_selective_scan) against the fp64 oracle."""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import samba_oracle as O
+from sliding_window_attention_samba_b200 import inputs as I
+from tests.helpers import TOL, dev, host, rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def L():
+    import torch
+    from sliding_window_attention_samba_b200 import _lib
+    torch.cuda.init()
+    return _lib
+
+
+def run_scan(L_, r, dt, softplus=True, with_z=True, h0=None, want_hT=True):
+    import torch
+    Bn, Ln, D = r["u"].shape
+    N = r["B"].shape[-1]
+    u, dtt, Bm, Cm = dev(r["u"], dt), dev(r["dt_raw"], dt), dev(r["B"], dt), dev(r["C"], dt)
+    z = dev(r["z"], dt) if with_z else None
+    y = torch.empty(Bn, Ln, D, device="cuda", dtype=u.dtype)
+    hT = torch.empty(Bn, D, N, device="cuda") if want_hT else None
+    L_.samba_selective_scan(u, dtt, dev(r["dt_bias"]), softplus, dev(r["A_log"]), Bm, Cm, dev(r["D"]), z,
+                            dev(h0) if h0 is not None else None, hT, y, Bn, Ln, D, N,
+                            1 if dt == "bf16" else 0)
+    torch.cuda.synchronize()
+    assert L_.samba_get_error() == 0
+    return host(y), (host(hT) if want_hT else None)
+
+
+def oracle_scan(r, softplus=True, with_z=True, h0=None):
+    delta = r["dt_raw"] + r["dt_bias"]
+    if softplus:
+        delta = O.softplus(delta)
+    A = -np.exp(r["A_log"].astype(np.float64))
+    return O.selective_scan(r["u"], delta, A, r["B"], r["C"], r["D"], r["z"] if with_z else None, h0)
+
+
+@pytest.mark.parametrize("dt,Bn,Ln,D", [("f32", 1, 256, 128), ("f32", 2, 200, 64), ("bf16", 1, 4096, 4096),
+                                        ("bf16", 3, 129, 256), ("bf16", 1, 1, 32), ("f32", 1, 63, 32)])
+def test_scan_matches_oracle(L, dt, Bn, Ln, D):
+    r = I.scan_inputs(0, Bn, Ln, D, 16, dt, with_h0=True)
+    y, hT = run_scan(L, r, dt, h0=r["h0"])
+    yo, ho = oracle_scan(r, h0=r["h0"])
+    assert rel_err(y, yo) <= TOL[dt]
+    assert rel_err(hT, ho) <= TOL[dt]
+
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+def test_scan_no_gate_no_softplus(L, dt):
+    r = I.scan_inputs(5, 2, 300, 64, 16, dt)
+    r["dt_raw"] = I.round_to(np.abs(r["dt_raw"]) * 0.05, dt)  # Delta given directly (>0)
+    r["dt_bias"] = np.zeros_like(r["dt_bias"])
+    y, hT = run_scan(L, r, dt, softplus=False, with_z=False)
+    yo, ho = oracle_scan(r, softplus=False, with_z=False)
+    assert rel_err(y, yo) <= TOL[dt] and rel_err(hT, ho) <= TOL[dt]
+
+
+def test_scan_lti_closed_form_on_gpu(L):
+    Ln, D, N = 500, 32, 16
+    dlt, uv = 0.02, 0.5
+    Bv = np.linspace(-1, 1, N)
+    Cv = np.cos(np.arange(N))
+    r = {"u": np.full((1, Ln, D), uv, np.float32), "dt_raw": np.full((1, Ln, D), dlt, np.float32),
+         "B": np.tile(Bv, (1, Ln, 1)).astype(np.float32), "C": np.tile(Cv, (1, Ln, 1)).astype(np.float32),
+         "z": None, "dt_bias": np.zeros(D, np.float32), "A_log": I.a_log_init(D, N), "D": np.zeros(D, np.float32)}
+    y, _ = run_scan(L, r, "f32", softplus=False, with_z=False)
+    a = np.exp(-dlt * np.arange(1, N + 1))
+    Bv32, Cv32 = r["B"][0, 0].astype(np.float64), r["C"][0, 0].astype(np.float64)
+    for t in (0, 1, 63, 64, 65, 499):
+        h = np.float32(dlt) * Bv32 * np.float32(uv) * (1 - a ** (t + 1)) / (1 - a)
+        assert abs(y[0, t, 0] - h @ Cv32) <= 1e-4 * max(1.0, abs(h @ Cv32))
+
+
+def test_scan_impulse_prefix_is_exactly_zero(L):
+    r = I.scan_inputs(2, 1, 400, 64, 16, "bf16")
+    r["u"][:, :237] = 0.0
+    y, _ = run_scan(L, r, "bf16")
+    assert np.all(y[0, :237] == 0.0)
+    assert np.any(y[0, 237] != 0.0)
+
+
+def test_scan_chunk_split_carries_state(L):
+    r = I.scan_inputs(7, 2, 1000, 128, 16, "f32")
+    y_full, h_full = run_scan(L, r, "f32")
+    cut = 333
+    first = {k: (v[:, :cut] if (v is not None and v.ndim == 3 and k != "h0") else v) for k, v in r.items()}
+    rest = {k: (v[:, cut:] if (v is not None and v.ndim == 3 and k != "h0") else v) for k, v in r.items()}
+    y1, h1 = run_scan(L, first, "f32")
+    y2, h2 = run_scan(L, rest, "f32", h0=h1.astype(np.float32))
+    assert rel_err(np.concatenate([y1, y2], 1), y_full) <= 1e-5
+    assert rel_err(h2, h_full) <= 1e-5
+
+
+def test_scan_empty_sequence_copies_state(L):
+    import torch
+    h0 = np.random.default_rng(0).standard_normal((2, 64, 16)).astype(np.float32)
+    hT = torch.empty(2, 64, 16, device="cuda")
+    u = torch.zeros(16, device="cuda")
+    L.samba_selective_scan(u, u, None, 1, torch.zeros(64, 16, device="cuda"), u, u, None, None, dev(h0), hT, u,
+                           2, 0, 64, 16, 0)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(hT), h0)
+
+
+def test_scan_batch_rows_independent_bit_exact(L):
+    r = I.scan_inputs(9, 3, 257, 64, 16, "bf16")
+    y3, h3 = run_scan(L, r, "bf16")
+    one = {k: (v[1:2] if (v is not None and v.ndim == 3) else v) for k, v in r.items()}
+    y1, h1 = run_scan(L, one, "bf16")
+    assert np.array_equal(y3[1:2], y1) and np.array_equal(h3[1:2], h1)
