@@ -105,6 +105,26 @@ samba_status samba_swa_fwd(const void* q, const void* k, const void* v, void* o,
                            int head_dim, int window, float rope_base, int64_t pos0, float softmax_scale,
                            samba_dtype dtype, void* workspace, size_t workspace_bytes, samba_stream stream);
 
+/* Same computation and arguments as samba_swa_fwd, for callers that cannot
+ * allocate device memory: for instance a plugin running inside a host
+ * application that owns all device memory and gives the plugin no allocator, so
+ * it has no way to obtain a workspace.  The paper has no counterpart: this is a
+ * library convenience.
+ * The scratch it needs with rope_base != 0 (the rotation table and rotated copies
+ * of q and k) lives in a fixed 16 MiB device array inside the library, held on
+ * every GPU that loads the library until the process exits.  It fits when
+ *   round256(3*1024*(head_dim/2)*8) + round256(B*L*Hq*head_dim*esize)
+ *                                   + round256(B*L*Hkv*head_dim*esize) <= 16 MiB
+ * (esize 2 for bf16, 4 for fp32); larger calls return SAMBA_ERR_UNSUPPORTED and
+ * launch nothing.  No cudaMalloc/cudaFree or other allocation is made.
+ * The first call on each device looks up the array's device address (set-up);
+ * make that first call before any stream capture.  All calls share the array and
+ * it keeps the last call's contents (each call rewrites what it reads); calls that
+ * overlap on the GPU (other streams, other host threads) race on it. */
+samba_status samba_swa_fwd_noalloc(const void* q, const void* k, const void* v, void* o, int B, int L, int Hq,
+                                   int Hkv, int head_dim, int window, float rope_base, int64_t pos0,
+                                   float softmax_scale, samba_dtype dtype, samba_stream stream);
+
 /* ------------------------------------------------------------------------
  * Building blocks of the block (also used by it)
  * ---------------------------------------------------------------------- */

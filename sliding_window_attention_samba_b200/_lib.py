@@ -81,6 +81,9 @@ _swa_ws = _sig("samba_swa_workspace_size", c_size_t, [c_int, c_int, c_int, c_int
 _swa = _sig("samba_swa_fwd", c_int,
             [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_float, c_int64,
              c_float, c_int, c_void_p, c_size_t, c_void_p])
+_swa_noalloc = _sig("samba_swa_fwd_noalloc", c_int,
+                    [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_float,
+                     c_int64, c_float, c_int, c_void_p])
 _rmsnorm = _sig("samba_rmsnorm", c_int, [c_void_p, c_void_p, c_void_p, c_int64, c_int, c_float, c_int, c_void_p])
 _conv = _sig("samba_causal_conv1d", c_int,
              [c_void_p, c_int64, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int,
@@ -155,6 +158,13 @@ def samba_swa_fwd(q, k, v, o, B, L, Hq, Hkv, head_dim, window, rope_base, pos0, 
     _check("samba_swa_fwd",
            _swa(_p(q), _p(k), _p(v), _p(o), B, L, Hq, Hkv, head_dim, window, rope_base, pos0, softmax_scale, dtype,
                 _p(workspace), workspace_bytes, _stream(stream)))
+
+
+def samba_swa_fwd_noalloc(q, k, v, o, B, L, Hq, Hkv, head_dim, window, rope_base, pos0, softmax_scale, dtype,
+                          stream=None):
+    _check("samba_swa_fwd_noalloc",
+           _swa_noalloc(_p(q), _p(k), _p(v), _p(o), B, L, Hq, Hkv, head_dim, window, rope_base, pos0,
+                        softmax_scale, dtype, _stream(stream)))
 
 
 def samba_rmsnorm(x, g, out, rows, dim, eps, dtype, stream=None):
