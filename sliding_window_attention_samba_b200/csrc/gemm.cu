@@ -377,7 +377,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_con
       tc_tile_coords(p, tile, mt, nt);
       const int acc = tc & 1;
       const uint32_t use = tc >> 1;
-      if (!mbar_wait(&S.tfull[acc], use & 1, err)) break;
+      // tcgen05.ld in the epilogue is warp-collective: keep the wait warp-uniform
+      const bool got = mbar_wait(&S.tfull[acc], use & 1, err);
+      if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       const uint32_t tbase = tmem + acc * TC_MAXN + ((uint32_t)(q * 32) << 16);
       const int64_t row = (int64_t)mt * TC_BM + q * 32 + lane;

@@ -1,11 +1,318 @@
-// Tensor-core (tcgen05) sliding-window attention: placeholder until the
-// banded tcgen05 kernel lands; the CUDA-core kernel serves every case.
+// Banded sliding-window GQA attention on the 5th-generation tensor cores
+// [Samba 3.4 "Window Specification", "Implementation": query t attends keys
+// t-w+1 .. t; GQA kv head = h / (Hq/Hkv)].
+//
+// One CTA = one 128-query tile of one query head.  It visits only the 128-key
+// tiles that intersect the band of its queries (17 tiles for w = 2048), masks
+// just the two edge tiles, and keeps all matrix products on tcgen05:
+//   warp 0      TMA producer: Q once, then K_j and V_j per key tile (3 stages,
+//               128-byte swizzle, no multicast); the K/V rows are shared by the
+//               8 query heads of a group through L2.
+//   warp 1      owns TMEM (S0 | S1 | O) and issues, from one thread,
+//               S_j = Q K_j^T (M128 N128 K16 x4) into S[j%2] and
+//               O += P_j V_j  (M128 N64 K16 x8, V read MN-major).
+//   warps 2..5  softmax, one query row per thread (TMEM lane): S_j -> registers,
+//               band mask on edge tiles, online max/sum in the log2 domain,
+//               P_j = exp2(s - m) as bf16 into 128B-swizzled smem.  O is
+//               rescaled in TMEM only when the running max grows by more than
+//               2^8 (P then stays below 256), so the rescale is rare.
+//   epilogue    O / l -> bf16 -> global, by the softmax threads.
+// All waits are bounded (error word + early exit on timeout).
+#include <stdlib.h>
+#include <string.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
 namespace samba {
 
-bool swa_tc_supported(const SwaArgs&) { return false; }
-samba_status launch_swa_tc(const SwaArgs&, cudaStream_t) { return SAMBA_ERR_UNSUPPORTED; }
+namespace {
+
+constexpr int AT_BM = 128;       // queries per CTA
+constexpr int AT_BN = 128;       // keys per tile
+constexpr int AT_D = 64;         // head dim handled here
+constexpr int AT_STAGES = 3;     // K/V stages
+constexpr int AT_THREADS = 192;  // 6 warps
+constexpr float kRescaleThresh = 8.0f;  // log2 units
+
+constexpr uint32_t kTileBytes = AT_BM * AT_D * 2;  // 16 KB (Q, K or V tile)
+
+struct AtSmem {
+  bf16 Q[AT_BM * AT_D];
+  bf16 K[AT_STAGES][AT_BN * AT_D];
+  bf16 V[AT_STAGES][AT_BN * AT_D];
+  bf16 P[2][2][AT_BM * 64];  // [buffer][key half][row][64 keys], 128B-swizzled
+  uint64_t q_full;
+  uint64_t kv_full[AT_STAGES], kv_empty[AT_STAGES];
+  uint64_t s_full[2], s_free[2], p_full[2], pv_done[2];
+  uint32_t tmem_base;
+};
+
+struct AtParams {
+  CUtensorMap tmQ, tmK, tmV;
+  bf16* o;
+  int64_t ld_o;
+  int L, window, Hq, Hkv;
+  float scale_log2;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__global__ void __launch_bounds__(AT_THREADS, 1) swa_tc_kernel(const __grid_constant__ AtParams p, int* err) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  AtSmem& S = *reinterpret_cast<AtSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = warp_id_sync();
+  const int lane = threadIdx.x & 31;
+  const int t0 = blockIdx.x * AT_BM;
+  const int h = blockIdx.y;
+  const int b = blockIdx.z;
+  const int g = h / (p.Hq / p.Hkv);
+
+  // key tiles intersecting the band of rows t0 .. t0+127
+  const int lo = t0 - p.window + 1;
+  const int kb0 = lo <= 0 ? 0 : (lo / AT_BN) * AT_BN;
+  const int ntile = (t0 - kb0) / AT_BN + 1;
+
+  if (warp == 0 && lane == 0) {
+    mbar_init(&S.q_full, 1);
+    for (int s = 0; s < AT_STAGES; ++s) {
+      mbar_init(&S.kv_full[s], 1);
+      mbar_init(&S.kv_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&S.s_full[i], 1);
+      mbar_init(&S.s_free[i], 4);
+      mbar_init(&S.p_full[i], 4);
+      mbar_init(&S.pv_done[i], 1);
+    }
+    fence_mbar_init();
+    tma_prefetch_desc(&p.tmQ);
+    tma_prefetch_desc(&p.tmK);
+    tma_prefetch_desc(&p.tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(&S.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+  const uint32_t tO = tmem + 256;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (elect_one()) {
+      mbar_arrive_expect_tx(&S.q_full, kTileBytes);
+      tma_load_3d(S.Q, &p.tmQ, &S.q_full, h * AT_D, t0, b);
+      for (int j = 0; j < ntile; ++j) {
+        const int s = j % AT_STAGES;
+        const uint32_t use = j / AT_STAGES;
+        if (!mbar_wait(&S.kv_empty[s], (use & 1) ^ 1, err)) break;
+        mbar_arrive_expect_tx(&S.kv_full[s], 2 * kTileBytes);
+        const int kb = kb0 + j * AT_BN;
+        tma_load_3d(S.K[s], &p.tmK, &S.kv_full[s], g * AT_D, kb, b);
+        tma_load_3d(S.V[s], &p.tmV, &S.kv_full[s], g * AT_D, kb, b);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t idesc_s = idesc_bf16_f32(AT_BM, AT_BN, false);
+    const uint32_t idesc_o = idesc_bf16_f32(AT_BM, AT_D, true);  // V is N-contiguous (MN-major B)
+    if (elect_one()) {
+      bool ok = mbar_wait(&S.q_full, 0, err);
+      const uint32_t q_base = smem_u32(S.Q);
+      auto issue_s = [&](int j) -> bool {
+        const int s = j % AT_STAGES;
+        if (!mbar_wait(&S.kv_full[s], (j / AT_STAGES) & 1, err)) return false;
+        if (j >= 2 && !mbar_wait(&S.s_free[j & 1], ((j - 2) >> 1) & 1, err)) return false;
+        tc_fence_after();
+        const uint32_t k_base = smem_u32(S.K[s]);
+#pragma unroll
+        for (int k = 0; k < AT_D / 16; ++k)
+          umma_f16_ss((tmem + ((j & 1) ? 128u : 0u)), smem_desc(q_base + k * 32, 16, 1024, kLayoutSw128),
+                      smem_desc(k_base + k * 32, 16, 1024, kLayoutSw128), idesc_s, k != 0);
+        umma_commit(&S.s_full[j & 1]);
+        return true;
+      };
+      auto issue_pv = [&](int j) -> bool {
+        const int s = j % AT_STAGES;
+        if (!mbar_wait(&S.p_full[j & 1], (j >> 1) & 1, err)) return false;
+        tc_fence_after();
+        const uint32_t v_base = smem_u32(S.V[s]);
+#pragma unroll
+        for (int k = 0; k < AT_BN / 16; ++k) {
+          const uint32_t a_addr = smem_u32(S.P[j & 1][k >> 2]) + (k & 3) * 32;
+          const uint32_t b_addr = v_base + k * 16 * AT_D * 2;  // 16 keys x 128 B
+          umma_f16_ss(tO, smem_desc(a_addr, 16, 1024, kLayoutSw128), smem_desc(b_addr, 16, 1024, kLayoutSw128),
+                      idesc_o, (j | k) != 0);
+        }
+        umma_commit(&S.kv_empty[s]);
+        umma_commit(&S.pv_done[j & 1]);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int j = 0; ok && j < ntile; ++j) {
+        if (j + 1 < ntile) ok = issue_s(j + 1);
+        if (ok) ok = issue_pv(j);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warps
+    // Every tcgen05.ld/st below is warp-collective (.sync.aligned): the waits in
+    // front of them and the rescale decision are made warp-uniform.
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;  // query row within the tile == TMEM lane
+    const int t = t0 + r;
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
+      const bool w = mbar_wait(bar, par, err);
+      return __all_sync(0xffffffffu, w);
+    };
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < ntile; ++j) {
+      const int kb = kb0 + j * AT_BN;
+      const uint32_t tSj = tmem + ((j & 1) ? 128u : 0u);
+      if (!wait_all(&S.s_full[j & 1], (j >> 1) & 1)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sr[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tSj + lane_off + c * 32, sr + c * 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.s_free[j & 1]);
+
+      const bool edge = (kb + AT_BN - 1 > t0) || (kb < t0 + AT_BM - p.window);
+      float mt = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 128; ++i) {
+        float x = __uint_as_float(sr[i]) * p.scale_log2;
+        if (edge) {
+          const int s = kb + i;
+          if (s > t || s <= t - p.window || t >= p.L) x = -INFINITY;
+        }
+        sr[i] = __float_as_uint(x);
+        mt = fmaxf(mt, x);
+      }
+      // Online max with conditional rescale: a row moves its reference max only
+      // when the tile max exceeds it by more than 2^8; O is then rescaled in TMEM.
+      const bool need = mt > m_run + kRescaleThresh;
+      float alpha = 1.f;
+      if (need) {
+        if (m_run != -INFINITY) alpha = exp2f(m_run - mt);
+        l_run *= alpha;
+        m_run = mt;
+      }
+      if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        if (!wait_all(&S.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t orr[64];
+        tmem_ld32(tO + lane_off, orr);
+        tmem_ld32(tO + lane_off + 32, orr + 32);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 64; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
+        tmem_st16(tO + lane_off, orr);
+        tmem_st16(tO + lane_off + 16, orr + 16);
+        tmem_st16(tO + lane_off + 32, orr + 32);
+        tmem_st16(tO + lane_off + 48, orr + 48);
+        tmem_wait_st();
+      }
+      const float msub = m_run == -INFINITY ? 0.f : m_run;
+      // P buffer j%2 was last read by PV_{j-2}
+      if (j >= 2 && !wait_all(&S.pv_done[j & 1], ((j - 2) >> 1) & 1)) { ok = false; break; }
+      float ls = 0.f;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        unsigned char* prow = reinterpret_cast<unsigned char*>(S.P[j & 1][half]) + r * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          float e[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            e[q] = ex2_approx(__uint_as_float(sr[half * 64 + c * 8 + q]) - msub);
+            ls += e[q];
+          }
+          uint4 v4 = make_uint4(pack_bf16(e[0], e[1]), pack_bf16(e[2], e[3]), pack_bf16(e[4], e[5]),
+                                pack_bf16(e[6], e[7]));
+          *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = v4;
+        }
+      }
+      l_run += ls;
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.p_full[j & 1]);
+    }
+    // epilogue: wait for the last P.V, then O / l
+    if (ok && wait_all(&S.pv_done[(ntile - 1) & 1], ((ntile - 1) >> 1) & 1)) {
+      tc_fence_after();
+      uint32_t orr[64];
+      tmem_ld32(tO + lane_off, orr);
+      tmem_ld32(tO + lane_off + 32, orr + 32);
+      tmem_wait_ld();
+      if (t < p.L && l_run > 0.f) {
+        const float inv = 1.f / l_run;
+        bf16* op = p.o + ((int64_t)b * p.L + t) * p.ld_o + (int64_t)h * AT_D;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          float f[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) f[q] = __uint_as_float(orr[c * 8 + q]) * inv;
+          store8(op + c * 8, f);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+bool make_head_map(CUtensorMap* m, const void* base, int64_t ld, int H, int L, int B) {
+  uint64_t dims[3] = {(uint64_t)H * AT_D, (uint64_t)L, (uint64_t)B};
+  uint64_t strides[2] = {(uint64_t)ld, (uint64_t)ld * (uint64_t)L};
+  uint32_t box[3] = {AT_D, 128, 1};
+  return make_tmap(m, base, SAMBA_BF16, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+}  // namespace
+
+bool swa_tc_supported(const SwaArgs& a) {
+  if (a.dtype != SAMBA_BF16 || a.d != AT_D) return false;
+  if (a.ld_q % 8 || a.ld_k % 8 || a.ld_v % 8 || a.ld_o % 8) return false;
+  if (!aligned16(a.q) || !aligned16(a.k) || !aligned16(a.v) || !aligned16(a.o)) return false;
+  if (getenv("SAMBA_SWA_KERNEL") && getenv("SAMBA_SWA_KERNEL")[0] == 's') return false;
+  return true;
+}
+
+samba_status launch_swa_tc(const SwaArgs& a, cudaStream_t st) {
+  AtParams p;
+  memset(&p, 0, sizeof(p));
+  if (!make_head_map(&p.tmQ, a.q, a.ld_q, a.Hq, a.L, a.B) || !make_head_map(&p.tmK, a.k, a.ld_k, a.Hkv, a.L, a.B) ||
+      !make_head_map(&p.tmV, a.v, a.ld_v, a.Hkv, a.L, a.B))
+    return SAMBA_ERR_CUDA;
+  p.o = (bf16*)a.o;
+  p.ld_o = a.ld_o;
+  p.L = a.L;
+  p.window = a.window;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  const size_t smem = sizeof(AtSmem) + 1024;
+  if (!ensure_smem_attr(swa_tc_kernel, smem)) return SAMBA_ERR_CUDA;
+  dim3 grid((a.L + AT_BM - 1) / AT_BM, a.Hq, a.B);
+  swa_tc_kernel<<<grid, AT_THREADS, smem, st>>>(p, device_error_word());
+  SAMBA_CHECK_LAUNCH();
+  return SAMBA_OK;
+}
 
 }  // namespace samba

@@ -115,3 +115,19 @@ def test_swa_gqa_equals_repeated_kv(L):
     o = run_swa(L, r["q"], r["k"], r["v"], 50, 10000.0, 0, "f32")
     o_mha = run_swa(L, r["q"], np.repeat(r["k"], 4, 2), np.repeat(r["v"], 4, 2), 50, 10000.0, 0, "f32")
     assert rel_err(o, o_mha) <= 1e-6
+
+
+@pytest.mark.parametrize("Bn,Ln,w", [(1, 1000, 2048), (2, 777, 128), (1, 2500, 300), (1, 130, 1)])
+def test_swa_tensor_core_kernel_matches_cuda_core_kernel(L, Bn, Ln, w):
+    """The tcgen05 kernel (default for bf16, head_dim 64) against the CUDA-core
+    kernel on the same bf16 inputs: both accumulate in fp32; they differ by the
+    bf16 rounding of P on the tensor-core path."""
+    import os
+    r = I.swa_inputs(9, Bn, Ln, 8, 2, 64, "bf16")
+    o_tc = run_swa(L, r["q"], r["k"], r["v"], w, 10000.0, 0, "bf16")
+    os.environ["SAMBA_SWA_KERNEL"] = "simt"
+    try:
+        o_simt = run_swa(L, r["q"], r["k"], r["v"], w, 10000.0, 0, "bf16")
+    finally:
+        del os.environ["SAMBA_SWA_KERNEL"]
+    assert rel_err(o_tc, o_simt) <= 1e-2
