@@ -179,11 +179,12 @@ def attribution_pass(torch, L, s, blocks, x, T, Bn, Ln, reps=2):
     bf = torch.bfloat16
     st = torch.cuda.current_stream()
     w, _ = blocks[0]
-    xn = torch.empty(T, s.d_model, device=dev, dtype=bf)
-    hz = torch.empty(T, 2 * s.d_inner, device=dev, dtype=bf)
-    u = torch.empty(T, s.d_inner, device=dev, dtype=bf)
-    xdbl = torch.empty(T, s.dt_rank + 2 * s.d_state, device=dev, dtype=bf)
-    dlt = torch.empty(T, s.d_inner, device=dev, dtype=bf)
+    # realistic operand values: N(0,1) activations, step sizes Delta in [1e-3, 1e-1]
+    xn = torch.empty(T, s.d_model, device=dev, dtype=bf).normal_()
+    hz = torch.empty(T, 2 * s.d_inner, device=dev, dtype=bf).normal_()
+    u = torch.empty(T, s.d_inner, device=dev, dtype=bf).normal_()
+    xdbl = torch.empty(T, s.dt_rank + 2 * s.d_state, device=dev, dtype=bf).normal_()
+    dlt = (torch.rand(T, s.d_inner, device=dev) * 0.099 + 0.001).to(bf)
     y = torch.empty(T, s.d_inner, device=dev, dtype=bf)
     big = torch.empty(T, s.d_ff, device=dev, dtype=bf)
     xo = torch.empty(T, s.d_model, device=dev, dtype=bf)

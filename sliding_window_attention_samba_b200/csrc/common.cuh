@@ -100,6 +100,15 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// Byte offset that aligns a dynamic shared-memory array to `align`.  Offsetting
+// the __shared__ array itself (instead of round-tripping the pointer through an
+// integer) keeps the shared address space visible to the compiler, so accesses
+// compile to shared-memory instructions rather than generic ones.
+__device__ __forceinline__ uint32_t smem_align_pad(const void* base, uint32_t align) {
+  const uint32_t a = smem_u32(base);
+  return ((a + align - 1) & ~(align - 1)) - a;
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -283,7 +283,7 @@ __device__ __forceinline__ void tc_epilogue_tile(const TcParams& p, uint32_t tba
 template <int EPI>
 __global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_constant__ TcParams p, int* err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  TcSmem& S = *reinterpret_cast<TcSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  TcSmem& S = *reinterpret_cast<TcSmem*>(smem_raw + smem_align_pad(smem_raw, 1024));
   const int warp = warp_id_sync();
   const int lane = threadIdx.x & 31;
   const int ntiles = p.m_tiles * p.n_tiles;

@@ -11,8 +11,12 @@
 //     staged through shared memory by TMA, NSTAGE deep.
 //   * 8 warps split each chunk in time: warp w owns tokens [8w, 8w+8), lane l
 //     owns channel l and its 16 fp32 states in registers.
+//   * B and C of a chunk are converted to fp32 once into a shared tile (all 32
+//     lanes of a warp read the same values, so per-lane conversion would repeat
+//     it 32 times).
 //   * Walk 1: each lane runs its 8 tokens from a zero state, keeping the 8x16
 //     decays exp(Delta A) in registers, and publishes (prod of decays, end state).
+//     States are processed in pairs with packed fp32x2 FMA/MUL.
 //   * Combine: 256 threads each own two (channel, state) pairs and chain the
 //     8 warp aggregates sequentially from the carry of the previous chunk
 //     (kept in registers across chunks); this yields every warp's entry state.
@@ -44,16 +48,13 @@ struct ScanSmem {
   T Bm[kStages][kChunk * kN];
   T Cm[kStages][kChunk * kN];
   T y[2][kChunk * kCh];
+  float BC[2][kChunk][2 * kN];  // fp32 copy of B | C per token, converted once per chunk
   float aggP[kWarps][kN][kCh];
   float aggH[kWarps][kN][kCh];
   uint64_t full[kStages];
 };
 
-template <typename T>
-__device__ __forceinline__ void load16(const T* p, float* f) {
-  load8(p, f);
-  load8(p + 8, f + 8);
-}
+__device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
 
 template <typename T, bool kSoftplus, bool kHasZ>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -64,7 +65,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float* __restrict__ Dskip, const float* __restrict__ h0, float* __restrict__ hT,
                         int L, int D, int* err) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  ScanSmem<T>& S = *reinterpret_cast<ScanSmem<T>*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  ScanSmem<T>& S = *reinterpret_cast<ScanSmem<T>*>(smem_raw + smem_align_pad(smem_raw, 128));
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -99,13 +100,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_load_3d(S.Bm[s], &tm_B, &S.full[s], 0, t0, b);
     tma_load_3d(S.Cm[s], &tm_C, &S.full[s], 0, t0, b);
   };
+  // wait for chunk c's stage, then convert its B and C to fp32 (one element per thread pass)
+  auto arrive_chunk = [&](int c) -> bool {
+    const int s = c % kStages;
+    const bool ok = mbar_wait(&S.full[s], (c / kStages) & 1, err);
+    if (ok) {
+      float* dst = &S.BC[c & 1][0][0];
+      for (int e = tid; e < kChunk * 2 * kN; e += kThreads) {
+        const int row = e / (2 * kN), col = e % (2 * kN);
+        dst[e] = col < kN ? Elt<T>::to_f(S.Bm[s][row * kN + col]) : Elt<T>::to_f(S.Cm[s][row * kN + col - kN]);
+      }
+    }
+    return ok;
+  };
   if (tid == 0)
     for (int c = 0; c < kStages - 1 && c < nchunk; ++c) issue(c);
 
-  // Per-lane constants: A * log2(e) so that exp(Delta A) = 2^(Delta A log2 e).
-  float A2[kN];
+  // Per-lane constants: A * log2(e), as pairs of states.
+  float2 A2[kN / 2];
 #pragma unroll
-  for (int n = 0; n < kN; ++n) A2[n] = -expf(A_log[(size_t)d * kN + n]) * 1.4426950408889634f;
+  for (int n = 0; n < kN / 2; ++n)
+    A2[n] = make_float2(-expf(A_log[(size_t)d * kN + 2 * n]) * 1.4426950408889634f,
+                        -expf(A_log[(size_t)d * kN + 2 * n + 1]) * 1.4426950408889634f);
   const float bias = dt_bias ? dt_bias[d] : 0.f;
   const float Dd = Dskip ? Dskip[d] : 0.f;
 
@@ -114,29 +130,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int cn = (tid >> 5) * 2;
   float carry[2];
 #pragma unroll
-  for (int j = 0; j < 2; ++j)
-    carry[j] = h0 ? h0[((size_t)b * D + d0 + cl) * kN + cn + j] : 0.f;
+  for (int j = 0; j < 2; ++j) carry[j] = h0 ? h0[((size_t)b * D + d0 + cl) * kN + cn + j] : 0.f;
 
-  bool ok = true;
-  for (int c = 0; c < nchunk; ++c) {
+  bool ok = nchunk > 0 ? __syncthreads_and(arrive_chunk(0)) : true;
+  for (int c = 0; c < nchunk && ok; ++c) {
     const int s = c % kStages;
     if (tid == 0 && c + kStages - 1 < nchunk) issue(c + kStages - 1);
-    ok = mbar_wait(&S.full[s], (c / kStages) & 1, err);
-    if (__syncthreads_or(!ok)) break;
+    const float* BC = &S.BC[c & 1][0][0];
 
-    const int tb = warp * kTs;           // first token of this warp within the chunk
-    const int tg = c * kChunk + tb;      // global index of that token
-    float dA[kTs][kN];
+    const int tb = warp * kTs;       // first token of this warp within the chunk
+    const int tg = c * kChunk + tb;  // global index of that token
+    float2 dA[kTs][kN / 2];
     float du[kTs];
-    float h[kN];
+    float2 h[kN / 2];
 #pragma unroll
-    for (int n = 0; n < kN; ++n) h[n] = 0.f;
+    for (int n = 0; n < kN / 2; ++n) h[n] = make_float2(0.f, 0.f);
 
-    // ---- walk 1: local scan from zero, decays cached
+    // ---- walk 1: local scan from zero, decays cached (pairs of states per FMA2)
 #pragma unroll
     for (int i = 0; i < kTs; ++i) {
       const int row = tb + i;
-      float dtv = Elt<T>::to_f(S.dt[s][row * kCh + lane]) + bias;
+      const float dtv = Elt<T>::to_f(S.dt[s][row * kCh + lane]) + bias;
       float delta;
       if (kSoftplus) {
         if constexpr (sizeof(T) == 4) delta = softplus_acc(dtv);
@@ -147,21 +161,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       float uv = Elt<T>::to_f(S.u[s][row * kCh + lane]);
       if (tg + i >= L) { delta = 0.f; uv = 0.f; }
       du[i] = delta * uv;
-      float Bt[kN];
-      load16(&S.Bm[s][row * kN], Bt);
+      const float2 dl = f2(delta), dd = f2(du[i]);
+      const float4* Bp = reinterpret_cast<const float4*>(BC + row * 2 * kN);
 #pragma unroll
-      for (int n = 0; n < kN; ++n) {
-        dA[i][n] = ex2_approx(delta * A2[n]);
-        h[n] = fmaf(dA[i][n], h[n], du[i] * Bt[n]);
+      for (int q = 0; q < kN / 4; ++q) {
+        const float4 Bq = Bp[q];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int n = 2 * q + hh;
+          const float2 x = __fmul2_rn(dl, A2[n]);
+          dA[i][n] = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          const float2 bu = __fmul2_rn(dd, hh ? make_float2(Bq.z, Bq.w) : make_float2(Bq.x, Bq.y));
+          h[n] = __ffma2_rn(dA[i][n], h[n], bu);
+        }
       }
     }
 #pragma unroll
-    for (int n = 0; n < kN; ++n) {
-      float p = dA[0][n];
+    for (int n = 0; n < kN / 2; ++n) {
+      float2 p = dA[0][n];
 #pragma unroll
-      for (int i = 1; i < kTs; ++i) p *= dA[i][n];
-      S.aggP[warp][n][lane] = p;
-      S.aggH[warp][n][lane] = h[n];
+      for (int i = 1; i < kTs; ++i) p = __fmul2_rn(p, dA[i][n]);
+      S.aggP[warp][2 * n][lane] = p.x;
+      S.aggP[warp][2 * n + 1][lane] = p.y;
+      S.aggH[warp][2 * n][lane] = h[n].x;
+      S.aggH[warp][2 * n + 1][lane] = h[n].y;
     }
     __syncthreads();
 
@@ -183,20 +206,28 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---- walk 2: exact states from the entry state, outputs
 #pragma unroll
-    for (int n = 0; n < kN; ++n) h[n] = S.aggH[warp][n][lane];
+    for (int n = 0; n < kN / 2; ++n) h[n] = make_float2(S.aggH[warp][2 * n][lane], S.aggH[warp][2 * n + 1][lane]);
     T* ytile = S.y[c & 1];
 #pragma unroll
     for (int i = 0; i < kTs; ++i) {
       const int row = tb + i;
-      float Bt[kN], Ct[kN];
-      load16(&S.Bm[s][row * kN], Bt);
-      load16(&S.Cm[s][row * kN], Ct);
-      float y = 0.f;
+      const float4* Bp = reinterpret_cast<const float4*>(BC + row * 2 * kN);
+      const float4* Cp = Bp + kN / 4;
+      const float2 dd = f2(du[i]);
+      float2 y2 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int n = 0; n < kN; ++n) {
-        h[n] = fmaf(dA[i][n], h[n], du[i] * Bt[n]);
-        y = fmaf(Ct[n], h[n], y);
+      for (int q = 0; q < kN / 4; ++q) {
+        const float4 Bq = Bp[q];
+        const float4 Cq = Cp[q];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int n = 2 * q + hh;
+          const float2 bu = __fmul2_rn(dd, hh ? make_float2(Bq.z, Bq.w) : make_float2(Bq.x, Bq.y));
+          h[n] = __ffma2_rn(dA[i][n], h[n], bu);
+          y2 = __ffma2_rn(hh ? make_float2(Cq.z, Cq.w) : make_float2(Cq.x, Cq.y), h[n], y2);
+        }
       }
+      float y = y2.x + y2.y;
       const float uv = Elt<T>::to_f(S.u[s][row * kCh + lane]);
       y = fmaf(Dd, uv, y);
       if (kHasZ) {
@@ -207,7 +238,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       ytile[row * kCh + lane] = Elt<T>::from_f(y);
     }
     fence_proxy_async_smem();
-    __syncthreads();
+    // next chunk's stage has (usually) landed: convert its B and C while we are here
+    bool nxt = true;
+    if (c + 1 < nchunk) nxt = arrive_chunk(c + 1);
+    ok = __syncthreads_and(nxt);
     if (tid == 0) {
       tma_store_3d(&tm_y, ytile, d0, c * kChunk, b);
       tma_store_commit();

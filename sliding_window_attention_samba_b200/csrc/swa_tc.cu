@@ -63,7 +63,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 
 __global__ void __launch_bounds__(AT_THREADS, 1) swa_tc_kernel(const __grid_constant__ AtParams p, int* err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  AtSmem& S = *reinterpret_cast<AtSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  AtSmem& S = *reinterpret_cast<AtSmem*>(smem_raw + smem_align_pad(smem_raw, 1024));
   const int warp = warp_id_sync();
   const int lane = threadIdx.x & 31;
   const int t0 = blockIdx.x * AT_BM;
@@ -187,18 +187,28 @@ __global__ void __launch_bounds__(AT_THREADS, 1) swa_tc_kernel(const __grid_cons
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.s_free[j & 1]);
 
+      // Row max on the raw scores (the softmax scale is positive and folded into
+      // the exponent below).  Only the two edge tiles need the band mask; there the
+      // valid key offsets of row t are (t - w - kb, t - kb], empty for t >= L.
       const bool edge = (kb + AT_BN - 1 > t0) || (kb < t0 + AT_BM - p.window);
-      float mt = -INFINITY;
+      float m8[8];
 #pragma unroll
-      for (int i = 0; i < 128; ++i) {
-        float x = __uint_as_float(sr[i]) * p.scale_log2;
-        if (edge) {
-          const int s = kb + i;
-          if (s > t || s <= t - p.window || t >= p.L) x = -INFINITY;
+      for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
+      if (edge) {
+        const int hi = t < p.L ? t - kb : -1;
+        const int lo = t - p.window - kb;
+#pragma unroll
+        for (int i = 0; i < 128; ++i) {
+          if (i > hi || i <= lo) sr[i] = __float_as_uint(-INFINITY);
+          m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(sr[i]));
         }
-        sr[i] = __float_as_uint(x);
-        mt = fmaxf(mt, x);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 128; ++i) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(sr[i]));
       }
+      const float mraw = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      const float mt = mraw * p.scale_log2;  // -inf stays -inf
       // Online max with conditional rescale: a row moves its reference max only
       // when the tile max exceeds it by more than 2^8; O is then rescaled in TMEM.
       const bool need = mt > m_run + kRescaleThresh;
@@ -226,7 +236,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1) swa_tc_kernel(const __grid_cons
       const float msub = m_run == -INFINITY ? 0.f : m_run;
       // P buffer j%2 was last read by PV_{j-2}
       if (j >= 2 && !wait_all(&S.pv_done[j & 1], ((j - 2) >> 1) & 1)) { ok = false; break; }
-      float ls = 0.f;
+      float ls8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // independent partial sums
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         unsigned char* prow = reinterpret_cast<unsigned char*>(S.P[j & 1][half]) + r * 128;
@@ -235,15 +245,15 @@ __global__ void __launch_bounds__(AT_THREADS, 1) swa_tc_kernel(const __grid_cons
           float e[8];
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
-            e[q] = ex2_approx(__uint_as_float(sr[half * 64 + c * 8 + q]) - msub);
-            ls += e[q];
+            e[q] = ex2_approx(fmaf(__uint_as_float(sr[half * 64 + c * 8 + q]), p.scale_log2, -msub));
+            ls8[q] += e[q];
           }
           uint4 v4 = make_uint4(pack_bf16(e[0], e[1]), pack_bf16(e[2], e[3]), pack_bf16(e[4], e[5]),
                                 pack_bf16(e[6], e[7]));
           *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = v4;
         }
       }
-      l_run += ls;
+      l_run += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
