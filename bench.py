@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--impl", default="samba", choices=["samba", "reference"])
     ap.add_argument("--seq-len", type=int, default=None, help="override L (parity/debug runs only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="prefill", choices=["prefill", "decode"],
+                    help="prefill: 4-block L=131072 stack (the headline); decode: B=32 samba_step stream")
     return ap.parse_args()
 
 
@@ -380,8 +382,105 @@ def oracle_sample(sample_len=1024):
     return sample_len / dt, f"1 block, batch 1, first {sample_len} tokens of the L=131072 sequence (fp64 numpy)"
 
 
+def decode_bytes_per_step(s, Bn):
+    """Algorithmic HBM bytes of one decode step: every weight once, the ring K/V
+    read (full window), the SSM state read+written, the conv state read+written."""
+    es = 2
+    w = (2 * s.d_inner * s.d_model + (s.dt_rank + 2 * s.d_state) * s.d_inner + s.d_inner * s.dt_rank +
+         s.d_model * s.d_inner + (s.n_q + 2 * s.n_kv) * s.head_dim * s.d_model + s.d_model * s.n_q * s.head_dim +
+         2 * 3 * s.d_ff * s.d_model) * es
+    ring = 2 * Bn * s.window * s.n_kv * s.head_dim * es
+    ssm = 2 * Bn * s.d_inner * s.d_state * 4
+    conv = 2 * Bn * s.d_inner * (s.d_conv - 1) * es
+    return w + ring + ssm + conv
+
+
+def run_decode(args):
+    """Streaming decode: prefill P tokens at batch 32, then time samba_step replays."""
+    import torch
+    from sliding_window_attention_samba_b200 import _lib as L
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    shape, Bn, P, _, seed = I.WORKLOADS["decode_bf16_B32"]
+    s = shape
+    cfg = L.make_config(s)
+    (w, wst), = make_stack(torch, L, s, 1, seed, dev)
+    bf = torch.bfloat16
+    ssm = torch.zeros(Bn, s.d_inner, s.d_state, device=dev)
+    conv = torch.zeros(Bn, s.d_inner, s.d_conv - 1, device=dev, dtype=bf)
+    kr = torch.zeros(Bn, s.window, s.n_kv, s.head_dim, device=dev, dtype=bf)
+    vr = torch.zeros_like(kr)
+    pos = torch.zeros(Bn, dtype=torch.int64, device=dev)
+    st = L.make_state(ssm, conv, kr, vr, pos)
+    ws_bytes = max(L.samba_block_workspace_size(cfg, Bn, P), L.samba_step_workspace_size(cfg, Bn))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(I.tensor_key(seed, "decode.x") & ((1 << 63) - 1))
+    x = torch.randn(Bn, P, s.d_model, generator=g, device=dev).to(bf)
+    xo = torch.empty_like(x)
+    L.samba_block_fwd(cfg, wst, x, xo, st, None, Bn, P, ws, ws_bytes)
+    xt = torch.randn(Bn, s.d_model, generator=g, device=dev).to(bf)
+    yt = torch.empty_like(xt)
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        L.samba_step(cfg, wst, xt, yt, st, Bn, ws, ws_bytes, stream=stream)  # first call outside capture
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            L.samba_step(cfg, wst, xt, yt, st, Bn, ws, ws_bytes, stream=stream)
+        for _ in range(args.warmup):
+            graph.replay()
+        stream.synchronize()
+        assert L.samba_get_error(stream) == 0
+        clocks = ClockSampler(0)
+        clocks.start()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        e1.record(stream)
+        stream.synchronize()
+        clk = clocks.stop()
+        t = e0.elapsed_time(e1) * 1e-3
+        # end to end: host token in, host token out, every step
+        xh = xt.cpu().pin_memory()
+        yh = torch.empty_like(xh).pin_memory()
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        n_e2e = max(1, min(args.steps, 2000))
+        f0.record(stream)
+        for _ in range(n_e2e):
+            xt.copy_(xh, non_blocking=True)
+            graph.replay()
+            yh.copy_(yt, non_blocking=True)
+        f1.record(stream)
+        stream.synchronize()
+        t_e2e = f0.elapsed_time(f1) * 1e-3
+    assert L.samba_get_error() == 0
+    hbm, _, _, src = load_peaks()
+    bps = decode_bytes_per_step(s, Bn)
+    per_step = t / args.steps
+    line = {"metric": "decode tokens/s (batch 32, one Samba block, 2048-slot ring)", "value": Bn * args.steps / t,
+            "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": per_step * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "decode_bf16_B32", "batch": Bn, "prefill": P, "window": s.window,
+                       "d_model": s.d_model, "graph": "one samba_step captured, replayed per step"},
+            "e2e": {"value": Bn * n_e2e / t_e2e, "unit": "tokens/s", "h2d_bytes_per_step": xh.numel() * 2,
+                    "d2h_bytes_per_step": yh.numel() * 2},
+            "roofline": {"bound": "hbm", "achieved": bps / per_step / 1e9, "peak": hbm, "unit": "GB/s",
+                         "frac": bps / per_step / 1e9 / hbm, "traffic": None,
+                         "kernel": "whole decode step (weights + ring + states per step)",
+                         "peak_source": src, "bytes_per_step": bps},
+            "clocks": clk}
+    print(json.dumps(line))
+
+
 def main():
     args = parse()
+    if args.workload == "decode":
+        return run_decode(args)
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))

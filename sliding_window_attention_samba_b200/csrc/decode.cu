@@ -3,6 +3,8 @@
 // fixed-size and the SWA keeps only the last w keys; the blog page's
 // ring-buffer KV cache of w slots].  Plus the prefill -> decode-state handoff
 // (ring fill, position set).
+#include <string.h>
+
 #include "common.cuh"
 #include "decode.h"
 
@@ -50,7 +52,7 @@ __global__ void scan_step_kernel(const T* __restrict__ u, const T* __restrict__ 
 #pragma unroll
   for (int n = 0; n < 16; ++n) {
     const float A = -expf(A_log[(size_t)c * 16 + n]);
-    const float dA = expf(delta * A);
+    const float dA = sizeof(T) == 4 ? expf(delta * A) : ex2_approx(delta * A * 1.4426950408889634f);
     const float hn = fmaf(dA, hp[n], du * Elt<T>::to_f(Bp[n]));
     hp[n] = hn;
     yv = fmaf(Elt<T>::to_f(Cp[n]), hn, yv);
@@ -161,6 +163,243 @@ __global__ void attn_decode_kernel(const T* __restrict__ qkv, int64_t ld, const 
   }
 }
 
+// Split-ring decode attention for bf16, head_dim 64, up to 8 query heads per kv
+// head: a cluster of kSplit CTAs per (kv head, batch row), each CTA attending to
+// a slice of the valid ring slots (flash-decoding), partial (max, sum, o) merged
+// across the cluster through distributed shared memory.
+constexpr int kSplit = 8;
+constexpr int kSliceMax = 256;  // slots per CTA (window <= kSplit * kSliceMax)
+constexpr int kHd = 64;
+constexpr int kKvPad = kHd + 8;  // bf16 row pitch in smem (144 B: conflict-free 16-B reads)
+
+struct DecPart {
+  float m[8], l[8];
+  float o[8][kHd];
+};
+
+__device__ __forceinline__ uint32_t dec_cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Returns 0; peer loads add it to their address so that they depend on the
+// barrier and cannot be scheduled above it.
+__device__ __forceinline__ uint32_t dec_cluster_sync() {
+  uint32_t tok;
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;\n\tmov.u32 %0, 0;"
+               : "=r"(tok)::"memory");
+  return tok;
+}
+__device__ __forceinline__ float dec_ld_remote(const float* p, uint32_t rank, uint32_t tok) {
+  uint32_t ra;
+  asm("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(p) + tok), "r"(rank));
+  float v;
+  asm("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra));
+  return v;
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t* r, const void* row_addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(row_addr)));
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Each warp owns 32 keys of the CTA's slice; the up to 8 query heads of the
+// group are the rows of warp-level m16n8k16 tensor-core products (rows 8..15
+// are zero padding): S = Q K^T, then O = P V with P taken straight from the S
+// accumulators.  Max/sum/O are combined across the 8 warps in shared memory,
+// then across the cluster's CTAs through distributed shared memory.
+__global__ void __launch_bounds__(256, 1)
+    attn_decode_split_kernel(const bf16* __restrict__ qkv, int64_t ld, const int64_t* __restrict__ pos,
+                             const bf16* __restrict__ k_ring, const bf16* __restrict__ v_ring, bf16* __restrict__ o,
+                             int Hq, int Hkv, int window, float scale_log2) {
+  extern __shared__ __align__(16) unsigned char dec_dyn[];  // K slice | V slice (bf16, padded rows)
+  bf16* Ks = reinterpret_cast<bf16*>(dec_dyn);
+  bf16* Vs = Ks + kSliceMax * kKvPad;
+  __shared__ DecPart part;
+  __shared__ float wm[8][8], wl[8][8];  // [warp][head] partial max / sum
+  __shared__ float wo[8][8][kHd];       // [warp][head][dim] partial O
+  const uint32_t rank = dec_cluster_rank();
+  const int g = blockIdx.y, b = blockIdx.z;
+  const int grp = Hq / Hkv;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t P = pos[b];
+  const int nvalid = (int)(P + 1 < window ? P + 1 : window);
+  const int slice = ((nvalid + kSplit - 1) / kSplit + 31) & ~31;
+  const int s0 = (int)rank * slice;
+  const int n = max(0, min(nvalid, s0 + slice) - s0);
+  const size_t kvw = (size_t)Hkv * kHd;
+  // ---- K/V slice -> smem (16-byte vectors, all loads in flight before the stores);
+  // rows past n are zero-filled so that the tensor-core tiles read finite values
+  constexpr int kVecPerThread = kSliceMax * (kHd / 8) / 256;  // 8
+  uint4 kreg[kVecPerThread], vreg[kVecPerThread];
+#pragma unroll
+  for (int it = 0; it < kVecPerThread; ++it) {
+    const int e = threadIdx.x + 256 * it;
+    const int j = e / (kHd / 8), c = e % (kHd / 8);
+    kreg[it] = vreg[it] = make_uint4(0u, 0u, 0u, 0u);
+    if (j < n) {
+      const size_t off = ((size_t)b * window + s0 + j) * kvw + (size_t)g * kHd + c * 8;
+      kreg[it] = *reinterpret_cast<const uint4*>(k_ring + off);
+      vreg[it] = *reinterpret_cast<const uint4*>(v_ring + off);
+    }
+  }
+#pragma unroll
+  for (int it = 0; it < kVecPerThread; ++it) {
+    const int e = threadIdx.x + 256 * it;
+    const int j = e / (kHd / 8), c = e % (kHd / 8);
+    if (j < slice) {
+      *reinterpret_cast<uint4*>(&Ks[j * kKvPad + c * 8]) = kreg[it];
+      *reinterpret_cast<uint4*>(&Vs[j * kKvPad + c * 8]) = vreg[it];
+    }
+  }
+  // Q fragments (A operand, rows = heads): a0/a2 hold head lane/4, a1/a3 padding
+  const int qr = lane >> 2, qc = 2 * (lane & 3);
+  uint32_t qa[kHd / 16][4];
+#pragma unroll
+  for (int ks = 0; ks < kHd / 16; ++ks) {
+    qa[ks][1] = qa[ks][3] = 0u;
+    if (qr < grp) {
+      const bf16* qrow = qkv + (size_t)b * ld + (size_t)(g * grp + qr) * kHd + ks * 16 + qc;
+      qa[ks][0] = *reinterpret_cast<const uint32_t*>(qrow);
+      qa[ks][2] = *reinterpret_cast<const uint32_t*>(qrow + 8);
+    } else {
+      qa[ks][0] = qa[ks][2] = 0u;
+    }
+  }
+  __syncthreads();
+
+  const int kb = warp * 32;  // this warp's keys within the slice
+  const bool active = kb < n;
+  // ---- S = Q K^T over this warp's 32 keys (4 n-tiles of 8 keys)
+  float sacc[4][4];
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sacc[nt][i] = 0.f;
+    if (active) {
+#pragma unroll
+      for (int ks = 0; ks < kHd / 16; ++ks) {
+        const bf16* kp = &Ks[(kb + nt * 8 + qr) * kKvPad + ks * 16 + qc];
+        mma_bf16_16816(sacc[nt], qa[ks], *reinterpret_cast<const uint32_t*>(kp),
+                       *reinterpret_cast<const uint32_t*>(kp + 8));
+      }
+    }
+  }
+  // scale into the log2 domain, mask keys past n, warp max per head (row qr)
+  float mx = -INFINITY;
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const int key = kb + nt * 8 + qc + c;
+      const float v = key < n ? sacc[nt][c] * scale_log2 : -INFINITY;
+      sacc[nt][c] = v;
+      mx = fmaxf(mx, v);
+    }
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+  if ((lane & 3) == 0) wm[warp][qr] = mx;
+  __syncthreads();
+  float M = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) M = fmaxf(M, wm[w][qr]);
+  const float msub = M == -INFINITY ? 0.f : M;
+  // P = exp2(s - M) (bf16 for the product), row sums
+  float ls = 0.f;
+  uint32_t pa[2][4];  // A fragments of P for the two 16-key steps
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt) {
+    const float p0 = ex2_approx(sacc[nt][0] - msub), p1 = ex2_approx(sacc[nt][1] - msub);
+    ls += p0 + p1;
+    pa[nt >> 1][(nt & 1) ? 2 : 0] = pack_bf16x2(p0, p1);
+    pa[nt >> 1][(nt & 1) ? 3 : 1] = 0u;
+  }
+  ls += __shfl_xor_sync(0xffffffffu, ls, 1);
+  ls += __shfl_xor_sync(0xffffffffu, ls, 2);
+  if ((lane & 3) == 0) wl[warp][qr] = ls;
+  // ---- O_w = P V over this warp's 32 keys (2 k-steps x 8 n-tiles of dims)
+  float oacc[kHd / 8][4];
+#pragma unroll
+  for (int nt = 0; nt < kHd / 8; ++nt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) oacc[nt][i] = 0.f;
+  if (active) {
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+#pragma unroll
+      for (int np = 0; np < kHd / 16; ++np) {
+        uint32_t vb[4];
+        const int key = kb + ks * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
+        const int dim = np * 16 + 8 * (lane >> 4);
+        ldmatrix_x4_trans(vb, &Vs[key * kKvPad + dim]);
+        mma_bf16_16816(oacc[2 * np], pa[ks], vb[0], vb[1]);
+        mma_bf16_16816(oacc[2 * np + 1], pa[ks], vb[2], vb[3]);
+      }
+    }
+  }
+#pragma unroll
+  for (int nt = 0; nt < kHd / 8; ++nt) {
+    wo[warp][qr][nt * 8 + qc] = oacc[nt][0];
+    wo[warp][qr][nt * 8 + qc + 1] = oacc[nt][1];
+  }
+  __syncthreads();
+  // ---- CTA partial per head: m = M, l = sum_w, o = sum_w
+  for (int e = threadIdx.x; e < grp * kHd; e += 256) {
+    const int h = e / kHd, d = e % kHd;
+    float acc = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) acc += wo[w][h][d];
+    part.o[h][d] = acc;
+    if (d == 0) {
+      float mm = -INFINITY, ll = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) {
+        mm = fmaxf(mm, wm[w][h]);
+        ll += wl[w][h];
+      }
+      part.m[h] = mm;
+      part.l[h] = ll;
+    }
+  }
+  __syncthreads();
+  const uint32_t tok = dec_cluster_sync();
+  // ---- merge: rank r finalises query head r of the group
+  if ((int)rank < grp && threadIdx.x < kHd) {
+    const int hw = (int)rank;
+    float ms[kSplit], ls[kSplit], os[kSplit], M = -INFINITY;
+#pragma unroll
+    for (int s = 0; s < kSplit; ++s) {
+      ms[s] = dec_ld_remote(&part.m[hw], s, tok);
+      ls[s] = dec_ld_remote(&part.l[hw], s, tok);
+      os[s] = dec_ld_remote(&part.o[hw][threadIdx.x], s, tok);
+    }
+#pragma unroll
+    for (int s = 0; s < kSplit; ++s) M = fmaxf(M, ms[s]);
+    float Lsum = 0.f, O = 0.f;
+#pragma unroll
+    for (int s = 0; s < kSplit; ++s) {
+      const float wgt = ms[s] == -INFINITY ? 0.f : ex2_approx(ms[s] - M);
+      Lsum += wgt * ls[s];
+      O += wgt * os[s];
+    }
+    const int h = g * grp + hw;
+    o[(size_t)b * Hq * kHd + (size_t)h * kHd + threadIdx.x] = __float2bfloat16_rn(O / Lsum);
+  }
+  (void)dec_cluster_sync();  // peers' shared memory stays valid until every merge is done
+}
+
 __global__ void pos_add_kernel(int64_t* pos, int B, int64_t inc, int set) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < B) pos[i] = set ? inc : pos[i] + inc;
@@ -239,6 +478,28 @@ samba_status launch_attn_decode(const void* qkv, int64_t ld, const int64_t* pos,
                                 const void* v_ring, void* o, int B, int Hq, int Hkv, int hd, int window, float scale,
                                 samba_dtype dt, cudaStream_t st) {
   if (hd > 128) return SAMBA_ERR_UNSUPPORTED;
+  if (dt == SAMBA_BF16 && hd == kHd && Hq / Hkv <= 8 && window <= kSplit * kSliceMax && ld % 8 == 0) {
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(kSplit, Hkv, B);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.dynamicSmemBytes = 2 * kSliceMax * kKvPad * sizeof(bf16);
+    cfg.stream = st;
+    if (!ensure_smem_attr(attn_decode_split_kernel, cfg.dynamicSmemBytes)) return SAMBA_ERR_CUDA;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kSplit;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, attn_decode_split_kernel, (const bf16*)qkv, ld, pos, (const bf16*)k_ring,
+                           (const bf16*)v_ring, (bf16*)o, Hq, Hkv, window, scale * 1.4426950408889634f) !=
+        cudaSuccess)
+      return SAMBA_ERR_CUDA;
+    SAMBA_CHECK_LAUNCH();
+    return SAMBA_OK;
+  }
   const int grp = Hq / Hkv;
   const int threads = ((grp * 32) < 128 ? 128 : grp * 32);
   if (threads > 1024) return SAMBA_ERR_UNSUPPORTED;

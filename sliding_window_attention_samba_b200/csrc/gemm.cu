@@ -507,6 +507,7 @@ samba_status launch_gemm(const GemmArgs& a, cudaStream_t st) {
   if (a.epi == kEpiSoftplus && !a.bias) return SAMBA_ERR_INVALID_ARG;
   if (a.epi == kEpiRope && (!a.rope_tab || a.head_dim <= 0 || a.rope_cols % a.head_dim)) return SAMBA_ERR_INVALID_ARG;
   if (a.M == 0) return SAMBA_OK;
+  if (!force_simt() && a.M <= 64 && gemm_skinny_supported(a)) return launch_gemm_skinny(a, st);
   if (!force_simt() && gemm_tc_supported(a)) return launch_gemm_tc(a, st);
   if (a.epi == kEpiRope && 64 % a.head_dim != 0) return SAMBA_ERR_UNSUPPORTED;
   return launch_gemm_simt(a, st);

@@ -1,0 +1,381 @@
+// Skinny projections for decode (M = batch <= 64 tokens): out = epi(X W^T).
+//
+// At batch 32 a decode step is bound by streaming the weights once, and the
+// down/out projections have only N/128 = 16 tiles of 128 output features, far
+// too few CTAs to pull HBM bandwidth.  Design:
+//   * swap-AB on the tensor cores: the 128 weight rows of a tile are the UMMA M
+//     side (TMEM lanes), the zero-padded batch is the UMMA N side (16..64);
+//   * split-K across a thread-block cluster of S <= 8 CTAs (one n-tile per
+//     cluster), each CTA streaming a K range of the weight tile through a
+//     4-stage TMA ring into tcgen05.mma;
+//   * the S fp32 partial tiles are reduced through distributed shared memory
+//     (ld.shared::cluster) and the epilogue (residual, SwiGLU, softplus+bias,
+//     RoPE at per-row positions) is applied in the same kernel, so no partial
+//     sums ever reach HBM.
+// No cluster multicast is used (each CTA loads its own tiles).
+#include <stdlib.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace samba {
+
+namespace {
+
+constexpr int SK_BM = 128;     // weight rows (output features) per tile
+constexpr int SK_BK = 64;
+constexpr int SK_STAGES = 8;  // upper bound; the stage count is ring bytes / stage bytes
+constexpr int SK_MAXB = 64;    // max padded batch
+constexpr int SK_THREADS = 192;
+
+// Shared memory: a ring of stages (W tile | W2 tile (SwiGLU) | X tile) that is
+// reused, once every MMA has completed, for the fp32 partial tile(s) of the
+// cluster reduction; barriers and the TMEM address live after it.
+constexpr int SK_RING_BYTES = 200 * 1024;
+constexpr int SK_RED_PITCH = SK_MAXB + 1;
+static_assert(2 * SK_BM * SK_RED_PITCH * 4 <= SK_RING_BYTES, "reduction tiles must fit in the ring");
+
+struct SkSmem {
+  unsigned char ring[SK_RING_BYTES];
+  uint64_t full[SK_STAGES], empty[SK_STAGES], done;
+  uint32_t tmem_base;
+};
+
+struct SkParams {
+  CUtensorMap tmW[3];
+  CUtensorMap tmW2;
+  CUtensorMap tmX;
+  GemmArgs a;
+  int MB;          // padded batch (UMMA N)
+  int stages;      // ring stages in use
+  int stage_bytes; // bytes per stage (multiple of 1024)
+  int S;           // cluster size = K splits
+  int kb_total, kps;
+  int seg_start[3];
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// All threads of all CTAs of the cluster (non-.aligned form: callers may arrive
+// from diverged role branches).
+// Returns 0; peer loads add it to their address so that they depend on the
+// barrier and cannot be scheduled above it.
+__device__ __forceinline__ uint32_t cluster_sync_all() {
+  uint32_t tok;
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;\n\tmov.u32 %0, 0;"
+               : "=r"(tok)::"memory");
+  return tok;
+}
+// Peer shared-memory load.  Not volatile and no memory clobber: the loads are
+// ordered by the cluster barrier before them, and this lets the compiler issue
+// the loads of all peers back to back instead of one round trip at a time.
+__device__ __forceinline__ float ld_dsmem_f32(const float* local_ptr, uint32_t rank, uint32_t tok) {
+  uint32_t raddr;
+  asm("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(raddr) : "r"(smem_u32(local_ptr) + tok), "r"(rank));
+  float v;
+  asm("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(raddr));
+  return v;
+}
+
+// Fire-and-forget store of 4 floats into a peer CTA's shared memory.
+__device__ __forceinline__ void st_dsmem_v4(const float* local_ptr, uint32_t rank, float4 v, uint32_t tok) {
+  uint32_t raddr;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(raddr) : "r"(smem_u32(local_ptr) + tok), "r"(rank));
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(raddr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+               : "memory");
+}
+
+__device__ __forceinline__ float2 rope_cs_sk(const float2* __restrict__ tab, int half, int64_t p, int i) {
+  const float2 c0 = tab[(0 * kRopeRadix + (p & 1023)) * half + i];
+  const float2 c1 = tab[(1 * kRopeRadix + ((p >> 10) & 1023)) * half + i];
+  const float2 c2 = tab[(2 * kRopeRadix + ((p >> 20) & 1023)) * half + i];
+  const float cr = c0.x * c1.x - c0.y * c1.y, sr = c0.x * c1.y + c0.y * c1.x;
+  return make_float2(cr * c2.x - sr * c2.y, cr * c2.y + sr * c2.x);
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(SK_THREADS, 1) gemm_skinny_kernel(const __grid_constant__ SkParams p, int* err) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  SkSmem& S = *reinterpret_cast<SkSmem*>(smem_raw + smem_align_pad(smem_raw, 1024));
+  const GemmArgs& a = p.a;
+  const int warp = warp_id_sync();
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int ntile = blockIdx.x / p.S;
+  const int n0 = ntile * SK_BM;  // first output feature of this tile
+  const int kb_begin = (int)rank * p.kps;
+  const int kb_end = min(p.kb_total, kb_begin + p.kps);
+  const int nkb = max(0, kb_end - kb_begin);
+  constexpr bool kDual = EPI == kEpiSwiglu;
+
+  constexpr uint32_t kWBytes = SK_BM * SK_BK * 2;
+  auto stW = [&](int s) { return S.ring + (size_t)s * p.stage_bytes; };
+  auto stW2 = [&](int s) { return S.ring + (size_t)s * p.stage_bytes + kWBytes; };
+  auto stX = [&](int s) { return S.ring + (size_t)s * p.stage_bytes + (kDual ? 2 : 1) * kWBytes; };
+  float* red = reinterpret_cast<float*>(S.ring);  // [acc][row][SK_RED_PITCH], valid after `done`
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < SK_STAGES; ++s) {
+      mbar_init(&S.full[s], 1);
+      mbar_init(&S.empty[s], 1);
+    }
+    mbar_init(&S.done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&S.tmem_base, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+
+  if (warp == 0) {
+    if (elect_one()) {
+      int seg = 0;
+      while (seg < a.nseg - 1 && n0 >= p.seg_start[seg + 1]) ++seg;
+      const int wrow = n0 - p.seg_start[seg];
+      const uint32_t bytes = (uint32_t)(SK_BM * SK_BK * 2) * (kDual ? 2 : 1) + (uint32_t)p.MB * SK_BK * 2;
+      for (int i = 0; i < nkb; ++i) {
+        const int s = i % p.stages;
+        if (!mbar_wait(&S.empty[s], ((i / p.stages) & 1) ^ 1, err)) break;
+        mbar_arrive_expect_tx(&S.full[s], bytes);
+        const int kx = (kb_begin + i) * SK_BK;
+        tma_load_2d(stW(s), &p.tmW[seg], &S.full[s], kx, wrow);
+        if (kDual) tma_load_2d(stW2(s), &p.tmW2, &S.full[s], kx, wrow);
+        tma_load_2d(stX(s), &p.tmX, &S.full[s], kx, 0);
+      }
+    }
+  } else if (warp == 1) {
+    const uint32_t idesc = idesc_bf16_f32(SK_BM, p.MB);
+    if (elect_one()) {
+      bool ok = true;
+      for (int i = 0; i < nkb; ++i) {
+        const int s = i % p.stages;
+        if (!mbar_wait(&S.full[s], (i / p.stages) & 1, err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t wb = smem_u32(stW(s)), w2b = smem_u32(stW2(s)), xb = smem_u32(stX(s));
+#pragma unroll
+        for (int k = 0; k < SK_BK / 16; ++k) {
+          const uint64_t bd = smem_desc(xb + k * 32, 16, 1024, kLayoutSw128);
+          umma_f16_ss(tmem, smem_desc(wb + k * 32, 16, 1024, kLayoutSw128), bd, idesc, (i | k) != 0);
+          if (kDual)
+            umma_f16_ss(tmem + SK_MAXB, smem_desc(w2b + k * 32, 16, 1024, kLayoutSw128), bd, idesc, (i | k) != 0);
+        }
+        umma_commit(&S.empty[s]);
+      }
+      if (ok) umma_commit(&S.done);
+    }
+  }
+  // Every row of the tile has one owner rank that finalises it: contiguous
+  // slices of 128/S rows, or, for RoPE tiles, the two rows (i, i + hd/2) of
+  // each rotated pair together.  Receive buffers (in the now idle ring):
+  //   recv[acc][src][slot][MB]  with slot < rows per owner.
+  const bool rope_tile = EPI == kEpiRope && n0 < a.rope_cols;
+  const int rows_per = SK_BM / p.S;
+  const int MB = p.MB;
+  auto owner_of = [&](int r, int& slot) -> int {
+    if (rope_tile) {
+      const int hd = a.head_dim, half = hd / 2;
+      const int pair = (r / hd) * half + (r % half);
+      const int per_pairs = (SK_BM / 2) / p.S;
+      slot = 2 * (pair % per_pairs) + ((r % hd) >= half ? 1 : 0);
+      return pair / per_pairs;
+    }
+    slot = r % rows_per;
+    return r / rows_per;
+  };
+  auto recv = [&](int acc, int src, int slot) -> float* {
+    return red + ((size_t)(acc * p.S + src) * rows_per + slot) * MB;
+  };
+  uint32_t tok = 0;
+  if (warp >= 2) {
+    // TMEM -> registers (zeros if this CTA had no K range)
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    bool got = true;
+    if (nkb > 0) got = __all_sync(0xffffffffu, mbar_wait(&S.done, 0, err));
+    if (got) tc_fence_after();
+    float v[2][SK_MAXB];
+#pragma unroll
+    for (int acc = 0; acc < (kDual ? 2 : 1); ++acc) {
+#pragma unroll
+      for (int c = 0; c < SK_MAXB; c += 16) {
+        if (c < MB) {
+          uint32_t r[16];
+          if (nkb > 0 && got) {
+            tmem_ld16(tmem + acc * SK_MAXB + lane_off + c, r);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) r[i] = 0u;
+          }
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[acc][c + i] = __uint_as_float(r[i]);
+        }
+      }
+    }
+    tc_fence_before();
+    // all MMAs of all CTAs are complete once everyone passes this barrier, so
+    // every ring may be overwritten by the pushes below
+    tok = cluster_sync_all();
+    int slot;
+    const int own = owner_of(row, slot);
+#pragma unroll
+    for (int acc = 0; acc < (kDual ? 2 : 1); ++acc)
+#pragma unroll
+      for (int c = 0; c < SK_MAXB; c += 4)
+        if (c < MB) st_dsmem_v4(recv(acc, (int)rank, slot) + c, own,
+                                make_float4(v[acc][c], v[acc][c + 1], v[acc][c + 2], v[acc][c + 3]), tok);
+  } else {
+    tc_fence_before();
+    tok = cluster_sync_all();
+  }
+  tok = cluster_sync_all();  // every push has landed; nothing remote is touched after this
+
+  // ---- reduction of the S received partials of this rank's rows + epilogue
+  const int M = (int)a.M;
+  bf16* out = (bf16*)a.out;
+  if (rope_tile) {
+    const int hd = a.head_dim, half = hd / 2;
+    const int per_pairs = (SK_BM / 2) / p.S;
+    for (int e = threadIdx.x; e < per_pairs * M; e += SK_THREADS) {
+      const int pl = e / M, b = e % M;
+      const int pair = (int)rank * per_pairs + pl;
+      const int hh = pair / half, i = pair % half;
+      const int r1 = hh * hd + i, r2 = r1 + half;
+      float x1 = 0.f, x2 = 0.f;
+      for (int s = 0; s < p.S; ++s) {
+        x1 += recv(0, s, 2 * pl)[b];
+        x2 += recv(0, s, 2 * pl + 1)[b];
+      }
+      const int64_t pos = a.pos_dev ? a.pos_dev[b] : a.pos0 + b % a.seq_len;
+      const float2 cs = rope_cs_sk(a.rope_tab, half, pos, i);
+      bf16* o = out + (int64_t)b * a.ldo + n0;
+      if (n0 + r1 < a.N) o[r1] = __float2bfloat16_rn(x1 * cs.x - x2 * cs.y);
+      if (n0 + r2 < a.N) o[r2] = __float2bfloat16_rn(x2 * cs.x + x1 * cs.y);
+    }
+  } else {
+    const int rb = (int)rank * rows_per;
+    for (int e = threadIdx.x; e < rows_per * M; e += SK_THREADS) {
+      const int sl = e % rows_per, b = e / rows_per;  // consecutive threads -> consecutive features
+      const int n = n0 + rb + sl;
+      float v = 0.f, v2 = 0.f;
+      for (int s = 0; s < p.S; ++s) {
+        v += recv(0, s, sl)[b];
+        if (kDual) v2 += recv(1, s, sl)[b];
+      }
+      if (n >= a.N) continue;
+      if (EPI == kEpiSwiglu) v = v * (v2 * sigmoid_fast(v2));
+      if (EPI == kEpiSoftplus) v = softplus_fast(v + a.bias[n]);
+      if (EPI == kEpiResid) {
+        if (a.tap) ((bf16*)a.tap)[(int64_t)b * a.ldt + n] = __float2bfloat16_rn(v);
+        v += __bfloat162float(((const bf16*)a.resid)[(int64_t)b * a.ldr + n]);
+      }
+      out[(int64_t)b * a.ldo + n] = __float2bfloat16_rn(v);
+    }
+  }
+  (void)tok;
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+}  // namespace
+
+bool gemm_skinny_supported(const GemmArgs& a) {
+  if (a.dtype != SAMBA_BF16 || a.M < 1 || a.M > SK_MAXB || a.K % SK_BK) return false;
+  if (a.lda % 8 || a.ldo % 8 || !aligned16(a.A) || !aligned16(a.out)) return false;
+  if (a.epi == kEpiRope && (a.head_dim < 16 || SK_BM % a.head_dim || a.rope_cols % SK_BM)) return false;
+  int start = 0;
+  for (int s = 0; s < a.nseg; ++s) {
+    if (!aligned16(a.seg[s].W) || (a.seg[s].W2 && !aligned16(a.seg[s].W2))) return false;
+    if (s + 1 < a.nseg && (start + a.seg[s].n) % SK_BM) return false;  // tiles never straddle segments
+    start += a.seg[s].n;
+  }
+  if (a.epi == kEpiSwiglu && a.nseg != 1) return false;
+  const char* e = getenv("SAMBA_GEMM_KERNEL");
+  return !(e && e[0] == 's');
+}
+
+template <int EPI>
+static samba_status skinny_launch(const SkParams& p, int ntiles, cudaStream_t st) {
+  const size_t smem = sizeof(SkSmem) + 1024;
+  auto kern = gemm_skinny_kernel<EPI>;
+  if (!ensure_smem_attr(kern, smem)) return SAMBA_ERR_CUDA;
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(ntiles * p.S, 1, 1);
+  cfg.blockDim = dim3(SK_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = p.S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, p, device_error_word()) != cudaSuccess) return SAMBA_ERR_CUDA;
+  SAMBA_CHECK_LAUNCH();
+  return SAMBA_OK;
+}
+
+samba_status launch_gemm_skinny(const GemmArgs& a, cudaStream_t st) {
+  if (!gemm_skinny_supported(a)) return SAMBA_ERR_UNSUPPORTED;
+  SkParams p;
+  memset(&p, 0, sizeof(p));
+  p.a = a;
+  p.MB = (int)((a.M + 15) / 16) * 16;
+  {
+    const int xb = ((p.MB * SK_BK * 2) + 1023) / 1024 * 1024;
+    p.stage_bytes = (a.epi == kEpiSwiglu ? 2 : 1) * SK_BM * SK_BK * 2 + xb;
+    p.stages = SK_RING_BYTES / p.stage_bytes;
+    if (p.stages > SK_STAGES) p.stages = SK_STAGES;
+  }
+  const int ntiles = (a.N + SK_BM - 1) / SK_BM;
+  p.kb_total = a.K / SK_BK;
+  // splits: about one CTA per SM (one wave; a CTA uses most of an SM's shared
+  // memory), at most 8 (portable cluster size) and at most one k-block each
+  const int want = num_sms() / ntiles;
+  int S = 1;
+  while (S * 2 <= want && S * 2 <= 8 && S * 2 <= p.kb_total) S *= 2;
+  p.S = S;
+  p.kps = (p.kb_total + S - 1) / S;
+  {
+    uint64_t dims[2] = {(uint64_t)a.K, (uint64_t)a.M};
+    uint64_t strides[1] = {(uint64_t)a.lda};
+    uint32_t box[2] = {SK_BK, (uint32_t)p.MB};
+    if (!make_tmap(&p.tmX, a.A, SAMBA_BF16, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return SAMBA_ERR_CUDA;
+  }
+  int start = 0;
+  for (int s = 0; s < a.nseg; ++s) {
+    p.seg_start[s] = start;
+    uint64_t dims[2] = {(uint64_t)a.K, (uint64_t)a.seg[s].n};
+    uint64_t strides[1] = {(uint64_t)a.K};
+    uint32_t box[2] = {SK_BK, SK_BM};
+    if (!make_tmap(&p.tmW[s], a.seg[s].W, SAMBA_BF16, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return SAMBA_ERR_CUDA;
+    if (a.epi == kEpiSwiglu &&
+        !make_tmap(&p.tmW2, a.seg[s].W2, SAMBA_BF16, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return SAMBA_ERR_CUDA;
+    start += a.seg[s].n;
+  }
+  switch (a.epi) {
+    case kEpiNone: return skinny_launch<kEpiNone>(p, ntiles, st);
+    case kEpiResid: return skinny_launch<kEpiResid>(p, ntiles, st);
+    case kEpiSwiglu: return skinny_launch<kEpiSwiglu>(p, ntiles, st);
+    case kEpiSoftplus: return skinny_launch<kEpiSoftplus>(p, ntiles, st);
+    case kEpiRope: return skinny_launch<kEpiRope>(p, ntiles, st);
+  }
+  return SAMBA_ERR_INVALID_ARG;
+}
+
+}  // namespace samba

@@ -93,6 +93,8 @@ samba_status launch_gemm(const GemmArgs& a, cudaStream_t st);       // picks the
 samba_status launch_gemm_simt(const GemmArgs& a, cudaStream_t st);  // CUDA-core fp32 FMA kernel
 samba_status launch_gemm_tc(const GemmArgs& a, cudaStream_t st);    // tcgen05 kernel (bf16)
 bool gemm_tc_supported(const GemmArgs& a);
+samba_status launch_gemm_skinny(const GemmArgs& a, cudaStream_t st);  // M <= 64: swap-AB, cluster split-K
+bool gemm_skinny_supported(const GemmArgs& a);
 
 // ---------------- sliding-window attention ----------------
 struct SwaArgs {

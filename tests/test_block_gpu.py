@@ -183,3 +183,18 @@ def test_step_state_save_restore_bit_exact_and_graph(L):
         gr.replay()
         torch.cuda.synchronize()
         assert torch.equal(yout, ys1[i]), i
+
+
+def test_decode_steps_wide_bf16_batch4(L):
+    """Batch-4 decode at the 2048-wide shapes (skinny tensor-core projections,
+    per-row RoPE positions, ring attention) against the oracle's longer prefill."""
+    shape = I.WIDE
+    W = I.block_weights(shape, 6)
+    P, S = 300, 3
+    x = I.block_input(shape, 6, 4, P + S)
+    g = GpuBlock(L, shape, W, 4, P + S)
+    g.prefill(x[:, :P], taps=False)
+    full = O.block_fwd(x, W, shape)
+    for i in range(S):
+        y = host(g.step(x[:, P + i]))
+        assert rel_err(y - x[:, P + i], full["x_out"][:, P + i] - x[:, P + i]) <= TOL["bf16"], i
