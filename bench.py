@@ -48,8 +48,10 @@ def parse():
     ap.add_argument("--impl", default="samba", choices=["samba", "reference"])
     ap.add_argument("--seq-len", type=int, default=None, help="override L (parity/debug runs only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="prefill", choices=["prefill", "decode"],
-                    help="prefill: 4-block L=131072 stack (the headline); decode: B=32 samba_step stream")
+    ap.add_argument("--workload", default="prefill", choices=["prefill", "decode", "sweep"],
+                    help="prefill: 4-block L=131072 stack (the headline); decode: B=32 samba_step stream; "
+                         "sweep: scan and SWA alone at L = 4K..1M")
+    ap.add_argument("--max-len", type=int, default=1048576, help="sweep: largest L")
     return ap.parse_args()
 
 
@@ -477,10 +479,81 @@ def run_decode(args):
     print(json.dumps(line))
 
 
+def run_sweep(args):
+    """Mixer-only length sweep, batch 1, d_model 2048 shapes: the selective scan
+    (d_inner 4096, d_state 16; u, dt, z, B, C ~ N(0,1), Delta = softplus(dt + b))
+    and SWA (32/4 heads of 64, window 2048, RoPE) timed separately per L."""
+    import torch
+    from sliding_window_attention_samba_b200 import _lib as L
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    hbm, tf_burst, _, src = load_peaks()
+    bf = torch.bfloat16
+    D, N, Hq, Hkv, hd, w = 4096, 16, 32, 4, 64, 2048
+    A_log = torch.from_numpy(I.a_log_init(D, N)).to(dev)
+    dtb = torch.from_numpy(I.dt_bias_init(3, "scan.dt_bias", D)).to(dev)
+    Dk = torch.ones(D, device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(I.tensor_key(I.MIXER_SWEEP_SEED, "sweep") & ((1 << 63) - 1))
+    for Ln in I.MIXER_SWEEP_L:
+        if Ln > args.max_len:
+            break
+        u = torch.randn(1, Ln, D, generator=g, device=dev).to(bf)
+        dt = torch.randn(1, Ln, D, generator=g, device=dev).to(bf)
+        z = torch.randn(1, Ln, D, generator=g, device=dev).to(bf)
+        Bm = torch.randn(1, Ln, N, generator=g, device=dev).to(bf)
+        Cm = torch.randn(1, Ln, N, generator=g, device=dev).to(bf)
+        y = torch.empty_like(u)
+        hT = torch.empty(1, D, N, device=dev)
+
+        def scan():
+            L.samba_selective_scan(u, dt, dtb, 1, A_log, Bm, Cm, Dk, z, None, hT, y, 1, Ln, D, N, 1)
+        reps = max(2, min(20, (1 << 22) // Ln))
+        t_scan = _time(torch, scan, args.warmup, reps)
+        del u, dt, z, y
+        q = torch.randn(1, Ln, Hq, hd, generator=g, device=dev).to(bf)
+        k = torch.randn(1, Ln, Hkv, hd, generator=g, device=dev).to(bf)
+        v = torch.randn(1, Ln, Hkv, hd, generator=g, device=dev).to(bf)
+        o = torch.empty_like(q)
+        wsn = L.samba_swa_workspace_size(1, Ln, Hq, Hkv, hd, 10000.0, 1)
+        ws = torch.empty(wsn, dtype=torch.uint8, device=dev)
+
+        def swa():
+            L.samba_swa_fwd(q, k, v, o, 1, Ln, Hq, Hkv, hd, w, 10000.0, 0, 0.0, 1, ws, wsn)
+        t_swa = _time(torch, swa, args.warmup, reps)
+        del q, k, v, o, ws
+        torch.cuda.empty_cache()
+        assert L.samba_get_error() == 0
+        sb = Ln * (8 * D + 4 * N)
+        sf = swa_flops(I.WIDE, 1, Ln)
+        print(json.dumps({"workload": "mixer_sweep", "seq_len": Ln, "dtype": "bf16",
+                          "scan": {"ms": t_scan * 1e3, "gbs": sb / t_scan / 1e9, "frac_of_" + src + "_hbm": sb / t_scan / 1e9 / hbm,
+                                   "tokens_per_s": Ln / t_scan},
+                          "swa": {"ms": t_swa * 1e3, "tflops": sf / t_swa / 1e12,
+                                  "frac_of_" + src + "_bf16_burst": sf / t_swa / 1e12 / tf_burst,
+                                  "tokens_per_s": Ln / t_swa, "includes": "RoPE of q and k (standalone entry)"}}))
+
+
+def _time(torch, fn, warmup, reps):
+    for _ in range(max(1, warmup)):
+        fn()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) * 1e-3 / reps
+
+
 def main():
     args = parse()
     if args.workload == "decode":
         return run_decode(args)
+    if args.workload == "sweep":
+        return run_sweep(args)
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))

@@ -287,6 +287,256 @@ __global__ void __launch_bounds__(AT_THREADS, 1) swa_tc_kernel(const __grid_cons
   }
 }
 
+// ---------------------------------------------------------------------------
+// Two query heads per CTA (same kv head): two softmax warpgroups ping-pong on
+// the exp/FMA pipes while sharing every K/V tile.
+//   warp 0      TMA: Q of both heads, then K_j/V_j (3 stages)
+//   warp 1      TMEM owner + MMA issuer: S_A, S_B (M128 N128) and O_A, O_B (M128 N64)
+//   warps 2..5  softmax of head A, warps 6..9 softmax of head B (TMEM lane
+//               quadrant = warp % 4 in both groups)
+// The scores are read from TMEM twice (row max, then exponentials), which keeps
+// the softmax threads at ~100 registers so that 10 warps fit the register file.
+constexpr int A2_THREADS = 320;
+
+struct At2Smem {
+  bf16 Q[2][AT_BM * AT_D];
+  bf16 K[AT_STAGES][AT_BN * AT_D];
+  bf16 V[AT_STAGES][AT_BN * AT_D];
+  bf16 P[2][2][AT_BM * 64];  // [warpgroup][key half][row][64 keys], 128B-swizzled
+  uint64_t q_full;
+  uint64_t kv_full[AT_STAGES], kv_empty[AT_STAGES];
+  uint64_t s_full[2], s_free[2], p_full[2], pv_done[2];
+  uint32_t tmem_base;
+};
+
+__global__ void __launch_bounds__(A2_THREADS, 1) swa_tc2_kernel(const __grid_constant__ AtParams p, int* err) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  At2Smem& S = *reinterpret_cast<At2Smem*>(smem_raw + smem_align_pad(smem_raw, 1024));
+  const int warp = warp_id_sync();
+  const int lane = threadIdx.x & 31;
+  const int t0 = blockIdx.x * AT_BM;
+  const int h0 = blockIdx.y * 2;
+  const int b = blockIdx.z;
+  const int g = h0 / (p.Hq / p.Hkv);
+  const int lo = t0 - p.window + 1;
+  const int kb0 = lo <= 0 ? 0 : (lo / AT_BN) * AT_BN;
+  const int ntile = (t0 - kb0) / AT_BN + 1;
+
+  if (warp == 0 && lane == 0) {
+    mbar_init(&S.q_full, 1);
+    for (int s = 0; s < AT_STAGES; ++s) {
+      mbar_init(&S.kv_full[s], 1);
+      mbar_init(&S.kv_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&S.s_full[i], 1);
+      mbar_init(&S.s_free[i], 4);
+      mbar_init(&S.p_full[i], 4);
+      mbar_init(&S.pv_done[i], 1);
+    }
+    fence_mbar_init();
+    tma_prefetch_desc(&p.tmQ);
+    tma_prefetch_desc(&p.tmK);
+    tma_prefetch_desc(&p.tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(&S.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+  // TMEM: S_A [0,128) S_B [128,256) O_A [256,320) O_B [320,384)
+
+  if (warp == 0) {
+    if (elect_one()) {
+      mbar_arrive_expect_tx(&S.q_full, 2 * kTileBytes);
+      tma_load_3d(S.Q[0], &p.tmQ, &S.q_full, h0 * AT_D, t0, b);
+      tma_load_3d(S.Q[1], &p.tmQ, &S.q_full, (h0 + 1) * AT_D, t0, b);
+      for (int j = 0; j < ntile; ++j) {
+        const int s = j % AT_STAGES;
+        if (!mbar_wait(&S.kv_empty[s], ((j / AT_STAGES) & 1) ^ 1, err)) break;
+        mbar_arrive_expect_tx(&S.kv_full[s], 2 * kTileBytes);
+        const int kb = kb0 + j * AT_BN;
+        tma_load_3d(S.K[s], &p.tmK, &S.kv_full[s], g * AT_D, kb, b);
+        tma_load_3d(S.V[s], &p.tmV, &S.kv_full[s], g * AT_D, kb, b);
+      }
+    }
+  } else if (warp == 1) {
+    const uint32_t idesc_s = idesc_bf16_f32(AT_BM, AT_BN, false);
+    const uint32_t idesc_o = idesc_bf16_f32(AT_BM, AT_D, true);
+    if (elect_one()) {
+      bool ok = mbar_wait(&S.q_full, 0, err);
+      auto issue_s = [&](int wg, int j) -> bool {
+        const int s = j % AT_STAGES;
+        if (wg == 0 && !mbar_wait(&S.kv_full[s], (j / AT_STAGES) & 1, err)) return false;
+        if (j >= 1 && !mbar_wait(&S.s_free[wg], (j - 1) & 1, err)) return false;
+        tc_fence_after();
+        const uint32_t q_base = smem_u32(S.Q[wg]);
+        const uint32_t k_base = smem_u32(S.K[s]);
+#pragma unroll
+        for (int k = 0; k < AT_D / 16; ++k)
+          umma_f16_ss(tmem + wg * 128u, smem_desc(q_base + k * 32, 16, 1024, kLayoutSw128),
+                      smem_desc(k_base + k * 32, 16, 1024, kLayoutSw128), idesc_s, k != 0);
+        umma_commit(&S.s_full[wg]);
+        return true;
+      };
+      auto issue_pv = [&](int wg, int j) -> bool {
+        const int s = j % AT_STAGES;
+        if (!mbar_wait(&S.p_full[wg], j & 1, err)) return false;
+        tc_fence_after();
+        const uint32_t v_base = smem_u32(S.V[s]);
+#pragma unroll
+        for (int k = 0; k < AT_BN / 16; ++k) {
+          const uint32_t a_addr = smem_u32(S.P[wg][k >> 2]) + (k & 3) * 32;
+          const uint32_t b_addr = v_base + k * 16 * AT_D * 2;
+          umma_f16_ss(tmem + 256u + wg * 64u, smem_desc(a_addr, 16, 1024, kLayoutSw128),
+                      smem_desc(b_addr, 16, 1024, kLayoutSw128), idesc_o, (j | k) != 0);
+        }
+        if (wg == 1) umma_commit(&S.kv_empty[s]);  // both heads are done with K_j, V_j
+        umma_commit(&S.pv_done[wg]);
+        return true;
+      };
+      if (ok) ok = issue_s(0, 0);
+      if (ok) ok = issue_s(1, 0);
+      for (int j = 0; ok && j < ntile; ++j) {
+        ok = issue_pv(0, j);
+        if (ok && j + 1 < ntile) ok = issue_s(0, j + 1);
+        if (ok) ok = issue_pv(1, j);
+        if (ok && j + 1 < ntile) ok = issue_s(1, j + 1);
+      }
+    }
+  } else {
+    const int wg = (warp - 2) >> 2;  // 0: head h0, 1: head h0 + 1
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;
+    const int t = t0 + r;
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const uint32_t tS = tmem + wg * 128u + lane_off;
+    const uint32_t tO = tmem + 256u + wg * 64u + lane_off;
+    auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
+      const bool w = mbar_wait(bar, par, err);
+      return __all_sync(0xffffffffu, w);
+    };
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < ntile; ++j) {
+      const int kb = kb0 + j * AT_BN;
+      if (!wait_all(&S.s_full[wg], j & 1)) { ok = false; break; }
+      tc_fence_after();
+      const bool edge = (kb + AT_BN - 1 > t0) || (kb < t0 + AT_BM - p.window);
+      const int hi = t < p.L ? t - kb : -1;  // valid key offsets of row t: (lo_i, hi]
+      const int lo_i = t - p.window - kb;
+      // pass 1: row max of the raw scores
+      float m8[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sr[32];
+        tmem_ld32(tS + c * 32, sr);
+        tmem_wait_ld();
+        if (edge) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int kk = c * 32 + i;
+            const float x = (kk > hi || kk <= lo_i) ? -INFINITY : __uint_as_float(sr[i]);
+            m8[i & 7] = fmaxf(m8[i & 7], x);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(sr[i]));
+        }
+      }
+      const float mraw = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      const float mt = mraw * p.scale_log2;
+      const bool need = mt > m_run + kRescaleThresh;
+      float alpha = 1.f;
+      if (need) {
+        if (m_run != -INFINITY) alpha = exp2f(m_run - mt);
+        l_run *= alpha;
+        m_run = mt;
+      }
+      // PV_{j-1} must be complete before O is rescaled and before P is overwritten
+      if (j >= 1 && !wait_all(&S.pv_done[wg], (j - 1) & 1)) { ok = false; break; }
+      tc_fence_after();
+      if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t orr[16];
+          tmem_ld16(tO + c * 16, orr);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
+          tmem_st16(tO + c * 16, orr);
+        }
+        tmem_wait_st();
+      }
+      const float msub = m_run == -INFINITY ? 0.f : m_run;
+      // pass 2: P = exp2(s * scale - m) as bf16 into the swizzled P tile
+      float ls8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sr[32];
+        tmem_ld32(tS + c * 32, sr);
+        tmem_wait_ld();
+        unsigned char* prow = reinterpret_cast<unsigned char*>(S.P[wg][c >> 1]) + r * 128;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          const int chunk = (c & 1) * 4 + cc;  // 16-byte chunk (8 keys) within the 64-key half
+          float e[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int i = cc * 8 + q;
+            const int kk = c * 32 + i;
+            float x = fmaf(__uint_as_float(sr[i]), p.scale_log2, -msub);
+            if (edge && (kk > hi || kk <= lo_i)) x = -INFINITY;
+            e[q] = ex2_approx(x);
+            ls8[q] += e[q];
+          }
+          uint4 v4 = make_uint4(pack_bf16(e[0], e[1]), pack_bf16(e[2], e[3]), pack_bf16(e[4], e[5]),
+                                pack_bf16(e[6], e[7]));
+          *reinterpret_cast<uint4*>(prow + ((chunk ^ (r & 7)) << 4)) = v4;
+        }
+      }
+      l_run += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
+      tc_fence_before();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&S.s_free[wg]);
+        mbar_arrive(&S.p_full[wg]);
+      }
+    }
+    if (ok && wait_all(&S.pv_done[wg], (ntile - 1) & 1)) {
+      tc_fence_after();
+      uint32_t orr[64];
+      tmem_ld32(tO, orr);
+      tmem_ld32(tO + 32, orr + 32);
+      tmem_wait_ld();
+      if (t < p.L && l_run > 0.f) {
+        const float inv = 1.f / l_run;
+        bf16* op = p.o + ((int64_t)b * p.L + t) * p.ld_o + (int64_t)(h0 + wg) * AT_D;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          float f[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) f[q] = __uint_as_float(orr[c * 8 + q]) * inv;
+          store8(op + c * 8, f);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 bool make_head_map(CUtensorMap* m, const void* base, int64_t ld, int H, int L, int B) {
   uint64_t dims[3] = {(uint64_t)H * AT_D, (uint64_t)L, (uint64_t)B};
   uint64_t strides[2] = {(uint64_t)ld, (uint64_t)ld * (uint64_t)L};
@@ -317,6 +567,15 @@ samba_status launch_swa_tc(const SwaArgs& a, cudaStream_t st) {
   p.Hq = a.Hq;
   p.Hkv = a.Hkv;
   p.scale_log2 = a.scale * 1.4426950408889634f;
+  const int grp = a.Hq / a.Hkv;
+  if (grp % 2 == 0 && !(getenv("SAMBA_SWA_KERNEL") && getenv("SAMBA_SWA_KERNEL")[0] == '1')) {
+    const size_t smem = sizeof(At2Smem) + 1024;
+    if (!ensure_smem_attr(swa_tc2_kernel, smem)) return SAMBA_ERR_CUDA;
+    dim3 grid((a.L + AT_BM - 1) / AT_BM, a.Hq / 2, a.B);
+    swa_tc2_kernel<<<grid, A2_THREADS, smem, st>>>(p, device_error_word());
+    SAMBA_CHECK_LAUNCH();
+    return SAMBA_OK;
+  }
   const size_t smem = sizeof(AtSmem) + 1024;
   if (!ensure_smem_attr(swa_tc_kernel, smem)) return SAMBA_ERR_CUDA;
   dim3 grid((a.L + AT_BM - 1) / AT_BM, a.Hq, a.B);
