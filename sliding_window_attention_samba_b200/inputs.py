@@ -12,7 +12,8 @@ Generator (counter based, so any slice of any tensor can be drawn on its own):
 * Each tensor gets its own key: ``key = mix(seed * 0x9E3779B97F4A7C15 ^ fnv1a64(name))``.
 * Element i of a normal tensor uses counters 2i+1 and 2i+2 for two uniforms
   ``u = ((x >> 11) + 1) * 2**-53`` in (0, 1] and Box-Muller's cosine branch
-  ``sqrt(-2 ln u1) * cos(2 pi u2)`` (Box & Muller 1958), in fp64.
+  ``sqrt(-2 ln u1) * cos(2 pi u2)`` (Box & Muller 1958), in fp64, evaluated with
+  multi-threaded torch CPU ops so that full-size tensors take seconds.
 * The fp64 value is scaled, rounded to fp32 (round to nearest even) and, for
   bf16 tensors, rounded again from fp32 to bf16 (round to nearest even).
 
@@ -55,29 +56,54 @@ def tensor_key(seed: int, name: str) -> int:
 
 
 def _mix_arr(z: np.ndarray) -> np.ndarray:
+    """SplitMix64 finaliser on uint64 numpy arrays (reference form, small inputs)."""
     with np.errstate(over="ignore"):
         z = (z ^ (z >> np.uint64(30))) * _M1
         z = (z ^ (z >> np.uint64(27))) * _M2
         return z ^ (z >> np.uint64(31))
 
 
+def _s64(c: int) -> int:
+    """An unsigned 64-bit constant as the int64 with the same bits."""
+    return c - (1 << 64) if c >= (1 << 63) else c
+
+
+def _lsr(z, k: int):
+    """Logical right shift of int64 tensors (torch shifts are arithmetic)."""
+    return (z >> k) & ((1 << (64 - k)) - 1)
+
+
+def _mix_t(z):
+    """SplitMix64 finaliser on int64 torch tensors (wrapping 64-bit arithmetic,
+    identical bits to the unsigned definition)."""
+    z = (z ^ _lsr(z, 30)) * _s64(0xBF58476D1CE4E5B9)
+    z = (z ^ _lsr(z, 27)) * _s64(0x94D049BB133111EB)
+    return z ^ _lsr(z, 31)
+
+
 def uniforms(key: int, start: int, count: int) -> np.ndarray:
     """Uniforms in (0, 1] for counters start+1 .. start+count (fp64)."""
-    ctr = np.arange(start + 1, start + count + 1, dtype=np.uint64)
-    with np.errstate(over="ignore"):
-        z = np.uint64(key) + ctr * _GAMMA
-    x = _mix_arr(z)
-    return ((x >> np.uint64(11)).astype(np.float64) + 1.0) * (2.0 ** -53)
+    import torch
+    ctr = torch.arange(start + 1, start + count + 1, dtype=torch.int64)
+    z = _s64(key) + ctr * _s64(0x9E3779B97F4A7C15)
+    x = _mix_t(z)
+    return ((_lsr(x, 11).to(torch.float64) + 1.0) * (2.0 ** -53)).numpy()
 
 
-def normals(key: int, count: int, start: int = 0, chunk: int = 1 << 22) -> np.ndarray:
-    """Standard normals (fp64) for elements start .. start+count-1 of a tensor."""
+def normals(key: int, count: int, start: int = 0, chunk: int = 1 << 24) -> np.ndarray:
+    """Standard normals (fp64) for elements start .. start+count-1 of a tensor:
+    element i uses counters 2i+1, 2i+2 and Box-Muller's cosine branch.  Runs on
+    the host cores (torch CPU ops, multi-threaded)."""
+    import torch
     out = np.empty(count, dtype=np.float64)
+    two_pi = 2.0 * np.pi
     for off in range(0, count, chunk):
         n = min(chunk, count - off)
-        u = uniforms(key, 2 * (start + off), 2 * n)
+        ctr = torch.arange(2 * (start + off) + 1, 2 * (start + off + n) + 1, dtype=torch.int64)
+        x = _mix_t(_s64(key) + ctr * _s64(0x9E3779B97F4A7C15))
+        u = (_lsr(x, 11).to(torch.float64) + 1.0) * (2.0 ** -53)
         u1, u2 = u[0::2], u[1::2]
-        out[off:off + n] = np.sqrt(-2.0 * np.log(u1)) * np.cos(2.0 * np.pi * u2)
+        out[off:off + n] = (torch.sqrt(-2.0 * torch.log(u1)) * torch.cos(two_pi * u2)).numpy()
     return out
 
 
@@ -96,12 +122,14 @@ def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
 
 def round_to(x: np.ndarray, dtype: str) -> np.ndarray:
     """Round fp64 values to the storage dtype and return them as fp32 arrays
-    (bf16 values are exactly representable in fp32)."""
-    x32 = np.asarray(x, dtype=np.float64).astype(np.float32)
+    (bf16 values are exactly representable in fp32).  fp64 -> fp32 and fp32 ->
+    bf16 both round to nearest even."""
+    import torch
+    x32 = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float64)).to(torch.float32)
     if dtype == "f32":
-        return x32
+        return x32.numpy()
     if dtype == "bf16":
-        return bf16_bits_to_f32(to_bf16_bits(x32))
+        return x32.to(torch.bfloat16).to(torch.float32).numpy()
     raise ValueError(dtype)
 
 
@@ -147,7 +175,11 @@ WORKLOADS = {
     "block_bf16_B4_L4096": (WIDE, 4, 4096, 1, 1),
     "prefill_bf16_L131072_x4": (WIDE, 1, 131072, 4, 2),
     "decode_bf16_B32": (WIDE, 32, 4096, 1, 4),
+    "chunked_prefill_bf16_L1048576": (WIDE, 1, 1048576, 1, 5),
 }
+# chunk length of the chunked prefill (the blog page's "Chunked Prefilling for
+# 1M-Token Sequences": chunks of 32,768 tokens)
+CHUNKED_PREFILL_CHUNK = 32768
 MIXER_SWEEP_L = (4096, 16384, 65536, 262144, 1048576)
 MIXER_SWEEP_SEED = 3
 

@@ -63,20 +63,17 @@ class GpuBlock:
 
 
 def check_branches(shape, W, x, out, br, rs, tol):
-    eps = shape.norm_eps
+    """GPU branch outputs (tapped before each residual add) and residual stream
+    against the oracle's own fp64 stream; a branch sees the stream through an
+    RMSNorm, so the GPU's bf16 rounding of the stream stays a relative error of
+    the branch input."""
     x = x.astype(np.float64)
-    # each sub-layer recomputed by the oracle from the residual stream the GPU fed it
-    f0, _, _ = O.mamba_branch(O.rmsnorm(x, W["norm0"], eps), W, shape)
-    f1 = O.swiglu_mlp(O.rmsnorm(rs[0], W["norm1"], eps), W["mlp1_W1"], W["mlp1_W2"], W["mlp1_W3"])
-    f2, _, _, _ = O.attn_branch(O.rmsnorm(rs[1], W["norm2"], eps), W, shape, 0)
-    f3 = O.swiglu_mlp(O.rmsnorm(rs[2], W["norm3"], eps), W["mlp2_W1"], W["mlp2_W2"], W["mlp2_W3"])
-    errs = [rel_err(br[i], f) for i, f in enumerate([f0, f1, f2, f3])]
-    assert max(errs) <= tol, errs
-    # and end to end against the oracle's own residual stream
     ref = O.block_fwd(x, W, shape)
+    errs = [rel_err(br[i], ref["branch"][i]) for i in range(4)]
+    assert max(errs) <= tol, errs
+    for i in range(3):
+        assert rel_err(rs[i], ref["resid"][i]) <= tol, i
     assert rel_err(out, ref["x_out"]) <= tol
-    for i in range(4):
-        assert rel_err(br[i], ref["branch"][i]) <= 2 * tol, i
     return errs
 
 

@@ -30,6 +30,21 @@ def test_splitmix64_published_first_output():
     assert int(I._mix_arr(z)[0]) == 0xE220A8397B1DCDAF
 
 
+def test_torch_generator_matches_unsigned_definition():
+    # The int64 torch form of the counter generator gives the same bits as the
+    # unsigned SplitMix64 definition, at offsets past 2^32 too.
+    key = I.tensor_key(5, "w")
+    for start in (0, 7, (1 << 33) + 3):
+        ctr = np.arange(start + 1, start + 65, dtype=np.uint64)
+        with np.errstate(over="ignore"):
+            z = np.uint64(key) + ctr * np.uint64(0x9E3779B97F4A7C15)
+        ref = ((I._mix_arr(z) >> np.uint64(11)).astype(np.float64) + 1.0) * 2.0 ** -53
+        assert np.array_equal(I.uniforms(key, start, 64), ref)
+    a = I.normals(key, 100, start=0)
+    b = I.normals(key, 60, start=40)
+    assert np.array_equal(a[40:], b)  # element i depends only on its own counters
+
+
 def test_bf16_rounding_ties_to_even():
     x = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -2.5, 1.0 + 2 ** -7], dtype=np.float32)
     bits = I.to_bf16_bits(x)
