@@ -48,9 +48,11 @@ def parse():
     ap.add_argument("--impl", default="samba", choices=["samba", "reference"])
     ap.add_argument("--seq-len", type=int, default=None, help="override L (parity/debug runs only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="prefill", choices=["prefill", "decode", "sweep"],
-                    help="prefill: 4-block L=131072 stack (the headline); decode: B=32 samba_step stream; "
-                         "sweep: scan and SWA alone at L = 4K..1M")
+    ap.add_argument("--workload", default="prefill", choices=["prefill", "block", "decode", "sweep", "chunked"],
+                    help="prefill: 4-block L=131072 stack (the headline); block: one block at B=4, L=4096; "
+                         "decode: B=32 samba_step stream; "
+                         "sweep: scan and SWA alone at L = 4K..1M; "
+                         "chunked: one block over L=1M in 32K-token chunks (samba_block_fwd_chunk)")
     ap.add_argument("--max-len", type=int, default=1048576, help="sweep: largest L")
     return ap.parse_args()
 
@@ -247,6 +249,10 @@ def _scan_contig(torch, L, s, w, u, dlt, hz, y, Bn, Ln):
                            s.d_state, 1)
 
 
+def workload_of(args):
+    return "block_bf16_B4_L4096" if args.workload == "block" else WORKLOAD
+
+
 def run_cuda(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -254,7 +260,7 @@ def run_cuda(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    shape, Bn, Ln, n_blocks, seed = I.WORKLOADS[WORKLOAD]
+    shape, Bn, Ln, n_blocks, seed = I.WORKLOADS[workload_of(args)]
     if args.seq_len:
         Ln = args.seq_len
     s = shape
@@ -324,16 +330,26 @@ def run_cuda(args, rank, world, local_rank):
     # ---- per-kernel attribution (same kernels and shapes, one block)
     kt = attribution_pass(torch, L, s, blocks, x0.view(T, s.d_model), T, Bn, Ln) if rank == 0 else {}
 
-    def tmax(t):
-        if world == 1:
-            return t
-        tt = torch.tensor([t], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        return float(tt.item())
-
-    t_dev, t_e2e = tmax(t_dev), tmax(t_e2e)
+    t_dev, t_e2e = max_over_ranks(t_dev, world, dev), max_over_ranks(t_e2e, world, dev)
     return dict(t_dev=t_dev, t_e2e=t_e2e, clocks=clk, kt=kt, s=s, Bn=Bn, Ln=Ln, n_blocks=n_blocks,
                 h2d=xh.numel() * 2, d2h=yh.numel() * 2)
+
+
+def max_over_ranks(t, world, device):
+    """The slowest rank's time (every rank calls it, in the same order)."""
+    if world == 1:
+        return t
+    import torch
+    import torch.distributed as dist
+    tt = torch.tensor([t], device=device, dtype=torch.float64)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt.item())
+
+
+def replica_throughput(tokens_per_rank, world, t_max, steps, n_blocks):
+    """Whole-job tokens/s per block: the tokens all replicas pushed through each
+    block, over the slowest rank's time per step and block."""
+    return tokens_per_rank * world / (t_max / steps / n_blocks)
 
 
 def kernel_report(kt, s, T, Bn, Ln, peaks):
@@ -479,6 +495,111 @@ def run_decode(args):
     print(json.dumps(line))
 
 
+def run_chunked(args):
+    """One block over a 1M-token sequence fed as 32K-token chunks, each continuing
+    from the state the previous chunk left.  Device timing with the sequence
+    resident; end to end streams every chunk from pinned host memory and back,
+    so the device holds one chunk's input/output and workspace only.  For
+    comparison, the same sequence in one samba_block_fwd call when it fits."""
+    import torch
+    from sliding_window_attention_samba_b200 import _lib as L
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    wl = "chunked_prefill_bf16_L1048576"
+    shape, Bn, Ln, _, seed = I.WORKLOADS[wl]
+    if args.seq_len:
+        Ln = args.seq_len
+    C = min(I.CHUNKED_PREFILL_CHUNK, Ln)
+    nch = (Ln + C - 1) // C
+    s = shape
+    cfg = L.make_config(s)
+    (w, wst), = make_stack(torch, L, s, 1, seed, dev)
+    bf = torch.bfloat16
+    ssm = torch.zeros(Bn, s.d_inner, s.d_state, device=dev)
+    conv = torch.zeros(Bn, s.d_inner, s.d_conv - 1, device=dev, dtype=bf)
+    kr = torch.zeros(Bn, s.window, s.n_kv, s.head_dim, device=dev, dtype=bf)
+    vr = torch.zeros_like(kr)
+    pos = torch.zeros(Bn, dtype=torch.int64, device=dev)
+    st = L.make_state(ssm, conv, kr, vr, pos)
+    ws_bytes = L.samba_block_chunk_workspace_size(cfg, Bn, C)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(I.tensor_key(seed, "chunked.x") & ((1 << 63) - 1))
+    x = torch.randn(Bn, Ln, s.d_model, generator=g, device=dev).to(bf)
+    out = torch.empty_like(x)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for c in range(nch):
+            a, b = c * C, min(Ln, (c + 1) * C)
+            L.samba_block_fwd_chunk(cfg, wst, x[:, a:b], out[:, a:b], st, a, None, Bn, b - a, ws, ws_bytes)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert L.samba_get_error() == 0, "device error during warm-up"
+    clocks = ClockSampler(0)
+    clocks.start()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    t_dev = e0.elapsed_time(e1) * 1e-3
+    assert L.samba_get_error() == 0, "device error in the timed region"
+    # end to end, streamed: chunk in from pinned host memory, chunk out to it
+    xh = x.cpu().pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    del x, out
+    xc = torch.empty(Bn, C, s.d_model, device=dev, dtype=bf)
+    yc = torch.empty_like(xc)
+    torch.cuda.synchronize()
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.steps):
+        for c in range(nch):
+            a, b = c * C, min(Ln, (c + 1) * C)
+            xc[:, :b - a].copy_(xh[:, a:b], non_blocking=True)
+            L.samba_block_fwd_chunk(cfg, wst, xc, yc, st, a, None, Bn, b - a, ws, ws_bytes)
+            yh[:, a:b].copy_(yc[:, :b - a], non_blocking=True)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    t_e2e = f0.elapsed_time(f1) * 1e-3
+    assert L.samba_get_error() == 0
+    # one call over the whole sequence, if its workspace fits next to the rest
+    one = None
+    ws1 = L.samba_block_workspace_size(cfg, Bn, Ln)
+    free, _ = torch.cuda.mem_get_info()
+    if ws1 + 2 * xh.numel() * 2 + (4 << 30) < free:
+        del ws
+        ws_one = torch.empty(ws1, dtype=torch.uint8, device=dev)
+        xd = xh.to(dev)
+        yd = torch.empty_like(xd)
+        L.samba_block_fwd(cfg, wst, xd, yd, None, None, Bn, Ln, ws_one, ws1)
+        torch.cuda.synchronize()
+        t_one = _time(torch, lambda: L.samba_block_fwd(cfg, wst, xd, yd, None, None, Bn, Ln, ws_one, ws1), 1,
+                      max(1, args.steps))
+        one = {"value": Bn * Ln / t_one, "unit": "tokens/s", "workspace_gb": ws1 / 1e9}
+        del ws_one, xd, yd
+    tok = Bn * Ln * args.steps
+    line = {"metric": "chunked prefill tokens/s per Samba block at L=1M (32K-token chunks)", "value": tok / t_dev,
+            "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t_dev / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl, "batch": Bn, "seq_len": Ln, "chunk": C, "n_chunks": nch,
+                       "workspace_gb": ws_bytes / 1e9, "d_model": s.d_model, "window": s.window,
+                       "l2": "activations per chunk >> 126 MB L2; no flush needed"},
+            "e2e": {"value": tok / t_e2e, "unit": "tokens/s", "h2d_bytes_per_step": xh.numel() * 2,
+                    "d2h_bytes_per_step": yh.numel() * 2,
+                    "mode": "each chunk copied in from pinned host memory and out again, same stream"},
+            "single_call": one, "clocks": clk, "gpu_launches": (21 * nch - 1) * args.steps}
+    print(json.dumps(line))
+
+
 def run_sweep(args):
     """Mixer-only length sweep, batch 1, d_model 2048 shapes: the selective scan
     (d_inner 4096, d_state 16; u, dt, z, B, C ~ N(0,1), Delta = softplus(dt + b))
@@ -554,13 +675,15 @@ def main():
         return run_decode(args)
     if args.workload == "sweep":
         return run_sweep(args)
+    if args.workload == "chunked":
+        return run_chunked(args)
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
-    shape, Bn, Ln, n_blocks, _ = I.WORKLOADS[WORKLOAD]
+    shape, Bn, Ln, n_blocks, _ = I.WORKLOADS[workload_of(args)]
     if args.seq_len:
         Ln = args.seq_len
-    cfgd = {"workload": WORKLOAD, "model": "samba block stack (random init)", "global_batch": Bn * max(world, 1),
+    cfgd = {"workload": workload_of(args), "model": "samba block stack (random init)", "global_batch": Bn * max(world, 1),
             "seq_len": Ln, "n_blocks": n_blocks, "d_model": shape.d_model, "window": shape.window,
             "parallelism": f"replicas{max(world, 1)}", "l2": "activations per block >> 126 MB L2; no flush needed"}
 
@@ -590,16 +713,16 @@ def main():
     r = run_cuda(args, rank, world, local_rank)
     peaks = load_peaks()
     if rank == 0:
-        tok_block = Bn * Ln * world  # tokens through each block, all ranks
-        value = tok_block / (r["t_dev"] / args.steps / n_blocks)
-        e2e = tok_block / (r["t_e2e"] / args.steps / n_blocks)
+        value = replica_throughput(Bn * Ln, world, r["t_dev"], args.steps, n_blocks)
+        e2e = replica_throughput(Bn * Ln, world, r["t_e2e"], args.steps, n_blocks)
         roof, rep = kernel_report(r["kt"], r["s"], Bn * Ln, Bn, Ln, peaks)
         cpu = None
         if not args.no_cpu_baseline:
             v, desc = oracle_sample(1024)
             cpu = {"value": v, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle", "sample": desc}
         launches_per_block = 4 + 10 + 1 + 1 + 1 + 1  # norms, projections, conv, scan, rope table, swa
-        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        line = {"metric": METRIC if args.workload == "prefill" else "prefill tokens/s per Samba block (B=4, L=4096)",
+                "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": r["t_dev"] / args.steps * 1e3, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfgd,
                 "e2e": {"value": e2e, "unit": UNIT, "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},

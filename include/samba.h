@@ -220,7 +220,7 @@ size_t samba_block_workspace_size(const samba_block_config* cfg, int B, int L);
 /* One block over a fresh sequence (positions 0..L-1):
  *   x1 = x  + Mamba(RMSNorm(x)); x2 = x1 + MLP1(RMSNorm(x1));
  *   x3 = x2 + SWA(RMSNorm(x2));  x_out = x3 + MLP2(RMSNorm(x3)).
- * x_in, x_out: [B, L, d_model] dtype (must not alias).  If st != NULL it is
+ * x_in, x_out: [B, L, d_model] dtype (must not alias; may be NULL when L == 0).  If st != NULL it is
  * overwritten with the decode state after the last token (SSM state, the last
  * d_conv-1 pre-conv inputs, the last min(L, window) post-RoPE keys/values in
  * their ring slots, pos[b] = L).  taps may be NULL.
@@ -229,6 +229,33 @@ size_t samba_block_workspace_size(const samba_block_config* cfg, int B, int L);
 samba_status samba_block_fwd(const samba_block_config* cfg, const samba_block_weights* w, const void* x_in,
                              void* x_out, samba_decode_state* st, const samba_block_taps* taps, int B, int L,
                              void* workspace, size_t workspace_bytes, samba_stream stream);
+
+/* ------------------------------------------------------------------------
+ * Chunked prefill: the block over the next L tokens of sequences that have
+ * already seen pos0 tokens [blog page "Samba Guide: Hybrid Mamba & Sliding
+ * Window Architecture", "Production Deployment & Long-Context Best Practices",
+ * item 3 "Chunked Prefilling for 1M-Token Sequences": process a long prompt in
+ * chunks, carrying the recurrent state forward, so activation memory is bounded
+ * by the chunk].
+ *
+ * st holds the decode state after pos0 tokens (from samba_block_fwd, an earlier
+ * chunk, or samba_step); pos[b] must equal pos0 for every row, which a device
+ * check verifies (mismatch: SAMBA_ERR_DEVICE from samba_get_error; outputs and
+ * state are then undefined).  The chunk's conv inputs continue the d_conv-1
+ * carried inputs, its scan starts from st->ssm, its queries attend to the ring's
+ * keys of the min(pos0, window-1) preceding positions and to the chunk's own, and
+ * RoPE positions are pos0..pos0+L-1.  On return st holds the state after
+ * pos0 + L tokens, so x_out equals rows pos0..pos0+L-1 of samba_block_fwd over
+ * the whole prefix (up to rounding).  pos0 == 0 is samba_block_fwd with st.
+ * The workspace (samba_block_chunk_workspace_size) depends on B and L only and
+ * holds the chunk's activations plus B*(window-1+L) rows of keys and values.
+ * Requirements as samba_block_fwd; pos0 + L <= 2^30.
+ * ---------------------------------------------------------------------- */
+size_t samba_block_chunk_workspace_size(const samba_block_config* cfg, int B, int L);
+
+samba_status samba_block_fwd_chunk(const samba_block_config* cfg, const samba_block_weights* w, const void* x_in,
+                                   void* x_out, samba_decode_state* st, int64_t pos0, const samba_block_taps* taps,
+                                   int B, int L, void* workspace, size_t workspace_bytes, samba_stream stream);
 
 /* ------------------------------------------------------------------------
  * The Samba block, one decode step per sequence (constant cost per token;

@@ -29,6 +29,8 @@ c_size_t = ctypes.c_size_t
 c_float = ctypes.c_float
 
 SAMBA_F32, SAMBA_BF16 = 0, 1
+(SAMBA_OK, SAMBA_ERR_INVALID_ARG, SAMBA_ERR_UNSUPPORTED, SAMBA_ERR_CUDA, SAMBA_ERR_TIMEOUT,
+ SAMBA_ERR_DEVICE) = range(6)
 EPI_NONE, EPI_RESIDUAL, EPI_SWIGLU, EPI_SOFTPLUS_BIAS = 0, 1, 2, 3
 STATUS = {0: "SAMBA_OK", 1: "SAMBA_ERR_INVALID_ARG", 2: "SAMBA_ERR_UNSUPPORTED", 3: "SAMBA_ERR_CUDA",
           4: "SAMBA_ERR_TIMEOUT", 5: "SAMBA_ERR_DEVICE"}
@@ -95,6 +97,11 @@ _block_ws = _sig("samba_block_workspace_size", c_size_t, [ctypes.POINTER(BlockCo
 _block = _sig("samba_block_fwd", c_int,
               [ctypes.POINTER(BlockConfig), ctypes.POINTER(BlockWeights), c_void_p, c_void_p,
                ctypes.POINTER(DecodeState), ctypes.POINTER(BlockTaps), c_int, c_int, c_void_p, c_size_t, c_void_p])
+_chunk_ws = _sig("samba_block_chunk_workspace_size", c_size_t, [ctypes.POINTER(BlockConfig), c_int, c_int])
+_chunk = _sig("samba_block_fwd_chunk", c_int,
+              [ctypes.POINTER(BlockConfig), ctypes.POINTER(BlockWeights), c_void_p, c_void_p,
+               ctypes.POINTER(DecodeState), c_int64, ctypes.POINTER(BlockTaps), c_int, c_int, c_void_p, c_size_t,
+               c_void_p])
 _step_ws = _sig("samba_step_workspace_size", c_size_t, [ctypes.POINTER(BlockConfig), c_int])
 _step = _sig("samba_step", c_int,
              [ctypes.POINTER(BlockConfig), ctypes.POINTER(BlockWeights), c_void_p, c_void_p,
@@ -189,6 +196,17 @@ def samba_block_fwd(cfg: BlockConfig, w: BlockWeights, x_in, x_out, st: Optional
                     taps: Optional[BlockTaps], B, L, workspace, workspace_bytes, stream=None):
     _check("samba_block_fwd",
            _block(ctypes.byref(cfg), ctypes.byref(w), _p(x_in), _p(x_out), ctypes.byref(st) if st else None,
+                  ctypes.byref(taps) if taps else None, B, L, _p(workspace), workspace_bytes, _stream(stream)))
+
+
+def samba_block_chunk_workspace_size(cfg: BlockConfig, B, L) -> int:
+    return _chunk_ws(ctypes.byref(cfg), B, L)
+
+
+def samba_block_fwd_chunk(cfg: BlockConfig, w: BlockWeights, x_in, x_out, st: DecodeState, pos0,
+                          taps: Optional[BlockTaps], B, L, workspace, workspace_bytes, stream=None):
+    _check("samba_block_fwd_chunk",
+           _chunk(ctypes.byref(cfg), ctypes.byref(w), _p(x_in), _p(x_out), ctypes.byref(st) if st else None, pos0,
                   ctypes.byref(taps) if taps else None, B, L, _p(workspace), workspace_bytes, _stream(stream)))
 
 

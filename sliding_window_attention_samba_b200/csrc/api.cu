@@ -1,6 +1,7 @@
 // C ABI of libsamba: validation, workspace carving and the launch sequences of
 // the Samba block prefill and decode step [Samba 3.2 "Big-Picture
 // Architecture"; 3.4 "Detailed, Sentence-Based Technical Breakdown"].
+#include <algorithm>
 #include <mutex>
 #include <set>
 #include <utility>
@@ -94,11 +95,13 @@ struct Carve {
 };
 
 struct BlockPlan {
-  size_t tab, xn, hz, u, xdbl, dlt, y, x1, x2, x3, hmlp, qkv, o, total;
+  size_t tab, xn, hz, u, xdbl, dlt, y, x1, x2, x3, hmlp, qkv, o, kx, vx, convh, total;
   int xdw, qkvw;
 };
 
-static BlockPlan plan_block(const samba_block_config& c, int64_t T) {
+// Workspace of one block over T = B*L tokens; a chunked prefill (chunk_B > 0)
+// adds the K/V rows of the preceding window and a copy of the conv history.
+static BlockPlan plan_block(const samba_block_config& c, int64_t T, int chunk_B = 0) {
   BlockPlan p;
   const size_t es = dtype_size(c.dtype);
   p.xdw = c.dt_rank + 2 * c.d_state;
@@ -117,6 +120,10 @@ static BlockPlan plan_block(const samba_block_config& c, int64_t T) {
   p.hmlp = cv.take(T * c.d_ff * es);
   p.qkv = cv.take(T * p.qkvw * es);
   p.o = cv.take(T * c.n_q * c.head_dim * es);
+  const int64_t kv_rows = chunk_B > 0 ? T + (int64_t)chunk_B * (c.window - 1) : 0;
+  p.kx = cv.take(kv_rows * c.n_kv * c.head_dim * es);
+  p.vx = cv.take(kv_rows * c.n_kv * c.head_dim * es);
+  p.convh = cv.take((int64_t)chunk_B * c.d_inner * (c.d_conv - 1) * es);
   p.total = cv.off + 256;  // slack for aligning the caller's base pointer
   return p;
 }
@@ -354,16 +361,28 @@ size_t samba_block_workspace_size(const samba_block_config* cfg, int B, int L) {
   return plan_block(*cfg, (int64_t)B * L).total;
 }
 
-samba_status samba_block_fwd(const samba_block_config* cfg, const samba_block_weights* w, const void* x_in,
-                             void* x_out, samba_decode_state* stt, const samba_block_taps* taps, int B, int L,
-                             void* workspace, size_t workspace_bytes, samba_stream stream) {
+}  // extern "C"
+
+namespace samba {
+
+// One block over B x L tokens.  pos0 > 0 continues a prefill from the decode
+// state `stt` holds after pos0 tokens (chunked prefill): the conv history, the
+// SSM state and the ring's last window of K/V are the inputs before token 0,
+// RoPE positions start at pos0, and the state is advanced to pos0 + L.
+static samba_status block_forward(const samba_block_config* cfg, const samba_block_weights* w, const void* x_in,
+                                  void* x_out, samba_decode_state* stt, int64_t pos0, const samba_block_taps* taps,
+                                  int B, int L, void* workspace, size_t workspace_bytes, samba_stream stream) {
   TRY(validate_cfg(cfg));
   TRY(validate_weights(w));
-  if (!x_in || !x_out || B < 1 || L < 0 || x_in == x_out) return SAMBA_ERR_INVALID_ARG;
+  if (B < 1 || L < 0 || pos0 < 0) return SAMBA_ERR_INVALID_ARG;
+  if (L > 0 && (!x_in || !x_out || x_in == x_out)) return SAMBA_ERR_INVALID_ARG;
   if (stt && (!stt->ssm || !stt->conv || !stt->k_ring || !stt->v_ring || !stt->pos)) return SAMBA_ERR_INVALID_ARG;
+  const bool resume = pos0 > 0;
+  if (resume && !stt) return SAMBA_ERR_INVALID_ARG;
+  if (pos0 + (int64_t)L > (int64_t(1) << 30)) return SAMBA_ERR_UNSUPPORTED;
   const samba_block_config& c = *cfg;
   const int64_t T = (int64_t)B * L;
-  const BlockPlan P = plan_block(c, T);
+  const BlockPlan P = plan_block(c, T, resume ? B : 0);
   if (!workspace || workspace_bytes < P.total) return SAMBA_ERR_INVALID_ARG;
   if (!aligned16(x_in) || !aligned16(x_out)) return SAMBA_ERR_UNSUPPORTED;
   cudaStream_t st = (cudaStream_t)stream;
@@ -381,11 +400,10 @@ samba_status samba_block_fwd(const samba_block_config* cfg, const samba_block_we
   char* qkv = (char*)buf(P.qkv);
   float2* tab = (float2*)buf(P.tab);
 
+  if (T == 0 && resume) return launch_pos_check_set(stt->pos, B, pos0, pos0, st);
   if (T == 0) {
     if (stt) {
       TRY(launch_pos_update(stt->pos, B, 0, true, st));
-      ScanArgs z;  // zero SSM state
-      (void)z;
       cudaMemsetAsync(stt->ssm, 0, (size_t)B * Di * N * sizeof(float), st);
       cudaMemsetAsync(stt->conv, 0, (size_t)B * Di * (c.d_conv - 1) * es, st);
     }
@@ -403,6 +421,12 @@ samba_status samba_block_fwd(const samba_block_config* cfg, const samba_block_we
     ca.bias = w->conv_b;
     ca.u = buf(P.u);
     ca.state = stt ? stt->conv : nullptr;
+    if (resume) {  // the history is read from a copy: the kernel rewrites the state in place
+      const size_t bytes = (size_t)B * Di * (c.d_conv - 1) * es;
+      if (cudaMemcpyAsync(buf(P.convh), stt->conv, bytes, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+        return SAMBA_ERR_CUDA;
+      ca.hist = buf(P.convh);
+    }
     ca.B = B;
     ca.L = L;
     ca.D = Di;
@@ -430,6 +454,7 @@ samba_status samba_block_fwd(const samba_block_config* cfg, const samba_block_we
     a.ld_bc = P.xdw;
     a.A_log = w->A_log;
     a.Dskip = w->Dskip;
+    a.h0 = resume ? stt->ssm : nullptr;  // each thread reads its h0 entries before writing hT
     a.hT = stt ? stt->ssm : nullptr;
     a.B = B;
     a.L = L;
@@ -470,7 +495,7 @@ samba_status samba_block_fwd(const samba_block_config* cfg, const samba_block_we
       g.rope_cols = qw + kvw;
       g.head_dim = hd;
       g.seq_len = L;
-      g.pos0 = 0;
+      g.pos0 = pos0;
       g.rope_tab = tab;
     }
     TRY(launch_gemm(g, st));
@@ -491,9 +516,19 @@ samba_status samba_block_fwd(const samba_block_config* cfg, const samba_block_we
     a.window = c.window;
     a.scale = 1.0f / sqrtf((float)hd);
     a.dtype = dt;
+    if (resume) {  // keys of the h tokens before the chunk lead the chunk's own K/V rows
+      const int h = (int)std::min<int64_t>(pos0, c.window - 1);
+      TRY(launch_kv_window_gather(qkv, P.qkvw, qw, qw + kvw, stt->k_ring, stt->v_ring, buf(P.kx), buf(P.vx), B, L,
+                                  pos0, h, c.window, kvw, dt, st));
+      a.k = buf(P.kx);
+      a.v = buf(P.vx);
+      a.ld_k = a.ld_v = kvw;
+      a.qoff = h;
+    }
     TRY(launch_swa(a, st));
   }
-  if (stt) TRY(launch_ring_fill(qkv, P.qkvw, qw, qw + kvw, stt->k_ring, stt->v_ring, B, L, c.window, kvw, dt, st));
+  if (stt)
+    TRY(launch_ring_fill(qkv, P.qkvw, qw, qw + kvw, stt->k_ring, stt->v_ring, B, L, pos0, c.window, kvw, dt, st));
   {
     GemmArgs g = gemm1(buf(P.o), qw, w->Wo, T, Dm, qw, x3, Dm, dt);
     g.epi = kEpiResid;
@@ -506,9 +541,34 @@ samba_status samba_block_fwd(const samba_block_config* cfg, const samba_block_we
   // ---- MLP 2
   TRY(mlp_sublayer(c, w->norm_g[3], w->mlp2_W1, w->mlp2_W2, w->mlp2_W3, x3, x_out, xn, buf(P.hmlp),
                    taps ? taps->branch[3] : nullptr, T, st));
+  if (resume) return launch_pos_check_set(stt->pos, B, pos0, pos0 + L, st);
   if (stt) TRY(launch_pos_update(stt->pos, B, L, true, st));
   return SAMBA_OK;
 }
+
+}  // namespace samba
+
+extern "C" {
+
+samba_status samba_block_fwd(const samba_block_config* cfg, const samba_block_weights* w, const void* x_in,
+                             void* x_out, samba_decode_state* stt, const samba_block_taps* taps, int B, int L,
+                             void* workspace, size_t workspace_bytes, samba_stream stream) {
+  return block_forward(cfg, w, x_in, x_out, stt, 0, taps, B, L, workspace, workspace_bytes, stream);
+}
+
+// ------------------------------------------------------------------ chunked prefill
+size_t samba_block_chunk_workspace_size(const samba_block_config* cfg, int B, int L) {
+  if (validate_cfg(cfg) != SAMBA_OK || B < 1 || L < 0) return 0;
+  return plan_block(*cfg, (int64_t)B * L, B).total;
+}
+
+samba_status samba_block_fwd_chunk(const samba_block_config* cfg, const samba_block_weights* w, const void* x_in,
+                                   void* x_out, samba_decode_state* stt, int64_t pos0, const samba_block_taps* taps,
+                                   int B, int L, void* workspace, size_t workspace_bytes, samba_stream stream) {
+  if (!stt) return SAMBA_ERR_INVALID_ARG;
+  return block_forward(cfg, w, x_in, x_out, stt, pos0, taps, B, L, workspace, workspace_bytes, stream);
+}
+
 
 // ------------------------------------------------------------------ decode step
 size_t samba_step_workspace_size(const samba_block_config* cfg, int B) {

@@ -405,22 +405,57 @@ __global__ void pos_add_kernel(int64_t* pos, int B, int64_t inc, int set) {
   if (i < B) pos[i] = set ? inc : pos[i] + inc;
 }
 
-// prefill -> ring: positions max(0, L-w) .. L-1 into slot p mod w
+__global__ void pos_check_set_kernel(int64_t* pos, int B, int64_t expect, int64_t value, int* err) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < B) {
+    if (pos[i] != expect) raise_error(err, kErrDevice);
+    pos[i] = value;
+  }
+}
+
+// prefill -> ring: chunk tokens max(0, L-w) .. L-1 (absolute position pos0 + t) into slot (pos0 + t) mod w
 template <typename T>
 __global__ void ring_fill_kernel(const T* __restrict__ qkv, int64_t ld, int k_off, int v_off, T* __restrict__ k_ring,
-                                 T* __restrict__ v_ring, int L, int window, int kvw) {
+                                 T* __restrict__ v_ring, int L, int64_t pos0, int window, int kvw) {
   const int j = blockIdx.x;  // 0 .. min(L, w)-1
   const int b = blockIdx.y;
   const int n = min(L, window);
   if (j >= n) return;
   const int p = L - n + j;
-  const int slot = p % window;
+  const int slot = (int)((pos0 + p) % window);
   const T* src = qkv + ((size_t)b * L + p) * ld;
   T* kd = k_ring + ((size_t)b * window + slot) * kvw;
   T* vd = v_ring + ((size_t)b * window + slot) * kvw;
   for (int i = threadIdx.x; i < kvw; i += blockDim.x) {
     kd[i] = src[k_off + i];
     vd[i] = src[v_off + i];
+  }
+}
+
+// Row j of kx/vx: j < h is the ring entry of position pos0 - h + j, else chunk token j - h.
+// Rows are copied as 16-byte pieces (`vec` per row); dtype-agnostic.
+__global__ void kv_window_gather_kernel(const char* __restrict__ qkv, int64_t ld_b, int64_t k_off_b,
+                                        int64_t v_off_b, const char* __restrict__ k_ring,
+                                        const char* __restrict__ v_ring, char* __restrict__ kx,
+                                        char* __restrict__ vx, int L, int64_t pos0, int h, int window, int vec) {
+  const int j = blockIdx.x;
+  const int b = blockIdx.y;
+  const int64_t row_b = (int64_t)vec * 16;
+  const char *ks, *vs;
+  if (j < h) {
+    const int slot = (int)((pos0 - h + j) % window);
+    ks = k_ring + ((int64_t)b * window + slot) * row_b;
+    vs = v_ring + ((int64_t)b * window + slot) * row_b;
+  } else {
+    const char* src = qkv + ((int64_t)b * L + (j - h)) * ld_b;
+    ks = src + k_off_b;
+    vs = src + v_off_b;
+  }
+  char* kd = kx + ((int64_t)b * (h + L) + j) * row_b;
+  char* vd = vx + ((int64_t)b * (h + L) + j) * row_b;
+  for (int i = threadIdx.x; i < vec; i += blockDim.x) {
+    reinterpret_cast<uint4*>(kd)[i] = reinterpret_cast<const uint4*>(ks)[i];
+    reinterpret_cast<uint4*>(vd)[i] = reinterpret_cast<const uint4*>(vs)[i];
   }
 }
 
@@ -523,15 +558,39 @@ samba_status launch_pos_update(int64_t* pos, int B, int64_t value, bool set, cud
 }
 
 samba_status launch_ring_fill(const void* qkv, int64_t ld, int k_off, int v_off, void* k_ring, void* v_ring, int B,
-                              int L, int window, int kvw, samba_dtype dt, cudaStream_t st) {
+                              int L, int64_t pos0, int window, int kvw, samba_dtype dt, cudaStream_t st) {
   const int n = L < window ? L : window;
   if (n == 0) return SAMBA_OK;
   dim3 grid(n, B);
   SAMBA_DT_DISPATCH(dt,
                     (ring_fill_kernel<bf16><<<grid, 128, 0, st>>>((const bf16*)qkv, ld, k_off, v_off, (bf16*)k_ring,
-                                                                  (bf16*)v_ring, L, window, kvw)),
+                                                                  (bf16*)v_ring, L, pos0, window, kvw)),
                     (ring_fill_kernel<float><<<grid, 128, 0, st>>>((const float*)qkv, ld, k_off, v_off,
-                                                                   (float*)k_ring, (float*)v_ring, L, window, kvw)));
+                                                                   (float*)k_ring, (float*)v_ring, L, pos0, window,
+                                                                   kvw)));
+  SAMBA_CHECK_LAUNCH();
+  return SAMBA_OK;
+}
+
+samba_status launch_kv_window_gather(const void* qkv, int64_t ld, int k_off, int v_off, const void* k_ring,
+                                     const void* v_ring, void* kx, void* vx, int B, int L, int64_t pos0, int h,
+                                     int window, int kvw, samba_dtype dt, cudaStream_t st) {
+  const size_t es = dtype_size(dt);
+  const int vec = (int)(kvw * es / 16);  // 16-byte pieces per row
+  if ((kvw * es) % 16 || (ld * es) % 16 || (k_off * es) % 16 || (v_off * es) % 16 || h < 0 || h > pos0 ||
+      h >= window + 1)
+    return SAMBA_ERR_UNSUPPORTED;
+  if (h + L == 0) return SAMBA_OK;
+  dim3 grid(h + L, B);
+  kv_window_gather_kernel<<<grid, 64, 0, st>>>((const char*)qkv, ld * es, k_off * es, v_off * es,
+                                               (const char*)k_ring, (const char*)v_ring, (char*)kx, (char*)vx, L,
+                                               pos0, h, window, vec);
+  SAMBA_CHECK_LAUNCH();
+  return SAMBA_OK;
+}
+
+samba_status launch_pos_check_set(int64_t* pos, int B, int64_t expect, int64_t value, cudaStream_t st) {
+  pos_check_set_kernel<<<(B + 127) / 128, 128, 0, st>>>(pos, B, expect, value, device_error_word());
   SAMBA_CHECK_LAUNCH();
   return SAMBA_OK;
 }

@@ -16,7 +16,15 @@ samba_status launch_attn_decode(const void* qkv, int64_t ld, const int64_t* pos,
                                 const void* v_ring, void* o, int B, int Hq, int Hkv, int hd, int window, float scale,
                                 samba_dtype dt, cudaStream_t st);
 samba_status launch_pos_update(int64_t* pos, int B, int64_t value, bool set, cudaStream_t st);
+// prefill -> ring: the last min(L, w) tokens of a prefill whose token 0 is at absolute position pos0
 samba_status launch_ring_fill(const void* qkv, int64_t ld, int k_off, int v_off, void* k_ring, void* v_ring, int B,
-                              int L, int window, int kvw, samba_dtype dt, cudaStream_t st);
+                              int L, int64_t pos0, int window, int kvw, samba_dtype dt, cudaStream_t st);
+// K/V rows of a prefill chunk preceded by the h ring entries of positions pos0-h .. pos0-1:
+// kx, vx [B, h + L, kvw] (contiguous)
+samba_status launch_kv_window_gather(const void* qkv, int64_t ld, int k_off, int v_off, const void* k_ring,
+                                     const void* v_ring, void* kx, void* vx, int B, int L, int64_t pos0, int h,
+                                     int window, int kvw, samba_dtype dt, cudaStream_t st);
+// pos[b] must equal `expect` (else the device error word is set); then pos[b] = value
+samba_status launch_pos_check_set(int64_t* pos, int B, int64_t expect, int64_t value, cudaStream_t st);
 
 }  // namespace samba

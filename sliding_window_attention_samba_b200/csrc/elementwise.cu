@@ -67,8 +67,8 @@ constexpr int kMaxK = 8;
 
 template <typename T, int K>
 __global__ void conv_silu_kernel(const T* __restrict__ x, int64_t ld_x, const float* __restrict__ w,
-                                 const float* __restrict__ bias, T* __restrict__ u, T* __restrict__ state, int L,
-                                 int D) {
+                                 const float* __restrict__ bias, T* __restrict__ u, T* __restrict__ state,
+                                 const T* __restrict__ hist_in, int L, int D) {
   const int cg = blockIdx.x * blockDim.x + threadIdx.x;  // channel group of 8
   const int c0 = cg * 8;
   const int t0 = blockIdx.y * kConvRun;
@@ -82,15 +82,18 @@ __global__ void conv_silu_kernel(const T* __restrict__ x, int64_t ld_x, const fl
     bb[i] = bias ? bias[c0 + i] : 0.f;
   }
   const T* xb = x + (size_t)b * L * ld_x + c0;
+  // input at token t < 0: the carried history (slot K-1+t of each channel), or zero
+  auto before = [&](int t, float* f) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      f[i] = hist_in ? Elt<T>::to_f(hist_in[((size_t)b * D + c0 + i) * (K - 1) + (K - 1) + t]) : 0.f;
+  };
   float hist[K][8];  // hist[j] = x[t-(K-1)+j]
 #pragma unroll
   for (int j = 0; j < K - 1; ++j) {
     const int t = t0 - (K - 1) + j;
     if (t >= 0) load8(xb + (size_t)t * ld_x, hist[j]);
-    else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) hist[j][i] = 0.f;
-    }
+    else before(t, hist[j]);
   }
   const int tend = min(t0 + kConvRun, L);
   for (int t = t0; t < tend; ++t) {
@@ -116,10 +119,7 @@ __global__ void conv_silu_kernel(const T* __restrict__ x, int64_t ld_x, const fl
       const int t = L - (K - 1) + j;
       float f[8];
       if (t >= 0) load8(xb + (size_t)t * ld_x, f);
-      else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) f[i] = 0.f;
-      }
+      else before(t, f);
 #pragma unroll
       for (int i = 0; i < 8; ++i) state[((size_t)b * D + c0 + i) * (K - 1) + j] = Elt<T>::from_f(f[i]);
     }
@@ -137,8 +137,8 @@ samba_status launch_conv_k(const ConvArgs& a, cudaStream_t st) {
   const int groups = a.D / 8;
   dim3 block(128);
   dim3 grid((groups + 127) / 128, (a.L + kConvRun - 1) / kConvRun, a.B);
-  conv_silu_kernel<T, K><<<grid, block, 0, st>>>((const T*)a.x, a.ld_x, a.w, a.bias, (T*)a.u, (T*)a.state, a.L,
-                                                 a.D);
+  conv_silu_kernel<T, K><<<grid, block, 0, st>>>((const T*)a.x, a.ld_x, a.w, a.bias, (T*)a.u, (T*)a.state,
+                                                 (const T*)a.hist, a.L, a.D);
   SAMBA_CHECK_LAUNCH();
   return SAMBA_OK;
 }
@@ -161,8 +161,12 @@ samba_status launch_causal_conv(const ConvArgs& a, cudaStream_t st) {
   if (!a.x || !a.w || !a.u || a.B < 1 || a.L < 0 || a.D < 1 || a.ld_x < a.D) return SAMBA_ERR_INVALID_ARG;
   if (a.k < 2 || a.k > kMaxK || a.D % 8 || a.ld_x % 8 || !aligned16(a.x) || !aligned16(a.u))
     return SAMBA_ERR_UNSUPPORTED;
+  if (a.hist && a.hist == a.state) return SAMBA_ERR_INVALID_ARG;
   if (a.L == 0) {
-    if (a.state) {
+    if (a.state && a.hist) {  // no new inputs: the history is the state
+      const size_t bytes = (size_t)a.B * a.D * (a.k - 1) * dtype_size(a.dtype);
+      if (cudaMemcpyAsync(a.state, a.hist, bytes, cudaMemcpyDeviceToDevice, st) != cudaSuccess) return SAMBA_ERR_CUDA;
+    } else if (a.state) {
       const size_t n = (size_t)a.B * a.D * (a.k - 1);
       if (a.dtype == SAMBA_BF16) conv_state_zero_kernel<bf16><<<(unsigned)((n + 255) / 256), 256, 0, st>>>((bf16*)a.state, n);
       else conv_state_zero_kernel<float><<<(unsigned)((n + 255) / 256), 256, 0, st>>>((float*)a.state, n);

@@ -51,7 +51,9 @@ struct ConvArgs {
   const float* w = nullptr;
   const float* bias = nullptr;
   void* u = nullptr;
-  void* state = nullptr;
+  void* state = nullptr;       // out: [B, D, k-1] the last k-1 inputs, oldest first (may be NULL)
+  const void* hist = nullptr;  // in: [B, D, k-1] the k-1 inputs before token 0, oldest first; NULL = zeros.
+                               // Must not alias `state`.
   int B = 0, L = 0, D = 0, k = 0;
   samba_dtype dtype = SAMBA_BF16;
 };
@@ -99,11 +101,12 @@ bool gemm_skinny_supported(const GemmArgs& a);
 // ---------------- sliding-window attention ----------------
 struct SwaArgs {
   const void* q = nullptr;  // [B, L, Hq, d] rows of stride ld_q elements per token
-  const void* k = nullptr;  // [B, L, Hkv, d]
+  const void* k = nullptr;  // [B, L + qoff, Hkv, d]
   const void* v = nullptr;
   void* o = nullptr;        // [B, L, Hq, d]
   int64_t ld_q = 0, ld_k = 0, ld_v = 0, ld_o = 0;  // elements between consecutive tokens
   int B = 0, L = 0, Hq = 0, Hkv = 0, d = 0, window = 0;
+  int qoff = 0;             // query row t is key row t + qoff (keys of earlier tokens lead the K/V rows)
   float scale = 0.f;
   samba_dtype dtype = SAMBA_BF16;
 };

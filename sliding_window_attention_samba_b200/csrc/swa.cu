@@ -27,6 +27,8 @@ __global__ void __launch_bounds__(SW_Q) swa_simt_kernel(const SwaArgs a) {
   const int g = h / (a.Hq / a.Hkv);
   const int t = t0 + tid;
   const bool active = t < a.L;
+  const int Lk = a.L + a.qoff;  // key rows per batch row
+  const int tk = t + a.qoff;    // this query's own key row
   const float sl2 = a.scale * 1.4426950408889634f;  // scores in log2 units
 
   float q[D], o[D];
@@ -38,10 +40,10 @@ __global__ void __launch_bounds__(SW_Q) swa_simt_kernel(const SwaArgs a) {
   }
   float m = -INFINITY, l = 0.f;
 
-  const int kmin = max(0, t0 - a.window + 1);
-  const int kmax = min(a.L - 1, t0 + SW_Q - 1);
-  const T* kbase = (const T*)a.k + (size_t)b * a.L * a.ld_k + (size_t)g * D;
-  const T* vbase = (const T*)a.v + (size_t)b * a.L * a.ld_v + (size_t)g * D;
+  const int kmin = max(0, t0 + a.qoff - a.window + 1);
+  const int kmax = min(Lk - 1, t0 + a.qoff + SW_Q - 1);
+  const T* kbase = (const T*)a.k + (size_t)b * Lk * a.ld_k + (size_t)g * D;
+  const T* vbase = (const T*)a.v + (size_t)b * Lk * a.ld_v + (size_t)g * D;
   for (int kb = kmin; kb <= kmax; kb += SW_K) {
     for (int e = tid; e < SW_K * D; e += SW_Q) {
       const int j = e / D, i = e % D;
@@ -59,7 +61,7 @@ __global__ void __launch_bounds__(SW_Q) swa_simt_kernel(const SwaArgs a) {
         float acc = 0.f;
 #pragma unroll
         for (int i = 0; i < D; ++i) acc = fmaf(q[i], Ks[j][i], acc);
-        const bool in_band = s <= t && s > t - a.window;
+        const bool in_band = s <= tk && s > tk - a.window;
         sc[j] = in_band ? acc : -INFINITY;
         bmax = fmaxf(bmax, sc[j]);
       }
@@ -114,7 +116,7 @@ samba_status launch_swa_simt(const SwaArgs& a, cudaStream_t st) {
 }
 
 samba_status launch_swa(const SwaArgs& a, cudaStream_t st) {
-  if (!a.q || !a.k || !a.v || !a.o || a.B < 1 || a.L < 0 || a.Hq < 1 || a.Hkv < 1 || a.window < 1)
+  if (!a.q || !a.k || !a.v || !a.o || a.B < 1 || a.L < 0 || a.Hq < 1 || a.Hkv < 1 || a.window < 1 || a.qoff < 0)
     return SAMBA_ERR_INVALID_ARG;
   if (a.Hq % a.Hkv) return SAMBA_ERR_INVALID_ARG;
   if (a.L == 0) return SAMBA_OK;

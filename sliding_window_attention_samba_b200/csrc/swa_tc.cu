@@ -53,6 +53,7 @@ struct AtParams {
   bf16* o;
   int64_t ld_o;
   int L, window, Hq, Hkv;
+  int qoff, Lk;  // query row t is key row t + qoff; Lk = L + qoff key rows
   float scale_log2;
 };
 
@@ -71,10 +72,11 @@ __global__ void __launch_bounds__(AT_THREADS, 1) swa_tc_kernel(const __grid_cons
   const int b = blockIdx.z;
   const int g = h / (p.Hq / p.Hkv);
 
-  // key tiles intersecting the band of rows t0 .. t0+127
-  const int lo = t0 - p.window + 1;
+  // key tiles intersecting the band of rows t0 .. t0+127 (key rows tk0 .. tk0+127)
+  const int tk0 = t0 + p.qoff;
+  const int lo = tk0 - p.window + 1;
   const int kb0 = lo <= 0 ? 0 : (lo / AT_BN) * AT_BN;
-  const int ntile = (t0 - kb0) / AT_BN + 1;
+  const int ntile = (min(tk0 + AT_BM - 1, p.Lk - 1) - kb0) / AT_BN + 1;
 
   if (warp == 0 && lane == 0) {
     mbar_init(&S.q_full, 1);
@@ -166,7 +168,8 @@ __global__ void __launch_bounds__(AT_THREADS, 1) swa_tc_kernel(const __grid_cons
     // front of them and the rescale decision are made warp-uniform.
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;  // query row within the tile == TMEM lane
-    const int t = t0 + r;
+    const int tq = t0 + r;         // query row
+    const int t = tk0 + r;         // its key row
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
       const bool w = mbar_wait(bar, par, err);
@@ -190,12 +193,12 @@ __global__ void __launch_bounds__(AT_THREADS, 1) swa_tc_kernel(const __grid_cons
       // Row max on the raw scores (the softmax scale is positive and folded into
       // the exponent below).  Only the two edge tiles need the band mask; there the
       // valid key offsets of row t are (t - w - kb, t - kb], empty for t >= L.
-      const bool edge = (kb + AT_BN - 1 > t0) || (kb < t0 + AT_BM - p.window);
+      const bool edge = (kb + AT_BN - 1 > tk0) || (kb < tk0 + AT_BM - p.window);
       float m8[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
       if (edge) {
-        const int hi = t < p.L ? t - kb : -1;
+        const int hi = tq < p.L ? t - kb : -1;
         const int lo = t - p.window - kb;
 #pragma unroll
         for (int i = 0; i < 128; ++i) {
@@ -266,9 +269,9 @@ __global__ void __launch_bounds__(AT_THREADS, 1) swa_tc_kernel(const __grid_cons
       tmem_ld32(tO + lane_off, orr);
       tmem_ld32(tO + lane_off + 32, orr + 32);
       tmem_wait_ld();
-      if (t < p.L && l_run > 0.f) {
+      if (tq < p.L && l_run > 0.f) {
         const float inv = 1.f / l_run;
-        bf16* op = p.o + ((int64_t)b * p.L + t) * p.ld_o + (int64_t)h * AT_D;
+        bf16* op = p.o + ((int64_t)b * p.L + tq) * p.ld_o + (int64_t)h * AT_D;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           float f[8];
@@ -318,9 +321,10 @@ __global__ void __launch_bounds__(A2_THREADS, 1) swa_tc2_kernel(const __grid_con
   const int h0 = blockIdx.y * 2;
   const int b = blockIdx.z;
   const int g = h0 / (p.Hq / p.Hkv);
-  const int lo = t0 - p.window + 1;
+  const int tk0 = t0 + p.qoff;  // key row of query row t0
+  const int lo = tk0 - p.window + 1;
   const int kb0 = lo <= 0 ? 0 : (lo / AT_BN) * AT_BN;
-  const int ntile = (t0 - kb0) / AT_BN + 1;
+  const int ntile = (min(tk0 + AT_BM - 1, p.Lk - 1) - kb0) / AT_BN + 1;
 
   if (warp == 0 && lane == 0) {
     mbar_init(&S.q_full, 1);
@@ -411,7 +415,8 @@ __global__ void __launch_bounds__(A2_THREADS, 1) swa_tc2_kernel(const __grid_con
     const int wg = (warp - 2) >> 2;  // 0: head h0, 1: head h0 + 1
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
-    const int t = t0 + r;
+    const int tq = t0 + r;  // query row
+    const int t = tk0 + r;  // its key row
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const uint32_t tS = tmem + wg * 128u + lane_off;
     const uint32_t tO = tmem + 256u + wg * 64u + lane_off;
@@ -425,8 +430,8 @@ __global__ void __launch_bounds__(A2_THREADS, 1) swa_tc2_kernel(const __grid_con
       const int kb = kb0 + j * AT_BN;
       if (!wait_all(&S.s_full[wg], j & 1)) { ok = false; break; }
       tc_fence_after();
-      const bool edge = (kb + AT_BN - 1 > t0) || (kb < t0 + AT_BM - p.window);
-      const int hi = t < p.L ? t - kb : -1;  // valid key offsets of row t: (lo_i, hi]
+      const bool edge = (kb + AT_BN - 1 > tk0) || (kb < tk0 + AT_BM - p.window);
+      const int hi = tq < p.L ? t - kb : -1;  // valid key offsets of row t: (lo_i, hi]
       const int lo_i = t - p.window - kb;
       // pass 1: row max of the raw scores
       float m8[8];
@@ -516,9 +521,9 @@ __global__ void __launch_bounds__(A2_THREADS, 1) swa_tc2_kernel(const __grid_con
       tmem_ld32(tO, orr);
       tmem_ld32(tO + 32, orr + 32);
       tmem_wait_ld();
-      if (t < p.L && l_run > 0.f) {
+      if (tq < p.L && l_run > 0.f) {
         const float inv = 1.f / l_run;
-        bf16* op = p.o + ((int64_t)b * p.L + t) * p.ld_o + (int64_t)(h0 + wg) * AT_D;
+        bf16* op = p.o + ((int64_t)b * p.L + tq) * p.ld_o + (int64_t)(h0 + wg) * AT_D;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           float f[8];
@@ -557,12 +562,15 @@ bool swa_tc_supported(const SwaArgs& a) {
 samba_status launch_swa_tc(const SwaArgs& a, cudaStream_t st) {
   AtParams p;
   memset(&p, 0, sizeof(p));
-  if (!make_head_map(&p.tmQ, a.q, a.ld_q, a.Hq, a.L, a.B) || !make_head_map(&p.tmK, a.k, a.ld_k, a.Hkv, a.L, a.B) ||
-      !make_head_map(&p.tmV, a.v, a.ld_v, a.Hkv, a.L, a.B))
+  const int Lk = a.L + a.qoff;
+  if (!make_head_map(&p.tmQ, a.q, a.ld_q, a.Hq, a.L, a.B) || !make_head_map(&p.tmK, a.k, a.ld_k, a.Hkv, Lk, a.B) ||
+      !make_head_map(&p.tmV, a.v, a.ld_v, a.Hkv, Lk, a.B))
     return SAMBA_ERR_CUDA;
   p.o = (bf16*)a.o;
   p.ld_o = a.ld_o;
   p.L = a.L;
+  p.qoff = a.qoff;
+  p.Lk = Lk;
   p.window = a.window;
   p.Hq = a.Hq;
   p.Hkv = a.Hkv;
