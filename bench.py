@@ -369,9 +369,24 @@ def kernel_report(kt, s, T, Bn, Ln, peaks):
     conv_bytes = T * s.d_inner * 4
     rep["conv"] = {"gbs": conv_bytes / kt["conv"] / 1e9, "ms": kt["conv"] * 1e3}
     rep["rmsnorm"] = {"gbs": T * s.d_model * 4 / kt["rmsnorm"] / 1e9, "ms": kt["rmsnorm"] * 1e3}
-    roof = {"bound": "tensor", "achieved": round(g_flops / n_g / (g_time / n_g) / 1e12, 2), "peak": tf_sus,
-            "unit": "TFLOP/s", "frac": round(g_flops / g_time / 1e12 / tf_sus, 4), "traffic": None,
-            "kernel": "gemm_tc (all projections of a block, flop-weighted)", "peak_source": src + " sustained bf16"}
+    rep["gemm"]["frac_of_" + src + "_burst_bf16_peak"] = g_flops / g_time / 1e12 / tf_burst
+    # Dominant kernel: the SwiGLU up-projection (gemm_tc_kernel<2>, ~32% of the
+    # step in the launch list).  Timed alone by the attribution pass, so against
+    # the burst peak.  DRAM traffic per launch from an ncu capture of this kernel
+    # at M = 16384 (dram__bytes_read.sum 203.3 MB, dram__bytes_write.sum 237.3 MB),
+    # scaled to this M: the activation reads and the output writes grow with M,
+    # the 67 MB of weights are read once whatever M is.
+    name = "mlp1_up"
+    up = [fl for (n, M, N, K, e, fl) in gl if n == name][0]
+    w_bytes = 2 * s.d_ff * s.d_model * 2
+    scale = T / 16384
+    traffic = (203.3e6 - w_bytes) * scale + w_bytes + 237.3e6 * scale
+    roof = {"bound": "tensor", "achieved": round(up / kt[name] / 1e12, 2), "peak": tf_burst, "unit": "TFLOP/s",
+            "frac": round(up / kt[name] / 1e12 / tf_burst, 4), "traffic": round(traffic),
+            "algorithmic_bytes": T * s.d_model * 2 + w_bytes + T * s.d_ff * 2,
+            "kernel": "gemm_tc_kernel<2>: SwiGLU up-projection [T, d_model] x [2 d_ff, d_model]^T",
+            "peak_source": src + " burst bf16 (kernel timed alone)",
+            "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum at M=16384, scaled to M"}
     return roof, rep
 
 

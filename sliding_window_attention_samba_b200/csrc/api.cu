@@ -181,13 +181,15 @@ static GemmArgs gemm1(const void* A, int64_t lda, const void* W, int64_t M, int 
 // SwiGLU MLP sub-layer: x_next = x + W3 ((W1 xn) * SiLU(W2 xn))  [Samba 3.4 "SwiGLU Formulation"]
 static samba_status mlp_sublayer(const samba_block_config& c, const float* g, const void* W1, const void* W2,
                                  const void* W3, const void* x, void* x_next, void* xn, void* hmlp, void* tap,
-                                 int64_t T, cudaStream_t st) {
-  TRY(launch_rmsnorm(x, c.d_model, g, xn, c.d_model, T, c.d_model, c.norm_eps, c.dtype, st));
+                                 int64_t T, cudaStream_t st, bool pdl = false) {
+  TRY(launch_rmsnorm(x, c.d_model, g, xn, c.d_model, T, c.d_model, c.norm_eps, c.dtype, st, pdl));
   GemmArgs up = gemm1(xn, c.d_model, W1, T, c.d_ff, c.d_model, hmlp, c.d_ff, c.dtype);
   up.seg[0].W2 = W2;
   up.epi = kEpiSwiglu;
+  up.pdl = pdl;
   TRY(launch_gemm(up, st));
   GemmArgs dn = gemm1(hmlp, c.d_ff, W3, T, c.d_model, c.d_ff, x_next, c.d_model, c.dtype);
+  dn.pdl = pdl;
   dn.epi = kEpiResid;
   dn.resid = x;
   dn.ldr = c.d_model;
@@ -365,52 +367,33 @@ size_t samba_block_workspace_size(const samba_block_config* cfg, int B, int L) {
 
 namespace samba {
 
-// One block over B x L tokens.  pos0 > 0 continues a prefill from the decode
-// state `stt` holds after pos0 tokens (chunked prefill): the conv history, the
-// SSM state and the ring's last window of K/V are the inputs before token 0,
-// RoPE positions start at pos0, and the state is advanced to pos0 + L.
-static samba_status block_forward(const samba_block_config* cfg, const samba_block_weights* w, const void* x_in,
-                                  void* x_out, samba_decode_state* stt, int64_t pos0, const samba_block_taps* taps,
-                                  int B, int L, void* workspace, size_t workspace_bytes, samba_stream stream) {
-  TRY(validate_cfg(cfg));
-  TRY(validate_weights(w));
-  if (B < 1 || L < 0 || pos0 < 0) return SAMBA_ERR_INVALID_ARG;
-  if (L > 0 && (!x_in || !x_out || x_in == x_out)) return SAMBA_ERR_INVALID_ARG;
-  if (stt && (!stt->ssm || !stt->conv || !stt->k_ring || !stt->v_ring || !stt->pos)) return SAMBA_ERR_INVALID_ARG;
-  const bool resume = pos0 > 0;
-  if (resume && !stt) return SAMBA_ERR_INVALID_ARG;
-  if (pos0 + (int64_t)L > (int64_t(1) << 30)) return SAMBA_ERR_UNSUPPORTED;
-  const samba_block_config& c = *cfg;
-  const int64_t T = (int64_t)B * L;
-  const BlockPlan P = plan_block(c, T, resume ? B : 0);
-  if (!workspace || workspace_bytes < P.total) return SAMBA_ERR_INVALID_ARG;
-  if (!aligned16(x_in) || !aligned16(x_out)) return SAMBA_ERR_UNSUPPORTED;
-  cudaStream_t st = (cudaStream_t)stream;
+// Shapes, workspace plan and stream shared by the sub-layers of one call.
+struct LayerCtx {
+  const samba_block_config& c;
+  const BlockPlan& P;
+  char* base;  // workspace, 256-byte aligned
+  int B, L;
+  int64_t T;
+  cudaStream_t st;
+};
+
+// Mamba sub-layer over B x L tokens: x_out = x_in + Mamba(RMSNorm(x_in))
+// [Samba 3.4 "The Mamba Layer"].  stt: NULL, or the decode state, overwritten
+// with the state after the last token (resume: the layer continues from it).
+static samba_status mamba_sublayer(const LayerCtx& X, const samba_block_weights* w, const void* x_in, void* x_out,
+                                   samba_decode_state* stt, bool resume, void* tap) {
+  const samba_block_config& c = X.c;
+  const BlockPlan& P = X.P;
+  const int B = X.B, L = X.L;
+  const int64_t T = X.T;
+  cudaStream_t st = X.st;
   const samba_dtype dt = c.dtype;
-  char* base = (char*)(((uintptr_t)workspace + 255) & ~uintptr_t(255));
-  auto buf = [&](size_t off) -> void* { return base + off; };
+  auto buf = [&](size_t off) -> void* { return X.base + off; };
   const int Di = c.d_inner, Dm = c.d_model, N = c.d_state, R = c.dt_rank;
   const size_t es = dtype_size(dt);
-  void* x1 = (taps && taps->resid[0]) ? taps->resid[0] : buf(P.x1);
-  void* x2 = (taps && taps->resid[1]) ? taps->resid[1] : buf(P.x2);
-  void* x3 = (taps && taps->resid[2]) ? taps->resid[2] : buf(P.x3);
   void* xn = buf(P.xn);
   char* hz = (char*)buf(P.hz);
   char* xdbl = (char*)buf(P.xdbl);
-  char* qkv = (char*)buf(P.qkv);
-  float2* tab = (float2*)buf(P.tab);
-
-  if (T == 0 && resume) return launch_pos_check_set(stt->pos, B, pos0, pos0, st);
-  if (T == 0) {
-    if (stt) {
-      TRY(launch_pos_update(stt->pos, B, 0, true, st));
-      cudaMemsetAsync(stt->ssm, 0, (size_t)B * Di * N * sizeof(float), st);
-      cudaMemsetAsync(stt->conv, 0, (size_t)B * Di * (c.d_conv - 1) * es, st);
-    }
-    return SAMBA_OK;
-  }
-
-  // ---- Mamba sub-layer [Samba 3.4 "The Mamba Layer"]
   TRY(launch_rmsnorm(x_in, Dm, w->norm_g[0], xn, Dm, T, Dm, c.norm_eps, dt, st));
   TRY(launch_gemm(gemm1(xn, Dm, w->W_in, T, 2 * Di, Dm, hz, 2 * Di, dt), st));  // H | X W_g
   {
@@ -465,19 +448,37 @@ static samba_status block_forward(const samba_block_config* cfg, const samba_blo
     TRY(launch_selective_scan(a, st));
   }
   {
-    GemmArgs g = gemm1(buf(P.y), Di, w->W_out, T, Dm, Di, x1, Dm, dt);
+    GemmArgs g = gemm1(buf(P.y), Di, w->W_out, T, Dm, Di, x_out, Dm, dt);
     g.epi = kEpiResid;
     g.resid = x_in;
     g.ldr = Dm;
-    g.tap = taps ? taps->branch[0] : nullptr;
+    g.tap = tap;
     g.ldt = Dm;
     TRY(launch_gemm(g, st));
   }
-  // ---- MLP 1
-  TRY(mlp_sublayer(c, w->norm_g[1], w->mlp1_W1, w->mlp1_W2, w->mlp1_W3, x1, x2, xn, buf(P.hmlp),
-                   taps ? taps->branch[1] : nullptr, T, st));
-  // ---- SWA sub-layer [Samba 3.4 "The Sliding Window Attention (SWA) Layer"]
-  TRY(launch_rmsnorm(x2, Dm, w->norm_g[2], xn, Dm, T, Dm, c.norm_eps, dt, st));
+  return SAMBA_OK;
+}
+
+// SWA sub-layer over B x L tokens: x_out = x_in + SWA(RMSNorm(x_in))
+// [Samba 3.4 "The Sliding Window Attention (SWA) Layer"]; RoPE positions start
+// at pos0.  stt: NULL, or the decode state whose ring receives the last
+// min(L, window) keys/values (resume: the ring also supplies the keys of the
+// min(pos0, window-1) tokens before this chunk).
+static samba_status swa_sublayer(const LayerCtx& X, const samba_block_weights* w, const void* x_in, void* x_out,
+                                 samba_decode_state* stt, int64_t pos0, bool resume, void* tap) {
+  const samba_block_config& c = X.c;
+  const BlockPlan& P = X.P;
+  const int B = X.B, L = X.L;
+  const int64_t T = X.T;
+  cudaStream_t st = X.st;
+  const samba_dtype dt = c.dtype;
+  auto buf = [&](size_t off) -> void* { return X.base + off; };
+  const int Dm = c.d_model;
+  const size_t es = dtype_size(dt);
+  void* xn = buf(P.xn);
+  char* qkv = (char*)buf(P.qkv);
+  float2* tab = (float2*)buf(P.tab);
+  TRY(launch_rmsnorm(x_in, Dm, w->norm_g[2], xn, Dm, T, Dm, c.norm_eps, dt, st));
   const int hd = c.head_dim;
   const int qw = c.n_q * hd, kvw = c.n_kv * hd;
   {
@@ -530,14 +531,64 @@ static samba_status block_forward(const samba_block_config* cfg, const samba_blo
   if (stt)
     TRY(launch_ring_fill(qkv, P.qkvw, qw, qw + kvw, stt->k_ring, stt->v_ring, B, L, pos0, c.window, kvw, dt, st));
   {
-    GemmArgs g = gemm1(buf(P.o), qw, w->Wo, T, Dm, qw, x3, Dm, dt);
+    GemmArgs g = gemm1(buf(P.o), qw, w->Wo, T, Dm, qw, x_out, Dm, dt);
     g.epi = kEpiResid;
-    g.resid = x2;
+    g.resid = x_in;
     g.ldr = Dm;
-    g.tap = taps ? taps->branch[2] : nullptr;
+    g.tap = tap;
     g.ldt = Dm;
     TRY(launch_gemm(g, st));
   }
+  return SAMBA_OK;
+}
+
+// One block over B x L tokens.  pos0 > 0 continues a prefill from the decode
+// state `stt` holds after pos0 tokens (chunked prefill): the conv history, the
+// SSM state and the ring's last window of K/V are the inputs before token 0,
+// RoPE positions start at pos0, and the state is advanced to pos0 + L.
+static samba_status block_forward(const samba_block_config* cfg, const samba_block_weights* w, const void* x_in,
+                                  void* x_out, samba_decode_state* stt, int64_t pos0, const samba_block_taps* taps,
+                                  int B, int L, void* workspace, size_t workspace_bytes, samba_stream stream) {
+  TRY(validate_cfg(cfg));
+  TRY(validate_weights(w));
+  if (B < 1 || L < 0 || pos0 < 0) return SAMBA_ERR_INVALID_ARG;
+  if (L > 0 && (!x_in || !x_out || x_in == x_out)) return SAMBA_ERR_INVALID_ARG;
+  if (stt && (!stt->ssm || !stt->conv || !stt->k_ring || !stt->v_ring || !stt->pos)) return SAMBA_ERR_INVALID_ARG;
+  const bool resume = pos0 > 0;
+  if (resume && !stt) return SAMBA_ERR_INVALID_ARG;
+  if (pos0 + (int64_t)L > (int64_t(1) << 30)) return SAMBA_ERR_UNSUPPORTED;
+  const samba_block_config& c = *cfg;
+  const int64_t T = (int64_t)B * L;
+  const BlockPlan P = plan_block(c, T, resume ? B : 0);
+  if (!workspace || workspace_bytes < P.total) return SAMBA_ERR_INVALID_ARG;
+  if (!aligned16(x_in) || !aligned16(x_out)) return SAMBA_ERR_UNSUPPORTED;
+  cudaStream_t st = (cudaStream_t)stream;
+  const samba_dtype dt = c.dtype;
+  char* base = (char*)(((uintptr_t)workspace + 255) & ~uintptr_t(255));
+  auto buf = [&](size_t off) -> void* { return base + off; };
+  const int Di = c.d_inner, N = c.d_state;
+  const size_t es = dtype_size(dt);
+  void* x1 = (taps && taps->resid[0]) ? taps->resid[0] : buf(P.x1);
+  void* x2 = (taps && taps->resid[1]) ? taps->resid[1] : buf(P.x2);
+  void* x3 = (taps && taps->resid[2]) ? taps->resid[2] : buf(P.x3);
+  void* xn = buf(P.xn);
+
+  if (T == 0 && resume) return launch_pos_check_set(stt->pos, B, pos0, pos0, st);
+  if (T == 0) {
+    if (stt) {
+      TRY(launch_pos_update(stt->pos, B, 0, true, st));
+      cudaMemsetAsync(stt->ssm, 0, (size_t)B * Di * N * sizeof(float), st);
+      cudaMemsetAsync(stt->conv, 0, (size_t)B * Di * (c.d_conv - 1) * es, st);
+    }
+    return SAMBA_OK;
+  }
+
+  const LayerCtx X{c, P, base, B, L, T, st};
+  TRY(mamba_sublayer(X, w, x_in, x1, stt, resume, taps ? taps->branch[0] : nullptr));
+  // ---- MLP 1
+  TRY(mlp_sublayer(c, w->norm_g[1], w->mlp1_W1, w->mlp1_W2, w->mlp1_W3, x1, x2, xn, buf(P.hmlp),
+                   taps ? taps->branch[1] : nullptr, T, st));
+  TRY(swa_sublayer(X, w, x2, x3, stt, pos0, resume, taps ? taps->branch[2] : nullptr));
   // ---- MLP 2
   TRY(mlp_sublayer(c, w->norm_g[3], w->mlp2_W1, w->mlp2_W2, w->mlp2_W3, x3, x_out, xn, buf(P.hmlp),
                    taps ? taps->branch[3] : nullptr, T, st));
@@ -591,7 +642,7 @@ samba_status samba_step(const samba_block_config* cfg, const samba_block_weights
   const samba_dtype dt = c.dtype;
   char* base = (char*)(((uintptr_t)workspace + 255) & ~uintptr_t(255));
   auto buf = [&](size_t off) -> void* { return base + off; };
-  const int Di = c.d_inner, Dm = c.d_model, N = c.d_state, R = c.dt_rank;
+  const int Di = c.d_inner, Dm = c.d_model, R = c.dt_rank;
   const size_t es = dtype_size(dt);
   void* xn = buf(P.xn);
   char* hz = (char*)buf(P.hz);
@@ -601,15 +652,22 @@ samba_status samba_step(const samba_block_config* cfg, const samba_block_weights
   void *x1 = buf(P.x1), *x2 = buf(P.x2), *x3 = buf(P.x3);
 
   // ---- Mamba, one step
-  TRY(launch_rmsnorm(x_t, Dm, w->norm_g[0], xn, Dm, B, Dm, c.norm_eps, dt, st));
-  TRY(launch_gemm(gemm1(xn, Dm, w->W_in, B, 2 * Di, Dm, hz, 2 * Di, dt), st));
+  // Every launch of the step is a programmatic dependent of the one before it:
+  // a kernel sets up (and the projections fetch their first weight tiles) while
+  // its predecessor finishes.
+  auto gemm_pdl = [&](GemmArgs g) {
+    g.pdl = true;
+    return launch_gemm(g, st);
+  };
+  TRY(launch_rmsnorm(x_t, Dm, w->norm_g[0], xn, Dm, B, Dm, c.norm_eps, dt, st, true));
+  TRY(gemm_pdl(gemm1(xn, Dm, w->W_in, B, 2 * Di, Dm, hz, 2 * Di, dt)));
   TRY(launch_conv_step(hz, 2 * Di, w->conv_w, w->conv_b, stt->conv, buf(P.u), B, Di, c.d_conv, dt, st));
-  TRY(launch_gemm(gemm1(buf(P.u), Di, w->W_x, B, P.xdw, Di, xdbl, P.xdw, dt), st));
+  TRY(gemm_pdl(gemm1(buf(P.u), Di, w->W_x, B, P.xdw, Di, xdbl, P.xdw, dt)));
   {
     GemmArgs g = gemm1(xdbl, P.xdw, w->W_dt, B, Di, R, buf(P.dlt), Di, dt);
     g.epi = kEpiSoftplus;
     g.bias = w->dt_bias;
-    TRY(launch_gemm(g, st));
+    TRY(gemm_pdl(g));
   }
   TRY(launch_scan_step(buf(P.u), buf(P.dlt), hz + (size_t)Di * es, 2 * Di, xdbl, P.xdw, R, w->A_log, w->Dskip,
                        stt->ssm, buf(P.y), B, Di, dt, st));
@@ -618,11 +676,12 @@ samba_status samba_step(const samba_block_config* cfg, const samba_block_weights
     g.epi = kEpiResid;
     g.resid = x_t;
     g.ldr = Dm;
-    TRY(launch_gemm(g, st));
+    TRY(gemm_pdl(g));
   }
-  TRY(mlp_sublayer(c, w->norm_g[1], w->mlp1_W1, w->mlp1_W2, w->mlp1_W3, x1, x2, xn, buf(P.hmlp), nullptr, B, st));
+  TRY(mlp_sublayer(c, w->norm_g[1], w->mlp1_W1, w->mlp1_W2, w->mlp1_W3, x1, x2, xn, buf(P.hmlp), nullptr, B, st,
+                   true));
   // ---- SWA over the ring
-  TRY(launch_rmsnorm(x2, Dm, w->norm_g[2], xn, Dm, B, Dm, c.norm_eps, dt, st));
+  TRY(launch_rmsnorm(x2, Dm, w->norm_g[2], xn, Dm, B, Dm, c.norm_eps, dt, st, true));
   const int hd = c.head_dim;
   const int qw = c.n_q * hd, kvw = c.n_kv * hd;
   {
@@ -635,14 +694,14 @@ samba_status samba_step(const samba_block_config* cfg, const samba_block_weights
     g.seg[2].W = w->Wv;
     g.seg[2].n = kvw;
     if (c.rope_base != 0.f) {
-      TRY(launch_build_rope_table(tab, hd, c.rope_base, st));
+      TRY(launch_build_rope_table(tab, hd, c.rope_base, st, true));
       g.epi = kEpiRope;
       g.rope_cols = qw + kvw;
       g.head_dim = hd;
       g.pos_dev = stt->pos;
       g.rope_tab = tab;
     }
-    TRY(launch_gemm(g, st));
+    TRY(gemm_pdl(g));
   }
   TRY(launch_ring_write(qkv, P.qkvw, qw, qw + kvw, stt->pos, stt->k_ring, stt->v_ring, B, c.window, kvw, dt, st));
   TRY(launch_attn_decode(qkv, P.qkvw, stt->pos, stt->k_ring, stt->v_ring, buf(P.o), B, c.n_q, c.n_kv, hd, c.window,
@@ -652,10 +711,11 @@ samba_status samba_step(const samba_block_config* cfg, const samba_block_weights
     g.epi = kEpiResid;
     g.resid = x2;
     g.ldr = Dm;
-    TRY(launch_gemm(g, st));
+    TRY(gemm_pdl(g));
   }
-  TRY(mlp_sublayer(c, w->norm_g[3], w->mlp2_W1, w->mlp2_W2, w->mlp2_W3, x3, y_t, xn, buf(P.hmlp), nullptr, B, st));
-  return launch_pos_update(stt->pos, B, 1, false, st);
+  TRY(mlp_sublayer(c, w->norm_g[3], w->mlp2_W1, w->mlp2_W2, w->mlp2_W3, x3, y_t, xn, buf(P.hmlp), nullptr, B, st,
+                   true));
+  return launch_pos_update(stt->pos, B, 1, false, st, true);
 }
 
 }  // extern "C"

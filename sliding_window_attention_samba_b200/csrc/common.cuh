@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <string.h>
 #include <cudaTypedefs.h>
 #include <stdint.h>
 
@@ -303,6 +304,15 @@ __device__ __forceinline__ bool elect_one() {
   return pred != 0;
 }
 
+// Programmatic dependent launch.  A kernel launched with launch_k(..., pdl=true)
+// may begin while the previous kernel of the stream is still running; it calls
+// pdl_wait() before it reads or writes any memory that earlier kernels read or
+// write (weights, which nothing writes, may be fetched before), and pdl_trigger()
+// to let the next kernel of the stream begin early in turn.  Both are no-ops
+// for a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
@@ -334,6 +344,25 @@ inline bool ensure_smem_attr(K kern, size_t bytes) {
 // elements (innermost first); strides[i] is the stride of dim i+1.
 bool make_tmap(CUtensorMap* m, const void* base, samba_dtype dt, int rank, const uint64_t* dims,
                const uint64_t* strides_elems, const uint32_t* box, CUtensorMapSwizzle swz);
+
+// Launch `kern` on `st`; with pdl, as a programmatic dependent of the previous
+// kernel on the stream (see pdl_wait).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+                            Args... args) {
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
 
 #define SAMBA_CHECK_LAUNCH()                                 \
   do {                                                       \

@@ -17,6 +17,8 @@ template <typename T>
 __global__ void conv_step_kernel(const T* __restrict__ hz, int64_t ld_hz, const float* __restrict__ w,
                                  const float* __restrict__ bias, T* __restrict__ state, T* __restrict__ u, int B,
                                  int D, int k) {
+  pdl_wait();
+  pdl_trigger();
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= B * D) return;
   const int b = idx / D, c = idx % D;
@@ -39,6 +41,8 @@ __global__ void scan_step_kernel(const T* __restrict__ u, const T* __restrict__ 
                                  int64_t ld_z, const T* __restrict__ xdbl, int64_t ld_x, int r_off,
                                  const float* __restrict__ A_log, const float* __restrict__ Dskip,
                                  float* __restrict__ ssm, T* __restrict__ y, int B, int D) {
+  pdl_wait();
+  pdl_trigger();
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= B * D) return;
   const int b = idx / D, c = idx % D;
@@ -68,6 +72,8 @@ template <typename T>
 __global__ void ring_write_kernel(const T* __restrict__ qkv, int64_t ld, int k_off, int v_off,
                                   const int64_t* __restrict__ pos, T* __restrict__ k_ring, T* __restrict__ v_ring,
                                   int window, int kvw) {
+  pdl_wait();
+  pdl_trigger();
   const int b = blockIdx.x;
   const int64_t slot = pos[b] % window;
   const T* src = qkv + (size_t)b * ld;
@@ -89,6 +95,8 @@ template <typename T>
 __global__ void attn_decode_kernel(const T* __restrict__ qkv, int64_t ld, const int64_t* __restrict__ pos,
                                    const T* __restrict__ k_ring, const T* __restrict__ v_ring, T* __restrict__ o,
                                    int Hq, int Hkv, int hd, int window, float scale) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ float dsm[];
   const int g = blockIdx.x, b = blockIdx.y;
   const int grp = Hq / Hkv;
@@ -224,6 +232,8 @@ __global__ void __launch_bounds__(256, 1)
     attn_decode_split_kernel(const bf16* __restrict__ qkv, int64_t ld, const int64_t* __restrict__ pos,
                              const bf16* __restrict__ k_ring, const bf16* __restrict__ v_ring, bf16* __restrict__ o,
                              int Hq, int Hkv, int window, float scale_log2) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(16) unsigned char dec_dyn[];  // K slice | V slice (bf16, padded rows)
   bf16* Ks = reinterpret_cast<bf16*>(dec_dyn);
   bf16* Vs = Ks + kSliceMax * kKvPad;
@@ -401,6 +411,8 @@ __global__ void __launch_bounds__(256, 1)
 }
 
 __global__ void pos_add_kernel(int64_t* pos, int B, int64_t inc, int set) {
+  pdl_wait();
+  pdl_trigger();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < B) pos[i] = set ? inc : pos[i] + inc;
 }
@@ -474,12 +486,13 @@ samba_status launch_conv_step(const void* hz, int64_t ld_hz, const float* w, con
                               int B, int D, int k, samba_dtype dt, cudaStream_t st) {
   if (k < 2 || k > 8) return SAMBA_ERR_UNSUPPORTED;
   const int n = B * D;
+  cudaError_t e;
   SAMBA_DT_DISPATCH(dt,
-                    (conv_step_kernel<bf16><<<(n + 255) / 256, 256, 0, st>>>((const bf16*)hz, ld_hz, w, bias,
-                                                                             (bf16*)state, (bf16*)u, B, D, k)),
-                    (conv_step_kernel<float><<<(n + 255) / 256, 256, 0, st>>>((const float*)hz, ld_hz, w, bias,
-                                                                              (float*)state, (float*)u, B, D, k)));
-  SAMBA_CHECK_LAUNCH();
+                    (e = launch_k(conv_step_kernel<bf16>, dim3((n + 255) / 256), dim3(256), 0, st, true,
+                                  (const bf16*)hz, ld_hz, w, bias, (bf16*)state, (bf16*)u, B, D, k)),
+                    (e = launch_k(conv_step_kernel<float>, dim3((n + 255) / 256), dim3(256), 0, st, true,
+                                  (const float*)hz, ld_hz, w, bias, (float*)state, (float*)u, B, D, k)));
+  if (e != cudaSuccess) return SAMBA_ERR_CUDA;
   return SAMBA_OK;
 }
 
@@ -487,25 +500,27 @@ samba_status launch_scan_step(const void* u, const void* dlt, const void* z, int
                               int64_t ld_x, int r_off, const float* A_log, const float* Dskip, float* ssm, void* y,
                               int B, int D, samba_dtype dt, cudaStream_t st) {
   const int n = B * D;
+  cudaError_t e;
   SAMBA_DT_DISPATCH(dt,
-                    (scan_step_kernel<bf16><<<(n + 127) / 128, 128, 0, st>>>(
-                        (const bf16*)u, (const bf16*)dlt, (const bf16*)z, ld_z, (const bf16*)xdbl, ld_x, r_off, A_log,
-                        Dskip, ssm, (bf16*)y, B, D)),
-                    (scan_step_kernel<float><<<(n + 127) / 128, 128, 0, st>>>(
-                        (const float*)u, (const float*)dlt, (const float*)z, ld_z, (const float*)xdbl, ld_x, r_off,
-                        A_log, Dskip, ssm, (float*)y, B, D)));
-  SAMBA_CHECK_LAUNCH();
+                    (e = launch_k(scan_step_kernel<bf16>, dim3((n + 127) / 128), dim3(128), 0, st, true,
+                                  (const bf16*)u, (const bf16*)dlt, (const bf16*)z, ld_z, (const bf16*)xdbl, ld_x,
+                                  r_off, A_log, Dskip, ssm, (bf16*)y, B, D)),
+                    (e = launch_k(scan_step_kernel<float>, dim3((n + 127) / 128), dim3(128), 0, st, true,
+                                  (const float*)u, (const float*)dlt, (const float*)z, ld_z, (const float*)xdbl, ld_x,
+                                  r_off, A_log, Dskip, ssm, (float*)y, B, D)));
+  if (e != cudaSuccess) return SAMBA_ERR_CUDA;
   return SAMBA_OK;
 }
 
 samba_status launch_ring_write(const void* qkv, int64_t ld, int k_off, int v_off, const int64_t* pos, void* k_ring,
                                void* v_ring, int B, int window, int kvw, samba_dtype dt, cudaStream_t st) {
+  cudaError_t e;
   SAMBA_DT_DISPATCH(dt,
-                    (ring_write_kernel<bf16><<<B, 128, 0, st>>>((const bf16*)qkv, ld, k_off, v_off, pos,
-                                                                (bf16*)k_ring, (bf16*)v_ring, window, kvw)),
-                    (ring_write_kernel<float><<<B, 128, 0, st>>>((const float*)qkv, ld, k_off, v_off, pos,
-                                                                 (float*)k_ring, (float*)v_ring, window, kvw)));
-  SAMBA_CHECK_LAUNCH();
+                    (e = launch_k(ring_write_kernel<bf16>, dim3(B), dim3(128), 0, st, true, (const bf16*)qkv, ld,
+                                  k_off, v_off, pos, (bf16*)k_ring, (bf16*)v_ring, window, kvw)),
+                    (e = launch_k(ring_write_kernel<float>, dim3(B), dim3(128), 0, st, true, (const float*)qkv, ld,
+                                  k_off, v_off, pos, (float*)k_ring, (float*)v_ring, window, kvw)));
+  if (e != cudaSuccess) return SAMBA_ERR_CUDA;
   return SAMBA_OK;
 }
 
@@ -521,13 +536,15 @@ samba_status launch_attn_decode(const void* qkv, int64_t ld, const int64_t* pos,
     cfg.dynamicSmemBytes = 2 * kSliceMax * kKvPad * sizeof(bf16);
     cfg.stream = st;
     if (!ensure_smem_attr(attn_decode_split_kernel, cfg.dynamicSmemBytes)) return SAMBA_ERR_CUDA;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = kSplit;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     if (cudaLaunchKernelEx(&cfg, attn_decode_split_kernel, (const bf16*)qkv, ld, pos, (const bf16*)k_ring,
                            (const bf16*)v_ring, (bf16*)o, Hq, Hkv, window, scale * 1.4426950408889634f) !=
         cudaSuccess)
@@ -540,20 +557,22 @@ samba_status launch_attn_decode(const void* qkv, int64_t ld, const int64_t* pos,
   if (threads > 1024) return SAMBA_ERR_UNSUPPORTED;
   const size_t smem = 2 * kDecKB * (hd + 1) * sizeof(float);
   dim3 grid(Hkv, B);
+  cudaError_t e;
   SAMBA_DT_DISPATCH(dt,
-                    (attn_decode_kernel<bf16><<<grid, threads, smem, st>>>(
-                        (const bf16*)qkv, ld, pos, (const bf16*)k_ring, (const bf16*)v_ring, (bf16*)o, Hq, Hkv, hd,
-                        window, scale)),
-                    (attn_decode_kernel<float><<<grid, threads, smem, st>>>(
-                        (const float*)qkv, ld, pos, (const float*)k_ring, (const float*)v_ring, (float*)o, Hq, Hkv,
-                        hd, window, scale)));
-  SAMBA_CHECK_LAUNCH();
+                    (e = launch_k(attn_decode_kernel<bf16>, grid, dim3(threads), smem, st, true, (const bf16*)qkv, ld,
+                                  pos, (const bf16*)k_ring, (const bf16*)v_ring, (bf16*)o, Hq, Hkv, hd, window,
+                                  scale)),
+                    (e = launch_k(attn_decode_kernel<float>, grid, dim3(threads), smem, st, true, (const float*)qkv,
+                                  ld, pos, (const float*)k_ring, (const float*)v_ring, (float*)o, Hq, Hkv, hd, window,
+                                  scale)));
+  if (e != cudaSuccess) return SAMBA_ERR_CUDA;
   return SAMBA_OK;
 }
 
-samba_status launch_pos_update(int64_t* pos, int B, int64_t value, bool set, cudaStream_t st) {
-  pos_add_kernel<<<(B + 127) / 128, 128, 0, st>>>(pos, B, value, set ? 1 : 0);
-  SAMBA_CHECK_LAUNCH();
+samba_status launch_pos_update(int64_t* pos, int B, int64_t value, bool set, cudaStream_t st, bool pdl) {
+  if (launch_k(pos_add_kernel, dim3((B + 127) / 128), dim3(128), 0, st, pdl, pos, B, value, set ? 1 : 0) !=
+      cudaSuccess)
+    return SAMBA_ERR_CUDA;
   return SAMBA_OK;
 }
 

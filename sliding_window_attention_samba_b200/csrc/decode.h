@@ -1,4 +1,6 @@
-// Internal launchers of the decode-step kernels (not part of the C ABI).
+// Internal launchers of the decode-step kernels (not part of the C ABI).  The
+// single-token kernels (conv_step, scan_step, ring_write, attn_decode) are
+// launched as programmatic dependents of the previous kernel (see pdl_wait).
 #pragma once
 
 #include "kernels.h"
@@ -15,7 +17,7 @@ samba_status launch_ring_write(const void* qkv, int64_t ld, int k_off, int v_off
 samba_status launch_attn_decode(const void* qkv, int64_t ld, const int64_t* pos, const void* k_ring,
                                 const void* v_ring, void* o, int B, int Hq, int Hkv, int hd, int window, float scale,
                                 samba_dtype dt, cudaStream_t st);
-samba_status launch_pos_update(int64_t* pos, int B, int64_t value, bool set, cudaStream_t st);
+samba_status launch_pos_update(int64_t* pos, int B, int64_t value, bool set, cudaStream_t st, bool pdl = false);
 // prefill -> ring: the last min(L, w) tokens of a prefill whose token 0 is at absolute position pos0
 samba_status launch_ring_fill(const void* qkv, int64_t ld, int k_off, int v_off, void* k_ring, void* v_ring, int B,
                               int L, int64_t pos0, int window, int kvw, samba_dtype dt, cudaStream_t st);

@@ -13,6 +13,8 @@ namespace samba {
 template <typename T>
 __global__ void rmsnorm_kernel(const T* __restrict__ x, int64_t ld_x, const float* __restrict__ g,
                                T* __restrict__ out, int64_t ld_out, int64_t rows, int dim, float eps) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
@@ -39,20 +41,20 @@ __global__ void rmsnorm_kernel(const T* __restrict__ x, int64_t ld_x, const floa
 }
 
 samba_status launch_rmsnorm(const void* x, int64_t ld_x, const float* g, void* out, int64_t ld_out, int64_t rows,
-                            int dim, float eps, samba_dtype dt, cudaStream_t st) {
+                            int dim, float eps, samba_dtype dt, cudaStream_t st, bool pdl) {
   if (!x || !g || !out || rows < 0 || dim <= 0) return SAMBA_ERR_INVALID_ARG;
   if (dim % 8 || ld_x % 8 || ld_out % 8 || !aligned16(x) || !aligned16(out) || !aligned16(g))
     return SAMBA_ERR_UNSUPPORTED;
   if (rows == 0) return SAMBA_OK;
   const int warps = 8;
   dim3 grid((unsigned)((rows + warps - 1) / warps));
-  if (dt == SAMBA_BF16)
-    rmsnorm_kernel<bf16><<<grid, warps * 32, 0, st>>>((const bf16*)x, ld_x, g, (bf16*)out, ld_out, rows, dim, eps);
-  else
-    rmsnorm_kernel<float><<<grid, warps * 32, 0, st>>>((const float*)x, ld_x, g, (float*)out, ld_out, rows, dim,
-                                                       eps);
-  SAMBA_CHECK_LAUNCH();
-  return SAMBA_OK;
+  const cudaError_t e =
+      dt == SAMBA_BF16
+          ? launch_k(rmsnorm_kernel<bf16>, grid, dim3(warps * 32), 0, st, pdl, (const bf16*)x, ld_x, g, (bf16*)out,
+                     ld_out, rows, dim, eps)
+          : launch_k(rmsnorm_kernel<float>, grid, dim3(warps * 32), 0, st, pdl, (const float*)x, ld_x, g,
+                     (float*)out, ld_out, rows, dim, eps);
+  return e == cudaSuccess ? SAMBA_OK : SAMBA_ERR_CUDA;
 }
 
 // ===========================================================================
@@ -188,6 +190,8 @@ size_t rope_table_bytes(int head_dim) {
 }
 
 __global__ void build_rope_table_kernel(float2* tab, int half, int head_dim, double base) {
+  pdl_wait();
+  pdl_trigger();
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   const int total = kRopeLevels * kRopeRadix * half;
   if (idx >= total) return;
@@ -202,12 +206,13 @@ __global__ void build_rope_table_kernel(float2* tab, int half, int head_dim, dou
   tab[idx] = make_float2((float)c, (float)s);
 }
 
-samba_status launch_build_rope_table(float2* tab, int head_dim, float base, cudaStream_t st) {
+samba_status launch_build_rope_table(float2* tab, int head_dim, float base, cudaStream_t st, bool pdl) {
   const int half = head_dim / 2;
   const int total = kRopeLevels * kRopeRadix * half;
-  build_rope_table_kernel<<<(total + 255) / 256, 256, 0, st>>>(tab, half, head_dim, (double)base);
-  SAMBA_CHECK_LAUNCH();
-  return SAMBA_OK;
+  return launch_k(build_rope_table_kernel, dim3((total + 255) / 256), dim3(256), 0, st, pdl, tab, half, head_dim,
+                  (double)base) == cudaSuccess
+             ? SAMBA_OK
+             : SAMBA_ERR_CUDA;
 }
 
 template <typename T>

@@ -6,7 +6,7 @@
 // Two kernels:
 //  * gemm_tc: bf16 operands, fp32 accumulation on the 5th-generation tensor
 //    cores.  Persistent, warp specialised (warp 0: TMA producer, warp 1: MMA
-//    issuer + TMEM owner, warps 2-5: epilogue).  A 4-stage ring of 128x64 A and
+//    issuer + TMEM owner, warps 2-9: epilogue).  A 4-stage ring of 128x64 A and
 //    up to 256x64 B tiles in 128-byte-swizzled shared memory feeds
 //    tcgen05.mma (M=128, N<=256, K=16) issued by one thread into a double
 //    buffered 2x256-column TMEM accumulator, so the epilogue of one tile
@@ -168,7 +168,8 @@ samba_status simt_dispatch(const GemmArgs& a, cudaStream_t st) {
 // tcgen05 kernel
 // ===========================================================================
 constexpr int TC_BM = 128, TC_BK = 64, TC_STAGES = 4, TC_MAXN = 256;
-constexpr int TC_THREADS = 192;
+constexpr int TC_EPI_WARPS = 8;  // two per TMEM lane quadrant, each taking half of the tile's columns
+constexpr int TC_THREADS = 64 + 32 * TC_EPI_WARPS;
 constexpr uint32_t TC_A_BYTES = TC_BM * TC_BK * 2;
 constexpr uint32_t TC_B_BYTES = TC_MAXN * TC_BK * 2;
 
@@ -187,23 +188,42 @@ struct TcParams {
   int bn;          // output columns per tile
   int umma_n;      // accumulator columns per tile (2*bn for SwiGLU)
   int n_tiles, m_tiles, k_blocks;
+  int group_n;  // n-tiles per raster group (divides n_tiles)
   int seg_start[3];
 };
 
+// Tile order: groups of group_n n-tiles; within a group every m-tile in turn,
+// the group's n-tiles consecutive.  The CTAs in flight then share one group's
+// weight panel (kept in L2 for the whole sweep) and each A row block is read
+// once per group, instead of every wave streaming the whole weight matrix.
 __device__ __forceinline__ void tc_tile_coords(const TcParams& p, int tile, int& mt, int& nt) {
-  mt = tile / p.n_tiles;
-  nt = tile % p.n_tiles;
+  const int per_group = p.group_n * p.m_tiles;
+  const int g = tile / per_group, w = tile % per_group;
+  mt = w / p.group_n;
+  nt = g * p.group_n + w % p.group_n;
 }
 
+// Columns [c_lo, c_hi) of one 32-column-chunk split: half 0 takes the first
+// ceil(n/2) of n units, half 1 the rest.
+__device__ __forceinline__ void half_range(int n, int half, int& lo, int& hi) {
+  const int split = (n + 1) / 2;
+  lo = half ? split : 0;
+  hi = half ? n : split;
+}
+
+// One epilogue warp's share of a tile: TMEM lane quadrant = 32 rows, and half
+// `half` of the tile's column units (32-column chunks; 64-column heads for RoPE).
 template <int EPI>
-__device__ __forceinline__ void tc_epilogue_tile(const TcParams& p, uint32_t tbase, int64_t row, int nt) {
+__device__ __forceinline__ void tc_epilogue_tile(const TcParams& p, uint32_t tbase, int64_t row, int nt, int half) {
   const GemmArgs& a = p.a;
   const bool in_range = row < a.M;
   const int col0 = nt * p.bn;
   bf16* out = (bf16*)a.out;
   uint32_t r[32], r2[32];
+  int u_lo, u_hi;
   if (EPI == kEpiSwiglu) {
-    for (int cc = 0; cc < p.bn; cc += 32) {
+    half_range(p.bn / 32, half, u_lo, u_hi);
+    for (int cc = u_lo * 32; cc < u_hi * 32; cc += 32) {
       tmem_ld32(tbase + cc, r);
       tmem_ld32(tbase + p.bn + cc, r2);
       tmem_wait_ld();
@@ -223,17 +243,18 @@ __device__ __forceinline__ void tc_epilogue_tile(const TcParams& p, uint32_t tba
   }
   if (EPI == kEpiRope && col0 < a.rope_cols) {
     // heads of 64 columns: rotate (i, i+32) pairs
-    const int half = a.head_dim / 2;  // 32
+    const int hd2 = a.head_dim / 2;  // 32
     const int64_t pos = in_range ? rope_position(a, row) : 0;
-    for (int hc = 0; hc < p.bn; hc += 2 * half) {
+    half_range(p.bn / (2 * hd2), half, u_lo, u_hi);
+    for (int hc = u_lo * 2 * hd2; hc < u_hi * 2 * hd2; hc += 2 * hd2) {
       tmem_ld32(tbase + hc, r);
-      tmem_ld32(tbase + hc + half, r2);
+      tmem_ld32(tbase + hc + hd2, r2);
       tmem_wait_ld();
       if (in_range) {
         float lo[32], hi[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float2 cs = rope_cs(a.rope_tab, half, pos, i);
+          const float2 cs = rope_cs(a.rope_tab, hd2, pos, i);
           const float x1 = __uint_as_float(r[i]), x2 = __uint_as_float(r2[i]);
           lo[i] = x1 * cs.x - x2 * cs.y;
           hi[i] = x2 * cs.x + x1 * cs.y;
@@ -242,13 +263,14 @@ __device__ __forceinline__ void tc_epilogue_tile(const TcParams& p, uint32_t tba
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           store8(o + 8 * i, lo + 8 * i);
-          store8(o + half + 8 * i, hi + 8 * i);
+          store8(o + hd2 + 8 * i, hi + 8 * i);
         }
       }
     }
     return;
   }
-  for (int cc = 0; cc < p.bn; cc += 32) {
+  half_range(p.bn / 32, half, u_lo, u_hi);
+  for (int cc = u_lo * 32; cc < u_hi * 32; cc += 32) {
     tmem_ld32(tbase + cc, r);
     tmem_wait_ld();
     if (!in_range) continue;
@@ -271,8 +293,15 @@ __device__ __forceinline__ void tc_epilogue_tile(const TcParams& p, uint32_t tba
         for (int j = 0; j < 8; ++j) f[8 * i + j] += g[j];
       }
     } else if (EPI == kEpiSoftplus) {
+      const float4* bp = reinterpret_cast<const float4*>(a.bias + col);  // 16-byte aligned (checked at launch)
 #pragma unroll
-      for (int i = 0; i < 32; ++i) f[i] = softplus_fast(f[i] + a.bias[col + i]);
+      for (int i = 0; i < 8; ++i) {
+        const float4 b4 = bp[i];
+        f[4 * i + 0] = softplus_fast(f[4 * i + 0] + b4.x);
+        f[4 * i + 1] = softplus_fast(f[4 * i + 1] + b4.y);
+        f[4 * i + 2] = softplus_fast(f[4 * i + 2] + b4.z);
+        f[4 * i + 3] = softplus_fast(f[4 * i + 3] + b4.w);
+      }
     }
     bf16* o = out + row * a.ldo + col;
 #pragma unroll
@@ -295,7 +324,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_con
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.tfull[i], 1);
-      mbar_init(&S.tempty[i], 4);
+      mbar_init(&S.tempty[i], TC_EPI_WARPS);
     }
     fence_mbar_init();
     tma_prefetch_desc(&p.tmA);
@@ -369,8 +398,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_con
       }
     }
   } else {
-    // ---------------- epilogue warps 2..5 -> TMEM lane quadrant warp % 4
+    // ---------------- epilogue warps 2..9 -> TMEM lane quadrant warp % 4, column half (warp - 2) / 4
     const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
     int tc = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tc) {
       int mt, nt;
@@ -383,7 +413,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_con
       tc_fence_after();
       const uint32_t tbase = tmem + acc * TC_MAXN + ((uint32_t)(q * 32) << 16);
       const int64_t row = (int64_t)mt * TC_BM + q * 32 + lane;
-      tc_epilogue_tile<EPI>(p, tbase, row, nt);
+      tc_epilogue_tile<EPI>(p, tbase, row, nt, half);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.tempty[acc]);
@@ -439,6 +469,7 @@ bool gemm_tc_supported(const GemmArgs& a) {
   if (!tc_bn_for(a, bn)) return false;
   if (a.epi == kEpiRope && (a.head_dim != 64 || a.rope_cols % 64 != 0)) return false;
   if (a.epi == kEpiResid && (a.ldr % 8 || (a.tap && a.ldt % 8))) return false;
+  if (a.epi == kEpiSoftplus && !aligned16(a.bias)) return false;
   for (int s = 0; s < a.nseg; ++s)
     if (!aligned16(a.seg[s].W) || (a.seg[s].W2 && !aligned16(a.seg[s].W2))) return false;
   return true;
@@ -453,6 +484,13 @@ samba_status launch_gemm_tc(const GemmArgs& a, cudaStream_t st) {
   p.umma_n = a.epi == kEpiSwiglu ? 2 * p.bn : p.bn;
   p.n_tiles = a.N / p.bn;
   p.m_tiles = (int)((a.M + TC_BM - 1) / TC_BM);
+  {
+    // largest divisor of n_tiles whose weight panel stays within 32 MB of L2
+    const size_t panel = (size_t)p.umma_n * a.K * 2;  // bytes of B per n-tile
+    p.group_n = 1;
+    for (int g = 1; g <= p.n_tiles; ++g)
+      if (p.n_tiles % g == 0 && (size_t)g * panel <= (size_t(32) << 20)) p.group_n = g;
+  }
   p.k_blocks = a.K / TC_BK;
   {
     uint64_t dims[2] = {(uint64_t)a.K, (uint64_t)a.M};

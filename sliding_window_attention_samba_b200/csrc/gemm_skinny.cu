@@ -140,7 +140,20 @@ __global__ void __launch_bounds__(SK_THREADS, 1) gemm_skinny_kernel(const __grid
       while (seg < a.nseg - 1 && n0 >= p.seg_start[seg + 1]) ++seg;
       const int wrow = n0 - p.seg_start[seg];
       const uint32_t bytes = (uint32_t)(SK_BM * SK_BK * 2) * (kDual ? 2 : 1) + (uint32_t)p.MB * SK_BK * 2;
-      for (int i = 0; i < nkb; ++i) {
+      // The weights are never written by a kernel: the first ring stages are
+      // fetched before waiting for the previous kernel (programmatic dependent
+      // launch), the activations only after it.
+      const int npre = min(nkb, p.stages);
+      for (int i = 0; i < npre; ++i) {
+        mbar_arrive_expect_tx(&S.full[i], bytes);
+        const int kx = (kb_begin + i) * SK_BK;
+        tma_load_2d(stW(i), &p.tmW[seg], &S.full[i], kx, wrow);
+        if (kDual) tma_load_2d(stW2(i), &p.tmW2, &S.full[i], kx, wrow);
+      }
+      pdl_wait();
+      pdl_trigger();
+      for (int i = 0; i < npre; ++i) tma_load_2d(stX(i), &p.tmX, &S.full[i], (kb_begin + i) * SK_BK, 0);
+      for (int i = npre; i < nkb; ++i) {
         const int s = i % p.stages;
         if (!mbar_wait(&S.empty[s], ((i / p.stages) & 1) ^ 1, err)) break;
         mbar_arrive_expect_tx(&S.full[s], bytes);
@@ -150,7 +163,11 @@ __global__ void __launch_bounds__(SK_THREADS, 1) gemm_skinny_kernel(const __grid
         tma_load_2d(stX(s), &p.tmX, &S.full[s], kx, 0);
       }
     }
-  } else if (warp == 1) {
+  } else {
+    pdl_wait();  // the epilogue reads and writes activations
+    pdl_trigger();
+  }
+  if (warp == 1) {
     const uint32_t idesc = idesc_bf16_f32(SK_BM, p.MB);
     if (elect_one()) {
       bool ok = true;
@@ -316,13 +333,15 @@ static samba_status skinny_launch(const SkParams& p, int ntiles, cudaStream_t st
   cfg.blockDim = dim3(SK_THREADS, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = p.S;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = p.a.pdl ? 2 : 1;
   if (cudaLaunchKernelEx(&cfg, kern, p, device_error_word()) != cudaSuccess) return SAMBA_ERR_CUDA;
   SAMBA_CHECK_LAUNCH();
   return SAMBA_OK;

@@ -35,14 +35,14 @@ samba_status launch_selective_scan(const ScanArgs& a, cudaStream_t st);
 constexpr int kRopeLevels = 3;
 constexpr int kRopeRadix = 1024;
 size_t rope_table_bytes(int head_dim);
-samba_status launch_build_rope_table(float2* tab, int head_dim, float base, cudaStream_t st);
+samba_status launch_build_rope_table(float2* tab, int head_dim, float base, cudaStream_t st, bool pdl = false);
 // out[b,t,h,:] = RoPE(x[b,t,h,:], pos0 + t); x may alias out.
 samba_status launch_rope_apply(const void* x, void* out, int B, int L, int H, int head_dim, int64_t pos0,
                                const float2* tab, samba_dtype dt, cudaStream_t st);
 
 // ---------------- RMSNorm ----------------
 samba_status launch_rmsnorm(const void* x, int64_t ld_x, const float* g, void* out, int64_t ld_out, int64_t rows,
-                            int dim, float eps, samba_dtype dt, cudaStream_t st);
+                            int dim, float eps, samba_dtype dt, cudaStream_t st, bool pdl = false);
 
 // ---------------- causal conv ----------------
 struct ConvArgs {
@@ -90,6 +90,7 @@ struct GemmArgs {
   const int64_t* pos_dev = nullptr;
   const float2* rope_tab = nullptr;
   samba_dtype dtype = SAMBA_BF16;
+  bool pdl = false;  // launch as a programmatic dependent of the previous kernel (decode path)
 };
 samba_status launch_gemm(const GemmArgs& a, cudaStream_t st);       // picks the kernel
 samba_status launch_gemm_simt(const GemmArgs& a, cudaStream_t st);  // CUDA-core fp32 FMA kernel

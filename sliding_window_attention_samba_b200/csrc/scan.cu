@@ -105,11 +105,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int s = c % kStages;
     const bool ok = mbar_wait(&S.full[s], (c / kStages) & 1, err);
     if (ok) {
-      float* dst = &S.BC[c & 1][0][0];
-      for (int e = tid; e < kChunk * 2 * kN; e += kThreads) {
-        const int row = e / (2 * kN), col = e % (2 * kN);
-        dst[e] = col < kN ? Elt<T>::to_f(S.Bm[s][row * kN + col]) : Elt<T>::to_f(S.Cm[s][row * kN + col - kN]);
-      }
+      // 64 rows x (16 B | 16 C) = 256 runs of 8 values: one per thread
+      static_assert(kChunk * 4 == kThreads, "one 8-value run of B or C per thread");
+      const int row = tid >> 2, part = tid & 3;
+      const T* src = (part < 2 ? S.Bm[s] : S.Cm[s]) + row * kN + (part & 1) * 8;
+      float f[8];
+      load8(src, f);
+      float4* dst = reinterpret_cast<float4*>(&S.BC[c & 1][row][part * 8]);
+      dst[0] = make_float4(f[0], f[1], f[2], f[3]);
+      dst[1] = make_float4(f[4], f[5], f[6], f[7]);
     }
     return ok;
   };
@@ -189,15 +193,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
 
     // ---- combine across the 8 warps, chained from the previous chunk's carry
+    // (all aggregates are loaded before the first entry state is stored: the
+    // dependent chain is then 8 FMAs, not 8 shared-memory round trips)
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
+      float P[kWarps], hl[kWarps];
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        P[w] = S.aggP[w][cn + j][cl];
+        hl[w] = S.aggH[w][cn + j][cl];
+      }
       float H = carry[j];
 #pragma unroll
       for (int w = 0; w < kWarps; ++w) {
-        const float P = S.aggP[w][cn + j][cl];
-        const float hl = S.aggH[w][cn + j][cl];
         S.aggH[w][cn + j][cl] = H;
-        H = fmaf(P, H, hl);
+        H = fmaf(P[w], H, hl[w]);
       }
       carry[j] = H;
     }
@@ -214,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float4* Bp = reinterpret_cast<const float4*>(BC + row * 2 * kN);
       const float4* Cp = Bp + kN / 4;
       const float2 dd = f2(du[i]);
-      float2 y2 = make_float2(0.f, 0.f);
+      float2 y2[4];  // four partial sums: the readout is not one serial chain of 8 FMAs
 #pragma unroll
       for (int q = 0; q < kN / 4; ++q) {
         const float4 Bq = Bp[q];
@@ -224,10 +234,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int n = 2 * q + hh;
           const float2 bu = __fmul2_rn(dd, hh ? make_float2(Bq.z, Bq.w) : make_float2(Bq.x, Bq.y));
           h[n] = __ffma2_rn(dA[i][n], h[n], bu);
-          y2 = __ffma2_rn(hh ? make_float2(Cq.z, Cq.w) : make_float2(Cq.x, Cq.y), h[n], y2);
+          const float2 cq = hh ? make_float2(Cq.z, Cq.w) : make_float2(Cq.x, Cq.y);
+          y2[q] = hh ? __ffma2_rn(cq, h[n], y2[q]) : __fmul2_rn(cq, h[n]);
         }
       }
-      float y = y2.x + y2.y;
+      const float2 ya = __fadd2_rn(__fadd2_rn(y2[0], y2[1]), __fadd2_rn(y2[2], y2[3]));
+      float y = ya.x + ya.y;
       const float uv = Elt<T>::to_f(S.u[s][row * kCh + lane]);
       y = fmaf(Dd, uv, y);
       if (kHasZ) {

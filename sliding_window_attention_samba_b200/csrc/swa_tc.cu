@@ -57,6 +57,36 @@ struct AtParams {
   float scale_log2;
 };
 
+// three-input maximum (one instruction on sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x for a pair of x <= 0 on the FMA pipe, to take part of the exponentials off
+// the MUFU unit.  Range reduction: x is clamped to >= -126 (so the exponent
+// field below cannot wrap) and n = round(x) is
+// taken with the 1.5*2^23 shift (the sum's low mantissa bits hold n, the
+// difference is exact); f = x - n lies in [-1/2, 1/2]; 2^f is a degree-3
+// polynomial fitted here by relative-error-weighted least squares on Chebyshev
+// nodes of [-1/2, 1/2] (max relative error 7.5e-5, far below the bf16 rounding
+// of P); 2^n is added to the exponent field, i.e. bits(p) + bits(shifted sum)
+// * 2^23 modulo 2^32 (the shift constant's bits vanish under that product).
+// Results for x <= -126 (masked keys: x = -inf) are exact zeros.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  x = make_float2(fmaxf(x.x, -126.f), fmaxf(x.y, -126.f));
+  const float2 r = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
+  const float2 n = __fadd2_rn(r, make_float2(-12582912.f, -12582912.f));
+  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+  float2 q = __ffma2_rn(make_float2(0.05517137f, 0.05517137f), f, make_float2(0.24261110f, 0.24261110f));
+  q = __ffma2_rn(q, f, make_float2(0.69326103f, 0.69326103f));
+  q = __ffma2_rn(q, f, make_float2(0.99992806f, 0.99992806f));
+  const float2 y = make_float2(__uint_as_float(__float_as_uint(q.x) + __float_as_uint(r.x) * 8388608u),
+                               __uint_as_float(__float_as_uint(q.y) + __float_as_uint(r.y) * 8388608u));
+  return make_float2(x.x > -126.f ? y.x : 0.f, x.y > -126.f ? y.y : 0.f);  // masked keys give exact zeros
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -201,14 +231,12 @@ __global__ void __launch_bounds__(AT_THREADS, 1) swa_tc_kernel(const __grid_cons
         const int hi = tq < p.L ? t - kb : -1;
         const int lo = t - p.window - kb;
 #pragma unroll
-        for (int i = 0; i < 128; ++i) {
+        for (int i = 0; i < 128; ++i)
           if (i > hi || i <= lo) sr[i] = __float_as_uint(-INFINITY);
-          m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(sr[i]));
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 128; ++i) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(sr[i]));
       }
+#pragma unroll
+      for (int i = 0; i < 128; i += 2)
+        m8[(i >> 1) & 7] = fmax3(m8[(i >> 1) & 7], __uint_as_float(sr[i]), __uint_as_float(sr[i + 1]));
       const float mraw = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
                                fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       const float mt = mraw * p.scale_log2;  // -inf stays -inf
@@ -239,7 +267,8 @@ __global__ void __launch_bounds__(AT_THREADS, 1) swa_tc_kernel(const __grid_cons
       const float msub = m_run == -INFINITY ? 0.f : m_run;
       // P buffer j%2 was last read by PV_{j-2}
       if (j >= 2 && !wait_all(&S.pv_done[j & 1], ((j - 2) >> 1) & 1)) { ok = false; break; }
-      float ls8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // independent partial sums
+      const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nm2 = make_float2(-msub, -msub);
+      float2 ls2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         unsigned char* prow = reinterpret_cast<unsigned char*>(S.P[j & 1][half]) + r * 128;
@@ -247,16 +276,19 @@ __global__ void __launch_bounds__(AT_THREADS, 1) swa_tc_kernel(const __grid_cons
         for (int c = 0; c < 8; ++c) {
           float e[8];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            e[q] = ex2_approx(fmaf(__uint_as_float(sr[half * 64 + c * 8 + q]), p.scale_log2, -msub));
-            ls8[q] += e[q];
+          for (int q = 0; q < 4; ++q) {
+            const int i = half * 64 + c * 8 + 2 * q;
+            const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), sc2, nm2);
+            e[2 * q] = ex2_approx(x.x);
+            e[2 * q + 1] = ex2_approx(x.y);
+            ls2[q] = __fadd2_rn(ls2[q], make_float2(e[2 * q], e[2 * q + 1]));
           }
           uint4 v4 = make_uint4(pack_bf16(e[0], e[1]), pack_bf16(e[2], e[3]), pack_bf16(e[4], e[5]),
                                 pack_bf16(e[6], e[7]));
           *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = v4;
         }
       }
-      l_run += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
+      l_run += ((ls2[0].x + ls2[0].y) + (ls2[1].x + ls2[1].y)) + ((ls2[2].x + ls2[2].y) + (ls2[3].x + ls2[3].y));
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
@@ -312,6 +344,9 @@ struct At2Smem {
   uint32_t tmem_base;
 };
 
+// kPolyPairs: pairs (of the four per 8-key group) whose exponentials run on the
+// FMA pipe (exp2_poly2) instead of the MUFU unit.
+template <int kPolyPairs>
 __global__ void __launch_bounds__(A2_THREADS, 1) swa_tc2_kernel(const __grid_constant__ AtParams p, int* err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   At2Smem& S = *reinterpret_cast<At2Smem*>(smem_raw + smem_align_pad(smem_raw, 1024));
@@ -402,13 +437,15 @@ __global__ void __launch_bounds__(A2_THREADS, 1) swa_tc2_kernel(const __grid_con
         umma_commit(&S.pv_done[wg]);
         return true;
       };
+      // S_{j+1} of a head is issued as soon as its softmax has read S_j (before
+      // it has finished P_j), then PV_j once P_j is in shared memory.
       if (ok) ok = issue_s(0, 0);
       if (ok) ok = issue_s(1, 0);
       for (int j = 0; ok && j < ntile; ++j) {
-        ok = issue_pv(0, j);
-        if (ok && j + 1 < ntile) ok = issue_s(0, j + 1);
-        if (ok) ok = issue_pv(1, j);
+        if (j + 1 < ntile) ok = issue_s(0, j + 1);
+        if (ok) ok = issue_pv(0, j);
         if (ok && j + 1 < ntile) ok = issue_s(1, j + 1);
+        if (ok) ok = issue_pv(1, j);
       }
     }
   } else {
@@ -433,26 +470,30 @@ __global__ void __launch_bounds__(A2_THREADS, 1) swa_tc2_kernel(const __grid_con
       const bool edge = (kb + AT_BN - 1 > tk0) || (kb < tk0 + AT_BM - p.window);
       const int hi = tq < p.L ? t - kb : -1;  // valid key offsets of row t: (lo_i, hi]
       const int lo_i = t - p.window - kb;
-      // pass 1: row max of the raw scores
+      // pass 1: row max of the raw scores, two 32-column loads per TMEM round trip
       float m8[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t sr[32];
-        tmem_ld32(tS + c * 32, sr);
-        tmem_wait_ld();
+      auto max_chunk = [&](uint32_t (&sr)[32], int c) {
         if (edge) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const int kk = c * 32 + i;
-            const float x = (kk > hi || kk <= lo_i) ? -INFINITY : __uint_as_float(sr[i]);
-            m8[i & 7] = fmaxf(m8[i & 7], x);
+            if (kk > hi || kk <= lo_i) sr[i] = __float_as_uint(-INFINITY);
           }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(sr[i]));
         }
+#pragma unroll
+        for (int i = 0; i < 32; i += 2)
+          m8[(i >> 1) & 7] = fmax3(m8[(i >> 1) & 7], __uint_as_float(sr[i]), __uint_as_float(sr[i + 1]));
+      };
+#pragma unroll
+      for (int c = 0; c < 4; c += 2) {
+        uint32_t sa[32], sb[32];
+        tmem_ld32(tS + c * 32, sa);
+        tmem_ld32(tS + (c + 1) * 32, sb);
+        tmem_wait_ld();
+        max_chunk(sa, c);
+        max_chunk(sb, c + 1);
       }
       const float mraw = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
                                fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
@@ -480,40 +521,63 @@ __global__ void __launch_bounds__(A2_THREADS, 1) swa_tc2_kernel(const __grid_con
         tmem_wait_st();
       }
       const float msub = m_run == -INFINITY ? 0.f : m_run;
-      // pass 2: P = exp2(s * scale - m) as bf16 into the swizzled P tile
-      float ls8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      // pass 2: P = exp2(s * scale - m) as bf16 into the swizzled P tile.  The band
+      // mask is applied in a separate (tile-uniform) branch so that the 15 of 17
+      // interior tiles of a band pay nothing for it; scale-subtract and row sums
+      // run as packed fp32x2 operations.
+      const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nm2 = make_float2(-msub, -msub);
+      float2 ls2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      // software pipeline: the load of chunk c+1 is in flight while chunk c is exponentiated
+      uint32_t sbuf[2][32];
+      tmem_ld32(tS, sbuf[0]);
+      tmem_wait_ld();
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t sr[32];
-        tmem_ld32(tS + c * 32, sr);
-        tmem_wait_ld();
+        if (c + 1 < 4) tmem_ld32(tS + (c + 1) * 32, sbuf[(c + 1) & 1]);
+        uint32_t (&sr)[32] = sbuf[c & 1];
+        if (edge) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int kk = c * 32 + i;
+            if (kk > hi || kk <= lo_i) sr[i] = __float_as_uint(-INFINITY);
+          }
+        }
         unsigned char* prow = reinterpret_cast<unsigned char*>(S.P[wg][c >> 1]) + r * 128;
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           const int chunk = (c & 1) * 4 + cc;  // 16-byte chunk (8 keys) within the 64-key half
           float e[8];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const int i = cc * 8 + q;
-            const int kk = c * 32 + i;
-            float x = fmaf(__uint_as_float(sr[i]), p.scale_log2, -msub);
-            if (edge && (kk > hi || kk <= lo_i)) x = -INFINITY;
-            e[q] = ex2_approx(x);
-            ls8[q] += e[q];
+          for (int q = 0; q < 4; ++q) {
+            const int i = cc * 8 + 2 * q;
+            const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), sc2, nm2);
+            if (q < kPolyPairs) {
+              const float2 y = exp2_poly2(x);
+              e[2 * q] = y.x;
+              e[2 * q + 1] = y.y;
+            } else {
+              e[2 * q] = ex2_approx(x.x);
+              e[2 * q + 1] = ex2_approx(x.y);
+            }
+            ls2[q] = __fadd2_rn(ls2[q], make_float2(e[2 * q], e[2 * q + 1]));
           }
           uint4 v4 = make_uint4(pack_bf16(e[0], e[1]), pack_bf16(e[2], e[3]), pack_bf16(e[4], e[5]),
                                 pack_bf16(e[6], e[7]));
           *reinterpret_cast<uint4*>(prow + ((chunk ^ (r & 7)) << 4)) = v4;
         }
+        if (c + 1 < 4) {
+          tmem_wait_ld();
+          if (c + 1 == 3) {  // every score of this tile is in registers: S may be overwritten
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.s_free[wg]);
+          }
+        }
       }
-      l_run += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
-      tc_fence_before();
+      l_run += ((ls2[0].x + ls2[0].y) + (ls2[1].x + ls2[1].y)) + ((ls2[2].x + ls2[2].y) + (ls2[3].x + ls2[3].y));
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&S.s_free[wg]);
-        mbar_arrive(&S.p_full[wg]);
-      }
+      if (lane == 0) mbar_arrive(&S.p_full[wg]);
     }
     if (ok && wait_all(&S.pv_done[wg], (ntile - 1) & 1)) {
       tc_fence_after();
@@ -577,10 +641,15 @@ samba_status launch_swa_tc(const SwaArgs& a, cudaStream_t st) {
   p.scale_log2 = a.scale * 1.4426950408889634f;
   const int grp = a.Hq / a.Hkv;
   if (grp % 2 == 0 && !(getenv("SAMBA_SWA_KERNEL") && getenv("SAMBA_SWA_KERNEL")[0] == '1')) {
+    // share of the exponentials on the FMA pipe: SAMBA_SWA_POLY = 0..3 pairs of 4 (default 1)
+    const char* pe = getenv("SAMBA_SWA_POLY");
+    const int poly = (pe && pe[0] >= '0' && pe[0] <= '3') ? pe[0] - '0' : 1;
+    auto kern = poly == 0 ? swa_tc2_kernel<0> : poly == 2 ? swa_tc2_kernel<2> : poly == 3 ? swa_tc2_kernel<3>
+                                                                                            : swa_tc2_kernel<1>;
     const size_t smem = sizeof(At2Smem) + 1024;
-    if (!ensure_smem_attr(swa_tc2_kernel, smem)) return SAMBA_ERR_CUDA;
+    if (!ensure_smem_attr(kern, smem)) return SAMBA_ERR_CUDA;
     dim3 grid((a.L + AT_BM - 1) / AT_BM, a.Hq / 2, a.B);
-    swa_tc2_kernel<<<grid, A2_THREADS, smem, st>>>(p, device_error_word());
+    kern<<<grid, A2_THREADS, smem, st>>>(p, device_error_word());
     SAMBA_CHECK_LAUNCH();
     return SAMBA_OK;
   }
