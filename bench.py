@@ -48,11 +48,16 @@ def parse():
     ap.add_argument("--impl", default="samba", choices=["samba", "reference"])
     ap.add_argument("--seq-len", type=int, default=None, help="override L (parity/debug runs only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="prefill", choices=["prefill", "block", "decode", "sweep", "chunked"],
+    ap.add_argument("--workload", default="prefill",
+                    choices=["prefill", "block", "decode", "sweep", "chunked", "model", "model_decode"],
                     help="prefill: 4-block L=131072 stack (the headline); block: one block at B=4, L=4096; "
                          "decode: B=32 samba_step stream; "
                          "sweep: scan and SWA alone at L = 4K..1M; "
-                         "chunked: one block over L=1M in 32K-token chunks (samba_block_fwd_chunk)")
+                         "chunked: one block over L=1M in 32K-token chunks (samba_block_fwd_chunk); "
+                         "model: prompt processing of a Samba-1.7B-layout stack vs a GQA Transformer of the "
+                         "same width (samba_model_prefill), 128K tokens per step at L = 4K..128K; "
+                         "model_decode: decode tokens/s of the same two stacks at batch 16 over 64K generated "
+                         "tokens (samba_model_step, CUDA graph replay)")
     ap.add_argument("--max-len", type=int, default=1048576, help="sweep: largest L")
     return ap.parse_args()
 
@@ -615,6 +620,198 @@ def run_chunked(args):
     print(json.dumps(line))
 
 
+def make_layers(torch, s, layout, seed, dev):
+    """Random-init weights of a layout of sub-layers (N(0, 0.02) matrices, S4D-Real
+    A, D = 1, Delta bias in [1e-3, 1e-1], unit norm gains); each dict holds only
+    what its kind reads."""
+    g = torch.Generator(device=dev)
+    bf = torch.bfloat16
+    out = []
+    for li, kind in enumerate(layout):
+        g.manual_seed(I.tensor_key(seed, f"model.L{li}") & ((1 << 63) - 1))
+
+        def mat(o, i):
+            return (torch.randn(o, i, generator=g, device=dev) * 0.02).to(bf)
+
+        if kind == "mamba":
+            w = {"norm0": torch.ones(s.d_model, device=dev), "W_in": mat(2 * s.d_inner, s.d_model),
+                 "conv_w": torch.randn(s.d_inner, s.d_conv, generator=g, device=dev) * 0.02,
+                 "W_x": mat(s.dt_rank + 2 * s.d_state, s.d_inner), "W_dt": mat(s.d_inner, s.dt_rank),
+                 "dt_bias": torch.from_numpy(I.dt_bias_init(seed, f"model.L{li}.dt_bias", s.d_inner)).to(dev),
+                 "A_log": torch.from_numpy(I.a_log_init(s.d_inner, s.d_state)).to(dev),
+                 "D": torch.ones(s.d_inner, device=dev), "W_out": mat(s.d_model, s.d_inner)}
+        elif kind == "swa":
+            w = {"norm2": torch.ones(s.d_model, device=dev), "Wq": mat(s.n_q * s.head_dim, s.d_model),
+                 "Wk": mat(s.n_kv * s.head_dim, s.d_model), "Wv": mat(s.n_kv * s.head_dim, s.d_model),
+                 "Wo": mat(s.d_model, s.n_q * s.head_dim)}
+        else:
+            w = {"norm1": torch.ones(s.d_model, device=dev), "mlp1_W1": mat(s.d_ff, s.d_model),
+                 "mlp1_W2": mat(s.d_ff, s.d_model), "mlp1_W3": mat(s.d_model, s.d_ff)}
+        out.append(w)
+    return out
+
+
+def run_model(args):
+    """Prompt processing of two stacks of the same width built from this
+    library's kernels: the paper's Samba-1.7B layout (8 x [Mamba, MLP, Mamba,
+    MLP, SWA, MLP]: 16 Mamba, 8 SWA, 24 MLP) and a GQA Transformer of the
+    Llama-3-1.6B shape (24 x [attention over the whole prefix, MLP]), both with a
+    32000-token vocabulary.  As in the pages' throughput protocol, every step
+    processes 131072 prompt tokens: batch = 131072 / L for L = 4K .. 128K."""
+    import dataclasses
+    import torch
+    from sliding_window_attention_samba_b200 import _lib as L
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    s = I.WIDE
+    vocab, total = 32000, 131072
+    kind = {"mamba": L.LAYER_MAMBA, "mlp": L.LAYER_MLP, "swa": L.LAYER_SWA}
+    samba_layout = ["mamba", "mlp", "mamba", "mlp", "swa", "mlp"] * 8
+    tfm_layout = ["swa", "mlp"] * 24
+    bf = torch.bfloat16
+    g = torch.Generator(device=dev)
+    g.manual_seed(7)
+    common = {"emb": torch.randn(vocab, s.d_model, generator=g, device=dev).to(bf),
+              "head": (torch.randn(vocab, s.d_model, generator=g, device=dev) * 0.02).to(bf),
+              "gfin": torch.ones(s.d_model, device=dev)}
+    stacks = {"samba": (samba_layout, make_layers(torch, s, samba_layout, 6, dev)),
+              "transformer": (tfm_layout, make_layers(torch, s, tfm_layout, 7, dev))}
+    n_params = {k: sum(t.numel() for w in ws for t in w.values()) + 2 * vocab * s.d_model
+                for k, (_, ws) in stacks.items()}
+    lens = [Ln for Ln in (4096, 16384, 65536, 131072) if Ln <= (args.seq_len or 131072)]
+    ws_bytes = max(L.samba_model_workspace_size(
+        L.make_model(L.make_config(s), [], [], common["emb"], common["gfin"], common["head"], vocab),
+        total // Ln, Ln) for Ln in lens)
+    wsp = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    results = []
+    clocks = ClockSampler(0)
+    clocks.start()
+    for Ln in lens:
+        Bn = total // Ln
+        ids = torch.randint(0, vocab, (Bn, Ln), generator=g, device=dev, dtype=torch.int32)
+        logits = torch.empty(Bn, vocab, device=dev, dtype=bf)
+        row = {"seq_len": Ln, "batch": Bn}
+        for name, (layout, ws_) in stacks.items():
+            shape = s if name == "samba" else dataclasses.replace(s, window=Ln)  # full causal attention
+            m = L.make_model(L.make_config(shape), [kind[k] for k in layout], ws_, common["emb"], common["gfin"],
+                             common["head"], vocab)
+
+            def run(m=m):
+                L.samba_model_prefill(m, ids, logits, Bn, Ln, wsp, ws_bytes)
+
+            t = _time(torch, run, 1, max(1, args.steps))
+            row[name + "_tokens_per_s"] = Bn * Ln / t
+            row[name + "_ms_per_step"] = t * 1e3
+        row["ratio"] = row["samba_tokens_per_s"] / row["transformer_tokens_per_s"]
+        results.append(row)
+        print(json.dumps(dict(workload="prompt_processing", **row)))
+    clk = clocks.stop()
+    assert L.samba_get_error() == 0
+    last = results[-1]
+    print(json.dumps({"metric": f"prompt tokens/s, Samba-1.7B layout, L={last['seq_len']}",
+                      "value": last["samba_tokens_per_s"], "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+                      "warmup": 1, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                      "dtype": "bf16", "data": "synthetic",
+                      "config": {"workload": "prompt_processing_128K_tokens", "d_model": s.d_model,
+                                 "vocab": vocab, "samba_layers": "8 x [Mamba, MLP, Mamba, MLP, SWA, MLP]",
+                                 "transformer_layers": "24 x [GQA attention (full causal), MLP]",
+                                 "params": n_params, "tokens_per_step": total},
+                      "transformer_value": last["transformer_tokens_per_s"], "ratio": last["ratio"],
+                      "by_length": results, "clocks": clk}))
+
+
+def run_model_decode(args):
+    """Decode throughput of the two stacks of run_model at batch 16 (the pages'
+    generation protocol: 64K generated tokens).  Samba's step cost does not
+    depend on the context; the Transformer's attention reads its whole KV cache.
+    One step is captured in a CUDA graph and replayed at contexts P = 0, 2K, 8K,
+    16K, 32K, 64K (the cache holds P valid entries; its values do not change the
+    work), and the time to generate 64K tokens is the trapezoid over P."""
+    import dataclasses
+    import torch
+    from sliding_window_attention_samba_b200 import _lib as L
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    s = I.WIDE
+    vocab, Bn, gen = 32000, 16, 65536
+    bf = torch.bfloat16
+    kind = {"mamba": L.LAYER_MAMBA, "mlp": L.LAYER_MLP, "swa": L.LAYER_SWA}
+    g = torch.Generator(device=dev)
+    g.manual_seed(8)
+    common = {"emb": torch.randn(vocab, s.d_model, generator=g, device=dev).to(bf),
+              "head": (torch.randn(vocab, s.d_model, generator=g, device=dev) * 0.02).to(bf),
+              "gfin": torch.ones(s.d_model, device=dev)}
+    cache = gen + 256
+    setups = {"samba": (["mamba", "mlp", "mamba", "mlp", "swa", "mlp"] * 8, s),
+              "transformer": (["swa", "mlp"] * 24, dataclasses.replace(s, window=cache))}
+    points = [0, 2048, 8192, 16384, 32768, gen - 1]
+    reps = max(10, args.steps)
+    out = {}
+    clocks = ClockSampler(0)
+    clocks.start()
+    for name, (layout, shape) in setups.items():
+        ws_layers = make_layers(torch, shape, layout, 9 if name == "samba" else 10, dev)
+        m = L.make_model(L.make_config(shape), [kind[k] for k in layout], ws_layers, common["emb"], common["gfin"],
+                         common["head"], vocab)
+        states = []
+        for k in layout:
+            d = {}
+            if k == "mamba":
+                d["ssm"] = torch.zeros(Bn, s.d_inner, s.d_state, device=dev)
+                d["conv"] = torch.zeros(Bn, s.d_inner, s.d_conv - 1, device=dev, dtype=bf)
+            elif k == "swa":
+                d["k_ring"] = torch.randn(Bn, shape.window, s.n_kv, s.head_dim, generator=g, device=dev).to(bf)
+                d["v_ring"] = torch.randn_like(d["k_ring"].float()).to(bf)
+            states.append(d)
+        st_arr = L.make_layer_states(states)
+        pos = torch.zeros(Bn, dtype=torch.int64, device=dev)
+        ids_t = torch.randint(0, vocab, (Bn,), generator=g, device=dev, dtype=torch.int32)
+        logits = torch.empty(Bn, vocab, device=dev, dtype=bf)
+        n = L.samba_model_step_workspace_size(m, Bn)
+        wsp = torch.empty(n, dtype=torch.uint8, device=dev)
+        stream = torch.cuda.Stream()
+        stream.wait_stream(torch.cuda.current_stream())
+        per = {}
+        with torch.cuda.stream(stream):
+            L.samba_model_step(m, ids_t, logits, st_arr, pos, Bn, wsp, n, stream=stream)
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=stream):
+                L.samba_model_step(m, ids_t, logits, st_arr, pos, Bn, wsp, n, stream=stream)
+            for P in points:
+                pos.fill_(P)
+                for _ in range(3):
+                    graph.replay()
+                pos.fill_(P)
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                for _ in range(reps):
+                    graph.replay()
+                e1.record(stream)
+                stream.synchronize()
+                per[P] = e0.elapsed_time(e1) * 1e-3 / reps
+        del graph
+        assert L.samba_get_error(stream) == 0
+        t_gen = sum((points[i + 1] - points[i]) * (per[points[i]] + per[points[i + 1]]) / 2
+                    for i in range(len(points) - 1))
+        out[name] = {"step_ms_at_context": {str(P): round(per[P] * 1e3, 4) for P in points},
+                     "tokens_per_s_64K_generation": Bn * gen / t_gen,
+                     "params": sum(t.numel() for w in ws_layers for t in w.values()) + 2 * vocab * s.d_model}
+        del states, st_arr, ws_layers, wsp
+        torch.cuda.empty_cache()
+    clk = clocks.stop()
+    sv, tv = out["samba"]["tokens_per_s_64K_generation"], out["transformer"]["tokens_per_s_64K_generation"]
+    print(json.dumps({"metric": "decode tokens/s over 64K generated tokens, batch 16, Samba-1.7B layout",
+                      "value": sv, "unit": "tokens/s", "n_gpus": 1, "steps": reps, "warmup": 3,
+                      "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                      "data": "synthetic",
+                      "config": {"workload": "decode_batch16_64K", "batch": Bn, "generated": gen, "vocab": vocab,
+                                 "samba_layers": "8 x [Mamba, MLP, Mamba, MLP, SWA, MLP], 2048-slot rings",
+                                 "transformer_layers": f"24 x [GQA attention, MLP], {cache}-slot KV cache",
+                                 "graph": "one samba_model_step captured, replayed per step"},
+                      "transformer_value": tv, "ratio": sv / tv, "by_model": out, "clocks": clk}))
+
+
 def run_sweep(args):
     """Mixer-only length sweep, batch 1, d_model 2048 shapes: the selective scan
     (d_inner 4096, d_state 16; u, dt, z, B, C ~ N(0,1), Delta = softplus(dt + b))
@@ -692,6 +889,10 @@ def main():
         return run_sweep(args)
     if args.workload == "chunked":
         return run_chunked(args)
+    if args.workload == "model":
+        return run_model(args)
+    if args.workload == "model_decode":
+        return run_model_decode(args)
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))

@@ -258,6 +258,69 @@ samba_status samba_block_fwd_chunk(const samba_block_config* cfg, const samba_bl
                                    int B, int L, void* workspace, size_t workspace_bytes, samba_stream stream);
 
 /* ------------------------------------------------------------------------
+ * A language-model stack: token embedding, a sequence of pre-RMSNorm residual
+ * sub-layers, final RMSNorm, vocabulary projection [Samba §3.2 "Big-Picture
+ * Architecture": token embeddings enter the first layer, the layers repeat
+ * Mamba -> MLP -> Mamba -> MLP -> SWA -> MLP (2:1 Mamba to SWA), each preceded
+ * by RMSNorm and followed by a residual add, and the last layer's output is
+ * projected to vocabulary logits].  The same entry point runs any layout, e.g.
+ * a GQA Transformer as (SWA with window >= L, MLP) pairs.
+ * ---------------------------------------------------------------------- */
+typedef enum { SAMBA_LAYER_MAMBA = 0, SAMBA_LAYER_MLP = 1, SAMBA_LAYER_SWA = 2 } samba_layer_kind;
+
+typedef struct {
+  samba_block_config cfg;             /* shapes shared by all layers; window >= L is full causal attention */
+  int n_layers;
+  const int* kinds;                   /* host [n_layers] samba_layer_kind */
+  const samba_block_weights* layers;  /* host [n_layers]; a layer reads only the fields of its kind:
+                                         Mamba: norm_g[0], W_in, conv_w, conv_b, W_x, W_dt, dt_bias,
+                                         A_log, Dskip, W_out;  MLP: norm_g[1], mlp1_W1..W3;
+                                         SWA: norm_g[2], Wq, Wk, Wv, Wo */
+  const void* embedding;              /* device [vocab, d_model] dtype */
+  const float* final_norm;            /* device [d_model] fp32 gain */
+  const void* lm_head;                /* device [vocab, d_model] dtype */
+  int vocab;
+} samba_model;
+
+size_t samba_model_workspace_size(const samba_model* m, int B, int L);
+
+/* Prompt processing: the logits of the last position of each of B sequences.
+ * ids: device int32 [B, L], each in [0, vocab) (an id outside it latches
+ * SAMBA_ERR_DEVICE for samba_get_error and embeds as a zero row); logits:
+ * device [B, vocab] dtype.  The stack runs layer by layer over all B*L tokens
+ * (workspace: one block's activations plus two residual streams). */
+samba_status samba_model_prefill(const samba_model* m, const int32_t* ids, void* logits, int B, int L,
+                                 void* workspace, size_t workspace_bytes, samba_stream stream);
+
+/* Decode state of one sub-layer of a model: Mamba layers use ssm
+ * [B, d_inner, d_state] fp32 and conv [B, d_inner, d_conv-1]; SWA layers k_ring
+ * and v_ring [B, cfg.window, n_kv, head_dim] (post-RoPE, slot = position mod
+ * window; a window at least the longest sequence is a full KV cache); MLP
+ * layers none (their fields are ignored).  A new sequence starts from zeroed
+ * states and pos = 0. */
+typedef struct {
+  float* ssm;
+  void* conv;
+  void* k_ring;
+  void* v_ring;
+} samba_layer_state;
+
+size_t samba_model_step_workspace_size(const samba_model* m, int B);
+
+/* One decode step of the stack for one new token per sequence [the same layers
+ * at a single t; Samba §5's constant-cost decoding for Mamba, a window-sized
+ * ring for SWA]: ids_t device int32 [B]; logits device [B, vocab] dtype;
+ * states host [n_layers]; pos device int64 [B], the tokens each sequence has
+ * seen (the new token's position), incremented on return.  Feeding tokens
+ * t = 0..T-1 one by one gives, at step t, the logits samba_model_prefill gives
+ * for the prefix of t+1 tokens (up to rounding).  Rings above 2048 slots
+ * (head_dim 64, bf16) use a split attention whose partials live in the
+ * workspace.  Positions are read on the device: the call can be captured in a
+ * CUDA graph and replayed. */
+samba_status samba_model_step(const samba_model* m, const int32_t* ids_t, void* logits, samba_layer_state* states,
+                              int64_t* pos, int B, void* workspace, size_t workspace_bytes, samba_stream stream);
+
+/* ------------------------------------------------------------------------
  * The Samba block, one decode step per sequence (constant cost per token;
  * [Samba 5 / Figure 2b discussion of decoding; the blog page's ring-buffer KV])
  *

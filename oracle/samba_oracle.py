@@ -264,6 +264,30 @@ def block_fwd(x, W, cfg, want_state: bool = False):
     return r
 
 
+def model_prefill(ids, layers, embedding, final_norm, lm_head, cfg):
+    """Language-model stack [Samba §3.2 "Big-Picture Architecture": token
+    embeddings enter the first layer; each intermediate layer (Mamba, SWA or MLP)
+    is preceded by RMSNorm and followed by a residual add; the last layer's output
+    is projected to vocabulary logits].  A final RMSNorm (gain final_norm) comes
+    before the projection (the pages do not print one; the reading of a pre-norm
+    stack).  layers: list of (kind, W), kind in {"mamba", "mlp", "swa"}; an MLP
+    layer reads norm1 and mlp1_W1..W3, Mamba norm0, SWA norm2.
+    ids: int [B, L].  Returns the logits of the last position, [B, vocab]."""
+    x = _f(embedding)[np.asarray(ids)]
+    eps = cfg.norm_eps
+    for kind, W in layers:
+        if kind == "mamba":
+            f = mamba_branch(rmsnorm(x, W["norm0"], eps), W, cfg)[0]
+        elif kind == "mlp":
+            f = swiglu_mlp(rmsnorm(x, W["norm1"], eps), W["mlp1_W1"], W["mlp1_W2"], W["mlp1_W3"])
+        elif kind == "swa":
+            f = attn_branch(rmsnorm(x, W["norm2"], eps), W, cfg, 0)[0]
+        else:
+            raise ValueError(kind)
+        x = x + f
+    return linear(rmsnorm(x[:, -1], final_norm, eps), lm_head)
+
+
 def empty_state(cfg, batch: int):
     return dict(ssm=np.zeros((batch, cfg.d_inner, cfg.d_state)),
                 conv=np.zeros((batch, cfg.d_inner, cfg.d_conv - 1)),

@@ -56,6 +56,19 @@ class BlockWeights(ctypes.Structure):
                 ("mlp2_W1", c_void_p), ("mlp2_W2", c_void_p), ("mlp2_W3", c_void_p)]
 
 
+class Model(ctypes.Structure):
+    _fields_ = [("cfg", BlockConfig), ("n_layers", c_int), ("kinds", ctypes.POINTER(c_int)),
+                ("layers", ctypes.POINTER(BlockWeights)), ("embedding", c_void_p), ("final_norm", c_void_p),
+                ("lm_head", c_void_p), ("vocab", c_int)]
+
+
+LAYER_MAMBA, LAYER_MLP, LAYER_SWA = 0, 1, 2
+
+
+class LayerState(ctypes.Structure):
+    _fields_ = [("ssm", c_void_p), ("conv", c_void_p), ("k_ring", c_void_p), ("v_ring", c_void_p)]
+
+
 class DecodeState(ctypes.Structure):
     _fields_ = [("ssm", c_void_p), ("conv", c_void_p), ("k_ring", c_void_p), ("v_ring", c_void_p),
                 ("pos", c_void_p)]
@@ -102,6 +115,13 @@ _chunk = _sig("samba_block_fwd_chunk", c_int,
               [ctypes.POINTER(BlockConfig), ctypes.POINTER(BlockWeights), c_void_p, c_void_p,
                ctypes.POINTER(DecodeState), c_int64, ctypes.POINTER(BlockTaps), c_int, c_int, c_void_p, c_size_t,
                c_void_p])
+_model_ws = _sig("samba_model_workspace_size", c_size_t, [ctypes.POINTER(Model), c_int, c_int])
+_model = _sig("samba_model_prefill", c_int,
+              [ctypes.POINTER(Model), c_void_p, c_void_p, c_int, c_int, c_void_p, c_size_t, c_void_p])
+_mstep_ws = _sig("samba_model_step_workspace_size", c_size_t, [ctypes.POINTER(Model), c_int])
+_mstep = _sig("samba_model_step", c_int,
+              [ctypes.POINTER(Model), c_void_p, c_void_p, ctypes.POINTER(LayerState), c_void_p, c_int, c_void_p,
+               c_size_t, c_void_p])
 _step_ws = _sig("samba_step_workspace_size", c_size_t, [ctypes.POINTER(BlockConfig), c_int])
 _step = _sig("samba_step", c_int,
              [ctypes.POINTER(BlockConfig), ctypes.POINTER(BlockWeights), c_void_p, c_void_p,
@@ -210,6 +230,33 @@ def samba_block_fwd_chunk(cfg: BlockConfig, w: BlockWeights, x_in, x_out, st: De
                   ctypes.byref(taps) if taps else None, B, L, _p(workspace), workspace_bytes, _stream(stream)))
 
 
+def samba_model_workspace_size(m: Model, B, L) -> int:
+    return _model_ws(ctypes.byref(m), B, L)
+
+
+def samba_model_prefill(m: Model, ids, logits, B, L, workspace, workspace_bytes, stream=None):
+    _check("samba_model_prefill",
+           _model(ctypes.byref(m), _p(ids), _p(logits), B, L, _p(workspace), workspace_bytes, _stream(stream)))
+
+
+def samba_model_step_workspace_size(m: Model, B) -> int:
+    return _mstep_ws(ctypes.byref(m), B)
+
+
+def make_layer_states(states: Sequence[dict]):
+    """Host array of LayerState from dicts of device tensors (ssm, conv, k_ring, v_ring; absent = NULL)."""
+    n = len(states)
+    arr = (LayerState * max(n, 1))(*[LayerState(_p(d.get("ssm")), _p(d.get("conv")), _p(d.get("k_ring")),
+                                                 _p(d.get("v_ring"))) for d in states])
+    return arr
+
+
+def samba_model_step(m: Model, ids_t, logits, states, pos, B, workspace, workspace_bytes, stream=None):
+    _check("samba_model_step",
+           _mstep(ctypes.byref(m), _p(ids_t), _p(logits), ctypes.cast(states, ctypes.POINTER(LayerState)), _p(pos),
+                  B, _p(workspace), workspace_bytes, _stream(stream)))
+
+
 def samba_step_workspace_size(cfg: BlockConfig, B) -> int:
     return _step_ws(ctypes.byref(cfg), B)
 
@@ -234,12 +281,26 @@ def make_weights(wt: dict) -> BlockWeights:
     """wt: dict of device tensors keyed like inputs.block_weights()."""
     w = BlockWeights()
     for i in range(4):
-        w.norm_g[i] = _p(wt[f"norm{i}"])
+        w.norm_g[i] = _p(wt.get(f"norm{i}"))
     for name in ("W_in", "conv_w", "conv_b", "W_x", "W_dt", "dt_bias", "A_log", "W_out", "Wq", "Wk", "Wv", "Wo",
                  "mlp1_W1", "mlp1_W2", "mlp1_W3", "mlp2_W1", "mlp2_W2", "mlp2_W3"):
         setattr(w, name, _p(wt.get(name)))
-    w.Dskip = _p(wt["D"])
+    w.Dskip = _p(wt.get("D"))
     return w
+
+
+def make_model(cfg: BlockConfig, kinds: Sequence[int], layers: Sequence[dict], embedding, final_norm, lm_head,
+               vocab: int) -> Model:
+    """kinds: LAYER_* per sub-layer; layers: dicts of device tensors keyed like
+    inputs.block_weights() (a layer's kind decides which it reads).  The host
+    arrays live as attributes of the returned struct; keep the tensors alive."""
+    n = len(kinds)
+    ka = (c_int * max(n, 1))(*kinds)
+    la = (BlockWeights * max(n, 1))(*[make_weights(d) for d in layers])
+    m = Model(cfg, n, ctypes.cast(ka, ctypes.POINTER(c_int)), ctypes.cast(la, ctypes.POINTER(BlockWeights)),
+              _p(embedding), _p(final_norm), _p(lm_head), vocab)
+    m._keep = (ka, la)
+    return m
 
 
 def make_state(ssm, conv, k_ring, v_ring, pos) -> DecodeState:

@@ -2,6 +2,7 @@
 // the Samba block prefill and decode step [Samba 3.2 "Big-Picture
 // Architecture"; 3.4 "Detailed, Sentence-Based Technical Breakdown"].
 #include <algorithm>
+#include <initializer_list>
 #include <mutex>
 #include <set>
 #include <utility>
@@ -542,6 +543,98 @@ static samba_status swa_sublayer(const LayerCtx& X, const samba_block_weights* w
   return SAMBA_OK;
 }
 
+// Decode step of a Mamba sub-layer for one token per sequence (X.T = B rows):
+// conv-state shift, one recurrence step of the fp32 SSM state, gate, residual
+// [Samba 3.4 "The Mamba Layer" at a single t].  Every launch of a decode step is
+// a programmatic dependent of the one before it: a kernel sets up (and the
+// projections fetch their first weight tiles) while its predecessor finishes.
+static samba_status mamba_step_layer(const LayerCtx& X, const samba_block_weights* w, const void* x_in, void* x_out,
+                                     float* ssm, void* conv) {
+  const samba_block_config& c = X.c;
+  const BlockPlan& P = X.P;
+  const int B = X.B;
+  cudaStream_t st = X.st;
+  const samba_dtype dt = c.dtype;
+  auto buf = [&](size_t off) -> void* { return X.base + off; };
+  const int Di = c.d_inner, Dm = c.d_model, R = c.dt_rank;
+  const size_t es = dtype_size(dt);
+  void* xn = buf(P.xn);
+  char* hz = (char*)buf(P.hz);
+  char* xdbl = (char*)buf(P.xdbl);
+  auto gemm_pdl = [&](GemmArgs g) {
+    g.pdl = true;
+    return launch_gemm(g, st);
+  };
+  TRY(launch_rmsnorm(x_in, Dm, w->norm_g[0], xn, Dm, B, Dm, c.norm_eps, dt, st, true));
+  TRY(gemm_pdl(gemm1(xn, Dm, w->W_in, B, 2 * Di, Dm, hz, 2 * Di, dt)));
+  TRY(launch_conv_step(hz, 2 * Di, w->conv_w, w->conv_b, conv, buf(P.u), B, Di, c.d_conv, dt, st));
+  TRY(gemm_pdl(gemm1(buf(P.u), Di, w->W_x, B, P.xdw, Di, xdbl, P.xdw, dt)));
+  {
+    GemmArgs g = gemm1(xdbl, P.xdw, w->W_dt, B, Di, R, buf(P.dlt), Di, dt);
+    g.epi = kEpiSoftplus;
+    g.bias = w->dt_bias;
+    TRY(gemm_pdl(g));
+  }
+  TRY(launch_scan_step(buf(P.u), buf(P.dlt), hz + (size_t)Di * es, 2 * Di, xdbl, P.xdw, R, w->A_log, w->Dskip, ssm,
+                       buf(P.y), B, Di, dt, st));
+  GemmArgs g = gemm1(buf(P.y), Di, w->W_out, B, Dm, Di, x_out, Dm, dt);
+  g.epi = kEpiResid;
+  g.resid = x_in;
+  g.ldr = Dm;
+  return gemm_pdl(g);
+}
+
+// Decode step of an SWA sub-layer: q, k, v of the new token rotated at
+// position pos[b], k/v written to ring slot pos[b] mod window, attention over
+// the min(pos[b] + 1, window) valid slots, output projection, residual.
+// attn_ws: partials of the split attention for rings above 2048 slots.
+static samba_status swa_step_layer(const LayerCtx& X, const samba_block_weights* w, const void* x_in, void* x_out,
+                                   void* k_ring, void* v_ring, const int64_t* pos, void* attn_ws,
+                                   size_t attn_ws_bytes) {
+  const samba_block_config& c = X.c;
+  const BlockPlan& P = X.P;
+  const int B = X.B;
+  cudaStream_t st = X.st;
+  const samba_dtype dt = c.dtype;
+  auto buf = [&](size_t off) -> void* { return X.base + off; };
+  const int Dm = c.d_model;
+  void* xn = buf(P.xn);
+  char* qkv = (char*)buf(P.qkv);
+  float2* tab = (float2*)buf(P.tab);
+  TRY(launch_rmsnorm(x_in, Dm, w->norm_g[2], xn, Dm, B, Dm, c.norm_eps, dt, st, true));
+  const int hd = c.head_dim;
+  const int qw = c.n_q * hd, kvw = c.n_kv * hd;
+  {
+    GemmArgs g = gemm1(xn, Dm, w->Wq, B, P.qkvw, Dm, qkv, P.qkvw, dt);
+    g.nseg = 3;
+    g.seg[0].W = w->Wq;
+    g.seg[0].n = qw;
+    g.seg[1].W = w->Wk;
+    g.seg[1].n = kvw;
+    g.seg[2].W = w->Wv;
+    g.seg[2].n = kvw;
+    g.pdl = true;
+    if (c.rope_base != 0.f) {
+      TRY(launch_build_rope_table(tab, hd, c.rope_base, st, true));
+      g.epi = kEpiRope;
+      g.rope_cols = qw + kvw;
+      g.head_dim = hd;
+      g.pos_dev = pos;
+      g.rope_tab = tab;
+    }
+    TRY(launch_gemm(g, st));
+  }
+  TRY(launch_ring_write(qkv, P.qkvw, qw, qw + kvw, pos, k_ring, v_ring, B, c.window, kvw, dt, st));
+  TRY(launch_attn_decode(qkv, P.qkvw, pos, k_ring, v_ring, buf(P.o), B, c.n_q, c.n_kv, hd, c.window,
+                         1.0f / sqrtf((float)hd), dt, st, attn_ws, attn_ws_bytes));
+  GemmArgs g = gemm1(buf(P.o), qw, w->Wo, B, Dm, qw, x_out, Dm, dt);
+  g.epi = kEpiResid;
+  g.resid = x_in;
+  g.ldr = Dm;
+  g.pdl = true;
+  return launch_gemm(g, st);
+}
+
 // One block over B x L tokens.  pos0 > 0 continues a prefill from the decode
 // state `stt` holds after pos0 tokens (chunked prefill): the conv history, the
 // SSM state and the ring's last window of K/V are the inputs before token 0,
@@ -621,6 +714,173 @@ samba_status samba_block_fwd_chunk(const samba_block_config* cfg, const samba_bl
 }
 
 
+// ------------------------------------------------------------------ language-model stack
+}  // extern "C"
+
+namespace samba {
+
+struct ModelPlan {
+  BlockPlan P;                 // one sub-layer's activations over all B*L tokens
+  size_t xa, xb, xl, total;    // two residual streams, the normed last rows
+};
+
+static ModelPlan plan_model(const samba_block_config& c, int B, int L) {
+  ModelPlan m;
+  const int64_t T = (int64_t)B * L;
+  const size_t es = dtype_size(c.dtype);
+  m.P = plan_block(c, T);
+  Carve cv;
+  cv.off = m.P.total;
+  m.xa = cv.take(T * c.d_model * es);
+  m.xb = cv.take(T * c.d_model * es);
+  m.xl = cv.take((size_t)B * c.d_model * es);
+  m.total = cv.off + 256;
+  return m;
+}
+
+static samba_status validate_layer(int kind, const samba_block_weights& w) {
+  std::initializer_list<const void*> mamba = {w.norm_g[0], w.W_in, w.conv_w, w.W_x, w.W_dt,
+                                              w.dt_bias,   w.A_log, w.Dskip, w.W_out};
+  std::initializer_list<const void*> mlp = {w.norm_g[1], w.mlp1_W1, w.mlp1_W2, w.mlp1_W3};
+  std::initializer_list<const void*> swa = {w.norm_g[2], w.Wq, w.Wk, w.Wv, w.Wo};
+  const std::initializer_list<const void*>* req =
+      kind == SAMBA_LAYER_MAMBA ? &mamba : kind == SAMBA_LAYER_MLP ? &mlp : kind == SAMBA_LAYER_SWA ? &swa : nullptr;
+  if (!req) return SAMBA_ERR_INVALID_ARG;
+  for (const void* p : *req)
+    if (!p) return SAMBA_ERR_INVALID_ARG;
+  for (const void* p : *req)
+    if (!aligned16(p)) return SAMBA_ERR_UNSUPPORTED;
+  return SAMBA_OK;
+}
+
+}  // namespace samba
+
+extern "C" {
+
+size_t samba_model_workspace_size(const samba_model* m, int B, int L) {
+  if (!m || validate_cfg(&m->cfg) != SAMBA_OK || B < 1 || L < 1) return 0;
+  return plan_model(m->cfg, B, L).total;
+}
+
+samba_status samba_model_prefill(const samba_model* m, const int32_t* ids, void* logits, int B, int L,
+                                 void* workspace, size_t workspace_bytes, samba_stream stream) {
+  if (!m) return SAMBA_ERR_INVALID_ARG;
+  TRY(validate_cfg(&m->cfg));
+  if (!ids || !logits || B < 1 || L < 1 || m->n_layers < 0 || m->vocab < 1) return SAMBA_ERR_INVALID_ARG;
+  if (m->n_layers > 0 && (!m->kinds || !m->layers)) return SAMBA_ERR_INVALID_ARG;
+  if (!m->embedding || !m->final_norm || !m->lm_head) return SAMBA_ERR_INVALID_ARG;
+  for (int i = 0; i < m->n_layers; ++i) TRY(validate_layer(m->kinds[i], m->layers[i]));
+  if ((int64_t)L > (int64_t(1) << 30)) return SAMBA_ERR_UNSUPPORTED;
+  const samba_block_config& c = m->cfg;
+  const ModelPlan MP = plan_model(c, B, L);
+  if (!workspace || workspace_bytes < MP.total) return SAMBA_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  const samba_dtype dt = c.dtype;
+  const size_t es = dtype_size(dt);
+  char* base = (char*)(((uintptr_t)workspace + 255) & ~uintptr_t(255));
+  const int64_t T = (int64_t)B * L;
+  const int Dm = c.d_model;
+  char* cur = base + MP.xa;
+  char* nxt = base + MP.xb;
+  TRY(launch_embedding(ids, m->embedding, cur, T, Dm, m->vocab, dt, st));
+  const LayerCtx X{c, MP.P, base, B, L, T, st};
+  for (int i = 0; i < m->n_layers; ++i) {
+    const samba_block_weights& w = m->layers[i];
+    switch (m->kinds[i]) {
+      case SAMBA_LAYER_MAMBA: TRY(mamba_sublayer(X, &w, cur, nxt, nullptr, false, nullptr)); break;
+      case SAMBA_LAYER_SWA: TRY(swa_sublayer(X, &w, cur, nxt, nullptr, 0, false, nullptr)); break;
+      default:
+        TRY(mlp_sublayer(c, w.norm_g[1], w.mlp1_W1, w.mlp1_W2, w.mlp1_W3, cur, nxt, base + MP.P.xn,
+                         base + MP.P.hmlp, nullptr, T, st));
+        break;
+    }
+    std::swap(cur, nxt);
+  }
+  // final RMSNorm of each sequence's last position, then the vocabulary projection
+  TRY(launch_rmsnorm(cur + (size_t)(L - 1) * Dm * es, (int64_t)L * Dm, m->final_norm, base + MP.xl, Dm, B, Dm,
+                     c.norm_eps, dt, st));
+  return launch_gemm(gemm1(base + MP.xl, Dm, m->lm_head, B, m->vocab, Dm, logits, m->vocab, dt), st);
+}
+
+}  // extern "C"
+
+namespace samba {
+
+struct ModelStepPlan {
+  BlockPlan P;
+  size_t xa, xb, xl, attn, attn_bytes, total;
+};
+
+static ModelStepPlan plan_model_step(const samba_block_config& c, int B) {
+  ModelStepPlan m;
+  const size_t es = dtype_size(c.dtype);
+  m.P = plan_block(c, B);
+  Carve cv;
+  cv.off = m.P.total;
+  m.xa = cv.take((size_t)B * c.d_model * es);
+  m.xb = cv.take((size_t)B * c.d_model * es);
+  m.xl = cv.take((size_t)B * c.d_model * es);
+  m.attn_bytes = attn_decode_workspace_bytes(B, c.n_kv, c.window);
+  m.attn = cv.take(m.attn_bytes);
+  m.total = cv.off + 256;
+  return m;
+}
+
+}  // namespace samba
+
+extern "C" {
+
+size_t samba_model_step_workspace_size(const samba_model* m, int B) {
+  if (!m || validate_cfg(&m->cfg) != SAMBA_OK || B < 1) return 0;
+  return plan_model_step(m->cfg, B).total;
+}
+
+samba_status samba_model_step(const samba_model* m, const int32_t* ids_t, void* logits, samba_layer_state* states,
+                              int64_t* pos, int B, void* workspace, size_t workspace_bytes, samba_stream stream) {
+  if (!m) return SAMBA_ERR_INVALID_ARG;
+  TRY(validate_cfg(&m->cfg));
+  if (!ids_t || !logits || !pos || B < 1 || m->n_layers < 0 || m->vocab < 1) return SAMBA_ERR_INVALID_ARG;
+  if (m->n_layers > 0 && (!m->kinds || !m->layers || !states)) return SAMBA_ERR_INVALID_ARG;
+  if (!m->embedding || !m->final_norm || !m->lm_head) return SAMBA_ERR_INVALID_ARG;
+  for (int i = 0; i < m->n_layers; ++i) {
+    TRY(validate_layer(m->kinds[i], m->layers[i]));
+    const samba_layer_state& sl = states[i];
+    if (m->kinds[i] == SAMBA_LAYER_MAMBA && (!sl.ssm || !sl.conv)) return SAMBA_ERR_INVALID_ARG;
+    if (m->kinds[i] == SAMBA_LAYER_SWA && (!sl.k_ring || !sl.v_ring)) return SAMBA_ERR_INVALID_ARG;
+  }
+  const samba_block_config& c = m->cfg;
+  const ModelStepPlan MP = plan_model_step(c, B);
+  if (!workspace || workspace_bytes < MP.total) return SAMBA_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  const samba_dtype dt = c.dtype;
+  char* base = (char*)(((uintptr_t)workspace + 255) & ~uintptr_t(255));
+  const int Dm = c.d_model;
+  char* cur = base + MP.xa;
+  char* nxt = base + MP.xb;
+  TRY(launch_embedding(ids_t, m->embedding, cur, B, Dm, m->vocab, dt, st));
+  const LayerCtx X{c, MP.P, base, B, 1, (int64_t)B, st};
+  for (int i = 0; i < m->n_layers; ++i) {
+    const samba_block_weights& w = m->layers[i];
+    const samba_layer_state& sl = states[i];
+    switch (m->kinds[i]) {
+      case SAMBA_LAYER_MAMBA: TRY(mamba_step_layer(X, &w, cur, nxt, sl.ssm, sl.conv)); break;
+      case SAMBA_LAYER_SWA:
+        TRY(swa_step_layer(X, &w, cur, nxt, sl.k_ring, sl.v_ring, pos, base + MP.attn, MP.attn_bytes));
+        break;
+      default:
+        TRY(mlp_sublayer(c, w.norm_g[1], w.mlp1_W1, w.mlp1_W2, w.mlp1_W3, cur, nxt, base + MP.P.xn,
+                         base + MP.P.hmlp, nullptr, B, st, true));
+        break;
+    }
+    std::swap(cur, nxt);
+  }
+  TRY(launch_rmsnorm(cur, Dm, m->final_norm, base + MP.xl, Dm, B, Dm, c.norm_eps, dt, st, true));
+  GemmArgs g = gemm1(base + MP.xl, Dm, m->lm_head, B, m->vocab, Dm, logits, m->vocab, dt);
+  g.pdl = true;
+  TRY(launch_gemm(g, st));
+  return launch_pos_update(pos, B, 1, false, st, true);
+}
+
 // ------------------------------------------------------------------ decode step
 size_t samba_step_workspace_size(const samba_block_config* cfg, int B) {
   if (validate_cfg(cfg) != SAMBA_OK || B < 1) return 0;
@@ -639,82 +899,15 @@ samba_status samba_step(const samba_block_config* cfg, const samba_block_weights
   if (!workspace || workspace_bytes < P.total) return SAMBA_ERR_INVALID_ARG;
   if (!aligned16(x_t) || !aligned16(y_t)) return SAMBA_ERR_UNSUPPORTED;
   cudaStream_t st = (cudaStream_t)stream;
-  const samba_dtype dt = c.dtype;
   char* base = (char*)(((uintptr_t)workspace + 255) & ~uintptr_t(255));
-  auto buf = [&](size_t off) -> void* { return base + off; };
-  const int Di = c.d_inner, Dm = c.d_model, R = c.dt_rank;
-  const size_t es = dtype_size(dt);
-  void* xn = buf(P.xn);
-  char* hz = (char*)buf(P.hz);
-  char* xdbl = (char*)buf(P.xdbl);
-  char* qkv = (char*)buf(P.qkv);
-  float2* tab = (float2*)buf(P.tab);
-  void *x1 = buf(P.x1), *x2 = buf(P.x2), *x3 = buf(P.x3);
-
-  // ---- Mamba, one step
-  // Every launch of the step is a programmatic dependent of the one before it:
-  // a kernel sets up (and the projections fetch their first weight tiles) while
-  // its predecessor finishes.
-  auto gemm_pdl = [&](GemmArgs g) {
-    g.pdl = true;
-    return launch_gemm(g, st);
-  };
-  TRY(launch_rmsnorm(x_t, Dm, w->norm_g[0], xn, Dm, B, Dm, c.norm_eps, dt, st, true));
-  TRY(gemm_pdl(gemm1(xn, Dm, w->W_in, B, 2 * Di, Dm, hz, 2 * Di, dt)));
-  TRY(launch_conv_step(hz, 2 * Di, w->conv_w, w->conv_b, stt->conv, buf(P.u), B, Di, c.d_conv, dt, st));
-  TRY(gemm_pdl(gemm1(buf(P.u), Di, w->W_x, B, P.xdw, Di, xdbl, P.xdw, dt)));
-  {
-    GemmArgs g = gemm1(xdbl, P.xdw, w->W_dt, B, Di, R, buf(P.dlt), Di, dt);
-    g.epi = kEpiSoftplus;
-    g.bias = w->dt_bias;
-    TRY(gemm_pdl(g));
-  }
-  TRY(launch_scan_step(buf(P.u), buf(P.dlt), hz + (size_t)Di * es, 2 * Di, xdbl, P.xdw, R, w->A_log, w->Dskip,
-                       stt->ssm, buf(P.y), B, Di, dt, st));
-  {
-    GemmArgs g = gemm1(buf(P.y), Di, w->W_out, B, Dm, Di, x1, Dm, dt);
-    g.epi = kEpiResid;
-    g.resid = x_t;
-    g.ldr = Dm;
-    TRY(gemm_pdl(g));
-  }
-  TRY(mlp_sublayer(c, w->norm_g[1], w->mlp1_W1, w->mlp1_W2, w->mlp1_W3, x1, x2, xn, buf(P.hmlp), nullptr, B, st,
-                   true));
-  // ---- SWA over the ring
-  TRY(launch_rmsnorm(x2, Dm, w->norm_g[2], xn, Dm, B, Dm, c.norm_eps, dt, st, true));
-  const int hd = c.head_dim;
-  const int qw = c.n_q * hd, kvw = c.n_kv * hd;
-  {
-    GemmArgs g = gemm1(xn, Dm, w->Wq, B, P.qkvw, Dm, qkv, P.qkvw, dt);
-    g.nseg = 3;
-    g.seg[0].W = w->Wq;
-    g.seg[0].n = qw;
-    g.seg[1].W = w->Wk;
-    g.seg[1].n = kvw;
-    g.seg[2].W = w->Wv;
-    g.seg[2].n = kvw;
-    if (c.rope_base != 0.f) {
-      TRY(launch_build_rope_table(tab, hd, c.rope_base, st, true));
-      g.epi = kEpiRope;
-      g.rope_cols = qw + kvw;
-      g.head_dim = hd;
-      g.pos_dev = stt->pos;
-      g.rope_tab = tab;
-    }
-    TRY(gemm_pdl(g));
-  }
-  TRY(launch_ring_write(qkv, P.qkvw, qw, qw + kvw, stt->pos, stt->k_ring, stt->v_ring, B, c.window, kvw, dt, st));
-  TRY(launch_attn_decode(qkv, P.qkvw, stt->pos, stt->k_ring, stt->v_ring, buf(P.o), B, c.n_q, c.n_kv, hd, c.window,
-                         1.0f / sqrtf((float)hd), dt, st));
-  {
-    GemmArgs g = gemm1(buf(P.o), qw, w->Wo, B, Dm, qw, x3, Dm, dt);
-    g.epi = kEpiResid;
-    g.resid = x2;
-    g.ldr = Dm;
-    TRY(gemm_pdl(g));
-  }
-  TRY(mlp_sublayer(c, w->norm_g[3], w->mlp2_W1, w->mlp2_W2, w->mlp2_W3, x3, y_t, xn, buf(P.hmlp), nullptr, B, st,
-                   true));
+  const LayerCtx X{c, P, base, B, 1, (int64_t)B, st};
+  void *x1 = base + P.x1, *x2 = base + P.x2, *x3 = base + P.x3;
+  TRY(mamba_step_layer(X, w, x_t, x1, stt->ssm, stt->conv));
+  TRY(mlp_sublayer(c, w->norm_g[1], w->mlp1_W1, w->mlp1_W2, w->mlp1_W3, x1, x2, base + P.xn, base + P.hmlp, nullptr,
+                   B, st, true));
+  TRY(swa_step_layer(X, w, x2, x3, stt->k_ring, stt->v_ring, stt->pos, nullptr, 0));
+  TRY(mlp_sublayer(c, w->norm_g[3], w->mlp2_W1, w->mlp2_W2, w->mlp2_W3, x3, y_t, base + P.xn, base + P.hmlp, nullptr,
+                   B, st, true));
   return launch_pos_update(stt->pos, B, 1, false, st, true);
 }
 

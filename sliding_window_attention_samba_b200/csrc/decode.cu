@@ -228,27 +228,16 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // are zero padding): S = Q K^T, then O = P V with P taken straight from the S
 // accumulators.  Max/sum/O are combined across the 8 warps in shared memory,
 // then across the cluster's CTAs through distributed shared memory.
-__global__ void __launch_bounds__(256, 1)
-    attn_decode_split_kernel(const bf16* __restrict__ qkv, int64_t ld, const int64_t* __restrict__ pos,
-                             const bf16* __restrict__ k_ring, const bf16* __restrict__ v_ring, bf16* __restrict__ o,
-                             int Hq, int Hkv, int window, float scale_log2) {
-  pdl_wait();
-  pdl_trigger();
-  extern __shared__ __align__(16) unsigned char dec_dyn[];  // K slice | V slice (bf16, padded rows)
-  bf16* Ks = reinterpret_cast<bf16*>(dec_dyn);
-  bf16* Vs = Ks + kSliceMax * kKvPad;
-  __shared__ DecPart part;
-  __shared__ float wm[8][8], wl[8][8];  // [warp][head] partial max / sum
-  __shared__ float wo[8][8][kHd];       // [warp][head][dim] partial O
-  const uint32_t rank = dec_cluster_rank();
-  const int g = blockIdx.y, b = blockIdx.z;
-  const int grp = Hq / Hkv;
+// Partial attention of the grp <= 8 query heads of kv head g (batch row b) over
+// the ring slots [s0, s0 + n), n <= kSliceMax (the first `slice` rows of the
+// shared K/V tiles are written, rows past n as zeros).  Leaves the per-head
+// max, sum and unnormalised O in `part`.  All 256 threads take part.
+__device__ __forceinline__ void dec_slice_partial(const bf16* __restrict__ qkv, int64_t ld,
+                                                  const bf16* __restrict__ k_ring, const bf16* __restrict__ v_ring,
+                                                  int Hkv, int grp, int window, int g, int b, int s0, int n,
+                                                  int slice, float scale_log2, bf16* Ks, bf16* Vs, DecPart& part,
+                                                  float (&wm)[8][8], float (&wl)[8][8], float (&wo)[8][8][kHd]) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t P = pos[b];
-  const int nvalid = (int)(P + 1 < window ? P + 1 : window);
-  const int slice = ((nvalid + kSplit - 1) / kSplit + 31) & ~31;
-  const int s0 = (int)rank * slice;
-  const int n = max(0, min(nvalid, s0 + slice) - s0);
   const size_t kvw = (size_t)Hkv * kHd;
   // ---- K/V slice -> smem (16-byte vectors, all loads in flight before the stores);
   // rows past n are zero-filled so that the tensor-core tiles read finite values
@@ -383,6 +372,30 @@ __global__ void __launch_bounds__(256, 1)
       part.l[h] = ll;
     }
   }
+}
+
+__global__ void __launch_bounds__(256, 1)
+    attn_decode_split_kernel(const bf16* __restrict__ qkv, int64_t ld, const int64_t* __restrict__ pos,
+                             const bf16* __restrict__ k_ring, const bf16* __restrict__ v_ring, bf16* __restrict__ o,
+                             int Hq, int Hkv, int window, float scale_log2) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ __align__(16) unsigned char dec_dyn[];  // K slice | V slice (bf16, padded rows)
+  bf16* Ks = reinterpret_cast<bf16*>(dec_dyn);
+  bf16* Vs = Ks + kSliceMax * kKvPad;
+  __shared__ DecPart part;
+  __shared__ float wm[8][8], wl[8][8];  // [warp][head] partial max / sum
+  __shared__ float wo[8][8][kHd];       // [warp][head][dim] partial O
+  const uint32_t rank = dec_cluster_rank();
+  const int g = blockIdx.y, b = blockIdx.z;
+  const int grp = Hq / Hkv;
+  const int64_t P = pos[b];
+  const int nvalid = (int)(P + 1 < window ? P + 1 : window);
+  const int slice = ((nvalid + kSplit - 1) / kSplit + 31) & ~31;
+  const int s0 = (int)rank * slice;
+  const int n = max(0, min(nvalid, s0 + slice) - s0);
+  dec_slice_partial(qkv, ld, k_ring, v_ring, Hkv, grp, window, g, b, s0, n, slice, scale_log2, Ks, Vs, part, wm, wl,
+                    wo);
   __syncthreads();
   const uint32_t tok = dec_cluster_sync();
   // ---- merge: rank r finalises query head r of the group
@@ -408,6 +421,68 @@ __global__ void __launch_bounds__(256, 1)
     o[(size_t)b * Hq * kHd + (size_t)h * kHd + threadIdx.x] = __float2bfloat16_rn(O / Lsum);
   }
   (void)dec_cluster_sync();  // peers' shared memory stays valid until every merge is done
+}
+
+// Long caches (more than kSplit * kSliceMax slots, e.g. a full-attention KV
+// cache): one CTA per 256-slot slice, grid (cache / 256, Hkv, B); CTAs past the
+// valid slots publish an empty partial.  Partials go to `ws`, and
+// attn_decode_merge_kernel combines them (flash-decoding).
+__global__ void __launch_bounds__(256, 1)
+    attn_decode_long_kernel(const bf16* __restrict__ qkv, int64_t ld, const int64_t* __restrict__ pos,
+                            const bf16* __restrict__ k_ring, const bf16* __restrict__ v_ring,
+                            DecPart* __restrict__ ws, int Hq, int Hkv, int window, float scale_log2) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ __align__(16) unsigned char dec_dyn[];
+  bf16* Ks = reinterpret_cast<bf16*>(dec_dyn);
+  bf16* Vs = Ks + kSliceMax * kKvPad;
+  __shared__ DecPart part;
+  __shared__ float wm[8][8], wl[8][8];
+  __shared__ float wo[8][8][kHd];
+  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int grp = Hq / Hkv;
+  const int64_t P = pos[b];
+  const int nvalid = (int)(P + 1 < window ? P + 1 : window);
+  const int s0 = split * kSliceMax;
+  const int n = max(0, min(nvalid, s0 + kSliceMax) - s0);
+  DecPart* dst = ws + ((size_t)b * Hkv + g) * gridDim.x + split;
+  if (n == 0) {  // block-uniform: past the valid slots
+    if (threadIdx.x < 8) {
+      dst->m[threadIdx.x] = -INFINITY;
+      dst->l[threadIdx.x] = 0.f;
+    }
+    return;
+  }
+  dec_slice_partial(qkv, ld, k_ring, v_ring, Hkv, grp, window, g, b, s0, n, (n + 31) & ~31, scale_log2, Ks, Vs,
+                    part, wm, wl, wo);
+  __syncthreads();
+  for (int e = threadIdx.x; e < grp * kHd; e += 256) dst->o[e / kHd][e % kHd] = part.o[e / kHd][e % kHd];
+  if (threadIdx.x < grp) {
+    dst->m[threadIdx.x] = part.m[threadIdx.x];
+    dst->l[threadIdx.x] = part.l[threadIdx.x];
+  }
+}
+
+// o[b, h] = merge over the splits of (m, l, O) of query head h: one CTA of 64
+// threads (head dims) per (query head, batch row).
+__global__ void attn_decode_merge_kernel(const DecPart* __restrict__ ws, bf16* __restrict__ o, int Hq, int Hkv,
+                                         int nsplit) {
+  pdl_wait();
+  pdl_trigger();
+  const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
+  const int grp = Hq / Hkv, g = h / grp, hw = h % grp;
+  const DecPart* src = ws + ((size_t)b * Hkv + g) * nsplit;
+  float M = -INFINITY;
+  for (int s = 0; s < nsplit; ++s) M = fmaxf(M, src[s].m[hw]);
+  float Lsum = 0.f, O = 0.f;
+  for (int s = 0; s < nsplit; ++s) {
+    const float ms = src[s].m[hw];
+    if (ms == -INFINITY) continue;
+    const float wgt = ex2_approx(ms - M);
+    Lsum += wgt * src[s].l[hw];
+    O += wgt * src[s].o[hw][d];
+  }
+  o[(size_t)b * Hq * kHd + (size_t)h * kHd + d] = __float2bfloat16_rn(O / Lsum);
 }
 
 __global__ void pos_add_kernel(int64_t* pos, int B, int64_t inc, int set) {
@@ -524,10 +599,30 @@ samba_status launch_ring_write(const void* qkv, int64_t ld, int k_off, int v_off
   return SAMBA_OK;
 }
 
+size_t attn_decode_workspace_bytes(int B, int Hkv, int window) {
+  if (window <= kSplit * kSliceMax) return 0;
+  return (size_t)B * Hkv * ((window + kSliceMax - 1) / kSliceMax) * sizeof(DecPart);
+}
+
 samba_status launch_attn_decode(const void* qkv, int64_t ld, const int64_t* pos, const void* k_ring,
                                 const void* v_ring, void* o, int B, int Hq, int Hkv, int hd, int window, float scale,
-                                samba_dtype dt, cudaStream_t st) {
+                                samba_dtype dt, cudaStream_t st, void* ws, size_t ws_bytes) {
   if (hd > 128) return SAMBA_ERR_UNSUPPORTED;
+  if (dt == SAMBA_BF16 && hd == kHd && Hq / Hkv <= 8 && window > kSplit * kSliceMax && ld % 8 == 0) {
+    const int nsplit = (window + kSliceMax - 1) / kSliceMax;
+    if (!ws || ws_bytes < attn_decode_workspace_bytes(B, Hkv, window) || !aligned16(ws))
+      return SAMBA_ERR_INVALID_ARG;
+    const size_t smem = 2 * kSliceMax * kKvPad * sizeof(bf16);
+    if (!ensure_smem_attr(attn_decode_long_kernel, smem)) return SAMBA_ERR_CUDA;
+    if (launch_k(attn_decode_long_kernel, dim3(nsplit, Hkv, B), dim3(256), smem, st, true, (const bf16*)qkv, ld,
+                 pos, (const bf16*)k_ring, (const bf16*)v_ring, (DecPart*)ws, Hq, Hkv, window,
+                 scale * 1.4426950408889634f) != cudaSuccess)
+      return SAMBA_ERR_CUDA;
+    if (launch_k(attn_decode_merge_kernel, dim3(Hq, B), dim3(kHd), 0, st, true, (const DecPart*)ws, (bf16*)o, Hq,
+                 Hkv, nsplit) != cudaSuccess)
+      return SAMBA_ERR_CUDA;
+    return SAMBA_OK;
+  }
   if (dt == SAMBA_BF16 && hd == kHd && Hq / Hkv <= 8 && window <= kSplit * kSliceMax && ld % 8 == 0) {
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));

@@ -14,9 +14,12 @@ samba_status launch_scan_step(const void* u, const void* dlt, const void* z, int
                               int B, int D, samba_dtype dt, cudaStream_t st);
 samba_status launch_ring_write(const void* qkv, int64_t ld, int k_off, int v_off, const int64_t* pos, void* k_ring,
                                void* v_ring, int B, int window, int kvw, samba_dtype dt, cudaStream_t st);
+// Ring caches above 2048 slots (bf16, head_dim 64) need attn_decode_workspace_bytes() of workspace for the
+// per-slice partials; smaller ones none.
+size_t attn_decode_workspace_bytes(int B, int Hkv, int window);
 samba_status launch_attn_decode(const void* qkv, int64_t ld, const int64_t* pos, const void* k_ring,
                                 const void* v_ring, void* o, int B, int Hq, int Hkv, int hd, int window, float scale,
-                                samba_dtype dt, cudaStream_t st);
+                                samba_dtype dt, cudaStream_t st, void* ws = nullptr, size_t ws_bytes = 0);
 samba_status launch_pos_update(int64_t* pos, int B, int64_t value, bool set, cudaStream_t st, bool pdl = false);
 // prefill -> ring: the last min(L, w) tokens of a prefill whose token 0 is at absolute position pos0
 samba_status launch_ring_fill(const void* qkv, int64_t ld, int k_off, int v_off, void* k_ring, void* v_ring, int B,

@@ -58,6 +58,34 @@ samba_status launch_rmsnorm(const void* x, int64_t ld_x, const float* g, void* o
 }
 
 // ===========================================================================
+// Token embedding lookup [Samba 3.2: token embeddings enter the first layer]:
+// one warp per token, 16-byte pieces of the row.
+// ===========================================================================
+__global__ void embedding_kernel(const int32_t* __restrict__ ids, const uint4* __restrict__ table,
+                                 uint4* __restrict__ out, int64_t T, int vec, int vocab, int* err) {
+  const int64_t t = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  const int id = ids[t];
+  const bool ok = id >= 0 && id < vocab;
+  if (!ok && lane == 0) raise_error(err, kErrDevice);
+  for (int i = lane; i < vec; i += 32) out[t * vec + i] = ok ? table[(int64_t)id * vec + i] : make_uint4(0, 0, 0, 0);
+}
+
+samba_status launch_embedding(const int32_t* ids, const void* table, void* out, int64_t T, int d_model, int vocab,
+                              samba_dtype dt, cudaStream_t st) {
+  if (!ids || !table || !out || T < 0 || d_model <= 0 || vocab < 1) return SAMBA_ERR_INVALID_ARG;
+  const size_t row = (size_t)d_model * dtype_size(dt);
+  if (row % 16 || !aligned16(table) || !aligned16(out)) return SAMBA_ERR_UNSUPPORTED;
+  if (T == 0) return SAMBA_OK;
+  const int warps = 8;
+  embedding_kernel<<<(unsigned)((T + warps - 1) / warps), warps * 32, 0, st>>>(
+      ids, (const uint4*)table, (uint4*)out, T, (int)(row / 16), vocab, device_error_word());
+  SAMBA_CHECK_LAUNCH();
+  return SAMBA_OK;
+}
+
+// ===========================================================================
 // Short convolution [Samba 3.4 "Input Projection and Short Convolution"]
 //   u[b,t,c] = SiLU(sum_j w[c,j] x[b,t-(k-1)+j,c] + bias[c])
 // A thread owns 8 consecutive channels and a run of kRun tokens, keeping the

@@ -40,6 +40,11 @@ samba_status launch_build_rope_table(float2* tab, int head_dim, float base, cuda
 samba_status launch_rope_apply(const void* x, void* out, int B, int L, int H, int head_dim, int64_t pos0,
                                const float2* tab, samba_dtype dt, cudaStream_t st);
 
+// ---------------- token embedding ----------------
+// out[t, :] = table[ids[t], :]; ids outside [0, vocab) latch kErrDevice and give zeros.
+samba_status launch_embedding(const int32_t* ids, const void* table, void* out, int64_t T, int d_model, int vocab,
+                              samba_dtype dt, cudaStream_t st);
+
 // ---------------- RMSNorm ----------------
 samba_status launch_rmsnorm(const void* x, int64_t ld_x, const float* g, void* out, int64_t ld_out, int64_t rows,
                             int dim, float eps, samba_dtype dt, cudaStream_t st, bool pdl = false);

@@ -363,3 +363,30 @@ def test_ring_slot_map_bit_exact():
         # the newest position p < L with p mod w == slot
         p = L - 1 - ((L - 1 - slot) % cfg.window)
         assert np.array_equal(r["state"]["k_ring"][0, slot], kr[0, p])
+
+
+# ---------------------------------------------------------------- language-model stack
+def test_model_stack_composes_the_block():
+    # [Mamba, MLP, SWA, MLP'] with MLP' carrying the block's second MLP is the block;
+    # the embedding lookup is an identity when the table holds the inputs row by row.
+    cfg = I.TINY
+    W = I.block_weights(cfg, 5)
+    x = I.block_input(cfg, 5, 1, 90)
+    W2 = dict(W, norm1=W["norm3"], mlp1_W1=W["mlp2_W1"], mlp1_W2=W["mlp2_W2"], mlp1_W3=W["mlp2_W3"])
+    g = RNG.standard_normal(cfg.d_model)
+    head = RNG.standard_normal((11, cfg.d_model))
+    ids = np.arange(90)[None]
+    got = O.model_prefill(ids, [("mamba", W), ("mlp", W), ("swa", W), ("mlp", W2)], x[0], g, head, cfg)
+    xo = O.block_fwd(x, W, cfg)["x_out"][:, -1]
+    want = (xo / np.sqrt((xo ** 2).mean(-1, keepdims=True) + cfg.norm_eps) * g) @ head.T
+    assert np.allclose(got, want, rtol=1e-12, atol=1e-12)
+
+
+def test_model_without_layers_reads_the_last_token():
+    # no layers, one-hot embeddings, identity head: logits are sqrt(d) at the last id
+    cfg = I.TINY
+    d = cfg.d_model
+    ids = np.array([[3, 17, 5], [60, 2, 41]])
+    logits = O.model_prefill(ids, [], np.eye(d), np.ones(d), np.eye(d), cfg)
+    assert list(logits.argmax(1)) == [5, 41]
+    assert np.allclose(logits.max(1), np.sqrt(d / (1 + d * cfg.norm_eps)), rtol=1e-12)
