@@ -49,8 +49,10 @@ def parse():
     ap.add_argument("--seq-len", type=int, default=None, help="override L (parity/debug runs only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default="prefill",
-                    choices=["prefill", "block", "decode", "sweep", "chunked", "model", "model_decode"],
+                    choices=["prefill", "block", "block38", "decode", "sweep", "chunked", "model",
+                             "model_decode"],
                     help="prefill: 4-block L=131072 stack (the headline); block: one block at B=4, L=4096; "
+                         "block38: one block at the 3.8B model's widths (head_dim 256), L=131072; "
                          "decode: B=32 samba_step stream; "
                          "sweep: scan and SWA alone at L = 4K..1M; "
                          "chunked: one block over L=1M in 32K-token chunks (samba_block_fwd_chunk); "
@@ -255,7 +257,7 @@ def _scan_contig(torch, L, s, w, u, dlt, hz, y, Bn, Ln):
 
 
 def workload_of(args):
-    return "block_bf16_B4_L4096" if args.workload == "block" else WORKLOAD
+    return {"block": "block_bf16_B4_L4096", "block38": "block38_bf16_L131072"}.get(args.workload, WORKLOAD)
 
 
 def run_cuda(args, rank, world, local_rank):
@@ -378,16 +380,17 @@ def kernel_report(kt, s, T, Bn, Ln, peaks):
     # Dominant kernel: the SwiGLU up-projection (gemm_tc_kernel<2>, ~32% of the
     # step in the launch list).  Timed alone by the attribution pass, so against
     # the burst peak.  DRAM traffic per launch from an ncu capture of this kernel
-    # at M = 16384 (dram__bytes_read.sum 203.3 MB, dram__bytes_write.sum 237.3 MB),
+    # at M = 16384 (dram__bytes_read.sum 204.2 MB, dram__bytes_write.sum 237.0 MB),
     # scaled to this M: the activation reads and the output writes grow with M,
     # the 67 MB of weights are read once whatever M is.
     name = "mlp1_up"
     up = [fl for (n, M, N, K, e, fl) in gl if n == name][0]
     w_bytes = 2 * s.d_ff * s.d_model * 2
     scale = T / 16384
-    traffic = (203.3e6 - w_bytes) * scale + w_bytes + 237.3e6 * scale
+    # measured at the 2048-wide shapes only
+    traffic = (204.2e6 - w_bytes) * scale + w_bytes + 237.0e6 * scale if s == I.WIDE else None
     roof = {"bound": "tensor", "achieved": round(up / kt[name] / 1e12, 2), "peak": tf_burst, "unit": "TFLOP/s",
-            "frac": round(up / kt[name] / 1e12 / tf_burst, 4), "traffic": round(traffic),
+            "frac": round(up / kt[name] / 1e12 / tf_burst, 4), "traffic": round(traffic) if traffic else None,
             "algorithmic_bytes": T * s.d_model * 2 + w_bytes + T * s.d_ff * 2,
             "kernel": "gemm_tc_kernel<2>: SwiGLU up-projection [T, d_model] x [2 d_ff, d_model]^T",
             "peak_source": src + " burst bf16 (kernel timed alone)",
@@ -937,7 +940,9 @@ def main():
             v, desc = oracle_sample(1024)
             cpu = {"value": v, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle", "sample": desc}
         launches_per_block = 4 + 10 + 1 + 1 + 1 + 1  # norms, projections, conv, scan, rope table, swa
-        line = {"metric": METRIC if args.workload == "prefill" else "prefill tokens/s per Samba block (B=4, L=4096)",
+        metric = {"prefill": METRIC, "block": "prefill tokens/s per Samba block (B=4, L=4096)",
+                  "block38": "prefill tokens/s per Samba block at the 3.8B widths (L=128K)"}[args.workload]
+        line = {"metric": metric,
                 "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": r["t_dev"] / args.steps * 1e3, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfgd,

@@ -94,7 +94,7 @@ samba_status samba_selective_scan(const void* u, const void* dt, const float* dt
  *   q, o : [B, L, Hq, head_dim] dtype      k, v : [B, L, Hkv, head_dim] dtype
  * RoPE pairs channel i with i + head_dim/2 and uses theta_i = rope_base^(-2i/head_dim);
  * angles are formed from fp64 tables so that positions up to 2^30 keep ~1e-7 rad.
- * Requirements: Hq % Hkv == 0, head_dim in {16, 32, 64, 128}, window >= 1,
+ * Requirements: Hq % Hkv == 0, head_dim in {16, 32, 64} (any dtype) or 256 (bf16), window >= 1,
  * pos0 >= 0, pos0 + L <= 2^30.  With rope_base != 0 the rotated copies of q and k
  * live in the workspace.
  * ---------------------------------------------------------------------- */
@@ -224,8 +224,9 @@ size_t samba_block_workspace_size(const samba_block_config* cfg, int B, int L);
  * overwritten with the decode state after the last token (SSM state, the last
  * d_conv-1 pre-conv inputs, the last min(L, window) post-RoPE keys/values in
  * their ring slots, pos[b] = L).  taps may be NULL.
- * Requirements: d_state == 16, head_dim == 64 for bf16 (16..128 for fp32),
- * d_model, d_inner, d_ff multiples of 64, n_q % n_kv == 0. */
+ * Requirements: d_state == 16, head_dim in {16, 32, 64} (64 or 256 on the bf16
+ * tensor-core path), d_model, d_inner, d_ff multiples of 64, dt_rank a multiple
+ * of 8, n_q % n_kv == 0.  samba_step supports head_dim <= 64. */
 samba_status samba_block_fwd(const samba_block_config* cfg, const samba_block_weights* w, const void* x_in,
                              void* x_out, samba_decode_state* st, const samba_block_taps* taps, int B, int L,
                              void* workspace, size_t workspace_bytes, samba_stream stream);

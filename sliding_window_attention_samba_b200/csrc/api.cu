@@ -137,7 +137,9 @@ static samba_status validate_cfg(const samba_block_config* c) {
   if (c->dtype != SAMBA_F32 && c->dtype != SAMBA_BF16) return SAMBA_ERR_INVALID_ARG;
   if (c->n_q % c->n_kv) return SAMBA_ERR_INVALID_ARG;
   if (c->d_state != 16 || c->d_conv < 2 || c->d_conv > 8) return SAMBA_ERR_UNSUPPORTED;
-  if (c->head_dim != 16 && c->head_dim != 32 && c->head_dim != 64) return SAMBA_ERR_UNSUPPORTED;
+  // head_dim 256 (the 3.8B shapes) runs on the bf16 tensor-core path only
+  if (c->head_dim != 16 && c->head_dim != 32 && c->head_dim != 64 && !(c->head_dim == 256 && c->dtype == SAMBA_BF16))
+    return SAMBA_ERR_UNSUPPORTED;
   if (c->d_model % 64 || c->d_inner % 64 || c->d_ff % 64) return SAMBA_ERR_UNSUPPORTED;
   const size_t es = dtype_size(c->dtype);
   if ((c->dt_rank * es) % 16) return SAMBA_ERR_UNSUPPORTED;
@@ -282,7 +284,8 @@ samba_status samba_swa_fwd(const void* q, const void* k, const void* v, void* o,
   if (!q || !k || !v || !o || B < 1 || L < 0 || Hq < 1 || Hkv < 1 || window < 1 || pos0 < 0 || rope_base < 0.f)
     return SAMBA_ERR_INVALID_ARG;
   if (Hq % Hkv) return SAMBA_ERR_INVALID_ARG;
-  if (head_dim != 16 && head_dim != 32 && head_dim != 64 && head_dim != 128) return SAMBA_ERR_UNSUPPORTED;
+  if (head_dim != 16 && head_dim != 32 && head_dim != 64 && !(head_dim == 256 && dtype == SAMBA_BF16))
+    return SAMBA_ERR_UNSUPPORTED;
   if (pos0 + (int64_t)L > (int64_t(1) << 30)) return SAMBA_ERR_UNSUPPORTED;
   if (L == 0) return SAMBA_OK;
   SwaArgs a;

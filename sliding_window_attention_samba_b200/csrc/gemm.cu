@@ -171,7 +171,6 @@ constexpr int TC_BM = 128, TC_BK = 64, TC_STAGES = 4, TC_MAXN = 256;
 constexpr int TC_EPI_WARPS = 8;  // two per TMEM lane quadrant, each taking half of the tile's columns
 constexpr int TC_THREADS = 64 + 32 * TC_EPI_WARPS;
 constexpr uint32_t TC_A_BYTES = TC_BM * TC_BK * 2;
-constexpr uint32_t TC_B_BYTES = TC_MAXN * TC_BK * 2;
 
 struct TcSmem {
   bf16 A[TC_STAGES][TC_BM * TC_BK];
@@ -242,24 +241,30 @@ __device__ __forceinline__ void tc_epilogue_tile(const TcParams& p, uint32_t tba
     return;
   }
   if (EPI == kEpiRope && col0 < a.rope_cols) {
-    // heads of 64 columns: rotate (i, i+32) pairs
-    const int hd2 = a.head_dim / 2;  // 32
+    // heads of head_dim columns (a multiple of 64): rotate (i, i + hd/2) pairs,
+    // 32 pairs per step; the warp's share is half of the tile's heads (or, for
+    // one head per tile, half of its pair chunks)
+    const int hd = a.head_dim, hd2 = hd / 2;
     const int64_t pos = in_range ? rope_position(a, row) : 0;
-    half_range(p.bn / (2 * hd2), half, u_lo, u_hi);
-    for (int hc = u_lo * 2 * hd2; hc < u_hi * 2 * hd2; hc += 2 * hd2) {
-      tmem_ld32(tbase + hc, r);
-      tmem_ld32(tbase + hc + hd2, r2);
+    const int nunits = p.bn / 64;  // (head, 32-pair chunk) units
+    half_range(nunits, half, u_lo, u_hi);
+    for (int u = u_lo; u < u_hi; ++u) {
+      const int hh = (u * 64) / hd;         // head within the tile
+      const int j0 = (u * 32) % hd2;        // first pair index of this unit
+      const int hc = hh * hd;
+      tmem_ld32(tbase + hc + j0, r);
+      tmem_ld32(tbase + hc + hd2 + j0, r2);
       tmem_wait_ld();
       if (in_range) {
         float lo[32], hi[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float2 cs = rope_cs(a.rope_tab, hd2, pos, i);
+          const float2 cs = rope_cs(a.rope_tab, hd2, pos, j0 + i);
           const float x1 = __uint_as_float(r[i]), x2 = __uint_as_float(r2[i]);
           lo[i] = x1 * cs.x - x2 * cs.y;
           hi[i] = x2 * cs.x + x1 * cs.y;
         }
-        bf16* o = out + row * a.ldo + col0 + hc;
+        bf16* o = out + row * a.ldo + col0 + hc + j0;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           store8(o + 8 * i, lo + 8 * i);
@@ -269,11 +274,14 @@ __device__ __forceinline__ void tc_epilogue_tile(const TcParams& p, uint32_t tba
     }
     return;
   }
-  half_range(p.bn / 32, half, u_lo, u_hi);
+  // 32-column chunks; a tile width of 16 mod 32 ends in a 16-column chunk (the
+  // TMEM columns past it are read but not stored)
+  half_range((p.bn + 31) / 32, half, u_lo, u_hi);
   for (int cc = u_lo * 32; cc < u_hi * 32; cc += 32) {
     tmem_ld32(tbase + cc, r);
     tmem_wait_ld();
     if (!in_range) continue;
+    const int nv = min(4, (p.bn - cc) / 8);  // valid 8-column groups: 4, or 2 in a 16-column tail
     float f[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(r[i]);
@@ -282,11 +290,13 @@ __device__ __forceinline__ void tc_epilogue_tile(const TcParams& p, uint32_t tba
       if (a.tap) {
         bf16* t = (bf16*)a.tap + row * a.ldt + col;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) store8(t + 8 * i, f + 8 * i);
+        for (int i = 0; i < 4; ++i)
+          if (i < nv) store8(t + 8 * i, f + 8 * i);
       }
       const bf16* rs = (const bf16*)a.resid + row * a.ldr + col;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
+        if (i >= nv) continue;
         float g[8];
         load8(rs + 8 * i, g);
 #pragma unroll
@@ -296,6 +306,7 @@ __device__ __forceinline__ void tc_epilogue_tile(const TcParams& p, uint32_t tba
       const float4* bp = reinterpret_cast<const float4*>(a.bias + col);  // 16-byte aligned (checked at launch)
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
+        if (i >= 2 * nv) continue;
         const float4 b4 = bp[i];
         f[4 * i + 0] = softplus_fast(f[4 * i + 0] + b4.x);
         f[4 * i + 1] = softplus_fast(f[4 * i + 1] + b4.y);
@@ -305,7 +316,8 @@ __device__ __forceinline__ void tc_epilogue_tile(const TcParams& p, uint32_t tba
     }
     bf16* o = out + row * a.ldo + col;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) store8(o + 8 * i, f + 8 * i);
+    for (int i = 0; i < 4; ++i)
+      if (i < nv) store8(o + 8 * i, f + 8 * i);
   }
 }
 
@@ -432,7 +444,7 @@ bool tc_bn_for(const GemmArgs& a, int& bn) {
     bn = 128;
     return a.nseg == 1 && a.N % 128 == 0;
   }
-  if (a.nseg == 1 && a.N <= TC_MAXN && a.N % 32 == 0) {
+  if (a.nseg == 1 && a.N <= TC_MAXN && a.N % 16 == 0) {
     bn = a.N;
     return true;
   }
@@ -463,11 +475,14 @@ samba_status tc_launch(TcParams& p, cudaStream_t st) {
 }  // namespace
 
 bool gemm_tc_supported(const GemmArgs& a) {
-  if (a.dtype != SAMBA_BF16 || a.K % TC_BK != 0 || a.lda % 8 || a.ldo % 8 || a.M < 1) return false;
+  // K need not be a multiple of 64: the tensor maps end at K and fill the last
+  // k-block with zeros
+  if (a.dtype != SAMBA_BF16 || a.K % 8 != 0 || a.lda % 8 || a.ldo % 8 || a.M < 1) return false;
   if (!aligned16(a.A) || !aligned16(a.out)) return false;
   int bn;
   if (!tc_bn_for(a, bn)) return false;
-  if (a.epi == kEpiRope && (a.head_dim != 64 || a.rope_cols % 64 != 0)) return false;
+  if (a.epi == kEpiRope && (a.head_dim % 64 != 0 || a.rope_cols % a.head_dim != 0)) return false;
+  if (a.epi == kEpiRope && bn % a.head_dim != 0) return false;  // whole heads per tile
   if (a.epi == kEpiResid && (a.ldr % 8 || (a.tap && a.ldt % 8))) return false;
   if (a.epi == kEpiSoftplus && !aligned16(a.bias)) return false;
   for (int s = 0; s < a.nseg; ++s)
@@ -491,7 +506,7 @@ samba_status launch_gemm_tc(const GemmArgs& a, cudaStream_t st) {
     for (int g = 1; g <= p.n_tiles; ++g)
       if (p.n_tiles % g == 0 && (size_t)g * panel <= (size_t(32) << 20)) p.group_n = g;
   }
-  p.k_blocks = a.K / TC_BK;
+  p.k_blocks = (a.K + TC_BK - 1) / TC_BK;
   {
     uint64_t dims[2] = {(uint64_t)a.K, (uint64_t)a.M};
     uint64_t strides[1] = {(uint64_t)a.lda};

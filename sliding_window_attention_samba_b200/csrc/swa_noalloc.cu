@@ -70,7 +70,8 @@ extern "C" samba_status samba_swa_fwd_noalloc(const void* q, const void* k, cons
   if (!q || !k || !v || !o || B < 1 || L < 0 || Hq < 1 || Hkv < 1 || window < 1 || pos0 < 0 || rope_base < 0.f)
     return SAMBA_ERR_INVALID_ARG;
   if (Hq % Hkv) return SAMBA_ERR_INVALID_ARG;
-  if (head_dim != 16 && head_dim != 32 && head_dim != 64 && head_dim != 128) return SAMBA_ERR_UNSUPPORTED;
+  if (head_dim != 16 && head_dim != 32 && head_dim != 64 && !(head_dim == 256 && dtype == SAMBA_BF16))
+    return SAMBA_ERR_UNSUPPORTED;
   if (pos0 + (int64_t)L > (int64_t(1) << 30)) return SAMBA_ERR_UNSUPPORTED;
   if (L == 0) return SAMBA_OK;
   SwaArgs a;

@@ -323,6 +323,257 @@ __global__ void __launch_bounds__(AT_THREADS, 1) swa_tc_kernel(const __grid_cons
 }
 
 // ---------------------------------------------------------------------------
+// Head dim 256 (the 3.8B shapes: 11 query heads over one kv head), one query
+// head per CTA.  Q (128 x 256) and each K/V tile (64 keys x 256) are four
+// 64-column 128B-swizzled sub-tiles; S = Q K^T is 16 K16 steps into a
+// double-buffered 64-column S; O = P V is M128 x N256 (V MN-major across four
+// 64-wide atoms, 8 KB apart) accumulated over four K16 key steps.  TMEM:
+// S0 | S1 | O = 64 + 64 + 256 columns.  Shared memory: Q 64 KB, two K/V stages
+// 128 KB, two P tiles 32 KB.  Roles as in swa_tc_kernel.
+constexpr int H_BN = 64;      // keys per tile
+constexpr int H_D = 256;      // head dim
+constexpr int H_STAGES = 2;
+constexpr uint32_t kHQBytes = AT_BM * H_D * 2;    // 64 KB
+constexpr uint32_t kHKVBytes = H_BN * H_D * 2;    // 32 KB (K or V tile)
+
+struct AtHSmem {
+  bf16 Q[4][AT_BM * 64];             // [d atom][row][64]
+  bf16 K[H_STAGES][4][H_BN * 64];    // [stage][d atom][key][64]
+  bf16 V[H_STAGES][4][H_BN * 64];
+  bf16 P[2][AT_BM * 64];             // [buffer][row][64 keys]
+  uint64_t q_full;
+  uint64_t kv_full[H_STAGES], kv_empty[H_STAGES];
+  uint64_t s_full[2], s_free[2], p_full[2], pv_done[2];
+  uint32_t tmem_base;
+};
+
+__global__ void __launch_bounds__(AT_THREADS, 1) swa_tc256_kernel(const __grid_constant__ AtParams p, int* err) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  AtHSmem& S = *reinterpret_cast<AtHSmem*>(smem_raw + smem_align_pad(smem_raw, 1024));
+  const int warp = warp_id_sync();
+  const int lane = threadIdx.x & 31;
+  const int t0 = blockIdx.x * AT_BM;
+  const int h = blockIdx.y;
+  const int b = blockIdx.z;
+  const int g = h / (p.Hq / p.Hkv);
+  const int tk0 = t0 + p.qoff;
+  const int lo = tk0 - p.window + 1;
+  const int kb0 = lo <= 0 ? 0 : (lo / H_BN) * H_BN;
+  const int ntile = (min(tk0 + AT_BM - 1, p.Lk - 1) - kb0) / H_BN + 1;
+
+  if (warp == 0 && lane == 0) {
+    mbar_init(&S.q_full, 1);
+    for (int s = 0; s < H_STAGES; ++s) {
+      mbar_init(&S.kv_full[s], 1);
+      mbar_init(&S.kv_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&S.s_full[i], 1);
+      mbar_init(&S.s_free[i], 4);
+      mbar_init(&S.p_full[i], 4);
+      mbar_init(&S.pv_done[i], 1);
+    }
+    fence_mbar_init();
+    tma_prefetch_desc(&p.tmQ);
+    tma_prefetch_desc(&p.tmK);
+    tma_prefetch_desc(&p.tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(&S.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+  const uint32_t tO = tmem + 256;
+
+  if (warp == 0) {
+    if (elect_one()) {
+      mbar_arrive_expect_tx(&S.q_full, kHQBytes);
+#pragma unroll
+      for (int a = 0; a < 4; ++a) tma_load_3d(S.Q[a], &p.tmQ, &S.q_full, h * H_D + a * 64, t0, b);
+      for (int j = 0; j < ntile; ++j) {
+        const int s = j % H_STAGES;
+        if (!mbar_wait(&S.kv_empty[s], ((j / H_STAGES) & 1) ^ 1, err)) break;
+        mbar_arrive_expect_tx(&S.kv_full[s], 2 * kHKVBytes);
+        const int kb = kb0 + j * H_BN;
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          tma_load_3d(S.K[s][a], &p.tmK, &S.kv_full[s], g * H_D + a * 64, kb, b);
+          tma_load_3d(S.V[s][a], &p.tmV, &S.kv_full[s], g * H_D + a * 64, kb, b);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    const uint32_t idesc_s = idesc_bf16_f32(AT_BM, H_BN, false);
+    const uint32_t idesc_o = idesc_bf16_f32(AT_BM, H_D, true);  // V MN-major
+    if (elect_one()) {
+      bool ok = mbar_wait(&S.q_full, 0, err);
+      auto issue_s = [&](int j) -> bool {
+        const int s = j % H_STAGES;
+        if (!mbar_wait(&S.kv_full[s], (j / H_STAGES) & 1, err)) return false;
+        if (j >= 2 && !mbar_wait(&S.s_free[j & 1], ((j - 2) >> 1) & 1, err)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < H_D / 16; ++k) {
+          const uint32_t qa = smem_u32(S.Q[k >> 2]) + (k & 3) * 32;
+          const uint32_t ka = smem_u32(S.K[s][k >> 2]) + (k & 3) * 32;
+          umma_f16_ss(tmem + ((j & 1) ? 64u : 0u), smem_desc(qa, 16, 1024, kLayoutSw128),
+                      smem_desc(ka, 16, 1024, kLayoutSw128), idesc_s, k != 0);
+        }
+        umma_commit(&S.s_full[j & 1]);
+        return true;
+      };
+      auto issue_pv = [&](int j) -> bool {
+        const int s = j % H_STAGES;
+        if (!mbar_wait(&S.p_full[j & 1], (j >> 1) & 1, err)) return false;
+        tc_fence_after();
+        const uint32_t v_base = smem_u32(S.V[s][0]);
+        const uint32_t atom = (uint32_t)(H_BN * 64 * 2);  // bytes between 64-wide atoms along N
+#pragma unroll
+        for (int k = 0; k < H_BN / 16; ++k) {
+          const uint32_t a_addr = smem_u32(S.P[j & 1]) + k * 32;
+          const uint32_t b_addr = v_base + k * 16 * 128;  // 16 keys x 128 B
+          umma_f16_ss(tO, smem_desc(a_addr, 16, 1024, kLayoutSw128), smem_desc(b_addr, atom, 1024, kLayoutSw128),
+                      idesc_o, (j | k) != 0);
+        }
+        umma_commit(&S.kv_empty[s]);
+        umma_commit(&S.pv_done[j & 1]);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int j = 0; ok && j < ntile; ++j) {
+        if (j + 1 < ntile) ok = issue_s(j + 1);
+        if (ok) ok = issue_pv(j);
+      }
+    }
+  } else {
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;
+    const int tq = t0 + r;
+    const int t = tk0 + r;
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
+      const bool w = mbar_wait(bar, par, err);
+      return __all_sync(0xffffffffu, w);
+    };
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < ntile; ++j) {
+      const int kb = kb0 + j * H_BN;
+      const uint32_t tSj = tmem + ((j & 1) ? 64u : 0u);
+      if (!wait_all(&S.s_full[j & 1], (j >> 1) & 1)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sr[64];
+      tmem_ld32(tSj + lane_off, sr);
+      tmem_ld32(tSj + lane_off + 32, sr + 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.s_free[j & 1]);
+      const bool edge = (kb + H_BN - 1 > tk0) || (kb < tk0 + AT_BM - p.window);
+      if (edge) {
+        const int hi = tq < p.L ? t - kb : -1;
+        const int lo_i = t - p.window - kb;
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+          if (i > hi || i <= lo_i) sr[i] = __float_as_uint(-INFINITY);
+      }
+      float m8[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 64; i += 2)
+        m8[(i >> 1) & 7] = fmax3(m8[(i >> 1) & 7], __uint_as_float(sr[i]), __uint_as_float(sr[i + 1]));
+      const float mraw = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      const float mt = mraw * p.scale_log2;
+      const bool need = mt > m_run + kRescaleThresh;
+      float alpha = 1.f;
+      if (need) {
+        if (m_run != -INFINITY) alpha = exp2f(m_run - mt);
+        l_run *= alpha;
+        m_run = mt;
+      }
+      if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        if (!wait_all(&S.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < H_D / 32; ++c) {
+          uint32_t orr[32];
+          tmem_ld32(tO + lane_off + c * 32, orr);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
+          tmem_st16(tO + lane_off + c * 32, orr);
+          tmem_st16(tO + lane_off + c * 32 + 16, orr + 16);
+        }
+        tmem_wait_st();
+      }
+      const float msub = m_run == -INFINITY ? 0.f : m_run;
+      if (j >= 2 && !wait_all(&S.pv_done[j & 1], ((j - 2) >> 1) & 1)) { ok = false; break; }
+      const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nm2 = make_float2(-msub, -msub);
+      float2 ls2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      unsigned char* prow = reinterpret_cast<unsigned char*>(S.P[j & 1]) + r * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        float e[8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int i = c * 8 + 2 * q;
+          const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), sc2, nm2);
+          if (q == 0) {
+            const float2 y = exp2_poly2(x);
+            e[0] = y.x;
+            e[1] = y.y;
+          } else {
+            e[2 * q] = ex2_approx(x.x);
+            e[2 * q + 1] = ex2_approx(x.y);
+          }
+          ls2[q] = __fadd2_rn(ls2[q], make_float2(e[2 * q], e[2 * q + 1]));
+        }
+        uint4 v4 = make_uint4(pack_bf16(e[0], e[1]), pack_bf16(e[2], e[3]), pack_bf16(e[4], e[5]),
+                              pack_bf16(e[6], e[7]));
+        *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = v4;
+      }
+      l_run += ((ls2[0].x + ls2[0].y) + (ls2[1].x + ls2[1].y)) + ((ls2[2].x + ls2[2].y) + (ls2[3].x + ls2[3].y));
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.p_full[j & 1]);
+    }
+    if (ok && wait_all(&S.pv_done[(ntile - 1) & 1], ((ntile - 1) >> 1) & 1)) {
+      tc_fence_after();
+      const bool store = tq < p.L && l_run > 0.f;
+      const float inv = store ? 1.f / l_run : 0.f;
+      bf16* op = p.o + ((int64_t)b * p.L + tq) * p.ld_o + (int64_t)h * H_D;
+#pragma unroll
+      for (int c = 0; c < H_D / 32; ++c) {
+        uint32_t orr[32];
+        tmem_ld32(tO + lane_off + c * 32, orr);
+        tmem_wait_ld();
+        if (store) {
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8) {
+            float f[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) f[q] = __uint_as_float(orr[q8 * 8 + q]) * inv;
+            store8(op + c * 32 + q8 * 8, f);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Two query heads per CTA (same kv head): two softmax warpgroups ping-pong on
 // the exp/FMA pipes while sharing every K/V tile.
 //   warp 0      TMA: Q of both heads, then K_j/V_j (3 stages)
@@ -606,17 +857,18 @@ __global__ void __launch_bounds__(A2_THREADS, 1) swa_tc2_kernel(const __grid_con
   }
 }
 
-bool make_head_map(CUtensorMap* m, const void* base, int64_t ld, int H, int L, int B) {
-  uint64_t dims[3] = {(uint64_t)H * AT_D, (uint64_t)L, (uint64_t)B};
+// [B, L, H * d] rows of stride ld; boxes of 64 columns x `rows` rows (128B swizzle)
+bool make_head_map(CUtensorMap* m, const void* base, int64_t ld, int H, int d, int L, int B, int rows) {
+  uint64_t dims[3] = {(uint64_t)H * d, (uint64_t)L, (uint64_t)B};
   uint64_t strides[2] = {(uint64_t)ld, (uint64_t)ld * (uint64_t)L};
-  uint32_t box[3] = {AT_D, 128, 1};
+  uint32_t box[3] = {64, (uint32_t)rows, 1};
   return make_tmap(m, base, SAMBA_BF16, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 }  // namespace
 
 bool swa_tc_supported(const SwaArgs& a) {
-  if (a.dtype != SAMBA_BF16 || a.d != AT_D) return false;
+  if (a.dtype != SAMBA_BF16 || (a.d != AT_D && a.d != H_D)) return false;
   if (a.ld_q % 8 || a.ld_k % 8 || a.ld_v % 8 || a.ld_o % 8) return false;
   if (!aligned16(a.q) || !aligned16(a.k) || !aligned16(a.v) || !aligned16(a.o)) return false;
   if (getenv("SAMBA_SWA_KERNEL") && getenv("SAMBA_SWA_KERNEL")[0] == 's') return false;
@@ -627,8 +879,10 @@ samba_status launch_swa_tc(const SwaArgs& a, cudaStream_t st) {
   AtParams p;
   memset(&p, 0, sizeof(p));
   const int Lk = a.L + a.qoff;
-  if (!make_head_map(&p.tmQ, a.q, a.ld_q, a.Hq, a.L, a.B) || !make_head_map(&p.tmK, a.k, a.ld_k, a.Hkv, Lk, a.B) ||
-      !make_head_map(&p.tmV, a.v, a.ld_v, a.Hkv, Lk, a.B))
+  const int kv_rows = a.d == H_D ? H_BN : AT_BN;
+  if (!make_head_map(&p.tmQ, a.q, a.ld_q, a.Hq, a.d, a.L, a.B, AT_BM) ||
+      !make_head_map(&p.tmK, a.k, a.ld_k, a.Hkv, a.d, Lk, a.B, kv_rows) ||
+      !make_head_map(&p.tmV, a.v, a.ld_v, a.Hkv, a.d, Lk, a.B, kv_rows))
     return SAMBA_ERR_CUDA;
   p.o = (bf16*)a.o;
   p.ld_o = a.ld_o;
@@ -640,6 +894,14 @@ samba_status launch_swa_tc(const SwaArgs& a, cudaStream_t st) {
   p.Hkv = a.Hkv;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   const int grp = a.Hq / a.Hkv;
+  if (a.d == H_D) {
+    const size_t smem = sizeof(AtHSmem) + 1024;
+    if (!ensure_smem_attr(swa_tc256_kernel, smem)) return SAMBA_ERR_CUDA;
+    dim3 grid((a.L + AT_BM - 1) / AT_BM, a.Hq, a.B);
+    swa_tc256_kernel<<<grid, AT_THREADS, smem, st>>>(p, device_error_word());
+    SAMBA_CHECK_LAUNCH();
+    return SAMBA_OK;
+  }
   if (grp % 2 == 0 && !(getenv("SAMBA_SWA_KERNEL") && getenv("SAMBA_SWA_KERNEL")[0] == '1')) {
     // share of the exponentials on the FMA pipe: SAMBA_SWA_POLY = 0..3 pairs of 4 (default 1)
     const char* pe = getenv("SAMBA_SWA_POLY");

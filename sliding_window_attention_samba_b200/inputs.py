@@ -169,6 +169,11 @@ TINY = BlockShape(d_model=64, d_inner=128, d_state=16, d_conv=4, dt_rank=4, n_q=
 WIDE = BlockShape(d_model=2048, d_inner=4096, d_state=16, d_conv=4, dt_rank=128, n_q=32, n_kv=4,
                   head_dim=64, window=2048, d_ff=8192, dtype="bf16")
 
+# the 3.8B model's widths (d_model 2816, MLP 9984, 11 query heads over 1 kv
+# head, hence head_dim 256; d_inner = 2 d_model, dt_rank = d_model / 16)
+WIDE38 = BlockShape(d_model=2816, d_inner=5632, d_state=16, d_conv=4, dt_rank=176, n_q=11, n_kv=1,
+                    head_dim=256, window=2048, d_ff=9984, dtype="bf16")
+
 # name -> (shape, batch, seq_len, n_blocks, seed)
 WORKLOADS = {
     "tiny_f32_L256": (TINY, 1, 256, 1, 0),
@@ -176,6 +181,7 @@ WORKLOADS = {
     "prefill_bf16_L131072_x4": (WIDE, 1, 131072, 4, 2),
     "decode_bf16_B32": (WIDE, 32, 4096, 1, 4),
     "chunked_prefill_bf16_L1048576": (WIDE, 1, 1048576, 1, 5),
+    "block38_bf16_L131072": (WIDE38, 1, 131072, 1, 6),
 }
 # chunk length of the chunked prefill (the blog page's "Chunked Prefilling for
 # 1M-Token Sequences": chunks of 32,768 tokens)
