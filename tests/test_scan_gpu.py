@@ -116,3 +116,12 @@ def test_scan_batch_rows_independent_bit_exact(L):
     one = {k: (v[1:2] if (v is not None and v.ndim == 3) else v) for k, v in r.items()}
     y1, h1 = run_scan(L, one, "bf16")
     assert np.array_equal(y3[1:2], y1) and np.array_equal(h3[1:2], h1)
+
+
+@pytest.mark.parametrize("Ln", [31, 32, 33, 64, 65, 96, 130, 4097])
+def test_scan_ragged_lengths_bf16(L, Ln):
+    """Lengths around the 64-token chunk and the 8-token warp sub-chunks."""
+    r = I.scan_inputs(8, 1, Ln, 64, 16, "bf16", with_h0=True)
+    y, hT = run_scan(L, r, "bf16", h0=r["h0"])
+    yo, ho = oracle_scan(r, h0=r["h0"])
+    assert rel_err(y, yo) <= TOL["bf16"] and rel_err(hT, ho) <= TOL["bf16"]
