@@ -168,7 +168,8 @@ samba_status simt_dispatch(const GemmArgs& a, cudaStream_t st) {
 // tcgen05 kernel
 // ===========================================================================
 constexpr int TC_BM = 128, TC_BK = 64, TC_STAGES = 4, TC_MAXN = 256;
-constexpr int TC_EPI_WARPS = 8;  // two per TMEM lane quadrant, each taking half of the tile's columns
+constexpr int TC_EPI_PARTS = 2;                  // epilogue warps per TMEM lane quadrant (column parts)
+constexpr int TC_EPI_WARPS = 4 * TC_EPI_PARTS;
 constexpr int TC_THREADS = 64 + 32 * TC_EPI_WARPS;
 constexpr uint32_t TC_A_BYTES = TC_BM * TC_BK * 2;
 
@@ -202,18 +203,17 @@ __device__ __forceinline__ void tc_tile_coords(const TcParams& p, int tile, int&
   nt = g * p.group_n + w % p.group_n;
 }
 
-// Columns [c_lo, c_hi) of one 32-column-chunk split: half 0 takes the first
-// ceil(n/2) of n units, half 1 the rest.
-__device__ __forceinline__ void half_range(int n, int half, int& lo, int& hi) {
-  const int split = (n + 1) / 2;
-  lo = half ? split : 0;
-  hi = half ? n : split;
+// Units [lo, hi) of part `part` when n units (32-column chunks; 64-column
+// RoPE units) are split over TC_EPI_PARTS warps of one lane quadrant.
+__device__ __forceinline__ void part_range(int n, int part, int& lo, int& hi) {
+  lo = (n * part) / TC_EPI_PARTS;
+  hi = (n * (part + 1)) / TC_EPI_PARTS;
 }
 
-// One epilogue warp's share of a tile: TMEM lane quadrant = 32 rows, and half
-// `half` of the tile's column units (32-column chunks; 64-column heads for RoPE).
+// One epilogue warp's share of a tile: TMEM lane quadrant = 32 rows, and part
+// `part` of the tile's column units (32-column chunks; 64-column RoPE units).
 template <int EPI>
-__device__ __forceinline__ void tc_epilogue_tile(const TcParams& p, uint32_t tbase, int64_t row, int nt, int half) {
+__device__ __forceinline__ void tc_epilogue_tile(const TcParams& p, uint32_t tbase, int64_t row, int nt, int part) {
   const GemmArgs& a = p.a;
   const bool in_range = row < a.M;
   const int col0 = nt * p.bn;
@@ -221,7 +221,7 @@ __device__ __forceinline__ void tc_epilogue_tile(const TcParams& p, uint32_t tba
   uint32_t r[32], r2[32];
   int u_lo, u_hi;
   if (EPI == kEpiSwiglu) {
-    half_range(p.bn / 32, half, u_lo, u_hi);
+    part_range(p.bn / 32, part, u_lo, u_hi);
     for (int cc = u_lo * 32; cc < u_hi * 32; cc += 32) {
       tmem_ld32(tbase + cc, r);
       tmem_ld32(tbase + p.bn + cc, r2);
@@ -247,7 +247,7 @@ __device__ __forceinline__ void tc_epilogue_tile(const TcParams& p, uint32_t tba
     const int hd = a.head_dim, hd2 = hd / 2;
     const int64_t pos = in_range ? rope_position(a, row) : 0;
     const int nunits = p.bn / 64;  // (head, 32-pair chunk) units
-    half_range(nunits, half, u_lo, u_hi);
+    part_range(nunits, part, u_lo, u_hi);
     for (int u = u_lo; u < u_hi; ++u) {
       const int hh = (u * 64) / hd;         // head within the tile
       const int j0 = (u * 32) % hd2;        // first pair index of this unit
@@ -276,7 +276,7 @@ __device__ __forceinline__ void tc_epilogue_tile(const TcParams& p, uint32_t tba
   }
   // 32-column chunks; a tile width of 16 mod 32 ends in a 16-column chunk (the
   // TMEM columns past it are read but not stored)
-  half_range((p.bn + 31) / 32, half, u_lo, u_hi);
+  part_range((p.bn + 31) / 32, part, u_lo, u_hi);
   for (int cc = u_lo * 32; cc < u_hi * 32; cc += 32) {
     tmem_ld32(tbase + cc, r);
     tmem_wait_ld();
@@ -410,9 +410,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_con
       }
     }
   } else {
-    // ---------------- epilogue warps 2..9 -> TMEM lane quadrant warp % 4, column half (warp - 2) / 4
+    // ---------------- epilogue warps 2.. -> TMEM lane quadrant warp % 4, column part (warp - 2) / 4
     const int q = warp & 3;
-    const int half = (warp - 2) >> 2;
+    const int part = (warp - 2) >> 2;
     int tc = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tc) {
       int mt, nt;
@@ -425,7 +425,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_con
       tc_fence_after();
       const uint32_t tbase = tmem + acc * TC_MAXN + ((uint32_t)(q * 32) << 16);
       const int64_t row = (int64_t)mt * TC_BM + q * 32 + lane;
-      tc_epilogue_tile<EPI>(p, tbase, row, nt, half);
+      tc_epilogue_tile<EPI>(p, tbase, row, nt, part);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.tempty[acc]);
