@@ -126,22 +126,33 @@ __global__ void conv_silu_kernel(const T* __restrict__ x, int64_t ld_x, const fl
     else before(t, hist[j]);
   }
   const int tend = min(t0 + kConvRun, L);
-  for (int t = t0; t < tend; ++t) {
-    load8(xb + (size_t)t * ld_x, hist[K - 1]);
-    float o[8];
+  // kConvAhead tokens' loads in flight at a time, then their outputs
+  constexpr int kConvAhead = 4;
+  for (int tb = t0; tb < tend; tb += kConvAhead) {
+    float xr[kConvAhead][8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float acc = bb[i];
+    for (int k = 0; k < kConvAhead; ++k)
+      if (tb + k < tend) load8(xb + (size_t)(tb + k) * ld_x, xr[k]);
 #pragma unroll
-      for (int j = 0; j < K; ++j) acc = fmaf(wr[i][j], hist[j][i], acc);
-      if constexpr (sizeof(T) == 4) o[i] = acc * sigmoid_acc(acc);
-      else o[i] = acc * sigmoid_fast(acc);
+    for (int k = 0; k < kConvAhead; ++k) {
+      if (tb + k >= tend) break;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) hist[K - 1][i] = xr[k][i];
+      float o[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float acc = bb[i];
+#pragma unroll
+        for (int j = 0; j < K; ++j) acc = fmaf(wr[i][j], hist[j][i], acc);
+        if constexpr (sizeof(T) == 4) o[i] = acc * sigmoid_acc(acc);
+        else o[i] = acc * sigmoid_fast(acc);
+      }
+      store8(u + ((size_t)b * L + tb + k) * D + c0, o);
+#pragma unroll
+      for (int j = 0; j < K - 1; ++j)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) hist[j][i] = hist[j + 1][i];
     }
-    store8(u + ((size_t)b * L + t) * D + c0, o);
-#pragma unroll
-    for (int j = 0; j < K - 1; ++j)
-#pragma unroll
-      for (int i = 0; i < 8; ++i) hist[j][i] = hist[j + 1][i];
   }
   // conv state: the last K-1 inputs of the sequence, oldest first, [B, D, K-1]
   if (state && t0 <= L - 1 && L - 1 < t0 + kConvRun) {
