@@ -168,9 +168,15 @@ samba_status simt_dispatch(const GemmArgs& a, cudaStream_t st) {
 // tcgen05 kernel
 // ===========================================================================
 constexpr int TC_BM = 128, TC_BK = 64, TC_STAGES = 4, TC_MAXN = 256;
-constexpr int TC_EPI_PARTS = 2;                  // epilogue warps per TMEM lane quadrant (column parts)
-constexpr int TC_EPI_WARPS = 4 * TC_EPI_PARTS;
-constexpr int TC_THREADS = 64 + 32 * TC_EPI_WARPS;
+// Epilogue warps per TMEM lane quadrant (column parts).  Two keep up with the
+// mainloop of every projection with K >= 2048; the dt projection (K = 128,
+// softplus) has almost no mainloop, so its epilogue sets the pace and gets four.
+template <int EPI>
+struct TcEpi {
+  static constexpr int parts = EPI == kEpiSoftplus ? 4 : 2;
+  static constexpr int warps = 4 * parts;
+  static constexpr int threads = 64 + 32 * warps;
+};
 constexpr uint32_t TC_A_BYTES = TC_BM * TC_BK * 2;
 
 struct TcSmem {
@@ -204,10 +210,10 @@ __device__ __forceinline__ void tc_tile_coords(const TcParams& p, int tile, int&
 }
 
 // Units [lo, hi) of part `part` when n units (32-column chunks; 64-column
-// RoPE units) are split over TC_EPI_PARTS warps of one lane quadrant.
-__device__ __forceinline__ void part_range(int n, int part, int& lo, int& hi) {
-  lo = (n * part) / TC_EPI_PARTS;
-  hi = (n * (part + 1)) / TC_EPI_PARTS;
+// RoPE units) are split over `parts` warps of one lane quadrant.
+__device__ __forceinline__ void part_range(int n, int part, int parts, int& lo, int& hi) {
+  lo = (n * part) / parts;
+  hi = (n * (part + 1)) / parts;
 }
 
 // One epilogue warp's share of a tile: TMEM lane quadrant = 32 rows, and part
@@ -221,7 +227,7 @@ __device__ __forceinline__ void tc_epilogue_tile(const TcParams& p, uint32_t tba
   uint32_t r[32], r2[32];
   int u_lo, u_hi;
   if (EPI == kEpiSwiglu) {
-    part_range(p.bn / 32, part, u_lo, u_hi);
+    part_range(p.bn / 32, part, TcEpi<EPI>::parts, u_lo, u_hi);
     for (int cc = u_lo * 32; cc < u_hi * 32; cc += 32) {
       tmem_ld32(tbase + cc, r);
       tmem_ld32(tbase + p.bn + cc, r2);
@@ -247,7 +253,7 @@ __device__ __forceinline__ void tc_epilogue_tile(const TcParams& p, uint32_t tba
     const int hd = a.head_dim, hd2 = hd / 2;
     const int64_t pos = in_range ? rope_position(a, row) : 0;
     const int nunits = p.bn / 64;  // (head, 32-pair chunk) units
-    part_range(nunits, part, u_lo, u_hi);
+    part_range(nunits, part, TcEpi<EPI>::parts, u_lo, u_hi);
     for (int u = u_lo; u < u_hi; ++u) {
       const int hh = (u * 64) / hd;         // head within the tile
       const int j0 = (u * 32) % hd2;        // first pair index of this unit
@@ -276,7 +282,7 @@ __device__ __forceinline__ void tc_epilogue_tile(const TcParams& p, uint32_t tba
   }
   // 32-column chunks; a tile width of 16 mod 32 ends in a 16-column chunk (the
   // TMEM columns past it are read but not stored)
-  part_range((p.bn + 31) / 32, part, u_lo, u_hi);
+  part_range((p.bn + 31) / 32, part, TcEpi<EPI>::parts, u_lo, u_hi);
   for (int cc = u_lo * 32; cc < u_hi * 32; cc += 32) {
     tmem_ld32(tbase + cc, r);
     tmem_wait_ld();
@@ -322,7 +328,7 @@ __device__ __forceinline__ void tc_epilogue_tile(const TcParams& p, uint32_t tba
 }
 
 template <int EPI>
-__global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_constant__ TcParams p, int* err) {
+__global__ void __launch_bounds__(TcEpi<EPI>::threads, 1) gemm_tc_kernel(const __grid_constant__ TcParams p, int* err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   TcSmem& S = *reinterpret_cast<TcSmem*>(smem_raw + smem_align_pad(smem_raw, 1024));
   const int warp = warp_id_sync();
@@ -336,7 +342,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_con
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.tfull[i], 1);
-      mbar_init(&S.tempty[i], TC_EPI_WARPS);
+      mbar_init(&S.tempty[i], TcEpi<EPI>::warps);
     }
     fence_mbar_init();
     tma_prefetch_desc(&p.tmA);
@@ -467,7 +473,7 @@ samba_status tc_launch(TcParams& p, cudaStream_t st) {
     return SAMBA_ERR_CUDA;
   const int ntiles = p.m_tiles * p.n_tiles;
   const int grid = ntiles < num_sms() ? ntiles : num_sms();
-  kern<<<grid, TC_THREADS, smem, st>>>(p, device_error_word());
+  kern<<<grid, TcEpi<EPI>::threads, smem, st>>>(p, device_error_word());
   SAMBA_CHECK_LAUNCH();
   return SAMBA_OK;
 }
