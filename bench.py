@@ -405,7 +405,7 @@ def kernel_report(kt, s, T, Bn, Ln, peaks):
     # Dominant kernel: the SwiGLU up-projection (gemm_tc_kernel<2>, ~32% of the
     # step in the launch list).  Timed alone by the attribution pass, so against
     # the burst peak.  DRAM traffic per launch from an ncu capture of this kernel
-    # at M = 16384 (dram__bytes_read.sum 209.8 MB, dram__bytes_write.sum 236.0 MB),
+    # at M = 16384 (dram__bytes_read.sum 207.1 MB, dram__bytes_write.sum 236.8 MB),
     # scaled to this M: the activation reads and the output writes grow with M,
     # the 67 MB of weights are read once whatever M is.
     name = "mlp1_up"
@@ -413,7 +413,7 @@ def kernel_report(kt, s, T, Bn, Ln, peaks):
     w_bytes = 2 * s.d_ff * s.d_model * 2
     scale = T / 16384
     # measured at the 2048-wide shapes only
-    traffic = (209.8e6 - w_bytes) * scale + w_bytes + 236.0e6 * scale if s == I.WIDE else None
+    traffic = (207.1e6 - w_bytes) * scale + w_bytes + 236.8e6 * scale if s == I.WIDE else None
     roof = {"bound": "tensor", "achieved": round(up / kt[name] / 1e12, 2), "peak": tf_burst, "unit": "TFLOP/s",
             "frac": round(up / kt[name] / 1e12 / tf_burst, 4), "traffic": round(traffic) if traffic else None,
             "algorithmic_bytes": T * s.d_model * 2 + w_bytes + T * s.d_ff * 2,
