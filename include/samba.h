@@ -25,6 +25,11 @@
  *     transpose of the pages' X W notation.
  *   - No exception, C++ type or torch type crosses this boundary; the library is
  *     stateless apart from the device error word and is reentrant.
+ *   - Size limits of the launch grids: a batch B (and a head count) of at most
+ *     65535, and at most 65535 * 32 = 2,097,120 tokens per sequence in one call
+ *     of an entry point that runs the causal conv (longer prompts go through
+ *     samba_block_fwd_chunk).  Larger shapes return SAMBA_ERR_UNSUPPORTED before
+ *     anything is launched.
  */
 #ifndef SAMBA_H_
 #define SAMBA_H_

@@ -653,6 +653,7 @@ static samba_status block_forward(const samba_block_config* cfg, const samba_blo
   const bool resume = pos0 > 0;
   if (resume && !stt) return SAMBA_ERR_INVALID_ARG;
   if (pos0 + (int64_t)L > (int64_t(1) << 30)) return SAMBA_ERR_UNSUPPORTED;
+  if (B > kMaxGridYZ || L > kMaxConvTokens) return SAMBA_ERR_UNSUPPORTED;
   const samba_block_config& c = *cfg;
   const int64_t T = (int64_t)B * L;
   const BlockPlan P = plan_block(c, T, resume ? B : 0);
@@ -770,6 +771,7 @@ samba_status samba_model_prefill(const samba_model* m, const int32_t* ids, void*
   if (!m) return SAMBA_ERR_INVALID_ARG;
   TRY(validate_cfg(&m->cfg));
   if (!ids || !logits || B < 1 || L < 1 || m->n_layers < 0 || m->vocab < 1) return SAMBA_ERR_INVALID_ARG;
+  if (B > kMaxGridYZ || L > kMaxConvTokens) return SAMBA_ERR_UNSUPPORTED;
   if (m->n_layers > 0 && (!m->kinds || !m->layers)) return SAMBA_ERR_INVALID_ARG;
   if (!m->embedding || !m->final_norm || !m->lm_head) return SAMBA_ERR_INVALID_ARG;
   for (int i = 0; i < m->n_layers; ++i) TRY(validate_layer(m->kinds[i], m->layers[i]));
@@ -843,6 +845,7 @@ samba_status samba_model_step(const samba_model* m, const int32_t* ids_t, void* 
   if (!m) return SAMBA_ERR_INVALID_ARG;
   TRY(validate_cfg(&m->cfg));
   if (!ids_t || !logits || !pos || B < 1 || m->n_layers < 0 || m->vocab < 1) return SAMBA_ERR_INVALID_ARG;
+  if (B > kMaxGridYZ) return SAMBA_ERR_UNSUPPORTED;
   if (m->n_layers > 0 && (!m->kinds || !m->layers || !states)) return SAMBA_ERR_INVALID_ARG;
   if (!m->embedding || !m->final_norm || !m->lm_head) return SAMBA_ERR_INVALID_ARG;
   for (int i = 0; i < m->n_layers; ++i) {
@@ -896,6 +899,7 @@ samba_status samba_step(const samba_block_config* cfg, const samba_block_weights
   TRY(validate_cfg(cfg));
   TRY(validate_weights(w));
   if (!x_t || !y_t || !stt || B < 1 || x_t == y_t) return SAMBA_ERR_INVALID_ARG;
+  if (B > kMaxGridYZ) return SAMBA_ERR_UNSUPPORTED;
   if (!stt->ssm || !stt->conv || !stt->k_ring || !stt->v_ring || !stt->pos) return SAMBA_ERR_INVALID_ARG;
   const samba_block_config& c = *cfg;
   const BlockPlan P = plan_block(c, B);

@@ -559,6 +559,7 @@ __global__ void kv_window_gather_kernel(const char* __restrict__ qkv, int64_t ld
 
 samba_status launch_conv_step(const void* hz, int64_t ld_hz, const float* w, const float* bias, void* state, void* u,
                               int B, int D, int k, samba_dtype dt, cudaStream_t st) {
+  if (B > kMaxGridYZ || (int64_t)B * D > INT32_MAX) return SAMBA_ERR_UNSUPPORTED;
   if (k < 2 || k > 8) return SAMBA_ERR_UNSUPPORTED;
   const int n = B * D;
   cudaError_t e;
@@ -574,6 +575,7 @@ samba_status launch_conv_step(const void* hz, int64_t ld_hz, const float* w, con
 samba_status launch_scan_step(const void* u, const void* dlt, const void* z, int64_t ld_z, const void* xdbl,
                               int64_t ld_x, int r_off, const float* A_log, const float* Dskip, float* ssm, void* y,
                               int B, int D, samba_dtype dt, cudaStream_t st) {
+  if (B > kMaxGridYZ || (int64_t)B * D > INT32_MAX) return SAMBA_ERR_UNSUPPORTED;
   const int n = B * D;
   cudaError_t e;
   SAMBA_DT_DISPATCH(dt,
@@ -607,6 +609,7 @@ size_t attn_decode_workspace_bytes(int B, int Hkv, int window) {
 samba_status launch_attn_decode(const void* qkv, int64_t ld, const int64_t* pos, const void* k_ring,
                                 const void* v_ring, void* o, int B, int Hq, int Hkv, int hd, int window, float scale,
                                 samba_dtype dt, cudaStream_t st, void* ws, size_t ws_bytes) {
+  if (B > kMaxGridYZ) return SAMBA_ERR_UNSUPPORTED;
   if (hd > 128) return SAMBA_ERR_UNSUPPORTED;
   if (dt == SAMBA_BF16 && hd == kHd && Hq / Hkv <= 8 && window > kSplit * kSliceMax && ld % 8 == 0) {
     const int nsplit = (window + kSliceMax - 1) / kSliceMax;
@@ -673,6 +676,7 @@ samba_status launch_pos_update(int64_t* pos, int B, int64_t value, bool set, cud
 
 samba_status launch_ring_fill(const void* qkv, int64_t ld, int k_off, int v_off, void* k_ring, void* v_ring, int B,
                               int L, int64_t pos0, int window, int kvw, samba_dtype dt, cudaStream_t st) {
+  if (B > kMaxGridYZ) return SAMBA_ERR_UNSUPPORTED;
   const int n = L < window ? L : window;
   if (n == 0) return SAMBA_OK;
   dim3 grid(n, B);
@@ -689,6 +693,7 @@ samba_status launch_ring_fill(const void* qkv, int64_t ld, int k_off, int v_off,
 samba_status launch_kv_window_gather(const void* qkv, int64_t ld, int k_off, int v_off, const void* k_ring,
                                      const void* v_ring, void* kx, void* vx, int B, int L, int64_t pos0, int h,
                                      int window, int kvw, samba_dtype dt, cudaStream_t st) {
+  if (B > kMaxGridYZ) return SAMBA_ERR_UNSUPPORTED;
   const size_t es = dtype_size(dt);
   const int vec = (int)(kvw * es / 16);  // 16-byte pieces per row
   if ((kvw * es) % 16 || (ld * es) % 16 || (k_off * es) % 16 || (v_off * es) % 16 || h < 0 || h > pos0 ||

@@ -92,7 +92,7 @@ samba_status launch_embedding(const int32_t* ids, const void* table, void* out, 
 // last k-1 inputs in registers (each input is read once from HBM per run plus
 // k-1 halo rows).  Also writes the conv state (last k-1 inputs) when asked.
 // ===========================================================================
-constexpr int kConvRun = 32;
+constexpr int kConvRun = kConvRunTokens;
 constexpr int kMaxK = 8;
 
 template <typename T, int K>
@@ -176,6 +176,7 @@ __global__ void conv_state_zero_kernel(T* state, size_t n) {
 template <typename T, int K>
 samba_status launch_conv_k(const ConvArgs& a, cudaStream_t st) {
   const int groups = a.D / 8;
+  if (a.B > kMaxGridYZ || a.L > kMaxConvTokens) return SAMBA_ERR_UNSUPPORTED;
   dim3 block(128);
   dim3 grid((groups + 127) / 128, (a.L + kConvRun - 1) / kConvRun, a.B);
   conv_silu_kernel<T, K><<<grid, block, 0, st>>>((const T*)a.x, a.ld_x, a.w, a.bias, (T*)a.u, (T*)a.state,

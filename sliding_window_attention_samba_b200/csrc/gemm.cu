@@ -151,6 +151,7 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(const GemmArgs a) {
 
 template <typename T>
 samba_status simt_dispatch(const GemmArgs& a, cudaStream_t st) {
+  if ((a.M + SB_M - 1) / SB_M > kMaxGridYZ) return SAMBA_ERR_UNSUPPORTED;
   dim3 grid((a.N + SB_N - 1) / SB_N, (unsigned)((a.M + SB_M - 1) / SB_M));
   switch (a.epi) {
     case kEpiNone: gemm_simt_kernel<T, kEpiNone><<<grid, 256, 0, st>>>(a); break;

@@ -8,6 +8,12 @@
 
 namespace samba {
 
+// Grid limits the launchers check before launching: batch rows and heads go to
+// grid y/z (at most 65535 each); the conv kernel puts 32-token runs on grid y.
+constexpr int kMaxGridYZ = 65535;
+constexpr int kConvRunTokens = 32;
+constexpr int64_t kMaxConvTokens = (int64_t)kMaxGridYZ * kConvRunTokens;
+
 // ---------------- selective scan ----------------
 struct ScanArgs {
   const void* u = nullptr;

@@ -315,7 +315,7 @@ samba_status launch_dispatch(const ScanArgs& a, cudaStream_t st) {
 samba_status validate_scan(const ScanArgs& a) {
   if (!a.u || !a.dt || !a.A_log || !a.Bm || !a.Cm || !a.y) return SAMBA_ERR_INVALID_ARG;
   if (a.B < 1 || a.L < 0 || a.D < 1 || a.N < 1) return SAMBA_ERR_INVALID_ARG;
-  if (a.N != kN || a.D % kCh != 0) return SAMBA_ERR_UNSUPPORTED;
+  if (a.N != kN || a.D % kCh != 0 || a.B > kMaxGridYZ) return SAMBA_ERR_UNSUPPORTED;
   const size_t es = dtype_size(a.dtype);
   const void* ptrs[] = {a.u, a.dt, a.Bm, a.Cm, a.y, a.z};
   for (const void* p : ptrs)

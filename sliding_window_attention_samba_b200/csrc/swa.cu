@@ -119,6 +119,7 @@ samba_status launch_swa(const SwaArgs& a, cudaStream_t st) {
   if (!a.q || !a.k || !a.v || !a.o || a.B < 1 || a.L < 0 || a.Hq < 1 || a.Hkv < 1 || a.window < 1 || a.qoff < 0)
     return SAMBA_ERR_INVALID_ARG;
   if (a.Hq % a.Hkv) return SAMBA_ERR_INVALID_ARG;
+  if (a.B > kMaxGridYZ || a.Hq > kMaxGridYZ) return SAMBA_ERR_UNSUPPORTED;
   if (a.L == 0) return SAMBA_OK;
   if (swa_tc_supported(a)) return launch_swa_tc(a, st);
   return launch_swa_simt(a, st);

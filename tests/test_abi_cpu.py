@@ -81,3 +81,36 @@ def test_invalid_arguments_rejected_before_launch(lib):
     w = lib.BlockWeights()
     with pytest.raises(lib.SambaError):
         lib.samba_block_fwd(cfg, w, 1 << 20, 2 << 20, None, None, 1, 8, 1 << 22, 1 << 30, 0)
+
+
+def test_grid_limits_rejected_before_launch(lib):
+    """Shapes beyond the launch grids (batch > 65535; more than 65535 conv runs of
+    32 tokens in one call) come back as SAMBA_ERR_UNSUPPORTED from host-side
+    validation, before any CUDA call (none can run on this machine)."""
+    from sliding_window_attention_samba_b200 import inputs as I
+    h = lib.lib_handle()
+    fake = ctypes.c_void_p(1 << 20)
+    big_b = 65536
+    rc = h.samba_selective_scan(fake, fake, None, 1, fake, fake, fake, None, None, None, None, fake,
+                                big_b, 16, 32, 16, 1, None, 0, None)
+    assert rc == lib.SAMBA_ERR_UNSUPPORTED
+    rc = h.samba_swa_fwd(fake, fake, fake, fake, big_b, 16, 4, 4, 64, 8, ctypes.c_float(0.0), 0,
+                         ctypes.c_float(0.0), 1, None, 0, None)
+    assert rc == lib.SAMBA_ERR_UNSUPPORTED
+    cfg = lib.make_config(I.TINY)
+    w = lib.BlockWeights()
+    for i in range(4):
+        w.norm_g[i] = 1 << 20
+    for name, _ in lib.BlockWeights._fields_[1:]:
+        setattr(w, name, 1 << 20)
+    st = lib.make_state(1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20)
+    with pytest.raises(lib.SambaError) as e:
+        lib.samba_step(cfg, w, 1 << 20, 2 << 20, st, big_b, 1 << 22, 1 << 40, 0)
+    assert e.value.code == lib.SAMBA_ERR_UNSUPPORTED
+    with pytest.raises(lib.SambaError) as e:
+        lib.samba_block_fwd(cfg, w, 1 << 20, 2 << 20, None, None, 1, 65535 * 32 + 1, 1 << 22, 1 << 40, 0)
+    assert e.value.code == lib.SAMBA_ERR_UNSUPPORTED
+    # the largest accepted batch still gets as far as the workspace check
+    with pytest.raises(lib.SambaError) as e:
+        lib.samba_step(cfg, w, 1 << 20, 2 << 20, st, 65535, 1 << 22, 16, 0)
+    assert e.value.code == lib.SAMBA_ERR_INVALID_ARG
