@@ -114,3 +114,23 @@ def test_grid_limits_rejected_before_launch(lib):
     with pytest.raises(lib.SambaError) as e:
         lib.samba_step(cfg, w, 1 << 20, 2 << 20, st, 65535, 1 << 22, 16, 0)
     assert e.value.code == lib.SAMBA_ERR_INVALID_ARG
+
+
+def test_plain_c_consumer_builds_and_runs(tmp_path, lib):
+    """The header is valid C99 (no C++ or torch types cross the boundary): a C
+    program compiled with -std=c99 -Wall -Werror links libsamba.so and runs its
+    host-side calls."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    libdir = os.path.dirname(lib.LIB_PATH)
+    exe = str(tmp_path / "consumer")
+    src = os.path.join(ROOT, "tests", "abi_c", "consumer.c")
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"), src,
+                        "-L", libdir, "-lsamba", "-Wl,-rpath," + libdir, "-o", exe], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.startswith("consumer ok")
