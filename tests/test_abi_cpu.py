@@ -134,3 +134,12 @@ def test_plain_c_consumer_builds_and_runs(tmp_path, lib):
     r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0, r.stderr
     assert r.stdout.startswith("consumer ok")
+    # the same header and program as C++ (extern "C" linkage)
+    cxx = shutil.which("g++") or shutil.which("c++")
+    if cxx is not None:
+        exe2 = str(tmp_path / "consumer_cxx")
+        r = subprocess.run([cxx, "-x", "c++", "-std=c++17", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                            src, "-L", libdir, "-lsamba", "-Wl,-rpath," + libdir, "-o", exe2],
+                           capture_output=True, text=True)
+        assert r.returncode == 0, r.stderr
+        assert subprocess.run([exe2], capture_output=True, text=True, timeout=60).returncode == 0
