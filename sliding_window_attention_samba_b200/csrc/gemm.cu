@@ -6,7 +6,8 @@
 // Two kernels:
 //  * gemm_tc: bf16 operands, fp32 accumulation on the 5th-generation tensor
 //    cores.  Persistent, warp specialised (warp 0: TMA producer, warp 1: MMA
-//    issuer + TMEM owner, warps 2-9: epilogue).  A 4-stage ring of 128x64 A and
+//    issuer + TMEM owner, warps 2..: epilogue, two per TMEM lane quadrant, four
+//    for the softplus instance).  A 4-stage ring of 128x64 A and
 //    up to 256x64 B tiles in 128-byte-swizzled shared memory feeds
 //    tcgen05.mma (M=128, N<=256, K=16) issued by one thread into a double
 //    buffered 2x256-column TMEM accumulator, so the epilogue of one tile
