@@ -674,8 +674,9 @@ static samba_status block_forward(const samba_block_config* cfg, const samba_blo
   if (T == 0) {
     if (stt) {
       TRY(launch_pos_update(stt->pos, B, 0, true, st));
-      cudaMemsetAsync(stt->ssm, 0, (size_t)B * Di * N * sizeof(float), st);
-      cudaMemsetAsync(stt->conv, 0, (size_t)B * Di * (c.d_conv - 1) * es, st);
+      if (cudaMemsetAsync(stt->ssm, 0, (size_t)B * Di * N * sizeof(float), st) != cudaSuccess ||
+          cudaMemsetAsync(stt->conv, 0, (size_t)B * Di * (c.d_conv - 1) * es, st) != cudaSuccess)
+        return SAMBA_ERR_CUDA;
     }
     return SAMBA_OK;
   }
