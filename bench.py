@@ -954,7 +954,7 @@ def main():
     shape, Bn, Ln, n_blocks, _ = I.WORKLOADS[workload_of(args)]
     if args.seq_len:
         Ln = args.seq_len
-    cfgd = {"workload": workload_of(args), "model": "samba block stack (random init)", "global_batch": Bn * max(world, 1),
+    cfgd = {"workload": workload_of(args), "weights": "random init", "global_batch": Bn * max(world, 1),
             "seq_len": Ln, "n_blocks": n_blocks, "d_model": shape.d_model, "window": shape.window,
             "parallelism": f"replicas{max(world, 1)}", "l2": "activations per block >> 126 MB L2; no flush needed"}
 
