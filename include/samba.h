@@ -60,6 +60,22 @@ const char* samba_status_string(samba_status s);
 /* Library version string (static). */
 const char* samba_version(void);
 
+/* Measurement hook for benchmarks and profilers (no effect unless installed).
+ * While installed, every launch of a projection with epilogue kind `epi` (the
+ * samba_linear kinds: 0 none, 1 residual, 2 SwiGLU, 3 softplus + bias; 4 the
+ * Q/K/V projection with RoPE inside the block) records start_events[i] on its
+ * stream immediately before the kernel and stop_events[i] immediately after it,
+ * i = 0, 1, ... in launch order; launches past `capacity` are not recorded.
+ * Events are cudaEvent_t created by the caller with timing enabled and must
+ * outlive the hook.  epi < 0 removes the hook (the arrays may then be NULL).
+ * Installing or removing the hook resets the launch count; it is process-wide,
+ * so install it only while one host thread launches.  Returns
+ * SAMBA_ERR_INVALID_ARG for NULL arrays or entries, capacity < 1 or epi > 4. */
+samba_status samba_set_gemm_timing(int epi, void* const* start_events, void* const* stop_events, int capacity);
+
+/* Launches recorded by the hook since it was installed. */
+int samba_gemm_timing_count(void);
+
 /* Synchronises `stream`, returns and clears the device error word of the
  * current device: SAMBA_OK, SAMBA_ERR_TIMEOUT or SAMBA_ERR_DEVICE, or
  * SAMBA_ERR_CUDA if the synchronisation itself failed. */

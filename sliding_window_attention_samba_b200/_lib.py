@@ -87,6 +87,8 @@ def _sig(name, restype, argtypes):
 
 _status_string = _sig("samba_status_string", ctypes.c_char_p, [c_int])
 _version = _sig("samba_version", ctypes.c_char_p, [])
+_set_timing = _sig("samba_set_gemm_timing", c_int, [c_int, c_void_p, c_void_p, c_int])
+_timing_count = _sig("samba_gemm_timing_count", c_int, [])
 _get_error = _sig("samba_get_error", c_int, [c_void_p])
 _scan_ws = _sig("samba_selective_scan_workspace_size", c_size_t, [c_int, c_int, c_int, c_int])
 _scan = _sig("samba_selective_scan", c_int,
@@ -159,6 +161,30 @@ def samba_status_string(code: int) -> str:
 
 def samba_version() -> str:
     return _version().decode()
+
+
+def samba_set_gemm_timing(epi: int, start_events=(), stop_events=()):
+    """Install (epi >= 0) or remove (epi < 0) the projection timing hook.  The
+    events are torch.cuda.Event(enable_timing=True) objects that have been
+    recorded once (so that their CUDA events exist); keep them alive while
+    the hook is installed."""
+    if epi < 0:
+        _check("samba_set_gemm_timing", _set_timing(-1, None, None, 0))
+        return
+    n = len(start_events)
+    if n != len(stop_events) or n == 0:
+        raise ValueError("need equally many start and stop events")
+    hs = [int(e.cuda_event) for e in start_events]
+    he = [int(e.cuda_event) for e in stop_events]
+    if not all(hs) or not all(he):
+        raise ValueError("record every event once before installing the hook")
+    a = (c_void_p * n)(*hs)
+    b = (c_void_p * n)(*he)
+    _check("samba_set_gemm_timing", _set_timing(epi, ctypes.cast(a, c_void_p), ctypes.cast(b, c_void_p), n))
+
+
+def samba_gemm_timing_count() -> int:
+    return _timing_count()
 
 
 def samba_get_error(stream=None) -> int:

@@ -221,6 +221,12 @@ const char* samba_status_string(samba_status s) {
 
 const char* samba_version(void) { return "samba-b200 0.1 (sm_100a)"; }
 
+samba_status samba_set_gemm_timing(int epi, void* const* start_events, void* const* stop_events, int capacity) {
+  return gemm_timing_set(epi, start_events, stop_events, capacity);
+}
+
+int samba_gemm_timing_count(void) { return gemm_timing_count(); }
+
 samba_status samba_get_error(samba_stream stream) {
   if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return SAMBA_ERR_CUDA;
   int* w = device_error_word();

@@ -18,6 +18,10 @@
 //    kernel does not take.
 #include <stdlib.h>
 
+#include <atomic>
+#include <mutex>
+#include <vector>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -555,6 +559,67 @@ static bool force_simt() {
   return e && e[0] == 's';
 }
 
+// ---- measurement hook: CUDA events around the launches of one epilogue kind
+// (no effect, beyond one relaxed atomic load per launch, unless installed)
+namespace {
+std::mutex g_tm_mu;
+std::atomic<int> g_tm_epi{-1};
+std::vector<cudaEvent_t> g_tm_start, g_tm_stop;
+int g_tm_count = 0;
+
+// Records the next start event on `st` and returns its stop event, or nullptr.
+cudaEvent_t timing_begin(int epi, cudaStream_t st) {
+  if (g_tm_epi.load(std::memory_order_relaxed) != epi) return nullptr;
+  cudaEvent_t s0 = nullptr, s1 = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_tm_mu);
+    if (g_tm_epi.load(std::memory_order_relaxed) != epi || g_tm_count >= (int)g_tm_start.size()) return nullptr;
+    s0 = g_tm_start[g_tm_count];
+    s1 = g_tm_stop[g_tm_count];
+    ++g_tm_count;
+  }
+  if (cudaEventRecord(s0, st) != cudaSuccess) {
+    (void)cudaGetLastError();  // a bad event handle must not fail the launch that follows
+    return nullptr;
+  }
+  return s1;
+}
+
+void timing_end(cudaEvent_t s1, cudaStream_t st) {
+  if (s1 && cudaEventRecord(s1, st) != cudaSuccess) (void)cudaGetLastError();
+}
+}  // namespace
+
+samba_status gemm_timing_set(int epi, void* const* start, void* const* stop, int capacity) {
+  std::lock_guard<std::mutex> lk(g_tm_mu);
+  g_tm_epi.store(-1);
+  g_tm_start.clear();
+  g_tm_stop.clear();
+  g_tm_count = 0;
+  if (epi < 0) return SAMBA_OK;
+  if (epi > kEpiRope || !start || !stop || capacity < 1) return SAMBA_ERR_INVALID_ARG;
+  for (int i = 0; i < capacity; ++i)
+    if (!start[i] || !stop[i]) return SAMBA_ERR_INVALID_ARG;
+  for (int i = 0; i < capacity; ++i) {
+    g_tm_start.push_back((cudaEvent_t)start[i]);
+    g_tm_stop.push_back((cudaEvent_t)stop[i]);
+  }
+  g_tm_epi.store(epi);
+  return SAMBA_OK;
+}
+
+int gemm_timing_count() {
+  std::lock_guard<std::mutex> lk(g_tm_mu);
+  return g_tm_count;
+}
+
+static samba_status gemm_dispatch(const GemmArgs& a, cudaStream_t st) {
+  if (!force_simt() && a.M <= 64 && gemm_skinny_supported(a)) return launch_gemm_skinny(a, st);
+  if (!force_simt() && gemm_tc_supported(a)) return launch_gemm_tc(a, st);
+  if (a.epi == kEpiRope && 64 % a.head_dim != 0) return SAMBA_ERR_UNSUPPORTED;
+  return launch_gemm_simt(a, st);
+}
+
 samba_status launch_gemm(const GemmArgs& a, cudaStream_t st) {
   if (!a.A || !a.out || a.M < 0 || a.N <= 0 || a.K <= 0 || a.nseg < 1 || a.nseg > 3) return SAMBA_ERR_INVALID_ARG;
   int nsum = 0;
@@ -568,10 +633,10 @@ samba_status launch_gemm(const GemmArgs& a, cudaStream_t st) {
   if (a.epi == kEpiSoftplus && !a.bias) return SAMBA_ERR_INVALID_ARG;
   if (a.epi == kEpiRope && (!a.rope_tab || a.head_dim <= 0 || a.rope_cols % a.head_dim)) return SAMBA_ERR_INVALID_ARG;
   if (a.M == 0) return SAMBA_OK;
-  if (!force_simt() && a.M <= 64 && gemm_skinny_supported(a)) return launch_gemm_skinny(a, st);
-  if (!force_simt() && gemm_tc_supported(a)) return launch_gemm_tc(a, st);
-  if (a.epi == kEpiRope && 64 % a.head_dim != 0) return SAMBA_ERR_UNSUPPORTED;
-  return launch_gemm_simt(a, st);
+  const cudaEvent_t tstop = timing_begin(a.epi, st);
+  const samba_status r = gemm_dispatch(a, st);
+  timing_end(tstop, st);
+  return r;
 }
 
 }  // namespace samba

@@ -104,6 +104,10 @@ struct GemmArgs {
   bool pdl = false;  // launch as a programmatic dependent of the previous kernel (decode path)
 };
 samba_status launch_gemm(const GemmArgs& a, cudaStream_t st);       // picks the kernel
+// Measurement hook: while installed, launches of epilogue kind `epi` record
+// start[i] / stop[i] on their stream around the kernel (i counts the launches).
+samba_status gemm_timing_set(int epi, void* const* start, void* const* stop, int capacity);
+int gemm_timing_count();
 samba_status launch_gemm_simt(const GemmArgs& a, cudaStream_t st);  // CUDA-core fp32 FMA kernel
 samba_status launch_gemm_tc(const GemmArgs& a, cudaStream_t st);    // tcgen05 kernel (bf16)
 bool gemm_tc_supported(const GemmArgs& a);

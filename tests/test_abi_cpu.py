@@ -143,3 +143,20 @@ def test_plain_c_consumer_builds_and_runs(tmp_path, lib):
                            capture_output=True, text=True)
         assert r.returncode == 0, r.stderr
         assert subprocess.run([exe2], capture_output=True, text=True, timeout=60).returncode == 0
+
+
+def test_gemm_timing_hook_host_side(lib):
+    """The measurement hook validates its arguments and counts nothing until a
+    projection launches (no device call happens in install/remove)."""
+    h = lib.lib_handle()
+    V = ctypes.c_void_p
+    a = (V * 2)(1 << 20, 1 << 21)
+    b = (V * 2)(1 << 22, 1 << 23)
+    assert h.samba_set_gemm_timing(-1, None, None, 0) == 0
+    assert h.samba_set_gemm_timing(2, None, None, 1) == lib.SAMBA_ERR_INVALID_ARG
+    assert h.samba_set_gemm_timing(5, a, b, 2) == lib.SAMBA_ERR_INVALID_ARG
+    assert h.samba_set_gemm_timing(2, a, b, 0) == lib.SAMBA_ERR_INVALID_ARG
+    assert h.samba_set_gemm_timing(2, (V * 2)(1 << 20, None), b, 2) == lib.SAMBA_ERR_INVALID_ARG
+    assert h.samba_set_gemm_timing(2, a, b, 2) == 0
+    assert h.samba_gemm_timing_count() == 0
+    assert h.samba_set_gemm_timing(-1, None, None, 0) == 0
