@@ -11,10 +11,14 @@ ranks (each rank runs its own replica: no data-path collective).
 
 Printed JSON line (rank 0): value (device time, inputs resident in HBM), e2e
 (same metric through the C ABI with pinned host input/output copied inside the
-timed region), roofline of the dominant kernel (from a CUDA-event attribution
-pass over the same kernels), the oracle CPU baseline, clocks sampled during the
-timed region.  `--impl reference` times the fp64 CPU oracle on a bounded sample
-of the same workload instead.
+timed region), roofline of the dominant kernel (CUDA events around its launches
+inside the timed region), per-kernel figures (scan HBM GB/s, SWA and projection
+TF/s) from an attribution pass over the same kernels, the oracle CPU baseline,
+clocks sampled during the timed region; at one GPU also `decode` (batch 32,
+65 536 graph-replayed samba_step calls after a 4096-token prefill, against its
+HBM roofline) and `sweep` (scan and SWA alone at L = 4K .. 1M).  `--impl
+reference` times the fp64 CPU oracle on a bounded sample of the same workload
+instead (the same sample as the line's cpu_baseline).
 """
 from __future__ import annotations
 
@@ -36,7 +40,7 @@ import numpy as np  # noqa: E402
 from sliding_window_attention_samba_b200 import inputs as I  # noqa: E402
 
 WORKLOAD = "prefill_bf16_L131072_x4"
-METRIC = "prefill tokens/s per Samba block at L=128K"
+METRIC = "prefill tokens/s per Samba block at L=128K; scan HBM GB/s & SWA TC util vs peak"
 UNIT = "tokens/s"
 
 
@@ -48,6 +52,8 @@ def parse():
     ap.add_argument("--impl", default="samba", choices=["samba", "reference"])
     ap.add_argument("--seq-len", type=int, default=None, help="override L (parity/debug runs only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="prefill line only: skip the decode and mixer-sweep measurements")
     ap.add_argument("--workload", default="prefill",
                     choices=["prefill", "block", "block38", "decode", "sweep", "chunked", "model",
                              "model_decode"],
@@ -65,11 +71,39 @@ def parse():
 
 
 def load_peaks():
+    """(HBM GB/s, burst bf16 TF/s, sustained bf16 TF/s, source): the pool's
+    measured figures when the driver wrote them, else the profiling recipe's
+    fallback (6.65 TB/s, 1.59 PF/s burst, ~1.4 PF/s sustained)."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
         return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), d.get("bf16_tflops_sustained", 1400.0), "measured"
     return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def peak_clock_mhz(kind):
+    """SM clock (MHz) at which a peak was taken: from MEASURED_PEAKS.json when it
+    records one (any numeric field whose name mentions the peak kind and a
+    clock), else the recipe's statement for the fallback sustained figure
+    (~1.4 PF/s at ~1.3 GHz).  None when unknown."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        def walk(d, path=""):
+            for k, v in d.items():
+                name = (path + "." + k).lower()
+                if isinstance(v, dict):
+                    yield from walk(v, name)
+                elif isinstance(v, (int, float)) and ("mhz" in name or "clock" in name):
+                    yield name, float(v)
+        cands = list(walk(json.load(open(p))))
+        sus = [v for n, v in cands if "sustain" in n and 300 < v < 3000]
+        burst = [v for n, v in cands if "sustain" not in n and ("bf16" in n or "gemm" in n) and 300 < v < 3000]
+        if kind == "sustained" and sus:
+            return sus[0]
+        if kind == "burst" and burst:
+            return burst[0]
+        return None
+    return 1300.0 if kind == "sustained" else None
 
 
 # ---------------------------------------------------------------------------
@@ -409,7 +443,7 @@ def replica_throughput(tokens_per_rank, world, t_max, steps, n_blocks):
     return tokens_per_rank * world / (t_max / steps / n_blocks)
 
 
-def kernel_report(kt, s, T, Bn, Ln, peaks, t_up_live=None):
+def kernel_report(kt, s, T, Bn, Ln, peaks, t_up_live=None, clocks=None):
     hbm, tf_burst, tf_sus, src = peaks
     gl = gemm_list(s, T)
     g_flops = sum(fl for (n, M, N, K, e, fl) in gl if n in kt)
@@ -443,16 +477,32 @@ def kernel_report(kt, s, T, Bn, Ln, peaks, t_up_live=None):
     traffic = (207.1e6 - w_bytes) * scale + w_bytes + 236.8e6 * scale if s == I.WIDE else None
     t_alone = kt[name]
     live = t_up_live is not None and 0.5 * t_alone <= t_up_live[0] <= 2.0 * t_alone
-    t_k, peak = (t_up_live[0], tf_sus) if live else (t_alone, tf_burst)
-    roof = {"bound": "tensor", "achieved": round(up / t_k / 1e12, 2), "peak": peak, "unit": "TFLOP/s",
-            "frac": round(up / t_k / 1e12 / peak, 4), "traffic": round(traffic) if traffic else None,
+    t_k, peak, kind = (t_up_live[0], tf_sus, "sustained") if live else (t_alone, tf_burst, "burst")
+    achieved = up / t_k / 1e12
+    note = None
+    if achieved > peak and kind == "sustained":
+        # the sustained figure was taken at a lower clock than this run's: it is
+        # not this kernel's ceiling, so the burst figure is the denominator
+        note = (f"the sustained bf16 figure ({tf_sus} TF/s) is below this kernel's measured rate; "
+                f"the burst figure is used as the peak")
+        peak, kind = tf_burst, "burst"
+    pk_mhz = peak_clock_mhz(kind)
+    run_mhz = (clocks or {}).get("sm_mhz")
+    frac_clk = (achieved / run_mhz) / (peak / pk_mhz) if (pk_mhz and run_mhz) else None
+    roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4), "traffic": round(traffic) if traffic else None,
+            "frac_clock_normalised": round(frac_clk, 4) if frac_clk else None,
+            "clock_normalisation": (f"(achieved / {run_mhz:.0f} MHz median SM clock of this run) / "
+                                    f"(peak / {pk_mhz:.0f} MHz at which the peak was taken)")
+            if frac_clk else "peak clock unknown",
+            "denominator_note": note,
             "algorithmic_flops": up,
             "algorithmic_bytes": T * s.d_model * 2 + w_bytes + T * s.d_ff * 2,
             "kernel": "gemm_tc_kernel<2>: SwiGLU up-projection [T, d_model] x [2 d_ff, d_model]^T",
             "timing": (f"CUDA events around each of its {t_up_live[1]} launches inside the timed region"
                        if live else "attribution pass: the kernel alone, CUDA events"),
-            "peak_source": src + (" sustained bf16 (kernel timed inside the long step)" if live
-                                  else " burst bf16 (kernel timed alone)"),
+            "peak_source": src + (" sustained bf16 (kernel timed inside the long step)" if kind == "sustained"
+                                  else " burst bf16"),
             "alone_tflops": round(up / t_alone / 1e12, 2),
             "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum at M=16384, scaled to M"}
     return roof, rep
@@ -470,17 +520,26 @@ def cpu_threads():
         return os.cpu_count()
 
 
-def oracle_sample(sample_len=1024):
+ORACLE_SAMPLE_LEN = 2304
+_ORACLE_IN = {}
+
+
+def oracle_sample(sample_len=ORACLE_SAMPLE_LEN):
     """fp64 oracle of one block at the workload's shapes on a bounded sample:
-    batch 1, the first `sample_len` tokens.  Returns (tokens/s per block, desc)."""
+    batch 1, the first `sample_len` tokens of the sequence (2304: the last 256
+    attend over the full 2048-key window).  Weights and input are drawn once
+    per process, outside the timing.  Returns (tokens/s per block, desc)."""
     from oracle import samba_oracle as O
     shape = I.WORKLOADS[WORKLOAD][0]
-    W = I.block_weights(shape, 2)
-    x = I.block_input(shape, 2, 1, sample_len)
+    if sample_len not in _ORACLE_IN:
+        _ORACLE_IN[sample_len] = (I.block_weights(shape, 2), I.block_input(shape, 2, 1, sample_len))
+    W, x = _ORACLE_IN[sample_len]
     t0 = time.perf_counter()
     O.block_fwd(x, W, shape)
     dt = time.perf_counter() - t0
-    return sample_len / dt, f"1 block, batch 1, first {sample_len} tokens of the L=131072 sequence (fp64 numpy)"
+    return sample_len / dt, (f"1 block, batch 1, the first {sample_len} tokens of the L=131072 sequence "
+                             f"(the last {sample_len - shape.window} at the full {shape.window}-key window); "
+                             f"fp64 numpy, BLAS threads = cores")
 
 
 def decode_bytes_per_step(s, Bn):
@@ -496,8 +555,13 @@ def decode_bytes_per_step(s, Bn):
     return w + ring + ssm + conv
 
 
-def run_decode(args):
-    """Streaming decode: prefill P tokens at batch 32, then time samba_step replays."""
+DECODE_STEPS = 65536
+
+
+def measure_decode(steps, warmup):
+    """Streaming decode at batch 32 (one block at the 2048-wide shapes, 2048-slot
+    ring): prefill 4096 tokens, then `steps` replays of one captured samba_step.
+    Returns the measurement as a dict (device time, end to end, roofline)."""
     import torch
     from sliding_window_attention_samba_b200 import _lib as L
     torch.cuda.set_device(0)
@@ -520,6 +584,7 @@ def run_decode(args):
     x = torch.randn(Bn, P, s.d_model, generator=g, device=dev).to(bf)
     xo = torch.empty_like(x)
     L.samba_block_fwd(cfg, wst, x, xo, st, None, Bn, P, ws, ws_bytes)
+    del x, xo
     xt = torch.randn(Bn, s.d_model, generator=g, device=dev).to(bf)
     yt = torch.empty_like(xt)
     stream = torch.cuda.Stream()
@@ -529,7 +594,7 @@ def run_decode(args):
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, stream=stream):
             L.samba_step(cfg, wst, xt, yt, st, Bn, ws, ws_bytes, stream=stream)
-        for _ in range(args.warmup):
+        for _ in range(max(3, warmup)):
             graph.replay()
         stream.synchronize()
         assert L.samba_get_error(stream) == 0
@@ -538,7 +603,7 @@ def run_decode(args):
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(args.steps):
+        for _ in range(steps):
             graph.replay()
         e1.record(stream)
         stream.synchronize()
@@ -549,7 +614,7 @@ def run_decode(args):
         yh = torch.empty_like(xh).pin_memory()
         f0 = torch.cuda.Event(enable_timing=True)
         f1 = torch.cuda.Event(enable_timing=True)
-        n_e2e = max(1, min(args.steps, 2000))
+        n_e2e = max(1, min(steps, 2000))
         f0.record(stream)
         for _ in range(n_e2e):
             xt.copy_(xh, non_blocking=True)
@@ -558,26 +623,35 @@ def run_decode(args):
         f1.record(stream)
         stream.synchronize()
         t_e2e = f0.elapsed_time(f1) * 1e-3
+    del graph
     assert L.samba_get_error() == 0
     hbm, _, _, src = load_peaks()
     bps = decode_bytes_per_step(s, Bn)
-    per_step = t / args.steps
-    line = {"metric": "decode tokens/s (batch 32, one Samba block, 2048-slot ring)", "value": Bn * args.steps / t,
-            "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": per_step * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "decode_bf16_B32", "batch": Bn, "prefill": P, "window": s.window,
-                       "d_model": s.d_model, "graph": "one samba_step captured, replayed per step"},
+    per_step = t / steps
+    return {"tokens_per_s": Bn * steps / t, "ms_per_step": per_step * 1e3, "steps": steps, "batch": Bn,
+            "prefill": P, "window": s.window,
             "e2e": {"value": Bn * n_e2e / t_e2e, "unit": "tokens/s", "h2d_bytes_per_step": xh.numel() * 2,
-                    "d2h_bytes_per_step": yh.numel() * 2},
+                    "d2h_bytes_per_step": yh.numel() * 2, "steps": n_e2e},
             "roofline": {"bound": "hbm", "achieved": bps / per_step / 1e9, "peak": hbm, "unit": "GB/s",
                          "frac": bps / per_step / 1e9 / hbm, "traffic": None,
                          "kernel": "whole decode step (weights + ring + states per step)",
                          "peak_source": src, "bytes_per_step": bps},
-            "clocks": clk,
+            "clocks": clk, "graph": "one samba_step captured, replayed per step",
             # per step: 4 RMSNorms, 10 skinny projections, conv step, recurrence
             # step, RoPE table, ring write, attention, position increment
-            "gpu_launches": 20 * args.steps}
+            "gpu_launches": 20 * steps}
+
+
+def run_decode(args):
+    """Streaming decode: prefill P tokens at batch 32, then time samba_step replays."""
+    d = measure_decode(args.steps, args.warmup)
+    line = {"metric": "decode tokens/s (batch 32, one Samba block, 2048-slot ring)", "value": d["tokens_per_s"],
+            "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": d["ms_per_step"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "decode_bf16_B32", "batch": d["batch"], "prefill": d["prefill"],
+                       "window": d["window"], "d_model": I.WIDE.d_model, "graph": d["graph"]},
+            "e2e": d["e2e"], "roofline": d["roofline"], "clocks": d["clocks"], "gpu_launches": d["gpu_launches"]}
     print(json.dumps(line))
 
 
@@ -902,10 +976,11 @@ def run_model_decode(args):
                       "transformer_value": tv, "ratio": sv / tv, "by_model": out, "clocks": clk}))
 
 
-def run_sweep(args):
+def measure_sweep(warmup, max_len):
     """Mixer-only length sweep, batch 1, d_model 2048 shapes: the selective scan
     (d_inner 4096, d_state 16; u, dt, z, B, C ~ N(0,1), Delta = softplus(dt + b))
-    and SWA (32/4 heads of 64, window 2048, RoPE) timed separately per L."""
+    and SWA (32/4 heads of 64, window 2048, RoPE) timed separately per L.
+    Returns one dict per L."""
     import torch
     from sliding_window_attention_samba_b200 import _lib as L
     torch.cuda.set_device(0)
@@ -918,8 +993,9 @@ def run_sweep(args):
     Dk = torch.ones(D, device=dev)
     g = torch.Generator(device=dev)
     g.manual_seed(I.tensor_key(I.MIXER_SWEEP_SEED, "sweep") & ((1 << 63) - 1))
+    rows = []
     for Ln in I.MIXER_SWEEP_L:
-        if Ln > args.max_len:
+        if Ln > max_len:
             break
         u = torch.randn(1, Ln, D, generator=g, device=dev).to(bf)
         dt = torch.randn(1, Ln, D, generator=g, device=dev).to(bf)
@@ -931,8 +1007,8 @@ def run_sweep(args):
 
         def scan():
             L.samba_selective_scan(u, dt, dtb, 1, A_log, Bm, Cm, Dk, z, None, hT, y, 1, Ln, D, N, 1)
-        reps = max(2, min(20, (1 << 22) // Ln))
-        t_scan = _time(torch, scan, args.warmup, reps)
+        reps = max(3, min(20, (1 << 22) // Ln))
+        t_scan = _time(torch, scan, warmup, reps)
         del u, dt, z, y
         q = torch.randn(1, Ln, Hq, hd, generator=g, device=dev).to(bf)
         k = torch.randn(1, Ln, Hkv, hd, generator=g, device=dev).to(bf)
@@ -943,18 +1019,31 @@ def run_sweep(args):
 
         def swa():
             L.samba_swa_fwd(q, k, v, o, 1, Ln, Hq, Hkv, hd, w, 10000.0, 0, 0.0, 1, ws, wsn)
-        t_swa = _time(torch, swa, args.warmup, reps)
+        t_swa = _time(torch, swa, warmup, reps)
+
+        def swa_kernel():  # the attention kernel alone (RoPE off: no table, no rotation pass)
+            L.samba_swa_fwd(q, k, v, o, 1, Ln, Hq, Hkv, hd, w, 0.0, 0, 0.0, 1, ws, wsn)
+        t_swak = _time(torch, swa_kernel, warmup, reps)
         del q, k, v, o, ws
         torch.cuda.empty_cache()
         assert L.samba_get_error() == 0
         sb = Ln * (8 * D + 4 * N)
         sf = swa_flops(I.WIDE, 1, Ln)
-        print(json.dumps({"workload": "mixer_sweep", "seq_len": Ln, "dtype": "bf16",
-                          "scan": {"ms": t_scan * 1e3, "gbs": sb / t_scan / 1e9, "frac_of_" + src + "_hbm": sb / t_scan / 1e9 / hbm,
-                                   "tokens_per_s": Ln / t_scan},
-                          "swa": {"ms": t_swa * 1e3, "tflops": sf / t_swa / 1e12,
-                                  "frac_of_" + src + "_bf16_burst": sf / t_swa / 1e12 / tf_burst,
-                                  "tokens_per_s": Ln / t_swa, "includes": "RoPE of q and k (standalone entry)"}}))
+        rows.append({"seq_len": Ln, "reps": reps,
+                     "scan": {"ms": t_scan * 1e3, "gbs": sb / t_scan / 1e9,
+                              "frac_of_" + src + "_hbm": sb / t_scan / 1e9 / hbm, "tokens_per_s": Ln / t_scan,
+                              "includes": "softplus(dt + bias) in the kernel"},
+                     "swa": {"ms": t_swa * 1e3, "tflops": sf / t_swa / 1e12,
+                             "frac_of_" + src + "_bf16_burst": sf / t_swa / 1e12 / tf_burst,
+                             "tokens_per_s": Ln / t_swa, "includes": "RoPE of q and k (standalone entry)",
+                             "kernel_ms": t_swak * 1e3, "kernel_tflops": sf / t_swak / 1e12,
+                             "kernel_frac_of_" + src + "_bf16_burst": sf / t_swak / 1e12 / tf_burst}})
+    return rows
+
+
+def run_sweep(args):
+    for r in measure_sweep(args.warmup, args.max_len):
+        print(json.dumps({"workload": "mixer_sweep", "dtype": "bf16", **r}))
 
 
 def _time(torch, fn, warmup, reps):
@@ -998,7 +1087,7 @@ def main():
             return
         vals = []
         for i in range(args.warmup + args.steps):
-            v, desc = oracle_sample(256)
+            v, desc = oracle_sample()
             if i >= args.warmup:
                 vals.append(v)
         v = statistics.mean(vals)
@@ -1021,11 +1110,20 @@ def main():
     if rank == 0:
         value = replica_throughput(Bn * Ln, world, r["t_dev"], args.steps, n_blocks)
         e2e = replica_throughput(Bn * Ln, world, r["t_e2e"], args.steps, n_blocks)
-        roof, rep = kernel_report(r["kt"], r["s"], Bn * Ln, Bn, Ln, peaks, r.get("t_up_live"))
+        roof, rep = kernel_report(r["kt"], r["s"], Bn * Ln, Bn, Ln, peaks, r.get("t_up_live"), r["clocks"])
         cpu = None
         if not args.no_cpu_baseline:
-            v, desc = oracle_sample(1024)
+            v, desc = oracle_sample()
             cpu = {"value": v, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle", "sample": desc}
+        extra = {}
+        if world == 1 and not args.no_extras:
+            # the other single-GPU figures of the metric: decode at batch 32
+            # (65 536 graph-replayed steps) and the mixer sweep L = 4K .. 1M
+            import torch
+            torch.cuda.empty_cache()
+            extra["decode"] = measure_decode(DECODE_STEPS, args.warmup)
+            torch.cuda.empty_cache()
+            extra["sweep"] = measure_sweep(args.warmup, args.max_len)
         launches_per_block = 4 + 10 + 1 + 1 + 1 + 1  # norms, projections, conv, scan, rope table, swa
         metric = {"prefill": METRIC, "block": "prefill tokens/s per Samba block (B=4, L=4096)",
                   "block38": "prefill tokens/s per Samba block at the 3.8B widths (L=128K)"}[args.workload]
@@ -1037,7 +1135,7 @@ def main():
                         "mode": "pinned host input in and output out every step, on a copy stream overlapping "
                                 "the previous/next step's compute (double-buffered)"},
                 "roofline": roof, "kernels": rep, "cpu_baseline": cpu, "clocks": r["clocks"],
-                "gpu_launches": launches_per_block * n_blocks * args.steps}
+                "gpu_launches": launches_per_block * n_blocks * args.steps, **extra}
         print(json.dumps(line))
     if world > 1:
         import torch.distributed as dist

@@ -76,6 +76,18 @@ samba_status samba_set_gemm_timing(int epi, void* const* start_events, void* con
 /* Launches recorded by the hook since it was installed. */
 int samba_gemm_timing_count(void);
 
+/* Failure-detection test hook (the paper has no counterpart).  While set
+ * (stop_after_chunks >= 0), every selective-scan launch stops issuing its
+ * input loads after that many 64-token chunks, and its bounded waits give up
+ * after wait_limit_ns (1 ms .. 2 s) instead of 2 s: the wait for the next chunk
+ * then runs out, the kernel latches SAMBA_ERR_TIMEOUT in the device error word,
+ * waits for its own output stores and returns, leaving the context usable.
+ * Outputs past the stop are unspecified.  stop_after_chunks = -1 clears the hook
+ * (wait_limit_ns is then ignored).  Process-wide; the scan reads it at each
+ * launch on the host.  SAMBA_ERR_INVALID_ARG for stop_after_chunks < -1 or a
+ * limit outside the range. */
+samba_status samba_debug_scan_stall(int stop_after_chunks, uint64_t wait_limit_ns);
+
 /* Synchronises `stream`, returns and clears the device error word of the
  * current device: SAMBA_OK, SAMBA_ERR_TIMEOUT or SAMBA_ERR_DEVICE, or
  * SAMBA_ERR_CUDA if the synchronisation itself failed. */
@@ -138,8 +150,11 @@ samba_status samba_swa_fwd(const void* q, const void* k, const void* v, void* o,
  *                                   + round256(B*L*Hkv*head_dim*esize) <= 16 MiB
  * (esize 2 for bf16, 4 for fp32); larger calls return SAMBA_ERR_UNSUPPORTED and
  * launch nothing.  No cudaMalloc/cudaFree or other allocation is made.
- * The first call on each device looks up the array's device address (set-up);
- * make that first call before any stream capture.  All calls share the array and
+ * The first call on each device looks up the array's device address (set-up),
+ * and a call after the device's context was replaced (cudaDeviceReset) looks it
+ * up again; make the first call on a device before any stream capture.  Shapes
+ * beyond the launch grids (B or Hq > 65535) are rejected before any launch, like
+ * the size check above.  All calls share the array and
  * it keeps the last call's contents (each call rewrites what it reads); calls that
  * overlap on the GPU (other streams, other host threads) race on it. */
 samba_status samba_swa_fwd_noalloc(const void* q, const void* k, const void* v, void* o, int B, int L, int Hq,

@@ -90,6 +90,7 @@ _version = _sig("samba_version", ctypes.c_char_p, [])
 _set_timing = _sig("samba_set_gemm_timing", c_int, [c_int, c_void_p, c_void_p, c_int])
 _timing_count = _sig("samba_gemm_timing_count", c_int, [])
 _get_error = _sig("samba_get_error", c_int, [c_void_p])
+_scan_stall = _sig("samba_debug_scan_stall", c_int, [c_int, ctypes.c_uint64])
 _scan_ws = _sig("samba_selective_scan_workspace_size", c_size_t, [c_int, c_int, c_int, c_int])
 _scan = _sig("samba_selective_scan", c_int,
              [c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
@@ -185,6 +186,12 @@ def samba_set_gemm_timing(epi: int, start_events=(), stop_events=()):
 
 def samba_gemm_timing_count() -> int:
     return _timing_count()
+
+
+def samba_debug_scan_stall(stop_after_chunks: int, wait_limit_ns: int = 0) -> None:
+    """Set (stop_after_chunks >= 0) or clear (-1) the scan's failure-detection
+    test hook (see include/samba.h)."""
+    _check("samba_debug_scan_stall", _scan_stall(stop_after_chunks, wait_limit_ns))
 
 
 def samba_get_error(stream=None) -> int:

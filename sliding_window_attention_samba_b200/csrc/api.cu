@@ -19,18 +19,52 @@ namespace samba {
 // ---------------------------------------------------------------------------
 __device__ int g_error_word = 0;
 
+// Identity of the calling thread's current CUDA context.  A module-scope
+// __device__ variable lives in the context that loaded the module, so a
+// device address cached for it is only valid while that context lives: after
+// cudaDeviceReset the device gets a new primary context and the address is
+// looked up again.
+uintptr_t current_context_id() {
+  typedef CUresult (*GetCurrentFn)(CUcontext*);
+  static GetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<GetCurrentFn>(p);
+  });
+  CUcontext c = nullptr;
+  if (!fn || fn(&c) != CUDA_SUCCESS) return 0;
+  return reinterpret_cast<uintptr_t>(c);
+}
+
 int* device_error_word() {
   static int* addr[64] = {nullptr};
+  static uintptr_t ctx[64] = {0};
   static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  const uintptr_t c = current_context_id();  // 0 before the runtime's first call made one current
   std::lock_guard<std::mutex> lk(mu);
-  if (!addr[dev]) {
+  if (!addr[dev] || ctx[dev] != c) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
     addr[dev] = static_cast<int*>(p);
+    ctx[dev] = c;
   }
   return addr[dev];
+}
+
+// ---------------------------------------------------------------------------
+// Failure-detection test hook of the selective scan
+// ---------------------------------------------------------------------------
+static std::mutex g_stall_mu;
+static StallHook g_stall = {-1, kWaitLimitNs};
+StallHook scan_stall_hook() {
+  std::lock_guard<std::mutex> lk(g_stall_mu);
+  return g_stall;
 }
 
 // ---------------------------------------------------------------------------
@@ -227,6 +261,16 @@ samba_status samba_set_gemm_timing(int epi, void* const* start_events, void* con
 
 int samba_gemm_timing_count(void) { return gemm_timing_count(); }
 
+samba_status samba_debug_scan_stall(int stop_after_chunks, uint64_t wait_limit_ns) {
+  if (stop_after_chunks < -1) return SAMBA_ERR_INVALID_ARG;
+  if (stop_after_chunks >= 0 && (wait_limit_ns < 1000000ull || wait_limit_ns > kWaitLimitNs))
+    return SAMBA_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_stall_mu);
+  g_stall.stop_chunk = stop_after_chunks;
+  g_stall.wait_limit_ns = stop_after_chunks >= 0 ? wait_limit_ns : kWaitLimitNs;
+  return SAMBA_OK;
+}
+
 samba_status samba_get_error(samba_stream stream) {
   if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return SAMBA_ERR_CUDA;
   int* w = device_error_word();
@@ -293,6 +337,7 @@ samba_status samba_swa_fwd(const void* q, const void* k, const void* v, void* o,
   if (head_dim != 16 && head_dim != 32 && head_dim != 64 && !(head_dim == 256 && dtype == SAMBA_BF16))
     return SAMBA_ERR_UNSUPPORTED;
   if (pos0 + (int64_t)L > (int64_t(1) << 30)) return SAMBA_ERR_UNSUPPORTED;
+  if (B > kMaxGridYZ || Hq > kMaxGridYZ) return SAMBA_ERR_UNSUPPORTED;  // before the RoPE launches
   if (L == 0) return SAMBA_OK;
   SwaArgs a;
   a.q = q;

@@ -20,6 +20,7 @@ namespace samba {
 enum : int { kErrNone = 0, kErrTimeout = 1, kErrDevice = 2 };
 
 int* device_error_word();  // device address of the error word of the current device
+uintptr_t current_context_id();  // the calling thread's current CUDA context (0: none yet)
 
 __device__ __forceinline__ void raise_error(int* err, int code) {
   if (err) atomicCAS(err, 0, code);
@@ -145,19 +146,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait until the phase with the given parity completed.  Gives up after
-// `limit_ns` of wall time, latches kErrTimeout and returns false.
+// `limit_ns` of wall time (default 2 s), latches kErrTimeout and returns false.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 63u && globaltimer_ns() - t0 > kWaitLimitNs) {
+    if ((it & 63u) == 63u && globaltimer_ns() - t0 > limit_ns) {
       raise_error(err, kErrTimeout);
       return false;
     }
   }
 }
+
+// Failure-detection test hook (host side): while set, selective-scan launches
+// stop issuing their input loads after `stop_chunk` chunks and give up waiting
+// after `wait_limit_ns`, so that the bounded-wait path runs without any fault.
+struct StallHook {
+  int stop_chunk;          // -1: off
+  uint64_t wait_limit_ns;  // wait limit while the hook is set
+};
+StallHook scan_stall_hook();
 
 // ---------------------------------------------------------------------------
 // TMA (no multicast anywhere in this library)

@@ -63,7 +63,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ CUtensorMap tm_y,
                         const float* __restrict__ A_log, const float* __restrict__ dt_bias,
                         const float* __restrict__ Dskip, const float* __restrict__ h0, float* __restrict__ hT,
-                        int L, int D, int* err) {
+                        int L, int D, int* err, int stop_chunk, uint64_t wait_limit_ns) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   ScanSmem<T>& S = *reinterpret_cast<ScanSmem<T>*>(smem_raw + smem_align_pad(smem_raw, 128));
 
@@ -91,6 +91,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
 
   auto issue = [&](int c) {
+    if (c >= stop_chunk) return;  // failure-detection test hook: nothing issued past here
     const int s = c % kStages;
     const int t0 = c * kChunk;
     mbar_arrive_expect_tx(&S.full[s], stage_bytes);
@@ -103,7 +104,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // wait for chunk c's stage, then convert its B and C to fp32 (one element per thread pass)
   auto arrive_chunk = [&](int c) -> bool {
     const int s = c % kStages;
-    const bool ok = mbar_wait(&S.full[s], (c / kStages) & 1, err);
+    const bool ok = mbar_wait(&S.full[s], (c / kStages) & 1, err, wait_limit_ns);
     if (ok) {
       // 64 rows x (16 B | 16 C) = 256 runs of 8 values: one per thread
       static_assert(kChunk * 4 == kThreads, "one 8-value run of B or C per thread");
@@ -296,8 +297,10 @@ samba_status launch_typed(const ScanArgs& a, cudaStream_t st) {
   if (!ensure_smem_attr(kern, smem))
     return SAMBA_ERR_CUDA;
   dim3 grid(a.D / kCh, a.B);
+  const StallHook hk = scan_stall_hook();
   kern<<<grid, kThreads, smem, st>>>(mu, mdt, mz, mB, mC, my, a.A_log, a.dt_bias, a.Dskip, a.h0, a.hT, a.L, a.D,
-                                     device_error_word());
+                                     device_error_word(), hk.stop_chunk < 0 ? INT32_MAX : hk.stop_chunk,
+                                     hk.stop_chunk < 0 ? kWaitLimitNs : hk.wait_limit_ns);
   SAMBA_CHECK_LAUNCH();
   return SAMBA_OK;
 }

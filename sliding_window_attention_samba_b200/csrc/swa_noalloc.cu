@@ -12,9 +12,10 @@
 //   * The scratch is a file-scope static __device__ array of kNoallocScratchBytes
 //     (16 MiB).  Every GPU that loads the library holds it until the process exits.
 //   * Host code never passes the array's name to a kernel (on the host it is only
-//     a stand-in symbol); the device address is looked up once per device with
+//     a stand-in symbol); the device address is looked up with
 //     cudaGetSymbolAddress, with that device current, on the first call made on
-//     that device.  Make that first call before any stream capture.
+//     that device (and again if the device's context was replaced, e.g. by
+//     cudaDeviceReset).  Make that first call before any stream capture.
 //   * Calls reject sizes whose scratch would not fit (SAMBA_ERR_UNSUPPORTED) and
 //     never call cudaMalloc/cudaFree or any allocating routine.
 //   * All calls share the one array and it keeps the last call's contents; the
@@ -34,17 +35,22 @@ constexpr size_t kNoallocScratchBytes = size_t(16) << 20;  // 16 MiB
 
 static __device__ __align__(256) unsigned char g_swa_noalloc_scratch[kNoallocScratchBytes];
 
-// Device address of the scratch array on the current device (set-up on first use).
+// Device address of the scratch array on the current device (set-up on first
+// use, and again whenever the device's context changed, e.g. after
+// cudaDeviceReset: the array lives in the context that loaded the module).
 unsigned char* noalloc_scratch_ptr() {
   static unsigned char* ptr[64] = {nullptr};
+  static uintptr_t ctx[64] = {0};
   static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  const uintptr_t c = current_context_id();
   std::lock_guard<std::mutex> lk(mu);
-  if (!ptr[dev]) {
+  if (!ptr[dev] || ctx[dev] != c) {
     unsigned char* p = nullptr;
     if (cudaGetSymbolAddress((void**)&p, g_swa_noalloc_scratch) != cudaSuccess) return nullptr;
     ptr[dev] = p;
+    ctx[dev] = c;
   }
   return ptr[dev];
 }
@@ -73,6 +79,7 @@ extern "C" samba_status samba_swa_fwd_noalloc(const void* q, const void* k, cons
   if (head_dim != 16 && head_dim != 32 && head_dim != 64 && !(head_dim == 256 && dtype == SAMBA_BF16))
     return SAMBA_ERR_UNSUPPORTED;
   if (pos0 + (int64_t)L > (int64_t(1) << 30)) return SAMBA_ERR_UNSUPPORTED;
+  if (B > kMaxGridYZ || Hq > kMaxGridYZ) return SAMBA_ERR_UNSUPPORTED;  // before any launch
   if (L == 0) return SAMBA_OK;
   SwaArgs a;
   a.q = q;

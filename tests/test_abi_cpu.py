@@ -97,6 +97,17 @@ def test_grid_limits_rejected_before_launch(lib):
     rc = h.samba_swa_fwd(fake, fake, fake, fake, big_b, 16, 4, 4, 64, 8, ctypes.c_float(0.0), 0,
                          ctypes.c_float(0.0), 1, None, 0, None)
     assert rc == lib.SAMBA_ERR_UNSUPPORTED
+    # with RoPE on, the grid check still comes before the table and rotation launches
+    # (a CUDA call here would return SAMBA_ERR_CUDA instead)
+    rc = h.samba_swa_fwd(fake, fake, fake, fake, big_b, 1, 1, 1, 16, 8, ctypes.c_float(10000.0), 0,
+                         ctypes.c_float(0.0), 1, fake, ctypes.c_size_t(1 << 40), None)
+    assert rc == lib.SAMBA_ERR_UNSUPPORTED
+    rc = h.samba_swa_fwd_noalloc(fake, fake, fake, fake, big_b, 1, 1, 1, 16, 8, ctypes.c_float(10000.0), 0,
+                                 ctypes.c_float(0.0), 1, None)
+    assert rc == lib.SAMBA_ERR_UNSUPPORTED
+    rc = h.samba_swa_fwd_noalloc(fake, fake, fake, fake, 1, 1, big_b, 1, 16, 8, ctypes.c_float(0.0), 0,
+                                 ctypes.c_float(0.0), 1, None)
+    assert rc == lib.SAMBA_ERR_UNSUPPORTED
     cfg = lib.make_config(I.TINY)
     w = lib.BlockWeights()
     for i in range(4):
@@ -160,3 +171,14 @@ def test_gemm_timing_hook_host_side(lib):
     assert h.samba_set_gemm_timing(2, a, b, 2) == 0
     assert h.samba_gemm_timing_count() == 0
     assert h.samba_set_gemm_timing(-1, None, None, 0) == 0
+
+
+def test_scan_stall_hook_arguments(lib):
+    """The failure-detection hook validates its arguments on the host; setting and
+    clearing it makes no device call."""
+    h = lib.lib_handle()
+    assert h.samba_debug_scan_stall(-2, 0) == lib.SAMBA_ERR_INVALID_ARG
+    assert h.samba_debug_scan_stall(3, 10) == lib.SAMBA_ERR_INVALID_ARG          # below 1 ms
+    assert h.samba_debug_scan_stall(3, 3_000_000_000) == lib.SAMBA_ERR_INVALID_ARG  # above 2 s
+    assert h.samba_debug_scan_stall(3, 5_000_000) == 0
+    assert h.samba_debug_scan_stall(-1, 0) == 0

@@ -6,7 +6,7 @@ import pytest
 
 from oracle import samba_oracle as O
 from sliding_window_attention_samba_b200 import inputs as I
-from tests.helpers import TOL, block_weights_dev, dev, host, rel_err
+from tests.helpers import TOL, attn_err, block_weights_dev, dev, host, rel_err, stream_slack
 
 pytestmark = pytest.mark.gpu
 
@@ -62,19 +62,37 @@ class GpuBlock:
         return y
 
 
+def branch_err(i, got, ref, dt):
+    """The SWA branch (i = 2) in bf16 is attention over bf16-stored rotated q/k
+    followed by the output projection: its rows inherit the attention output's
+    row-to-row scale spread (a query's first tokens average few values), so it
+    is held to the attention reading; every other branch to the elementwise one."""
+    return (attn_err if (i == 2 and dt == "bf16") else rel_err)(got, ref)
+
+
 def check_branches(shape, W, x, out, br, rs, tol):
     """GPU branch outputs (tapped before each residual add) and residual stream
     against the oracle's own fp64 stream; a branch sees the stream through an
-    RMSNorm, so the GPU's bf16 rounding of the stream stays a relative error of
-    the branch input."""
+    RMSNorm, so the GPU's rounding of the stream stays a relative error of the
+    branch input.  The stream values are checked with the allowance for their own
+    storage rounding (one half-ulp per residual add that produced them)."""
     x = x.astype(np.float64)
+    dt = shape.dtype
     ref = O.block_fwd(x, W, shape)
-    errs = [rel_err(br[i], ref["branch"][i]) for i in range(4)]
+    errs = [branch_err(i, br[i], ref["branch"][i], dt) for i in range(4)]
     assert max(errs) <= tol, errs
     for i in range(3):
-        assert rel_err(rs[i], ref["resid"][i]) <= tol, i
-    assert rel_err(out, ref["x_out"]) <= tol
+        assert rel_err(rs[i], ref["resid"][i], slack=stream_slack(ref["resid"], dt, i)) <= tol, i
+    assert rel_err(out - x, ref["x_out"] - x, slack=stream_slack(ref["resid"], dt)) <= tol
     return errs
+
+
+def step_err(y, xt, full, t, dt):
+    """Decode output y at position t against the oracle's prefill of the longer
+    sequence: the block's contribution y - x_t, with the stream's storage
+    allowance taken from the oracle's own streams at t."""
+    res = [r[:, t] for r in full["resid"]]
+    return rel_err(y - xt, full["x_out"][:, t] - xt, slack=stream_slack(res, dt))
 
 
 def test_block_tiny_f32(L):
@@ -115,7 +133,7 @@ def test_prefill_then_step_tiny_f32(L, P, S):
     g.prefill(x[:, :P], taps=False)
     for i in range(S):
         y = host(g.step(x[:, P + i]))
-        assert rel_err(y - x[:, P + i], full["x_out"][:, P + i] - x[:, P + i]) <= TOL["f32"], i
+        assert step_err(y, x[:, P + i], full, P + i, "f32") <= TOL["f32"], i
     assert rel_err(host(g.ssm), full["state"]["ssm"]) <= TOL["f32"]
     assert np.array_equal(host(g.pos), full["state"]["pos"])
 
@@ -144,7 +162,7 @@ def test_prefill_state_handoff_wide_bf16(L):
     full = O.block_fwd(x, W, shape)
     for i in range(2):
         y = host(g.step(x[:, P + i]))
-        assert rel_err(y - x[:, P + i], full["x_out"][:, P + i] - x[:, P + i]) <= TOL["bf16"]
+        assert step_err(y, x[:, P + i], full, P + i, "bf16") <= TOL["bf16"]
 
 
 def test_step_state_save_restore_bit_exact_and_graph(L):
@@ -194,4 +212,76 @@ def test_decode_steps_wide_bf16_batch4(L):
     full = O.block_fwd(x, W, shape)
     for i in range(S):
         y = host(g.step(x[:, P + i]))
-        assert rel_err(y - x[:, P + i], full["x_out"][:, P + i] - x[:, P + i]) <= TOL["bf16"], i
+        assert step_err(y, x[:, P + i], full, P + i, "bf16") <= TOL["bf16"], i
+
+
+def _ring_map_exact(ring, oracle_k, cur, w):
+    """The ring's slot -> position map after `cur` tokens, bit-exact: every slot
+    holds the key of the latest position p < cur with p mod w == slot (slots
+    never written yet, when cur < w, are skipped).  A slot's position is read as
+    the oracle key nearest to the stored one."""
+    Bn = ring.shape[0]
+    flat = oracle_k[:, :cur].reshape(Bn, cur, -1)
+    for b in range(Bn):
+        for slot in range(min(w, cur)):
+            p_expect = cur - 1 - ((cur - 1 - slot) % w)
+            dist = np.linalg.norm(flat[b] - ring[b, slot].reshape(1, -1), axis=1)
+            assert int(np.argmin(dist)) == p_expect, (b, slot, cur)
+
+
+def test_decode_ring_wraps_32x_tiny_f32(L):
+    """2100 decode steps over a 64-slot ring (32.8 wraps) after a 10-token
+    prefill, batch 2: every step's output against the oracle's prefill of the
+    whole sequence; the position counter and the ring's slot -> position map
+    bit-exact at checkpoints around and far past the wraps."""
+    import torch
+    shape = I.TINY
+    w = shape.window
+    P, S, Bn = 10, 2100, 2
+    W = I.block_weights(shape, 21, conv_bias=True)
+    x = I.block_input(shape, 21, Bn, P + S)
+    full = O.block_fwd(x, W, shape)
+    g = GpuBlock(L, shape, W, Bn, P + S)
+    g.prefill(x[:, :P], taps=False)
+    xd = dev(x, "f32")
+    ys = torch.empty(S, Bn, shape.d_model, device="cuda")
+    checks = {w - P - 1, w - P, 1000, S - 1}
+    for i in range(S):
+        L.samba_step(g.cfg, g.w, xd[:, P + i].contiguous(), ys[i], g.st, Bn, g.ws, g.ws.numel())
+        if i in checks:
+            cur = P + i + 1
+            assert np.array_equal(host(g.pos), np.full(Bn, cur))
+            _ring_map_exact(host(g.k_ring), full["attn"]["k"], cur, w)
+    torch.cuda.synchronize()
+    assert L.samba_get_error() == 0
+    yh = host(ys)
+    errs = [step_err(yh[i], x[:, P + i], full, P + i, "f32") for i in range(S)]
+    assert max(errs) <= TOL["f32"], int(np.argmax(errs))
+
+
+def test_decode_ring_wraps_wide_bf16(L):
+    """800 decode steps of the 2048-wide block over a 256-slot ring (3.5 wraps)
+    after a 100-token prefill: sampled steps around each wrap against the
+    oracle's prefill of the whole sequence, the ring map bit-exact at the end."""
+    import dataclasses
+    import torch
+    shape = dataclasses.replace(I.WIDE, window=256)
+    w = shape.window
+    P, S = 100, 800
+    W = I.block_weights(shape, 22)
+    x = I.block_input(shape, 22, 1, P + S)
+    full = O.block_fwd(x, W, shape)
+    g = GpuBlock(L, shape, W, 1, P + S)
+    g.prefill(x[:, :P], taps=False)
+    xd = dev(x, "bf16")
+    ys = torch.empty(S, 1, shape.d_model, device="cuda", dtype=torch.bfloat16)
+    for i in range(S):
+        L.samba_step(g.cfg, g.w, xd[:, P + i].contiguous(), ys[i], g.st, 1, g.ws, g.ws.numel())
+    torch.cuda.synchronize()
+    assert L.samba_get_error() == 0
+    yh = host(ys)
+    for i in (0, 1, w - P - 1, w - P, w - P + 1, 2 * w - P, 3 * w - P, S - 1):
+        assert step_err(yh[i], x[:, P + i], full, P + i, "bf16") <= TOL["bf16"], i
+    cur = P + S
+    assert np.array_equal(host(g.pos), np.full(1, cur))
+    _ring_map_exact(host(g.k_ring), full["attn"]["k"], cur, w)

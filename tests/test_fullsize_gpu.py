@@ -15,7 +15,8 @@ import pytest
 
 from oracle import samba_oracle as O
 from sliding_window_attention_samba_b200 import inputs as I
-from tests.helpers import TOL, block_weights_dev, dev, host, rel_err
+from tests.helpers import TOL, attn_err, block_weights_dev, dev, host, rel_err, stream_slack
+from tests.test_block_gpu import branch_err, step_err
 
 pytestmark = pytest.mark.gpu
 
@@ -62,8 +63,9 @@ def test_prefill_stack_L131072_prefix(L):
         assert torch.isfinite(nxt).all()
         ref = O.block_fwd(xo, W, shape)
         for i in range(4):
-            assert rel_err(host(br[i][:, :P]), ref["branch"][i]) <= TOL["bf16"], (li, i)
-        assert rel_err(host(nxt[:, :P]), ref["x_out"]) <= TOL["bf16"], li
+            assert branch_err(i, host(br[i][:, :P]), ref["branch"][i], "bf16") <= TOL["bf16"], (li, i)
+        assert rel_err(host(nxt[:, :P]) - xo, ref["x_out"] - xo,
+                       slack=stream_slack(ref["resid"], "bf16")) <= TOL["bf16"], li
         xo = ref["x_out"]
         cur, nxt = nxt, cur
         del Wd
@@ -83,9 +85,10 @@ def test_block_B4_L4096_one_full_row(L):
     torch.cuda.synchronize()
     assert L.samba_get_error() == 0
     row = 2
-    ref = O.block_fwd(x[row:row + 1], W, shape)["x_out"]
+    ref = O.block_fwd(x[row:row + 1], W, shape)
     got = host(out[row:row + 1])
-    assert rel_err(got - x[row:row + 1], ref - x[row:row + 1]) <= TOL["bf16"]
+    assert rel_err(got - x[row:row + 1], ref["x_out"] - x[row:row + 1],
+                   slack=stream_slack(ref["resid"], "bf16")) <= TOL["bf16"]
 
 
 def test_decode_B32_after_4096_prefill(L):
@@ -113,10 +116,9 @@ def test_decode_B32_after_4096_prefill(L):
     assert L.samba_get_error() == 0
     assert np.array_equal(host(st_t[4]), np.full(Bn, P + S))
     row = 17
-    ref = O.block_fwd(x[row:row + 1], W, shape)["x_out"][0]
+    ref = O.block_fwd(x[row:row + 1], W, shape)
     for i in range(S):
-        d = x[row, P + i]
-        assert rel_err(ys[i][row] - d, ref[P + i] - d) <= TOL["bf16"], i
+        assert step_err(ys[i][row:row + 1], x[row:row + 1, P + i], ref, P + i, "bf16") <= TOL["bf16"], i
 
 
 def test_scan_L1M_sampled_channels(L):
@@ -199,4 +201,4 @@ def test_swa_L1M_sampled_rows(L):
             sc = kr[0, :, h // grp] @ qr[0, 0, h] / np.sqrt(hd)
             p = np.exp(sc - sc.max())
             ref[h] = (p / p.sum()) @ vh[0, :, h // grp].astype(np.float64)
-        assert rel_err(host(o[0, t]), ref) <= TOL["bf16"], t
+        assert attn_err(host(o[0, t]), ref) <= TOL["bf16"], t

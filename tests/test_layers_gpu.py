@@ -7,7 +7,7 @@ import pytest
 
 from oracle import samba_oracle as O
 from sliding_window_attention_samba_b200 import inputs as I
-from tests.helpers import TOL, dev, host, rel_err
+from tests.helpers import TOL, dev, host, rel_err, sum_slack
 
 pytestmark = pytest.mark.gpu
 
@@ -73,19 +73,18 @@ def _linear(L, dt, M, N, K, epi, force_simt=False):
     assert L.samba_get_error() == 0
     h = O.linear(x, W)
     ref = {0: h, 1: resid + h, 2: h * O.silu(O.linear(x, W2)), 3: O.softplus(h + bias)}[epi]
-    # the residual epilogue is checked on the branch part; the sum is dominated by resid
+    # the residual epilogue is checked on the branch part (the sum is dominated by
+    # resid); the single rounding of the stored sum is not error of the branch
     if epi == 1:
-        return rel_err(host(out) - resid, h)
+        got = host(out)
+        return rel_err(got - resid, h, slack=sum_slack(got, dt))
     return rel_err(host(out), ref)
 
 
 @pytest.mark.parametrize("epi", [0, 1, 2, 3])
 @pytest.mark.parametrize("M,N,K", [(300, 256, 2048), (128, 160, 4096), (1000, 512, 128), (77, 2048, 1024)])
 def test_linear_tensor_core_bf16(L, epi, M, N, K):
-    if epi == 1:
-        assert _linear(L, "bf16", M, N, K, epi) <= 0.05  # bf16 rounding of resid+h relative to the small h
-    else:
-        assert _linear(L, "bf16", M, N, K, epi) <= TOL["bf16"]
+    assert _linear(L, "bf16", M, N, K, epi) <= TOL["bf16"]
 
 
 @pytest.mark.parametrize("epi", [0, 2, 3])
@@ -124,5 +123,4 @@ _SKINNY_SHAPES = [(1, 2048, 8192), (7, 160, 4096), (32, 8192, 2048), (64, 4096, 
 def test_linear_skinny_decode_bf16(L, epi, M, N, K):
     """M <= 64 (decode batch): swap-AB tensor-core tiles, split-K over a thread-block
     cluster reduced through distributed shared memory."""
-    err = _linear(L, "bf16", M, N, K, epi)
-    assert err <= (0.05 if epi == 1 else TOL["bf16"])
+    assert _linear(L, "bf16", M, N, K, epi) <= TOL["bf16"]

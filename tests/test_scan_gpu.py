@@ -125,3 +125,29 @@ def test_scan_ragged_lengths_bf16(L, Ln):
     y, hT = run_scan(L, r, "bf16", h0=r["h0"])
     yo, ho = oracle_scan(r, h0=r["h0"])
     assert rel_err(y, yo) <= TOL["bf16"] and rel_err(hT, ho) <= TOL["bf16"]
+
+
+def test_scan_bounded_wait_times_out_and_recovers(L):
+    """Failure detection without a fault: the test hook makes the scan's loader
+    stop after 3 of 8 chunks and shortens the wait limit to 5 ms.  The consumer's
+    wait for chunk 3 runs out, the kernel latches SAMBA_ERR_TIMEOUT, drains its
+    own output stores and returns; the context stays usable, and the next call
+    without the hook matches the oracle."""
+    r = I.scan_inputs(6, 1, 512, 64, 16, "bf16", with_h0=True)
+    L.samba_debug_scan_stall(3, 5_000_000)
+    try:
+        import torch
+        Bn, Ln, D = r["u"].shape
+        u, dtt = dev(r["u"], "bf16"), dev(r["dt_raw"], "bf16")
+        y = torch.empty_like(u)
+        L.samba_selective_scan(u, dtt, dev(r["dt_bias"]), 1, dev(r["A_log"]), dev(r["B"], "bf16"),
+                               dev(r["C"], "bf16"), dev(r["D"]), dev(r["z"], "bf16"), dev(r["h0"]), None, y,
+                               Bn, Ln, D, 16, 1)
+        assert L.samba_get_error() == L.SAMBA_ERR_TIMEOUT
+    finally:
+        L.samba_debug_scan_stall(-1)
+    assert L.samba_get_error() == 0  # the word was cleared by the read
+    y, hT = run_scan(L, r, "bf16", h0=r["h0"])
+    yo, ho = oracle_scan(r, h0=r["h0"])
+    assert rel_err(y, yo) <= TOL["bf16"]
+    assert rel_err(hT, ho) <= TOL["bf16"]

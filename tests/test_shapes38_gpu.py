@@ -7,7 +7,7 @@ import pytest
 
 from oracle import samba_oracle as O
 from sliding_window_attention_samba_b200 import inputs as I
-from tests.helpers import TOL, dev, host, rel_err
+from tests.helpers import TOL, attn_err, dev, host, rel_err, sum_slack
 from tests.test_block_gpu import GpuBlock, check_branches
 
 pytestmark = pytest.mark.gpu
@@ -36,7 +36,7 @@ def test_swa_head_dim_256_gqa11(L, Bn, Ln, window, pos0):
     assert L.samba_get_error() == 0
     pos = np.arange(pos0, pos0 + Ln)
     ref = O.swa(O.rope(r["q"], pos, 1e4), O.rope(r["k"], pos, 1e4), r["v"], window)
-    assert rel_err(host(o), ref) <= TOL["bf16"]
+    assert attn_err(host(o), ref) <= TOL["bf16"]
 
 
 @pytest.mark.parametrize("M,N,K,epi", [(300, 208, 5632, 0), (1000, 5632, 176, 3), (257, 176, 2816, 0),
@@ -53,7 +53,8 @@ def test_projection_tails(L, M, N, K, epi):
     assert L.samba_get_error() == 0
     h = O.linear(x, W)
     if epi == 1:
-        assert rel_err(host(out) - resid, h) <= 0.05
+        got = host(out)
+        assert rel_err(got - resid, h, slack=sum_slack(got, "bf16")) <= TOL["bf16"]
     else:
         ref = O.softplus(h + bias) if epi == 3 else h
         assert rel_err(host(out), ref) <= TOL["bf16"]

@@ -40,6 +40,7 @@ def _pair(L_, dt, Bn, Ln, Hq, Hkv, d, w, base, pos0, seed):
     ("bf16", 1, 1024, 32, 4, 64, 256, 10000.0, 0),
     ("f32", 2, 300, 4, 2, 16, 64, 10000.0, 12345),
     ("bf16", 1, 200, 8, 2, 64, 50, 0.0, 0),
+    ("bf16", 1, 1500, 11, 1, 256, 2048, 10000.0, 7),  # head_dim 256: 11.9 MiB of scratch
 ])
 def test_noalloc_matches_workspace_entry_two_calls(L, dt, Bn, Ln, Hq, Hkv, d, w, base, pos0):
     # two calls in a row with different inputs: the shared scratch keeps the first
@@ -48,6 +49,20 @@ def test_noalloc_matches_workspace_entry_two_calls(L, dt, Bn, Ln, Hq, Hkv, d, w,
         got, ref = _pair(L, dt, Bn, Ln, Hq, Hkv, d, w, base, pos0, seed)
         assert not np.isnan(got).any()
         assert rel_err(got, ref) <= TOL[dt]
+
+
+def test_noalloc_back_to_back_calls_with_other_shapes(L):
+    # consecutive calls with a different head_dim, table size, rope base and
+    # position: each call rebuilds the table and the rotated copies it reads, so
+    # none depends on what the previous call left in the shared scratch
+    cases = [("bf16", 1, 600, 11, 1, 256, 512, 10000.0, 3, 21),
+             ("bf16", 2, 333, 8, 2, 64, 100, 500000.0, 1000, 22),
+             ("f32", 1, 257, 4, 2, 32, 64, 10000.0, 0, 23),
+             ("bf16", 1, 600, 11, 1, 256, 512, 20000.0, 99, 24)]
+    for dt, Bn, Ln, Hq, Hkv, d, w, base, pos0, seed in cases:
+        got, ref = _pair(L, dt, Bn, Ln, Hq, Hkv, d, w, base, pos0, seed)
+        assert not np.isnan(got).any()
+        assert rel_err(got, ref) <= TOL[dt], (d, base)
 
 
 def test_noalloc_rejects_sizes_beyond_the_fixed_scratch(L):
