@@ -6,25 +6,31 @@
 //   h_t     = exp(Delta_t A) (.) h_{t-1} + Delta_t u_t B_t
 //   y_t     = <C_t, h_t> + D u_t,   y_t *= SiLU(z_t)
 //
-// Design (one CTA = 32 channels of one batch row, the whole sequence):
-//   * 64-token chunks of u, dt, z (32 channels wide) and B, C (16 wide) are
-//     staged through shared memory by TMA, NSTAGE deep.
-//   * 8 warps split each chunk in time: warp w owns tokens [8w, 8w+8), lane l
-//     owns channel l and its 16 fp32 states in registers.
-//   * B and C of a chunk are converted to fp32 once into a shared tile (all 32
-//     lanes of a warp read the same values, so per-lane conversion would repeat
-//     it 32 times).
-//   * Walk 1: each lane runs its 8 tokens from a zero state, keeping the 8x16
-//     decays exp(Delta A) in registers, and publishes (prod of decays, end state).
-//     States are processed in pairs with packed fp32x2 FMA/MUL.
-//   * Combine: 256 threads each own two (channel, state) pairs and chain the
-//     8 warp aggregates sequentially from the carry of the previous chunk
-//     (kept in registers across chunks); this yields every warp's entry state.
-//   * Walk 2: each lane re-runs its tokens from the right entry state with the
-//     cached decays (one exp per element in total), emits y into a shared tile
-//     written back by a TMA store.
-// No inter-CTA communication, no workspace, no spin waits except the TMA
-// mbarrier waits (bounded, error word on timeout).
+// Design (one CTA = 16 channels of one batch row for the whole sequence, two
+// CTAs per SM):
+//   * 64-token chunks of u, dt, z (16 channels wide) and B, C (16 wide) are
+//     staged through shared memory by TMA, kStages deep.
+//   * Lane l of every warp owns channel l & 15 and half of its 16 fp32 states
+//     (l >> 4 selects states 0-7 or 8-15).  Warp w owns tokens [8w, 8w + 8) of
+//     every chunk.
+//   * Each warp converts its own 8 rows once (B, C to fp32; Delta, Delta u,
+//     the SiLU(z) gate and D u gate per token and channel), so the walks never
+//     repeat per-token work between the two lanes of a channel.
+//   * Walk 1: each lane runs its 8 tokens from a zero state, keeping the 8x8
+//     decays exp(Delta A) in registers (one exp per element), and forms the
+//     slice aggregate (product of decays P, end state H).
+//   * Carry chain: warp w waits for its entry state E_w (an mbarrier per warp
+//     slot), passes E_{w+1} = P (.) E_w + H to warp w + 1 through shared memory,
+//     warp 7 hands the next chunk's entry state to warp 0.  There is no
+//     CTA-wide barrier in the steady state: warps drift one hop apart, so the
+//     exp-heavy walk 1 of one warp overlaps the FMA-heavy walk 2 of another.
+//   * Walk 2: each lane re-runs its tokens from E_w with the cached decays,
+//     the two lanes of a channel add their partial read-outs with one shuffle
+//     per token pair, and y goes to a shared tile written back by a TMA store.
+//   * Warp 7's lane 0 recycles input stages (once every warp converted the
+//     chunk) and stores y tiles (once every warp wrote its rows).
+// Every wait is bounded (error word on timeout); a timed-out CTA drains its
+// own copies in flight before it returns.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -32,238 +38,326 @@ namespace samba {
 
 namespace {
 
-constexpr int kCh = 32;       // channels per CTA
-constexpr int kWarps = 8;     // time sub-chunks per chunk
-constexpr int kTs = 8;        // tokens per warp sub-chunk
+constexpr int kCh = 16;               // channels per CTA
+constexpr int kWarps = 8;             // token slices per chunk
+constexpr int kTs = 8;                // tokens per warp slice
 constexpr int kChunk = kWarps * kTs;  // 64 tokens
-constexpr int kN = 16;        // state size
-constexpr int kStages = 3;
+constexpr int kN = 16;                // state size
+constexpr int kHalf = 8;              // states per lane
 constexpr int kThreads = kWarps * 32;
+constexpr int kYBuf = 3;              // y tiles in flight
+
+template <typename T> struct ScanCfg { static constexpr int kStages = sizeof(T) == 2 ? 4 : 2; };
 
 template <typename T>
 struct ScanSmem {
-  T u[kStages][kChunk * kCh];
-  T dt[kStages][kChunk * kCh];
-  T z[kStages][kChunk * kCh];
-  T Bm[kStages][kChunk * kN];
-  T Cm[kStages][kChunk * kN];
-  T y[2][kChunk * kCh];
-  float BC[2][kChunk][2 * kN];  // fp32 copy of B | C per token, converted once per chunk
-  float aggP[kWarps][kN][kCh];
-  float aggH[kWarps][kN][kCh];
-  uint64_t full[kStages];
+  static constexpr int S = ScanCfg<T>::kStages;
+  T u[S][kChunk * kCh];  // [token][channel]
+  T dt[S][kChunk * kCh];
+  T z[S][kChunk * kCh];
+  T Bm[S][kChunk * kN];  // [token][state]
+  T Cm[S][kChunk * kN];
+  T y[kYBuf][kChunk * kCh];
+  float BC[kWarps][kTs][2 * kN];   // each warp's rows: B | C in fp32
+  float2 dd[kWarps][kTs][kCh];     // (Delta, Delta u)
+  float2 gg[kWarps][kTs][kCh];     // (gate, D u gate)
+  float4 E[2][kWarps][2][32];      // entry states [chunk parity][warp slot][state quad][lane]
+  uint64_t full[S];                // stage landed (TMA transaction count)
+  uint64_t sfree[S];               // every warp converted the stage's chunk (8 arrivals)
+  uint64_t ydone[kYBuf];           // every warp wrote its y rows (8 arrivals)
+  uint64_t eready[kWarps];         // entry state of slot w published (32 arrivals)
+  int abort;
 };
 
 __device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
 
+template <typename T>
+__device__ __forceinline__ void load4(const T* p, float* f) {
+  if constexpr (sizeof(T) == 2) {
+    const uint2 v = *reinterpret_cast<const uint2*>(p);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.y));
+    f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
+  } else {
+    const float4 v = *reinterpret_cast<const float4*>(p);
+    f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+  }
+}
+
 template <typename T, bool kSoftplus, bool kHasZ>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     scan_chunked_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_dt,
                         const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_B,
                         const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ CUtensorMap tm_y,
                         const float* __restrict__ A_log, const float* __restrict__ dt_bias,
                         const float* __restrict__ Dskip, const float* __restrict__ h0, float* __restrict__ hT,
                         int L, int D, int* err, int stop_chunk, uint64_t wait_limit_ns) {
+  constexpr int S = ScanCfg<T>::kStages;
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  ScanSmem<T>& S = *reinterpret_cast<ScanSmem<T>*>(smem_raw + smem_align_pad(smem_raw, 128));
+  ScanSmem<T>& Sm = *reinterpret_cast<ScanSmem<T>*>(smem_raw + smem_align_pad(smem_raw, 128));
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
+  const int ch = lane & 15;   // channel within the CTA
+  const int hf = lane >> 4;   // state half
   const int d0 = blockIdx.x * kCh;
   const int b = blockIdx.y;
-  const int d = d0 + lane;
+  const int d = d0 + ch;
   const int nchunk = (L + kChunk - 1) / kChunk;
+  const bool producer = warp == kWarps - 1 && lane == 0;
 
   constexpr uint32_t kStageBytes = (3 * kChunk * kCh + 2 * kChunk * kN) * sizeof(T);
   const uint32_t stage_bytes = kHasZ ? kStageBytes : kStageBytes - kChunk * kCh * sizeof(T);
 
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(&S.full[s], 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&Sm.full[s], 1);
+      mbar_init(&Sm.sfree[s], kWarps);
+    }
+    for (int i = 0; i < kYBuf; ++i) mbar_init(&Sm.ydone[i], kWarps);
+    for (int w = 0; w < kWarps; ++w) mbar_init(&Sm.eready[w], 32);
+    Sm.abort = 0;
     fence_mbar_init();
+  }
+  __syncthreads();
+
+  // Bounded wait that also gives up once another warp of the CTA gave up.
+  auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 0;; ++it) {
+      if (mbar_try_wait(bar, parity)) return true;
+      if ((it & 15u) == 15u) {
+        if (*reinterpret_cast<volatile int*>(&Sm.abort)) return false;
+        if (globaltimer_ns() - t0 > wait_limit_ns) {
+          raise_error(err, kErrTimeout);
+          *reinterpret_cast<volatile int*>(&Sm.abort) = 1;
+          return false;
+        }
+      }
+    }
+  };
+
+  int issued = 0;  // chunks whose loads the producer issued
+  auto issue = [&](int c) {
+    if (c >= stop_chunk || c >= nchunk) return;  // failure-detection test hook: nothing issued past stop
+    const int s = c % S;
+    const int t0 = c * kChunk;
+    mbar_arrive_expect_tx(&Sm.full[s], stage_bytes);
+    tma_load_3d(Sm.u[s], &tm_u, &Sm.full[s], d0, t0, b);
+    tma_load_3d(Sm.dt[s], &tm_dt, &Sm.full[s], d0, t0, b);
+    if (kHasZ) tma_load_3d(Sm.z[s], &tm_z, &Sm.full[s], d0, t0, b);
+    tma_load_3d(Sm.Bm[s], &tm_B, &Sm.full[s], 0, t0, b);
+    tma_load_3d(Sm.Cm[s], &tm_C, &Sm.full[s], 0, t0, b);
+    issued = c + 1;
+  };
+  if (producer) {
     tma_prefetch_desc(&tm_u);
     tma_prefetch_desc(&tm_dt);
     tma_prefetch_desc(&tm_B);
     tma_prefetch_desc(&tm_C);
     tma_prefetch_desc(&tm_y);
     if (kHasZ) tma_prefetch_desc(&tm_z);
+    for (int c = 0; c < S; ++c) issue(c);
   }
-  __syncthreads();
 
-  auto issue = [&](int c) {
-    if (c >= stop_chunk) return;  // failure-detection test hook: nothing issued past here
-    const int s = c % kStages;
-    const int t0 = c * kChunk;
-    mbar_arrive_expect_tx(&S.full[s], stage_bytes);
-    tma_load_3d(S.u[s], &tm_u, &S.full[s], d0, t0, b);
-    tma_load_3d(S.dt[s], &tm_dt, &S.full[s], d0, t0, b);
-    if (kHasZ) tma_load_3d(S.z[s], &tm_z, &S.full[s], d0, t0, b);
-    tma_load_3d(S.Bm[s], &tm_B, &S.full[s], 0, t0, b);
-    tma_load_3d(S.Cm[s], &tm_C, &S.full[s], 0, t0, b);
-  };
-  // wait for chunk c's stage, then convert its B and C to fp32 (one element per thread pass)
-  auto arrive_chunk = [&](int c) -> bool {
-    const int s = c % kStages;
-    const bool ok = mbar_wait(&S.full[s], (c / kStages) & 1, err, wait_limit_ns);
-    if (ok) {
-      // 64 rows x (16 B | 16 C) = 256 runs of 8 values: one per thread
-      static_assert(kChunk * 4 == kThreads, "one 8-value run of B or C per thread");
-      const int row = tid >> 2, part = tid & 3;
-      const T* src = (part < 2 ? S.Bm[s] : S.Cm[s]) + row * kN + (part & 1) * 8;
+  // Walk constants: A * log2(e) for this lane's 8 states, as pairs.
+  float2 A2[kHalf / 2];
+#pragma unroll
+  for (int k = 0; k < kHalf / 2; ++k) {
+    const float* a = A_log + (size_t)d * kN + hf * kHalf + 2 * k;
+    A2[k] = make_float2(-expf(a[0]) * 1.4426950408889634f, -expf(a[1]) * 1.4426950408889634f);
+  }
+  // Conversion-role constants: row pr of the warp slice, channels pc .. pc + 3.
+  const int pr = lane >> 2, pc = (lane & 3) * 4;
+  float bias4[4], D4[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    bias4[j] = dt_bias ? dt_bias[d0 + pc + j] : 0.f;
+    D4[j] = Dskip ? Dskip[d0 + pc + j] : 0.f;
+  }
+
+  bool ok = true;
+  int consumed = 0;  // chunks whose stage this warp saw land
+  for (int c = 0; c < nchunk && ok; ++c) {
+    const int s = c % S;
+    // ---- this warp's rows of chunk c: wait for the stage, convert once
+    // (every decision to stop is taken by the whole warp, so that no lane
+    // leaves the loop while the others still meet at a warp barrier)
+    if (!__all_sync(0xffffffffu, wait(&Sm.full[s], (c / S) & 1))) { ok = false; break; }
+    consumed = c + 1;
+    {
+      const int row = warp * kTs + pr;
+      const int tg = c * kChunk + row;
+      float uu[4], dv[4], zz[4];
+      load4(Sm.u[s] + row * kCh + pc, uu);
+      load4(Sm.dt[s] + row * kCh + pc, dv);
+      if (kHasZ) load4(Sm.z[s] + row * kCh + pc, zz);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float delta = dv[j] + bias4[j];
+        if (kSoftplus) {
+          if constexpr (sizeof(T) == 4) delta = softplus_acc(delta);
+          else delta = softplus_fast(delta);
+        }
+        float uv = uu[j];
+        if (tg >= L) { delta = 0.f; uv = 0.f; }  // padding past the sequence: state unchanged
+        float g = 1.f;
+        if (kHasZ) {
+          if constexpr (sizeof(T) == 4) g = zz[j] * sigmoid_acc(zz[j]);
+          else g = zz[j] * sigmoid_fast(zz[j]);
+        }
+        Sm.dd[warp][pr][pc + j] = make_float2(delta, delta * uv);
+        Sm.gg[warp][pr][pc + j] = make_float2(g, D4[j] * uv * g);
+      }
+      // B | C of the 8 rows: 4 runs of 8 values per row, one run per lane
+      const int part = lane & 3;
+      const T* src = (part < 2 ? Sm.Bm[s] : Sm.Cm[s]) + row * kN + (part & 1) * 8;
       float f[8];
       load8(src, f);
-      float4* dst = reinterpret_cast<float4*>(&S.BC[c & 1][row][part * 8]);
+      float4* dst = reinterpret_cast<float4*>(&Sm.BC[warp][pr][part * 8]);
       dst[0] = make_float4(f[0], f[1], f[2], f[3]);
       dst[1] = make_float4(f[4], f[5], f[6], f[7]);
     }
-    return ok;
-  };
-  if (tid == 0)
-    for (int c = 0; c < kStages - 1 && c < nchunk; ++c) issue(c);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&Sm.sfree[s]);
+    if (warp == kWarps - 1) {
+      bool pok = true;
+      if (producer && c + S < nchunk) {  // recycle the stage once every warp converted it
+        pok = wait(&Sm.sfree[s], (c / S) & 1);
+        if (pok) issue(c + S);
+      }
+      if (!__shfl_sync(0xffffffffu, pok, 0)) { ok = false; break; }
+    }
 
-  // Per-lane constants: A * log2(e), as pairs of states.
-  float2 A2[kN / 2];
+    // ---- walk 1: local scan from zero, decays cached
+    float2 dA[kTs][kHalf / 2];
+    float2 h[kHalf / 2];
 #pragma unroll
-  for (int n = 0; n < kN / 2; ++n)
-    A2[n] = make_float2(-expf(A_log[(size_t)d * kN + 2 * n]) * 1.4426950408889634f,
-                        -expf(A_log[(size_t)d * kN + 2 * n + 1]) * 1.4426950408889634f);
-  const float bias = dt_bias ? dt_bias[d] : 0.f;
-  const float Dd = Dskip ? Dskip[d] : 0.f;
-
-  // Combine-role ownership: channel cl, states cn and cn+1; their carries.
-  const int cl = tid & 31;
-  const int cn = (tid >> 5) * 2;
-  float carry[2];
-#pragma unroll
-  for (int j = 0; j < 2; ++j) carry[j] = h0 ? h0[((size_t)b * D + d0 + cl) * kN + cn + j] : 0.f;
-
-  bool ok = nchunk > 0 ? __syncthreads_and(arrive_chunk(0)) : true;
-  for (int c = 0; c < nchunk && ok; ++c) {
-    const int s = c % kStages;
-    if (tid == 0 && c + kStages - 1 < nchunk) issue(c + kStages - 1);
-    const float* BC = &S.BC[c & 1][0][0];
-
-    const int tb = warp * kTs;       // first token of this warp within the chunk
-    const int tg = c * kChunk + tb;  // global index of that token
-    float2 dA[kTs][kN / 2];
-    float du[kTs];
-    float2 h[kN / 2];
-#pragma unroll
-    for (int n = 0; n < kN / 2; ++n) h[n] = make_float2(0.f, 0.f);
-
-    // ---- walk 1: local scan from zero, decays cached (pairs of states per FMA2)
+    for (int k = 0; k < kHalf / 2; ++k) h[k] = make_float2(0.f, 0.f);
 #pragma unroll
     for (int i = 0; i < kTs; ++i) {
-      const int row = tb + i;
-      const float dtv = Elt<T>::to_f(S.dt[s][row * kCh + lane]) + bias;
-      float delta;
-      if (kSoftplus) {
-        if constexpr (sizeof(T) == 4) delta = softplus_acc(dtv);
-        else delta = softplus_fast(dtv);
-      } else {
-        delta = dtv;
+      const float2 dl = Sm.dd[warp][i][ch];
+      const float2 dlt = f2(dl.x), du = f2(dl.y);
+      const float4* Bp = reinterpret_cast<const float4*>(&Sm.BC[warp][i][hf * kHalf]);
+      const float4 b0 = Bp[0], b1 = Bp[1];
+      const float2 bq[4] = {make_float2(b0.x, b0.y), make_float2(b0.z, b0.w), make_float2(b1.x, b1.y),
+                            make_float2(b1.z, b1.w)};
+#pragma unroll
+      for (int k = 0; k < kHalf / 2; ++k) {
+        const float2 x = __fmul2_rn(dlt, A2[k]);
+        dA[i][k] = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+        h[k] = __ffma2_rn(dA[i][k], h[k], __fmul2_rn(du, bq[k]));
       }
-      float uv = Elt<T>::to_f(S.u[s][row * kCh + lane]);
-      if (tg + i >= L) { delta = 0.f; uv = 0.f; }
-      du[i] = delta * uv;
-      const float2 dl = f2(delta), dd = f2(du[i]);
-      const float4* Bp = reinterpret_cast<const float4*>(BC + row * 2 * kN);
+    }
+    float2 P[kHalf / 2];
 #pragma unroll
-      for (int q = 0; q < kN / 4; ++q) {
-        const float4 Bq = Bp[q];
+    for (int k = 0; k < kHalf / 2; ++k) {
+      P[k] = dA[0][k];
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int n = 2 * q + hh;
-          const float2 x = __fmul2_rn(dl, A2[n]);
-          dA[i][n] = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-          const float2 bu = __fmul2_rn(dd, hh ? make_float2(Bq.z, Bq.w) : make_float2(Bq.x, Bq.y));
-          h[n] = __ffma2_rn(dA[i][n], h[n], bu);
+      for (int i = 1; i < kTs; ++i) P[k] = __fmul2_rn(P[k], dA[i][k]);
+    }
+
+    // ---- carry chain: entry state of this slice, hand the next one on
+    float2 e[kHalf / 2];
+    if (c == 0 && warp == 0) {
+#pragma unroll
+      for (int k = 0; k < kHalf / 2; ++k) {
+        if (h0) {
+          const float* hp = h0 + ((size_t)b * D + d) * kN + hf * kHalf + 2 * k;
+          e[k] = make_float2(hp[0], hp[1]);
+        } else {
+          e[k] = make_float2(0.f, 0.f);
+        }
+      }
+    } else {
+      const uint32_t par = warp == 0 ? ((c - 1) & 1) : (c & 1);
+      if (!__all_sync(0xffffffffu, wait(&Sm.eready[warp], par))) { ok = false; break; }
+      const float4 q0 = Sm.E[c & 1][warp][0][lane], q1 = Sm.E[c & 1][warp][1][lane];
+      e[0] = make_float2(q0.x, q0.y);
+      e[1] = make_float2(q0.z, q0.w);
+      e[2] = make_float2(q1.x, q1.y);
+      e[3] = make_float2(q1.z, q1.w);
+    }
+    {
+      float2 en[kHalf / 2];
+#pragma unroll
+      for (int k = 0; k < kHalf / 2; ++k) en[k] = __ffma2_rn(P[k], e[k], h[k]);
+      if (warp < kWarps - 1 || c + 1 < nchunk) {
+        const int nw = warp < kWarps - 1 ? warp + 1 : 0;
+        const int np = warp < kWarps - 1 ? (c & 1) : ((c + 1) & 1);
+        Sm.E[np][nw][0][lane] = make_float4(en[0].x, en[0].y, en[1].x, en[1].y);
+        Sm.E[np][nw][1][lane] = make_float4(en[2].x, en[2].y, en[3].x, en[3].y);
+        mbar_arrive(&Sm.eready[nw]);
+      } else if (hT) {  // the state after the last token
+        float* hp = hT + ((size_t)b * D + d) * kN + hf * kHalf;
+#pragma unroll
+        for (int k = 0; k < kHalf / 2; ++k) {
+          hp[2 * k] = en[k].x;
+          hp[2 * k + 1] = en[k].y;
         }
       }
     }
-#pragma unroll
-    for (int n = 0; n < kN / 2; ++n) {
-      float2 p = dA[0][n];
-#pragma unroll
-      for (int i = 1; i < kTs; ++i) p = __fmul2_rn(p, dA[i][n]);
-      S.aggP[warp][2 * n][lane] = p.x;
-      S.aggP[warp][2 * n + 1][lane] = p.y;
-      S.aggH[warp][2 * n][lane] = h[n].x;
-      S.aggH[warp][2 * n + 1][lane] = h[n].y;
-    }
-    __syncthreads();
 
-    // ---- combine across the 8 warps, chained from the previous chunk's carry
-    // (all aggregates are loaded before the first entry state is stored: the
-    // dependent chain is then 8 FMAs, not 8 shared-memory round trips)
+    // ---- walk 2: exact states from the entry state, read-out, gate
+    T* ytile = Sm.y[c % kYBuf];
+    float yp[kTs];
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      float P[kWarps], hl[kWarps];
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        P[w] = S.aggP[w][cn + j][cl];
-        hl[w] = S.aggH[w][cn + j][cl];
-      }
-      float H = carry[j];
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        S.aggH[w][cn + j][cl] = H;
-        H = fmaf(P[w], H, hl[w]);
-      }
-      carry[j] = H;
-    }
-    if (tid == 0) tma_store_wait_read<1>();  // y tile (c & 1) free again
-    __syncthreads();
-
-    // ---- walk 2: exact states from the entry state, outputs
-#pragma unroll
-    for (int n = 0; n < kN / 2; ++n) h[n] = make_float2(S.aggH[warp][2 * n][lane], S.aggH[warp][2 * n + 1][lane]);
-    T* ytile = S.y[c & 1];
+    for (int k = 0; k < kHalf / 2; ++k) h[k] = e[k];
 #pragma unroll
     for (int i = 0; i < kTs; ++i) {
-      const int row = tb + i;
-      const float4* Bp = reinterpret_cast<const float4*>(BC + row * 2 * kN);
-      const float4* Cp = Bp + kN / 4;
-      const float2 dd = f2(du[i]);
-      float2 y2[4];  // four partial sums: the readout is not one serial chain of 8 FMAs
+      const float2 du = f2(Sm.dd[warp][i][ch].y);
+      const float4* Bp = reinterpret_cast<const float4*>(&Sm.BC[warp][i][hf * kHalf]);
+      const float4* Cp = reinterpret_cast<const float4*>(&Sm.BC[warp][i][kN + hf * kHalf]);
+      const float4 b0 = Bp[0], b1 = Bp[1], c0 = Cp[0], c1 = Cp[1];
+      const float2 bq[4] = {make_float2(b0.x, b0.y), make_float2(b0.z, b0.w), make_float2(b1.x, b1.y),
+                            make_float2(b1.z, b1.w)};
+      const float2 cq[4] = {make_float2(c0.x, c0.y), make_float2(c0.z, c0.w), make_float2(c1.x, c1.y),
+                            make_float2(c1.z, c1.w)};
 #pragma unroll
-      for (int q = 0; q < kN / 4; ++q) {
-        const float4 Bq = Bp[q];
-        const float4 Cq = Cp[q];
+      for (int k = 0; k < kHalf / 2; ++k) h[k] = __ffma2_rn(dA[i][k], h[k], __fmul2_rn(du, bq[k]));
+      const float2 ya = __ffma2_rn(cq[1], h[1], __fmul2_rn(cq[0], h[0]));
+      const float2 yb = __ffma2_rn(cq[3], h[3], __fmul2_rn(cq[2], h[2]));
+      const float2 ys = __fadd2_rn(ya, yb);
+      yp[i] = ys.x + ys.y;
+    }
+    // the two lanes of a channel: lane half 0 finishes the even token of each
+    // pair, half 1 the odd one (one shuffle per pair)
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int n = 2 * q + hh;
-          const float2 bu = __fmul2_rn(dd, hh ? make_float2(Bq.z, Bq.w) : make_float2(Bq.x, Bq.y));
-          h[n] = __ffma2_rn(dA[i][n], h[n], bu);
-          const float2 cq = hh ? make_float2(Cq.z, Cq.w) : make_float2(Cq.x, Cq.y);
-          y2[q] = hh ? __ffma2_rn(cq, h[n], y2[q]) : __fmul2_rn(cq, h[n]);
-        }
-      }
-      const float2 ya = __fadd2_rn(__fadd2_rn(y2[0], y2[1]), __fadd2_rn(y2[2], y2[3]));
-      float y = ya.x + ya.y;
-      const float uv = Elt<T>::to_f(S.u[s][row * kCh + lane]);
-      y = fmaf(Dd, uv, y);
-      if (kHasZ) {
-        const float zv = Elt<T>::to_f(S.z[s][row * kCh + lane]);
-        if constexpr (sizeof(T) == 4) y *= zv * sigmoid_acc(zv);
-        else y *= zv * sigmoid_fast(zv);
-      }
-      ytile[row * kCh + lane] = Elt<T>::from_f(y);
+    for (int i = 0; i < kTs; i += 2) {
+      const float send = hf ? yp[i] : yp[i + 1];
+      const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
+      const int ti = i + hf;
+      const float ysum = (hf ? yp[i + 1] : yp[i]) + recv;
+      const float2 g = Sm.gg[warp][ti][ch];
+      ytile[(warp * kTs + ti) * kCh + ch] = Elt<T>::from_f(fmaf(ysum, g.x, g.y));
     }
     fence_proxy_async_smem();
-    // next chunk's stage has (usually) landed: convert its B and C while we are here
-    bool nxt = true;
-    if (c + 1 < nchunk) nxt = arrive_chunk(c + 1);
-    ok = __syncthreads_and(nxt);
-    if (tid == 0) {
-      tma_store_3d(&tm_y, ytile, d0, c * kChunk, b);
-      tma_store_commit();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&Sm.ydone[c % kYBuf]);
+    if (warp == kWarps - 1) {
+      bool pok = true;
+      if (producer) {  // every warp wrote its rows: store the tile
+        pok = wait(&Sm.ydone[c % kYBuf], (c / kYBuf) & 1);
+        if (pok) {
+          tma_store_3d(&tm_y, ytile, d0, c * kChunk, b);
+          tma_store_commit();
+          tma_store_wait_read<1>();  // the tile of chunk c - 1 has been read: reusable at chunk c + 2
+        }
+      }
+      if (!__shfl_sync(0xffffffffu, pok, 0)) { ok = false; break; }
     }
+    __syncwarp();
   }
-  if (tid == 0) tma_store_wait_all<0>();
-  if (ok && hT) {
-#pragma unroll
-    for (int j = 0; j < 2; ++j) hT[((size_t)b * D + d0 + cl) * kN + cn + j] = carry[j];
+  if (producer) {
+    tma_store_wait_all<0>();
+    // after a timeout, loads still in flight must land before the CTA leaves
+    for (int c = consumed; c < issued; ++c) {
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(&Sm.full[c % S], (c / S) & 1))
+        if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+    }
   }
 }
 

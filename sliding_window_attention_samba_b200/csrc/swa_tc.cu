@@ -857,6 +857,292 @@ __global__ void __launch_bounds__(A2_THREADS, 1) swa_tc2_kernel(const __grid_con
   }
 }
 
+// ---------------------------------------------------------------------------
+// Four query heads per CTA (four heads of one kv group at the same 128 query
+// rows), 64-key tiles.  Sixteen softmax warps (four per head, one per TMEM lane
+// quadrant) keep the exponential unit fed while any one head waits on its
+// matrix products; every K/V tile is read once for four heads.
+//   warp 0      TMA: Q of the four heads, then K_j / V_j (64 keys, 4 stages)
+//   warp 1      TMEM owner + MMA issuer.  It issues, per head and as soon as
+//               its inputs are ready (polled, no fixed head order),
+//               S_h(j) = Q_h K_j^T (M128 N64 K16 x4) and O_h += P_h(j) V_j
+//               (M128 N64 K16 x4); a K/V stage is released once all four
+//               heads' products of its tile completed.
+//   warps 2..17 softmax of head (warp - 2) / 4, query row = TMEM lane: the 64
+//               scores of a tile in registers, band mask on edge tiles, online
+//               max with lazy O rescale (> 2^8), P as bf16 into 128B-swizzled
+//               shared memory, one pair in four of the exponentials on the FMA
+//               pipe.
+// TMEM: S_h at columns 64h, O_h at 256 + 64h.
+constexpr int A4_HEADS = 4;
+constexpr int A4_BN = 64;
+constexpr int A4_STAGES = 4;
+constexpr int A4_THREADS = (2 + 4 * A4_HEADS) * 32;
+constexpr uint32_t kKV64Bytes = A4_BN * AT_D * 2;  // 8 KB
+
+struct At4Smem {
+  bf16 Q[A4_HEADS][AT_BM * AT_D];
+  bf16 K[A4_STAGES][A4_BN * AT_D];
+  bf16 V[A4_STAGES][A4_BN * AT_D];
+  bf16 P[A4_HEADS][AT_BM * A4_BN];  // [row][64 keys], 128B-swizzled
+  uint64_t q_full;
+  uint64_t kv_full[A4_STAGES], kv_empty[A4_STAGES];
+  uint64_t s_full[A4_HEADS], s_free[A4_HEADS], p_full[A4_HEADS], pv_done[A4_HEADS];
+  uint32_t tmem_base;
+};
+
+template <int kPolyPairs>
+__global__ void __launch_bounds__(A4_THREADS, 1) swa_tc4_kernel(const __grid_constant__ AtParams p, int* err) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  At4Smem& S = *reinterpret_cast<At4Smem*>(smem_raw + smem_align_pad(smem_raw, 1024));
+  const int warp = warp_id_sync();
+  const int lane = threadIdx.x & 31;
+  const int t0 = blockIdx.x * AT_BM;
+  const int h0 = blockIdx.y * A4_HEADS;
+  const int b = blockIdx.z;
+  const int g = h0 / (p.Hq / p.Hkv);
+  const int tk0 = t0 + p.qoff;  // key row of query row t0
+  const int lo = tk0 - p.window + 1;
+  const int kb0 = lo <= 0 ? 0 : (lo / A4_BN) * A4_BN;
+  const int ntile = (min(tk0 + AT_BM - 1, p.Lk - 1) - kb0) / A4_BN + 1;
+
+  if (warp == 0 && lane == 0) {
+    mbar_init(&S.q_full, 1);
+    for (int s = 0; s < A4_STAGES; ++s) {
+      mbar_init(&S.kv_full[s], 1);
+      mbar_init(&S.kv_empty[s], 1);
+    }
+    for (int i = 0; i < A4_HEADS; ++i) {
+      mbar_init(&S.s_full[i], 1);
+      mbar_init(&S.s_free[i], 4);
+      mbar_init(&S.p_full[i], 4);
+      mbar_init(&S.pv_done[i], 1);
+    }
+    fence_mbar_init();
+    tma_prefetch_desc(&p.tmQ);
+    tma_prefetch_desc(&p.tmK);
+    tma_prefetch_desc(&p.tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(&S.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+
+  if (warp == 0) {
+    if (elect_one()) {
+      mbar_arrive_expect_tx(&S.q_full, A4_HEADS * kTileBytes);
+      for (int hh = 0; hh < A4_HEADS; ++hh)
+        tma_load_3d(S.Q[hh], &p.tmQ, &S.q_full, (h0 + hh) * AT_D, t0, b);
+      for (int j = 0; j < ntile; ++j) {
+        const int s = j % A4_STAGES;
+        if (!mbar_wait(&S.kv_empty[s], ((j / A4_STAGES) & 1) ^ 1, err)) break;
+        mbar_arrive_expect_tx(&S.kv_full[s], 2 * kKV64Bytes);
+        const int kb = kb0 + j * A4_BN;
+        tma_load_3d(S.K[s], &p.tmK, &S.kv_full[s], g * AT_D, kb, b);
+        tma_load_3d(S.V[s], &p.tmV, &S.kv_full[s], g * AT_D, kb, b);
+      }
+    }
+  } else if (warp == 1) {
+    const uint32_t idesc_s = idesc_bf16_f32(AT_BM, A4_BN, false);
+    const uint32_t idesc_o = idesc_bf16_f32(AT_BM, AT_D, true);  // V is N-contiguous (MN-major B)
+    if (elect_one()) {
+      bool ok = mbar_wait(&S.q_full, 0, err);
+      int ns[A4_HEADS], npv[A4_HEADS], cnt[A4_STAGES];
+      for (int i = 0; i < A4_HEADS; ++i) ns[i] = npv[i] = 0;
+      for (int i = 0; i < A4_STAGES; ++i) cnt[i] = 0;
+      uint64_t t_last = globaltimer_ns();
+      while (ok) {
+        bool done = true, progress = false;
+#pragma unroll
+        for (int hh = 0; hh < A4_HEADS; ++hh) {
+          const int j = ns[hh];
+          if (j < ntile) {
+            done = false;
+            const int s = j % A4_STAGES;
+            if (mbar_test(&S.kv_full[s], (j / A4_STAGES) & 1) &&
+                (j == 0 || mbar_test(&S.s_free[hh], (j - 1) & 1))) {
+              tc_fence_after();
+              const uint32_t q_base = smem_u32(S.Q[hh]);
+              const uint32_t k_base = smem_u32(S.K[s]);
+#pragma unroll
+              for (int k = 0; k < AT_D / 16; ++k)
+                umma_f16_ss(tmem + hh * 64u, smem_desc(q_base + k * 32, 16, 1024, kLayoutSw128),
+                            smem_desc(k_base + k * 32, 16, 1024, kLayoutSw128), idesc_s, k != 0);
+              umma_commit(&S.s_full[hh]);
+              ns[hh] = j + 1;
+              progress = true;
+            }
+          }
+          const int jp = npv[hh];
+          if (jp < ntile) {
+            done = false;
+            if (jp < ns[hh] && mbar_test(&S.p_full[hh], jp & 1)) {
+              tc_fence_after();
+              const int s = jp % A4_STAGES;
+              const uint32_t a_base = smem_u32(S.P[hh]);
+              const uint32_t v_base = smem_u32(S.V[s]);
+#pragma unroll
+              for (int k = 0; k < A4_BN / 16; ++k)
+                umma_f16_ss(tmem + 256u + hh * 64u, smem_desc(a_base + k * 32, 16, 1024, kLayoutSw128),
+                            smem_desc(v_base + k * 16 * AT_D * 2, 16, 1024, kLayoutSw128), idesc_o,
+                            (jp | k) != 0);
+              umma_commit(&S.pv_done[hh]);
+              // the K/V stage of tile jp is released once all four heads' products
+              // of that tile are issued (they complete in issue order)
+              int c4 = 0;
+#pragma unroll
+              for (int i = 0; i < A4_STAGES; ++i)
+                if (i == s) c4 = ++cnt[i];
+              if (c4 == A4_HEADS) {
+#pragma unroll
+                for (int i = 0; i < A4_STAGES; ++i)
+                  if (i == s) cnt[i] = 0;
+                umma_commit(&S.kv_empty[s]);
+              }
+              npv[hh] = jp + 1;
+              progress = true;
+            }
+          }
+        }
+        if (done) break;
+        const uint64_t now = globaltimer_ns();
+        if (progress) {
+          t_last = now;
+        } else if (now - t_last > kWaitLimitNs) {
+          raise_error(err, kErrTimeout);
+          ok = false;
+        } else {
+          __nanosleep(32);
+        }
+      }
+    }
+  } else {
+    const int hh = (warp - 2) >> 2;
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;  // query row within the tile == TMEM lane
+    const int tq = t0 + r;
+    const int t = tk0 + r;
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const uint32_t tS = tmem + hh * 64u + lane_off;
+    const uint32_t tO = tmem + 256u + hh * 64u + lane_off;
+    auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
+      const bool w = mbar_wait(bar, par, err);
+      return __all_sync(0xffffffffu, w);
+    };
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+    for (int j = 0; j < ntile; ++j) {
+      const int kb = kb0 + j * A4_BN;
+      if (!wait_all(&S.s_full[hh], j & 1)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sr[64];
+      tmem_ld32(tS, sr);
+      tmem_ld32(tS + 32, sr + 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.s_free[hh]);
+      // band mask on the edge tiles: valid key offsets of row t are (t - w - kb, t - kb]
+      const bool edge = (kb + A4_BN - 1 > tk0) || (kb < tk0 + AT_BM - p.window);
+      if (edge) {
+        const int hi = tq < p.L ? t - kb : -1;
+        const int lo_i = t - p.window - kb;
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+          if (i > hi || i <= lo_i) sr[i] = __float_as_uint(-INFINITY);
+      }
+      float m8[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 64; i += 2)
+        m8[(i >> 1) & 7] = fmax3(m8[(i >> 1) & 7], __uint_as_float(sr[i]), __uint_as_float(sr[i + 1]));
+      const float mraw = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      const float mt = mraw * p.scale_log2;
+      const bool need = mt > m_run + kRescaleThresh;
+      float alpha = 1.f;
+      if (need) {
+        if (m_run != -INFINITY) alpha = exp2f(m_run - mt);
+        l_run *= alpha;
+        m_run = mt;
+      }
+      // O_h += P_h(j-1) V_{j-1} must be complete before O is rescaled and P rewritten
+      if (j >= 1 && !wait_all(&S.pv_done[hh], (j - 1) & 1)) { ok = false; break; }
+      tc_fence_after();
+      if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t orr[16];
+          tmem_ld16(tO + c * 16, orr);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
+          tmem_st16(tO + c * 16, orr);
+        }
+        tmem_wait_st();
+      }
+      const float msub = m_run == -INFINITY ? 0.f : m_run;
+      const float2 nm2 = make_float2(-msub, -msub);
+      float2 ls2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      unsigned char* prow = reinterpret_cast<unsigned char*>(S.P[hh]) + r * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {  // 16-byte chunk c holds keys 8c .. 8c + 7
+        float e[8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int i = c * 8 + 2 * q;
+          const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), sc2, nm2);
+          if (q < kPolyPairs) {
+            const float2 y = exp2_poly2(x);
+            e[2 * q] = y.x;
+            e[2 * q + 1] = y.y;
+          } else {
+            e[2 * q] = ex2_approx(x.x);
+            e[2 * q + 1] = ex2_approx(x.y);
+          }
+          ls2[q] = __fadd2_rn(ls2[q], make_float2(e[2 * q], e[2 * q + 1]));
+        }
+        *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) =
+            make_uint4(pack_bf16(e[0], e[1]), pack_bf16(e[2], e[3]), pack_bf16(e[4], e[5]), pack_bf16(e[6], e[7]));
+      }
+      l_run += ((ls2[0].x + ls2[0].y) + (ls2[1].x + ls2[1].y)) + ((ls2[2].x + ls2[2].y) + (ls2[3].x + ls2[3].y));
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.p_full[hh]);
+    }
+    if (ok && wait_all(&S.pv_done[hh], (ntile - 1) & 1)) {
+      tc_fence_after();
+      uint32_t orr[64];
+      tmem_ld32(tO, orr);
+      tmem_ld32(tO + 32, orr + 32);
+      tmem_wait_ld();
+      if (tq < p.L && l_run > 0.f) {
+        const float inv = 1.f / l_run;
+        bf16* op = p.o + ((int64_t)b * p.L + tq) * p.ld_o + (int64_t)(h0 + hh) * AT_D;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          float f[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) f[q] = __uint_as_float(orr[c * 8 + q]) * inv;
+          store8(op + c * 8, f);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 // [B, L, H * d] rows of stride ld; boxes of 64 columns x `rows` rows (128B swizzle)
 bool make_head_map(CUtensorMap* m, const void* base, int64_t ld, int H, int d, int L, int B, int rows) {
   uint64_t dims[3] = {(uint64_t)H * d, (uint64_t)L, (uint64_t)B};
@@ -902,7 +1188,26 @@ samba_status launch_swa_tc(const SwaArgs& a, cudaStream_t st) {
     SAMBA_CHECK_LAUNCH();
     return SAMBA_OK;
   }
-  if (grp % 2 == 0 && !(getenv("SAMBA_SWA_KERNEL") && getenv("SAMBA_SWA_KERNEL")[0] == '1')) {
+  const char* kenv = getenv("SAMBA_SWA_KERNEL");
+  if (grp % A4_HEADS == 0 && !(kenv && (kenv[0] == '1' || kenv[0] == '2'))) {
+    CUtensorMap tk, tv;
+    if (!make_head_map(&tk, a.k, a.ld_k, a.Hkv, a.d, Lk, a.B, A4_BN) ||
+        !make_head_map(&tv, a.v, a.ld_v, a.Hkv, a.d, Lk, a.B, A4_BN))
+      return SAMBA_ERR_CUDA;
+    p.tmK = tk;
+    p.tmV = tv;
+    const char* pe = getenv("SAMBA_SWA_POLY");
+    const int poly = (pe && pe[0] >= '0' && pe[0] <= '3') ? pe[0] - '0' : 1;
+    auto kern = poly == 0 ? swa_tc4_kernel<0> : poly == 2 ? swa_tc4_kernel<2> : poly == 3 ? swa_tc4_kernel<3>
+                                                                                            : swa_tc4_kernel<1>;
+    const size_t smem = sizeof(At4Smem) + 1024;
+    if (!ensure_smem_attr(kern, smem)) return SAMBA_ERR_CUDA;
+    dim3 grid((a.L + AT_BM - 1) / AT_BM, a.Hq / A4_HEADS, a.B);
+    kern<<<grid, A4_THREADS, smem, st>>>(p, device_error_word());
+    SAMBA_CHECK_LAUNCH();
+    return SAMBA_OK;
+  }
+  if (grp % 2 == 0 && !(kenv && kenv[0] == '1')) {
     // share of the exponentials on the FMA pipe: SAMBA_SWA_POLY = 0..3 pairs of 4 (default 1)
     const char* pe = getenv("SAMBA_SWA_POLY");
     const int poly = (pe && pe[0] >= '0' && pe[0] <= '3') ? pe[0] - '0' : 1;

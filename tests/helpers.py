@@ -7,14 +7,23 @@ denominator floored at the reference tensor's RMS,
     elem_err(g, o) = max_i |g_i - o_i| / max(|o_i|, rms(o)),
 
 reported together with the normwise ||g - o||_2 / ||o||_2; `rel_err` is the
-larger of the two and is the metric of every path except attention over
-RoPE-rotated bf16 queries and keys.
+larger of the two.  It is the metric of every single operation (RMSNorm, the
+short convolution, every projection epilogue, the selective scan, attention
+without RoPE) and of every fp32 path.
 
-There (`attn_err`) the elementwise form measures the bf16 rounding of the
-rotated q and k that any bf16 tensor-core attention performs, not the kernel:
-that rounding alone gives 4.6% on N(0,1) inputs against 0.28% l-infinity
-relative and 0.27% normwise, so attention outputs are held to
-max(l-inf relative, normwise).
+Two kinds of bf16 output are held to max(l-infinity relative, normwise)
+instead (`chain_err`), because there the elementwise form measures the bf16
+storage of intermediate tensors, which the path's data layout fixes, and not
+the kernels:
+  * attention over RoPE-rotated bf16 queries and keys: the bf16 rounding of
+    the rotated q and k alone gives 4.6% elementwise on N(0,1) inputs against
+    0.28% l-infinity relative and 0.27% normwise;
+  * composite bf16 paths whose intermediates are stored in bf16 before the
+    next step reads them (a block's branches and stream, the SSM state, a
+    stack's logits): with exact (fp64) arithmetic and only that storage
+    rounding, the 2048-wide Mamba branch is off by 2.1% elementwise (0.42%
+    normwise), its scan output by 5.1% and its final state by 7.6% (0.49%),
+    the SwiGLU branch by 1.6% on 256 tokens (0.35%).
 
 Where a check compares a difference S - a against a small b (the branch a
 residual epilogue adds, a decode step's contribution y - x) and S is stored in
@@ -71,11 +80,26 @@ def _norm_err_slack(g, o, slack) -> float:
     return float(np.linalg.norm(d) / max(np.linalg.norm(o), 1e-300))
 
 
-def attn_err(g, o) -> float:
-    """max(l-infinity relative, normwise): attention over RoPE-rotated bf16 q/k."""
-    if np.asarray(o).size == 0:
+def chain_err(g, o, slack=None) -> float:
+    """max(l-infinity relative, normwise): attention over RoPE-rotated bf16 q/k
+    and composite bf16 paths with bf16-stored intermediates."""
+    g, o = _arr(g), _arr(o)
+    if o.size == 0:
         return 0.0
-    return max(linf_rel(g, o), norm_err(g, o))
+    d = np.abs(g - o)
+    if slack is not None:
+        d = np.maximum(d - _arr(slack), 0.0)
+    return max(float(np.max(d) / max(float(np.max(np.abs(o))), 1e-300)),
+               float(np.linalg.norm(d) / max(np.linalg.norm(o), 1e-300)))
+
+
+attn_err = chain_err
+
+
+def path_err(g, o, dt: str, slack=None) -> float:
+    """A composite path's output: the elementwise metric in fp32, the chain
+    reading in bf16."""
+    return rel_err(g, o, slack) if dt == "f32" else chain_err(g, o, slack)
 
 
 def half_ulp(x, dt: str) -> np.ndarray:

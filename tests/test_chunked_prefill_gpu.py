@@ -11,7 +11,7 @@ import pytest
 
 from oracle import samba_oracle as O
 from sliding_window_attention_samba_b200 import inputs as I
-from tests.helpers import TOL, block_weights_dev, dev, host, rel_err, stream_slack, sum_slack
+from tests.helpers import TOL, block_weights_dev, dev, host, path_err, rel_err, stream_slack, sum_slack
 from tests.test_block_gpu import branch_err, step_err
 
 pytestmark = pytest.mark.gpu
@@ -80,11 +80,11 @@ def _run_chunks(L, shape, W, x, chunks, tol, steps=2):
             for i in range(4):
                 assert branch_err(i, br[i], ref["branch"][i][:, p:p + Lc], shape.dtype) <= tol, (ci, i)
             res = [r[:, p:p + Lc] for r in ref["resid"]]
-            assert rel_err(out - x[:, p:p + Lc], ref["x_out"][:, p:p + Lc] - x[:, p:p + Lc],
-                           slack=stream_slack(res, shape.dtype)) <= tol, ci
+            assert path_err(out - x[:, p:p + Lc], ref["x_out"][:, p:p + Lc] - x[:, p:p + Lc], shape.dtype,
+                            slack=stream_slack(res, shape.dtype)) <= tol, ci
         p += Lc
     assert np.array_equal(host(g.pos), np.full(Bn, total))
-    assert rel_err(host(g.ssm), refp["ssm"]) <= tol
+    assert path_err(host(g.ssm), refp["ssm"], shape.dtype) <= tol
     assert rel_err(host(g.conv), refp["conv"]) <= tol
     n = min(total, shape.window)
     slots = [(total - n + j) % shape.window for j in range(n)]
@@ -103,12 +103,12 @@ def test_chunked_prefill_tiny_f32(L, chunks):
     _run_chunks(L, shape, W, x, chunks, TOL["f32"])
 
 
-@pytest.mark.parametrize("kernel", ["", "1"])
+@pytest.mark.parametrize("kernel", ["", "2", "1"])
 def test_chunked_prefill_wide_bf16(L, kernel):
     """2048-wide block at B = 1 in chunks of 1000, 1500, 700: the second chunk
     starts 1000 tokens in (1000 earlier keys, not a tile multiple), the third past
-    the window (2047 earlier keys).  kernel "1" runs the one-head-per-CTA
-    tensor-core attention kernel instead of the two-head one."""
+    the window (2047 earlier keys).  kernel "2" / "1" run the two-head / one-head
+    per CTA tensor-core attention kernels instead of the four-head one."""
     shape = I.WIDE
     W = I.block_weights(shape, 8)
     chunks = [1000, 1500, 700]
@@ -149,7 +149,7 @@ def test_chunked_equals_single_call_wide_bf16(L):
     torch.cuda.synchronize()
     one = host(out)
     # both sides store their output in bf16: one half-ulp each
-    assert rel_err(got - x, one - x, slack=sum_slack(one, "bf16", 2)) <= TOL["bf16"]
+    assert path_err(got - x, one - x, "bf16", slack=sum_slack(one, "bf16", 2)) <= TOL["bf16"]
 
 
 def test_chunk_position_mismatch_sets_device_error(L):

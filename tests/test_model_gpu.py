@@ -10,7 +10,7 @@ import pytest
 
 from oracle import samba_oracle as O
 from sliding_window_attention_samba_b200 import inputs as I
-from tests.helpers import TOL, block_weights_dev, dev, host, rel_err
+from tests.helpers import TOL, block_weights_dev, dev, host, path_err, rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -63,7 +63,7 @@ def test_transformer_layout_full_attention_tiny_f32(L):
 
 def test_samba_2to1_stack_wide_bf16(L):
     got, ref = _run(L, I.WIDE, SAMBA_2_1, 1, 2304, 512, 23)
-    assert rel_err(got, ref) <= TOL["bf16"]
+    assert path_err(got, ref, "bf16") <= TOL["bf16"]
     assert int(np.argmax(got[0])) == int(np.argmax(ref[0]))
 
 
@@ -159,7 +159,7 @@ def test_model_step_full_cache_split_attention_bf16(L):
     for t in range(S):
         g.step(ids[:, t])
         if t in (0, 255, 256, 511, 699):
-            assert rel_err(host(g.logits), g.oracle(ids[:, :t + 1])) <= TOL["bf16"], t
+            assert path_err(host(g.logits), g.oracle(ids[:, :t + 1]), "bf16") <= TOL["bf16"], t
 
 
 def test_model_step_graph_replay_bit_exact(L):

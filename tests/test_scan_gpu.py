@@ -44,7 +44,9 @@ def oracle_scan(r, softplus=True, with_z=True, h0=None):
 
 
 @pytest.mark.parametrize("dt,Bn,Ln,D", [("f32", 1, 256, 128), ("f32", 2, 200, 64), ("bf16", 1, 4096, 4096),
-                                        ("bf16", 3, 129, 256), ("bf16", 1, 1, 32), ("f32", 1, 63, 32)])
+                                        ("bf16", 3, 129, 256), ("bf16", 1, 1, 32), ("f32", 1, 63, 32),
+                                        ("bf16", 2, 700, 48), ("f32", 1, 130, 16), ("bf16", 1, 64, 16),
+                                        ("bf16", 1, 65, 16), ("bf16", 1, 4097, 1040)])
 def test_scan_matches_oracle(L, dt, Bn, Ln, D):
     r = I.scan_inputs(0, Bn, Ln, D, 16, dt, with_h0=True)
     y, hT = run_scan(L, r, dt, h0=r["h0"])

@@ -71,11 +71,11 @@ def test_swa_config_shapes_peaked(L):
     assert attn_err(o, ref) <= TOL["bf16"]
 
 
-@pytest.mark.parametrize("kernel", ["", "1"])
+@pytest.mark.parametrize("kernel", ["", "2", "1"])
 def test_swa_config_shapes_peaked_x30(L, kernel):
     """q scaled x30 (score std 30: most rows put nearly all weight on one or two
     keys), at the config shapes (32/4 heads of 64, window 2048) past the window,
-    through the two-head and the one-head tensor-core kernels.  Without RoPE:
+    through the four-head, two-head and one-head tensor-core kernels.  Without RoPE:
     both sides then score the same bf16 q and k, while with RoPE the bf16 storage
     of the rotated q/k moves logits of std 30 by ~0.1, which flips near-ties
     between the two largest keys and is not a kernel error."""
@@ -162,4 +162,23 @@ def test_swa_tensor_core_kernel_matches_cuda_core_kernel(L, Bn, Ln, w):
         o_simt = run_swa(L, r["q"], r["k"], r["v"], w, 10000.0, 0, "bf16")
     finally:
         del os.environ["SAMBA_SWA_KERNEL"]
-    assert rel_err(o_tc, o_simt) <= 1e-2
+    assert attn_err(o_tc, o_simt) <= 1e-2
+
+
+@pytest.mark.parametrize("Bn,Ln,w,qh", [(1, 1000, 2048, 32), (2, 777, 128, 8), (1, 2500, 300, 16), (1, 130, 1, 8)])
+def test_swa_four_head_kernel_matches_two_head_kernel(L, Bn, Ln, w, qh):
+    """The four-heads-per-CTA kernel (64-key tiles, default when a kv group has a
+    multiple of four query heads) against the two-heads-per-CTA kernel (128-key
+    tiles) on the same bf16 inputs: same arithmetic per score, different tile
+    boundaries for the online softmax."""
+    import os
+    r = I.swa_inputs(14, Bn, Ln, qh, qh // 8 if qh >= 8 else 1, 64, "bf16")
+    o4 = run_swa(L, r["q"], r["k"], r["v"], w, 10000.0, 0, "bf16")
+    os.environ["SAMBA_SWA_KERNEL"] = "2"
+    try:
+        o2 = run_swa(L, r["q"], r["k"], r["v"], w, 10000.0, 0, "bf16")
+    finally:
+        del os.environ["SAMBA_SWA_KERNEL"]
+    assert attn_err(o4, o2) <= 1e-2
+    ref = oracle_swa(r["q"], r["k"], r["v"], w, 10000.0, 0)
+    assert attn_err(o4, ref) <= TOL["bf16"]
