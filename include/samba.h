@@ -238,7 +238,7 @@ typedef struct {
 
 /* Decode state of one block, all caller-owned device buffers. */
 typedef struct {
-  float* ssm;     /* [B, d_inner, d_state] fp32 recurrent state */
+  float* ssm;     /* [B, d_inner, d_state] fp32 recurrent state, 16-byte aligned */
   void* conv;     /* [B, d_inner, d_conv-1] dtype: last d_conv-1 pre-conv inputs, oldest first */
   void* k_ring;   /* [B, window, n_kv, head_dim] dtype: post-RoPE keys, slot = position mod window */
   void* v_ring;   /* [B, window, n_kv, head_dim] dtype */
@@ -262,7 +262,8 @@ size_t samba_block_workspace_size(const samba_block_config* cfg, int B, int L);
  * their ring slots, pos[b] = L).  taps may be NULL.
  * Requirements: d_state == 16, head_dim in {16, 32, 64} (64 or 256 on the bf16
  * tensor-core path), d_model, d_inner, d_ff multiples of 64, dt_rank a multiple
- * of 8, n_q % n_kv == 0.  samba_step supports head_dim <= 64. */
+ * of 8, n_q % n_kv == 0.  samba_step takes the same head dims (at head_dim 256
+ * its attention runs on the CUDA-core decode kernel). */
 samba_status samba_block_fwd(const samba_block_config* cfg, const samba_block_weights* w, const void* x_in,
                              void* x_out, samba_decode_state* st, const samba_block_taps* taps, int B, int L,
                              void* workspace, size_t workspace_bytes, samba_stream stream);

@@ -904,6 +904,7 @@ samba_status samba_model_step(const samba_model* m, const int32_t* ids_t, void* 
     TRY(validate_layer(m->kinds[i], m->layers[i]));
     const samba_layer_state& sl = states[i];
     if (m->kinds[i] == SAMBA_LAYER_MAMBA && (!sl.ssm || !sl.conv)) return SAMBA_ERR_INVALID_ARG;
+    if (m->kinds[i] == SAMBA_LAYER_MAMBA && !aligned16(sl.ssm)) return SAMBA_ERR_UNSUPPORTED;
     if (m->kinds[i] == SAMBA_LAYER_SWA && (!sl.k_ring || !sl.v_ring)) return SAMBA_ERR_INVALID_ARG;
   }
   const samba_block_config& c = m->cfg;
@@ -953,6 +954,7 @@ samba_status samba_step(const samba_block_config* cfg, const samba_block_weights
   if (!x_t || !y_t || !stt || B < 1 || x_t == y_t) return SAMBA_ERR_INVALID_ARG;
   if (B > kMaxGridYZ) return SAMBA_ERR_UNSUPPORTED;
   if (!stt->ssm || !stt->conv || !stt->k_ring || !stt->v_ring || !stt->pos) return SAMBA_ERR_INVALID_ARG;
+  if (!aligned16(stt->ssm)) return SAMBA_ERR_UNSUPPORTED;  // the state is moved in 16-byte pieces
   const samba_block_config& c = *cfg;
   const BlockPlan P = plan_block(c, B);
   if (!workspace || workspace_bytes < P.total) return SAMBA_ERR_INVALID_ARG;

@@ -93,7 +93,21 @@ __device__ __forceinline__ float sigmoid_acc(float x) { return 1.0f / (1.0f + ex
 __device__ __forceinline__ float sigmoid_fast(float x) { return fmaf(0.5f, tanh_approx(0.5f * x), 0.5f); }
 // softplus(x) = log(1 + e^x); for x > 20 the difference from x is below fp32 resolution.
 __device__ __forceinline__ float softplus_acc(float x) { return x > 20.f ? x : log1pf(expf(x)); }
-__device__ __forceinline__ float softplus_fast(float x) { return x > 20.f ? x : __logf(1.0f + __expf(x)); }
+// softplus(x) = max(x, 0) + log1p(e^-|x|) with a single MUFU operation: y =
+// e^-|x| in (0, 1] by ex2, then log1p(y) = y q(y) on the FMA pipe, q a degree-5
+// polynomial fitted here to log1p(y)/y on [0, 1] (relative-error-weighted least
+// squares on Chebyshev nodes; max relative error of y q(y) 9e-6 in fp32, far
+// below the bf16 resolution of the stored result).  Exact limits: x -> -inf
+// gives 0 (y underflows), large x gives x.
+__device__ __forceinline__ float softplus_1x(float x) {
+  const float y = ex2_approx(-fabsf(x) * 1.4426950408889634f);
+  float q = fmaf(-0.023869865f, y, 0.10122409f);
+  q = fmaf(q, y, -0.21005028f);
+  q = fmaf(q, y, 0.32520726f);
+  q = fmaf(q, y, -0.49936143f);
+  q = fmaf(q, y, 0.99999160f);
+  return fmaxf(x, 0.f) + y * q;
+}
 
 // ---------------------------------------------------------------------------
 // Shared-memory addresses, mbarriers with bounded waits
@@ -194,6 +208,27 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, uin
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
           smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+// L2 eviction-priority policies for TMA loads: a streamed operand (read once)
+// is marked evict-first so that it does not push a reused one (marked
+// evict-last) out of L2.
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* m, uint64_t* bar, int x, int y,
+                                                 uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%3, "
+      "%4}], [%2], %5;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(policy)
       : "memory");
 }
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* m, uint64_t* bar, int x, int y, int z) {

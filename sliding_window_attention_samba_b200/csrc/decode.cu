@@ -50,17 +50,32 @@ __global__ void scan_step_kernel(const T* __restrict__ u, const T* __restrict__ 
   const float uv = Elt<T>::to_f(u[(size_t)b * D + c]);
   const T* Bp = xdbl + (size_t)b * ld_x + r_off;
   const T* Cp = Bp + 16;
-  float* hp = ssm + ((size_t)b * D + c) * 16;
+  // the 16 states of (b, c) are 64 contiguous bytes: four 16-byte accesses per
+  // thread, so a warp's accesses cover whole 2 KB runs
+  float4* hp = reinterpret_cast<float4*>(ssm + ((size_t)b * D + c) * 16);
+  const float4* ap = reinterpret_cast<const float4*>(A_log + (size_t)c * 16);
+  float Bv[16], Cv[16], h[16], al[16];
+  load8(Bp, Bv);
+  load8(Bp + 8, Bv + 8);
+  load8(Cp, Cv);
+  load8(Cp + 8, Cv + 8);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float4 hv = hp[q], av = ap[q];
+    h[4 * q] = hv.x; h[4 * q + 1] = hv.y; h[4 * q + 2] = hv.z; h[4 * q + 3] = hv.w;
+    al[4 * q] = av.x; al[4 * q + 1] = av.y; al[4 * q + 2] = av.z; al[4 * q + 3] = av.w;
+  }
   float yv = 0.f;
   const float du = delta * uv;
 #pragma unroll
   for (int n = 0; n < 16; ++n) {
-    const float A = -expf(A_log[(size_t)c * 16 + n]);
+    const float A = -expf(al[n]);
     const float dA = sizeof(T) == 4 ? expf(delta * A) : ex2_approx(delta * A * 1.4426950408889634f);
-    const float hn = fmaf(dA, hp[n], du * Elt<T>::to_f(Bp[n]));
-    hp[n] = hn;
-    yv = fmaf(Elt<T>::to_f(Cp[n]), hn, yv);
+    h[n] = fmaf(dA, h[n], du * Bv[n]);
+    yv = fmaf(Cv[n], h[n], yv);
   }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) hp[q] = make_float4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
   yv = fmaf(Dskip ? Dskip[c] : 0.f, uv, yv);
   const float zv = Elt<T>::to_f(z[(size_t)b * ld_z + c]);
   const float s = sizeof(T) == 4 ? sigmoid_acc(zv) : sigmoid_fast(zv);
@@ -90,6 +105,7 @@ __global__ void ring_write_kernel(const T* __restrict__ qkv, int64_t ld, int k_o
 // softmax sum does not depend on their order.  CTA = (kv head, batch row),
 // one warp per query head of the group; K/V blocks shared through smem.
 constexpr int kDecKB = 64;
+constexpr int kDecMaxDpl = 8;  // head dims per lane: head_dim <= 256
 
 template <typename T>
 __global__ void attn_decode_kernel(const T* __restrict__ qkv, int64_t ld, const int64_t* __restrict__ pos,
@@ -107,9 +123,9 @@ __global__ void attn_decode_kernel(const T* __restrict__ qkv, int64_t ld, const 
   const int64_t P = pos[b];
   const int nvalid = (int)(P + 1 < window ? P + 1 : window);
   const T* qrow = qkv + (size_t)b * ld + (size_t)h * hd;
-  float q[4], oacc[4];
-  const int nd = (hd + 31) / 32;  // dims per lane (<= 4)
-  for (int r = 0; r < 4; ++r) {
+  float q[kDecMaxDpl], oacc[kDecMaxDpl];
+  const int nd = (hd + 31) / 32;  // dims per lane (<= 8: head_dim <= 256)
+  for (int r = 0; r < kDecMaxDpl; ++r) {
     const int i = lane + 32 * r;
     q[r] = (r < nd && i < hd) ? Elt<T>::to_f(qrow[i]) * scale : 0.f;
     oacc[r] = 0.f;
@@ -149,7 +165,7 @@ __global__ void attn_decode_kernel(const T* __restrict__ qkv, int64_t ld, const 
       }
       for (int off = 16; off; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
       l = l * corr + ps;
-      for (int r = 0; r < 4; ++r) oacc[r] *= corr;
+      for (int r = 0; r < kDecMaxDpl; ++r) oacc[r] *= corr;
       for (int j = 0; j < nb; ++j) {
         const float pj = __shfl_sync(0xffffffffu, p[j / 32], j % 32);
         for (int r = 0; r < nd; ++r) {
@@ -610,7 +626,7 @@ samba_status launch_attn_decode(const void* qkv, int64_t ld, const int64_t* pos,
                                 const void* v_ring, void* o, int B, int Hq, int Hkv, int hd, int window, float scale,
                                 samba_dtype dt, cudaStream_t st, void* ws, size_t ws_bytes) {
   if (B > kMaxGridYZ) return SAMBA_ERR_UNSUPPORTED;
-  if (hd > 128) return SAMBA_ERR_UNSUPPORTED;
+  if (hd > 32 * kDecMaxDpl) return SAMBA_ERR_UNSUPPORTED;
   if (dt == SAMBA_BF16 && hd == kHd && Hq / Hkv <= 8 && window > kSplit * kSliceMax && ld % 8 == 0) {
     const int nsplit = (window + kSliceMax - 1) / kSliceMax;
     if (!ws || ws_bytes < attn_decode_workspace_bytes(B, Hkv, window) || !aligned16(ws))
@@ -653,7 +669,9 @@ samba_status launch_attn_decode(const void* qkv, int64_t ld, const int64_t* pos,
   const int grp = Hq / Hkv;
   const int threads = ((grp * 32) < 128 ? 128 : grp * 32);
   if (threads > 1024) return SAMBA_ERR_UNSUPPORTED;
-  const size_t smem = 2 * kDecKB * (hd + 1) * sizeof(float);
+  const size_t smem = 2 * kDecKB * (hd + 1) * sizeof(float);  // 131.6 KB at head_dim 256
+  if (!ensure_smem_attr(attn_decode_kernel<bf16>, smem) || !ensure_smem_attr(attn_decode_kernel<float>, smem))
+    return SAMBA_ERR_CUDA;
   dim3 grid(Hkv, B);
   cudaError_t e;
   SAMBA_DT_DISPATCH(dt,

@@ -52,7 +52,7 @@ __device__ __forceinline__ float silu_t(float g) {
 template <typename T>
 __device__ __forceinline__ float softplus_t(float x) {
   if constexpr (sizeof(T) == 4) return softplus_acc(x);
-  else return softplus_fast(x);
+  else return softplus_1x(x);
 }
 
 __device__ __forceinline__ void seg_lookup(const GemmArgs& a, int n, int& s, int& row) {
@@ -286,6 +286,48 @@ __device__ __forceinline__ void tc_epilogue_tile(const TcParams& p, uint32_t tba
     }
     return;
   }
+  if (EPI == kEpiSoftplus) {
+    // Delta = softplus(acc + bias): the next chunk's TMEM load is in flight while
+    // this one is evaluated (the K = 128 main loop is short, so this read-out
+    // sets the kernel's pace); one MUFU operation per element
+    part_range((p.bn + 31) / 32, part, TcEpi<EPI>::parts, u_lo, u_hi);
+    auto chunk = [&](const uint32_t (&rc)[32], int u) {
+      const int cc = u * 32;
+      if (!in_range) return;
+      const int nv = min(4, (p.bn - cc) / 8);
+      const int col = col0 + cc;
+      const float4* bp = reinterpret_cast<const float4*>(a.bias + col);  // 16-byte aligned (checked at launch)
+      bf16* o = out + row * a.ldo + col;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {  // 8 columns at a time, stored at once
+        if (i >= nv) continue;
+        const float4 b0 = bp[2 * i], b1 = bp[2 * i + 1];
+        float f[8];
+        f[0] = softplus_1x(__uint_as_float(rc[8 * i + 0]) + b0.x);
+        f[1] = softplus_1x(__uint_as_float(rc[8 * i + 1]) + b0.y);
+        f[2] = softplus_1x(__uint_as_float(rc[8 * i + 2]) + b0.z);
+        f[3] = softplus_1x(__uint_as_float(rc[8 * i + 3]) + b0.w);
+        f[4] = softplus_1x(__uint_as_float(rc[8 * i + 4]) + b1.x);
+        f[5] = softplus_1x(__uint_as_float(rc[8 * i + 5]) + b1.y);
+        f[6] = softplus_1x(__uint_as_float(rc[8 * i + 6]) + b1.z);
+        f[7] = softplus_1x(__uint_as_float(rc[8 * i + 7]) + b1.w);
+        store8(o + 8 * i, f);
+      }
+    };
+    uint32_t ra[32], rb[32];
+    if (u_lo < u_hi) tmem_ld32(tbase + u_lo * 32, ra);
+    for (int u = u_lo; u < u_hi; u += 2) {  // two buffers, named statically
+      tmem_wait_ld();
+      if (u + 1 < u_hi) tmem_ld32(tbase + (u + 1) * 32, rb);
+      chunk(ra, u);
+      if (u + 1 < u_hi) {
+        tmem_wait_ld();
+        if (u + 2 < u_hi) tmem_ld32(tbase + (u + 2) * 32, ra);
+        chunk(rb, u + 1);
+      }
+    }
+    return;
+  }
   // 32-column chunks; a tile width of 16 mod 32 ends in a 16-column chunk (the
   // TMEM columns past it are read but not stored)
   part_range((p.bn + 31) / 32, part, TcEpi<EPI>::parts, u_lo, u_hi);
@@ -313,17 +355,6 @@ __device__ __forceinline__ void tc_epilogue_tile(const TcParams& p, uint32_t tba
         load8(rs + 8 * i, g);
 #pragma unroll
         for (int j = 0; j < 8; ++j) f[8 * i + j] += g[j];
-      }
-    } else if (EPI == kEpiSoftplus) {
-      const float4* bp = reinterpret_cast<const float4*>(a.bias + col);  // 16-byte aligned (checked at launch)
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        if (i >= 2 * nv) continue;
-        const float4 b4 = bp[i];
-        f[4 * i + 0] = softplus_fast(f[4 * i + 0] + b4.x);
-        f[4 * i + 1] = softplus_fast(f[4 * i + 1] + b4.y);
-        f[4 * i + 2] = softplus_fast(f[4 * i + 2] + b4.z);
-        f[4 * i + 3] = softplus_fast(f[4 * i + 3] + b4.w);
       }
     }
     bf16* o = out + row * a.ldo + col;
@@ -368,6 +399,9 @@ __global__ void __launch_bounds__(TcEpi<EPI>::threads, 1) gemm_tc_kernel(const _
     // ---------------- TMA producer
     if (elect_one()) {
       const uint32_t bytes = TC_A_BYTES + (uint32_t)p.umma_n * TC_BK * 2;
+      // activations stream through once per n-tile group; the group's weight
+      // panel is reused by every m-tile, so it is kept in L2 ahead of them
+      const uint64_t pol_a = l2_policy_evict_first(), pol_b = l2_policy_evict_last();
       int it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
@@ -381,12 +415,12 @@ __global__ void __launch_bounds__(TcEpi<EPI>::threads, 1) gemm_tc_kernel(const _
           const uint32_t j = it / TC_STAGES;
           if (!mbar_wait(&S.empty[s], (j & 1) ^ 1, err)) { ok = false; break; }
           mbar_arrive_expect_tx(&S.full[s], bytes);
-          tma_load_2d(S.A[s], &p.tmA, &S.full[s], kb * TC_BK, mt * TC_BM);
+          tma_load_2d_hint(S.A[s], &p.tmA, &S.full[s], kb * TC_BK, mt * TC_BM, pol_a);
           if (EPI == kEpiSwiglu) {
-            tma_load_2d(S.B[s], &p.tmB[0], &S.full[s], kb * TC_BK, brow);
-            tma_load_2d(S.B[s] + p.bn * TC_BK, &p.tmB2, &S.full[s], kb * TC_BK, brow);
+            tma_load_2d_hint(S.B[s], &p.tmB[0], &S.full[s], kb * TC_BK, brow, pol_b);
+            tma_load_2d_hint(S.B[s] + p.bn * TC_BK, &p.tmB2, &S.full[s], kb * TC_BK, brow, pol_b);
           } else {
-            tma_load_2d(S.B[s], &p.tmB[seg], &S.full[s], kb * TC_BK, brow);
+            tma_load_2d_hint(S.B[s], &p.tmB[seg], &S.full[s], kb * TC_BK, brow, pol_b);
           }
         }
       }

@@ -289,7 +289,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) gemm_skinny_kernel(const __grid
       }
       if (n >= a.N) continue;
       if (EPI == kEpiSwiglu) v = v * (v2 * sigmoid_fast(v2));
-      if (EPI == kEpiSoftplus) v = softplus_fast(v + a.bias[n]);
+      if (EPI == kEpiSoftplus) v = softplus_1x(v + a.bias[n]);
       if (EPI == kEpiResid) {
         if (a.tap) ((bf16*)a.tap)[(int64_t)b * a.ldt + n] = __float2bfloat16_rn(v);
         v += __bfloat162float(((const bf16*)a.resid)[(int64_t)b * a.ldr + n]);

@@ -46,6 +46,7 @@ constexpr int kN = 16;                // state size
 constexpr int kHalf = 8;              // states per lane
 constexpr int kThreads = kWarps * 32;
 constexpr int kYBuf = 3;              // y tiles in flight
+constexpr int kBCPitch = 2 * kN + 4;  // 36 floats: rows 16 bytes apart in the bank space
 
 template <typename T> struct ScanCfg { static constexpr int kStages = sizeof(T) == 2 ? 4 : 2; };
 
@@ -58,7 +59,7 @@ struct ScanSmem {
   T Bm[S][kChunk * kN];  // [token][state]
   T Cm[S][kChunk * kN];
   T y[kYBuf][kChunk * kCh];
-  float BC[kWarps][kTs][2 * kN];   // each warp's rows: B | C in fp32
+  float BC[kWarps][kTs][kBCPitch];  // each warp's rows: B | C in fp32 (row padded: conflict-free stores)
   float2 dd[kWarps][kTs][kCh];     // (Delta, Delta u)
   float2 gg[kWarps][kTs][kCh];     // (gate, D u gate)
   float4 E[2][kWarps][2][32];      // entry states [chunk parity][warp slot][state quad][lane]
@@ -70,19 +71,6 @@ struct ScanSmem {
 };
 
 __device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
-
-template <typename T>
-__device__ __forceinline__ void load4(const T* p, float* f) {
-  if constexpr (sizeof(T) == 2) {
-    const uint2 v = *reinterpret_cast<const uint2*>(p);
-    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.x));
-    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.y));
-    f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
-  } else {
-    const float4 v = *reinterpret_cast<const float4*>(p);
-    f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
-  }
-}
 
 template <typename T, bool kSoftplus, bool kHasZ>
 __global__ void __launch_bounds__(kThreads, 2)
@@ -139,6 +127,23 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
   };
 
+  // The carry hand-off is on the critical path of every chunk: poll it without
+  // suspending (a suspended waiter resumes later than a polling one), bounded.
+  auto wait_spin = [&](uint64_t* bar, uint32_t parity) -> bool {
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 0;; ++it) {
+      if (mbar_test(bar, parity)) return true;
+      if ((it & 255u) == 255u) {
+        if (*reinterpret_cast<volatile int*>(&Sm.abort)) return false;
+        if (globaltimer_ns() - t0 > wait_limit_ns) {
+          raise_error(err, kErrTimeout);
+          *reinterpret_cast<volatile int*>(&Sm.abort) = 1;
+          return false;
+        }
+      }
+    }
+  };
+
   int issued = 0;  // chunks whose loads the producer issued
   auto issue = [&](int c) {
     if (c >= stop_chunk || c >= nchunk) return;  // failure-detection test hook: nothing issued past stop
@@ -169,14 +174,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     const float* a = A_log + (size_t)d * kN + hf * kHalf + 2 * k;
     A2[k] = make_float2(-expf(a[0]) * 1.4426950408889634f, -expf(a[1]) * 1.4426950408889634f);
   }
-  // Conversion-role constants: row pr of the warp slice, channels pc .. pc + 3.
-  const int pr = lane >> 2, pc = (lane & 3) * 4;
-  float bias4[4], D4[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    bias4[j] = dt_bias ? dt_bias[d0 + pc + j] : 0.f;
-    D4[j] = Dskip ? Dskip[d0 + pc + j] : 0.f;
-  }
+  // Conversion-role constants: this lane's channel; row pr of the B | C runs.
+  const int pr = lane >> 2;
+  const float bias1 = dt_bias ? dt_bias[d] : 0.f;
+  const float D1 = Dskip ? Dskip[d] : 0.f;
 
   bool ok = true;
   int consumed = 0;  // chunks whose stage this warp saw land
@@ -188,31 +189,32 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (!__all_sync(0xffffffffu, wait(&Sm.full[s], (c / S) & 1))) { ok = false; break; }
     consumed = c + 1;
     {
-      const int row = warp * kTs + pr;
-      const int tg = c * kChunk + row;
-      float uu[4], dv[4], zz[4];
-      load4(Sm.u[s] + row * kCh + pc, uu);
-      load4(Sm.dt[s] + row * kCh + pc, dv);
-      if (kHasZ) load4(Sm.z[s] + row * kCh + pc, zz);
+      // per (token, channel): lane = (channel ch, token half hf), tokens hf*4 .. hf*4+3
+      // of the warp's slice, so each store writes whole 128-byte rows
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        float delta = dv[j] + bias4[j];
+      for (int k = 0; k < 4; ++k) {
+        const int i = hf * 4 + k;
+        const int row = warp * kTs + i;
+        const int tg = c * kChunk + row;
+        float delta = Elt<T>::to_f(Sm.dt[s][row * kCh + ch]) + bias1;
         if (kSoftplus) {
           if constexpr (sizeof(T) == 4) delta = softplus_acc(delta);
-          else delta = softplus_fast(delta);
+          else delta = softplus_1x(delta);
         }
-        float uv = uu[j];
+        float uv = Elt<T>::to_f(Sm.u[s][row * kCh + ch]);
         if (tg >= L) { delta = 0.f; uv = 0.f; }  // padding past the sequence: state unchanged
         float g = 1.f;
         if (kHasZ) {
-          if constexpr (sizeof(T) == 4) g = zz[j] * sigmoid_acc(zz[j]);
-          else g = zz[j] * sigmoid_fast(zz[j]);
+          const float zv = Elt<T>::to_f(Sm.z[s][row * kCh + ch]);
+          if constexpr (sizeof(T) == 4) g = zv * sigmoid_acc(zv);
+          else g = zv * sigmoid_fast(zv);
         }
-        Sm.dd[warp][pr][pc + j] = make_float2(delta, delta * uv);
-        Sm.gg[warp][pr][pc + j] = make_float2(g, D4[j] * uv * g);
+        Sm.dd[warp][i][ch] = make_float2(delta, delta * uv);
+        Sm.gg[warp][i][ch] = make_float2(g, D1 * uv * g);
       }
       // B | C of the 8 rows: 4 runs of 8 values per row, one run per lane
       const int part = lane & 3;
+      const int row = warp * kTs + pr;
       const T* src = (part < 2 ? Sm.Bm[s] : Sm.Cm[s]) + row * kN + (part & 1) * 8;
       float f[8];
       load8(src, f);
@@ -273,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     } else {
       const uint32_t par = warp == 0 ? ((c - 1) & 1) : (c & 1);
-      if (!__all_sync(0xffffffffu, wait(&Sm.eready[warp], par))) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, wait_spin(&Sm.eready[warp], par))) { ok = false; break; }
       const float4 q0 = Sm.E[c & 1][warp][0][lane], q1 = Sm.E[c & 1][warp][1][lane];
       e[0] = make_float2(q0.x, q0.y);
       e[1] = make_float2(q0.z, q0.w);

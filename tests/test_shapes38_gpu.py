@@ -67,3 +67,21 @@ def test_block_38b_shapes(L):
     g = GpuBlock(L, shape, W, 1, 2304)
     out, br, rs = g.prefill(x)
     check_branches(shape, W, x, out, br, rs, TOL["bf16"])
+
+
+def test_decode_steps_38b_shapes(L):
+    """samba_step at the 3.8B widths (11 query heads over one kv head of 256):
+    prefill 300 tokens, then 3 decode steps, against the oracle's prefill of the
+    longer sequence; positions exact."""
+    from tests.test_block_gpu import step_err
+    shape = I.WIDE38
+    W = I.block_weights(shape, 43)
+    P, S = 300, 3
+    x = I.block_input(shape, 43, 2, P + S)
+    g = GpuBlock(L, shape, W, 2, P + S)
+    g.prefill(x[:, :P], taps=False)
+    full = O.block_fwd(x, W, shape)
+    for i in range(S):
+        y = host(g.step(x[:, P + i]))
+        assert step_err(y, x[:, P + i], full, P + i, "bf16") <= TOL["bf16"], i
+    assert np.array_equal(host(g.pos), np.full(2, P + S))
