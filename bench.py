@@ -40,6 +40,8 @@ import numpy as np  # noqa: E402
 from sliding_window_attention_samba_b200 import inputs as I  # noqa: E402
 
 WORKLOAD = "prefill_bf16_L131072_x4"
+MUFU_EX2_PER_CLK_SM = 16  # ex2.approx results per clock per SM (sm_100a MUFU)
+N_SMS = 148
 METRIC = "prefill tokens/s per Samba block at L=128K; scan HBM GB/s & SWA TC util vs peak"
 UNIT = "tokens/s"
 
@@ -454,6 +456,16 @@ def kernel_report(kt, s, T, Bn, Ln, peaks, t_up_live=None, clocks=None):
     scan_bytes = T * (8 * s.d_inner + 4 * s.d_state)
     rep["scan"] = {"gbs": scan_bytes / kt["scan"] / 1e9, "frac_of_" + src + "_hbm": scan_bytes / kt["scan"] / 1e9 / hbm,
                    "ms": kt["scan"] * 1e3}
+    # The scan's binding unit is the exponential (MUFU) pipe: one ex2 per
+    # (token, channel, state) element at 16 per clock per SM (measured on this
+    # pool's B200 with a throughput microbenchmark: 4.6e12 ex2/s), at the run's
+    # median SM clock.
+    mhz = (clocks or {}).get("sm_mhz")
+    if mhz:
+        ex2_per_s = MUFU_EX2_PER_CLK_SM * N_SMS * mhz * 1e6
+        floor = T * s.d_inner * s.d_state / ex2_per_s
+        rep["scan"].update({"bound": "alu", "mufu_floor_ms": floor * 1e3, "frac_of_mufu_floor": floor / kt["scan"],
+                            "mufu_peak": f"{MUFU_EX2_PER_CLK_SM} ex2/clk/SM x {N_SMS} SMs x {mhz:.0f} MHz"})
     sf = swa_flops(s, Bn, Ln)
     rep["swa"] = {"tflops": sf / kt["swa"] / 1e12, "frac_of_" + src + "_bf16_peak": sf / kt["swa"] / 1e12 / tf_sus,
                   "ms": kt["swa"] * 1e3}

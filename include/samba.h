@@ -60,6 +60,11 @@ const char* samba_status_string(samba_status s);
 /* Library version string (static). */
 const char* samba_version(void);
 
+/* The CUDA error behind the calling thread's last SAMBA_ERR_CUDA return ("where:
+ * message (code)"), or "" if none was recorded.  Owned by the library; valid
+ * until the thread's next failing call. */
+const char* samba_last_cuda_error(void);
+
 /* Measurement hook for benchmarks and profilers (no effect unless installed).
  * While installed, every launch of a projection with epilogue kind `epi` (the
  * samba_linear kinds: 0 none, 1 residual, 2 SwiGLU, 3 softplus + bias; 4 the

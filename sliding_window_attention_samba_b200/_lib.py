@@ -37,9 +37,10 @@ STATUS = {0: "SAMBA_OK", 1: "SAMBA_ERR_INVALID_ARG", 2: "SAMBA_ERR_UNSUPPORTED",
 
 
 class SambaError(RuntimeError):
-    def __init__(self, fn: str, code: int):
-        super().__init__(f"{fn} returned {STATUS.get(code, code)}")
+    def __init__(self, fn: str, code: int, detail: str = ""):
+        super().__init__(f"{fn} returned {STATUS.get(code, code)}" + (f" [{detail}]" if detail else ""))
         self.code = code
+        self.detail = detail
 
 
 class BlockConfig(ctypes.Structure):
@@ -87,6 +88,7 @@ def _sig(name, restype, argtypes):
 
 _status_string = _sig("samba_status_string", ctypes.c_char_p, [c_int])
 _version = _sig("samba_version", ctypes.c_char_p, [])
+_last_cuda_error = _sig("samba_last_cuda_error", ctypes.c_char_p, [])
 _set_timing = _sig("samba_set_gemm_timing", c_int, [c_int, c_void_p, c_void_p, c_int])
 _timing_count = _sig("samba_gemm_timing_count", c_int, [])
 _get_error = _sig("samba_get_error", c_int, [c_void_p])
@@ -153,7 +155,12 @@ def _stream(stream) -> Optional[int]:
 
 def _check(fn: str, rc: int):
     if rc != 0:
-        raise SambaError(fn, rc)
+        detail = _last_cuda_error().decode() if rc == SAMBA_ERR_CUDA else ""
+        raise SambaError(fn, rc, detail)
+
+
+def samba_last_cuda_error() -> str:
+    return _last_cuda_error().decode()
 
 
 def samba_status_string(code: int) -> str:

@@ -4,8 +4,10 @@
 #include <algorithm>
 #include <initializer_list>
 #include <mutex>
+#include <map>
 #include <set>
 #include <utility>
+#include <stdio.h>
 #include <string.h>
 
 #include "common.cuh"
@@ -58,6 +60,16 @@ int* device_error_word() {
 }
 
 // ---------------------------------------------------------------------------
+// The CUDA error behind the last SAMBA_ERR_CUDA of the calling thread
+// ---------------------------------------------------------------------------
+static thread_local char g_cuda_err_msg[256] = {0};
+samba_status note_cuda_failure(const char* where, int cuda_error) {
+  snprintf(g_cuda_err_msg, sizeof(g_cuda_err_msg), "%s: %s (%d)", where,
+           cudaGetErrorString((cudaError_t)cuda_error), cuda_error);
+  return SAMBA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
 // Failure-detection test hook of the selective scan
 // ---------------------------------------------------------------------------
 static std::mutex g_stall_mu;
@@ -71,14 +83,16 @@ StallHook scan_stall_hook() {
 // Per-(kernel, device) record of raised shared-memory limits
 // ---------------------------------------------------------------------------
 static std::mutex g_attr_mu;
-static std::set<std::pair<const void*, int>> g_attr_done;
-bool smem_attr_done(const void* kern, int dev) {
+static std::map<std::pair<const void*, int>, size_t> g_attr_done;
+bool smem_attr_done(const void* kern, int dev, size_t bytes) {
   std::lock_guard<std::mutex> lk(g_attr_mu);
-  return g_attr_done.count({kern, dev}) != 0;
+  auto it = g_attr_done.find({kern, dev});
+  return it != g_attr_done.end() && it->second >= bytes;
 }
-void smem_attr_mark(const void* kern, int dev) {
+void smem_attr_mark(const void* kern, int dev, size_t bytes) {
   std::lock_guard<std::mutex> lk(g_attr_mu);
-  g_attr_done.insert({kern, dev});
+  size_t& v = g_attr_done[{kern, dev}];
+  if (bytes > v) v = bytes;
 }
 
 // ---------------------------------------------------------------------------
@@ -114,6 +128,8 @@ bool make_tmap(CUtensorMap* m, const void* base, samba_dtype dt, int rank, const
                   (cuuint32_t)rank, const_cast<void*>(base), gdim, gstride, bdim, estride,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    snprintf(g_cuda_err_msg, sizeof(g_cuda_err_msg), "cuTensorMapEncodeTiled: CUresult %d", (int)r);
   return r == CUDA_SUCCESS;
 }
 
@@ -254,6 +270,8 @@ const char* samba_status_string(samba_status s) {
 }
 
 const char* samba_version(void) { return "samba-b200 0.1 (sm_100a)"; }
+
+const char* samba_last_cuda_error(void) { return g_cuda_err_msg; }
 
 samba_status samba_set_gemm_timing(int epi, void* const* start_events, void* const* stop_events, int capacity) {
   return gemm_timing_set(epi, start_events, stop_events, capacity);

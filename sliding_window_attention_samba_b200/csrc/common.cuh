@@ -21,6 +21,9 @@ enum : int { kErrNone = 0, kErrTimeout = 1, kErrDevice = 2 };
 
 int* device_error_word();  // device address of the error word of the current device
 uintptr_t current_context_id();  // the calling thread's current CUDA context (0: none yet)
+// Records the CUDA error behind a SAMBA_ERR_CUDA return (calling thread;
+// samba_last_cuda_error reports it) and returns SAMBA_ERR_CUDA.
+samba_status note_cuda_failure(const char* where, int cuda_error);
 
 __device__ __forceinline__ void raise_error(int* err, int code) {
   if (err) atomicCAS(err, 0, code);
@@ -383,19 +386,23 @@ inline int num_sms() {
   return n;
 }
 
-// Raise a kernel's dynamic shared-memory limit once per (kernel, device).  Not
-// a stream operation, so later calls made under CUDA-graph capture skip it.
-bool smem_attr_done(const void* kern, int dev);
-void smem_attr_mark(const void* kern, int dev);
+// Raise a kernel's dynamic shared-memory limit per (kernel, device), again only
+// when a larger size is asked for.  Not a stream operation, so later calls made
+// under CUDA-graph capture (asking for no more than before) skip it.
+bool smem_attr_done(const void* kern, int dev, size_t bytes);
+void smem_attr_mark(const void* kern, int dev, size_t bytes);
 template <typename K>
 inline bool ensure_smem_attr(K kern, size_t bytes) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return false;
   const void* key = reinterpret_cast<const void*>(kern);
-  if (smem_attr_done(key, dev)) return true;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
+  if (smem_attr_done(key, dev, bytes)) return true;
+  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) {
+    note_cuda_failure("cudaFuncSetAttribute (dynamic shared memory)", e);
     return false;
-  smem_attr_mark(key, dev);
+  }
+  smem_attr_mark(key, dev, bytes);
   return true;
 }
 
@@ -423,10 +430,12 @@ inline cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_
   return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
-#define SAMBA_CHECK_LAUNCH()                                 \
-  do {                                                       \
-    cudaError_t e_ = cudaGetLastError();                     \
-    if (e_ != cudaSuccess) return SAMBA_ERR_CUDA;            \
+#define SAMBA_STR2_(x) #x
+#define SAMBA_STR_(x) SAMBA_STR2_(x)
+#define SAMBA_CHECK_LAUNCH()                                                              \
+  do {                                                                                    \
+    cudaError_t e_ = cudaGetLastError();                                                  \
+    if (e_ != cudaSuccess) return note_cuda_failure(__FILE__ ":" SAMBA_STR_(__LINE__), e_); \
   } while (0)
 
 }  // namespace samba

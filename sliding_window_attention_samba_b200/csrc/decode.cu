@@ -584,7 +584,7 @@ samba_status launch_conv_step(const void* hz, int64_t ld_hz, const float* w, con
                                   (const bf16*)hz, ld_hz, w, bias, (bf16*)state, (bf16*)u, B, D, k)),
                     (e = launch_k(conv_step_kernel<float>, dim3((n + 255) / 256), dim3(256), 0, st, true,
                                   (const float*)hz, ld_hz, w, bias, (float*)state, (float*)u, B, D, k)));
-  if (e != cudaSuccess) return SAMBA_ERR_CUDA;
+  if (e != cudaSuccess) return note_cuda_failure("decode kernel launch", e);
   return SAMBA_OK;
 }
 
@@ -601,7 +601,7 @@ samba_status launch_scan_step(const void* u, const void* dlt, const void* z, int
                     (e = launch_k(scan_step_kernel<float>, dim3((n + 127) / 128), dim3(128), 0, st, true,
                                   (const float*)u, (const float*)dlt, (const float*)z, ld_z, (const float*)xdbl, ld_x,
                                   r_off, A_log, Dskip, ssm, (float*)y, B, D)));
-  if (e != cudaSuccess) return SAMBA_ERR_CUDA;
+  if (e != cudaSuccess) return note_cuda_failure("decode kernel launch", e);
   return SAMBA_OK;
 }
 
@@ -613,7 +613,7 @@ samba_status launch_ring_write(const void* qkv, int64_t ld, int k_off, int v_off
                                   k_off, v_off, pos, (bf16*)k_ring, (bf16*)v_ring, window, kvw)),
                     (e = launch_k(ring_write_kernel<float>, dim3(B), dim3(128), 0, st, true, (const float*)qkv, ld,
                                   k_off, v_off, pos, (float*)k_ring, (float*)v_ring, window, kvw)));
-  if (e != cudaSuccess) return SAMBA_ERR_CUDA;
+  if (e != cudaSuccess) return note_cuda_failure("decode kernel launch", e);
   return SAMBA_OK;
 }
 
@@ -659,18 +659,21 @@ samba_status launch_attn_decode(const void* qkv, int64_t ld, const int64_t* pos,
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    if (cudaLaunchKernelEx(&cfg, attn_decode_split_kernel, (const bf16*)qkv, ld, pos, (const bf16*)k_ring,
-                           (const bf16*)v_ring, (bf16*)o, Hq, Hkv, window, scale * 1.4426950408889634f) !=
-        cudaSuccess)
-      return SAMBA_ERR_CUDA;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, attn_decode_split_kernel, (const bf16*)qkv, ld, pos,
+                                             (const bf16*)k_ring, (const bf16*)v_ring, (bf16*)o, Hq, Hkv, window,
+                                             scale * 1.4426950408889634f);
+    if (e != cudaSuccess) return note_cuda_failure("cudaLaunchKernelEx (decode attention cluster)", e);
     SAMBA_CHECK_LAUNCH();
     return SAMBA_OK;
   }
   const int grp = Hq / Hkv;
   const int threads = ((grp * 32) < 128 ? 128 : grp * 32);
   if (threads > 1024) return SAMBA_ERR_UNSUPPORTED;
-  const size_t smem = 2 * kDecKB * (hd + 1) * sizeof(float);  // 131.6 KB at head_dim 256
-  if (!ensure_smem_attr(attn_decode_kernel<bf16>, smem) || !ensure_smem_attr(attn_decode_kernel<float>, smem))
+  const size_t smem = 2 * kDecKB * (hd + 1) * sizeof(float);
+  // the limit is raised once to the largest head_dim's need (131.6 KB at 256),
+  // so that a smaller head_dim first does not leave it too low for a larger one
+  constexpr size_t kMaxSmem = 2 * kDecKB * (32 * kDecMaxDpl + 1) * sizeof(float);
+  if (!ensure_smem_attr(attn_decode_kernel<bf16>, kMaxSmem) || !ensure_smem_attr(attn_decode_kernel<float>, kMaxSmem))
     return SAMBA_ERR_CUDA;
   dim3 grid(Hkv, B);
   cudaError_t e;
@@ -681,7 +684,7 @@ samba_status launch_attn_decode(const void* qkv, int64_t ld, const int64_t* pos,
                     (e = launch_k(attn_decode_kernel<float>, grid, dim3(threads), smem, st, true, (const float*)qkv,
                                   ld, pos, (const float*)k_ring, (const float*)v_ring, (float*)o, Hq, Hkv, hd, window,
                                   scale)));
-  if (e != cudaSuccess) return SAMBA_ERR_CUDA;
+  if (e != cudaSuccess) return note_cuda_failure("decode kernel launch", e);
   return SAMBA_OK;
 }
 

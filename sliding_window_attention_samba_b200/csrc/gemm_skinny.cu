@@ -32,7 +32,10 @@ constexpr int SK_THREADS = 192;
 // Shared memory: a ring of stages (W tile | W2 tile (SwiGLU) | X tile) that is
 // reused, once every MMA has completed, for the fp32 partial tile(s) of the
 // cluster reduction; barriers and the TMEM address live after it.
-constexpr int SK_RING_BYTES = 200 * 1024;
+// 96 KB: two CTAs fit an SM, so that (with programmatic dependent launch) the
+// next projection's CTAs become resident and fetch their first weight stages
+// while the previous projection's CTAs reduce and write their outputs.
+constexpr int SK_RING_BYTES = 96 * 1024;
 constexpr int SK_RED_PITCH = SK_MAXB + 1;
 static_assert(2 * SK_BM * SK_RED_PITCH * 4 <= SK_RING_BYTES, "reduction tiles must fit in the ring");
 
@@ -98,7 +101,7 @@ __device__ __forceinline__ float2 rope_cs_sk(const float2* __restrict__ tab, int
 }
 
 template <int EPI>
-__global__ void __launch_bounds__(SK_THREADS, 1) gemm_skinny_kernel(const __grid_constant__ SkParams p, int* err) {
+__global__ void __launch_bounds__(SK_THREADS, 2) gemm_skinny_kernel(const __grid_constant__ SkParams p, int* err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   SkSmem& S = *reinterpret_cast<SkSmem*>(smem_raw + smem_align_pad(smem_raw, 1024));
   const GemmArgs& a = p.a;
@@ -342,7 +345,8 @@ static samba_status skinny_launch(const SkParams& p, int ntiles, cudaStream_t st
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = p.a.pdl ? 2 : 1;
-  if (cudaLaunchKernelEx(&cfg, kern, p, device_error_word()) != cudaSuccess) return SAMBA_ERR_CUDA;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p, device_error_word());
+  if (e != cudaSuccess) return note_cuda_failure("cudaLaunchKernelEx (skinny projection cluster)", e);
   SAMBA_CHECK_LAUNCH();
   return SAMBA_OK;
 }
@@ -361,8 +365,9 @@ samba_status launch_gemm_skinny(const GemmArgs& a, cudaStream_t st) {
   }
   const int ntiles = (a.N + SK_BM - 1) / SK_BM;
   p.kb_total = a.K / SK_BK;
-  // splits: about one CTA per SM (one wave; a CTA uses most of an SM's shared
-  // memory), at most 8 (portable cluster size) and at most one k-block each
+  // splits: about one CTA per SM (one wave; the SM's second CTA slot is left to
+  // the neighbouring projection), at most 8 (portable cluster size) and at most
+  // one k-block each
   const int want = num_sms() / ntiles;
   int S = 1;
   while (S * 2 <= want && S * 2 <= 8 && S * 2 <= p.kb_total) S *= 2;

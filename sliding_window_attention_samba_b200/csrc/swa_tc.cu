@@ -21,8 +21,6 @@
 #include <stdlib.h>
 #include <string.h>
 
-#include <cuda_fp16.h>
-
 #include "common.cuh"
 #include "kernels.h"
 
@@ -1145,301 +1143,6 @@ __global__ void __launch_bounds__(A4_THREADS, 1) swa_tc4_kernel(const __grid_con
   }
 }
 
-// ---------------------------------------------------------------------------
-// Two query heads per CTA with half-precision probabilities.  The exponentials
-// of P run as packed pairs (ex2.approx.f16x2: two results per MUFU operation)
-// on fp32 inputs rounded to f16, and P stays in f16 for the P V product, so V
-// tiles are converted from bf16 to f16 in shared memory (exact for |v| in the
-// f16 normal range [2^-14, 65504]; values below it keep an absolute accuracy
-// of 2^-24).  Row sums come from the tensor cores (L += P * ones), so the
-// softmax threads only scale, round, exponentiate and store:
-//   warp 0      TMA (Q of both heads, K_j / V_j, 3 stages)
-//   warp 1      TMEM owner + MMA issuer: S = Q K^T (bf16), O += P V (f16),
-//               L += P ones (f16, N 16)
-//   warps 2..9  softmax of head A (2..5) and head B (6..9)
-//   warps 10,11 convert V_j to f16 in place once it lands
-// TMEM: S_A 0..127, S_B 128..255, O_A 256..319, O_B 320..383, L_A 384..399,
-// L_B 400..415.
-constexpr int AH_THREADS = 384;
-constexpr int AH_CONV_THREADS = 64;
-
-struct AtHSmem2 {
-  bf16 Q[2][AT_BM * AT_D];
-  bf16 K[AT_STAGES][AT_BN * AT_D];
-  bf16 V[AT_STAGES][AT_BN * AT_D];  // f16 after conversion
-  __half P[2][2][AT_BM * 64];        // [head][key half][row][64 keys], 128B-swizzled
-  __half ones[16 * 64];              // 16 rows x 128 bytes of 1.0
-  uint64_t q_full;
-  uint64_t kv_full[AT_STAGES], kv_empty[AT_STAGES], v_ready[AT_STAGES];
-  uint64_t s_full[2], s_free[2], p_full[2], pv_done[2];
-  uint32_t tmem_base;
-};
-
-// kind::f16 instruction descriptor with f16 A and B, fp32 D
-__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool b_mn_major = false) {
-  return (1u << 4) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-
-__device__ __forceinline__ uint32_t ex2_h2(uint32_t x) {
-  asm("ex2.approx.f16x2 %0, %0;" : "+r"(x));
-  return x;
-}
-
-template <int kPolyPairs>
-__global__ void __launch_bounds__(AH_THREADS, 1) swa_tc2h_kernel(const __grid_constant__ AtParams p, int* err) {
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
-  AtHSmem2& S = *reinterpret_cast<AtHSmem2*>(smem_raw + smem_align_pad(smem_raw, 1024));
-  const int warp = warp_id_sync();
-  const int lane = threadIdx.x & 31;
-  const int t0 = blockIdx.x * AT_BM;
-  const int h0 = blockIdx.y * 2;
-  const int b = blockIdx.z;
-  const int g = h0 / (p.Hq / p.Hkv);
-  const int tk0 = t0 + p.qoff;
-  const int lo = tk0 - p.window + 1;
-  const int kb0 = lo <= 0 ? 0 : (lo / AT_BN) * AT_BN;
-  const int ntile = (min(tk0 + AT_BM - 1, p.Lk - 1) - kb0) / AT_BN + 1;
-
-  if (warp == 0 && lane == 0) {
-    mbar_init(&S.q_full, 1);
-    for (int s = 0; s < AT_STAGES; ++s) {
-      mbar_init(&S.kv_full[s], 1);
-      mbar_init(&S.kv_empty[s], 1);
-      mbar_init(&S.v_ready[s], AH_CONV_THREADS / 32);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&S.s_full[i], 1);
-      mbar_init(&S.s_free[i], 4);
-      mbar_init(&S.p_full[i], 4);
-      mbar_init(&S.pv_done[i], 1);
-    }
-    fence_mbar_init();
-    tma_prefetch_desc(&p.tmQ);
-    tma_prefetch_desc(&p.tmK);
-    tma_prefetch_desc(&p.tmV);
-  }
-  for (int i = threadIdx.x; i < 16 * 64 / 2; i += AH_THREADS)
-    reinterpret_cast<uint32_t*>(S.ones)[i] = 0x3C003C00u;  // f16 1.0 pairs
-  fence_proxy_async_smem();
-  if (warp == 1) {
-    tmem_alloc(&S.tmem_base, 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = S.tmem_base;
-
-  if (warp == 0) {
-    if (elect_one()) {
-      mbar_arrive_expect_tx(&S.q_full, 2 * kTileBytes);
-      tma_load_3d(S.Q[0], &p.tmQ, &S.q_full, h0 * AT_D, t0, b);
-      tma_load_3d(S.Q[1], &p.tmQ, &S.q_full, (h0 + 1) * AT_D, t0, b);
-      for (int j = 0; j < ntile; ++j) {
-        const int s = j % AT_STAGES;
-        if (!mbar_wait(&S.kv_empty[s], ((j / AT_STAGES) & 1) ^ 1, err)) break;
-        mbar_arrive_expect_tx(&S.kv_full[s], 2 * kTileBytes);
-        const int kb = kb0 + j * AT_BN;
-        tma_load_3d(S.K[s], &p.tmK, &S.kv_full[s], g * AT_D, kb, b);
-        tma_load_3d(S.V[s], &p.tmV, &S.kv_full[s], g * AT_D, kb, b);
-      }
-    }
-  } else if (warp == 1) {
-    const uint32_t idesc_s = idesc_bf16_f32(AT_BM, AT_BN, false);
-    const uint32_t idesc_o = idesc_f16_f32(AT_BM, AT_D, true);  // V is N-contiguous (MN-major B)
-    const uint32_t idesc_l = idesc_f16_f32(AT_BM, 16, false);
-    if (elect_one()) {
-      bool ok = mbar_wait(&S.q_full, 0, err);
-      const uint32_t ones_base = smem_u32(S.ones);
-      auto issue_s = [&](int wg, int j) -> bool {
-        const int s = j % AT_STAGES;
-        if (wg == 0 && !mbar_wait(&S.kv_full[s], (j / AT_STAGES) & 1, err)) return false;
-        if (j >= 1 && !mbar_wait(&S.s_free[wg], (j - 1) & 1, err)) return false;
-        tc_fence_after();
-        const uint32_t q_base = smem_u32(S.Q[wg]);
-        const uint32_t k_base = smem_u32(S.K[s]);
-#pragma unroll
-        for (int k = 0; k < AT_D / 16; ++k)
-          umma_f16_ss(tmem + wg * 128u, smem_desc(q_base + k * 32, 16, 1024, kLayoutSw128),
-                      smem_desc(k_base + k * 32, 16, 1024, kLayoutSw128), idesc_s, k != 0);
-        umma_commit(&S.s_full[wg]);
-        return true;
-      };
-      auto issue_pv = [&](int wg, int j) -> bool {
-        const int s = j % AT_STAGES;
-        if (wg == 0 && !mbar_wait(&S.v_ready[s], (j / AT_STAGES) & 1, err)) return false;
-        if (!mbar_wait(&S.p_full[wg], j & 1, err)) return false;
-        tc_fence_after();
-        const uint32_t v_base = smem_u32(S.V[s]);
-#pragma unroll
-        for (int k = 0; k < AT_BN / 16; ++k) {
-          const uint32_t a_addr = smem_u32(S.P[wg][k >> 2]) + (k & 3) * 32;
-          const uint64_t ad = smem_desc(a_addr, 16, 1024, kLayoutSw128);
-          umma_f16_ss(tmem + 256u + wg * 64u, ad, smem_desc(v_base + k * 16 * AT_D * 2, 16, 1024, kLayoutSw128),
-                      idesc_o, (j | k) != 0);
-          // every element of the ones tile is 1.0, so one 16-key slice serves every step
-          umma_f16_ss(tmem + 384u + wg * 16u, ad, smem_desc(ones_base + (k & 3) * 32, 16, 1024, kLayoutSw128),
-                      idesc_l, (j | k) != 0);
-        }
-        if (wg == 1) umma_commit(&S.kv_empty[s]);
-        umma_commit(&S.pv_done[wg]);
-        return true;
-      };
-      if (ok) ok = issue_s(0, 0);
-      if (ok) ok = issue_s(1, 0);
-      for (int j = 0; ok && j < ntile; ++j) {
-        if (j + 1 < ntile) ok = issue_s(0, j + 1);
-        if (ok) ok = issue_pv(0, j);
-        if (ok && j + 1 < ntile) ok = issue_s(1, j + 1);
-        if (ok) ok = issue_pv(1, j);
-      }
-    }
-  } else if (warp >= 10) {
-    // ---------------- V_j: bf16 -> f16 in place (each 32-bit word holds a pair)
-    const int ct = threadIdx.x - 10 * 32;
-    for (int j = 0; j < ntile; ++j) {
-      const int s = j % AT_STAGES;
-      if (!__all_sync(0xffffffffu, mbar_wait(&S.kv_full[s], (j / AT_STAGES) & 1, err))) break;
-      uint4* v4 = reinterpret_cast<uint4*>(S.V[s]);
-#pragma unroll 4
-      for (int i = ct; i < AT_BN * AT_D / 8; i += AH_CONV_THREADS) {
-        uint4 w = v4[i];
-        uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float a = __uint_as_float(wp[e] << 16), c = __uint_as_float(wp[e] & 0xFFFF0000u);
-          const __half2 h = __floats2half2_rn(a, c);
-          wp[e] = *reinterpret_cast<const uint32_t*>(&h);
-        }
-        v4[i] = w;
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.v_ready[s]);
-    }
-  } else {
-    const int wg = (warp - 2) >> 2;
-    const int q4 = warp & 3;
-    const int r = q4 * 32 + lane;
-    const int tq = t0 + r;
-    const int t = tk0 + r;
-    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    const uint32_t tS = tmem + wg * 128u + lane_off;
-    const uint32_t tO = tmem + 256u + wg * 64u + lane_off;
-    const uint32_t tL = tmem + 384u + wg * 16u + lane_off;
-    auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
-      const bool w = mbar_wait(bar, par, err);
-      return __all_sync(0xffffffffu, w);
-    };
-    float m_run = -INFINITY;
-    bool ok = true;
-    const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
-    for (int j = 0; j < ntile; ++j) {
-      const int kb = kb0 + j * AT_BN;
-      if (!wait_all(&S.s_full[wg], j & 1)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t sr[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr + c * 32);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.s_free[wg]);
-      const bool edge = (kb + AT_BN - 1 > tk0) || (kb < tk0 + AT_BM - p.window);
-      if (edge) {
-        const int hi = tq < p.L ? t - kb : -1;
-        const int lo_i = t - p.window - kb;
-#pragma unroll
-        for (int i = 0; i < 128; ++i)
-          if (i > hi || i <= lo_i) sr[i] = __float_as_uint(-INFINITY);
-      }
-      float m8[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
-#pragma unroll
-      for (int i = 0; i < 128; i += 2)
-        m8[(i >> 1) & 7] = fmax3(m8[(i >> 1) & 7], __uint_as_float(sr[i]), __uint_as_float(sr[i + 1]));
-      const float mraw = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-      const float mt = mraw * p.scale_log2;
-      const bool need = mt > m_run + kRescaleThresh;
-      float alpha = 1.f;
-      if (need) {
-        if (m_run != -INFINITY) alpha = exp2f(m_run - mt);
-        m_run = mt;
-      }
-      if (j >= 1 && !wait_all(&S.pv_done[wg], (j - 1) & 1)) { ok = false; break; }
-      tc_fence_after();
-      if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {  // O and its row sums, in TMEM
-#pragma unroll
-        for (int c = 0; c < 5; ++c) {
-          uint32_t orr[16];
-          const uint32_t a = c < 4 ? tO + c * 16 : tL;
-          tmem_ld16(a, orr);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 16; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
-          tmem_st16(a, orr);
-        }
-        tmem_wait_st();
-      }
-      const float msub = m_run == -INFINITY ? 0.f : m_run;
-      const float2 nm2 = make_float2(-msub, -msub);
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        unsigned char* prow = reinterpret_cast<unsigned char*>(S.P[wg][half]) + r * 128;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {  // 16-byte chunk c: keys 8c .. 8c + 7 of this half
-          uint32_t hv[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int i = half * 64 + c * 8 + 2 * q;
-            const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), sc2, nm2);
-            if (q < kPolyPairs) {  // on the FMA pipe, then rounded to f16
-              const float2 y = exp2_poly2(x);
-              const __half2 yh = __floats2half2_rn(y.x, y.y);
-              hv[q] = *reinterpret_cast<const uint32_t*>(&yh);
-            } else {
-              const __half2 xh = __floats2half2_rn(x.x, x.y);
-              hv[q] = ex2_h2(*reinterpret_cast<const uint32_t*>(&xh));
-            }
-          }
-          *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-        }
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.p_full[wg]);
-    }
-    if (ok && wait_all(&S.pv_done[wg], (ntile - 1) & 1)) {
-      tc_fence_after();
-      uint32_t orr[64], lr[16];
-      tmem_ld32(tO, orr);
-      tmem_ld32(tO + 32, orr + 32);
-      tmem_ld16(tL, lr);
-      tmem_wait_ld();
-      const float l = __uint_as_float(lr[0]);
-      if (tq < p.L && l > 0.f) {
-        const float inv = 1.f / l;
-        bf16* op = p.o + ((int64_t)b * p.L + tq) * p.ld_o + (int64_t)(h0 + wg) * AT_D;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          float f[8];
-#pragma unroll
-          for (int q = 0; q < 8; ++q) f[q] = __uint_as_float(orr[c * 8 + q]) * inv;
-          store8(op + c * 8, f);
-        }
-      }
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
-  }
-}
-
 // [B, L, H * d] rows of stride ld; boxes of 64 columns x `rows` rows (128B swizzle)
 bool make_head_map(CUtensorMap* m, const void* base, int64_t ld, int H, int d, int L, int B, int rows) {
   uint64_t dims[3] = {(uint64_t)H * d, (uint64_t)L, (uint64_t)B};
@@ -1486,18 +1189,6 @@ samba_status launch_swa_tc(const SwaArgs& a, cudaStream_t st) {
     return SAMBA_OK;
   }
   const char* kenv = getenv("SAMBA_SWA_KERNEL");
-  if (grp % 2 == 0 && kenv && kenv[0] == 'h') {
-    const char* pe = getenv("SAMBA_SWA_POLY");
-    const int poly = (pe && pe[0] >= '0' && pe[0] <= '3') ? pe[0] - '0' : 1;
-    auto kern = poly == 0 ? swa_tc2h_kernel<0> : poly == 2 ? swa_tc2h_kernel<2> : poly == 3 ? swa_tc2h_kernel<3>
-                                                                                             : swa_tc2h_kernel<1>;
-    const size_t smem = sizeof(AtHSmem2) + 1024;
-    if (!ensure_smem_attr(kern, smem)) return SAMBA_ERR_CUDA;
-    dim3 grid((a.L + AT_BM - 1) / AT_BM, a.Hq / 2, a.B);
-    kern<<<grid, AH_THREADS, smem, st>>>(p, device_error_word());
-    SAMBA_CHECK_LAUNCH();
-    return SAMBA_OK;
-  }
   if (grp % A4_HEADS == 0 && !(kenv && (kenv[0] == '1' || kenv[0] == '2'))) {
     CUtensorMap tk, tv;
     if (!make_head_map(&tk, a.k, a.ld_k, a.Hkv, a.d, Lk, a.B, A4_BN) ||
