@@ -498,14 +498,18 @@ def kernel_report(kt, s, T, Bn, Ln, peaks, t_up_live=None, clocks=None):
         note = (f"the sustained bf16 figure ({tf_sus} TF/s) is below this kernel's measured rate; "
                 f"the burst figure is used as the peak")
         peak, kind = tf_burst, "burst"
-    pk_mhz = peak_clock_mhz(kind)
     run_mhz = (clocks or {}).get("sm_mhz")
-    frac_clk = (achieved / run_mhz) / (peak / pk_mhz) if (pk_mhz and run_mhz) else None
+    # per-clock comparison with a peak whose clock is known (the chosen peak's,
+    # else the sustained figure's): (achieved / run MHz) / (peak / peak MHz)
+    norm_kind = kind if peak_clock_mhz(kind) else "sustained"
+    pk_mhz = peak_clock_mhz(norm_kind)
+    pk_val = peak if norm_kind == kind else tf_sus
+    frac_clk = (achieved / run_mhz) / (pk_val / pk_mhz) if (pk_mhz and run_mhz) else None
     roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
             "frac": round(achieved / peak, 4), "traffic": round(traffic) if traffic else None,
             "frac_clock_normalised": round(frac_clk, 4) if frac_clk else None,
             "clock_normalisation": (f"(achieved / {run_mhz:.0f} MHz median SM clock of this run) / "
-                                    f"(peak / {pk_mhz:.0f} MHz at which the peak was taken)")
+                                    f"({norm_kind} peak {pk_val} TF/s / {pk_mhz:.0f} MHz at which it was taken)")
             if frac_clk else "peak clock unknown",
             "denominator_note": note,
             "algorithmic_flops": up,

@@ -201,6 +201,7 @@ struct TcParams {
   int umma_n;      // accumulator columns per tile (2*bn for SwiGLU)
   int n_tiles, m_tiles, k_blocks;
   int group_n;  // n-tiles per raster group (divides n_tiles)
+  int a_evict_first;  // activations streamed with an evict-first L2 policy
   int seg_start[3];
 };
 
@@ -399,9 +400,13 @@ __global__ void __launch_bounds__(TcEpi<EPI>::threads, 1) gemm_tc_kernel(const _
     // ---------------- TMA producer
     if (elect_one()) {
       const uint32_t bytes = TC_A_BYTES + (uint32_t)p.umma_n * TC_BK * 2;
-      // activations stream through once per n-tile group; the group's weight
-      // panel is reused by every m-tile, so it is kept in L2 ahead of them
-      const uint64_t pol_a = l2_policy_evict_first(), pol_b = l2_policy_evict_last();
+      // The group's weight panel is reused by every m-tile: kept in L2 ahead of
+      // the activations.  When K is long, a 128-row activation block (>= 1 MB)
+      // is the bulk of the traffic and is streamed evict-first; shorter blocks
+      // are left at normal priority, since the group's n-tiles read each one
+      // several times while it is in flight.
+      const uint64_t pol_a = p.a_evict_first ? l2_policy_evict_first() : l2_policy_evict_normal();
+      const uint64_t pol_b = l2_policy_evict_last();
       int it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
@@ -553,6 +558,7 @@ samba_status launch_gemm_tc(const GemmArgs& a, cudaStream_t st) {
       if (p.n_tiles % g == 0 && (size_t)g * panel <= (size_t(32) << 20)) p.group_n = g;
   }
   p.k_blocks = (a.K + TC_BK - 1) / TC_BK;
+  p.a_evict_first = a.K >= 4096 ? 1 : 0;
   {
     uint64_t dims[2] = {(uint64_t)a.K, (uint64_t)a.M};
     uint64_t strides[1] = {(uint64_t)a.lda};
