@@ -32,18 +32,23 @@ constexpr int SK_THREADS = 192;
 // Shared memory: a ring of stages (W tile | W2 tile (SwiGLU) | X tile) that is
 // reused, once every MMA has completed, for the fp32 partial tile(s) of the
 // cluster reduction; barriers and the TMEM address live after it.
-// 96 KB: two CTAs fit an SM, so that (with programmatic dependent launch) the
-// next projection's CTAs become resident and fetch their first weight stages
-// while the previous projection's CTAs reduce and write their outputs.
+// 96 KB for single-weight projections: two CTAs fit an SM, so that (with
+// programmatic dependent launch) the next projection's CTAs become resident and
+// fetch their first weight stages while the previous projection's CTAs reduce
+// and write their outputs.  200 KB for the SwiGLU pair: its stages carry two
+// weight tiles, and bytes in flight matter more there than the overlap.
 constexpr int SK_RING_BYTES = 96 * 1024;
+constexpr int SK_RING_BYTES_DUAL = 200 * 1024;
 constexpr int SK_RED_PITCH = SK_MAXB + 1;
 static_assert(2 * SK_BM * SK_RED_PITCH * 4 <= SK_RING_BYTES, "reduction tiles must fit in the ring");
 
+template <int kRing>
 struct SkSmem {
-  unsigned char ring[SK_RING_BYTES];
+  unsigned char ring[kRing];
   uint64_t full[SK_STAGES], empty[SK_STAGES], done;
   uint32_t tmem_base;
 };
+template <int EPI> constexpr int sk_ring_bytes() { return EPI == kEpiSwiglu ? SK_RING_BYTES_DUAL : SK_RING_BYTES; }
 
 struct SkParams {
   CUtensorMap tmW[3];
@@ -103,7 +108,8 @@ __device__ __forceinline__ float2 rope_cs_sk(const float2* __restrict__ tab, int
 template <int EPI>
 __global__ void __launch_bounds__(SK_THREADS, 2) gemm_skinny_kernel(const __grid_constant__ SkParams p, int* err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  SkSmem& S = *reinterpret_cast<SkSmem*>(smem_raw + smem_align_pad(smem_raw, 1024));
+  SkSmem<sk_ring_bytes<EPI>()>& S =
+      *reinterpret_cast<SkSmem<sk_ring_bytes<EPI>()>*>(smem_raw + smem_align_pad(smem_raw, 1024));
   const GemmArgs& a = p.a;
   const int warp = warp_id_sync();
   const int lane = threadIdx.x & 31;
@@ -327,7 +333,7 @@ bool gemm_skinny_supported(const GemmArgs& a) {
 
 template <int EPI>
 static samba_status skinny_launch(const SkParams& p, int ntiles, cudaStream_t st) {
-  const size_t smem = sizeof(SkSmem) + 1024;
+  const size_t smem = sizeof(SkSmem<sk_ring_bytes<EPI>()>) + 1024;
   auto kern = gemm_skinny_kernel<EPI>;
   if (!ensure_smem_attr(kern, smem)) return SAMBA_ERR_CUDA;
   cudaLaunchConfig_t cfg;
@@ -360,7 +366,7 @@ samba_status launch_gemm_skinny(const GemmArgs& a, cudaStream_t st) {
   {
     const int xb = ((p.MB * SK_BK * 2) + 1023) / 1024 * 1024;
     p.stage_bytes = (a.epi == kEpiSwiglu ? 2 : 1) * SK_BM * SK_BK * 2 + xb;
-    p.stages = SK_RING_BYTES / p.stage_bytes;
+    p.stages = (a.epi == kEpiSwiglu ? SK_RING_BYTES_DUAL : SK_RING_BYTES) / p.stage_bytes;
     if (p.stages > SK_STAGES) p.stages = SK_STAGES;
   }
   const int ntiles = (a.N + SK_BM - 1) / SK_BM;
