@@ -47,7 +47,9 @@ typedef enum {
   SAMBA_ERR_UNSUPPORTED = 2,  /* valid but not handled by these kernels (misaligned, N != 16, ...) */
   SAMBA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed (launch, tensor-map encode) */
   SAMBA_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up (from samba_get_error) */
-  SAMBA_ERR_DEVICE = 5        /* a device-side check failed (from samba_get_error) */
+  SAMBA_ERR_DEVICE = 5,       /* a device-side check failed (from samba_get_error) */
+  SAMBA_ERR_BOUNDS = 6        /* debug-check build: an index bounds check or a workspace
+                                 guard band failed (from samba_get_error) */
 } samba_status;
 
 typedef enum { SAMBA_F32 = 0, SAMBA_BF16 = 1 } samba_dtype;
@@ -94,9 +96,44 @@ int samba_gemm_timing_count(void);
 samba_status samba_debug_scan_stall(int stop_after_chunks, uint64_t wait_limit_ns);
 
 /* Synchronises `stream`, returns and clears the device error word of the
- * current device: SAMBA_OK, SAMBA_ERR_TIMEOUT or SAMBA_ERR_DEVICE, or
- * SAMBA_ERR_CUDA if the synchronisation itself failed. */
+ * current device: SAMBA_OK, SAMBA_ERR_TIMEOUT, SAMBA_ERR_DEVICE or (debug-check
+ * build) SAMBA_ERR_BOUNDS, or SAMBA_ERR_CUDA if the synchronisation itself
+ * failed.  The word keeps the first error latched since it was last read. */
 samba_status samba_get_error(samba_stream stream);
+
+/* ------------------------------------------------------------------------
+ * Debug-check build.  libsamba_debug.so is the same library compiled with
+ * SAMBA_DEBUG_CHECKS=1 (same symbols, same results):
+ *   - device index checks: before the accesses they guard (tile and chunk
+ *     coordinates, ring slots, key ranges, reduction slots, output rows), the
+ *     kernels check the index against the extent it must stay in; a failed
+ *     check skips the access and latches SAMBA_ERR_BOUNDS with its site, and the
+ *     kernel runs on (no trap, no assert);
+ *   - workspace guard bands: every sub-buffer the library carves from a
+ *     workspace is followed by a 4 KiB band that is filled with a pattern
+ *     before the call's kernels and verified after them; the workspace-size
+ *     queries include the bands.
+ * ---------------------------------------------------------------------- */
+
+/* 1 in the debug-check build, 0 in the release build. */
+int samba_debug_checks_enabled(void);
+
+/* Where the check behind the calling thread's last SAMBA_ERR_BOUNDS from
+ * samba_get_error failed ("file.cu:line", or "workspace guard band <i>
+ * overwritten"); "" if none.  Owned by the library, per thread. */
+const char* samba_last_check_site(void);
+
+/* Self-test of the debug checks; makes no out-of-bounds access of any kind.
+ * kind 0: a kernel evaluates one device check on an index the host chose out
+ *         of range and skips the access it guards;
+ * kind 1: two sub-buffers of 4 KiB are carved from `workspace` with their guard
+ *         bands, one byte inside the first band (memory of the caller's
+ *         workspace) is changed between the fill and the verification.
+ * Both then latch SAMBA_ERR_BOUNDS for samba_get_error.  Returns
+ * SAMBA_ERR_UNSUPPORTED in the release build, SAMBA_ERR_INVALID_ARG for another
+ * kind or (kind 1) a workspace smaller than samba_debug_selftest_workspace_size(). */
+size_t samba_debug_selftest_workspace_size(void);
+samba_status samba_debug_check_selftest(int kind, void* workspace, size_t workspace_bytes, samba_stream stream);
 
 /* ------------------------------------------------------------------------
  * Selective scan (S6)  [Samba 3.4 "The State Space Model Update (S6)",

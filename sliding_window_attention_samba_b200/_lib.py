@@ -13,11 +13,15 @@ import os
 from typing import Optional, Sequence
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libsamba.so")
+# SAMBA_DEBUG_CHECKS=1 selects the debug-check build (device index checks and
+# workspace guard bands; same symbols and results)
+DEBUG_CHECKS = os.environ.get("SAMBA_DEBUG_CHECKS", "0") not in ("", "0")
+LIB_PATH = os.path.join(_HERE, "libsamba_debug.so" if DEBUG_CHECKS else "libsamba.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m sliding_window_attention_samba_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python -m sliding_window_attention_samba_b200.build"
+        f"{' --debug-checks' if DEBUG_CHECKS else ''}` "
         "(the CUDA path has no CPU fallback)")
 
 _L = ctypes.CDLL(LIB_PATH)
@@ -30,10 +34,10 @@ c_float = ctypes.c_float
 
 SAMBA_F32, SAMBA_BF16 = 0, 1
 (SAMBA_OK, SAMBA_ERR_INVALID_ARG, SAMBA_ERR_UNSUPPORTED, SAMBA_ERR_CUDA, SAMBA_ERR_TIMEOUT,
- SAMBA_ERR_DEVICE) = range(6)
+ SAMBA_ERR_DEVICE, SAMBA_ERR_BOUNDS) = range(7)
 EPI_NONE, EPI_RESIDUAL, EPI_SWIGLU, EPI_SOFTPLUS_BIAS = 0, 1, 2, 3
 STATUS = {0: "SAMBA_OK", 1: "SAMBA_ERR_INVALID_ARG", 2: "SAMBA_ERR_UNSUPPORTED", 3: "SAMBA_ERR_CUDA",
-          4: "SAMBA_ERR_TIMEOUT", 5: "SAMBA_ERR_DEVICE"}
+          4: "SAMBA_ERR_TIMEOUT", 5: "SAMBA_ERR_DEVICE", 6: "SAMBA_ERR_BOUNDS"}
 
 
 class SambaError(RuntimeError):
@@ -93,6 +97,10 @@ _set_timing = _sig("samba_set_gemm_timing", c_int, [c_int, c_void_p, c_void_p, c
 _timing_count = _sig("samba_gemm_timing_count", c_int, [])
 _get_error = _sig("samba_get_error", c_int, [c_void_p])
 _scan_stall = _sig("samba_debug_scan_stall", c_int, [c_int, ctypes.c_uint64])
+_dbg_enabled = _sig("samba_debug_checks_enabled", c_int, [])
+_check_site = _sig("samba_last_check_site", ctypes.c_char_p, [])
+_selftest_ws = _sig("samba_debug_selftest_workspace_size", c_size_t, [])
+_selftest = _sig("samba_debug_check_selftest", c_int, [c_int, c_void_p, c_size_t, c_void_p])
 _scan_ws = _sig("samba_selective_scan_workspace_size", c_size_t, [c_int, c_int, c_int, c_int])
 _scan = _sig("samba_selective_scan", c_int,
              [c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
@@ -203,6 +211,23 @@ def samba_debug_scan_stall(stop_after_chunks: int, wait_limit_ns: int = 0) -> No
 
 def samba_get_error(stream=None) -> int:
     return _get_error(_stream(stream))
+
+
+def samba_debug_checks_enabled() -> int:
+    return _dbg_enabled()
+
+
+def samba_last_check_site() -> str:
+    return _check_site().decode()
+
+
+def samba_debug_selftest_workspace_size() -> int:
+    return _selftest_ws()
+
+
+def samba_debug_check_selftest(kind: int, workspace=None, workspace_bytes: int = 0, stream=None) -> int:
+    """Returns the status code (SAMBA_ERR_UNSUPPORTED in the release build)."""
+    return _selftest(kind, _p(workspace), workspace_bytes, _stream(stream))
 
 
 def samba_selective_scan_workspace_size(B, L, D, N) -> int:

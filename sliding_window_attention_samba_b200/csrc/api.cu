@@ -10,6 +10,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#define SAMBA_TU_ID 1  // site id of this file in debug-check reports
 #include "common.cuh"
 #include "decode.h"
 #include "kernels.h"
@@ -67,6 +68,21 @@ samba_status note_cuda_failure(const char* where, int cuda_error) {
   snprintf(g_cuda_err_msg, sizeof(g_cuda_err_msg), "%s: %s (%d)", where,
            cudaGetErrorString((cudaError_t)cuda_error), cuda_error);
   return SAMBA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Site of the last failed debug check read by samba_get_error (calling thread)
+// ---------------------------------------------------------------------------
+static thread_local char g_check_site[96] = {0};
+static void note_check_site(int word) {
+  static const char* const files[16] = {"?", "api.cu", "decode.cu", "elementwise.cu", "gemm.cu", "gemm_skinny.cu",
+                                        "scan.cu", "swa.cu", "swa_noalloc.cu", "swa_tc.cu", "?", "?", "?", "?",
+                                        "?", "workspace guard band"};
+  const int tu = (word >> 4) & 15, line = (word >> 8) & 0x7fffff;
+  if (tu == kGuardSiteTu)
+    snprintf(g_check_site, sizeof(g_check_site), "%s %d overwritten", files[tu], line);
+  else
+    snprintf(g_check_site, sizeof(g_check_site), "%s:%d", files[tu], line);
 }
 
 // ---------------------------------------------------------------------------
@@ -136,18 +152,45 @@ bool make_tmap(CUtensorMap* m, const void* base, samba_dtype dt, int rank, const
 // ---------------------------------------------------------------------------
 // Workspace carving (256-byte aligned sub-buffers)
 // ---------------------------------------------------------------------------
+// Workspace carving: 256-byte aligned sub-buffers.  In the debug-check build
+// every sub-buffer is followed by a guard band that is filled with a pattern
+// before the call's kernels run and verified after them (guards_arm /
+// guards_check), so a kernel that writes past the end of its buffer is
+// reported as SAMBA_ERR_BOUNDS naming the band.
 struct Carve {
   size_t off = 0;
+  int nguard = 0;
+  size_t guard[kMaxGuards];
   size_t take(size_t bytes) {
     const size_t o = off;
     off = (off + bytes + 255) & ~size_t(255);
+    if (kGuardBytes && nguard < kMaxGuards) {
+      guard[nguard++] = off;
+      off += kGuardBytes;
+    }
     return o;
   }
 };
 
+static samba_status guards_arm(char* base, const Carve& c, cudaStream_t st) {
+  if (!c.nguard) return SAMBA_OK;
+  GuardList g;
+  g.n = c.nguard;
+  for (int i = 0; i < c.nguard; ++i) g.off[i] = c.guard[i];
+  return launch_guard_fill(base, g, st);
+}
+static samba_status guards_check(char* base, const Carve& c, cudaStream_t st) {
+  if (!c.nguard) return SAMBA_OK;
+  GuardList g;
+  g.n = c.nguard;
+  for (int i = 0; i < c.nguard; ++i) g.off[i] = c.guard[i];
+  return launch_guard_check(base, g, st);
+}
+
 struct BlockPlan {
   size_t tab, xn, hz, u, xdbl, dlt, y, x1, x2, x3, hmlp, qkv, o, kx, vx, convh, total;
   int xdw, qkvw;
+  Carve cv;  // the carving (guard bands of the debug-check build)
 };
 
 // Workspace of one block over T = B*L tokens; a chunked prefill (chunk_B > 0)
@@ -176,6 +219,7 @@ static BlockPlan plan_block(const samba_block_config& c, int64_t T, int chunk_B 
   p.vx = cv.take(kv_rows * c.n_kv * c.head_dim * es);
   p.convh = cv.take((int64_t)chunk_B * c.d_inner * (c.d_conv - 1) * es);
   p.total = cv.off + 256;  // slack for aligning the caller's base pointer
+  p.cv = cv;
   return p;
 }
 
@@ -265,6 +309,7 @@ const char* samba_status_string(samba_status s) {
     case SAMBA_ERR_CUDA: return "SAMBA_ERR_CUDA";
     case SAMBA_ERR_TIMEOUT: return "SAMBA_ERR_TIMEOUT";
     case SAMBA_ERR_DEVICE: return "SAMBA_ERR_DEVICE";
+    case SAMBA_ERR_BOUNDS: return "SAMBA_ERR_BOUNDS";
   }
   return "SAMBA_ERR_UNKNOWN";
 }
@@ -299,8 +344,40 @@ samba_status samba_get_error(samba_stream stream) {
     const int zero = 0;
     if (cudaMemcpy(w, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return SAMBA_ERR_CUDA;
   }
+  if ((v & 15) == kErrBounds) {
+    note_check_site(v);
+    return SAMBA_ERR_BOUNDS;
+  }
   return v == kErrTimeout ? SAMBA_ERR_TIMEOUT : (v ? SAMBA_ERR_DEVICE : SAMBA_OK);
 }
+
+int samba_debug_checks_enabled(void) { return SAMBA_DEBUG_CHECKS; }
+
+size_t samba_debug_selftest_workspace_size(void) {
+  Carve cv;
+  cv.take(4096);
+  cv.take(4096);
+  return cv.off + 256;
+}
+
+samba_status samba_debug_check_selftest(int kind, void* workspace, size_t workspace_bytes, samba_stream stream) {
+  cudaStream_t st = (cudaStream_t)stream;
+  if (kind != 0 && kind != 1) return SAMBA_ERR_INVALID_ARG;
+  if (!SAMBA_DEBUG_CHECKS) return SAMBA_ERR_UNSUPPORTED;
+  if (kind == 0) return launch_dcheck_selftest(st);
+  if (!workspace || workspace_bytes < samba_debug_selftest_workspace_size()) return SAMBA_ERR_INVALID_ARG;
+  char* base = (char*)(((uintptr_t)workspace + 255) & ~uintptr_t(255));
+  Carve cv;
+  cv.take(4096);
+  cv.take(4096);
+  TRY(guards_arm(base, cv, st));
+  // one byte of the first band: inside the caller's workspace, outside every sub-buffer
+  if (cudaMemsetAsync(base + cv.guard[0] + 17, 0x11, 1, st) != cudaSuccess)
+    return note_cuda_failure("cudaMemsetAsync (guard self-test)", cudaGetLastError());
+  return guards_check(base, cv, st);
+}
+
+const char* samba_last_check_site(void) { return g_check_site; }
 
 // ------------------------------------------------------------------ scan
 size_t samba_selective_scan_workspace_size(int, int, int, int) { return 0; }
@@ -382,11 +459,14 @@ samba_status samba_swa_fwd(const void* q, const void* k, const void* v, void* o,
     float2* tab = (float2*)(base + cv.take(rope_table_bytes(head_dim)));
     void* qr = base + cv.take((size_t)B * L * Hq * head_dim * es);
     void* kr = base + cv.take((size_t)B * L * Hkv * head_dim * es);
+    TRY(guards_arm(base, cv, st));
     TRY(launch_build_rope_table(tab, head_dim, rope_base, st));
     TRY(launch_rope_apply(q, qr, B, L, Hq, head_dim, pos0, tab, dtype, st));
     TRY(launch_rope_apply(k, kr, B, L, Hkv, head_dim, pos0, tab, dtype, st));
     a.q = qr;
     a.k = kr;
+    TRY(launch_swa(a, st));
+    return guards_check(base, cv, st);
   }
   return launch_swa(a, st);
 }
@@ -751,6 +831,7 @@ static samba_status block_forward(const samba_block_config* cfg, const samba_blo
   }
 
   const LayerCtx X{c, P, base, B, L, T, st};
+  TRY(guards_arm(base, P.cv, st));
   TRY(mamba_sublayer(X, w, x_in, x1, stt, resume, taps ? taps->branch[0] : nullptr));
   // ---- MLP 1
   TRY(mlp_sublayer(c, w->norm_g[1], w->mlp1_W1, w->mlp1_W2, w->mlp1_W3, x1, x2, xn, buf(P.hmlp),
@@ -759,6 +840,7 @@ static samba_status block_forward(const samba_block_config* cfg, const samba_blo
   // ---- MLP 2
   TRY(mlp_sublayer(c, w->norm_g[3], w->mlp2_W1, w->mlp2_W2, w->mlp2_W3, x3, x_out, xn, buf(P.hmlp),
                    taps ? taps->branch[3] : nullptr, T, st));
+  TRY(guards_check(base, P.cv, st));
   if (resume) return launch_pos_check_set(stt->pos, B, pos0, pos0 + L, st);
   if (stt) TRY(launch_pos_update(stt->pos, B, L, true, st));
   return SAMBA_OK;
@@ -796,6 +878,7 @@ namespace samba {
 struct ModelPlan {
   BlockPlan P;                 // one sub-layer's activations over all B*L tokens
   size_t xa, xb, xl, total;    // two residual streams, the normed last rows
+  Carve cv;
 };
 
 static ModelPlan plan_model(const samba_block_config& c, int B, int L) {
@@ -803,12 +886,13 @@ static ModelPlan plan_model(const samba_block_config& c, int B, int L) {
   const int64_t T = (int64_t)B * L;
   const size_t es = dtype_size(c.dtype);
   m.P = plan_block(c, T);
-  Carve cv;
+  Carve cv = m.P.cv;  // keeps the block's guard bands
   cv.off = m.P.total;
   m.xa = cv.take(T * c.d_model * es);
   m.xb = cv.take(T * c.d_model * es);
   m.xl = cv.take((size_t)B * c.d_model * es);
   m.total = cv.off + 256;
+  m.cv = cv;
   return m;
 }
 
@@ -857,6 +941,7 @@ samba_status samba_model_prefill(const samba_model* m, const int32_t* ids, void*
   const int Dm = c.d_model;
   char* cur = base + MP.xa;
   char* nxt = base + MP.xb;
+  TRY(guards_arm(base, MP.cv, st));
   TRY(launch_embedding(ids, m->embedding, cur, T, Dm, m->vocab, dt, st));
   const LayerCtx X{c, MP.P, base, B, L, T, st};
   for (int i = 0; i < m->n_layers; ++i) {
@@ -874,7 +959,8 @@ samba_status samba_model_prefill(const samba_model* m, const int32_t* ids, void*
   // final RMSNorm of each sequence's last position, then the vocabulary projection
   TRY(launch_rmsnorm(cur + (size_t)(L - 1) * Dm * es, (int64_t)L * Dm, m->final_norm, base + MP.xl, Dm, B, Dm,
                      c.norm_eps, dt, st));
-  return launch_gemm(gemm1(base + MP.xl, Dm, m->lm_head, B, m->vocab, Dm, logits, m->vocab, dt), st);
+  TRY(launch_gemm(gemm1(base + MP.xl, Dm, m->lm_head, B, m->vocab, Dm, logits, m->vocab, dt), st));
+  return guards_check(base, MP.cv, st);
 }
 
 }  // extern "C"
@@ -884,13 +970,14 @@ namespace samba {
 struct ModelStepPlan {
   BlockPlan P;
   size_t xa, xb, xl, attn, attn_bytes, total;
+  Carve cv;
 };
 
 static ModelStepPlan plan_model_step(const samba_block_config& c, int B) {
   ModelStepPlan m;
   const size_t es = dtype_size(c.dtype);
   m.P = plan_block(c, B);
-  Carve cv;
+  Carve cv = m.P.cv;
   cv.off = m.P.total;
   m.xa = cv.take((size_t)B * c.d_model * es);
   m.xb = cv.take((size_t)B * c.d_model * es);
@@ -898,6 +985,7 @@ static ModelStepPlan plan_model_step(const samba_block_config& c, int B) {
   m.attn_bytes = attn_decode_workspace_bytes(B, c.n_kv, c.window);
   m.attn = cv.take(m.attn_bytes);
   m.total = cv.off + 256;
+  m.cv = cv;
   return m;
 }
 
@@ -934,6 +1022,7 @@ samba_status samba_model_step(const samba_model* m, const int32_t* ids_t, void* 
   const int Dm = c.d_model;
   char* cur = base + MP.xa;
   char* nxt = base + MP.xb;
+  TRY(guards_arm(base, MP.cv, st));
   TRY(launch_embedding(ids_t, m->embedding, cur, B, Dm, m->vocab, dt, st));
   const LayerCtx X{c, MP.P, base, B, 1, (int64_t)B, st};
   for (int i = 0; i < m->n_layers; ++i) {
@@ -955,6 +1044,7 @@ samba_status samba_model_step(const samba_model* m, const int32_t* ids_t, void* 
   GemmArgs g = gemm1(base + MP.xl, Dm, m->lm_head, B, m->vocab, Dm, logits, m->vocab, dt);
   g.pdl = true;
   TRY(launch_gemm(g, st));
+  TRY(guards_check(base, MP.cv, st));
   return launch_pos_update(pos, B, 1, false, st, true);
 }
 
@@ -981,12 +1071,14 @@ samba_status samba_step(const samba_block_config* cfg, const samba_block_weights
   char* base = (char*)(((uintptr_t)workspace + 255) & ~uintptr_t(255));
   const LayerCtx X{c, P, base, B, 1, (int64_t)B, st};
   void *x1 = base + P.x1, *x2 = base + P.x2, *x3 = base + P.x3;
+  TRY(guards_arm(base, P.cv, st));
   TRY(mamba_step_layer(X, w, x_t, x1, stt->ssm, stt->conv));
   TRY(mlp_sublayer(c, w->norm_g[1], w->mlp1_W1, w->mlp1_W2, w->mlp1_W3, x1, x2, base + P.xn, base + P.hmlp, nullptr,
                    B, st, true));
   TRY(swa_step_layer(X, w, x2, x3, stt->k_ring, stt->v_ring, stt->pos, nullptr, 0));
   TRY(mlp_sublayer(c, w->norm_g[3], w->mlp2_W1, w->mlp2_W2, w->mlp2_W3, x3, y_t, base + P.xn, base + P.hmlp, nullptr,
                    B, st, true));
+  TRY(guards_check(base, P.cv, st));
   return launch_pos_update(stt->pos, B, 1, false, st, true);
 }
 

@@ -17,7 +17,10 @@ namespace samba {
 // ---------------------------------------------------------------------------
 // Device error word (one per device, latched; read and cleared by samba_get_error)
 // ---------------------------------------------------------------------------
-enum : int { kErrNone = 0, kErrTimeout = 1, kErrDevice = 2 };
+enum : int { kErrNone = 0, kErrTimeout = 1, kErrDevice = 2, kErrBounds = 3 };
+// The word holds the first error latched since it was last read: the code in
+// bits 0..3; for kErrBounds also the check's site, the source file id in bits
+// 4..7 (SAMBA_TU_ID of the translation unit) and its line in bits 8..30.
 
 int* device_error_word();  // device address of the error word of the current device
 uintptr_t current_context_id();  // the calling thread's current CUDA context (0: none yet)
@@ -28,6 +31,30 @@ samba_status note_cuda_failure(const char* where, int cuda_error);
 __device__ __forceinline__ void raise_error(int* err, int code) {
   if (err) atomicCAS(err, 0, code);
 }
+
+// ---------------------------------------------------------------------------
+// Debug-build checks.  Built with -DSAMBA_DEBUG_CHECKS=1 (libsamba_debug.so),
+// SAMBA_DCHECK(err, cond) evaluates an index or range condition before the
+// access it guards; when it fails it latches kErrBounds with the check's site
+// in the device error word and evaluates to false, so that the caller skips
+// the access (no trap, no assert: the context stays usable).  In the release
+// build it is the constant true and costs nothing.
+// ---------------------------------------------------------------------------
+#ifndef SAMBA_TU_ID
+#define SAMBA_TU_ID 0
+#endif
+#ifndef SAMBA_DEBUG_CHECKS
+#define SAMBA_DEBUG_CHECKS 0
+#endif
+__device__ __forceinline__ bool dcheck_fail(int* err, int tu, int line) {
+  raise_error(err, kErrBounds | ((tu & 15) << 4) | ((line & 0x7fffff) << 8));
+  return false;
+}
+#if SAMBA_DEBUG_CHECKS
+#define SAMBA_DCHECK(err, cond) ((cond) ? true : ::samba::dcheck_fail((err), SAMBA_TU_ID, __LINE__))
+#else
+#define SAMBA_DCHECK(err, cond) true
+#endif
 
 // ---------------------------------------------------------------------------
 // Element types

@@ -5,6 +5,7 @@
 // (ring fill, position set).
 #include <string.h>
 
+#define SAMBA_TU_ID 2  // site id of this file in debug-check reports
 #include "common.cuh"
 #include "decode.h"
 

@@ -1,5 +1,6 @@
 // HBM-bound helper kernels: RMSNorm, causal depthwise conv + SiLU, RoPE tables
 // and the standalone RoPE rotation.
+#define SAMBA_TU_ID 3  // site id of this file in debug-check reports
 #include "common.cuh"
 #include "kernels.h"
 
@@ -291,6 +292,58 @@ samba_status launch_rope_apply(const void* x, void* out, int B, int L, int H, in
     rope_apply_kernel<float><<<grid, 256, 0, st>>>((const float*)x, (float*)out, rows, L, H, head_dim, pos0, tab);
   SAMBA_CHECK_LAUNCH();
   return SAMBA_OK;
+}
+
+// ===========================================================================
+// Workspace guard bands of the debug-check build: a fixed 16-byte pattern,
+// one thread per 16 bytes, one CTA row per band.
+// ===========================================================================
+__device__ __forceinline__ uint4 guard_pattern() { return make_uint4(0xA5C3E187u, 0x5A3C1E78u, 0xC0FFEE11u, 0x0DDBA115u); }
+
+__global__ void guard_fill_kernel(char* base, GuardList g) {
+  const int band = blockIdx.y;
+  uint4* p = reinterpret_cast<uint4*>(base + g.off[band]);
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < (int)(kGuardBytes / 16); i += gridDim.x * blockDim.x)
+    p[i] = guard_pattern();
+}
+
+__global__ void guard_check_kernel(const char* base, GuardList g, int* err) {
+  const int band = blockIdx.y;
+  const uint4* p = reinterpret_cast<const uint4*>(base + g.off[band]);
+  const uint4 e = guard_pattern();
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < (int)(kGuardBytes / 16); i += gridDim.x * blockDim.x) {
+    const uint4 v = p[i];
+    if (v.x != e.x || v.y != e.y || v.z != e.z || v.w != e.w)
+      raise_error(err, kErrBounds | (kGuardSiteTu << 4) | (band << 8));
+  }
+}
+
+// The guarded store's index is masked into the array as well, so that the
+// kernel stays in bounds even in a build whose checks are compiled out.
+__global__ void dcheck_selftest_kernel(int* err, int idx, int n, int* sink) {
+  __shared__ int buf[32];
+  buf[threadIdx.x & 31] = 0;
+  __syncthreads();
+  if (SAMBA_DCHECK(err, idx >= 0 && idx < n)) buf[idx & 31] = 1;
+  __syncthreads();
+  if (threadIdx.x == 0 && sink) *sink = buf[0];
+}
+
+samba_status launch_dcheck_selftest(cudaStream_t st) {
+  dcheck_selftest_kernel<<<1, 32, 0, st>>>(device_error_word(), 32, 32, nullptr);
+  return cudaGetLastError() == cudaSuccess ? SAMBA_OK : SAMBA_ERR_CUDA;
+}
+
+samba_status launch_guard_fill(char* base, const GuardList& g, cudaStream_t st) {
+  if (!kGuardBytes || g.n <= 0) return SAMBA_OK;
+  guard_fill_kernel<<<dim3(1, g.n), 256, 0, st>>>(base, g);
+  return cudaGetLastError() == cudaSuccess ? SAMBA_OK : SAMBA_ERR_CUDA;
+}
+
+samba_status launch_guard_check(const char* base, const GuardList& g, cudaStream_t st) {
+  if (!kGuardBytes || g.n <= 0) return SAMBA_OK;
+  guard_check_kernel<<<dim3(1, g.n), 256, 0, st>>>(base, g, device_error_word());
+  return cudaGetLastError() == cudaSuccess ? SAMBA_OK : SAMBA_ERR_CUDA;
 }
 
 }  // namespace samba

@@ -22,6 +22,7 @@
 #include <mutex>
 #include <vector>
 
+#define SAMBA_TU_ID 4  // site id of this file in debug-check reports
 #include "common.cuh"
 #include "kernels.h"
 

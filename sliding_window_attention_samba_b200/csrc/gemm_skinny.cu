@@ -16,6 +16,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#define SAMBA_TU_ID 5  // site id of this file in debug-check reports
 #include "common.cuh"
 #include "kernels.h"
 
@@ -39,8 +40,13 @@ constexpr int SK_THREADS = 192;
 // weight tiles, and bytes in flight matter more there than the overlap.
 constexpr int SK_RING_BYTES = 96 * 1024;
 constexpr int SK_RING_BYTES_DUAL = 200 * 1024;
-constexpr int SK_RED_PITCH = SK_MAXB + 1;
-static_assert(2 * SK_BM * SK_RED_PITCH * 4 <= SK_RING_BYTES, "reduction tiles must fit in the ring");
+// Receive buffers of the cluster reduction: recv[acc][src][batch][slot] with
+// the slot (the owner's output features) innermost, padded by 4 floats, so that
+// the reduction reads 8 consecutive features of one batch row as two 16-byte
+// loads per source and writes them as one 16-byte store.
+constexpr int SK_RED_PAD = 4;
+// largest receive area: 2 accumulators x S sources x 64 rows x (128/S + 4) floats, S <= 8
+static_assert(2 * SK_MAXB * (SK_BM + 8 * SK_RED_PAD) * 4 <= SK_RING_BYTES, "reduction tiles must fit in the ring");
 
 template <int kRing>
 struct SkSmem {
@@ -95,6 +101,12 @@ __device__ __forceinline__ void st_dsmem_v4(const float* local_ptr, uint32_t ran
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(raddr) : "r"(smem_u32(local_ptr) + tok), "r"(rank));
   asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(raddr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
                : "memory");
+}
+
+__device__ __forceinline__ void st_dsmem_f32(const float* local_ptr, uint32_t rank, float v, uint32_t tok) {
+  uint32_t raddr;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(raddr) : "r"(smem_u32(local_ptr) + tok), "r"(rank));
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(raddr), "f"(v) : "memory");
 }
 
 __device__ __forceinline__ float2 rope_cs_sk(const float2* __restrict__ tab, int half, int64_t p, int i) {
@@ -199,24 +211,25 @@ __global__ void __launch_bounds__(SK_THREADS, 2) gemm_skinny_kernel(const __grid
   }
   // Every row of the tile has one owner rank that finalises it: contiguous
   // slices of 128/S rows, or, for RoPE tiles, the two rows (i, i + hd/2) of
-  // each rotated pair together.  Receive buffers (in the now idle ring):
-  //   recv[acc][src][slot][MB]  with slot < rows per owner.
+  // each rotated pair together (slots [0, P) the first rows of the owner's P
+  // pairs, [P, 2P) the second).  Receive buffers in the now idle ring.
   const bool rope_tile = EPI == kEpiRope && n0 < a.rope_cols;
   const int rows_per = SK_BM / p.S;
+  const int pitch = rows_per + SK_RED_PAD;
   const int MB = p.MB;
+  const int per_pairs = (SK_BM / 2) / p.S;
   auto owner_of = [&](int r, int& slot) -> int {
     if (rope_tile) {
       const int hd = a.head_dim, half = hd / 2;
       const int pair = (r / hd) * half + (r % half);
-      const int per_pairs = (SK_BM / 2) / p.S;
-      slot = 2 * (pair % per_pairs) + ((r % hd) >= half ? 1 : 0);
+      slot = pair % per_pairs + ((r % hd) >= half ? per_pairs : 0);
       return pair / per_pairs;
     }
     slot = r % rows_per;
     return r / rows_per;
   };
-  auto recv = [&](int acc, int src, int slot) -> float* {
-    return red + ((size_t)(acc * p.S + src) * rows_per + slot) * MB;
+  auto recv = [&](int acc, int src, int b) -> float* {
+    return red + ((size_t)(acc * p.S + src) * MB + b) * pitch;
   };
   uint32_t tok = 0;
   if (warp >= 2) {
@@ -227,83 +240,110 @@ __global__ void __launch_bounds__(SK_THREADS, 2) gemm_skinny_kernel(const __grid
     bool got = true;
     if (nkb > 0) got = __all_sync(0xffffffffu, mbar_wait(&S.done, 0, err));
     if (got) tc_fence_after();
-    float v[2][SK_MAXB];
+    uint32_t v[2][SK_MAXB];
 #pragma unroll
-    for (int acc = 0; acc < (kDual ? 2 : 1); ++acc) {
+    for (int acc = 0; acc < (kDual ? 2 : 1); ++acc)
 #pragma unroll
-      for (int c = 0; c < SK_MAXB; c += 16) {
+      for (int c = 0; c < SK_MAXB; c += 16)
         if (c < MB) {
-          uint32_t r[16];
           if (nkb > 0 && got) {
-            tmem_ld16(tmem + acc * SK_MAXB + lane_off + c, r);
-            tmem_wait_ld();
+            tmem_ld16(tmem + acc * SK_MAXB + lane_off + c, &v[acc][c]);
           } else {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) r[i] = 0u;
+            for (int i = 0; i < 16; ++i) v[acc][c + i] = 0u;
           }
-#pragma unroll
-          for (int i = 0; i < 16; ++i) v[acc][c + i] = __uint_as_float(r[i]);
         }
-      }
-    }
+    if (nkb > 0 && got) tmem_wait_ld();
     tc_fence_before();
     // all MMAs of all CTAs are complete once everyone passes this barrier, so
     // every ring may be overwritten by the pushes below
     tok = cluster_sync_all();
     int slot;
     const int own = owner_of(row, slot);
+    // the 32 lanes of a warp hold consecutive rows, i.e. consecutive slots of
+    // one or two owners: each store below writes a contiguous run of the peer
 #pragma unroll
     for (int acc = 0; acc < (kDual ? 2 : 1); ++acc)
 #pragma unroll
-      for (int c = 0; c < SK_MAXB; c += 4)
-        if (c < MB) st_dsmem_v4(recv(acc, (int)rank, slot) + c, own,
-                                make_float4(v[acc][c], v[acc][c + 1], v[acc][c + 2], v[acc][c + 3]), tok);
+      for (int c = 0; c < SK_MAXB; ++c)
+        if (c < MB) st_dsmem_f32(recv(acc, (int)rank, c) + slot, own, __uint_as_float(v[acc][c]), tok);
   } else {
     tc_fence_before();
     tok = cluster_sync_all();
   }
   tok = cluster_sync_all();  // every push has landed; nothing remote is touched after this
 
-  // ---- reduction of the S received partials of this rank's rows + epilogue
+  // ---- reduction of the S received partials of this rank's rows + epilogue:
+  // one item = 8 consecutive output features of one batch row (RoPE: 8 pairs)
   const int M = (int)a.M;
   bf16* out = (bf16*)a.out;
-  if (rope_tile) {
-    const int hd = a.head_dim, half = hd / 2;
-    const int per_pairs = (SK_BM / 2) / p.S;
-    for (int e = threadIdx.x; e < per_pairs * M; e += SK_THREADS) {
-      const int pl = e / M, b = e % M;
-      const int pair = (int)rank * per_pairs + pl;
-      const int hh = pair / half, i = pair % half;
-      const int r1 = hh * hd + i, r2 = r1 + half;
-      float x1 = 0.f, x2 = 0.f;
-      for (int s = 0; s < p.S; ++s) {
-        x1 += recv(0, s, 2 * pl)[b];
-        x2 += recv(0, s, 2 * pl + 1)[b];
-      }
+  const int G = (rope_tile ? per_pairs : rows_per) / 8;  // feature groups per batch row
+  for (int e = threadIdx.x; e < G * M; e += SK_THREADS) {
+    const int g = e % G, b = e / G;  // consecutive threads -> consecutive groups of one row
+    if (rope_tile) {
+      const int hd = a.head_dim, half = hd / 2;
+      const int pair0 = (int)rank * per_pairs + 8 * g;
+      const int hh = pair0 / half, i0 = pair0 % half;  // 8 pairs inside one head (8 | half)
+      const int r1 = hh * hd + i0, r2 = r1 + half;
       const int64_t pos = a.pos_dev ? a.pos_dev[b] : a.pos0 + b % a.seq_len;
-      const float2 cs = rope_cs_sk(a.rope_tab, half, pos, i);
+      float x1[8], x2[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) x1[j] = x2[j] = 0.f;
+      for (int sidx = 0; sidx < p.S; ++sidx) {
+        const float* q = recv(0, sidx, b);
+        const float4 a0 = *reinterpret_cast<const float4*>(q + 8 * g);
+        const float4 a1 = *reinterpret_cast<const float4*>(q + 8 * g + 4);
+        const float4 c0 = *reinterpret_cast<const float4*>(q + per_pairs + 8 * g);
+        const float4 c1 = *reinterpret_cast<const float4*>(q + per_pairs + 8 * g + 4);
+        x1[0] += a0.x; x1[1] += a0.y; x1[2] += a0.z; x1[3] += a0.w;
+        x1[4] += a1.x; x1[5] += a1.y; x1[6] += a1.z; x1[7] += a1.w;
+        x2[0] += c0.x; x2[1] += c0.y; x2[2] += c0.z; x2[3] += c0.w;
+        x2[4] += c1.x; x2[5] += c1.y; x2[6] += c1.z; x2[7] += c1.w;
+      }
+      float o1[8], o2[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float2 cs = rope_cs_sk(a.rope_tab, half, pos, i0 + j);
+        o1[j] = x1[j] * cs.x - x2[j] * cs.y;
+        o2[j] = x2[j] * cs.x + x1[j] * cs.y;
+      }
       bf16* o = out + (int64_t)b * a.ldo + n0;
-      if (n0 + r1 < a.N) o[r1] = __float2bfloat16_rn(x1 * cs.x - x2 * cs.y);
-      if (n0 + r2 < a.N) o[r2] = __float2bfloat16_rn(x2 * cs.x + x1 * cs.y);
-    }
-  } else {
-    const int rb = (int)rank * rows_per;
-    for (int e = threadIdx.x; e < rows_per * M; e += SK_THREADS) {
-      const int sl = e % rows_per, b = e / rows_per;  // consecutive threads -> consecutive features
-      const int n = n0 + rb + sl;
-      float v = 0.f, v2 = 0.f;
-      for (int s = 0; s < p.S; ++s) {
-        v += recv(0, s, sl)[b];
-        if (kDual) v2 += recv(1, s, sl)[b];
+      if (n0 + r1 < a.N) store8(o + r1, o1);
+      if (n0 + r2 < a.N) store8(o + r2, o2);
+    } else {
+      const int n = n0 + (int)rank * rows_per + 8 * g;
+      if (n >= a.N) continue;  // N % 8 == 0: a group is wholly inside or outside
+      float extra[8];
+      if (EPI == kEpiResid) load8((const bf16*)a.resid + (int64_t)b * a.ldr + n, extra);
+      if (EPI == kEpiSoftplus) load8(a.bias + n, extra);
+      float v[8], v2[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = v2[j] = 0.f;
+      for (int sidx = 0; sidx < p.S; ++sidx) {
+        const float* q = recv(0, sidx, b) + 8 * g;
+        const float4 a0 = *reinterpret_cast<const float4*>(q);
+        const float4 a1 = *reinterpret_cast<const float4*>(q + 4);
+        v[0] += a0.x; v[1] += a0.y; v[2] += a0.z; v[3] += a0.w;
+        v[4] += a1.x; v[5] += a1.y; v[6] += a1.z; v[7] += a1.w;
+        if (kDual) {
+          const float* q2 = recv(1, sidx, b) + 8 * g;
+          const float4 c0 = *reinterpret_cast<const float4*>(q2);
+          const float4 c1 = *reinterpret_cast<const float4*>(q2 + 4);
+          v2[0] += c0.x; v2[1] += c0.y; v2[2] += c0.z; v2[3] += c0.w;
+          v2[4] += c1.x; v2[5] += c1.y; v2[6] += c1.z; v2[7] += c1.w;
+        }
       }
-      if (n >= a.N) continue;
-      if (EPI == kEpiSwiglu) v = v * (v2 * sigmoid_fast(v2));
-      if (EPI == kEpiSoftplus) v = softplus_1x(v + a.bias[n]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (EPI == kEpiSwiglu) v[j] = v[j] * (v2[j] * sigmoid_fast(v2[j]));
+        if (EPI == kEpiSoftplus) v[j] = softplus_1x(v[j] + extra[j]);
+      }
       if (EPI == kEpiResid) {
-        if (a.tap) ((bf16*)a.tap)[(int64_t)b * a.ldt + n] = __float2bfloat16_rn(v);
-        v += __bfloat162float(((const bf16*)a.resid)[(int64_t)b * a.ldr + n]);
+        if (a.tap) store8((bf16*)a.tap + (int64_t)b * a.ldt + n, v);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] += extra[j];
       }
-      out[(int64_t)b * a.ldo + n] = __float2bfloat16_rn(v);
+      store8(out + (int64_t)b * a.ldo + n, v);
     }
   }
   (void)tok;
@@ -319,6 +359,11 @@ __global__ void __launch_bounds__(SK_THREADS, 2) gemm_skinny_kernel(const __grid
 bool gemm_skinny_supported(const GemmArgs& a) {
   if (a.dtype != SAMBA_BF16 || a.M < 1 || a.M > SK_MAXB || a.K % SK_BK) return false;
   if (a.lda % 8 || a.ldo % 8 || !aligned16(a.A) || !aligned16(a.out)) return false;
+  // the epilogue moves 8 consecutive features at a time (16-byte accesses)
+  if (a.N % 8) return false;
+  if (a.epi == kEpiResid && (a.ldr % 8 || !aligned16(a.resid) || (a.tap && (a.ldt % 8 || !aligned16(a.tap)))))
+    return false;
+  if (a.epi == kEpiSoftplus && !aligned16(a.bias)) return false;
   if (a.epi == kEpiRope && (a.head_dim < 16 || SK_BM % a.head_dim || a.rope_cols % SK_BM)) return false;
   int start = 0;
   for (int s = 0; s < a.nseg; ++s) {

@@ -14,6 +14,25 @@ constexpr int kMaxGridYZ = 65535;
 constexpr int kConvRunTokens = 32;
 constexpr int64_t kMaxConvTokens = (int64_t)kMaxGridYZ * kConvRunTokens;
 
+// ---------------- debug-check build: workspace guard bands ----------------
+#if defined(SAMBA_DEBUG_CHECKS) && SAMBA_DEBUG_CHECKS
+constexpr size_t kGuardBytes = 4096;
+#else
+constexpr size_t kGuardBytes = 0;
+#endif
+constexpr int kMaxGuards = 48;
+constexpr int kGuardSiteTu = 15;  // site file id that names a guard band (the line is its index)
+struct GuardList {
+  int n = 0;
+  size_t off[kMaxGuards];
+};
+// Fill each band [base + off[i], + kGuardBytes) with a fixed pattern / verify
+// it after the call (a changed band latches kErrBounds naming its index).
+samba_status launch_guard_fill(char* base, const GuardList& g, cudaStream_t st);
+samba_status launch_guard_check(const char* base, const GuardList& g, cudaStream_t st);
+// One device check on an index made out of range on purpose (debug-check self-test).
+samba_status launch_dcheck_selftest(cudaStream_t st);
+
 // ---------------- selective scan ----------------
 struct ScanArgs {
   const void* u = nullptr;

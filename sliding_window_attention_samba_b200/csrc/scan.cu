@@ -31,6 +31,7 @@
 //     chunk) and stores y tiles (once every warp wrote its rows).
 // Every wait is bounded (error word on timeout); a timed-out CTA drains its
 // own copies in flight before it returns.
+#define SAMBA_TU_ID 6  // site id of this file in debug-check reports
 #include "common.cuh"
 #include "kernels.h"
 

@@ -6,6 +6,7 @@
 // This file holds the CUDA-core kernel (fp32 path, small head dims, and the
 // reference-precision path).  Only key blocks that intersect the band of the
 // CTA's 128 queries are visited, so work is O(L * w), never O(L^2).
+#define SAMBA_TU_ID 7  // site id of this file in debug-check reports
 #include "common.cuh"
 #include "kernels.h"
 

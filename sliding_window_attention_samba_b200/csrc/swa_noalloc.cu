@@ -24,6 +24,7 @@
 //     different host threads on the same device) race on the array.
 #include <mutex>
 
+#define SAMBA_TU_ID 8  // site id of this file in debug-check reports
 #include "common.cuh"
 #include "kernels.h"
 

@@ -21,6 +21,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#define SAMBA_TU_ID 9  // site id of this file in debug-check reports
 #include "common.cuh"
 #include "kernels.h"
 
