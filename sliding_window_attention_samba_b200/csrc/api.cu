@@ -10,12 +10,23 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #define SAMBA_TU_ID 1  // site id of this file in debug-check reports
 #include "common.cuh"
 #include "decode.h"
 #include "kernels.h"
 
 namespace samba {
+
+// NVTX range around an entry point or a sub-layer's launches (host-side
+// markers for profilers; inert unless a tool is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // ---------------------------------------------------------------------------
 // Device error word
@@ -278,7 +289,9 @@ static GemmArgs gemm1(const void* A, int64_t lda, const void* W, int64_t M, int 
 // SwiGLU MLP sub-layer: x_next = x + W3 ((W1 xn) * SiLU(W2 xn))  [Samba 3.4 "SwiGLU Formulation"]
 static samba_status mlp_sublayer(const samba_block_config& c, const float* g, const void* W1, const void* W2,
                                  const void* W3, const void* x, void* x_next, void* xn, void* hmlp, void* tap,
-                                 int64_t T, cudaStream_t st, bool pdl = false) {
+                                 int64_t T, cudaStream_t st, bool pdl = false, int64_t* pos_inc = nullptr,
+                                 bool* pos_done = nullptr) {
+  NvtxRange nvtx_("samba.mlp");
   TRY(launch_rmsnorm(x, c.d_model, g, xn, c.d_model, T, c.d_model, c.norm_eps, c.dtype, st, pdl));
   GemmArgs up = gemm1(xn, c.d_model, W1, T, c.d_ff, c.d_model, hmlp, c.d_ff, c.dtype);
   up.seg[0].W2 = W2;
@@ -292,6 +305,14 @@ static samba_status mlp_sublayer(const samba_block_config& c, const float* g, co
   dn.ldr = c.d_model;
   dn.tap = tap;
   dn.ldt = c.d_model;
+  if (pos_inc) {  // decode: the step's last projection also advances the positions
+    GemmArgs dp = dn;
+    dp.pos_inc = pos_inc;
+    if (gemm_takes_skinny(dp)) {
+      dn = dp;
+      *pos_done = true;
+    }
+  }
   return launch_gemm(dn, st);
 }
 
@@ -386,6 +407,7 @@ samba_status samba_selective_scan(const void* u, const void* dt, const float* dt
                                   const float* A_log, const void* Bm, const void* Cm, const float* Dskip,
                                   const void* z, const float* h0, float* hT, void* y, int B, int L, int D, int N,
                                   samba_dtype dtype, void*, size_t, samba_stream stream) {
+  NvtxRange nvtx_("samba_selective_scan");
   if (dtype != SAMBA_F32 && dtype != SAMBA_BF16) return SAMBA_ERR_INVALID_ARG;
   ScanArgs a;
   a.u = u;
@@ -424,6 +446,7 @@ size_t samba_swa_workspace_size(int B, int L, int Hq, int Hkv, int head_dim, flo
 samba_status samba_swa_fwd(const void* q, const void* k, const void* v, void* o, int B, int L, int Hq, int Hkv,
                            int head_dim, int window, float rope_base, int64_t pos0, float softmax_scale,
                            samba_dtype dtype, void* workspace, size_t workspace_bytes, samba_stream stream) {
+  NvtxRange nvtx_("samba_swa_fwd");
   cudaStream_t st = (cudaStream_t)stream;
   if (dtype != SAMBA_F32 && dtype != SAMBA_BF16) return SAMBA_ERR_INVALID_ARG;
   if (!q || !k || !v || !o || B < 1 || L < 0 || Hq < 1 || Hkv < 1 || window < 1 || pos0 < 0 || rope_base < 0.f)
@@ -535,6 +558,7 @@ struct LayerCtx {
 // with the state after the last token (resume: the layer continues from it).
 static samba_status mamba_sublayer(const LayerCtx& X, const samba_block_weights* w, const void* x_in, void* x_out,
                                    samba_decode_state* stt, bool resume, void* tap) {
+  NvtxRange nvtx_("samba.mamba");
   const samba_block_config& c = X.c;
   const BlockPlan& P = X.P;
   const int B = X.B, L = X.L;
@@ -619,6 +643,7 @@ static samba_status mamba_sublayer(const LayerCtx& X, const samba_block_weights*
 // min(pos0, window-1) tokens before this chunk).
 static samba_status swa_sublayer(const LayerCtx& X, const samba_block_weights* w, const void* x_in, void* x_out,
                                  samba_decode_state* stt, int64_t pos0, bool resume, void* tap) {
+  NvtxRange nvtx_("samba.swa");
   const samba_block_config& c = X.c;
   const BlockPlan& P = X.P;
   const int B = X.B, L = X.L;
@@ -702,6 +727,7 @@ static samba_status swa_sublayer(const LayerCtx& X, const samba_block_weights* w
 // projections fetch their first weight tiles) while its predecessor finishes.
 static samba_status mamba_step_layer(const LayerCtx& X, const samba_block_weights* w, const void* x_in, void* x_out,
                                      float* ssm, void* conv) {
+  NvtxRange nvtx_("samba.mamba_step");
   const samba_block_config& c = X.c;
   const BlockPlan& P = X.P;
   const int B = X.B;
@@ -743,6 +769,7 @@ static samba_status mamba_step_layer(const LayerCtx& X, const samba_block_weight
 static samba_status swa_step_layer(const LayerCtx& X, const samba_block_weights* w, const void* x_in, void* x_out,
                                    void* k_ring, void* v_ring, const int64_t* pos, void* attn_ws,
                                    size_t attn_ws_bytes) {
+  NvtxRange nvtx_("samba.swa_step");
   const samba_block_config& c = X.c;
   const BlockPlan& P = X.P;
   const int B = X.B;
@@ -766,17 +793,34 @@ static samba_status swa_step_layer(const LayerCtx& X, const samba_block_weights*
     g.seg[2].W = w->Wv;
     g.seg[2].n = kvw;
     g.pdl = true;
+    bool ring_done = false;
     if (c.rope_base != 0.f) {
-      TRY(launch_build_rope_table(tab, hd, c.rope_base, st, true));
       g.epi = kEpiRope;
       g.rope_cols = qw + kvw;
       g.head_dim = hd;
       g.pos_dev = pos;
-      g.rope_tab = tab;
+      g.rope_base = c.rope_base;  // the skinny projection evaluates the rotation from the position
+      if (!gemm_takes_skinny(g)) {
+        TRY(launch_build_rope_table(tab, hd, c.rope_base, st, true));
+        g.rope_tab = tab;
+      }
+      // the skinny projection writes the new token's k, v into the ring itself
+      GemmArgs gr = g;
+      gr.k_ring = k_ring;
+      gr.v_ring = v_ring;
+      gr.ring_window = c.window;
+      gr.ring_k_col = qw;
+      gr.ring_v_col = qw + kvw;
+      gr.ring_kvw = kvw;
+      if (gemm_takes_skinny(gr)) {
+        g = gr;
+        ring_done = true;
+      }
     }
     TRY(launch_gemm(g, st));
+    if (!ring_done)
+      TRY(launch_ring_write(qkv, P.qkvw, qw, qw + kvw, pos, k_ring, v_ring, B, c.window, kvw, dt, st));
   }
-  TRY(launch_ring_write(qkv, P.qkvw, qw, qw + kvw, pos, k_ring, v_ring, B, c.window, kvw, dt, st));
   TRY(launch_attn_decode(qkv, P.qkvw, pos, k_ring, v_ring, buf(P.o), B, c.n_q, c.n_kv, hd, c.window,
                          1.0f / sqrtf((float)hd), dt, st, attn_ws, attn_ws_bytes));
   GemmArgs g = gemm1(buf(P.o), qw, w->Wo, B, Dm, qw, x_out, Dm, dt);
@@ -794,6 +838,7 @@ static samba_status swa_step_layer(const LayerCtx& X, const samba_block_weights*
 static samba_status block_forward(const samba_block_config* cfg, const samba_block_weights* w, const void* x_in,
                                   void* x_out, samba_decode_state* stt, int64_t pos0, const samba_block_taps* taps,
                                   int B, int L, void* workspace, size_t workspace_bytes, samba_stream stream) {
+  NvtxRange nvtx_("samba_block_fwd");
   TRY(validate_cfg(cfg));
   TRY(validate_weights(w));
   if (B < 1 || L < 0 || pos0 < 0) return SAMBA_ERR_INVALID_ARG;
@@ -922,6 +967,7 @@ size_t samba_model_workspace_size(const samba_model* m, int B, int L) {
 
 samba_status samba_model_prefill(const samba_model* m, const int32_t* ids, void* logits, int B, int L,
                                  void* workspace, size_t workspace_bytes, samba_stream stream) {
+  NvtxRange nvtx_("samba_model_prefill");
   if (!m) return SAMBA_ERR_INVALID_ARG;
   TRY(validate_cfg(&m->cfg));
   if (!ids || !logits || B < 1 || L < 1 || m->n_layers < 0 || m->vocab < 1) return SAMBA_ERR_INVALID_ARG;
@@ -1000,6 +1046,7 @@ size_t samba_model_step_workspace_size(const samba_model* m, int B) {
 
 samba_status samba_model_step(const samba_model* m, const int32_t* ids_t, void* logits, samba_layer_state* states,
                               int64_t* pos, int B, void* workspace, size_t workspace_bytes, samba_stream stream) {
+  NvtxRange nvtx_("samba_model_step");
   if (!m) return SAMBA_ERR_INVALID_ARG;
   TRY(validate_cfg(&m->cfg));
   if (!ids_t || !logits || !pos || B < 1 || m->n_layers < 0 || m->vocab < 1) return SAMBA_ERR_INVALID_ARG;
@@ -1057,6 +1104,7 @@ size_t samba_step_workspace_size(const samba_block_config* cfg, int B) {
 samba_status samba_step(const samba_block_config* cfg, const samba_block_weights* w, const void* x_t, void* y_t,
                         samba_decode_state* stt, int B, void* workspace, size_t workspace_bytes,
                         samba_stream stream) {
+  NvtxRange nvtx_("samba_step");
   TRY(validate_cfg(cfg));
   TRY(validate_weights(w));
   if (!x_t || !y_t || !stt || B < 1 || x_t == y_t) return SAMBA_ERR_INVALID_ARG;
@@ -1076,10 +1124,11 @@ samba_status samba_step(const samba_block_config* cfg, const samba_block_weights
   TRY(mlp_sublayer(c, w->norm_g[1], w->mlp1_W1, w->mlp1_W2, w->mlp1_W3, x1, x2, base + P.xn, base + P.hmlp, nullptr,
                    B, st, true));
   TRY(swa_step_layer(X, w, x2, x3, stt->k_ring, stt->v_ring, stt->pos, nullptr, 0));
+  bool pos_done = false;
   TRY(mlp_sublayer(c, w->norm_g[3], w->mlp2_W1, w->mlp2_W2, w->mlp2_W3, x3, y_t, base + P.xn, base + P.hmlp, nullptr,
-                   B, st, true));
+                   B, st, true, stt->pos, &pos_done));
   TRY(guards_check(base, P.cv, st));
-  return launch_pos_update(stt->pos, B, 1, false, st, true);
+  return pos_done ? SAMBA_OK : launch_pos_update(stt->pos, B, 1, false, st, true);
 }
 
 }  // extern "C"

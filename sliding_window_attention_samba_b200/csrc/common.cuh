@@ -87,6 +87,23 @@ __device__ __forceinline__ void load8(const bf16* p, float* f) {
     f[2 * i + 1] = t.y;
   }
 }
+// 4 consecutive elements -> 4 floats (8-byte or 16-byte vector access)
+__device__ __forceinline__ void load4(const bf16* p, float* f) {
+  uint2 v = *reinterpret_cast<const uint2*>(p);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+  const float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
+  f[0] = a.x;
+  f[1] = a.y;
+  f[2] = b.x;
+  f[3] = b.y;
+}
+__device__ __forceinline__ void load4(const float* p, float* f) {
+  const float4 v = *reinterpret_cast<const float4*>(p);
+  f[0] = v.x;
+  f[1] = v.y;
+  f[2] = v.z;
+  f[3] = v.w;
+}
 __device__ __forceinline__ void load8(const float* p, float* f) {
   float4 a = *reinterpret_cast<const float4*>(p);
   float4 b = *reinterpret_cast<const float4*>(p + 4);

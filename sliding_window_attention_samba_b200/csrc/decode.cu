@@ -36,7 +36,10 @@ __global__ void conv_step_kernel(const T* __restrict__ hz, int64_t ld_hz, const 
   u[(size_t)b * D + c] = Elt<T>::from_f(acc * s);
 }
 
-// one recurrence step per (b, c), 16 fp32 states
+// One recurrence step per (b, c), 16 fp32 states: four lanes per channel, each
+// holding four states, so that the state, A_log, B and C are read and the
+// state written in contiguous runs of the warp (16-byte pieces per lane); the
+// read-out sum is completed across the four lanes with two shuffles.
 template <typename T>
 __global__ void scan_step_kernel(const T* __restrict__ u, const T* __restrict__ dlt, const T* __restrict__ z,
                                  int64_t ld_z, const T* __restrict__ xdbl, int64_t ld_x, int r_off,
@@ -44,54 +47,61 @@ __global__ void scan_step_kernel(const T* __restrict__ u, const T* __restrict__ 
                                  float* __restrict__ ssm, T* __restrict__ y, int B, int D) {
   pdl_wait();
   pdl_trigger();
-  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= B * D) return;
-  const int b = idx / D, c = idx % D;
-  const float delta = Elt<T>::to_f(dlt[(size_t)b * D + c]);
-  const float uv = Elt<T>::to_f(u[(size_t)b * D + c]);
-  const T* Bp = xdbl + (size_t)b * ld_x + r_off;
-  const T* Cp = Bp + 16;
-  // the 16 states of (b, c) are 64 contiguous bytes: four 16-byte accesses per
-  // thread, so a warp's accesses cover whole 2 KB runs
-  float4* hp = reinterpret_cast<float4*>(ssm + ((size_t)b * D + c) * 16);
-  const float4* ap = reinterpret_cast<const float4*>(A_log + (size_t)c * 16);
-  float Bv[16], Cv[16], h[16], al[16];
-  load8(Bp, Bv);
-  load8(Bp + 8, Bv + 8);
-  load8(Cp, Cv);
-  load8(Cp + 8, Cv + 8);
+  const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int q = (int)(gid & 3);  // states 4q .. 4q+3
+  const int64_t idx = gid >> 2;  // (b, c)
+  const bool live = idx < (int64_t)B * D;
+  const int b = live ? (int)(idx / D) : 0, c = live ? (int)(idx % D) : 0;
+  float yv = 0.f, uv = 0.f;
+  if (live) {
+    const float delta = Elt<T>::to_f(dlt[(size_t)b * D + c]);
+    uv = Elt<T>::to_f(u[(size_t)b * D + c]);
+    const T* Bp = xdbl + (size_t)b * ld_x + r_off + 4 * q;
+    const T* Cp = Bp + 16;
+    float4* hp = reinterpret_cast<float4*>(ssm + ((size_t)b * D + c) * 16 + 4 * q);
+    const float4 av = *reinterpret_cast<const float4*>(A_log + (size_t)c * 16 + 4 * q);
+    const float4 hv = *hp;
+    float Bv[4], Cv[4];
+    load4(Bp, Bv);
+    load4(Cp, Cv);
+    const float al[4] = {av.x, av.y, av.z, av.w};
+    float h[4] = {hv.x, hv.y, hv.z, hv.w};
+    const float du = delta * uv;
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const float4 hv = hp[q], av = ap[q];
-    h[4 * q] = hv.x; h[4 * q + 1] = hv.y; h[4 * q + 2] = hv.z; h[4 * q + 3] = hv.w;
-    al[4 * q] = av.x; al[4 * q + 1] = av.y; al[4 * q + 2] = av.z; al[4 * q + 3] = av.w;
+    for (int n = 0; n < 4; ++n) {
+      const float A = -expf(al[n]);
+      const float dA = sizeof(T) == 4 ? expf(delta * A) : ex2_approx(delta * A * 1.4426950408889634f);
+      h[n] = fmaf(dA, h[n], du * Bv[n]);
+      yv = fmaf(Cv[n], h[n], yv);
+    }
+    *hp = make_float4(h[0], h[1], h[2], h[3]);
   }
-  float yv = 0.f;
-  const float du = delta * uv;
-#pragma unroll
-  for (int n = 0; n < 16; ++n) {
-    const float A = -expf(al[n]);
-    const float dA = sizeof(T) == 4 ? expf(delta * A) : ex2_approx(delta * A * 1.4426950408889634f);
-    h[n] = fmaf(dA, h[n], du * Bv[n]);
-    yv = fmaf(Cv[n], h[n], yv);
+  // the four lanes of a channel are consecutive lanes of one warp
+  yv += __shfl_xor_sync(0xffffffffu, yv, 1);
+  yv += __shfl_xor_sync(0xffffffffu, yv, 2);
+  if (live && q == 0) {
+    yv = fmaf(Dskip ? Dskip[c] : 0.f, uv, yv);
+    const float zv = Elt<T>::to_f(z[(size_t)b * ld_z + c]);
+    const float s = sizeof(T) == 4 ? sigmoid_acc(zv) : sigmoid_fast(zv);
+    y[(size_t)b * D + c] = Elt<T>::from_f(yv * zv * s);
   }
-#pragma unroll
-  for (int q = 0; q < 4; ++q) hp[q] = make_float4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
-  yv = fmaf(Dskip ? Dskip[c] : 0.f, uv, yv);
-  const float zv = Elt<T>::to_f(z[(size_t)b * ld_z + c]);
-  const float s = sizeof(T) == 4 ? sigmoid_acc(zv) : sigmoid_fast(zv);
-  y[(size_t)b * D + c] = Elt<T>::from_f(yv * zv * s);
 }
 
-// k, v (post-RoPE) of the new token into ring slot pos mod w
+// k, v (post-RoPE) of the new token into ring slot pos mod w.  A negative
+// position (a corrupted state) latches SAMBA_ERR_DEVICE and writes nothing.
 template <typename T>
 __global__ void ring_write_kernel(const T* __restrict__ qkv, int64_t ld, int k_off, int v_off,
                                   const int64_t* __restrict__ pos, T* __restrict__ k_ring, T* __restrict__ v_ring,
-                                  int window, int kvw) {
+                                  int window, int kvw, int* err) {
   pdl_wait();
   pdl_trigger();
   const int b = blockIdx.x;
+  if (pos[b] < 0) {
+    if (threadIdx.x == 0) raise_error(err, kErrDevice);
+    return;
+  }
   const int64_t slot = pos[b] % window;
+  if (!SAMBA_DCHECK(err, slot >= 0 && slot < window && k_off + kvw <= ld && v_off + kvw <= ld)) return;
   const T* src = qkv + (size_t)b * ld;
   T* kd = k_ring + ((size_t)b * window + slot) * kvw;
   T* vd = v_ring + ((size_t)b * window + slot) * kvw;
@@ -394,7 +404,7 @@ __device__ __forceinline__ void dec_slice_partial(const bf16* __restrict__ qkv, 
 __global__ void __launch_bounds__(256, 1)
     attn_decode_split_kernel(const bf16* __restrict__ qkv, int64_t ld, const int64_t* __restrict__ pos,
                              const bf16* __restrict__ k_ring, const bf16* __restrict__ v_ring, bf16* __restrict__ o,
-                             int Hq, int Hkv, int window, float scale_log2) {
+                             int Hq, int Hkv, int window, float scale_log2, int* err) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ __align__(16) unsigned char dec_dyn[];  // K slice | V slice (bf16, padded rows)
@@ -410,7 +420,9 @@ __global__ void __launch_bounds__(256, 1)
   const int nvalid = (int)(P + 1 < window ? P + 1 : window);
   const int slice = ((nvalid + kSplit - 1) / kSplit + 31) & ~31;
   const int s0 = (int)rank * slice;
-  const int n = max(0, min(nvalid, s0 + slice) - s0);
+  int n = max(0, min(nvalid, s0 + slice) - s0);
+  // the slice's rows must fit the shared-memory slice and stay inside the ring
+  if (!SAMBA_DCHECK(err, slice <= kSliceMax && (n == 0 || s0 + n <= window))) n = 0;
   dec_slice_partial(qkv, ld, k_ring, v_ring, Hkv, grp, window, g, b, s0, n, slice, scale_log2, Ks, Vs, part, wm, wl,
                     wo);
   __syncthreads();
@@ -447,7 +459,7 @@ __global__ void __launch_bounds__(256, 1)
 __global__ void __launch_bounds__(256, 1)
     attn_decode_long_kernel(const bf16* __restrict__ qkv, int64_t ld, const int64_t* __restrict__ pos,
                             const bf16* __restrict__ k_ring, const bf16* __restrict__ v_ring,
-                            DecPart* __restrict__ ws, int Hq, int Hkv, int window, float scale_log2) {
+                            DecPart* __restrict__ ws, int Hq, int Hkv, int window, float scale_log2, int* err) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ __align__(16) unsigned char dec_dyn[];
@@ -461,7 +473,8 @@ __global__ void __launch_bounds__(256, 1)
   const int64_t P = pos[b];
   const int nvalid = (int)(P + 1 < window ? P + 1 : window);
   const int s0 = split * kSliceMax;
-  const int n = max(0, min(nvalid, s0 + kSliceMax) - s0);
+  int n = max(0, min(nvalid, s0 + kSliceMax) - s0);
+  if (!SAMBA_DCHECK(err, n == 0 || s0 + n <= window)) n = 0;
   DecPart* dst = ws + ((size_t)b * Hkv + g) * gridDim.x + split;
   if (n == 0) {  // block-uniform: past the valid slots
     if (threadIdx.x < 8) {
@@ -520,13 +533,14 @@ __global__ void pos_check_set_kernel(int64_t* pos, int B, int64_t expect, int64_
 // prefill -> ring: chunk tokens max(0, L-w) .. L-1 (absolute position pos0 + t) into slot (pos0 + t) mod w
 template <typename T>
 __global__ void ring_fill_kernel(const T* __restrict__ qkv, int64_t ld, int k_off, int v_off, T* __restrict__ k_ring,
-                                 T* __restrict__ v_ring, int L, int64_t pos0, int window, int kvw) {
+                                 T* __restrict__ v_ring, int L, int64_t pos0, int window, int kvw, int* err) {
   const int j = blockIdx.x;  // 0 .. min(L, w)-1
   const int b = blockIdx.y;
   const int n = min(L, window);
   if (j >= n) return;
   const int p = L - n + j;
   const int slot = (int)((pos0 + p) % window);
+  if (!SAMBA_DCHECK(err, p >= 0 && p < L && slot >= 0 && slot < window)) return;
   const T* src = qkv + ((size_t)b * L + p) * ld;
   T* kd = k_ring + ((size_t)b * window + slot) * kvw;
   T* vd = v_ring + ((size_t)b * window + slot) * kvw;
@@ -541,13 +555,15 @@ __global__ void ring_fill_kernel(const T* __restrict__ qkv, int64_t ld, int k_of
 __global__ void kv_window_gather_kernel(const char* __restrict__ qkv, int64_t ld_b, int64_t k_off_b,
                                         int64_t v_off_b, const char* __restrict__ k_ring,
                                         const char* __restrict__ v_ring, char* __restrict__ kx,
-                                        char* __restrict__ vx, int L, int64_t pos0, int h, int window, int vec) {
+                                        char* __restrict__ vx, int L, int64_t pos0, int h, int window, int vec,
+                                        int* err) {
   const int j = blockIdx.x;
   const int b = blockIdx.y;
   const int64_t row_b = (int64_t)vec * 16;
   const char *ks, *vs;
   if (j < h) {
     const int slot = (int)((pos0 - h + j) % window);
+    if (!SAMBA_DCHECK(err, pos0 - h + j >= 0 && slot < window)) return;
     ks = k_ring + ((int64_t)b * window + slot) * row_b;
     vs = v_ring + ((int64_t)b * window + slot) * row_b;
   } else {
@@ -596,10 +612,10 @@ samba_status launch_scan_step(const void* u, const void* dlt, const void* z, int
   const int n = B * D;
   cudaError_t e;
   SAMBA_DT_DISPATCH(dt,
-                    (e = launch_k(scan_step_kernel<bf16>, dim3((n + 127) / 128), dim3(128), 0, st, true,
+                    (e = launch_k(scan_step_kernel<bf16>, dim3((unsigned)((4 * (int64_t)n + 127) / 128)), dim3(128), 0, st, true,
                                   (const bf16*)u, (const bf16*)dlt, (const bf16*)z, ld_z, (const bf16*)xdbl, ld_x,
                                   r_off, A_log, Dskip, ssm, (bf16*)y, B, D)),
-                    (e = launch_k(scan_step_kernel<float>, dim3((n + 127) / 128), dim3(128), 0, st, true,
+                    (e = launch_k(scan_step_kernel<float>, dim3((unsigned)((4 * (int64_t)n + 127) / 128)), dim3(128), 0, st, true,
                                   (const float*)u, (const float*)dlt, (const float*)z, ld_z, (const float*)xdbl, ld_x,
                                   r_off, A_log, Dskip, ssm, (float*)y, B, D)));
   if (e != cudaSuccess) return note_cuda_failure("decode kernel launch", e);
@@ -611,9 +627,11 @@ samba_status launch_ring_write(const void* qkv, int64_t ld, int k_off, int v_off
   cudaError_t e;
   SAMBA_DT_DISPATCH(dt,
                     (e = launch_k(ring_write_kernel<bf16>, dim3(B), dim3(128), 0, st, true, (const bf16*)qkv, ld,
-                                  k_off, v_off, pos, (bf16*)k_ring, (bf16*)v_ring, window, kvw)),
+                                  k_off, v_off, pos, (bf16*)k_ring, (bf16*)v_ring, window, kvw,
+                                  device_error_word())),
                     (e = launch_k(ring_write_kernel<float>, dim3(B), dim3(128), 0, st, true, (const float*)qkv, ld,
-                                  k_off, v_off, pos, (float*)k_ring, (float*)v_ring, window, kvw)));
+                                  k_off, v_off, pos, (float*)k_ring, (float*)v_ring, window, kvw,
+                                  device_error_word())));
   if (e != cudaSuccess) return note_cuda_failure("decode kernel launch", e);
   return SAMBA_OK;
 }
@@ -636,7 +654,7 @@ samba_status launch_attn_decode(const void* qkv, int64_t ld, const int64_t* pos,
     if (!ensure_smem_attr(attn_decode_long_kernel, smem)) return SAMBA_ERR_CUDA;
     if (launch_k(attn_decode_long_kernel, dim3(nsplit, Hkv, B), dim3(256), smem, st, true, (const bf16*)qkv, ld,
                  pos, (const bf16*)k_ring, (const bf16*)v_ring, (DecPart*)ws, Hq, Hkv, window,
-                 scale * 1.4426950408889634f) != cudaSuccess)
+                 scale * 1.4426950408889634f, device_error_word()) != cudaSuccess)
       return SAMBA_ERR_CUDA;
     if (launch_k(attn_decode_merge_kernel, dim3(Hq, B), dim3(kHd), 0, st, true, (const DecPart*)ws, (bf16*)o, Hq,
                  Hkv, nsplit) != cudaSuccess)
@@ -662,7 +680,7 @@ samba_status launch_attn_decode(const void* qkv, int64_t ld, const int64_t* pos,
     cfg.numAttrs = 2;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, attn_decode_split_kernel, (const bf16*)qkv, ld, pos,
                                              (const bf16*)k_ring, (const bf16*)v_ring, (bf16*)o, Hq, Hkv, window,
-                                             scale * 1.4426950408889634f);
+                                             scale * 1.4426950408889634f, device_error_word());
     if (e != cudaSuccess) return note_cuda_failure("cudaLaunchKernelEx (decode attention cluster)", e);
     SAMBA_CHECK_LAUNCH();
     return SAMBA_OK;
@@ -704,10 +722,11 @@ samba_status launch_ring_fill(const void* qkv, int64_t ld, int k_off, int v_off,
   dim3 grid(n, B);
   SAMBA_DT_DISPATCH(dt,
                     (ring_fill_kernel<bf16><<<grid, 128, 0, st>>>((const bf16*)qkv, ld, k_off, v_off, (bf16*)k_ring,
-                                                                  (bf16*)v_ring, L, pos0, window, kvw)),
+                                                                  (bf16*)v_ring, L, pos0, window, kvw,
+                                                                  device_error_word())),
                     (ring_fill_kernel<float><<<grid, 128, 0, st>>>((const float*)qkv, ld, k_off, v_off,
                                                                    (float*)k_ring, (float*)v_ring, L, pos0, window,
-                                                                   kvw)));
+                                                                   kvw, device_error_word())));
   SAMBA_CHECK_LAUNCH();
   return SAMBA_OK;
 }
@@ -725,7 +744,7 @@ samba_status launch_kv_window_gather(const void* qkv, int64_t ld, int k_off, int
   dim3 grid(h + L, B);
   kv_window_gather_kernel<<<grid, 64, 0, st>>>((const char*)qkv, ld * es, k_off * es, v_off * es,
                                                (const char*)k_ring, (const char*)v_ring, (char*)kx, (char*)vx, L,
-                                               pos0, h, window, vec);
+                                               pos0, h, window, vec, device_error_word());
   SAMBA_CHECK_LAUNCH();
   return SAMBA_OK;
 }

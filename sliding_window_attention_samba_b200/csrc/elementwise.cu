@@ -41,12 +41,62 @@ __global__ void rmsnorm_kernel(const T* __restrict__ x, int64_t ld_x, const floa
   }
 }
 
+// Few rows (decode: one row per sequence): one CTA per row, each thread one
+// 8-element piece held in registers, the sum of squares reduced across the CTA
+// (one global load per element instead of two dependent passes of a warp).
+template <typename T>
+__global__ void rmsnorm_row_kernel(const T* __restrict__ x, int64_t ld_x, const float* __restrict__ g,
+                                   T* __restrict__ out, int64_t ld_out, int dim, float eps) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ float part[32];
+  const int64_t row = blockIdx.x;
+  const int c = threadIdx.x * 8;
+  const bool in = c < dim;
+  float f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, gg[8];
+  if (in) {
+    load8(x + row * ld_x + c, f);
+    load8(g + c, gg);
+  }
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) ss = fmaf(f[i], f[i], ss);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) part[warp] = ss;
+  __syncthreads();
+  if (warp == 0) {
+    float t = lane < (int)(blockDim.x >> 5) ? part[lane] : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    if (lane == 0) part[0] = t;
+  }
+  __syncthreads();
+  const float r = rsqrtf(part[0] / (float)dim + eps);
+  if (in) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) f[i] = f[i] * r * gg[i];
+    store8(out + row * ld_out + c, f);
+  }
+}
+
 samba_status launch_rmsnorm(const void* x, int64_t ld_x, const float* g, void* out, int64_t ld_out, int64_t rows,
                             int dim, float eps, samba_dtype dt, cudaStream_t st, bool pdl) {
   if (!x || !g || !out || rows < 0 || dim <= 0) return SAMBA_ERR_INVALID_ARG;
   if (dim % 8 || ld_x % 8 || ld_out % 8 || !aligned16(x) || !aligned16(out) || !aligned16(g))
     return SAMBA_ERR_UNSUPPORTED;
   if (rows == 0) return SAMBA_OK;
+  if (rows <= num_sms() && dim <= 8 * 1024) {
+    const int threads = ((dim / 8 + 31) / 32) * 32;
+    const cudaError_t e =
+        dt == SAMBA_BF16
+            ? launch_k(rmsnorm_row_kernel<bf16>, dim3((unsigned)rows), dim3(threads), 0, st, pdl, (const bf16*)x,
+                       ld_x, g, (bf16*)out, ld_out, dim, eps)
+            : launch_k(rmsnorm_row_kernel<float>, dim3((unsigned)rows), dim3(threads), 0, st, pdl, (const float*)x,
+                       ld_x, g, (float*)out, ld_out, dim, eps);
+    return e == cudaSuccess ? SAMBA_OK : SAMBA_ERR_CUDA;
+  }
   const int warps = 8;
   dim3 grid((unsigned)((rows + warps - 1) / warps));
   const cudaError_t e =

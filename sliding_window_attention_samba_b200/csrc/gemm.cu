@@ -416,6 +416,9 @@ __global__ void __launch_bounds__(TcEpi<EPI>::threads, 1) gemm_tc_kernel(const _
         int seg = 0;
         while (seg < p.a.nseg - 1 && nt * p.bn >= p.seg_start[seg + 1]) ++seg;
         const int brow = nt * p.bn - p.seg_start[seg];
+        // loads are clipped by the tensor maps; a bad tile is reported, not skipped (the pipeline stays in step)
+        (void)SAMBA_DCHECK(err, mt >= 0 && mt < p.m_tiles && nt >= 0 && nt < p.n_tiles && brow >= 0 &&
+                                    brow < p.a.seg[seg].n);
         for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
           const int s = it % TC_STAGES;
           const uint32_t j = it / TC_STAGES;
@@ -477,7 +480,7 @@ __global__ void __launch_bounds__(TcEpi<EPI>::threads, 1) gemm_tc_kernel(const _
       tc_fence_after();
       const uint32_t tbase = tmem + acc * TC_MAXN + ((uint32_t)(q * 32) << 16);
       const int64_t row = (int64_t)mt * TC_BM + q * 32 + lane;
-      tc_epilogue_tile<EPI>(p, tbase, row, nt, part);
+      if (SAMBA_DCHECK(err, mt < p.m_tiles && (nt + 1) * p.bn <= p.a.N)) tc_epilogue_tile<EPI>(p, tbase, row, nt, part);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.tempty[acc]);
@@ -654,8 +657,10 @@ int gemm_timing_count() {
   return g_tm_count;
 }
 
+bool gemm_takes_skinny(const GemmArgs& a) { return !force_simt() && a.M <= 64 && gemm_skinny_supported(a); }
+
 static samba_status gemm_dispatch(const GemmArgs& a, cudaStream_t st) {
-  if (!force_simt() && a.M <= 64 && gemm_skinny_supported(a)) return launch_gemm_skinny(a, st);
+  if (gemm_takes_skinny(a)) return launch_gemm_skinny(a, st);
   if (!force_simt() && gemm_tc_supported(a)) return launch_gemm_tc(a, st);
   if (a.epi == kEpiRope && 64 % a.head_dim != 0) return SAMBA_ERR_UNSUPPORTED;
   return launch_gemm_simt(a, st);
@@ -672,7 +677,9 @@ samba_status launch_gemm(const GemmArgs& a, cudaStream_t st) {
   if (nsum != a.N) return SAMBA_ERR_INVALID_ARG;
   if (a.epi == kEpiResid && !a.resid) return SAMBA_ERR_INVALID_ARG;
   if (a.epi == kEpiSoftplus && !a.bias) return SAMBA_ERR_INVALID_ARG;
-  if (a.epi == kEpiRope && (!a.rope_tab || a.head_dim <= 0 || a.rope_cols % a.head_dim)) return SAMBA_ERR_INVALID_ARG;
+  if (a.epi == kEpiRope && ((!a.rope_tab && !(a.rope_base > 0.f && gemm_takes_skinny(a))) || a.head_dim <= 0 ||
+                            a.rope_cols % a.head_dim))
+    return SAMBA_ERR_INVALID_ARG;
   if (a.M == 0) return SAMBA_OK;
   const cudaEvent_t tstop = timing_begin(a.epi, st);
   const samba_status r = gemm_dispatch(a, st);

@@ -67,6 +67,7 @@ struct SkParams {
   int S;           // cluster size = K splits
   int kb_total, kps;
   int seg_start[3];
+  double theta[64];  // RoPE without a table: base^(-2i/head_dim), i < head_dim / 2 (fp64)
 };
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -107,6 +108,19 @@ __device__ __forceinline__ void st_dsmem_f32(const float* local_ptr, uint32_t ra
   uint32_t raddr;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(raddr) : "r"(smem_u32(local_ptr) + tok), "r"(rank));
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(raddr), "f"(v) : "memory");
+}
+
+// (cos, sin) of pos * theta without a table: the angle is formed and reduced
+// modulo 2*pi in fp64 (exact product up to 2^-53 relative, Cody-Waite
+// two-term 2*pi), then evaluated in fp32 on [-pi, pi].
+__device__ __forceinline__ float2 rope_cs_direct(double theta, int64_t p) {
+  const double ang = (double)p * theta;
+  const double k = rint(ang * 0.15915494309189535);  // 1 / (2 pi)
+  double r = fma(-k, 6.283185307179586, ang);
+  r = fma(-k, 2.4492935982947064e-16, r);
+  float s, c;
+  sincosf((float)r, &s, &c);
+  return make_float2(c, s);
 }
 
 __device__ __forceinline__ float2 rope_cs_sk(const float2* __restrict__ tab, int half, int64_t p, int i) {
@@ -187,6 +201,9 @@ __global__ void __launch_bounds__(SK_THREADS, 2) gemm_skinny_kernel(const __grid
   } else {
     pdl_wait();  // the epilogue reads and writes activations
     pdl_trigger();
+    // every kernel before this one has completed: the step's position may advance
+    if (a.pos_inc && blockIdx.x == 0 && warp == 2)
+      for (int i = lane; i < (int)a.M; i += 32) a.pos_inc[i] += 1;
   }
   if (warp == 1) {
     const uint32_t idesc = idesc_bf16_f32(SK_BM, p.MB);
@@ -231,6 +248,8 @@ __global__ void __launch_bounds__(SK_THREADS, 2) gemm_skinny_kernel(const __grid
   auto recv = [&](int acc, int src, int b) -> float* {
     return red + ((size_t)(acc * p.S + src) * MB + b) * pitch;
   };
+  // the receive area (every source, batch row and slot) must fit the ring
+  const bool area_ok = SAMBA_DCHECK(err, (size_t)(kDual ? 2 : 1) * p.S * MB * pitch * 4 <= sizeof(S.ring));
   uint32_t tok = 0;
   if (warp >= 2) {
     // TMEM -> registers (zeros if this CTA had no K range)
@@ -260,10 +279,11 @@ __global__ void __launch_bounds__(SK_THREADS, 2) gemm_skinny_kernel(const __grid
     tok = cluster_sync_all();
     int slot;
     const int own = owner_of(row, slot);
+    const bool fits = area_ok && SAMBA_DCHECK(err, own >= 0 && own < p.S && slot >= 0 && slot < rows_per);
     // the 32 lanes of a warp hold consecutive rows, i.e. consecutive slots of
     // one or two owners: each store below writes a contiguous run of the peer
 #pragma unroll
-    for (int acc = 0; acc < (kDual ? 2 : 1); ++acc)
+    for (int acc = 0; acc < (kDual ? 2 : 1) && fits; ++acc)
 #pragma unroll
       for (int c = 0; c < SK_MAXB; ++c)
         if (c < MB) st_dsmem_f32(recv(acc, (int)rank, c) + slot, own, __uint_as_float(v[acc][c]), tok);
@@ -278,13 +298,14 @@ __global__ void __launch_bounds__(SK_THREADS, 2) gemm_skinny_kernel(const __grid
   const int M = (int)a.M;
   bf16* out = (bf16*)a.out;
   const int G = (rope_tile ? per_pairs : rows_per) / 8;  // feature groups per batch row
-  for (int e = threadIdx.x; e < G * M; e += SK_THREADS) {
+  for (int e = threadIdx.x; e < G * M && area_ok; e += SK_THREADS) {
     const int g = e % G, b = e / G;  // consecutive threads -> consecutive groups of one row
     if (rope_tile) {
       const int hd = a.head_dim, half = hd / 2;
       const int pair0 = (int)rank * per_pairs + 8 * g;
       const int hh = pair0 / half, i0 = pair0 % half;  // 8 pairs inside one head (8 | half)
       const int r1 = hh * hd + i0, r2 = r1 + half;
+      if (!SAMBA_DCHECK(err, i0 + 8 <= half && r2 + 8 <= SK_BM)) continue;
       const int64_t pos = a.pos_dev ? a.pos_dev[b] : a.pos0 + b % a.seq_len;
       float x1[8], x2[8];
 #pragma unroll
@@ -303,16 +324,27 @@ __global__ void __launch_bounds__(SK_THREADS, 2) gemm_skinny_kernel(const __grid
       float o1[8], o2[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const float2 cs = rope_cs_sk(a.rope_tab, half, pos, i0 + j);
+        const float2 cs = a.rope_tab ? rope_cs_sk(a.rope_tab, half, pos, i0 + j) : rope_cs_direct(p.theta[i0 + j], pos);
         o1[j] = x1[j] * cs.x - x2[j] * cs.y;
         o2[j] = x2[j] * cs.x + x1[j] * cs.y;
       }
       bf16* o = out + (int64_t)b * a.ldo + n0;
       if (n0 + r1 < a.N) store8(o + r1, o1);
       if (n0 + r2 < a.N) store8(o + r2, o2);
+      const int kc = n0 + r1 - a.ring_k_col;  // rotated key columns also go to the ring
+      if (a.k_ring && kc >= 0 && kc < a.ring_kvw) {
+        if (pos < 0) {
+          raise_error(err, kErrDevice);  // a corrupted position: nothing is written outside the ring
+        } else if (SAMBA_DCHECK(err, kc + half + 8 <= a.ring_kvw)) {
+          bf16* kr = (bf16*)a.k_ring + ((int64_t)b * a.ring_window + pos % a.ring_window) * a.ring_kvw;
+          store8(kr + kc, o1);
+          store8(kr + kc + half, o2);
+        }
+      }
     } else {
       const int n = n0 + (int)rank * rows_per + 8 * g;
       if (n >= a.N) continue;  // N % 8 == 0: a group is wholly inside or outside
+      if (!SAMBA_DCHECK(err, n + 8 <= a.N && b < M)) continue;
       float extra[8];
       if (EPI == kEpiResid) load8((const bf16*)a.resid + (int64_t)b * a.ldr + n, extra);
       if (EPI == kEpiSoftplus) load8(a.bias + n, extra);
@@ -344,6 +376,16 @@ __global__ void __launch_bounds__(SK_THREADS, 2) gemm_skinny_kernel(const __grid
         for (int j = 0; j < 8; ++j) v[j] += extra[j];
       }
       store8(out + (int64_t)b * a.ldo + n, v);
+      if (EPI == kEpiRope && a.v_ring) {  // value columns also go to the ring
+        const int vc = n - a.ring_v_col;
+        const int64_t pos = a.pos_dev[b];
+        if (vc >= 0 && vc < a.ring_kvw) {
+          if (pos < 0)
+            raise_error(err, kErrDevice);
+          else if (SAMBA_DCHECK(err, vc + 8 <= a.ring_kvw))
+            store8((bf16*)a.v_ring + ((int64_t)b * a.ring_window + pos % a.ring_window) * a.ring_kvw + vc, v);
+        }
+      }
     }
   }
   (void)tok;
@@ -365,6 +407,7 @@ bool gemm_skinny_supported(const GemmArgs& a) {
     return false;
   if (a.epi == kEpiSoftplus && !aligned16(a.bias)) return false;
   if (a.epi == kEpiRope && (a.head_dim < 16 || SK_BM % a.head_dim || a.rope_cols % SK_BM)) return false;
+  if (a.epi == kEpiRope && !a.rope_tab && !(a.rope_base > 0.f && a.head_dim / 2 <= 64)) return false;
   int start = 0;
   for (int s = 0; s < a.nseg; ++s) {
     if (!aligned16(a.seg[s].W) || (a.seg[s].W2 && !aligned16(a.seg[s].W2))) return false;
@@ -372,6 +415,12 @@ bool gemm_skinny_supported(const GemmArgs& a) {
     start += a.seg[s].n;
   }
   if (a.epi == kEpiSwiglu && a.nseg != 1) return false;
+  if (a.k_ring || a.v_ring) {  // ring columns: whole 8-column groups, rotated keys inside the RoPE columns
+    if (a.epi != kEpiRope || !a.pos_dev || a.ring_window < 1 || a.ring_kvw % 8 || a.ring_k_col % 8 ||
+        a.ring_v_col % 8 || !aligned16(a.k_ring) || !aligned16(a.v_ring) ||
+        a.ring_k_col + a.ring_kvw > a.rope_cols || a.ring_v_col < a.rope_cols)
+      return false;
+  }
   const char* e = getenv("SAMBA_GEMM_KERNEL");
   return !(e && e[0] == 's');
 }
@@ -408,6 +457,8 @@ samba_status launch_gemm_skinny(const GemmArgs& a, cudaStream_t st) {
   memset(&p, 0, sizeof(p));
   p.a = a;
   p.MB = (int)((a.M + 15) / 16) * 16;
+  if (a.epi == kEpiRope && !a.rope_tab)
+    for (int i = 0; i < a.head_dim / 2; ++i) p.theta[i] = pow((double)a.rope_base, -2.0 * i / (double)a.head_dim);
   {
     const int xb = ((p.MB * SK_BK * 2) + 1023) / 1024 * 1024;
     p.stage_bytes = (a.epi == kEpiSwiglu ? 2 : 1) * SK_BM * SK_BK * 2 + xb;

@@ -119,6 +119,18 @@ struct GemmArgs {
   int64_t pos0 = 0;
   const int64_t* pos_dev = nullptr;
   const float2* rope_tab = nullptr;
+  // skinny kernel only (see gemm_takes_skinny): rope_tab may be NULL when
+  // rope_base > 0, the rotation then evaluated from the position directly
+  float rope_base = 0.f;
+  // decode (skinny kernel only, see gemm_takes_skinny): also write the key and
+  // value columns [ring_k_col, +ring_kvw) and [ring_v_col, +ring_kvw) of row b
+  // into slot pos_dev[b] mod ring_window of k_ring / v_ring ([M, window, kvw])
+  void* k_ring = nullptr;
+  void* v_ring = nullptr;
+  int ring_window = 0, ring_k_col = 0, ring_v_col = 0, ring_kvw = 0;
+  // decode (skinny kernel only): add 1 to pos_inc[0 .. M) once the kernel's
+  // prerequisites have completed (the last projection of a step)
+  int64_t* pos_inc = nullptr;
   samba_dtype dtype = SAMBA_BF16;
   bool pdl = false;  // launch as a programmatic dependent of the previous kernel (decode path)
 };
@@ -132,6 +144,9 @@ samba_status launch_gemm_tc(const GemmArgs& a, cudaStream_t st);    // tcgen05 k
 bool gemm_tc_supported(const GemmArgs& a);
 samba_status launch_gemm_skinny(const GemmArgs& a, cudaStream_t st);  // M <= 64: swap-AB, cluster split-K
 bool gemm_skinny_supported(const GemmArgs& a);
+// launch_gemm runs these arguments on the skinny kernel (the only one that
+// honours the ring and pos_inc fields)
+bool gemm_takes_skinny(const GemmArgs& a);
 
 // ---------------- sliding-window attention ----------------
 struct SwaArgs {

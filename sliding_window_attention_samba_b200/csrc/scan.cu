@@ -293,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         Sm.E[np][nw][0][lane] = make_float4(en[0].x, en[0].y, en[1].x, en[1].y);
         Sm.E[np][nw][1][lane] = make_float4(en[2].x, en[2].y, en[3].x, en[3].y);
         mbar_arrive(&Sm.eready[nw]);
-      } else if (hT) {  // the state after the last token
+      } else if (hT && SAMBA_DCHECK(err, d < D && b < (int)gridDim.y)) {  // the state after the last token
         float* hp = hT + ((size_t)b * D + d) * kN + hf * kHalf;
 #pragma unroll
         for (int k = 0; k < kHalf / 2; ++k) {
@@ -344,7 +344,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (producer) {  // every warp wrote its rows: store the tile
         pok = wait(&Sm.ydone[c % kYBuf], (c / kYBuf) & 1);
         if (pok) {
-          tma_store_3d(&tm_y, ytile, d0, c * kChunk, b);
+          // the tensor map clips rows >= L and channels >= D; the tile's origin must lie inside
+          if (SAMBA_DCHECK(err, d0 < D && c * kChunk < L)) tma_store_3d(&tm_y, ytile, d0, c * kChunk, b);
           tma_store_commit();
           tma_store_wait_read<1>();  // the tile of chunk c - 1 has been read: reusable at chunk c + 2
         }

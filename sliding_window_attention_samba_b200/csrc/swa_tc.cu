@@ -108,6 +108,8 @@ __global__ void __launch_bounds__(AT_THREADS, 1) swa_tc_kernel(const __grid_cons
   const int lo = tk0 - p.window + 1;
   const int kb0 = lo <= 0 ? 0 : (lo / AT_BN) * AT_BN;
   const int ntile = (min(tk0 + AT_BM - 1, p.Lk - 1) - kb0) / AT_BN + 1;
+  // the visited key tiles start inside the key rows (loads past Lk are clipped by the tensor map)
+  (void)SAMBA_DCHECK(err, t0 < p.L && kb0 >= 0 && ntile >= 1 && kb0 + (ntile - 1) * AT_BN < p.Lk);
 
   if (warp == 0 && lane == 0) {
     mbar_init(&S.q_full, 1);
@@ -302,7 +304,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1) swa_tc_kernel(const __grid_cons
       tmem_ld32(tO + lane_off, orr);
       tmem_ld32(tO + lane_off + 32, orr + 32);
       tmem_wait_ld();
-      if (tq < p.L && l_run > 0.f) {
+      if (tq < p.L && l_run > 0.f && SAMBA_DCHECK(err, h < p.Hq)) {
         const float inv = 1.f / l_run;
         bf16* op = p.o + ((int64_t)b * p.L + tq) * p.ld_o + (int64_t)h * AT_D;
 #pragma unroll
@@ -361,6 +363,8 @@ __global__ void __launch_bounds__(AT_THREADS, 1) swa_tc256_kernel(const __grid_c
   const int lo = tk0 - p.window + 1;
   const int kb0 = lo <= 0 ? 0 : (lo / H_BN) * H_BN;
   const int ntile = (min(tk0 + AT_BM - 1, p.Lk - 1) - kb0) / H_BN + 1;
+  // the visited key tiles start inside the key rows (loads past Lk are clipped by the tensor map)
+  (void)SAMBA_DCHECK(err, t0 < p.L && kb0 >= 0 && ntile >= 1 && kb0 + (ntile - 1) * H_BN < p.Lk);
 
   if (warp == 0 && lane == 0) {
     mbar_init(&S.q_full, 1);
@@ -546,7 +550,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1) swa_tc256_kernel(const __grid_c
     }
     if (ok && wait_all(&S.pv_done[(ntile - 1) & 1], ((ntile - 1) >> 1) & 1)) {
       tc_fence_after();
-      const bool store = tq < p.L && l_run > 0.f;
+      const bool store = tq < p.L && l_run > 0.f && SAMBA_DCHECK(err, h < p.Hq);
       const float inv = store ? 1.f / l_run : 0.f;
       bf16* op = p.o + ((int64_t)b * p.L + tq) * p.ld_o + (int64_t)h * H_D;
 #pragma unroll
@@ -612,6 +616,8 @@ __global__ void __launch_bounds__(A2_THREADS, 1) swa_tc2_kernel(const __grid_con
   const int lo = tk0 - p.window + 1;
   const int kb0 = lo <= 0 ? 0 : (lo / AT_BN) * AT_BN;
   const int ntile = (min(tk0 + AT_BM - 1, p.Lk - 1) - kb0) / AT_BN + 1;
+  // the visited key tiles start inside the key rows (loads past Lk are clipped by the tensor map)
+  (void)SAMBA_DCHECK(err, t0 < p.L && kb0 >= 0 && ntile >= 1 && kb0 + (ntile - 1) * AT_BN < p.Lk);
 
   if (warp == 0 && lane == 0) {
     mbar_init(&S.q_full, 1);
@@ -837,7 +843,7 @@ __global__ void __launch_bounds__(A2_THREADS, 1) swa_tc2_kernel(const __grid_con
       tmem_ld32(tO, orr);
       tmem_ld32(tO + 32, orr + 32);
       tmem_wait_ld();
-      if (tq < p.L && l_run > 0.f) {
+      if (tq < p.L && l_run > 0.f && SAMBA_DCHECK(err, h0 + wg < p.Hq)) {
         const float inv = 1.f / l_run;
         bf16* op = p.o + ((int64_t)b * p.L + tq) * p.ld_o + (int64_t)(h0 + wg) * AT_D;
 #pragma unroll
@@ -906,6 +912,8 @@ __global__ void __launch_bounds__(A4_THREADS, 1) swa_tc4_kernel(const __grid_con
   const int lo = tk0 - p.window + 1;
   const int kb0 = lo <= 0 ? 0 : (lo / A4_BN) * A4_BN;
   const int ntile = (min(tk0 + AT_BM - 1, p.Lk - 1) - kb0) / A4_BN + 1;
+  // the visited key tiles start inside the key rows (loads past Lk are clipped by the tensor map)
+  (void)SAMBA_DCHECK(err, t0 < p.L && kb0 >= 0 && ntile >= 1 && kb0 + (ntile - 1) * A4_BN < p.Lk);
 
   if (warp == 0 && lane == 0) {
     mbar_init(&S.q_full, 1);
@@ -1123,7 +1131,7 @@ __global__ void __launch_bounds__(A4_THREADS, 1) swa_tc4_kernel(const __grid_con
       tmem_ld32(tO, orr);
       tmem_ld32(tO + 32, orr + 32);
       tmem_wait_ld();
-      if (tq < p.L && l_run > 0.f) {
+      if (tq < p.L && l_run > 0.f && SAMBA_DCHECK(err, h0 + hh < p.Hq)) {
         const float inv = 1.f / l_run;
         bf16* op = p.o + ((int64_t)b * p.L + tq) * p.ld_o + (int64_t)(h0 + hh) * AT_D;
 #pragma unroll

@@ -182,3 +182,27 @@ def test_scan_stall_hook_arguments(lib):
     assert h.samba_debug_scan_stall(3, 3_000_000_000) == lib.SAMBA_ERR_INVALID_ARG  # above 2 s
     assert h.samba_debug_scan_stall(3, 5_000_000) == 0
     assert h.samba_debug_scan_stall(-1, 0) == 0
+
+
+def test_debug_check_build_exports_and_flags(lib):
+    """libsamba_debug.so (built by __graft_entry__.build) exports the same
+    symbols; only it reports the checks enabled, and the release library refuses
+    the self-test before touching the device."""
+    assert lib.samba_debug_checks_enabled() == 0
+    assert lib.samba_debug_check_selftest(0, None, 0, 0) == lib.SAMBA_ERR_UNSUPPORTED
+    assert lib.samba_debug_check_selftest(7, None, 0, 0) == lib.SAMBA_ERR_INVALID_ARG
+    assert lib.samba_last_check_site() == ""
+    assert lib.samba_status_string(lib.SAMBA_ERR_BOUNDS) == "SAMBA_ERR_BOUNDS"
+    path = os.path.join(ROOT, "sliding_window_attention_samba_b200", "libsamba_debug.so")
+    if not os.path.exists(path):
+        pytest.skip("libsamba_debug.so not built")
+    dbg = ctypes.CDLL(path)
+    for n in declared_functions():
+        assert hasattr(dbg, n), n
+    dbg.samba_debug_checks_enabled.restype = ctypes.c_int
+    assert dbg.samba_debug_checks_enabled() == 1
+    # the guard bands are part of the workspace the size queries report
+    dbg.samba_debug_selftest_workspace_size.restype = ctypes.c_size_t
+    rel = ctypes.CDLL(lib.LIB_PATH)
+    rel.samba_debug_selftest_workspace_size.restype = ctypes.c_size_t
+    assert dbg.samba_debug_selftest_workspace_size() == rel.samba_debug_selftest_workspace_size() + 2 * 4096

@@ -282,3 +282,24 @@ def test_decode_ring_wraps_wide_bf16(L):
     cur = P + S
     assert np.array_equal(host(g.pos), np.full(1, cur))
     _ring_map_exact(host(g.k_ring), full["attn"]["k"], cur, w)
+
+
+@pytest.mark.parametrize("shape_name", ["TINY", "WIDE"])
+def test_step_refuses_negative_position(L, shape_name):
+    """A corrupted decode state (a negative position) is reported as
+    SAMBA_ERR_DEVICE and nothing is written into the rings: the ring write
+    (CUDA-core path) or the fused ring columns of the skinny QKV projection
+    check the position before forming a slot."""
+    import torch
+    shape = getattr(I, shape_name)
+    W = I.block_weights(shape, 9)
+    x = I.block_input(shape, 9, 2, 40)
+    g = GpuBlock(L, shape, W, 2, 40)
+    g.prefill(x[:, :39], taps=False)
+    k0, v0 = g.k_ring.clone(), g.v_ring.clone()
+    g.pos[1] = -5
+    g.step(x[:, 39])
+    torch.cuda.synchronize()
+    assert L.samba_get_error() == L.SAMBA_ERR_DEVICE
+    assert torch.equal(g.k_ring[1], k0[1]) and torch.equal(g.v_ring[1], v0[1])
+    assert L.samba_get_error() == L.SAMBA_OK  # read and cleared; the context stays usable
