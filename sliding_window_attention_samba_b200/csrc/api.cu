@@ -744,17 +744,36 @@ static samba_status mamba_step_layer(const LayerCtx& X, const samba_block_weight
     return launch_gemm(g, st);
   };
   TRY(launch_rmsnorm(x_in, Dm, w->norm_g[0], xn, Dm, B, Dm, c.norm_eps, dt, st, true));
-  TRY(gemm_pdl(gemm1(xn, Dm, w->W_in, B, 2 * Di, Dm, hz, 2 * Di, dt)));
-  TRY(launch_conv_step(hz, 2 * Di, w->conv_w, w->conv_b, conv, buf(P.u), B, Di, c.d_conv, dt, st));
-  TRY(gemm_pdl(gemm1(buf(P.u), Di, w->W_x, B, P.xdw, Di, xdbl, P.xdw, dt)));
   {
+    GemmArgs g = gemm1(xn, Dm, w->W_in, B, 2 * Di, Dm, hz, 2 * Di, dt);
+    // the skinny projection runs the short convolution step on its x columns itself
+    GemmArgs gc = g;
+    gc.conv_w = w->conv_w;
+    gc.conv_b = w->conv_b;
+    gc.conv_state = conv;
+    gc.conv_u = buf(P.u);
+    gc.conv_cols = Di;
+    gc.conv_k = c.d_conv;
+    if (gemm_takes_skinny(gc)) {
+      TRY(gemm_pdl(gc));
+    } else {
+      TRY(gemm_pdl(g));
+      TRY(launch_conv_step(hz, 2 * Di, w->conv_w, w->conv_b, conv, buf(P.u), B, Di, c.d_conv, dt, st));
+    }
+  }
+  TRY(gemm_pdl(gemm1(buf(P.u), Di, w->W_x, B, P.xdw, Di, xdbl, P.xdw, dt)));
+  if (scan_step_dt_supported(R, Di, P.xdw, dt) && aligned16(w->W_dt) && aligned16(w->A_log)) {
+    // the dt projection inside the recurrence step
+    TRY(launch_scan_step_dt(buf(P.u), hz + (size_t)Di * es, 2 * Di, xdbl, P.xdw, R, w->W_dt, w->dt_bias, w->A_log,
+                            w->Dskip, ssm, buf(P.y), B, Di, dt, st));
+  } else {
     GemmArgs g = gemm1(xdbl, P.xdw, w->W_dt, B, Di, R, buf(P.dlt), Di, dt);
     g.epi = kEpiSoftplus;
     g.bias = w->dt_bias;
     TRY(gemm_pdl(g));
+    TRY(launch_scan_step(buf(P.u), buf(P.dlt), hz + (size_t)Di * es, 2 * Di, xdbl, P.xdw, R, w->A_log, w->Dskip,
+                         ssm, buf(P.y), B, Di, dt, st));
   }
-  TRY(launch_scan_step(buf(P.u), buf(P.dlt), hz + (size_t)Di * es, 2 * Di, xdbl, P.xdw, R, w->A_log, w->Dskip, ssm,
-                       buf(P.y), B, Di, dt, st));
   GemmArgs g = gemm1(buf(P.y), Di, w->W_out, B, Dm, Di, x_out, Dm, dt);
   g.epi = kEpiResid;
   g.resid = x_in;

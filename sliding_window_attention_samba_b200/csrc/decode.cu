@@ -87,6 +87,97 @@ __global__ void scan_step_kernel(const T* __restrict__ u, const T* __restrict__ 
   }
 }
 
+// Recurrence step with the dt projection folded in [Samba 3.4 "Input-Dependent
+// Selective Gating": Delta = softplus(dt_low W_dt^T + b)]: a CTA takes 8
+// channels for 32 batch rows (one warp per row; lane = 8 * q + channel, lane q
+// holding states 4q .. 4q+3).  The CTA stages W_dt's 8 rows (before waiting
+// for the previous kernel: weights) and the 32 rows of dt_low in shared
+// memory; each lane forms a quarter of Delta's dot product and two shuffles
+// complete it, so Delta never goes through memory.  The state update and the
+// read-out are those of the kernel above.
+constexpr int kSdCh = 8;     // channels per CTA
+constexpr int kSdRows = 32;  // batch rows per CTA
+constexpr int kSdMaxR = 512;
+
+template <typename T>
+__global__ void __launch_bounds__(1024, 1)
+    scan_step_dt_kernel(const T* __restrict__ u, const T* __restrict__ z, int64_t ld_z, const T* __restrict__ xdbl,
+                        int64_t ld_x, int R, const T* __restrict__ W_dt, const float* __restrict__ dt_bias,
+                        const float* __restrict__ A_log, const float* __restrict__ Dskip, float* __restrict__ ssm,
+                        T* __restrict__ y, int B, int D) {
+  extern __shared__ __align__(16) unsigned char sd_smem[];
+  constexpr int kVec = 16 / sizeof(T);  // elements per 16-byte piece
+  const int pitch = R + kVec;            // padded rows (W rows of 8 channels land in distinct banks)
+  T* Ws = reinterpret_cast<T*>(sd_smem);
+  T* Xs = Ws + kSdCh * pitch;
+  const int c0 = blockIdx.x * kSdCh, b0 = blockIdx.y * kSdRows;
+  const int nv = R / kVec;  // 16-byte pieces per row
+  for (int e = threadIdx.x; e < kSdCh * nv; e += blockDim.x) {
+    const int r = e / nv, k = e % nv;
+    *reinterpret_cast<uint4*>(Ws + r * pitch + k * kVec) =
+        *reinterpret_cast<const uint4*>(W_dt + (size_t)(c0 + r) * R + k * kVec);
+  }
+  pdl_wait();
+  pdl_trigger();
+  for (int e = threadIdx.x; e < kSdRows * nv; e += blockDim.x) {
+    const int r = e / nv, k = e % nv;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (b0 + r < B) v = *reinterpret_cast<const uint4*>(xdbl + (size_t)(b0 + r) * ld_x + k * kVec);
+    *reinterpret_cast<uint4*>(Xs + r * pitch + k * kVec) = v;
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ci = lane & 7, q = lane >> 3;
+  const int b = b0 + warp, c = c0 + ci;
+  const bool live = b < B;
+  // Delta: lane q takes the 8-element pieces q, q + 4, q + 8, ... of the dot product
+  const int n8 = R / 8;
+  float acc = 0.f;
+  for (int k = q; k < n8; k += 4) {
+    float wv[8], xv[8];
+    load8(Ws + ci * pitch + k * 8, wv);
+    load8(Xs + warp * pitch + k * 8, xv);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc = fmaf(wv[j], xv[j], acc);
+  }
+  acc += __shfl_xor_sync(0xffffffffu, acc, 8);
+  acc += __shfl_xor_sync(0xffffffffu, acc, 16);
+  float yv = 0.f, uv = 0.f;
+  if (live) {
+    float delta = acc + (dt_bias ? dt_bias[c] : 0.f);
+    if constexpr (sizeof(T) == 4) delta = softplus_acc(delta);
+    else delta = softplus_1x(delta);
+    uv = Elt<T>::to_f(u[(size_t)b * D + c]);
+    const T* Bp = xdbl + (size_t)b * ld_x + R + 4 * q;
+    const T* Cp = Bp + 16;
+    float4* hp = reinterpret_cast<float4*>(ssm + ((size_t)b * D + c) * 16 + 4 * q);
+    const float4 av = *reinterpret_cast<const float4*>(A_log + (size_t)c * 16 + 4 * q);
+    const float4 hv = *hp;
+    float Bv[4], Cv[4];
+    load4(Bp, Bv);
+    load4(Cp, Cv);
+    const float al[4] = {av.x, av.y, av.z, av.w};
+    float h[4] = {hv.x, hv.y, hv.z, hv.w};
+    const float du = delta * uv;
+#pragma unroll
+    for (int n = 0; n < 4; ++n) {
+      const float A = -expf(al[n]);
+      const float dA = sizeof(T) == 4 ? expf(delta * A) : ex2_approx(delta * A * 1.4426950408889634f);
+      h[n] = fmaf(dA, h[n], du * Bv[n]);
+      yv = fmaf(Cv[n], h[n], yv);
+    }
+    *hp = make_float4(h[0], h[1], h[2], h[3]);
+  }
+  yv += __shfl_xor_sync(0xffffffffu, yv, 8);
+  yv += __shfl_xor_sync(0xffffffffu, yv, 16);
+  if (live && q == 0) {
+    yv = fmaf(Dskip ? Dskip[c] : 0.f, uv, yv);
+    const float zv = Elt<T>::to_f(z[(size_t)b * ld_z + c]);
+    const float s = sizeof(T) == 4 ? sigmoid_acc(zv) : sigmoid_fast(zv);
+    y[(size_t)b * D + c] = Elt<T>::from_f(yv * zv * s);
+  }
+}
+
 // k, v (post-RoPE) of the new token into ring slot pos mod w.  A negative
 // position (a corrupted state) latches SAMBA_ERR_DEVICE and writes nothing.
 template <typename T>
@@ -609,6 +700,7 @@ samba_status launch_scan_step(const void* u, const void* dlt, const void* z, int
                               int64_t ld_x, int r_off, const float* A_log, const float* Dskip, float* ssm, void* y,
                               int B, int D, samba_dtype dt, cudaStream_t st) {
   if (B > kMaxGridYZ || (int64_t)B * D > INT32_MAX) return SAMBA_ERR_UNSUPPORTED;
+  if (!aligned16(A_log) || !aligned16(ssm)) return SAMBA_ERR_UNSUPPORTED;  // 16-byte pieces of A and the state
   const int n = B * D;
   cudaError_t e;
   SAMBA_DT_DISPATCH(dt,
@@ -618,6 +710,35 @@ samba_status launch_scan_step(const void* u, const void* dlt, const void* z, int
                     (e = launch_k(scan_step_kernel<float>, dim3((unsigned)((4 * (int64_t)n + 127) / 128)), dim3(128), 0, st, true,
                                   (const float*)u, (const float*)dlt, (const float*)z, ld_z, (const float*)xdbl, ld_x,
                                   r_off, A_log, Dskip, ssm, (float*)y, B, D)));
+  if (e != cudaSuccess) return note_cuda_failure("decode kernel launch", e);
+  return SAMBA_OK;
+}
+
+bool scan_step_dt_supported(int R, int D, int64_t ld_x, samba_dtype dt) {
+  const int vec = dt == SAMBA_BF16 ? 8 : 4;
+  return R >= 8 && R <= kSdMaxR && R % 8 == 0 && D % kSdCh == 0 && ld_x % vec == 0;
+}
+
+samba_status launch_scan_step_dt(const void* u, const void* z, int64_t ld_z, const void* xdbl, int64_t ld_x, int R,
+                                 const void* W_dt, const float* dt_bias, const float* A_log, const float* Dskip,
+                                 float* ssm, void* y, int B, int D, samba_dtype dt, cudaStream_t st) {
+  if (!scan_step_dt_supported(R, D, ld_x, dt)) return SAMBA_ERR_UNSUPPORTED;
+  if (!aligned16(xdbl) || !aligned16(W_dt) || !aligned16(ssm) || !aligned16(A_log)) return SAMBA_ERR_UNSUPPORTED;
+  const int es = dt == SAMBA_BF16 ? 2 : 4;
+  const size_t smem = (size_t)(kSdCh + kSdRows) * (R + 16 / es) * es;
+  const dim3 grid(D / kSdCh, (B + kSdRows - 1) / kSdRows);
+  if (grid.y > (unsigned)kMaxGridYZ) return SAMBA_ERR_UNSUPPORTED;
+  constexpr size_t kMaxSmem = (size_t)(kSdCh + kSdRows) * (kSdMaxR + 4) * 4;
+  if (!ensure_smem_attr(scan_step_dt_kernel<bf16>, kMaxSmem) || !ensure_smem_attr(scan_step_dt_kernel<float>, kMaxSmem))
+    return SAMBA_ERR_CUDA;
+  cudaError_t e;
+  SAMBA_DT_DISPATCH(dt,
+                    (e = launch_k(scan_step_dt_kernel<bf16>, grid, dim3(1024), smem, st, true, (const bf16*)u,
+                                  (const bf16*)z, ld_z, (const bf16*)xdbl, ld_x, R, (const bf16*)W_dt, dt_bias, A_log,
+                                  Dskip, ssm, (bf16*)y, B, D)),
+                    (e = launch_k(scan_step_dt_kernel<float>, grid, dim3(1024), smem, st, true, (const float*)u,
+                                  (const float*)z, ld_z, (const float*)xdbl, ld_x, R, (const float*)W_dt, dt_bias,
+                                  A_log, Dskip, ssm, (float*)y, B, D)));
   if (e != cudaSuccess) return note_cuda_failure("decode kernel launch", e);
   return SAMBA_OK;
 }

@@ -12,6 +12,13 @@ samba_status launch_conv_step(const void* hz, int64_t ld_hz, const float* w, con
 samba_status launch_scan_step(const void* u, const void* dlt, const void* z, int64_t ld_z, const void* xdbl,
                               int64_t ld_x, int r_off, const float* A_log, const float* Dskip, float* ssm, void* y,
                               int B, int D, samba_dtype dt, cudaStream_t st);
+// The recurrence step with Delta = softplus(xdbl[:, :R] W_dt^T + dt_bias) formed
+// in the kernel (B, C at columns R, R + 16 of xdbl); supported for dt_rank R
+// <= 512, R % 8 == 0.
+bool scan_step_dt_supported(int R, int D, int64_t ld_x, samba_dtype dt);
+samba_status launch_scan_step_dt(const void* u, const void* z, int64_t ld_z, const void* xdbl, int64_t ld_x, int R,
+                                 const void* W_dt, const float* dt_bias, const float* A_log, const float* Dskip,
+                                 float* ssm, void* y, int B, int D, samba_dtype dt, cudaStream_t st);
 samba_status launch_ring_write(const void* qkv, int64_t ld, int k_off, int v_off, const int64_t* pos, void* k_ring,
                                void* v_ring, int B, int window, int kvw, samba_dtype dt, cudaStream_t st);
 // Ring caches above 2048 slots (bf16, head_dim 64) need attn_decode_workspace_bytes() of workspace for the

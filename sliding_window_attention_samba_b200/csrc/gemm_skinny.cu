@@ -375,6 +375,47 @@ __global__ void __launch_bounds__(SK_THREADS, 2) gemm_skinny_kernel(const __grid
 #pragma unroll
         for (int j = 0; j < 8; ++j) v[j] += extra[j];
       }
+      if (EPI == kEpiNone && a.conv_u && n < a.conv_cols) {
+        // short convolution step of channels n .. n+7 (the state keeps inputs as stored, in bf16)
+        if (!SAMBA_DCHECK(err, n + 8 <= a.conv_cols)) continue;
+        bf16* sp = (bf16*)a.conv_state + ((int64_t)b * a.conv_cols + n) * 3;
+        uint4 raw[3];
+#pragma unroll
+        for (int j = 0; j < 3; ++j) raw[j] = reinterpret_cast<const uint4*>(sp)[j];
+        const bf16* sv = reinterpret_cast<const bf16*>(raw);  // [channel][3], oldest first
+        bf16 xs[8];
+        float wv[32], uo[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) xs[j] = __float2bfloat16_rn(v[j]);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float4 w4 = reinterpret_cast<const float4*>(a.conv_w + (int64_t)(n + j) * 4)[0];
+          wv[4 * j] = w4.x;
+          wv[4 * j + 1] = w4.y;
+          wv[4 * j + 2] = w4.z;
+          wv[4 * j + 3] = w4.w;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          float acc = a.conv_b ? a.conv_b[n + j] : 0.f;
+          acc = fmaf(wv[4 * j], __bfloat162float(sv[3 * j]), acc);
+          acc = fmaf(wv[4 * j + 1], __bfloat162float(sv[3 * j + 1]), acc);
+          acc = fmaf(wv[4 * j + 2], __bfloat162float(sv[3 * j + 2]), acc);
+          acc = fmaf(wv[4 * j + 3], __bfloat162float(xs[j]), acc);
+          uo[j] = acc * sigmoid_fast(acc);
+        }
+        bf16 ns[24];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          ns[3 * j] = sv[3 * j + 1];
+          ns[3 * j + 1] = sv[3 * j + 2];
+          ns[3 * j + 2] = xs[j];
+        }
+#pragma unroll
+        for (int j = 0; j < 3; ++j) reinterpret_cast<uint4*>(sp)[j] = reinterpret_cast<const uint4*>(ns)[j];
+        store8((bf16*)a.conv_u + (int64_t)b * a.conv_cols + n, uo);
+        continue;
+      }
       store8(out + (int64_t)b * a.ldo + n, v);
       if (EPI == kEpiRope && a.v_ring) {  // value columns also go to the ring
         const int vc = n - a.ring_v_col;
@@ -415,6 +456,11 @@ bool gemm_skinny_supported(const GemmArgs& a) {
     start += a.seg[s].n;
   }
   if (a.epi == kEpiSwiglu && a.nseg != 1) return false;
+  if (a.conv_u) {  // the short convolution step on columns [0, conv_cols)
+    if (a.epi != kEpiNone || a.conv_k != 4 || a.conv_cols % 8 || a.conv_cols > a.N || !a.conv_w || !a.conv_state ||
+        !aligned16(a.conv_w) || !aligned16(a.conv_state) || !aligned16(a.conv_u))
+      return false;
+  }
   if (a.k_ring || a.v_ring) {  // ring columns: whole 8-column groups, rotated keys inside the RoPE columns
     if (a.epi != kEpiRope || !a.pos_dev || a.ring_window < 1 || a.ring_kvw % 8 || a.ring_k_col % 8 ||
         a.ring_v_col % 8 || !aligned16(a.k_ring) || !aligned16(a.v_ring) ||

@@ -128,6 +128,16 @@ struct GemmArgs {
   void* k_ring = nullptr;
   void* v_ring = nullptr;
   int ring_window = 0, ring_k_col = 0, ring_v_col = 0, ring_kvw = 0;
+  // decode (skinny kernel only, kEpiNone): columns [0, conv_cols) are the
+  // short convolution's new input x; instead of writing them to out, the kernel
+  // forms u = SiLU(conv_b + sum_j conv_w[c, j] win_j) over win = [conv_state
+  // (d_conv - 1 oldest first), x] into conv_u ([M, conv_cols]) and shifts x
+  // into conv_state ([M, conv_cols, d_conv - 1]); d_conv == 4
+  const float* conv_w = nullptr;
+  const float* conv_b = nullptr;
+  void* conv_state = nullptr;
+  void* conv_u = nullptr;
+  int conv_cols = 0, conv_k = 0;
   // decode (skinny kernel only): add 1 to pos_inc[0 .. M) once the kernel's
   // prerequisites have completed (the last projection of a step)
   int64_t* pos_inc = nullptr;
