@@ -543,6 +543,188 @@ __global__ void __launch_bounds__(256, 1)
   (void)dec_cluster_sync();  // peers' shared memory stays valid until every merge is done
 }
 
+// Streaming decode attention for bf16, head_dim 64, up to 8 query heads per kv
+// head, when there are enough (kv head, batch row) pairs to give every SM one:
+// one CTA per pair walks all min(pos + 1, w) valid ring slots in 64-slot tiles
+// that a producer warp streams through a TMA ring (no split, no merge across
+// CTAs).  Four consumer warps each take 16 slots of every tile and keep their
+// own online-softmax state (running max, sum, O) for the group's heads as rows
+// of m16n8k16 products (rows 8..15 padding): S = Q K^T, P = exp2(S - m), O +=
+// P V; the four partial states are merged in shared memory at the end.  K and
+// V tiles land 128-byte swizzled (16-byte piece j of row r at piece j ^ (r % 8)).
+constexpr int kStTile = 64;
+constexpr int kStStages = 6;
+constexpr int kStWarps = 4;
+constexpr int kStThreads = (kStWarps + 1) * 32;
+
+struct StSmem {
+  bf16 K[kStStages][kStTile * kHd];
+  bf16 V[kStStages][kStTile * kHd];
+  uint64_t full[kStStages], empty[kStStages];
+  float wm[kStWarps][8], wl[kStWarps][8];
+  float wo[kStWarps][8][kHd];
+};
+
+__device__ __forceinline__ uint32_t st_swz(int row, int col) {  // byte offset of element (row, col) of a tile
+  return (uint32_t)(row * 128 + ((((col >> 3) ^ row) & 7) << 4) + ((col & 7) << 1));
+}
+
+__global__ void __launch_bounds__(kStThreads, 1)
+    attn_decode_stream_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                              const bf16* __restrict__ qkv, int64_t ld, const int64_t* __restrict__ pos,
+                              bf16* __restrict__ o, int Hq, int Hkv, int window, float scale_log2, int* err) {
+  extern __shared__ __align__(1024) unsigned char st_raw[];
+  StSmem& S = *reinterpret_cast<StSmem*>(st_raw + smem_align_pad(st_raw, 1024));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = blockIdx.x, b = blockIdx.y;
+  const int grp = Hq / Hkv;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStStages; ++i) {
+      mbar_init(&S.full[i], 1);
+      mbar_init(&S.empty[i], kStWarps);
+    }
+    fence_mbar_init();
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  __syncthreads();
+  pdl_wait();  // the position, the query and this step's ring entry come from earlier kernels
+  pdl_trigger();
+  const int64_t P = pos[b];
+  const int nvalid = (int)(P + 1 < window ? P + 1 : window);
+  const int ntile = nvalid > 0 ? (nvalid + kStTile - 1) / kStTile : 0;
+  const int qr = lane >> 2, qc = 2 * (lane & 3);
+  float m_run = -INFINITY, l_run = 0.f;
+  float oacc[kHd / 8][4];
+#pragma unroll
+  for (int nt = 0; nt < kHd / 8; ++nt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) oacc[nt][i] = 0.f;
+
+  if (warp == kStWarps) {
+    // ---- producer: K and V tiles of slots [64t, 64t + 64) of ring row b
+    if (lane == 0) {
+      const int z0 = b * window;
+      int issued = 0;
+      for (int t = 0; t < ntile; ++t) {
+        const int s = t % kStStages;
+        if (t >= kStStages && !mbar_wait(&S.empty[s], ((t / kStStages) & 1) ^ 1, err)) break;
+        mbar_arrive_expect_tx(&S.full[s], 2u * kStTile * kHd * 2u);
+        tma_load_3d(S.K[s], &tmK, &S.full[s], 0, g, z0 + t * kStTile);
+        tma_load_3d(S.V[s], &tmV, &S.full[s], 0, g, z0 + t * kStTile);
+        issued = t + 1;
+      }
+      // the CTA leaves only once its own copies have landed (after a timeout too)
+      for (int t = issued > kStStages ? issued - kStStages : 0; t < issued; ++t)
+        (void)mbar_wait(&S.full[t % kStStages], (t / kStStages) & 1, err);
+    }
+  } else {
+    // ---- consumers: Q fragments (A operand, rows = heads), then the tiles
+    uint32_t qa[kHd / 16][4];
+#pragma unroll
+    for (int ks = 0; ks < kHd / 16; ++ks) {
+      qa[ks][1] = qa[ks][3] = 0u;
+      qa[ks][0] = qa[ks][2] = 0u;
+      if (qr < grp) {
+        const bf16* qrow = qkv + (size_t)b * ld + (size_t)(g * grp + qr) * kHd + ks * 16 + qc;
+        qa[ks][0] = *reinterpret_cast<const uint32_t*>(qrow);
+        qa[ks][2] = *reinterpret_cast<const uint32_t*>(qrow + 8);
+      }
+    }
+    const int kb = warp * 16;  // this warp's slots within a tile
+    for (int t = 0; t < ntile; ++t) {
+      const int s = t % kStStages;
+      if (!__all_sync(0xffffffffu, mbar_wait(&S.full[s], (t / kStStages) & 1, err))) break;
+      const unsigned char* Kt = reinterpret_cast<const unsigned char*>(S.K[s]);
+      const unsigned char* Vt = reinterpret_cast<const unsigned char*>(S.V[s]);
+      float sacc[2][4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) sacc[nt][i] = 0.f;
+        const int key = kb + nt * 8 + qr;
+#pragma unroll
+        for (int ks = 0; ks < kHd / 16; ++ks) {
+          const uint32_t b0 = *reinterpret_cast<const uint32_t*>(Kt + st_swz(key, ks * 16 + qc));
+          const uint32_t b1 = *reinterpret_cast<const uint32_t*>(Kt + st_swz(key, ks * 16 + 8 + qc));
+          mma_bf16_16816(sacc[nt], qa[ks], b0, b1);
+        }
+      }
+      // scale into the log2 domain, mask slots past the valid ones, online softmax per head (row qr)
+      float mx = -INFINITY;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int slot = t * kStTile + kb + nt * 8 + qc + c;
+          const float v = slot < nvalid ? sacc[nt][c] * scale_log2 : -INFINITY;
+          sacc[nt][c] = v;
+          mx = fmaxf(mx, v);
+        }
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      const float mnew = fmaxf(m_run, mx);
+      const float msub = mnew == -INFINITY ? 0.f : mnew;
+      const float corr = ex2_approx(m_run - msub);
+      m_run = mnew;
+      uint32_t pa[4];
+      float ps = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const float p0 = ex2_approx(sacc[nt][0] - msub), p1 = ex2_approx(sacc[nt][1] - msub);
+        ps += p0 + p1;
+        pa[nt ? 2 : 0] = pack_bf16x2(p0, p1);
+        pa[nt ? 3 : 1] = 0u;
+      }
+      l_run = l_run * corr + ps;
+#pragma unroll
+      for (int nt = 0; nt < kHd / 8; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) oacc[nt][i] *= corr;
+      // O += P V over the warp's 16 slots (V rows through ldmatrix.trans)
+#pragma unroll
+      for (int np = 0; np < kHd / 16; ++np) {
+        uint32_t vb[4];
+        const int key = kb + (lane & 7) + 8 * ((lane >> 3) & 1);
+        const int dim = np * 16 + 8 * (lane >> 4);
+        ldmatrix_x4_trans(vb, Vt + st_swz(key, dim));
+        mma_bf16_16816(oacc[2 * np], pa, vb[0], vb[1]);
+        mma_bf16_16816(oacc[2 * np + 1], pa, vb[2], vb[3]);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.empty[s]);
+    }
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+    if ((lane & 3) == 0) {
+      S.wm[warp][qr] = m_run;
+      S.wl[warp][qr] = l_run;
+    }
+#pragma unroll
+    for (int nt = 0; nt < kHd / 8; ++nt) {
+      S.wo[warp][qr][nt * 8 + qc] = oacc[nt][0];
+      S.wo[warp][qr][nt * 8 + qc + 1] = oacc[nt][1];
+    }
+  }
+  __syncthreads();
+  // ---- merge the four warps' states per head
+  for (int e = threadIdx.x; e < grp * kHd; e += kStThreads) {
+    const int h = e / kHd, d = e % kHd;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kStWarps; ++w) M = fmaxf(M, S.wm[w][h]);
+    float L = 0.f, O = 0.f;
+#pragma unroll
+    for (int w = 0; w < kStWarps; ++w) {
+      const float mw = S.wm[w][h];
+      const float wgt = mw == -INFINITY ? 0.f : ex2_approx(mw - M);
+      L += wgt * S.wl[w][h];
+      O += wgt * S.wo[w][h][d];
+    }
+    o[(size_t)b * Hq * kHd + (size_t)(g * grp + h) * kHd + d] = __float2bfloat16_rn(O / L);
+  }
+}
+
 // Long caches (more than kSplit * kSliceMax slots, e.g. a full-attention KV
 // cache): one CTA per 256-slot slice, grid (cache / 256, Hkv, B); CTAs past the
 // valid slots publish an empty partial.  Partials go to `ws`, and
@@ -780,6 +962,24 @@ samba_status launch_attn_decode(const void* qkv, int64_t ld, const int64_t* pos,
     if (launch_k(attn_decode_merge_kernel, dim3(Hq, B), dim3(kHd), 0, st, true, (const DecPart*)ws, (bf16*)o, Hq,
                  Hkv, nsplit) != cudaSuccess)
       return SAMBA_ERR_CUDA;
+    return SAMBA_OK;
+  }
+  if (dt == SAMBA_BF16 && hd == kHd && Hq / Hkv <= 8 && window <= 4096 && ld % 8 == 0 &&
+      (int64_t)B * Hkv >= (int64_t)num_sms() * 3 / 4 && aligned16(k_ring) && aligned16(v_ring)) {
+    // enough (kv head, row) pairs for every SM: one streaming CTA per pair
+    CUtensorMap tmK, tmV;
+    const uint64_t dims[3] = {(uint64_t)kHd, (uint64_t)Hkv, (uint64_t)B * (uint64_t)window};
+    const uint64_t strides[2] = {(uint64_t)kHd, (uint64_t)Hkv * kHd};
+    const uint32_t box[3] = {(uint32_t)kHd, 1u, (uint32_t)kStTile};
+    if (!make_tmap(&tmK, k_ring, SAMBA_BF16, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap(&tmV, v_ring, SAMBA_BF16, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return SAMBA_ERR_CUDA;
+    const size_t smem = sizeof(StSmem) + 1024;
+    if (!ensure_smem_attr(attn_decode_stream_kernel, smem)) return SAMBA_ERR_CUDA;
+    const cudaError_t e = launch_k(attn_decode_stream_kernel, dim3(Hkv, B), dim3(kStThreads), smem, st, true, tmK,
+                                   tmV, (const bf16*)qkv, ld, pos, (bf16*)o, Hq, Hkv, window,
+                                   scale * 1.4426950408889634f, device_error_word());
+    if (e != cudaSuccess) return note_cuda_failure("decode attention launch", e);
     return SAMBA_OK;
   }
   if (dt == SAMBA_BF16 && hd == kHd && Hq / Hkv <= 8 && window <= kSplit * kSliceMax && ld % 8 == 0) {

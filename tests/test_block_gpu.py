@@ -303,3 +303,20 @@ def test_step_refuses_negative_position(L, shape_name):
     assert L.samba_get_error() == L.SAMBA_ERR_DEVICE
     assert torch.equal(g.k_ring[1], k0[1]) and torch.equal(g.v_ring[1], v0[1])
     assert L.samba_get_error() == L.SAMBA_OK  # read and cleared; the context stays usable
+
+
+def test_decode_streaming_attention_B28(L):
+    """Enough (kv head, batch row) pairs for the streaming decode attention (one
+    CTA per pair walking every valid slot in 64-slot TMA tiles): 28 rows x 4 kv
+    heads at the 2048-wide shapes, 150 prefilled tokens (a partial last tile),
+    three steps against the oracle's longer prefill, every row."""
+    shape = I.WIDE
+    W = I.block_weights(shape, 12)
+    P, S = 150, 3
+    x = I.block_input(shape, 12, 28, P + S)
+    g = GpuBlock(L, shape, W, 28, P + S)
+    g.prefill(x[:, :P], taps=False)
+    full = O.block_fwd(x, W, shape)
+    for i in range(S):
+        y = host(g.step(x[:, P + i]))
+        assert step_err(y, x[:, P + i], full, P + i, "bf16") <= TOL["bf16"], i
