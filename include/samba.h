@@ -295,7 +295,14 @@ typedef struct {
 
 size_t samba_block_workspace_size(const samba_block_config* cfg, int B, int L);
 
-/* One block over a fresh sequence (positions 0..L-1):
+/* One block over a fresh sequence (positions 0..L-1) [Samba §3.2 "Big-Picture
+ * Architecture": every layer pre-RMSNorm with a residual add; §3.4 "Detailed,
+ * Sentence-Based Technical Breakdown": the Mamba layer per "The Mamba Layer",
+ * "Input-Dependent Selective Gating (The Delta Parameter)", "The State Space
+ * Model Update (S6)" and "Gated Output"; the SWA layer per "Window
+ * Specification" (keys t-w+1..t), "Positional Encoding" (RoPE, base 10,000)
+ * and the Llama-3-style GQA heads of the configuration; the MLPs per "The
+ * SwiGLU MLP Layer" ("SwiGLU Formulation")]:
  *   x1 = x  + Mamba(RMSNorm(x)); x2 = x1 + MLP1(RMSNorm(x1));
  *   x3 = x2 + SWA(RMSNorm(x2));  x_out = x3 + MLP2(RMSNorm(x3)).
  * x_in, x_out: [B, L, d_model] dtype (must not alias; may be NULL when L == 0).  If st != NULL it is
@@ -401,8 +408,13 @@ samba_status samba_model_step(const samba_model* m, const int32_t* ids_t, void* 
                               int64_t* pos, int B, void* workspace, size_t workspace_bytes, samba_stream stream);
 
 /* ------------------------------------------------------------------------
- * The Samba block, one decode step per sequence (constant cost per token;
- * [Samba 5 / Figure 2b discussion of decoding; the blog page's ring-buffer KV])
+ * The Samba block, one decode step per sequence (constant cost per token):
+ * the layers of samba_block_fwd for one new token [Samba §3.4 "The State Space
+ * Model Update (S6)": the recurrence advanced by one step from the carried
+ * state; "Window Specification": the new query attends to positions
+ * t-w+1..t; the decoding-throughput discussion of Figure 2b; the blog page
+ * "Samba Guide: Hybrid Mamba & Sliding Window Architecture", "Sliding Window
+ * KV Eviction Configuration": a w-slot ring, slot = position mod w]
  *
  * x_t, y_t: [B, d_model] dtype.  For each row b with p = pos[b]: the Mamba layer
  * advances the conv state and the SSM state by one step; the SWA layer writes

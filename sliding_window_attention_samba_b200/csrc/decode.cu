@@ -88,14 +88,16 @@ __global__ void scan_step_kernel(const T* __restrict__ u, const T* __restrict__ 
 }
 
 // Recurrence step with the dt projection folded in [Samba 3.4 "Input-Dependent
-// Selective Gating": Delta = softplus(dt_low W_dt^T + b)]: a CTA takes 8
-// channels for 32 batch rows (one warp per row; lane = 8 * q + channel, lane q
-// holding states 4q .. 4q+3).  The CTA stages W_dt's 8 rows (before waiting
-// for the previous kernel: weights) and the 32 rows of dt_low in shared
-// memory; each lane forms a quarter of Delta's dot product and two shuffles
-// complete it, so Delta never goes through memory.  The state update and the
-// read-out are those of the kernel above.
-constexpr int kSdCh = 8;     // channels per CTA
+// Selective Gating": Delta = softplus(dt_low W_dt^T + b)]: a CTA takes 16
+// channels for 32 batch rows (one warp per row; lane = 8 * q + i, lane q holding
+// states 4q .. 4q+3 of channels i and i + 8), so that one wave covers batch 32
+// at d_inner 4096.  Everything that does not come from the kernels before it
+// (the state, A_log, the biases, the 16 rows of W_dt into shared memory) is
+// fetched before waiting for them; then the 32 rows of dt_low are staged, each
+// lane forms a quarter of each Delta dot product and two shuffles complete it,
+// so Delta never goes through memory.  The state update and the read-out are
+// those of the kernel above.
+constexpr int kSdCh = 16;    // channels per CTA
 constexpr int kSdRows = 32;  // batch rows per CTA
 constexpr int kSdMaxR = 512;
 
@@ -112,53 +114,71 @@ __global__ void __launch_bounds__(1024, 1)
   T* Xs = Ws + kSdCh * pitch;
   const int c0 = blockIdx.x * kSdCh, b0 = blockIdx.y * kSdRows;
   const int nv = R / kVec;  // 16-byte pieces per row
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ci = lane & 7, q = lane >> 3;
+  const int b = b0 + warp;
+  const bool live = b < B;
+  // ---- before the wait: weights and the state (written only by this kernel's previous step)
   for (int e = threadIdx.x; e < kSdCh * nv; e += blockDim.x) {
     const int r = e / nv, k = e % nv;
     *reinterpret_cast<uint4*>(Ws + r * pitch + k * kVec) =
         *reinterpret_cast<const uint4*>(W_dt + (size_t)(c0 + r) * R + k * kVec);
   }
+  float4 hv[2], av[2];
+  float bias[2], dsk[2];
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    const int c = c0 + ci + 8 * hh;
+    av[hh] = *reinterpret_cast<const float4*>(A_log + (size_t)c * 16 + 4 * q);
+    hv[hh] = live ? *reinterpret_cast<const float4*>(ssm + ((size_t)b * D + c) * 16 + 4 * q)
+                  : make_float4(0.f, 0.f, 0.f, 0.f);
+    bias[hh] = dt_bias ? dt_bias[c] : 0.f;
+    dsk[hh] = Dskip ? Dskip[c] : 0.f;
+  }
   pdl_wait();
   pdl_trigger();
+  // ---- after it: dt_low rows (shared), B, C, u, z of this row
   for (int e = threadIdx.x; e < kSdRows * nv; e += blockDim.x) {
     const int r = e / nv, k = e % nv;
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (b0 + r < B) v = *reinterpret_cast<const uint4*>(xdbl + (size_t)(b0 + r) * ld_x + k * kVec);
     *reinterpret_cast<uint4*>(Xs + r * pitch + k * kVec) = v;
   }
-  __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int ci = lane & 7, q = lane >> 3;
-  const int b = b0 + warp, c = c0 + ci;
-  const bool live = b < B;
-  // Delta: lane q takes the 8-element pieces q, q + 4, q + 8, ... of the dot product
-  const int n8 = R / 8;
-  float acc = 0.f;
-  for (int k = q; k < n8; k += 4) {
-    float wv[8], xv[8];
-    load8(Ws + ci * pitch + k * 8, wv);
-    load8(Xs + warp * pitch + k * 8, xv);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc = fmaf(wv[j], xv[j], acc);
-  }
-  acc += __shfl_xor_sync(0xffffffffu, acc, 8);
-  acc += __shfl_xor_sync(0xffffffffu, acc, 16);
-  float yv = 0.f, uv = 0.f;
+  float Bv[4] = {0.f, 0.f, 0.f, 0.f}, Cv[4] = {0.f, 0.f, 0.f, 0.f}, uv[2] = {0.f, 0.f}, zv[2] = {0.f, 0.f};
   if (live) {
-    float delta = acc + (dt_bias ? dt_bias[c] : 0.f);
+    const T* Bp = xdbl + (size_t)b * ld_x + R + 4 * q;
+    load4(Bp, Bv);
+    load4(Bp + 16, Cv);
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int c = c0 + ci + 8 * hh;
+      uv[hh] = Elt<T>::to_f(u[(size_t)b * D + c]);
+      zv[hh] = Elt<T>::to_f(z[(size_t)b * ld_z + c]);
+    }
+  }
+  __syncthreads();
+  const int n8 = R / 8;
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    const int c = c0 + ci + 8 * hh;
+    // Delta: lane q takes the 8-element pieces q, q + 4, q + 8, ... of the dot product
+    float acc = 0.f;
+    for (int k = q; k < n8; k += 4) {
+      float wv[8], xv[8];
+      load8(Ws + (ci + 8 * hh) * pitch + k * 8, wv);
+      load8(Xs + warp * pitch + k * 8, xv);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc = fmaf(wv[j], xv[j], acc);
+    }
+    acc += __shfl_xor_sync(0xffffffffu, acc, 8);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 16);
+    float delta = acc + bias[hh];
     if constexpr (sizeof(T) == 4) delta = softplus_acc(delta);
     else delta = softplus_1x(delta);
-    uv = Elt<T>::to_f(u[(size_t)b * D + c]);
-    const T* Bp = xdbl + (size_t)b * ld_x + R + 4 * q;
-    const T* Cp = Bp + 16;
-    float4* hp = reinterpret_cast<float4*>(ssm + ((size_t)b * D + c) * 16 + 4 * q);
-    const float4 av = *reinterpret_cast<const float4*>(A_log + (size_t)c * 16 + 4 * q);
-    const float4 hv = *hp;
-    float Bv[4], Cv[4];
-    load4(Bp, Bv);
-    load4(Cp, Cv);
-    const float al[4] = {av.x, av.y, av.z, av.w};
-    float h[4] = {hv.x, hv.y, hv.z, hv.w};
-    const float du = delta * uv;
+    const float al[4] = {av[hh].x, av[hh].y, av[hh].z, av[hh].w};
+    float h[4] = {hv[hh].x, hv[hh].y, hv[hh].z, hv[hh].w};
+    const float du = delta * uv[hh];
+    float yv = 0.f;
 #pragma unroll
     for (int n = 0; n < 4; ++n) {
       const float A = -expf(al[n]);
@@ -166,15 +186,14 @@ __global__ void __launch_bounds__(1024, 1)
       h[n] = fmaf(dA, h[n], du * Bv[n]);
       yv = fmaf(Cv[n], h[n], yv);
     }
-    *hp = make_float4(h[0], h[1], h[2], h[3]);
-  }
-  yv += __shfl_xor_sync(0xffffffffu, yv, 8);
-  yv += __shfl_xor_sync(0xffffffffu, yv, 16);
-  if (live && q == 0) {
-    yv = fmaf(Dskip ? Dskip[c] : 0.f, uv, yv);
-    const float zv = Elt<T>::to_f(z[(size_t)b * ld_z + c]);
-    const float s = sizeof(T) == 4 ? sigmoid_acc(zv) : sigmoid_fast(zv);
-    y[(size_t)b * D + c] = Elt<T>::from_f(yv * zv * s);
+    if (live) *reinterpret_cast<float4*>(ssm + ((size_t)b * D + c) * 16 + 4 * q) = make_float4(h[0], h[1], h[2], h[3]);
+    yv += __shfl_xor_sync(0xffffffffu, yv, 8);
+    yv += __shfl_xor_sync(0xffffffffu, yv, 16);
+    if (live && q == 0) {
+      yv = fmaf(dsk[hh], uv[hh], yv);
+      const float s = sizeof(T) == 4 ? sigmoid_acc(zv[hh]) : sigmoid_fast(zv[hh]);
+      y[(size_t)b * D + c] = Elt<T>::from_f(yv * zv[hh] * s);
+    }
   }
 }
 
