@@ -13,6 +13,24 @@ namespace samba {
 
 namespace {
 
+__device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void ldmatrix_x4(uint32_t* r, const void* row_addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(row_addr)));
+}
+__device__ __forceinline__ void ldmatrix_x2(uint32_t* r, const void* row_addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1])
+               : "r"(smem_u32(row_addr)));
+}
+
 // conv state shift + one output:  window = [state (k-1, oldest first), x_new]
 template <typename T>
 __global__ void conv_step_kernel(const T* __restrict__ hz, int64_t ld_hz, const float* __restrict__ w,
@@ -157,21 +175,49 @@ __global__ void __launch_bounds__(1024, 1)
     }
   }
   __syncthreads();
+  // bf16 with R % 16 == 0: the CTA's [32 rows x 16 channels] of dt_low W_dt^T as
+  // four m16n8k16 tensor-core tiles (one warp each) through shared memory
+  __shared__ float Dpre[kSdRows][kSdCh + 1];
+  const bool tc_dot = sizeof(T) == 2 && R % 16 == 0;
+  if (tc_dot) {
+    if constexpr (sizeof(T) == 2) {
+      if (warp < 4) {
+        const int mt = warp >> 1, ntl = warp & 1;
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int ks = 0; ks < R / 16; ++ks) {
+          uint32_t af[4], bfr[2];
+          ldmatrix_x4(af, Xs + (mt * 16 + (lane & 15)) * pitch + ks * 16 + (lane >> 4) * 8);
+          ldmatrix_x2(bfr, Ws + (ntl * 8 + (lane & 7)) * pitch + ks * 16 + ((lane >> 3) & 1) * 8);
+          mma_bf16_16816(d, af, bfr[0], bfr[1]);
+        }
+        const int r0 = mt * 16 + (lane >> 2), cc = ntl * 8 + 2 * (lane & 3);
+        Dpre[r0][cc] = d[0];
+        Dpre[r0][cc + 1] = d[1];
+        Dpre[r0 + 8][cc] = d[2];
+        Dpre[r0 + 8][cc + 1] = d[3];
+      }
+    }
+    __syncthreads();
+  }
   const int n8 = R / 8;
 #pragma unroll
   for (int hh = 0; hh < 2; ++hh) {
     const int c = c0 + ci + 8 * hh;
-    // Delta: lane q takes the 8-element pieces q, q + 4, q + 8, ... of the dot product
     float acc = 0.f;
-    for (int k = q; k < n8; k += 4) {
-      float wv[8], xv[8];
-      load8(Ws + (ci + 8 * hh) * pitch + k * 8, wv);
-      load8(Xs + warp * pitch + k * 8, xv);
+    if (tc_dot) {
+      acc = Dpre[warp][ci + 8 * hh];
+    } else {
+      // Delta: lane q takes the 8-element pieces q, q + 4, q + 8, ... of the dot product
+      for (int k = q; k < n8; k += 4) {
+        float wv[8], xv[8];
+        load8(Ws + (ci + 8 * hh) * pitch + k * 8, wv);
+        load8(Xs + warp * pitch + k * 8, xv);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) acc = fmaf(wv[j], xv[j], acc);
+        for (int j = 0; j < 8; ++j) acc = fmaf(wv[j], xv[j], acc);
+      }
+      acc += __shfl_xor_sync(0xffffffffu, acc, 8);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 16);
     }
-    acc += __shfl_xor_sync(0xffffffffu, acc, 8);
-    acc += __shfl_xor_sync(0xffffffffu, acc, 16);
     float delta = acc + bias[hh];
     if constexpr (sizeof(T) == 4) delta = softplus_acc(delta);
     else delta = softplus_1x(delta);
@@ -343,13 +389,6 @@ __device__ __forceinline__ float dec_ld_remote(const float* p, uint32_t rank, ui
   return v;
 }
 
-__device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
 __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t* r, const void* row_addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])

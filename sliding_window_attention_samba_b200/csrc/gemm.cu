@@ -45,6 +45,26 @@ __device__ __forceinline__ float2 rope_cs(const float2* __restrict__ tab, int ha
   return make_float2(cr * c2.x - sr * c2.y, cr * c2.y + sr * c2.x);
 }
 
+// (cos, sin) of pairs i0 .. i0+15 at position p: the three table rows read as
+// 16-byte pieces (i0 a multiple of 16)
+__device__ __forceinline__ void rope_cs16(const float2* __restrict__ tab, int half, int64_t p, int i0, float2 (&cs)[16]) {
+  const float4* t0 = reinterpret_cast<const float4*>(tab + (0 * kRopeRadix + (p & 1023)) * half + i0);
+  const float4* t1 = reinterpret_cast<const float4*>(tab + (1 * kRopeRadix + ((p >> 10) & 1023)) * half + i0);
+  const float4* t2 = reinterpret_cast<const float4*>(tab + (2 * kRopeRadix + ((p >> 20) & 1023)) * half + i0);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float4 a = t0[k], b = t1[k], c = t2[k];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const float ax = e ? a.z : a.x, ay = e ? a.w : a.y;
+      const float bx = e ? b.z : b.x, by = e ? b.w : b.y;
+      const float cx = e ? c.z : c.x, cy = e ? c.w : c.y;
+      const float cr = ax * bx - ay * by, sr = ax * by + ay * bx;
+      cs[2 * k + e] = make_float2(cr * cx - sr * cy, cr * cy + sr * cx);
+    }
+  }
+}
+
 template <typename T>
 __device__ __forceinline__ float silu_t(float g) {
   if constexpr (sizeof(T) == 4) return g * sigmoid_acc(g);
@@ -262,6 +282,35 @@ __device__ __forceinline__ void tc_epilogue_tile(const TcParams& p, uint32_t tba
     const int64_t pos = in_range ? rope_position(a, row) : 0;
     const int nunits = p.bn / 64;  // (head, 32-pair chunk) units
     part_range(nunits, part, TcEpi<EPI>::parts, u_lo, u_hi);
+    if (hd == 64) {
+      // every unit is a whole head with pairs 0..31: the (cos, sin) of each
+      // 16-pair run is formed once and applied to all of this part's heads
+      for (int j0 = 0; j0 < 32; j0 += 16) {
+        float2 cs[16];
+        rope_cs16(a.rope_tab, 32, pos, j0, cs);
+        for (int u = u_lo; u < u_hi; ++u) {
+          const int hc = u * 64;
+          tmem_ld16(tbase + hc + j0, r);
+          tmem_ld16(tbase + hc + 32 + j0, r2);
+          tmem_wait_ld();
+          if (in_range) {
+            float lo[16], hi[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float x1 = __uint_as_float(r[i]), x2 = __uint_as_float(r2[i]);
+              lo[i] = x1 * cs[i].x - x2 * cs[i].y;
+              hi[i] = x2 * cs[i].x + x1 * cs[i].y;
+            }
+            bf16* o = out + row * a.ldo + col0 + hc + j0;
+            store8(o, lo);
+            store8(o + 8, lo + 8);
+            store8(o + 32, hi);
+            store8(o + 40, hi + 8);
+          }
+        }
+      }
+      return;
+    }
     for (int u = u_lo; u < u_hi; ++u) {
       const int hh = (u * 64) / hd;         // head within the tile
       const int j0 = (u * 32) % hd2;        // first pair index of this unit
