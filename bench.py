@@ -69,6 +69,8 @@ def parse():
                          "model_decode: decode tokens/s of the same two stacks at batch 16 over 64K generated "
                          "tokens (samba_model_step, CUDA graph replay)")
     ap.add_argument("--max-len", type=int, default=1048576, help="sweep: largest L")
+    ap.add_argument("--prefill", type=int, default=None,
+                    help="decode: override the 4096-token prefill (profiling runs only)")
     return ap.parse_args()
 
 
@@ -575,7 +577,7 @@ def decode_bytes_per_step(s, Bn):
 DECODE_STEPS = 65536
 
 
-def measure_decode(steps, warmup):
+def measure_decode(steps, warmup, prefill=None):
     """Streaming decode at batch 32 (one block at the 2048-wide shapes, 2048-slot
     ring): prefill 4096 tokens, then `steps` replays of one captured samba_step.
     Returns the measurement as a dict (device time, end to end, roofline)."""
@@ -584,6 +586,8 @@ def measure_decode(steps, warmup):
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
     shape, Bn, P, _, seed = I.WORKLOADS["decode_bf16_B32"]
+    if prefill:
+        P = prefill  # profiling runs only: a shorter prefill keeps the device footprint small
     s = shape
     cfg = L.make_config(s)
     (w, wst), = make_stack(torch, L, s, 1, seed, dev)
@@ -654,14 +658,16 @@ def measure_decode(steps, warmup):
                          "kernel": "whole decode step (weights + ring + states per step)",
                          "peak_source": src, "bytes_per_step": bps},
             "clocks": clk, "graph": "one samba_step captured, replayed per step",
-            # per step: 4 RMSNorms, 10 skinny projections, conv step, recurrence
-            # step, RoPE table, ring write, attention, position increment
-            "gpu_launches": 20 * steps}
+            # per step: 4 RMSNorms, 9 skinny projections (in_proj with the conv
+            # step, x_proj, out_proj, QKV with RoPE and the ring write, o_proj,
+            # 2 x SwiGLU up, 2 x down, the last advancing the positions), the
+            # recurrence step with the dt projection, the streaming attention
+            "gpu_launches": 15 * steps}
 
 
 def run_decode(args):
     """Streaming decode: prefill P tokens at batch 32, then time samba_step replays."""
-    d = measure_decode(args.steps, args.warmup)
+    d = measure_decode(args.steps, args.warmup, args.prefill)
     line = {"metric": "decode tokens/s (batch 32, one Samba block, 2048-slot ring)", "value": d["tokens_per_s"],
             "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": d["ms_per_step"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
