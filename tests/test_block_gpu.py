@@ -320,3 +320,35 @@ def test_decode_streaming_attention_B28(L):
     for i in range(S):
         y = host(g.step(x[:, P + i]))
         assert step_err(y, x[:, P + i], full, P + i, "bf16") <= TOL["bf16"], i
+
+
+def test_decode_wide_bf16_conv_bias(L):
+    """The short-conv step folded into the skinny in_proj epilogue, with a conv
+    bias (bf16, 2048-wide shapes): prefill + three steps against the oracle's
+    longer prefill."""
+    shape = I.WIDE
+    W = I.block_weights(shape, 13, conv_bias=True)
+    P, S = 70, 3
+    x = I.block_input(shape, 13, 2, P + S)
+    g = GpuBlock(L, shape, W, 2, P + S)
+    g.prefill(x[:, :P], taps=False)
+    full = O.block_fwd(x, W, shape)
+    for i in range(S):
+        y = host(g.step(x[:, P + i]))
+        assert step_err(y, x[:, P + i], full, P + i, "bf16") <= TOL["bf16"], i
+
+
+def test_decode_streaming_attention_window_4096(L):
+    """The streaming decode attention over a 4096-slot ring (its largest
+    window): 28 rows x 4 kv heads, 100 prefilled tokens, two steps."""
+    import dataclasses
+    shape = dataclasses.replace(I.WIDE, window=4096)
+    W = I.block_weights(shape, 14)
+    P, S = 100, 2
+    x = I.block_input(shape, 14, 28, P + S)
+    g = GpuBlock(L, shape, W, 28, P + S)
+    g.prefill(x[:, :P], taps=False)
+    full = O.block_fwd(x, W, shape)
+    for i in range(S):
+        y = host(g.step(x[:, P + i]))
+        assert step_err(y, x[:, P + i], full, P + i, "bf16") <= TOL["bf16"], i
