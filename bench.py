@@ -223,6 +223,12 @@ def swa_flops(s, Bn, Ln):
     return 4.0 * s.head_dim * s.n_q * pairs * Bn
 
 
+def dt_folded(s):
+    """The block forms Delta inside the scan kernel (bf16, dt_rank <= 128, a
+    multiple of 16): no separate dt projection launch."""
+    return s.dtype == "bf16" and s.dt_rank % 16 == 0 and 16 <= s.dt_rank <= 128
+
+
 def attribution_pass(torch, L, s, blocks, x, T, Bn, Ln, reps=2):
     """Times each kernel of one block separately through the component entry
     points (same kernels, same shapes, same stream) with CUDA events."""
@@ -262,7 +268,7 @@ def attribution_pass(torch, L, s, blocks, x, T, Bn, Ln, reps=2):
          "mlp1_up": (w["mlp1_W1"], w["mlp1_W2"], xn, big), "mlp1_down": (w["mlp1_W3"], None, big, xo),
          "qkv": (w["Wq"], None, xn, None), "o_proj": (w["Wo"], None, o, xo)}
     for (name, M, N, K, e, fl) in gemm_list(s, T):
-        if name in ("mlp2_up", "mlp2_down"):
+        if name in ("mlp2_up", "mlp2_down") or (name == "dt_proj" and dt_folded(s)):
             continue
         Wm, W2, a_in, out = W[name]
         a_t = torch.empty(M, K, device=dev, dtype=bf).normal_() if a_in is None or a_in.shape[1] != K else a_in
@@ -272,7 +278,10 @@ def attribution_pass(torch, L, s, blocks, x, T, Bn, Ln, reps=2):
             a_t, Wt, W2, w["dt_bias"] if e == 3 else None, x if e == 1 else None, o_t, M, N, K, e, 1))
     timed("conv", lambda: L.samba_causal_conv1d(hz, 2 * s.d_inner, w["conv_w"], None, u, None, Bn, Ln, s.d_inner,
                                                  s.d_conv, 1))
-    timed("scan", lambda: _scan_contig(torch, L, s, w, u, dlt, hz, y, Bn, Ln))
+    if dt_folded(s):  # the block's scan forms Delta itself from the x_proj output
+        timed("scan", lambda: _scan_xdbl(torch, L, s, w, u, xdbl, y, Bn, Ln))
+    else:
+        timed("scan", lambda: _scan_contig(torch, L, s, w, u, dlt, hz, y, Bn, Ln))
     timed("swa", lambda: L.samba_swa_fwd(q, kk, vv, o, Bn, Ln, s.n_q, s.n_kv, s.head_dim, s.window, 0.0, 0, 0.0, 1))
     return {k: sum(v) / len(v) for k, v in times.items()}
 
@@ -292,6 +301,16 @@ def _scan_contig(torch, L, s, w, u, dlt, hz, y, Bn, Ln):
     z, Bm, Cm = _SCAN_BUFS[key]
     L.samba_selective_scan(u, dlt, None, 0, w["A_log"], Bm, Cm, w["D"], z, None, None, y, Bn, Ln, s.d_inner,
                            s.d_state, 1)
+
+
+def _scan_xdbl(torch, L, s, w, u, xdbl, y, Bn, Ln):
+    """The scan with the dt projection folded in, on the x_proj output."""
+    key = ("z", Bn, Ln)
+    if key not in _SCAN_BUFS:
+        _SCAN_BUFS[key] = torch.empty(Bn * Ln, s.d_inner, device=u.device, dtype=torch.bfloat16).normal_()
+    z = _SCAN_BUFS[key]
+    L.samba_selective_scan_xdbl(u, xdbl, s.dt_rank, w["W_dt"], w["dt_bias"], w["A_log"], w["D"], z, None, None, y,
+                                Bn, Ln, s.d_inner, s.d_state, 1)
 
 
 def workload_of(args):
@@ -1147,7 +1166,8 @@ def main():
             extra["decode"] = measure_decode(DECODE_STEPS, args.warmup)
             torch.cuda.empty_cache()
             extra["sweep"] = measure_sweep(args.warmup, args.max_len)
-        launches_per_block = 4 + 10 + 1 + 1 + 1 + 1  # norms, projections, conv, scan, rope table, swa
+        # norms, projections (the dt projection inside the scan when folded), conv, scan, rope table, swa
+        launches_per_block = 4 + (9 if dt_folded(shape) else 10) + 1 + 1 + 1 + 1
         metric = {"prefill": METRIC, "block": "prefill tokens/s per Samba block (B=4, L=4096)",
                   "block38": "prefill tokens/s per Samba block at the 3.8B widths (L=128K)"}[args.workload]
         line = {"metric": metric,

@@ -159,6 +159,26 @@ samba_status samba_selective_scan(const void* u, const void* dt, const float* dt
                                   samba_stream stream);
 
 /* ------------------------------------------------------------------------
+ * The selective scan with the dt projection folded in, on the x_proj output
+ * of a Mamba layer [Samba §3.4 "Input-Dependent Selective Gating (The Delta
+ * Parameter)": Delta = softplus(dt_low W_dt^T + dt_bias), the low-rank
+ * bottleneck dt_low being the first dt_rank columns of x W_x^T; then "The
+ * State Space Model Update (S6)" and "Gated Output" as samba_selective_scan].
+ *
+ * x_dbl: [B, L, dt_rank + 2*N] dtype, row-major: dt_low | B_t | C_t per token.
+ * W_dt: [D, dt_rank] dtype.  dt_bias: [D] fp32 (may be NULL).  u, z, y:
+ * [B, L, D] dtype (z may be NULL).  A_log, Dskip, h0, hT as samba_selective_scan.
+ * Delta is formed inside the scan kernel in fp32 and never written to memory.
+ * Supported: bf16, N == 16, D % 16 == 0, dt_rank a multiple of 16 and at most
+ * 128, 16-byte aligned arrays; otherwise SAMBA_ERR_UNSUPPORTED (use
+ * samba_linear with the softplus epilogue and samba_selective_scan).
+ * ---------------------------------------------------------------------- */
+samba_status samba_selective_scan_xdbl(const void* u, const void* x_dbl, int dt_rank, const void* W_dt,
+                                       const float* dt_bias, const float* A_log, const float* Dskip, const void* z,
+                                       const float* h0, float* hT, void* y, int B, int L, int D, int N,
+                                       samba_dtype dtype, samba_stream stream);
+
+/* ------------------------------------------------------------------------
  * Causal sliding-window attention with grouped-query heads and RoPE
  *   [Samba 3.4 "Window Specification", "Positional Encoding", "Implementation"]
  *
@@ -423,6 +443,8 @@ samba_status samba_model_step(const samba_model* m, const int32_t* ids_t, void* 
  * read positions from device memory, so the call can be captured in a CUDA graph
  * and replayed.
  * ---------------------------------------------------------------------- */
+/* Workspace of samba_step: one block's activations for B tokens and, for rings
+ * above 2048 slots, the per-slice partials of the decode attention. */
 size_t samba_step_workspace_size(const samba_block_config* cfg, int B);
 
 samba_status samba_step(const samba_block_config* cfg, const samba_block_weights* w, const void* x_t, void* y_t,

@@ -105,6 +105,9 @@ _scan_ws = _sig("samba_selective_scan_workspace_size", c_size_t, [c_int, c_int, 
 _scan = _sig("samba_selective_scan", c_int,
              [c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
               c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_void_p, c_size_t, c_void_p])
+_scan_xdbl = _sig("samba_selective_scan_xdbl", c_int,
+                  [c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                   c_void_p, c_int, c_int, c_int, c_int, c_int, c_void_p])
 _swa_ws = _sig("samba_swa_workspace_size", c_size_t, [c_int, c_int, c_int, c_int, c_int, c_float, c_int])
 _swa = _sig("samba_swa_fwd", c_int,
             [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_float, c_int64,
@@ -243,6 +246,13 @@ def samba_selective_scan(u, dt, dt_bias, dt_softplus, A_log, Bm, Cm, Dskip, z, h
 
 def samba_swa_workspace_size(B, L, Hq, Hkv, head_dim, rope_base, dtype) -> int:
     return _swa_ws(B, L, Hq, Hkv, head_dim, rope_base, dtype)
+
+
+def samba_selective_scan_xdbl(u, x_dbl, dt_rank, W_dt, dt_bias, A_log, Dskip, z, h0, hT, y, B, L, D, N, dtype,
+                              stream=None):
+    _check("samba_selective_scan_xdbl",
+           _scan_xdbl(_p(u), _p(x_dbl), dt_rank, _p(W_dt), _p(dt_bias), _p(A_log), _p(Dskip), _p(z), _p(h0),
+                      _p(hT), _p(y), B, L, D, N, dtype, _stream(stream)))
 
 
 def samba_swa_fwd(q, k, v, o, B, L, Hq, Hkv, head_dim, window, rope_base, pos0, softmax_scale, dtype,

@@ -432,6 +432,40 @@ samba_status samba_selective_scan(const void* u, const void* dt, const float* dt
   return launch_selective_scan(a, (cudaStream_t)stream);
 }
 
+samba_status samba_selective_scan_xdbl(const void* u, const void* x_dbl, int dt_rank, const void* W_dt,
+                                       const float* dt_bias, const float* A_log, const float* Dskip, const void* z,
+                                       const float* h0, float* hT, void* y, int B, int L, int D, int N,
+                                       samba_dtype dtype, samba_stream stream) {
+  NvtxRange nvtx_("samba_selective_scan_xdbl");
+  if (dtype != SAMBA_F32 && dtype != SAMBA_BF16) return SAMBA_ERR_INVALID_ARG;
+  if (!x_dbl || !W_dt || dt_rank < 1 || N < 1) return SAMBA_ERR_INVALID_ARG;
+  ScanArgs a;
+  a.u = u;
+  a.dt_low = x_dbl;
+  a.ld_dtl = (int64_t)dt_rank + 2 * (int64_t)N;
+  a.R = dt_rank;
+  a.W_dt = W_dt;
+  a.z = z;
+  a.Bm = (const char*)x_dbl + (size_t)dt_rank * dtype_size(dtype);
+  a.Cm = (const char*)x_dbl + (size_t)(dt_rank + N) * dtype_size(dtype);
+  a.y = y;
+  a.ld_u = a.ld_z = a.ld_y = D;
+  a.ld_bc = a.ld_dtl;
+  a.dt_bias = dt_bias;
+  a.A_log = A_log;
+  a.Dskip = Dskip;
+  a.h0 = h0;
+  a.hT = hT;
+  a.B = B;
+  a.L = L;
+  a.D = D;
+  a.N = N;
+  a.softplus = true;
+  a.dtype = dtype;
+  if (!scan_dt_fold_supported(a)) return SAMBA_ERR_UNSUPPORTED;
+  return launch_selective_scan(a, (cudaStream_t)stream);
+}
+
 // ------------------------------------------------------------------ SWA
 size_t samba_swa_workspace_size(int B, int L, int Hq, int Hkv, int head_dim, float rope_base, samba_dtype dtype) {
   if (rope_base == 0.f || B <= 0 || L <= 0) return 0;
@@ -595,16 +629,26 @@ static samba_status mamba_sublayer(const LayerCtx& X, const samba_block_weights*
     TRY(launch_causal_conv(ca, st));
   }
   TRY(launch_gemm(gemm1(buf(P.u), Di, w->W_x, T, P.xdw, Di, xdbl, P.xdw, dt), st));  // dt_low | B | C
-  {
+  ScanArgs a;
+  // the dt projection folded into the scan where it can be (bf16, dt_rank <= 128)
+  a.dt_low = xdbl;
+  a.ld_dtl = P.xdw;
+  a.R = R;
+  a.W_dt = w->W_dt;
+  a.dtype = dt;
+  const bool fold = scan_dt_fold_supported(a) && !getenv("SAMBA_SCAN_UNFOLDED");
+  if (!fold) {
+    a.dt_low = nullptr;
+    a.W_dt = nullptr;
     GemmArgs g = gemm1(xdbl, P.xdw, w->W_dt, T, Di, R, buf(P.dlt), Di, dt);  // Delta = softplus(.. + b)
     g.epi = kEpiSoftplus;
     g.bias = w->dt_bias;
     TRY(launch_gemm(g, st));
   }
   {
-    ScanArgs a;
     a.u = buf(P.u);
-    a.dt = buf(P.dlt);
+    a.dt = fold ? nullptr : buf(P.dlt);
+    a.dt_bias = fold ? w->dt_bias : nullptr;
     a.z = hz + (size_t)Di * es;
     a.Bm = xdbl + (size_t)R * es;
     a.Cm = xdbl + (size_t)(R + N) * es;
@@ -620,7 +664,7 @@ static samba_status mamba_sublayer(const LayerCtx& X, const samba_block_weights*
     a.L = L;
     a.D = Di;
     a.N = N;
-    a.softplus = false;
+    a.softplus = fold;
     a.dtype = dt;
     TRY(launch_selective_scan(a, st));
   }
@@ -1115,9 +1159,16 @@ samba_status samba_model_step(const samba_model* m, const int32_t* ids_t, void* 
 }
 
 // ------------------------------------------------------------------ decode step
+// The step's workspace: one block's activations for B tokens, then (rings
+// above 2048 slots) the split decode attention's partials.
+static size_t step_attn_offset(const samba_block_config& c, int B) {
+  return plan_block(c, B).cv.off;  // 256-byte aligned end of the block's carve
+}
+
 size_t samba_step_workspace_size(const samba_block_config* cfg, int B) {
   if (validate_cfg(cfg) != SAMBA_OK || B < 1) return 0;
-  return plan_block(*cfg, B).total;
+  // + 256: slack for aligning the caller's base pointer
+  return step_attn_offset(*cfg, B) + attn_decode_workspace_bytes(B, cfg->n_kv, cfg->window) + 256;
 }
 
 samba_status samba_step(const samba_block_config* cfg, const samba_block_weights* w, const void* x_t, void* y_t,
@@ -1132,7 +1183,7 @@ samba_status samba_step(const samba_block_config* cfg, const samba_block_weights
   if (!aligned16(stt->ssm)) return SAMBA_ERR_UNSUPPORTED;  // the state is moved in 16-byte pieces
   const samba_block_config& c = *cfg;
   const BlockPlan P = plan_block(c, B);
-  if (!workspace || workspace_bytes < P.total) return SAMBA_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < samba_step_workspace_size(cfg, B)) return SAMBA_ERR_INVALID_ARG;
   if (!aligned16(x_t) || !aligned16(y_t)) return SAMBA_ERR_UNSUPPORTED;
   cudaStream_t st = (cudaStream_t)stream;
   char* base = (char*)(((uintptr_t)workspace + 255) & ~uintptr_t(255));
@@ -1142,7 +1193,9 @@ samba_status samba_step(const samba_block_config* cfg, const samba_block_weights
   TRY(mamba_step_layer(X, w, x_t, x1, stt->ssm, stt->conv));
   TRY(mlp_sublayer(c, w->norm_g[1], w->mlp1_W1, w->mlp1_W2, w->mlp1_W3, x1, x2, base + P.xn, base + P.hmlp, nullptr,
                    B, st, true));
-  TRY(swa_step_layer(X, w, x2, x3, stt->k_ring, stt->v_ring, stt->pos, nullptr, 0));
+  const size_t attn_bytes = attn_decode_workspace_bytes(B, c.n_kv, c.window);
+  TRY(swa_step_layer(X, w, x2, x3, stt->k_ring, stt->v_ring, stt->pos,
+                     attn_bytes ? base + step_attn_offset(c, B) : nullptr, attn_bytes));
   bool pos_done = false;
   TRY(mlp_sublayer(c, w->norm_g[3], w->mlp2_W1, w->mlp2_W2, w->mlp2_W3, x3, y_t, base + P.xn, base + P.hmlp, nullptr,
                    B, st, true, stt->pos, &pos_done));

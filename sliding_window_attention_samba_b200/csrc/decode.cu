@@ -1007,21 +1007,6 @@ samba_status launch_attn_decode(const void* qkv, int64_t ld, const int64_t* pos,
                                 samba_dtype dt, cudaStream_t st, void* ws, size_t ws_bytes) {
   if (B > kMaxGridYZ) return SAMBA_ERR_UNSUPPORTED;
   if (hd > 32 * kDecMaxDpl) return SAMBA_ERR_UNSUPPORTED;
-  if (dt == SAMBA_BF16 && hd == kHd && Hq / Hkv <= 8 && window > kSplit * kSliceMax && ld % 8 == 0) {
-    const int nsplit = (window + kSliceMax - 1) / kSliceMax;
-    if (!ws || ws_bytes < attn_decode_workspace_bytes(B, Hkv, window) || !aligned16(ws))
-      return SAMBA_ERR_INVALID_ARG;
-    const size_t smem = 2 * kSliceMax * kKvPad * sizeof(bf16);
-    if (!ensure_smem_attr(attn_decode_long_kernel, smem)) return SAMBA_ERR_CUDA;
-    if (launch_k(attn_decode_long_kernel, dim3(nsplit, Hkv, B), dim3(256), smem, st, true, (const bf16*)qkv, ld,
-                 pos, (const bf16*)k_ring, (const bf16*)v_ring, (DecPart*)ws, Hq, Hkv, window,
-                 scale * 1.4426950408889634f, device_error_word()) != cudaSuccess)
-      return SAMBA_ERR_CUDA;
-    if (launch_k(attn_decode_merge_kernel, dim3(Hq, B), dim3(kHd), 0, st, true, (const DecPart*)ws, (bf16*)o, Hq,
-                 Hkv, nsplit) != cudaSuccess)
-      return SAMBA_ERR_CUDA;
-    return SAMBA_OK;
-  }
   if (dt == SAMBA_BF16 && hd == kHd && Hq / Hkv <= 8 && window <= 4096 && ld % 8 == 0 &&
       (int64_t)B * Hkv >= (int64_t)num_sms() * 3 / 4 && aligned16(k_ring) && aligned16(v_ring)) {
     // enough (kv head, row) pairs for every SM: one streaming CTA per pair
@@ -1038,6 +1023,21 @@ samba_status launch_attn_decode(const void* qkv, int64_t ld, const int64_t* pos,
                                    tmV, (const bf16*)qkv, ld, pos, (bf16*)o, Hq, Hkv, window,
                                    scale * 1.4426950408889634f, device_error_word());
     if (e != cudaSuccess) return note_cuda_failure("decode attention launch", e);
+    return SAMBA_OK;
+  }
+  if (dt == SAMBA_BF16 && hd == kHd && Hq / Hkv <= 8 && window > kSplit * kSliceMax && ld % 8 == 0) {
+    const int nsplit = (window + kSliceMax - 1) / kSliceMax;
+    if (!ws || ws_bytes < attn_decode_workspace_bytes(B, Hkv, window) || !aligned16(ws))
+      return SAMBA_ERR_INVALID_ARG;
+    const size_t smem = 2 * kSliceMax * kKvPad * sizeof(bf16);
+    if (!ensure_smem_attr(attn_decode_long_kernel, smem)) return SAMBA_ERR_CUDA;
+    if (launch_k(attn_decode_long_kernel, dim3(nsplit, Hkv, B), dim3(256), smem, st, true, (const bf16*)qkv, ld,
+                 pos, (const bf16*)k_ring, (const bf16*)v_ring, (DecPart*)ws, Hq, Hkv, window,
+                 scale * 1.4426950408889634f, device_error_word()) != cudaSuccess)
+      return SAMBA_ERR_CUDA;
+    if (launch_k(attn_decode_merge_kernel, dim3(Hq, B), dim3(kHd), 0, st, true, (const DecPart*)ws, (bf16*)o, Hq,
+                 Hkv, nsplit) != cudaSuccess)
+      return SAMBA_ERR_CUDA;
     return SAMBA_OK;
   }
   if (dt == SAMBA_BF16 && hd == kHd && Hq / Hkv <= 8 && window <= kSplit * kSliceMax && ld % 8 == 0) {

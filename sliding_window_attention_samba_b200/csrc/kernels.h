@@ -36,7 +36,14 @@ samba_status launch_dcheck_selftest(cudaStream_t st);
 // ---------------- selective scan ----------------
 struct ScanArgs {
   const void* u = nullptr;
-  const void* dt = nullptr;
+  const void* dt = nullptr;       // Delta (or dt before softplus); NULL with dt_low below
+  // folded dt projection (bf16, dt_rank R <= 128, R % 16 == 0): Delta =
+  // softplus(dt_low W_dt^T + dt_bias) formed in the scan from dt_low [B, L, R]
+  // (row stride ld_dtl) and W_dt [D, R]
+  const void* dt_low = nullptr;
+  int64_t ld_dtl = 0;
+  int R = 0;
+  const void* W_dt = nullptr;
   const void* z = nullptr;
   const void* Bm = nullptr;
   const void* Cm = nullptr;
@@ -52,6 +59,7 @@ struct ScanArgs {
   samba_dtype dtype = SAMBA_BF16;
 };
 samba_status validate_scan(const ScanArgs& a);
+bool scan_dt_fold_supported(const ScanArgs& a);
 samba_status launch_selective_scan(const ScanArgs& a, cudaStream_t st);
 
 // ---------------- RoPE ----------------

@@ -31,6 +31,14 @@
 //     chunk) and stores y tiles (once every warp wrote its rows).
 // Every wait is bounded (error word on timeout); a timed-out CTA drains its
 // own copies in flight before it returns.
+//
+// With the dt projection folded in (kDt, bf16, dt_rank R <= 128, R % 16 == 0)
+// [Samba 3.4 "Input-Dependent Selective Gating": Delta = softplus(dt_low
+// W_dt^T + b)], the stages carry the chunk's rows of dt_low (128B-swizzled
+// boxes of 64 columns) instead of Delta, the CTA keeps its 16 rows of W_dt in
+// shared memory, and each warp forms Delta for its 8 tokens x 16 channels with
+// m16n8k16 tensor-core products (its 8 token rows repeated as the upper 8 rows
+// of the A tile) before the conversion, so Delta never goes through memory.
 #define SAMBA_TU_ID 6  // site id of this file in debug-check reports
 #include "common.cuh"
 #include "kernels.h"
@@ -51,11 +59,17 @@ constexpr int kBCPitch = 2 * kN + 4;  // 36 floats: rows 16 bytes apart in the b
 
 template <typename T> struct ScanCfg { static constexpr int kStages = sizeof(T) == 2 ? 4 : 2; };
 
-template <typename T>
+constexpr int kDtBox = 64;      // dt_low columns per TMA box (128 bytes of bf16)
+constexpr int kDtMaxBoxes = 2;  // dt_rank <= 128 on the folded path
+constexpr int kDtMaxR = kDtBox * kDtMaxBoxes;
+
+template <typename T, bool kDt>
 struct ScanSmem {
-  static constexpr int S = ScanCfg<T>::kStages;
-  T u[S][kChunk * kCh];  // [token][channel]
-  T dt[S][kChunk * kCh];
+  static constexpr int S = kDt ? 2 : ScanCfg<T>::kStages;
+  bf16 dtl[kDt ? S : 1][kDtMaxBoxes][kDt ? kChunk * kDtBox : 64];  // dt_low rows, 128B-swizzled (kDt)
+  bf16 Wd[kDt ? kCh : 1][kDt ? kDtMaxR + 8 : 64];                 // the CTA's rows of W_dt (kDt)
+  alignas(128) T u[S][kChunk * kCh];  // [token][channel]
+  T dt[kDt ? 1 : S][kChunk * kCh];
   T z[S][kChunk * kCh];
   T Bm[S][kChunk * kN];  // [token][state]
   T Cm[S][kChunk * kN];
@@ -73,17 +87,32 @@ struct ScanSmem {
 
 __device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
 
-template <typename T, bool kSoftplus, bool kHasZ>
+__device__ __forceinline__ void ldsm_x4(uint32_t* r, const void* row_addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(row_addr)));
+}
+__device__ __forceinline__ void mma_16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <typename T, bool kSoftplus, bool kHasZ, bool kDt>
 __global__ void __launch_bounds__(kThreads, 2)
     scan_chunked_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_dt,
                         const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_B,
                         const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ CUtensorMap tm_y,
                         const float* __restrict__ A_log, const float* __restrict__ dt_bias,
                         const float* __restrict__ Dskip, const float* __restrict__ h0, float* __restrict__ hT,
-                        int L, int D, int* err, int stop_chunk, uint64_t wait_limit_ns) {
-  constexpr int S = ScanCfg<T>::kStages;
-  extern __shared__ __align__(128) unsigned char smem_raw[];
-  ScanSmem<T>& Sm = *reinterpret_cast<ScanSmem<T>*>(smem_raw + smem_align_pad(smem_raw, 128));
+                        int L, int D, int* err, int stop_chunk, uint64_t wait_limit_ns,
+                        const bf16* __restrict__ W_dt, int R) {
+  using Smem = ScanSmem<T, kDt>;
+  constexpr int S = Smem::S;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  Smem& Sm = *reinterpret_cast<Smem*>(smem_raw + smem_align_pad(smem_raw, 1024));
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -97,7 +126,17 @@ __global__ void __launch_bounds__(kThreads, 2)
   const bool producer = warp == kWarps - 1 && lane == 0;
 
   constexpr uint32_t kStageBytes = (3 * kChunk * kCh + 2 * kChunk * kN) * sizeof(T);
-  const uint32_t stage_bytes = kHasZ ? kStageBytes : kStageBytes - kChunk * kCh * sizeof(T);
+  const int nbox = kDt ? (R + kDtBox - 1) / kDtBox : 0;
+  const uint32_t stage_bytes = (kHasZ ? kStageBytes : kStageBytes - kChunk * kCh * sizeof(T)) -
+                               (kDt ? kChunk * kCh * sizeof(T) - (uint32_t)nbox * kChunk * kDtBox * 2u : 0u);
+  if constexpr (kDt) {  // the CTA's 16 rows of W_dt (16-byte pieces; R % 16 == 0)
+    const int nv = R / 8;
+    for (int e = tid; e < kCh * nv; e += kThreads) {
+      const int r = e / nv, k = e % nv;
+      *reinterpret_cast<uint4*>(&Sm.Wd[r][k * 8]) =
+          *reinterpret_cast<const uint4*>(W_dt + (size_t)(d0 + r) * R + k * 8);
+    }
+  }
 
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
@@ -152,7 +191,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int t0 = c * kChunk;
     mbar_arrive_expect_tx(&Sm.full[s], stage_bytes);
     tma_load_3d(Sm.u[s], &tm_u, &Sm.full[s], d0, t0, b);
-    tma_load_3d(Sm.dt[s], &tm_dt, &Sm.full[s], d0, t0, b);
+    if constexpr (kDt) {
+      for (int k = 0; k < nbox; ++k) tma_load_3d(Sm.dtl[s][k], &tm_dt, &Sm.full[s], k * kDtBox, t0, b);
+    } else {
+      tma_load_3d(Sm.dt[s], &tm_dt, &Sm.full[s], d0, t0, b);
+    }
     if (kHasZ) tma_load_3d(Sm.z[s], &tm_z, &Sm.full[s], d0, t0, b);
     tma_load_3d(Sm.Bm[s], &tm_B, &Sm.full[s], 0, t0, b);
     tma_load_3d(Sm.Cm[s], &tm_C, &Sm.full[s], 0, t0, b);
@@ -179,6 +222,18 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int pr = lane >> 2;
   const float bias1 = dt_bias ? dt_bias[d] : 0.f;
   const float D1 = Dskip ? Dskip[d] : 0.f;
+  // folded dt projection: this lane's (token, channel) entries are the
+  // accumulator places of the m16n8k16 products: token lane / 4 of the warp's
+  // 8, channels 2q, 2q+1 (n-tile 0) and 8+2q, 9+2q (n-tile 1), q = lane % 4
+  float biasq[4] = {0.f, 0.f, 0.f, 0.f}, Dq[4] = {0.f, 0.f, 0.f, 0.f};
+  if (kDt) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int c = d0 + (e >> 1) * 8 + 2 * (lane & 3) + (e & 1);
+      biasq[e] = dt_bias ? dt_bias[c] : 0.f;
+      Dq[e] = Dskip ? Dskip[c] : 0.f;
+    }
+  }
 
   bool ok = true;
   int consumed = 0;  // chunks whose stage this warp saw land
@@ -189,11 +244,44 @@ __global__ void __launch_bounds__(kThreads, 2)
     // leaves the loop while the others still meet at a warp barrier)
     if (!__all_sync(0xffffffffu, wait(&Sm.full[s], (c / S) & 1))) { ok = false; break; }
     consumed = c + 1;
+    if constexpr (kDt) {
+      // Delta_pre[8 tokens x 16 channels] = dt_low rows x W_dt^T on the tensor cores
+      float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      const int arow = warp * kTs + (lane & 7);  // rows 8..15 of the A tile repeat rows 0..7
+      for (int ks = 0; ks < R / 16; ++ks) {
+        const int box = ks >> 2;
+        const int acol = (ks & 3) * 16 + ((lane >> 4) & 1) * 8;  // column within the 64-column box
+        const unsigned char* abase = reinterpret_cast<const unsigned char*>(Sm.dtl[s][box]);
+        uint32_t af[4], bfr[4];
+        ldsm_x4(af, abase + arow * 128 + ((((acol >> 3) ^ arow) & 7) << 4));
+        ldsm_x4(bfr, &Sm.Wd[((lane >> 4) & 1) * 8 + (lane & 7)][ks * 16 + ((lane >> 3) & 1) * 8]);
+        mma_16816(acc[0], af, bfr[0], bfr[1]);
+        mma_16816(acc[1], af, bfr[2], bfr[3]);
+      }
+      const int i = lane >> 2;  // token within the warp's slice
+      const int row = warp * kTs + i;
+      const int tg = c * kChunk + row;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int chq = (e >> 1) * 8 + 2 * (lane & 3) + (e & 1);
+        float delta = acc[e >> 1][e & 1] + biasq[e];
+        delta = softplus_1x(delta);
+        float uv = Elt<T>::to_f(Sm.u[s][row * kCh + chq]);
+        if (tg >= L) { delta = 0.f; uv = 0.f; }  // padding past the sequence: state unchanged
+        float g = 1.f;
+        if (kHasZ) {
+          const float zv = Elt<T>::to_f(Sm.z[s][row * kCh + chq]);
+          g = zv * sigmoid_fast(zv);
+        }
+        Sm.dd[warp][i][chq] = make_float2(delta, delta * uv);
+        Sm.gg[warp][i][chq] = make_float2(g, Dq[e] * uv * g);
+      }
+    }
     {
       // per (token, channel): lane = (channel ch, token half hf), tokens hf*4 .. hf*4+3
       // of the warp's slice, so each store writes whole 128-byte rows
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
+      for (int k = 0; k < 4 && !kDt; ++k) {
         const int i = hf * 4 + k;
         const int row = warp * kTs + i;
         const int tg = c * kChunk + row;
@@ -379,26 +467,34 @@ bool make_rows_map(CUtensorMap* m, const void* base, int64_t ld, int width, int 
   return make_tmap(m, base, dt, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
-template <typename T, bool kSoftplus, bool kHasZ>
+template <typename T, bool kSoftplus, bool kHasZ, bool kDt>
 samba_status launch_typed(const ScanArgs& a, cudaStream_t st) {
   CUtensorMap mu, mdt, mz, mB, mC, my;
-  bool ok = make_rows_map<T>(&mu, a.u, a.ld_u, a.D, kCh, a.L, a.B) &&
-            make_rows_map<T>(&mdt, a.dt, a.ld_dt, a.D, kCh, a.L, a.B) &&
-            make_rows_map<T>(&mB, a.Bm, a.ld_bc, kN, kN, a.L, a.B) &&
+  bool ok = make_rows_map<T>(&mu, a.u, a.ld_u, a.D, kCh, a.L, a.B);
+  if (kDt) {  // dt_low rows: 64-column boxes, 128B-swizzled, columns past R read as zeros
+    uint64_t dims[3] = {(uint64_t)a.R, (uint64_t)a.L, (uint64_t)a.B};
+    uint64_t strides[2] = {(uint64_t)a.ld_dtl, (uint64_t)a.ld_dtl * (uint64_t)a.L};
+    uint32_t box[3] = {(uint32_t)kDtBox, (uint32_t)kChunk, 1};
+    ok = ok && make_tmap(&mdt, a.dt_low, SAMBA_BF16, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+  } else {
+    ok = ok && make_rows_map<T>(&mdt, a.dt, a.ld_dt, a.D, kCh, a.L, a.B);
+  }
+  ok = ok && make_rows_map<T>(&mB, a.Bm, a.ld_bc, kN, kN, a.L, a.B) &&
             make_rows_map<T>(&mC, a.Cm, a.ld_bc, kN, kN, a.L, a.B) &&
             make_rows_map<T>(&my, a.y, a.ld_y, a.D, kCh, a.L, a.B);
   if (kHasZ) ok = ok && make_rows_map<T>(&mz, a.z, a.ld_z, a.D, kCh, a.L, a.B);
   else mz = mu;
   if (!ok) return SAMBA_ERR_CUDA;
-  const size_t smem = sizeof(ScanSmem<T>) + 128;
-  auto kern = scan_chunked_kernel<T, kSoftplus, kHasZ>;
+  const size_t smem = sizeof(ScanSmem<T, kDt>) + 1024;
+  auto kern = scan_chunked_kernel<T, kSoftplus, kHasZ, kDt>;
   if (!ensure_smem_attr(kern, smem))
     return SAMBA_ERR_CUDA;
   dim3 grid(a.D / kCh, a.B);
   const StallHook hk = scan_stall_hook();
   kern<<<grid, kThreads, smem, st>>>(mu, mdt, mz, mB, mC, my, a.A_log, a.dt_bias, a.Dskip, a.h0, a.hT, a.L, a.D,
                                      device_error_word(), hk.stop_chunk < 0 ? INT32_MAX : hk.stop_chunk,
-                                     hk.stop_chunk < 0 ? kWaitLimitNs : hk.wait_limit_ns);
+                                     hk.stop_chunk < 0 ? kWaitLimitNs : hk.wait_limit_ns,
+                                     (const bf16*)a.W_dt, a.R);
   SAMBA_CHECK_LAUNCH();
   return SAMBA_OK;
 }
@@ -406,25 +502,31 @@ samba_status launch_typed(const ScanArgs& a, cudaStream_t st) {
 template <typename T>
 samba_status launch_dispatch(const ScanArgs& a, cudaStream_t st) {
   if (a.softplus) {
-    return a.z ? launch_typed<T, true, true>(a, st) : launch_typed<T, true, false>(a, st);
+    return a.z ? launch_typed<T, true, true, false>(a, st) : launch_typed<T, true, false, false>(a, st);
   }
-  return a.z ? launch_typed<T, false, true>(a, st) : launch_typed<T, false, false>(a, st);
+  return a.z ? launch_typed<T, false, true, false>(a, st) : launch_typed<T, false, false, false>(a, st);
 }
 
 }  // namespace
 
+bool scan_dt_fold_supported(const ScanArgs& a) {
+  return a.dtype == SAMBA_BF16 && a.dt_low && a.W_dt && a.R >= 16 && a.R <= kDtMaxR && a.R % 16 == 0 &&
+         aligned16(a.dt_low) && aligned16(a.W_dt) && (a.ld_dtl * 2) % 16 == 0 && a.ld_dtl >= a.R;
+}
+
 samba_status validate_scan(const ScanArgs& a) {
-  if (!a.u || !a.dt || !a.A_log || !a.Bm || !a.Cm || !a.y) return SAMBA_ERR_INVALID_ARG;
+  if (!a.u || !(a.dt || a.dt_low) || !a.A_log || !a.Bm || !a.Cm || !a.y) return SAMBA_ERR_INVALID_ARG;
+  if (!a.dt && !scan_dt_fold_supported(a)) return SAMBA_ERR_UNSUPPORTED;
   if (a.B < 1 || a.L < 0 || a.D < 1 || a.N < 1) return SAMBA_ERR_INVALID_ARG;
   if (a.N != kN || a.D % kCh != 0 || a.B > kMaxGridYZ) return SAMBA_ERR_UNSUPPORTED;
   const size_t es = dtype_size(a.dtype);
   const void* ptrs[] = {a.u, a.dt, a.Bm, a.Cm, a.y, a.z};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return SAMBA_ERR_UNSUPPORTED;
-  const int64_t lds[] = {a.ld_u, a.ld_dt, a.ld_bc, a.ld_y, a.z ? a.ld_z : a.ld_u};
+  const int64_t lds[] = {a.ld_u, a.dt ? a.ld_dt : a.ld_u, a.ld_bc, a.ld_y, a.z ? a.ld_z : a.ld_u};
   for (int64_t ld : lds)
     if ((ld * (int64_t)es) % 16 != 0) return SAMBA_ERR_UNSUPPORTED;
-  if (a.ld_u < a.D || a.ld_dt < a.D || a.ld_y < a.D || a.ld_bc < a.N || (a.z && a.ld_z < a.D))
+  if (a.ld_u < a.D || (a.dt && a.ld_dt < a.D) || a.ld_y < a.D || a.ld_bc < a.N || (a.z && a.ld_z < a.D))
     return SAMBA_ERR_INVALID_ARG;
   return SAMBA_OK;
 }
@@ -439,6 +541,9 @@ samba_status launch_selective_scan(const ScanArgs& a, cudaStream_t st) {
       SAMBA_CHECK_LAUNCH();
     }
     return SAMBA_OK;
+  }
+  if (!a.dt) {  // the dt projection folded in (bf16; softplus always applied)
+    return a.z ? launch_typed<bf16, true, true, true>(a, st) : launch_typed<bf16, true, false, true>(a, st);
   }
   return a.dtype == SAMBA_BF16 ? launch_dispatch<bf16>(a, st) : launch_dispatch<float>(a, st);
 }

@@ -338,15 +338,17 @@ def test_decode_wide_bf16_conv_bias(L):
         assert step_err(y, x[:, P + i], full, P + i, "bf16") <= TOL["bf16"], i
 
 
-def test_decode_streaming_attention_window_4096(L):
-    """The streaming decode attention over a 4096-slot ring (its largest
-    window): 28 rows x 4 kv heads, 100 prefilled tokens, two steps."""
+@pytest.mark.parametrize("Bn", [28, 2])
+def test_decode_window_4096(L, Bn):
+    """A 4096-slot ring in samba_step: at 28 rows x 4 kv heads the streaming
+    decode attention (its largest window), at 2 rows the per-slice kernel with
+    the partials in samba_step's own workspace; 100 prefilled tokens, two steps."""
     import dataclasses
     shape = dataclasses.replace(I.WIDE, window=4096)
     W = I.block_weights(shape, 14)
     P, S = 100, 2
-    x = I.block_input(shape, 14, 28, P + S)
-    g = GpuBlock(L, shape, W, 28, P + S)
+    x = I.block_input(shape, 14, Bn, P + S)
+    g = GpuBlock(L, shape, W, Bn, P + S)
     g.prefill(x[:, :P], taps=False)
     full = O.block_fwd(x, W, shape)
     for i in range(S):

@@ -153,3 +153,42 @@ def test_scan_bounded_wait_times_out_and_recovers(L):
     yo, ho = oracle_scan(r, h0=r["h0"])
     assert rel_err(y, yo) <= TOL["bf16"]
     assert rel_err(hT, ho) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("Bn,Ln,D,R", [(1, 4096, 4096, 128), (2, 300, 64, 128), (1, 129, 32, 64), (2, 65, 48, 16)])
+def test_scan_xdbl_matches_oracle(L, Bn, Ln, D, R):
+    """The scan with the dt projection folded in (samba_selective_scan_xdbl):
+    Delta = softplus(dt_low W_dt^T + b) formed inside the kernel on tensor-core
+    tiles from the x_proj output [dt_low | B | C], against the oracle's
+    projection, softplus and scan in fp64 on the same (bf16) values."""
+    import torch
+    r = I.scan_inputs(7, Bn, Ln, D, 16, "bf16", with_h0=True)
+    dt_low = I.draw_normal(7, "scan.dt_low", (Bn, Ln, R), 1.0, "bf16")
+    W_dt = I.draw_normal(7, "scan.W_dt", (D, R), R ** -0.5, "bf16")
+    x_dbl = np.concatenate([dt_low, r["B"], r["C"]], axis=-1)
+    y = torch.empty(Bn, Ln, D, device="cuda", dtype=torch.bfloat16)
+    hT = torch.empty(Bn, D, 16, device="cuda")
+    L.samba_selective_scan_xdbl(dev(r["u"], "bf16"), dev(x_dbl, "bf16"), R, dev(W_dt, "bf16"), dev(r["dt_bias"]),
+                                dev(r["A_log"]), dev(r["D"]), dev(r["z"], "bf16"), dev(r["h0"]), hT, y, Bn, Ln, D,
+                                16, 1)
+    torch.cuda.synchronize()
+    assert L.samba_get_error() == 0
+    delta = O.softplus(O.linear(dt_low.astype(np.float64), W_dt.astype(np.float64)) + r["dt_bias"])
+    A = -np.exp(r["A_log"].astype(np.float64))
+    yo, ho = O.selective_scan(r["u"], delta, A, r["B"], r["C"], r["D"], r["z"], r["h0"])
+    assert rel_err(host(y), yo) <= TOL["bf16"]
+    assert rel_err(host(hT), ho) <= TOL["bf16"]
+
+
+def test_scan_xdbl_rejects_unsupported(L):
+    """Outside the folded kernel's range the entry point refuses before any launch."""
+    import torch
+    from sliding_window_attention_samba_b200._lib import SambaError
+    u = torch.zeros(1, 64, 64, device="cuda", dtype=torch.bfloat16)
+    x = torch.zeros(1, 64, 176 + 32, device="cuda", dtype=torch.bfloat16)
+    W = torch.zeros(64, 176, device="cuda", dtype=torch.bfloat16)
+    A = torch.zeros(64, 16, device="cuda")
+    y = torch.empty_like(u)
+    with pytest.raises(SambaError) as e:  # dt_rank 176 > 128
+        L.samba_selective_scan_xdbl(u, x, 176, W, None, A, None, None, None, None, y, 1, 64, 64, 16, 1)
+    assert e.value.code == L.SAMBA_ERR_UNSUPPORTED
