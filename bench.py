@@ -224,9 +224,10 @@ def swa_flops(s, Bn, Ln):
 
 
 def dt_folded(s):
-    """The block forms Delta inside the scan kernel (bf16, dt_rank <= 128, a
-    multiple of 16): no separate dt projection launch."""
-    return s.dtype == "bf16" and s.dt_rank % 16 == 0 and 16 <= s.dt_rank <= 128
+    """The block forms Delta inside the scan kernel (opt-in: SAMBA_SCAN_FOLD_DT=1;
+    bf16, dt_rank <= 128, a multiple of 16): no separate dt projection launch."""
+    return (os.environ.get("SAMBA_SCAN_FOLD_DT") == "1" and s.dtype == "bf16" and s.dt_rank % 16 == 0
+            and 16 <= s.dt_rank <= 128)
 
 
 def attribution_pass(torch, L, s, blocks, x, T, Bn, Ln, reps=2):

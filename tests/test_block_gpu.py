@@ -354,3 +354,19 @@ def test_decode_window_4096(L, Bn):
     for i in range(S):
         y = host(g.step(x[:, P + i]))
         assert step_err(y, x[:, P + i], full, P + i, "bf16") <= TOL["bf16"], i
+
+
+def test_block_wide_bf16_folded_dt(L):
+    """SAMBA_SCAN_FOLD_DT=1: the block's scan forms Delta itself from the x_proj
+    output (no dt projection launch); every branch against the oracle."""
+    shape = I.WIDE
+    W = I.block_weights(shape, 15)
+    x = I.block_input(shape, 15, 1, 300)
+    import os
+    os.environ["SAMBA_SCAN_FOLD_DT"] = "1"
+    try:
+        g = GpuBlock(L, shape, W, 1, 300)
+        out, br, rs = g.prefill(x)
+    finally:
+        del os.environ["SAMBA_SCAN_FOLD_DT"]
+    check_branches(shape, W, x, out, br, rs, TOL["bf16"])
