@@ -206,9 +206,18 @@ struct TcEpi {
 };
 constexpr uint32_t TC_A_BYTES = TC_BM * TC_BK * 2;
 
+// Output staging of the epilogue warps: each warp's 32 rows x 32 columns of
+// bf16 (64-byte rows, 16-byte pieces swizzled as the tensor map's 64B swizzle
+// expects: piece j of row r at j ^ ((r >> 1) & 3)), written back by a TMA
+// store so that the global writes are whole row segments rather than 16 bytes
+// in each of 32 rows per warp store.
+constexpr int TC_MAX_EPI_WARPS = 16;
+constexpr int TC_OST_BYTES = 32 * 64;
+
 struct TcSmem {
   bf16 A[TC_STAGES][TC_BM * TC_BK];
   bf16 B[TC_STAGES][TC_MAXN * TC_BK];
+  alignas(1024) unsigned char ost[TC_MAX_EPI_WARPS][TC_OST_BYTES];
   uint64_t full[TC_STAGES], empty[TC_STAGES], tfull[2], tempty[2];
   uint32_t tmem_base;
 };
@@ -217,6 +226,8 @@ struct TcParams {
   CUtensorMap tmA;
   CUtensorMap tmB[3];
   CUtensorMap tmB2;
+  CUtensorMap tmO;  // output, boxes of 32 rows x 32 columns, 64B swizzle (when tma_out)
+  int tma_out;      // the epilogue writes through the staging buffers and TMA stores
   GemmArgs a;
   int bn;          // output columns per tile
   int umma_n;      // accumulator columns per tile (2*bn for SwiGLU)
@@ -244,10 +255,54 @@ __device__ __forceinline__ void part_range(int n, int part, int parts, int& lo, 
   hi = (n * (part + 1)) / parts;
 }
 
+// A warp writes its 32 rows x 32 columns (row = lane) at columns
+// [col, col + 32) in four 8-column pieces: through the warp's staging buffer
+// and one TMA store (p.tma_out; rows past M and columns past N are clipped by
+// the tensor map), or directly (rows past M skipped, only valid pieces).
+__device__ __forceinline__ void tc_emit_begin(const TcParams& p) {
+  if (!p.tma_out) return;
+  if ((threadIdx.x & 31) == 0) tma_store_wait_read<0>();  // the previous store has read the buffer
+  __syncwarp();
+}
+__device__ __forceinline__ void tc_emit_piece(const TcParams& p, unsigned char* ost, int64_t row, int col, int j,
+                                              bool valid, const float* f8) {
+  const int lane = threadIdx.x & 31;
+  if (p.tma_out) {
+    uint4 v;
+    uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      __nv_bfloat162 h = __floats2bfloat162_rn(f8[2 * e], f8[2 * e + 1]);
+      w[e] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    *reinterpret_cast<uint4*>(ost + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) = v;
+    return;
+  }
+  if (valid && row < p.a.M) store8((bf16*)p.a.out + row * p.a.ldo + col + 8 * j, f8);
+}
+__device__ __forceinline__ void tc_emit_end(const TcParams& p, unsigned char* ost, int64_t row, int col) {
+  if (!p.tma_out) return;
+  const int lane = threadIdx.x & 31;
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(&p.tmO, ost, col, (int)(row - lane));
+    tma_store_commit();
+  }
+}
+__device__ __forceinline__ void tc_emit32(const TcParams& p, unsigned char* ost, int64_t row, int col, int nv,
+                                          const float* f) {
+  tc_emit_begin(p);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) tc_emit_piece(p, ost, row, col, j, j < nv, f + 8 * j);
+  tc_emit_end(p, ost, row, col);
+}
+
 // One epilogue warp's share of a tile: TMEM lane quadrant = 32 rows, and part
 // `part` of the tile's column units (32-column chunks; 64-column RoPE units).
 template <int EPI>
-__device__ __forceinline__ void tc_epilogue_tile(const TcParams& p, uint32_t tbase, int64_t row, int nt, int part) {
+__device__ __forceinline__ void tc_epilogue_tile(const TcParams& p, uint32_t tbase, int64_t row, int nt, int part,
+                                                 unsigned char* ost) {
   const GemmArgs& a = p.a;
   const bool in_range = row < a.M;
   const int col0 = nt * p.bn;
@@ -260,17 +315,13 @@ __device__ __forceinline__ void tc_epilogue_tile(const TcParams& p, uint32_t tba
       tmem_ld32(tbase + cc, r);
       tmem_ld32(tbase + p.bn + cc, r2);
       tmem_wait_ld();
-      if (in_range) {
-        float f[32];
+      float f[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float g = __uint_as_float(r2[i]);
-          f[i] = __uint_as_float(r[i]) * (g * sigmoid_fast(g));
-        }
-        bf16* o = out + row * a.ldo + col0 + cc;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) store8(o + 8 * i, f + 8 * i);
+      for (int i = 0; i < 32; ++i) {
+        const float g = __uint_as_float(r2[i]);
+        f[i] = __uint_as_float(r[i]) * (g * sigmoid_fast(g));
       }
+      tc_emit32(p, ost, row, col0 + cc, 4, f);
     }
     return;
   }
@@ -344,15 +395,15 @@ __device__ __forceinline__ void tc_epilogue_tile(const TcParams& p, uint32_t tba
     part_range((p.bn + 31) / 32, part, TcEpi<EPI>::parts, u_lo, u_hi);
     auto chunk = [&](const uint32_t (&rc)[32], int u) {
       const int cc = u * 32;
-      if (!in_range) return;
       const int nv = min(4, (p.bn - cc) / 8);
       const int col = col0 + cc;
       const float4* bp = reinterpret_cast<const float4*>(a.bias + col);  // 16-byte aligned (checked at launch)
-      bf16* o = out + row * a.ldo + col;
+      tc_emit_begin(p);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {  // 8 columns at a time, stored at once
-        if (i >= nv) continue;
-        const float4 b0 = bp[2 * i], b1 = bp[2 * i + 1];
+      for (int i = 0; i < 4; ++i) {  // 8 columns at a time
+        const bool valid = i < nv;
+        const float4 b0 = valid ? bp[2 * i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 b1 = valid ? bp[2 * i + 1] : make_float4(0.f, 0.f, 0.f, 0.f);
         float f[8];
         f[0] = softplus_1x(__uint_as_float(rc[8 * i + 0]) + b0.x);
         f[1] = softplus_1x(__uint_as_float(rc[8 * i + 1]) + b0.y);
@@ -362,8 +413,9 @@ __device__ __forceinline__ void tc_epilogue_tile(const TcParams& p, uint32_t tba
         f[5] = softplus_1x(__uint_as_float(rc[8 * i + 5]) + b1.y);
         f[6] = softplus_1x(__uint_as_float(rc[8 * i + 6]) + b1.z);
         f[7] = softplus_1x(__uint_as_float(rc[8 * i + 7]) + b1.w);
-        store8(o + 8 * i, f);
+        tc_emit_piece(p, ost, row, col, i, valid, f);
       }
+      tc_emit_end(p, ost, row, col);
     };
     uint32_t ra[32], rb[32];
     if (u_lo < u_hi) tmem_ld32(tbase + u_lo * 32, ra);
@@ -385,13 +437,12 @@ __device__ __forceinline__ void tc_epilogue_tile(const TcParams& p, uint32_t tba
   for (int cc = u_lo * 32; cc < u_hi * 32; cc += 32) {
     tmem_ld32(tbase + cc, r);
     tmem_wait_ld();
-    if (!in_range) continue;
     const int nv = min(4, (p.bn - cc) / 8);  // valid 8-column groups: 4, or 2 in a 16-column tail
     float f[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(r[i]);
     const int col = col0 + cc;
-    if (EPI == kEpiResid) {
+    if (EPI == kEpiResid && in_range) {
       if (a.tap) {
         bf16* t = (bf16*)a.tap + row * a.ldt + col;
 #pragma unroll
@@ -408,10 +459,7 @@ __device__ __forceinline__ void tc_epilogue_tile(const TcParams& p, uint32_t tba
         for (int j = 0; j < 8; ++j) f[8 * i + j] += g[j];
       }
     }
-    bf16* o = out + row * a.ldo + col;
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      if (i < nv) store8(o + 8 * i, f + 8 * i);
+    tc_emit32(p, ost, row, col, nv, f);
   }
 }
 
@@ -529,11 +577,14 @@ __global__ void __launch_bounds__(TcEpi<EPI>::threads, 1) gemm_tc_kernel(const _
       tc_fence_after();
       const uint32_t tbase = tmem + acc * TC_MAXN + ((uint32_t)(q * 32) << 16);
       const int64_t row = (int64_t)mt * TC_BM + q * 32 + lane;
-      if (SAMBA_DCHECK(err, mt < p.m_tiles && (nt + 1) * p.bn <= p.a.N)) tc_epilogue_tile<EPI>(p, tbase, row, nt, part);
+      if (SAMBA_DCHECK(err, mt < p.m_tiles && (nt + 1) * p.bn <= p.a.N))
+        tc_epilogue_tile<EPI>(p, tbase, row, nt, part, S.ost[warp - 2]);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.tempty[acc]);
     }
+    if (lane == 0) tma_store_wait_all<0>();  // this warp's output stores complete before the CTA exits
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
@@ -562,6 +613,8 @@ bool tc_bn_for(const GemmArgs& a, int& bn) {
   }
   return false;
 }
+
+static_assert(sizeof(TcSmem) + 1024 <= 232448, "tcgen05 GEMM shared memory above the 227 KB per-block limit");
 
 template <int EPI>
 samba_status tc_launch(TcParams& p, cudaStream_t st) {
@@ -612,6 +665,14 @@ samba_status launch_gemm_tc(const GemmArgs& a, cudaStream_t st) {
   }
   p.k_blocks = (a.K + TC_BK - 1) / TC_BK;
   p.a_evict_first = a.K >= 4096 ? 1 : 0;
+  {
+    // output through staging buffers and TMA stores (64B swizzle, 32 x 32 boxes)
+    uint64_t dims[2] = {(uint64_t)a.N, (uint64_t)a.M};
+    uint64_t strides[1] = {(uint64_t)a.ldo};
+    uint32_t box[2] = {32, 32};
+    if (!make_tmap(&p.tmO, a.out, SAMBA_BF16, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_64B)) return SAMBA_ERR_CUDA;
+    p.tma_out = 1;
+  }
   {
     uint64_t dims[2] = {(uint64_t)a.K, (uint64_t)a.M};
     uint64_t strides[1] = {(uint64_t)a.lda};
