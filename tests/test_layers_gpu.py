@@ -82,7 +82,8 @@ def _linear(L, dt, M, N, K, epi, force_simt=False):
 
 
 @pytest.mark.parametrize("epi", [0, 1, 2, 3])
-@pytest.mark.parametrize("M,N,K", [(300, 256, 2048), (128, 160, 4096), (1000, 512, 128), (77, 2048, 1024)])
+@pytest.mark.parametrize("M,N,K", [(300, 256, 2048), (128, 160, 4096), (1000, 512, 128), (77, 2048, 1024),
+                                   (200, 176, 256)])
 def test_linear_tensor_core_bf16(L, epi, M, N, K):
     assert _linear(L, "bf16", M, N, K, epi) <= TOL["bf16"]
 
