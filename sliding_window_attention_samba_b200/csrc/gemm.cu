@@ -12,7 +12,9 @@
 //    tcgen05.mma (M=128, N<=256, K=16) issued by one thread into a double
 //    buffered 2x256-column TMEM accumulator, so the epilogue of one tile
 //    overlaps the main loop of the next.  Epilogues (residual add, SwiGLU,
-//    softplus+bias, RoPE) are fused on the TMEM read-out.
+//    softplus+bias, RoPE) are fused on the TMEM read-out; each epilogue warp
+//    writes its 32 rows x 32 columns through a shared-memory staging buffer
+//    and a TMA store (RoPE tiles store directly).
 //  * gemm_simt: CUDA-core fp32 FMA tiles, used for fp32 data (no TF32: its
 //    ~1e-3 error would break the fp32 tolerance) and for shapes the tensor-core
 //    kernel does not take.

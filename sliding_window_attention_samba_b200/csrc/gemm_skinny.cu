@@ -8,10 +8,15 @@
 //   * split-K across a thread-block cluster of S <= 8 CTAs (one n-tile per
 //     cluster), each CTA streaming a K range of the weight tile through a
 //     4-stage TMA ring into tcgen05.mma;
-//   * the S fp32 partial tiles are reduced through distributed shared memory
-//     (ld.shared::cluster) and the epilogue (residual, SwiGLU, softplus+bias,
-//     RoPE at per-row positions) is applied in the same kernel, so no partial
-//     sums ever reach HBM.
+//   * the S fp32 partial tiles are pushed into their owner CTA's shared memory
+//     (st.shared::cluster, feature-innermost) and each owner finalises 8
+//     consecutive features of a batch row per thread with 16-byte accesses;
+//     the epilogue (residual, SwiGLU, softplus+bias, RoPE at per-row
+//     positions from a table or evaluated from the position) is applied in
+//     the same kernel, so no partial sums ever reach HBM;
+//   * decode-step folds: the short-conv step on in_proj's x columns, the new
+//     token's k, v into the ring slot by the QKV projection, the position
+//     advance by the step's last projection.
 // No cluster multicast is used (each CTA loads its own tiles).
 #include <stdlib.h>
 #include <string.h>
