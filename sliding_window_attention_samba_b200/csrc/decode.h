@@ -21,8 +21,12 @@ samba_status launch_scan_step_dt(const void* u, const void* z, int64_t ld_z, con
                                  float* ssm, void* y, int B, int D, samba_dtype dt, cudaStream_t st);
 samba_status launch_ring_write(const void* qkv, int64_t ld, int k_off, int v_off, const int64_t* pos, void* k_ring,
                                void* v_ring, int B, int window, int kvw, samba_dtype dt, cudaStream_t st);
-// Ring caches above 2048 slots (bf16, head_dim 64) need attn_decode_workspace_bytes() of workspace for the
-// per-slice partials; smaller ones none.
+// Decode attention over the ring (bf16, head_dim 64, up to 8 query heads per kv
+// head): with at least 3/4 of an SM's worth of (kv head, row) pairs per SM and
+// rings up to 4096 slots, one streaming CTA per pair; otherwise an 8-CTA
+// cluster per pair (rings up to 2048 slots) or, above 2048 slots, one CTA per
+// 256-slot slice whose partials need attn_decode_workspace_bytes() of
+// workspace (0 when not needed).  Other dtypes and head dims: a CUDA-core kernel.
 size_t attn_decode_workspace_bytes(int B, int Hkv, int window);
 samba_status launch_attn_decode(const void* qkv, int64_t ld, const int64_t* pos, const void* k_ring,
                                 const void* v_ring, void* o, int B, int Hq, int Hkv, int hd, int window, float scale,
