@@ -165,6 +165,24 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # the CUDA path
 # ---------------------------------------------------------------------------
+def graph_kernel_nodes(graph):
+    """Kernel nodes of a CUDA graph captured with keep_graph=True (the launches
+    one replay makes), or None where the runtime bindings cannot tell."""
+    try:
+        from cuda.bindings import runtime as rt
+        g = rt.cudaGraph_t(init_value=graph.raw_cuda_graph())
+        err, _, n = rt.cudaGraphGetNodes(g, 0)
+        if err != rt.cudaError_t.cudaSuccess:
+            return None
+        err, nodes, n = rt.cudaGraphGetNodes(g, n)
+        if err != rt.cudaError_t.cudaSuccess:
+            return None
+        kernel = rt.cudaGraphNodeType.cudaGraphNodeTypeKernel
+        return sum(1 for x in nodes[:n] if rt.cudaGraphNodeGetType(x)[1] == kernel)
+    except Exception:
+        return None
+
+
 def make_stack(torch, L, shape, n_blocks, seed, dev):
     """Random-init weights of the stack on the device (N(0, 0.02) matrices,
     S4D-Real A, D = 1, Delta bias in [1e-3, 1e-1], unit norm gains)."""
@@ -632,9 +650,11 @@ def measure_decode(steps, warmup, prefill=None):
     stream.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(stream):
         L.samba_step(cfg, wst, xt, yt, st, Bn, ws, ws_bytes, stream=stream)  # first call outside capture
-        graph = torch.cuda.CUDAGraph()
+        graph = torch.cuda.CUDAGraph(keep_graph=True)
         with torch.cuda.graph(graph, stream=stream):
             L.samba_step(cfg, wst, xt, yt, st, Bn, ws, ws_bytes, stream=stream)
+        nk = graph_kernel_nodes(graph)  # the step's kernel launches, read from the captured graph
+        graph.instantiate()
         for _ in range(max(3, warmup)):
             graph.replay()
         stream.synchronize()
@@ -678,11 +698,15 @@ def measure_decode(steps, warmup, prefill=None):
                          "kernel": "whole decode step (weights + ring + states per step)",
                          "peak_source": src, "bytes_per_step": bps},
             "clocks": clk, "graph": "one samba_step captured, replayed per step",
-            # per step: 4 RMSNorms, 9 skinny projections (in_proj with the conv
-            # step, x_proj, out_proj, QKV with RoPE and the ring write, o_proj,
-            # 2 x SwiGLU up, 2 x down, the last advancing the positions), the
-            # recurrence step with the dt projection, the streaming attention
-            "gpu_launches": 15 * steps}
+            # per step: the first RMSNorm (the other three ride on the
+            # projections around them: the norm fold), 9 skinny projections
+            # (in_proj with the conv step, x_proj, out_proj, QKV with RoPE and
+            # the ring write, o_proj, 2 x SwiGLU up, 2 x down, the last
+            # advancing the positions), the recurrence step with the dt
+            # projection, the streaming attention: 12 launches; 15 with the
+            # fold off (SAMBA_NORM_FOLD=0)
+            "gpu_launches": (nk if nk else 12) * steps,
+            "launches_per_step": {"value": nk if nk else 12, "source": "graph nodes" if nk else "claimed"}}
 
 
 def run_decode(args):
@@ -694,7 +718,8 @@ def run_decode(args):
             "dtype": "bf16", "data": "synthetic",
             "config": {"workload": "decode_bf16_B32", "batch": d["batch"], "prefill": d["prefill"],
                        "window": d["window"], "d_model": I.WIDE.d_model, "graph": d["graph"]},
-            "e2e": d["e2e"], "roofline": d["roofline"], "clocks": d["clocks"], "gpu_launches": d["gpu_launches"]}
+            "e2e": d["e2e"], "roofline": d["roofline"], "clocks": d["clocks"], "gpu_launches": d["gpu_launches"],
+            "launches_per_step": d["launches_per_step"]}
     print(json.dumps(line))
 
 

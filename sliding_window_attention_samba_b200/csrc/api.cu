@@ -199,7 +199,7 @@ static samba_status guards_check(char* base, const Carve& c, cudaStream_t st) {
 }
 
 struct BlockPlan {
-  size_t tab, xn, hz, u, xdbl, dlt, y, x1, x2, x3, hmlp, qkv, o, kx, vx, convh, total;
+  size_t tab, xn, hz, u, xdbl, dlt, y, x1, x2, x3, hmlp, qkv, o, kx, vx, convh, ss, total;
   int xdw, qkvw;
   Carve cv;  // the carving (guard bands of the debug-check build)
 };
@@ -229,6 +229,8 @@ static BlockPlan plan_block(const samba_block_config& c, int64_t T, int chunk_B 
   p.kx = cv.take(kv_rows * c.n_kv * c.head_dim * es);
   p.vx = cv.take(kv_rows * c.n_kv * c.head_dim * es);
   p.convh = cv.take((int64_t)chunk_B * c.d_inner * (c.d_conv - 1) * es);
+  // decode norm fold: partial sums of squares of norms 1..3, d_model/8 per row, for up to 64 rows
+  p.ss = cv.take((size_t)3 * std::min<int64_t>(T, 64) * (c.d_model / 8) * sizeof(float));
   p.total = cv.off + 256;  // slack for aligning the caller's base pointer
   p.cv = cv;
   return p;
@@ -290,13 +292,18 @@ static GemmArgs gemm1(const void* A, int64_t lda, const void* W, int64_t M, int 
 static samba_status mlp_sublayer(const samba_block_config& c, const float* g, const void* W1, const void* W2,
                                  const void* W3, const void* x, void* x_next, void* xn, void* hmlp, void* tap,
                                  int64_t T, cudaStream_t st, bool pdl = false, int64_t* pos_inc = nullptr,
-                                 bool* pos_done = nullptr) {
+                                 bool* pos_done = nullptr, const float* ss_in = nullptr, float* ss_out = nullptr,
+                                 const float* g_next = nullptr) {
   NvtxRange nvtx_("samba.mlp");
-  TRY(launch_rmsnorm(x, c.d_model, g, xn, c.d_model, T, c.d_model, c.norm_eps, c.dtype, st, pdl));
+  // ss_in (decode norm fold): xn already holds x (.) g from the producer of x
+  if (!ss_in) TRY(launch_rmsnorm(x, c.d_model, g, xn, c.d_model, T, c.d_model, c.norm_eps, c.dtype, st, pdl));
   GemmArgs up = gemm1(xn, c.d_model, W1, T, c.d_ff, c.d_model, hmlp, c.d_ff, c.dtype);
   up.seg[0].W2 = W2;
   up.epi = kEpiSwiglu;
   up.pdl = pdl;
+  up.ss_in = ss_in;
+  up.norm_dim = c.d_model;
+  up.norm_eps = c.norm_eps;
   TRY(launch_gemm(up, st));
   GemmArgs dn = gemm1(hmlp, c.d_ff, W3, T, c.d_model, c.d_ff, x_next, c.d_model, c.dtype);
   dn.pdl = pdl;
@@ -305,6 +312,11 @@ static samba_status mlp_sublayer(const samba_block_config& c, const float* g, co
   dn.ldr = c.d_model;
   dn.tap = tap;
   dn.ldt = c.d_model;
+  if (ss_out) {  // the next norm's input and sums of squares
+    dn.ss_out = ss_out;
+    dn.g_next = g_next;
+    dn.xg_out = xn;
+  }
   if (pos_inc) {  // decode: the step's last projection also advances the positions
     GemmArgs dp = dn;
     dp.pos_inc = pos_inc;
@@ -774,7 +786,7 @@ static samba_status swa_sublayer(const LayerCtx& X, const samba_block_weights* w
 // a programmatic dependent of the one before it: a kernel sets up (and the
 // projections fetch their first weight tiles) while its predecessor finishes.
 static samba_status mamba_step_layer(const LayerCtx& X, const samba_block_weights* w, const void* x_in, void* x_out,
-                                     float* ssm, void* conv) {
+                                     float* ssm, void* conv, float* ssf = nullptr) {
   NvtxRange nvtx_("samba.mamba_step");
   const samba_block_config& c = X.c;
   const BlockPlan& P = X.P;
@@ -826,6 +838,11 @@ static samba_status mamba_step_layer(const LayerCtx& X, const samba_block_weight
   g.epi = kEpiResid;
   g.resid = x_in;
   g.ldr = Dm;
+  if (ssf) {  // the MLP norm's input and sums of squares
+    g.ss_out = ssf;
+    g.g_next = w->norm_g[1];
+    g.xg_out = xn;
+  }
   return gemm_pdl(g);
 }
 
@@ -835,7 +852,8 @@ static samba_status mamba_step_layer(const LayerCtx& X, const samba_block_weight
 // attn_ws: partials of the split attention for rings above 2048 slots.
 static samba_status swa_step_layer(const LayerCtx& X, const samba_block_weights* w, const void* x_in, void* x_out,
                                    void* k_ring, void* v_ring, const int64_t* pos, void* attn_ws,
-                                   size_t attn_ws_bytes) {
+                                   size_t attn_ws_bytes, const float* ss_in = nullptr, float* ss_out = nullptr,
+                                   const float* g_next = nullptr) {
   NvtxRange nvtx_("samba.swa_step");
   const samba_block_config& c = X.c;
   const BlockPlan& P = X.P;
@@ -847,7 +865,7 @@ static samba_status swa_step_layer(const LayerCtx& X, const samba_block_weights*
   void* xn = buf(P.xn);
   char* qkv = (char*)buf(P.qkv);
   float2* tab = (float2*)buf(P.tab);
-  TRY(launch_rmsnorm(x_in, Dm, w->norm_g[2], xn, Dm, B, Dm, c.norm_eps, dt, st, true));
+  if (!ss_in) TRY(launch_rmsnorm(x_in, Dm, w->norm_g[2], xn, Dm, B, Dm, c.norm_eps, dt, st, true));
   const int hd = c.head_dim;
   const int qw = c.n_q * hd, kvw = c.n_kv * hd;
   {
@@ -860,6 +878,9 @@ static samba_status swa_step_layer(const LayerCtx& X, const samba_block_weights*
     g.seg[2].W = w->Wv;
     g.seg[2].n = kvw;
     g.pdl = true;
+    g.ss_in = ss_in;
+    g.norm_dim = Dm;
+    g.norm_eps = c.norm_eps;
     bool ring_done = false;
     if (c.rope_base != 0.f) {
       g.epi = kEpiRope;
@@ -895,6 +916,11 @@ static samba_status swa_step_layer(const LayerCtx& X, const samba_block_weights*
   g.resid = x_in;
   g.ldr = Dm;
   g.pdl = true;
+  if (ss_out) {  // the MLP norm's input and sums of squares
+    g.ss_out = ss_out;
+    g.g_next = g_next;
+    g.xg_out = xn;
+  }
   return launch_gemm(g, st);
 }
 
@@ -1163,6 +1189,37 @@ samba_status samba_model_step(const samba_model* m, const int32_t* ids_t, void* 
 }
 
 // ------------------------------------------------------------------ decode step
+}  // extern "C"
+
+namespace samba {
+
+// Whether every projection the decode-step norm fold involves runs on the
+// skinny kernel (bf16, batch <= 64, 16-byte aligned weights and gains, K
+// multiples of 64, QKV segments on 128-row tile boundaries with RoPE heads of
+// at most 128): out_proj and both MLP down projections produce x (.) g and the
+// sums of squares, both MLP up projections and the QKV projection consume
+// them.  SAMBA_NORM_FOLD=0 turns the fold off.
+static bool step_norm_fold_ok(const samba_block_config& c, const samba_block_weights* w, int B) {
+  const char* e = getenv("SAMBA_NORM_FOLD");
+  if (e && e[0] == '0') return false;
+  const char* gk = getenv("SAMBA_GEMM_KERNEL");
+  if (gk && gk[0] == 's') return false;
+  if (c.dtype != SAMBA_BF16 || B > 64) return false;
+  const int hd = c.head_dim, qw = c.n_q * hd, kvw = c.n_kv * hd;
+  if (c.d_model % 64 || c.d_inner % 64 || c.d_ff % 64 || qw % 64) return false;
+  if (qw % 128 || (qw + kvw) % 128) return false;  // tiles never straddle the Q | K | V segments
+  if (c.rope_base != 0.f && (hd < 16 || 128 % hd != 0 || hd / 2 > 64)) return false;
+  const void* ptrs[] = {w->W_out, w->mlp1_W1, w->mlp1_W2, w->mlp1_W3, w->mlp2_W1, w->mlp2_W2, w->mlp2_W3, w->Wq,
+                        w->Wk,    w->Wv,      w->Wo,      w->norm_g[1], w->norm_g[2], w->norm_g[3]};
+  for (const void* q : ptrs)
+    if (!q || !aligned16(q)) return false;
+  return true;
+}
+
+}  // namespace samba
+
+extern "C" {
+
 // The step's workspace: one block's activations for B tokens, then (rings
 // above 2048 slots) the split decode attention's partials.
 static size_t step_attn_offset(const samba_block_config& c, int B) {
@@ -1194,15 +1251,20 @@ samba_status samba_step(const samba_block_config* cfg, const samba_block_weights
   const LayerCtx X{c, P, base, B, 1, (int64_t)B, st};
   void *x1 = base + P.x1, *x2 = base + P.x2, *x3 = base + P.x3;
   TRY(guards_arm(base, P.cv, st));
-  TRY(mamba_step_layer(X, w, x_t, x1, stt->ssm, stt->conv));
+  // norm fold: norms 1..3 are completed by the projections around them, through
+  // three areas of B x d_model/8 partial sums of squares
+  float* ssf = step_norm_fold_ok(c, w, B) ? (float*)(base + P.ss) : nullptr;
+  const int64_t nss = (int64_t)B * (c.d_model / 8);
+  TRY(mamba_step_layer(X, w, x_t, x1, stt->ssm, stt->conv, ssf));
   TRY(mlp_sublayer(c, w->norm_g[1], w->mlp1_W1, w->mlp1_W2, w->mlp1_W3, x1, x2, base + P.xn, base + P.hmlp, nullptr,
-                   B, st, true));
+                   B, st, true, nullptr, nullptr, ssf, ssf ? ssf + nss : nullptr, w->norm_g[2]));
   const size_t attn_bytes = attn_decode_workspace_bytes(B, c.n_kv, c.window);
   TRY(swa_step_layer(X, w, x2, x3, stt->k_ring, stt->v_ring, stt->pos,
-                     attn_bytes ? base + step_attn_offset(c, B) : nullptr, attn_bytes));
+                     attn_bytes ? base + step_attn_offset(c, B) : nullptr, attn_bytes, ssf ? ssf + nss : nullptr,
+                     ssf ? ssf + 2 * nss : nullptr, w->norm_g[3]));
   bool pos_done = false;
   TRY(mlp_sublayer(c, w->norm_g[3], w->mlp2_W1, w->mlp2_W2, w->mlp2_W3, x3, y_t, base + P.xn, base + P.hmlp, nullptr,
-                   B, st, true, stt->pos, &pos_done));
+                   B, st, true, stt->pos, &pos_done, ssf ? ssf + 2 * nss : nullptr));
   TRY(guards_check(base, P.cv, st));
   return pos_done ? SAMBA_OK : launch_pos_update(stt->pos, B, 1, false, st, true);
 }

@@ -793,6 +793,8 @@ samba_status launch_gemm(const GemmArgs& a, cudaStream_t st) {
                             a.rope_cols % a.head_dim))
     return SAMBA_ERR_INVALID_ARG;
   if (a.M == 0) return SAMBA_OK;
+  // the norm fold is implemented by the skinny kernel only
+  if ((a.ss_in || a.ss_out) && !gemm_takes_skinny(a)) return SAMBA_ERR_UNSUPPORTED;
   const cudaEvent_t tstop = timing_begin(a.epi, st);
   const samba_status r = gemm_dispatch(a, st);
   timing_end(tstop, st);

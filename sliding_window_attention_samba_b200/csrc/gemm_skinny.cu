@@ -58,6 +58,7 @@ struct SkSmem {
   unsigned char ring[kRing];
   uint64_t full[SK_STAGES], empty[SK_STAGES], done;
   uint32_t tmem_base;
+  float rn[SK_MAXB];  // norm fold: each batch row's RMS scale
 };
 template <int EPI> constexpr int sk_ring_bytes() { return EPI == kEpiSwiglu ? SK_RING_BYTES_DUAL : SK_RING_BYTES; }
 
@@ -261,6 +262,20 @@ __global__ void __launch_bounds__(SK_THREADS, 2) gemm_skinny_kernel(const __grid
     const int q = warp & 3;
     const int row = q * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    if (a.ss_in) {
+      // norm fold, while the MMAs run: row b's RMS scale from its norm_dim/8
+      // partial sums of squares, in one fixed order (lane-strided, then a
+      // butterfly), so that every CTA and every run gets the same value
+      const int np = a.norm_dim / 8;
+      for (int b = q; b < (int)a.M; b += 4) {
+        const float* sp = a.ss_in + (int64_t)b * np;
+        float s = 0.f;
+        for (int j = lane; j < np; j += 32) s += sp[j];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (lane == 0) S.rn[b] = rsqrtf(s / (float)a.norm_dim + a.norm_eps);
+      }
+    }
     bool got = true;
     if (nkb > 0) got = __all_sync(0xffffffffu, mbar_wait(&S.done, 0, err));
     if (got) tc_fence_after();
@@ -315,6 +330,7 @@ __global__ void __launch_bounds__(SK_THREADS, 2) gemm_skinny_kernel(const __grid
       float x1[8], x2[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) x1[j] = x2[j] = 0.f;
+      const float rn = a.ss_in ? S.rn[b] : 1.f;
       for (int sidx = 0; sidx < p.S; ++sidx) {
         const float* q = recv(0, sidx, b);
         const float4 a0 = *reinterpret_cast<const float4*>(q + 8 * g);
@@ -329,6 +345,8 @@ __global__ void __launch_bounds__(SK_THREADS, 2) gemm_skinny_kernel(const __grid
       float o1[8], o2[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
+        x1[j] *= rn;
+        x2[j] *= rn;
         const float2 cs = a.rope_tab ? rope_cs_sk(a.rope_tab, half, pos, i0 + j) : rope_cs_direct(p.theta[i0 + j], pos);
         o1[j] = x1[j] * cs.x - x2[j] * cs.y;
         o2[j] = x2[j] * cs.x + x1[j] * cs.y;
@@ -351,6 +369,7 @@ __global__ void __launch_bounds__(SK_THREADS, 2) gemm_skinny_kernel(const __grid
       if (n >= a.N) continue;  // N % 8 == 0: a group is wholly inside or outside
       if (!SAMBA_DCHECK(err, n + 8 <= a.N && b < M)) continue;
       float extra[8];
+      const float rn = a.ss_in ? S.rn[b] : 1.f;
       if (EPI == kEpiResid) load8((const bf16*)a.resid + (int64_t)b * a.ldr + n, extra);
       if (EPI == kEpiSoftplus) load8(a.bias + n, extra);
       float v[8], v2[8];
@@ -372,6 +391,8 @@ __global__ void __launch_bounds__(SK_THREADS, 2) gemm_skinny_kernel(const __grid
       }
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
+        v[j] *= rn;
+        v2[j] *= rn;
         if (EPI == kEpiSwiglu) v[j] = v[j] * (v2[j] * sigmoid_fast(v2[j]));
         if (EPI == kEpiSoftplus) v[j] = softplus_1x(v[j] + extra[j]);
       }
@@ -379,6 +400,20 @@ __global__ void __launch_bounds__(SK_THREADS, 2) gemm_skinny_kernel(const __grid
         if (a.tap) store8((bf16*)a.tap + (int64_t)b * a.ldt + n, v);
 #pragma unroll
         for (int j = 0; j < 8; ++j) v[j] += extra[j];
+        if (a.ss_out) {  // the next norm's input: the stored row times its gain, and the row's sum of squares
+          float xg[8], sq = 0.f;
+          const float4 g0 = reinterpret_cast<const float4*>(a.g_next + n)[0];
+          const float4 g1 = reinterpret_cast<const float4*>(a.g_next + n)[1];
+          const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float vb = __bfloat162float(__float2bfloat16_rn(v[j]));
+            sq = fmaf(vb, vb, sq);
+            xg[j] = vb * gg[j];
+          }
+          store8((bf16*)a.xg_out + (int64_t)b * a.ldo + n, xg);
+          a.ss_out[(int64_t)b * (a.N / 8) + n / 8] = sq;
+        }
       }
       if (EPI == kEpiNone && a.conv_u && n < a.conv_cols) {
         // short convolution step of channels n .. n+7 (the state keeps inputs as stored, in bf16)
@@ -461,6 +496,9 @@ bool gemm_skinny_supported(const GemmArgs& a) {
     start += a.seg[s].n;
   }
   if (a.epi == kEpiSwiglu && a.nseg != 1) return false;
+  if (a.ss_in && (a.norm_dim <= 0 || a.norm_dim % 8)) return false;
+  if (a.ss_out && (a.epi != kEpiResid || !a.g_next || !a.xg_out || !aligned16(a.g_next) || !aligned16(a.xg_out)))
+    return false;
   if (a.conv_u) {  // the short convolution step on columns [0, conv_cols)
     if (a.epi != kEpiNone || a.conv_k != 4 || a.conv_cols % 8 || a.conv_cols > a.N || !a.conv_w || !a.conv_state ||
         !aligned16(a.conv_w) || !aligned16(a.conv_state) || !aligned16(a.conv_u))

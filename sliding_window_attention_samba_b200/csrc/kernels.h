@@ -146,6 +146,20 @@ struct GemmArgs {
   void* conv_state = nullptr;
   void* conv_u = nullptr;
   int conv_cols = 0, conv_k = 0;
+  // decode norm fold (skinny kernel only).  ss_in != NULL: the A rows are
+  // x (.) g of stream rows x, and ss_in[b * norm_dim/8 + j] holds the sum of
+  // squares of x[b, 8j .. 8j+8); output row b is scaled by
+  // rsqrt(sum_j ss_in[b, j] / norm_dim + norm_eps), which completes
+  // RMSNorm(x) W^T.  ss_out != NULL (kEpiResid): also writes bf16(out) (.) g_next
+  // to xg_out (row stride ldo) and the sums of squares of every 8 stored
+  // features to ss_out[b * N/8 + n/8] -- one writer per slot, summed in a fixed
+  // order by the consumer, so the result is deterministic
+  const float* ss_in = nullptr;
+  int norm_dim = 0;
+  float norm_eps = 0.f;
+  const float* g_next = nullptr;
+  void* xg_out = nullptr;
+  float* ss_out = nullptr;
   // decode (skinny kernel only): add 1 to pos_inc[0 .. M) once the kernel's
   // prerequisites have completed (the last projection of a step)
   int64_t* pos_inc = nullptr;

@@ -212,6 +212,40 @@ def test_decode_steps_wide_bf16_batch4(L):
         assert step_err(y, x[:, P + i], full, P + i, "bf16") <= TOL["bf16"], i
 
 
+def test_decode_norm_fold_on_off_wide_bf16_batch3(L, monkeypatch):
+    """The decode step's norm fold (the three RMSNorms after the first ride on
+    the projections around them: the producer writes x (.) g and per-8-feature
+    sums of squares, the consumer scales its rows by the RMS) against the plain
+    RMSNorm launches (SAMBA_NORM_FOLD=0): both within tolerance of the oracle,
+    close to each other, and the folded step bit-reproducible from the same
+    state (its sums are reduced in a fixed order)."""
+    import torch
+    shape = I.WIDE
+    W = I.block_weights(shape, 16)
+    P, S, Bn = 200, 3, 3
+    x = I.block_input(shape, 16, Bn, P + S)
+    g = GpuBlock(L, shape, W, Bn, P + S)
+    g.prefill(x[:, :P], taps=False)
+    full = O.block_fwd(x, W, shape)
+    state = (g.ssm, g.conv, g.k_ring, g.v_ring, g.pos)
+    snap = [t.clone() for t in state]
+
+    def run():
+        for t, s_ in zip(state, snap):
+            t.copy_(s_)
+        return [g.step(x[:, P + i]).clone() for i in range(S)]
+    folded, again = run(), run()
+    monkeypatch.setenv("SAMBA_NORM_FOLD", "0")
+    plain = run()
+    for i in range(S):
+        assert torch.equal(folded[i], again[i]), i
+        for y in (folded[i], plain[i]):
+            assert step_err(host(y), x[:, P + i], full, P + i, "bf16") <= TOL["bf16"], i
+        contrib = plain[i].float() - dev(x[:, P + i], g.dt).float()  # the block's part of the output
+        d = float((folded[i].float() - plain[i].float()).norm() / contrib.norm())
+        assert d <= 1e-2, (i, d)
+
+
 def _ring_map_exact(ring, oracle_k, cur, w):
     """The ring's slot -> position map after `cur` tokens, bit-exact: every slot
     holds the key of the latest position p < cur with p mod w == slot (slots
