@@ -1006,9 +1006,11 @@ def run_model_decode(args):
         per = {}
         with torch.cuda.stream(stream):
             L.samba_model_step(m, ids_t, logits, st_arr, pos, Bn, wsp, n, stream=stream)
-            graph = torch.cuda.CUDAGraph()
+            graph = torch.cuda.CUDAGraph(keep_graph=True)
             with torch.cuda.graph(graph, stream=stream):
                 L.samba_model_step(m, ids_t, logits, st_arr, pos, Bn, wsp, n, stream=stream)
+            nk = graph_kernel_nodes(graph)
+            graph.instantiate()
             for P in points:
                 pos.fill_(P)
                 for _ in range(3):
@@ -1027,7 +1029,7 @@ def run_model_decode(args):
         t_gen = sum((points[i + 1] - points[i]) * (per[points[i]] + per[points[i + 1]]) / 2
                     for i in range(len(points) - 1))
         out[name] = {"step_ms_at_context": {str(P): round(per[P] * 1e3, 4) for P in points},
-                     "tokens_per_s_64K_generation": Bn * gen / t_gen,
+                     "tokens_per_s_64K_generation": Bn * gen / t_gen, "launches_per_step": nk,
                      "params": sum(t.numel() for w in ws_layers for t in w.values()) + 2 * vocab * s.d_model}
         del states, st_arr, ws_layers, wsp
         torch.cuda.empty_cache()

@@ -785,8 +785,12 @@ static samba_status swa_sublayer(const LayerCtx& X, const samba_block_weights* w
 // [Samba 3.4 "The Mamba Layer" at a single t].  Every launch of a decode step is
 // a programmatic dependent of the one before it: a kernel sets up (and the
 // projections fetch their first weight tiles) while its predecessor finishes.
+// ss_in / ss_out / g_next: the norm fold (the layer's RMSNorm completed by its
+// input projection from the previous producer's sums of squares; its output
+// projection writes the next norm's input and sums of squares).
 static samba_status mamba_step_layer(const LayerCtx& X, const samba_block_weights* w, const void* x_in, void* x_out,
-                                     float* ssm, void* conv, float* ssf = nullptr) {
+                                     float* ssm, void* conv, const float* ss_in = nullptr, float* ss_out = nullptr,
+                                     const float* g_next = nullptr) {
   NvtxRange nvtx_("samba.mamba_step");
   const samba_block_config& c = X.c;
   const BlockPlan& P = X.P;
@@ -803,9 +807,12 @@ static samba_status mamba_step_layer(const LayerCtx& X, const samba_block_weight
     g.pdl = true;
     return launch_gemm(g, st);
   };
-  TRY(launch_rmsnorm(x_in, Dm, w->norm_g[0], xn, Dm, B, Dm, c.norm_eps, dt, st, true));
+  if (!ss_in) TRY(launch_rmsnorm(x_in, Dm, w->norm_g[0], xn, Dm, B, Dm, c.norm_eps, dt, st, true));
   {
     GemmArgs g = gemm1(xn, Dm, w->W_in, B, 2 * Di, Dm, hz, 2 * Di, dt);
+    g.ss_in = ss_in;
+    g.norm_dim = Dm;
+    g.norm_eps = c.norm_eps;
     // the skinny projection runs the short convolution step on its x columns itself
     GemmArgs gc = g;
     gc.conv_w = w->conv_w;
@@ -838,9 +845,9 @@ static samba_status mamba_step_layer(const LayerCtx& X, const samba_block_weight
   g.epi = kEpiResid;
   g.resid = x_in;
   g.ldr = Dm;
-  if (ssf) {  // the MLP norm's input and sums of squares
-    g.ss_out = ssf;
-    g.g_next = w->norm_g[1];
+  if (ss_out) {  // the next norm's input and sums of squares
+    g.ss_out = ss_out;
+    g.g_next = g_next;
     g.xg_out = xn;
   }
   return gemm_pdl(g);
@@ -1128,6 +1135,65 @@ static ModelStepPlan plan_model_step(const samba_block_config& c, int B) {
   return m;
 }
 
+// The decode norm fold: a layer's RMSNorm is completed by its input
+// projection(s), which scale their output rows by the RMS from per-8-feature
+// sums of squares, and the residual projection before it writes the norm's
+// input (the stream row times the norm's gain) and those sums.  Every
+// projection involved must run on the skinny kernel: bf16, batch <= 64, K
+// multiples of 64, QKV segments on 128-row tile boundaries with RoPE heads of
+// at most 128, 16-byte aligned weights and gains.  SAMBA_NORM_FOLD=0 turns it
+// off.
+static bool fold_dims_ok(const samba_block_config& c, int B) {
+  const char* e = getenv("SAMBA_NORM_FOLD");
+  if (e && e[0] == '0') return false;
+  const char* gk = getenv("SAMBA_GEMM_KERNEL");
+  if (gk && gk[0] == 's') return false;
+  if (c.dtype != SAMBA_BF16 || B > 64) return false;
+  const int hd = c.head_dim, qw = c.n_q * hd, kvw = c.n_kv * hd;
+  if (c.d_model % 64 || c.d_inner % 64 || c.d_ff % 64 || qw % 64) return false;
+  if (qw % 128 || (qw + kvw) % 128) return false;  // tiles never straddle the Q | K | V segments
+  if (c.rope_base != 0.f && (hd < 16 || 128 % hd != 0 || hd / 2 > 64)) return false;
+  return true;
+}
+
+static bool all_aligned16(std::initializer_list<const void*> ptrs) {
+  for (const void* q : ptrs)
+    if (!q || !aligned16(q)) return false;
+  return true;
+}
+
+// The weights and input gain of one sub-layer kind the fold touches.
+static bool fold_layer_ok(int k, const samba_block_weights& w) {
+  switch (k) {
+    case SAMBA_LAYER_MAMBA: return all_aligned16({w.W_in, w.W_out, w.norm_g[0]});
+    case SAMBA_LAYER_SWA: return all_aligned16({w.Wq, w.Wk, w.Wv, w.Wo, w.norm_g[2]});
+    default: return all_aligned16({w.mlp1_W1, w.mlp1_W2, w.mlp1_W3, w.norm_g[1]});
+  }
+}
+
+// The gain of a sub-layer's input norm.
+static const float* layer_input_gain(int k, const samba_block_weights& w) {
+  return k == SAMBA_LAYER_MAMBA ? w.norm_g[0] : k == SAMBA_LAYER_SWA ? w.norm_g[2] : w.norm_g[1];
+}
+
+// samba_step: norms 1..3 (out_proj and both MLP down projections produce,
+// both MLP up projections and the QKV projection consume).
+static bool step_norm_fold_ok(const samba_block_config& c, const samba_block_weights* w, int B) {
+  return fold_dims_ok(c, B) && all_aligned16({w->W_out, w->mlp1_W1, w->mlp1_W2, w->mlp1_W3, w->mlp2_W1, w->mlp2_W2,
+                                              w->mlp2_W3, w->Wq, w->Wk, w->Wv, w->Wo, w->norm_g[1], w->norm_g[2],
+                                              w->norm_g[3]});
+}
+
+// samba_model_step: every norm after the first sub-layer's, the final norm
+// included (the LM head consumes it).
+static bool model_norm_fold_ok(const samba_model* m, int B, const void* logits) {
+  if (m->n_layers < 1 || !fold_dims_ok(m->cfg, B)) return false;
+  if (m->vocab % 8 || !all_aligned16({m->lm_head, m->final_norm, logits})) return false;
+  for (int i = 0; i < m->n_layers; ++i)
+    if (!fold_layer_ok(m->kinds[i], m->layers[i])) return false;
+  return true;
+}
+
 }  // namespace samba
 
 extern "C" {
@@ -1165,60 +1231,49 @@ samba_status samba_model_step(const samba_model* m, const int32_t* ids_t, void* 
   TRY(guards_arm(base, MP.cv, st));
   TRY(launch_embedding(ids_t, m->embedding, cur, B, Dm, m->vocab, dt, st));
   const LayerCtx X{c, MP.P, base, B, 1, (int64_t)B, st};
+  // norm fold: every norm after the first sub-layer's rides on the projections
+  // around it, through two alternating areas of B x d_model/8 partial sums of
+  // squares (ss_in: the previous producer's, ss_out: this layer's)
+  const bool fold = model_norm_fold_ok(m, B, logits);
+  float* ss_in = nullptr;
+  float* ss_out = fold ? (float*)(base + MP.P.ss) : nullptr;
+  float* ss_spare = fold ? ss_out + (int64_t)B * (Dm / 8) : nullptr;
   for (int i = 0; i < m->n_layers; ++i) {
     const samba_block_weights& w = m->layers[i];
     const samba_layer_state& sl = states[i];
+    const float* g_next = !fold ? nullptr
+                          : i + 1 < m->n_layers ? layer_input_gain(m->kinds[i + 1], m->layers[i + 1])
+                                                : m->final_norm;
     switch (m->kinds[i]) {
-      case SAMBA_LAYER_MAMBA: TRY(mamba_step_layer(X, &w, cur, nxt, sl.ssm, sl.conv)); break;
+      case SAMBA_LAYER_MAMBA: TRY(mamba_step_layer(X, &w, cur, nxt, sl.ssm, sl.conv, ss_in, ss_out, g_next)); break;
       case SAMBA_LAYER_SWA:
-        TRY(swa_step_layer(X, &w, cur, nxt, sl.k_ring, sl.v_ring, pos, base + MP.attn, MP.attn_bytes));
+        TRY(swa_step_layer(X, &w, cur, nxt, sl.k_ring, sl.v_ring, pos, base + MP.attn, MP.attn_bytes, ss_in, ss_out,
+                           g_next));
         break;
       default:
         TRY(mlp_sublayer(c, w.norm_g[1], w.mlp1_W1, w.mlp1_W2, w.mlp1_W3, cur, nxt, base + MP.P.xn,
-                         base + MP.P.hmlp, nullptr, B, st, true));
+                         base + MP.P.hmlp, nullptr, B, st, true, nullptr, nullptr, ss_in, ss_out, g_next));
         break;
     }
     std::swap(cur, nxt);
+    if (fold) {
+      ss_in = ss_out;
+      std::swap(ss_out, ss_spare);
+    }
   }
-  TRY(launch_rmsnorm(cur, Dm, m->final_norm, base + MP.xl, Dm, B, Dm, c.norm_eps, dt, st, true));
-  GemmArgs g = gemm1(base + MP.xl, Dm, m->lm_head, B, m->vocab, Dm, logits, m->vocab, dt);
+  // the LM head: RMSNorm(x) from the last producer's x (.) g and sums (fold), else a norm launch
+  if (!fold) TRY(launch_rmsnorm(cur, Dm, m->final_norm, base + MP.xl, Dm, B, Dm, c.norm_eps, dt, st, true));
+  GemmArgs g = gemm1(base + (fold ? MP.P.xn : MP.xl), Dm, m->lm_head, B, m->vocab, Dm, logits, m->vocab, dt);
   g.pdl = true;
+  g.ss_in = ss_in;
+  g.norm_dim = Dm;
+  g.norm_eps = c.norm_eps;
   TRY(launch_gemm(g, st));
   TRY(guards_check(base, MP.cv, st));
   return launch_pos_update(pos, B, 1, false, st, true);
 }
 
 // ------------------------------------------------------------------ decode step
-}  // extern "C"
-
-namespace samba {
-
-// Whether every projection the decode-step norm fold involves runs on the
-// skinny kernel (bf16, batch <= 64, 16-byte aligned weights and gains, K
-// multiples of 64, QKV segments on 128-row tile boundaries with RoPE heads of
-// at most 128): out_proj and both MLP down projections produce x (.) g and the
-// sums of squares, both MLP up projections and the QKV projection consume
-// them.  SAMBA_NORM_FOLD=0 turns the fold off.
-static bool step_norm_fold_ok(const samba_block_config& c, const samba_block_weights* w, int B) {
-  const char* e = getenv("SAMBA_NORM_FOLD");
-  if (e && e[0] == '0') return false;
-  const char* gk = getenv("SAMBA_GEMM_KERNEL");
-  if (gk && gk[0] == 's') return false;
-  if (c.dtype != SAMBA_BF16 || B > 64) return false;
-  const int hd = c.head_dim, qw = c.n_q * hd, kvw = c.n_kv * hd;
-  if (c.d_model % 64 || c.d_inner % 64 || c.d_ff % 64 || qw % 64) return false;
-  if (qw % 128 || (qw + kvw) % 128) return false;  // tiles never straddle the Q | K | V segments
-  if (c.rope_base != 0.f && (hd < 16 || 128 % hd != 0 || hd / 2 > 64)) return false;
-  const void* ptrs[] = {w->W_out, w->mlp1_W1, w->mlp1_W2, w->mlp1_W3, w->mlp2_W1, w->mlp2_W2, w->mlp2_W3, w->Wq,
-                        w->Wk,    w->Wv,      w->Wo,      w->norm_g[1], w->norm_g[2], w->norm_g[3]};
-  for (const void* q : ptrs)
-    if (!q || !aligned16(q)) return false;
-  return true;
-}
-
-}  // namespace samba
-
-extern "C" {
 
 // The step's workspace: one block's activations for B tokens, then (rings
 // above 2048 slots) the split decode attention's partials.
@@ -1255,7 +1310,7 @@ samba_status samba_step(const samba_block_config* cfg, const samba_block_weights
   // three areas of B x d_model/8 partial sums of squares
   float* ssf = step_norm_fold_ok(c, w, B) ? (float*)(base + P.ss) : nullptr;
   const int64_t nss = (int64_t)B * (c.d_model / 8);
-  TRY(mamba_step_layer(X, w, x_t, x1, stt->ssm, stt->conv, ssf));
+  TRY(mamba_step_layer(X, w, x_t, x1, stt->ssm, stt->conv, nullptr, ssf, w->norm_g[1]));
   TRY(mlp_sublayer(c, w->norm_g[1], w->mlp1_W1, w->mlp1_W2, w->mlp1_W3, x1, x2, base + P.xn, base + P.hmlp, nullptr,
                    B, st, true, nullptr, nullptr, ssf, ssf ? ssf + nss : nullptr, w->norm_g[2]));
   const size_t attn_bytes = attn_decode_workspace_bytes(B, c.n_kv, c.window);

@@ -162,6 +162,42 @@ def test_model_step_full_cache_split_attention_bf16(L):
             assert path_err(host(g.logits), g.oracle(ids[:, :t + 1]), "bf16") <= TOL["bf16"], t
 
 
+def test_model_step_norm_fold_on_off_wide_bf16(L, monkeypatch):
+    """The decode norm fold over a whole 2:1 stack (every norm after the first
+    sub-layer's, the final one included, completed by the projections around
+    it) against the plain norm launches (SAMBA_NORM_FOLD=0): both against the
+    oracle's prefill of every prefix, close to each other, and the folded steps
+    bit-reproducible from the same states."""
+    import torch
+    Bn, S, vocab = 3, 6, 264
+    g = GpuModel(L, I.WIDE, SAMBA_2_1, vocab, 34, Bn)
+    ids = _ids(34, Bn, S, vocab)
+    tensors = [t for d in g.states for t in d.values()] + [g.pos]
+    s0 = [t.clone() for t in tensors]
+
+    def run():
+        for t_, s_ in zip(tensors, s0):
+            t_.copy_(s_)
+        out = []
+        for t in range(S):
+            g.step(ids[:, t])
+            out.append(g.logits.clone())
+        torch.cuda.synchronize()
+        assert L.samba_get_error() == 0
+        return out
+    folded, again = run(), run()
+    monkeypatch.setenv("SAMBA_NORM_FOLD", "0")
+    plain = run()
+    for t in range(S):
+        assert torch.equal(folded[t], again[t]), t
+        if t in (0, 2, S - 1):
+            ref = g.oracle(ids[:, :t + 1])
+            for y in (folded[t], plain[t]):
+                assert path_err(host(y), ref, "bf16") <= TOL["bf16"], t
+        d = float((folded[t].float() - plain[t].float()).norm() / plain[t].float().norm())
+        assert d <= 1e-2, (t, d)
+
+
 def test_model_step_graph_replay_bit_exact(L):
     import torch
     Bn, vocab = 3, 50
