@@ -50,8 +50,10 @@ constexpr int SK_RING_BYTES_DUAL = 200 * 1024;
 // the reduction reads 8 consecutive features of one batch row as two 16-byte
 // loads per source and writes them as one 16-byte store.
 constexpr int SK_RED_PAD = 4;
-// largest receive area: 2 accumulators x S sources x 64 rows x (128/S + 4) floats, S <= 8
+// largest receive area: 2 accumulators x S sources x 64 rows x (128/S + 4) floats, S <= 8;
+// one accumulator with S = 16 (the narrow projections' non-portable clusters)
 static_assert(2 * SK_MAXB * (SK_BM + 8 * SK_RED_PAD) * 4 <= SK_RING_BYTES, "reduction tiles must fit in the ring");
+static_assert(SK_MAXB * (SK_BM + 16 * SK_RED_PAD) * 4 <= SK_RING_BYTES, "reduction tiles must fit in the ring");
 
 template <int kRing>
 struct SkSmem {
@@ -540,6 +542,51 @@ static samba_status skinny_launch(const SkParams& p, int ntiles, cudaStream_t st
   return SAMBA_OK;
 }
 
+// Clusters of 16 CTAs (non-portable) for the narrow projections: whether this
+// device launches them for the kernel of epilogue EPI, asked once per device
+// and never under stream capture (a capture-time call could invalidate it).
+template <int EPI>
+static bool cluster16_ok(cudaStream_t st) {
+  static int state[64];  // per device: 0 not asked yet, 1 yes, -1 no
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (state[dev]) return state[dev] > 0;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return false;
+  const size_t smem = sizeof(SkSmem<sk_ring_bytes<EPI>()>) + 1024;
+  auto kern = gemm_skinny_kernel<EPI>;
+  bool ok = ensure_smem_attr(kern, smem) &&
+            cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+  if (ok) {
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(16, 1, 1);
+    cfg.blockDim = dim3(SK_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 16;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int n = 0;
+    ok = cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n >= 1;
+  }
+  if (!ok) (void)cudaGetLastError();  // a refusal here only means portable clusters
+  state[dev] = ok ? 1 : -1;
+  return ok;
+}
+
+static bool cluster16_ok_epi(int epi, cudaStream_t st) {
+  switch (epi) {
+    case kEpiNone: return cluster16_ok<kEpiNone>(st);
+    case kEpiResid: return cluster16_ok<kEpiResid>(st);
+    case kEpiSoftplus: return cluster16_ok<kEpiSoftplus>(st);
+  }
+  return false;  // SwiGLU (two accumulators) and RoPE (8-pair items) keep S <= 8
+}
+
 samba_status launch_gemm_skinny(const GemmArgs& a, cudaStream_t st) {
   if (!gemm_skinny_supported(a)) return SAMBA_ERR_UNSUPPORTED;
   SkParams p;
@@ -557,11 +604,14 @@ samba_status launch_gemm_skinny(const GemmArgs& a, cudaStream_t st) {
   const int ntiles = (a.N + SK_BM - 1) / SK_BM;
   p.kb_total = a.K / SK_BK;
   // splits: about one CTA per SM (one wave; the SM's second CTA slot is left to
-  // the neighbouring projection), at most 8 (portable cluster size) and at most
-  // one k-block each
+  // the neighbouring projection), at most 8 (portable cluster size; 16 below)
+  // and at least one k-block each
   const int want = num_sms() / ntiles;
   int S = 1;
   while (S * 2 <= want && S * 2 <= 8 && S * 2 <= p.kb_total) S *= 2;
+  // a projection too narrow to fill the SMs with 8-CTA clusters (x_proj: two
+  // tiles) splits K 16 ways where the device launches 16-CTA clusters
+  if (S == 8 && want >= 16 && p.kb_total >= 16 && cluster16_ok_epi(a.epi, st)) S = 16;
   p.S = S;
   p.kps = (p.kb_total + S - 1) / S;
   {
