@@ -441,10 +441,16 @@ samba_status samba_model_step(const samba_model* m, const int32_t* ids_t, void* 
  * RoPE(k)/v at ring slot p mod window and attends over the min(p+1, window)
  * most recent slots; pos[b] becomes p + 1.  All state updates are in place and
  * read positions from device memory, so the call can be captured in a CUDA graph
- * and replayed.
+ * and replayed.  On the bf16 tensor-core path (B <= 64) the three RMSNorms after
+ * the first are completed inside the projections around them (the producer of a
+ * stream row also writes the norm's input and per-8-feature sums of squares, the
+ * consumer scales its rows): the same result up to rounding, bit-reproducible
+ * from run to run; the environment variable SAMBA_NORM_FOLD=0 launches the norms
+ * separately instead.  samba_model_step does the same across its stack.
  * ---------------------------------------------------------------------- */
-/* Workspace of samba_step: one block's activations for B tokens and, for rings
- * above 2048 slots, the per-slice partials of the decode attention. */
+/* Workspace of samba_step: one block's activations for B tokens (with the norm
+ * fold's sums of squares) and, for rings above 2048 slots, the per-slice
+ * partials of the decode attention. */
 size_t samba_step_workspace_size(const samba_block_config* cfg, int B);
 
 samba_status samba_step(const samba_block_config* cfg, const samba_block_weights* w, const void* x_t, void* y_t,
