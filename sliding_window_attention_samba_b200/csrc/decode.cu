@@ -107,20 +107,23 @@ __global__ void scan_step_kernel(const T* __restrict__ u, const T* __restrict__ 
 
 // Recurrence step with the dt projection folded in [Samba 3.4 "Input-Dependent
 // Selective Gating": Delta = softplus(dt_low W_dt^T + b)]: a CTA takes 16
-// channels for 32 batch rows (one warp per row; lane = 8 * q + i, lane q holding
-// states 4q .. 4q+3 of channels i and i + 8), so that one wave covers batch 32
-// at d_inner 4096.  Everything that does not come from the kernels before it
-// (the state, A_log, the biases, the 16 rows of W_dt into shared memory) is
-// fetched before waiting for them; then the 32 rows of dt_low are staged, each
-// lane forms a quarter of each Delta dot product and two shuffles complete it,
-// so Delta never goes through memory.  The state update and the read-out are
-// those of the kernel above.
+// channels for 32 batch rows with 16 warps, warp w the rows w and w + 16
+// (lane = 8 * q + i, lane q holding states 4q .. 4q+3 of channels i and i + 8).
+// 512 threads at up to 64 registers put two CTAs on an SM, so that batch 32 at
+// d_inner 4096 (256 CTAs) runs in one wave.  Everything that does not come from
+// the kernels before it (the state, A, the 16 rows of W_dt into shared memory)
+// is fetched before waiting for them; then the 32 rows of dt_low
+// are staged and Delta is formed (tensor-core tiles for bf16 with R % 16 == 0,
+// else each lane a quarter of the dot product and two shuffles), so Delta never
+// goes through memory.  The state update and the read-out are those of the
+// kernel above.
 constexpr int kSdCh = 16;    // channels per CTA
 constexpr int kSdRows = 32;  // batch rows per CTA
+constexpr int kSdWarps = 16;  // two rows per warp
 constexpr int kSdMaxR = 512;
 
 template <typename T>
-__global__ void __launch_bounds__(1024, 1)
+__global__ void __launch_bounds__(kSdWarps * 32, 2)
     scan_step_dt_kernel(const T* __restrict__ u, const T* __restrict__ z, int64_t ld_z, const T* __restrict__ xdbl,
                         int64_t ld_x, int R, const T* __restrict__ W_dt, const float* __restrict__ dt_bias,
                         const float* __restrict__ A_log, const float* __restrict__ Dskip, float* __restrict__ ssm,
@@ -134,44 +137,52 @@ __global__ void __launch_bounds__(1024, 1)
   const int nv = R / kVec;  // 16-byte pieces per row
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ci = lane & 7, q = lane >> 3;
-  const int b = b0 + warp;
-  const bool live = b < B;
-  // ---- before the wait: weights and the state (written only by this kernel's previous step)
+  // ---- before the wait: weights, A and the state (written only by this kernel's previous step)
   for (int e = threadIdx.x; e < kSdCh * nv; e += blockDim.x) {
     const int r = e / nv, k = e % nv;
     *reinterpret_cast<uint4*>(Ws + r * pitch + k * kVec) =
         *reinterpret_cast<const uint4*>(W_dt + (size_t)(c0 + r) * R + k * kVec);
   }
-  float4 hv[2], av[2];
-  float bias[2], dsk[2];
+  float4 hv[2][2], av[2];  // [row][channel half], [channel half]: A (x log2 e for bf16)
 #pragma unroll
   for (int hh = 0; hh < 2; ++hh) {
     const int c = c0 + ci + 8 * hh;
-    av[hh] = *reinterpret_cast<const float4*>(A_log + (size_t)c * 16 + 4 * q);
-    hv[hh] = live ? *reinterpret_cast<const float4*>(ssm + ((size_t)b * D + c) * 16 + 4 * q)
-                  : make_float4(0.f, 0.f, 0.f, 0.f);
-    bias[hh] = dt_bias ? dt_bias[c] : 0.f;
-    dsk[hh] = Dskip ? Dskip[c] : 0.f;
+    const float4 al = *reinterpret_cast<const float4*>(A_log + (size_t)c * 16 + 4 * q);
+    const float sc = sizeof(T) == 4 ? -1.f : -1.4426950408889634f;
+    av[hh] = make_float4(sc * expf(al.x), sc * expf(al.y), sc * expf(al.z), sc * expf(al.w));
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      const int b = b0 + warp + kSdWarps * rr;
+      hv[rr][hh] = b < B ? *reinterpret_cast<const float4*>(ssm + ((size_t)b * D + c) * 16 + 4 * q)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   }
   pdl_wait();
   pdl_trigger();
-  // ---- after it: dt_low rows (shared), B, C, u, z of this row
+  // ---- after it: dt_low rows (shared), B, C, u, z of this warp's rows
   for (int e = threadIdx.x; e < kSdRows * nv; e += blockDim.x) {
     const int r = e / nv, k = e % nv;
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (b0 + r < B) v = *reinterpret_cast<const uint4*>(xdbl + (size_t)(b0 + r) * ld_x + k * kVec);
     *reinterpret_cast<uint4*>(Xs + r * pitch + k * kVec) = v;
   }
-  float Bv[4] = {0.f, 0.f, 0.f, 0.f}, Cv[4] = {0.f, 0.f, 0.f, 0.f}, uv[2] = {0.f, 0.f}, zv[2] = {0.f, 0.f};
-  if (live) {
-    const T* Bp = xdbl + (size_t)b * ld_x + R + 4 * q;
-    load4(Bp, Bv);
-    load4(Bp + 16, Cv);
+  float Bv[2][4], Cv[2][4], uv[2][2], zv[2][2];
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int c = c0 + ci + 8 * hh;
-      uv[hh] = Elt<T>::to_f(u[(size_t)b * D + c]);
-      zv[hh] = Elt<T>::to_f(z[(size_t)b * ld_z + c]);
+  for (int rr = 0; rr < 2; ++rr) {
+    const int b = b0 + warp + kSdWarps * rr;
+#pragma unroll
+    for (int n = 0; n < 4; ++n) Bv[rr][n] = Cv[rr][n] = 0.f;
+    uv[rr][0] = uv[rr][1] = zv[rr][0] = zv[rr][1] = 0.f;
+    if (b < B) {
+      const T* Bp = xdbl + (size_t)b * ld_x + R + 4 * q;
+      load4(Bp, Bv[rr]);
+      load4(Bp + 16, Cv[rr]);
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int c = c0 + ci + 8 * hh;
+        uv[rr][hh] = Elt<T>::to_f(u[(size_t)b * D + c]);
+        zv[rr][hh] = Elt<T>::to_f(z[(size_t)b * ld_z + c]);
+      }
     }
   }
   __syncthreads();
@@ -201,44 +212,50 @@ __global__ void __launch_bounds__(1024, 1)
   }
   const int n8 = R / 8;
 #pragma unroll
-  for (int hh = 0; hh < 2; ++hh) {
-    const int c = c0 + ci + 8 * hh;
-    float acc = 0.f;
-    if (tc_dot) {
-      acc = Dpre[warp][ci + 8 * hh];
-    } else {
-      // Delta: lane q takes the 8-element pieces q, q + 4, q + 8, ... of the dot product
-      for (int k = q; k < n8; k += 4) {
-        float wv[8], xv[8];
-        load8(Ws + (ci + 8 * hh) * pitch + k * 8, wv);
-        load8(Xs + warp * pitch + k * 8, xv);
+  for (int rr = 0; rr < 2; ++rr) {
+    const int row = warp + kSdWarps * rr;  // row within the CTA
+    const int b = b0 + row;
+    const bool live = b < B;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc = fmaf(wv[j], xv[j], acc);
+    for (int hh = 0; hh < 2; ++hh) {
+      const int c = c0 + ci + 8 * hh;
+      float acc = 0.f;
+      if (tc_dot) {
+        acc = Dpre[row][ci + 8 * hh];
+      } else {
+        // Delta: lane q takes the 8-element pieces q, q + 4, q + 8, ... of the dot product
+        for (int k = q; k < n8; k += 4) {
+          float wv[8], xv[8];
+          load8(Ws + (ci + 8 * hh) * pitch + k * 8, wv);
+          load8(Xs + row * pitch + k * 8, xv);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc = fmaf(wv[j], xv[j], acc);
+        }
+        acc += __shfl_xor_sync(0xffffffffu, acc, 8);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 16);
       }
-      acc += __shfl_xor_sync(0xffffffffu, acc, 8);
-      acc += __shfl_xor_sync(0xffffffffu, acc, 16);
-    }
-    float delta = acc + bias[hh];
-    if constexpr (sizeof(T) == 4) delta = softplus_acc(delta);
-    else delta = softplus_1x(delta);
-    const float al[4] = {av[hh].x, av[hh].y, av[hh].z, av[hh].w};
-    float h[4] = {hv[hh].x, hv[hh].y, hv[hh].z, hv[hh].w};
-    const float du = delta * uv[hh];
-    float yv = 0.f;
+      float delta = acc + (dt_bias ? dt_bias[c] : 0.f);
+      if constexpr (sizeof(T) == 4) delta = softplus_acc(delta);
+      else delta = softplus_1x(delta);
+      const float A[4] = {av[hh].x, av[hh].y, av[hh].z, av[hh].w};
+      float h[4] = {hv[rr][hh].x, hv[rr][hh].y, hv[rr][hh].z, hv[rr][hh].w};
+      const float du = delta * uv[rr][hh];
+      float yv = 0.f;
 #pragma unroll
-    for (int n = 0; n < 4; ++n) {
-      const float A = -expf(al[n]);
-      const float dA = sizeof(T) == 4 ? expf(delta * A) : ex2_approx(delta * A * 1.4426950408889634f);
-      h[n] = fmaf(dA, h[n], du * Bv[n]);
-      yv = fmaf(Cv[n], h[n], yv);
-    }
-    if (live) *reinterpret_cast<float4*>(ssm + ((size_t)b * D + c) * 16 + 4 * q) = make_float4(h[0], h[1], h[2], h[3]);
-    yv += __shfl_xor_sync(0xffffffffu, yv, 8);
-    yv += __shfl_xor_sync(0xffffffffu, yv, 16);
-    if (live && q == 0) {
-      yv = fmaf(dsk[hh], uv[hh], yv);
-      const float s = sizeof(T) == 4 ? sigmoid_acc(zv[hh]) : sigmoid_fast(zv[hh]);
-      y[(size_t)b * D + c] = Elt<T>::from_f(yv * zv[hh] * s);
+      for (int n = 0; n < 4; ++n) {
+        const float dA = sizeof(T) == 4 ? expf(delta * A[n]) : ex2_approx(delta * A[n]);
+        h[n] = fmaf(dA, h[n], du * Bv[rr][n]);
+        yv = fmaf(Cv[rr][n], h[n], yv);
+      }
+      if (live)
+        *reinterpret_cast<float4*>(ssm + ((size_t)b * D + c) * 16 + 4 * q) = make_float4(h[0], h[1], h[2], h[3]);
+      yv += __shfl_xor_sync(0xffffffffu, yv, 8);
+      yv += __shfl_xor_sync(0xffffffffu, yv, 16);
+      if (live && q == 0) {
+        yv = fmaf(Dskip ? Dskip[c] : 0.f, uv[rr][hh], yv);
+        const float sg = sizeof(T) == 4 ? sigmoid_acc(zv[rr][hh]) : sigmoid_fast(zv[rr][hh]);
+        y[(size_t)b * D + c] = Elt<T>::from_f(yv * zv[rr][hh] * sg);
+      }
     }
   }
 }
@@ -973,10 +990,10 @@ samba_status launch_scan_step_dt(const void* u, const void* z, int64_t ld_z, con
     return SAMBA_ERR_CUDA;
   cudaError_t e;
   SAMBA_DT_DISPATCH(dt,
-                    (e = launch_k(scan_step_dt_kernel<bf16>, grid, dim3(1024), smem, st, true, (const bf16*)u,
+                    (e = launch_k(scan_step_dt_kernel<bf16>, grid, dim3(kSdWarps * 32), smem, st, true, (const bf16*)u,
                                   (const bf16*)z, ld_z, (const bf16*)xdbl, ld_x, R, (const bf16*)W_dt, dt_bias, A_log,
                                   Dskip, ssm, (bf16*)y, B, D)),
-                    (e = launch_k(scan_step_dt_kernel<float>, grid, dim3(1024), smem, st, true, (const float*)u,
+                    (e = launch_k(scan_step_dt_kernel<float>, grid, dim3(kSdWarps * 32), smem, st, true, (const float*)u,
                                   (const float*)z, ld_z, (const float*)xdbl, ld_x, R, (const float*)W_dt, dt_bias,
                                   A_log, Dskip, ssm, (float*)y, B, D)));
   if (e != cudaSuccess) return note_cuda_failure("decode kernel launch", e);
