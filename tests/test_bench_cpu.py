@@ -72,3 +72,14 @@ def test_scan_bytes_per_token():
 def test_replica_throughput_counts_all_ranks():
     assert bench.replica_throughput(131072, 4, 2.0, 10, 4) == pytest.approx(4 * 131072 * 10 * 4 / 2.0)
     assert np.isclose(bench.replica_throughput(1, 1, 1.0, 1, 1), 1.0)
+
+
+def test_graph_kernel_nodes_without_a_graph_is_unknown():
+    """The decode lines' launch count comes from the captured graph's kernel
+    nodes; where the handle cannot be read (no GPU, no graph kept) the helper
+    reports None and the line falls back to its stated count instead of
+    inventing one."""
+    class NoGraph:
+        def raw_cuda_graph(self):
+            raise RuntimeError("keep_graph was not set")
+    assert bench.graph_kernel_nodes(NoGraph()) is None
