@@ -374,6 +374,12 @@ __global__ void __launch_bounds__(SK_THREADS, 2) gemm_skinny_kernel(const __grid
       const float rn = a.ss_in ? S.rn[b] : 1.f;
       if (EPI == kEpiResid) load8((const bf16*)a.resid + (int64_t)b * a.ldr + n, extra);
       if (EPI == kEpiSoftplus) load8(a.bias + n, extra);
+      // norm fold: the next norm's gain, fetched together with the residual
+      float4 gn0 = make_float4(0.f, 0.f, 0.f, 0.f), gn1 = gn0;
+      if (EPI == kEpiResid && a.ss_out) {
+        gn0 = reinterpret_cast<const float4*>(a.g_next + n)[0];
+        gn1 = reinterpret_cast<const float4*>(a.g_next + n)[1];
+      }
       float v[8], v2[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) v[j] = v2[j] = 0.f;
@@ -404,9 +410,7 @@ __global__ void __launch_bounds__(SK_THREADS, 2) gemm_skinny_kernel(const __grid
         for (int j = 0; j < 8; ++j) v[j] += extra[j];
         if (a.ss_out) {  // the next norm's input: the stored row times its gain, and the row's sum of squares
           float xg[8], sq = 0.f;
-          const float4 g0 = reinterpret_cast<const float4*>(a.g_next + n)[0];
-          const float4 g1 = reinterpret_cast<const float4*>(a.g_next + n)[1];
-          const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+          const float gg[8] = {gn0.x, gn0.y, gn0.z, gn0.w, gn1.x, gn1.y, gn1.z, gn1.w};
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const float vb = __bfloat162float(__float2bfloat16_rn(v[j]));
