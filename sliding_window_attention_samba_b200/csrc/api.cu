@@ -289,6 +289,10 @@ static GemmArgs gemm1(const void* A, int64_t lda, const void* W, int64_t M, int 
 }
 
 // SwiGLU MLP sub-layer: x_next = x + W3 ((W1 xn) * SiLU(W2 xn))  [Samba 3.4 "SwiGLU Formulation"]
+// Decode (pdl): pos_inc / pos_done let the down projection advance the
+// positions; ss_in / ss_out / g_next are the norm fold (the up projection
+// completes this sub-layer's RMSNorm, the down projection writes the next one's
+// input and sums of squares).
 static samba_status mlp_sublayer(const samba_block_config& c, const float* g, const void* W1, const void* W2,
                                  const void* W3, const void* x, void* x_next, void* xn, void* hmlp, void* tap,
                                  int64_t T, cudaStream_t st, bool pdl = false, int64_t* pos_inc = nullptr,
@@ -857,6 +861,7 @@ static samba_status mamba_step_layer(const LayerCtx& X, const samba_block_weight
 // position pos[b], k/v written to ring slot pos[b] mod window, attention over
 // the min(pos[b] + 1, window) valid slots, output projection, residual.
 // attn_ws: partials of the split attention for rings above 2048 slots.
+// ss_in / ss_out / g_next: the norm fold, as for the Mamba step layer.
 static samba_status swa_step_layer(const LayerCtx& X, const samba_block_weights* w, const void* x_in, void* x_out,
                                    void* k_ring, void* v_ring, const int64_t* pos, void* attn_ws,
                                    size_t attn_ws_bytes, const float* ss_in = nullptr, float* ss_out = nullptr,
