@@ -75,9 +75,9 @@ def parse():
 
 
 def load_peaks():
-    """(HBM GB/s, burst bf16 TF/s, sustained bf16 TF/s, source): the pool's
-    measured figures when the driver wrote them, else the profiling recipe's
-    fallback (6.65 TB/s, 1.59 PF/s burst, ~1.4 PF/s sustained)."""
+    """(HBM GB/s, burst bf16 TF/s, sustained bf16 TF/s, source): the measured
+    figures of MEASURED_PEAKS.json when present, else fallback figures for the
+    B200 (6.65 TB/s, 1.59 PF/s burst, ~1.4 PF/s sustained)."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
@@ -88,7 +88,7 @@ def load_peaks():
 def peak_clock_mhz(kind):
     """SM clock (MHz) at which a peak was taken: from MEASURED_PEAKS.json when it
     records one (any numeric field whose name mentions the peak kind and a
-    clock), else the recipe's statement for the fallback sustained figure
+    clock), else the clock of the fallback sustained figure
     (~1.4 PF/s at ~1.3 GHz).  None when unknown."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
